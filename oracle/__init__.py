@@ -1,0 +1,293 @@
+"""FP64 CPU oracle for the Kimi Delta Attention (KDA) hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA library (``gated_delta_rule_73_b200``) and never imports it; the
+library never imports this package.
+
+Pages cited (titles as published; the section, figure or Q&A item follows):
+
+* "Kimi K3 の KDA(1): KDA が Gated MLA と AttnRes とどのように連携するか"
+  (news.ainew.jp) -- cited as *Kimi K3 KDA(1)*.
+* "Kimi K3 模型结构（2）：序列维度（下），chunkwise 并行与下界衰减"
+  (xhh.club) -- cited as *Kimi K3 structure (2)*.
+* "Complex KDA: 理解并增强 Kimi Delta Attention 的表达能力" (ai-feeds.com)
+  -- cited as *Complex KDA summary*.
+* "GDN, KDA の整理" (taxfree.dev) -- cited as *GDN, KDA notes*.
+* "[논문리뷰] Complex KDA: Understanding and Enhancing the Expressivity of
+  Kimi Delta Attention" (blog.secrett2633.cloud) -- cited as *CKDA review*.
+
+Functions
+---------
+``recurrence_c``      plain C FP64 token recurrence (threaded over sequences).
+``recurrence_np``     numpy FP64 twin of the same recurrence (vectorised over
+                      sequences, loop over tokens).
+``recurrence_loops``  pure-Python loops, for tiny cases only.
+``chunkwise_np``      FP64 chunkwise-algebra form (cumulative decay, A_kk,
+                      UT inverse, WY vectors, inter-chunk state update).
+``conv_silu_np``      causal depthwise short convolution + SiLU.
+``bounded_log_decay`` g = -5 * sigmoid(exp(A_h) * z).
+``sigmoid``           beta = sigmoid(b).
+``prologue_np``       the three together (raw inputs -> q, k, v, g, beta).
+
+Every function is pinned by tests in ``tests/test_oracle_pins.py`` against
+closed forms, special cases, brute force and the worked example printed on the
+pages.  No function here is "parity unpinned".
+
+Conventions shared with the library's ABI (but not its code): layouts are
+``q, k, g: [B, T, H, dk]``, ``v, out: [B, T, H, dv]``, ``beta: [B, T, H]``,
+``S: [B, H, dk, dv]`` with rows = key channels; ``o_t = scale * S_t^T q_t``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+
+L2NORM_EPS = 1e-6   # reading: epsilon inside the square root (pages give none)
+G_MIN = -5.0        # Kimi K3 structure (2), Q&A on the -5 lower bound
+
+
+def build() -> str:
+    """Compile the C oracle into ``oracle/libkda_oracle.so`` (gcc, -O2)."""
+    if (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", _LIB, _SRC,
+             "-lm", "-lpthread"])
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.kda_oracle_recurrence.argtypes = [dp] * 8 + [ctypes.c_long] * 5 + [
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_int]
+        lib.kda_oracle_recurrence.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def recurrence_c(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False,
+                 scale=1.0, eps=L2NORM_EPS, nthreads=None):
+    """FP64 token recurrence in plain C (``kda_oracle.c``).
+
+    Decay, then erase, then write, then read the post-write state:
+    Kimi K3 KDA(1) section 1.2.1; GDN, KDA notes section "Kimi Delta
+    Attention".  Returns ``(out [B,T,H,dv], S_T [B,H,dk,dv])``.
+    """
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and g.shape == q.shape
+    assert v.shape == (B, T, H, dv) and beta.shape == (B, T, H)
+    S0a = None if S0 is None else _f64(S0)
+    if S0a is not None:
+        assert S0a.shape == (B, H, dk, dv)
+    out = np.zeros((B, T, H, dv), dtype=np.float64)
+    S_T = np.zeros((B, H, dk, dv), dtype=np.float64)
+    nt = nthreads if nthreads is not None else (os.cpu_count() or 1)
+    rc = _load().kda_oracle_recurrence(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0a), _ptr(out), _ptr(S_T),
+        B, T, H, dk, dv, int(bool(l2norm)), int(bool(complex_gate)), float(scale),
+        float(eps), int(nt))
+    if rc != 0:
+        raise ValueError("kda_oracle_recurrence rejected its arguments")
+    return out, S_T
+
+
+def _normalise(x, eps):
+    return x / np.sqrt(np.sum(x * x, axis=-1, keepdims=True) + eps)
+
+
+def recurrence_np(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False,
+                  scale=1.0, eps=L2NORM_EPS):
+    """numpy FP64 twin of :func:`recurrence_c` (same definition, vectorised
+    over the independent (b, h) sequences, loop over tokens)."""
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if l2norm:
+        q, k = _normalise(q, eps), _normalise(k, eps)
+    S = np.zeros((B, H, dk, dv)) if S0 is None else _f64(S0).copy()
+    out = np.zeros((B, T, H, dv))
+    alpha = g if complex_gate else np.exp(g)
+    for t in range(T):
+        St = alpha[:, t, :, :, None] * S                       # decay rows
+        pred = np.einsum("bhij,bhi->bhj", St, k[:, t])          # St^T k
+        r = v[:, t] - pred
+        S = St + beta[:, t, :, None, None] * k[:, t, :, :, None] * r[:, :, None, :]
+        out[:, t] = scale * np.einsum("bhij,bhi->bhj", S, q[:, t])
+    return out, S
+
+
+def recurrence_loops(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False,
+                     scale=1.0, eps=L2NORM_EPS):
+    """Pure-Python scalar loops of the same recurrence (tiny cases only)."""
+    import math
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    out = np.zeros((B, T, H, dv))
+    S_T = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = [[0.0] * dv for _ in range(dk)] if S0 is None else \
+                [[float(S0[b, h, i, j]) for j in range(dv)] for i in range(dk)]
+            for t in range(T):
+                qt = [float(x) for x in q[b, t, h]]
+                kt = [float(x) for x in k[b, t, h]]
+                if l2norm:
+                    nq = math.sqrt(sum(x * x for x in qt) + eps)
+                    nk = math.sqrt(sum(x * x for x in kt) + eps)
+                    qt = [x / nq for x in qt]
+                    kt = [x / nk for x in kt]
+                for i in range(dk):
+                    a = float(g[b, t, h, i]) if complex_gate else math.exp(float(g[b, t, h, i]))
+                    for j in range(dv):
+                        S[i][j] *= a
+                for j in range(dv):
+                    p = sum(S[i][j] * kt[i] for i in range(dk))
+                    rj = float(v[b, t, h, j]) - p
+                    for i in range(dk):
+                        S[i][j] += float(beta[b, t, h]) * kt[i] * rj
+                for j in range(dv):
+                    out[b, t, h, j] = scale * sum(S[i][j] * qt[i] for i in range(dk))
+            S_T[b, h] = np.array(S)
+    return out, S_T
+
+
+def chunkwise_np(q, k, v, g, beta, S0=None, *, C=64, l2norm=True, complex_gate=False,
+                 scale=1.0, eps=L2NORM_EPS):
+    """FP64 chunkwise-parallel form, written from the pages' chunk algebra.
+
+    Kimi K3 structure (2), Q&A items on the chunkwise algorithm and on the
+    intra-chunk matrix A: chunks of C tokens, one state update per chunk, a
+    UT transform (one C x C triangular inverse) for the WY auxiliary vectors,
+    ``A = Tril[(Q * Gamma)(K / Gamma)^T]`` with the diagonal kept (Kimi K3
+    KDA(1) section 1.2.1: the read sees the token's own write) and
+    ``O = (Gamma * Q) S + A V~``.  The forms of A_kk, W, U and V~ are derived
+    from the recurrence (the pages name them without formulas):
+
+      Gamma_r = prod_{s<=r} alpha_s                 (within the chunk)
+      A_kk    = tril(beta_r (K*Gamma)(K/Gamma)^T, -1)
+      Tm      = (I + A_kk)^{-1}
+      W = Tm diag(beta) (K*Gamma),   U = Tm diag(beta) V
+      V~ = U - W S
+      O  = (Q*Gamma) S + tril((Q*Gamma)(K/Gamma)^T) V~
+      S <- diag(Gamma_C) S + (K * Gamma_C/Gamma)^T V~
+
+    FP64 holds exp(+-320), so the plain K/Gamma is used (no sub-tiling).
+    """
+    q, k, v, g, beta = map(_f64, (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if l2norm:
+        q, k = _normalise(q, eps), _normalise(k, eps)
+    alpha = g if complex_gate else np.exp(g)
+    out = np.zeros((B, T, H, dv))
+    S_T = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else _f64(S0)[b, h].copy()
+            for s in range(0, T, C):
+                e = min(s + C, T)
+                n = e - s
+                Q, K, V = q[b, s:e, h], k[b, s:e, h], v[b, s:e, h]
+                bt = beta[b, s:e, h]
+                Gam = np.cumprod(alpha[b, s:e, h], axis=0)            # n x dk
+                Kg, Ki, Qg = K * Gam, K / Gam, Q * Gam
+                Akk = np.tril(bt[:, None] * (Kg @ Ki.T), -1)
+                Tm = np.linalg.inv(np.eye(n) + Akk)
+                W = Tm @ (bt[:, None] * Kg)
+                U = Tm @ (bt[:, None] * V)
+                Vt = U - W @ S
+                Aqk = np.tril(Qg @ Ki.T)
+                out[b, s:e, h] = scale * (Qg @ S + Aqk @ Vt)
+                GC = Gam[-1]
+                S = GC[:, None] * S + (K * (GC[None, :] / Gam)).T @ Vt
+            S_T[b, h] = S
+    return out, S_T
+
+
+def sigmoid(x):
+    x = _f64(x)
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def bounded_log_decay(z, A):
+    """g = G_MIN * sigmoid(exp(A_h) * z), G_MIN = -5.
+
+    Kimi K3 structure (2), Q&A "衰减函数与 Kimi Linear 的负 softplus 有何不同";
+    GDN, KDA notes section "Kimi Delta Attention" (-5 < g < 0).
+    ``z``: [..., H, dk]; ``A``: [H] (the per-head log-scale).
+    """
+    z = _f64(z)
+    A = _f64(A)
+    return G_MIN * sigmoid(np.exp(A)[:, None] * z)
+
+
+def conv_silu_np(x, w):
+    """Causal depthwise short convolution (kernel 4, no bias, zero history)
+    followed by SiLU.
+
+    Kimi K3 KDA(1) section 1.2.1: ``ShortConvolution(hidden_size=12288,
+    kernel_size=4, activation='silu')``, each channel independent, the current
+    token and the three before it.  Tap order follows a causal Conv1d weight
+    ``[channels, 4]``: ``y_t = sum_j w[c, j] * x_{t-3+j}`` (tap 3 = current).
+    ``x``: [B, T, Cch]; ``w``: [Cch, 4].
+    """
+    x = _f64(x)
+    w = _f64(w)
+    B, T, Cch = x.shape
+    Kw = w.shape[1]
+    y = np.zeros_like(x)
+    for j in range(Kw):
+        shift = Kw - 1 - j            # x_{t - shift}
+        if shift == 0:
+            y += w[None, None, :, j] * x
+        elif shift < T:
+            y[:, shift:, :] += w[None, None, :, j] * x[:, :T - shift, :]
+    return y * sigmoid(y)
+
+
+def prologue_np(q_pre, k_pre, v_pre, conv_w, z, A, b_logit):
+    """Raw branch inputs -> (q, k, v, g, beta), FP64.
+
+    ``q_pre, k_pre``: [B, T, H, dk]; ``v_pre``: [B, T, H, dv];
+    ``conv_w``: [3, H*dk, 4] (q, k, v taps; requires dk == dv);
+    ``z``: [B, T, H, dk]; ``A``: [H]; ``b_logit``: [B, T, H].
+    The L2 norm of q and k is left to the recurrence (``l2norm=True``).
+    """
+    q_pre, k_pre, v_pre = map(_f64, (q_pre, k_pre, v_pre))
+    B, T, H, dk = q_pre.shape
+    cw = _f64(conv_w)
+    outs = []
+    for i, x in enumerate((q_pre, k_pre, v_pre)):
+        d = x.shape[-1]
+        y = conv_silu_np(x.reshape(B, T, H * d), cw[i])
+        outs.append(y.reshape(B, T, H, d))
+    g = bounded_log_decay(z, A)
+    beta = sigmoid(b_logit)
+    return outs[0], outs[1], outs[2], g, beta
