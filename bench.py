@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one ``kda_chunk_fwd`` over the prefill workload (B=1, T=4096, H=16,
+dk=dv=128, bf16 q/k/v/g/beta, FP32 S0 -> out, S_T), inputs resident in HBM.
+The workload's inputs (86 MB) fit in the 126 MB L2, so a 256 MiB buffer is
+written between timed steps (outside the timed events).  Under torchrun every
+rank runs its own batch (weak scaling, no collective on the data path);
+``value`` is the tokens of all ranks over the slowest rank's time.
+
+Also measured on rank 0 at N=1 (the ``rows`` object): the fused-prologue
+length sweep at T=8192 (B=1, H=96), the decode step (N=256, H=96) and the
+Complex-KDA workload (B=8, T=8192, H=32) next to unsigned KDA of the same
+shape.  ``cpu_baseline`` times the FP64 oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_workloads as W  # noqa: E402
+
+METRIC = "chunk_kda fwd tokens/s & % of BF16 roofline; decode step state GB/s vs HBM"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+# algorithmic counts per token-head and per head (d = 128, C = 64): bf16 q,k,v,g,out
+# (4*256 + 256 bytes) + bf16 beta; FP32 S0 and S_T per head; FLOPs of the
+# triangular intra-chunk products, the three state GEMMs and the C x C inverse
+PREFILL_FLOP_PER_TOKEN_HEAD = 5 * 64 * 128 + 6 * 128 * 128 + 64 * 64 / 3
+
+
+def token_head_bytes(d, elt=2, beta_elt=2):
+    return 4 * d * elt + d * elt + beta_elt
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """Polls NVML (read-only) for SM clock and clock-event reasons while timing."""
+
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+               "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown"}
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            self.h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS.items():
+                    if r & getattr(N, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return 0
+    import numpy as np
+    import oracle
+    cfg = W.WORKLOADS["prefill"]
+    x = W.workload_inputs("prefill")
+    heads = 2       # a bounded sample of the workload per step
+    sel = {n: x[n][:, :, :heads].double().numpy() for n in ("q", "k", "v", "g", "beta")}
+    S0 = x["S0"][:, :heads].double().numpy()
+    threads = os.cpu_count() or 1
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        oracle.recurrence_c(sel["q"], sel["k"], sel["v"], sel["g"], sel["beta"], S0, nthreads=threads)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tok = cfg["B"] * cfg["T"] * heads
+    value = tok / statistics.mean(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill B=1 T=4096 H=16 dk=dv=128 (oracle sample: 2 heads)",
+                       "B": 1, "T": 4096, "H": 16, "dk": 128, "dv": 128},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, heads), "kind": "oracle",
+                             "sample": f"{heads} of 16 heads x 4096 tokens of the prefill workload per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def time_calls(fn, reps, flush=None, stream=None):
+    """Per-call CUDA-event times (ms) on the current stream, L2 flushed before each."""
+    out = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        out.append((a, b))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in out]
+
+
+def cpu_baseline_prefill():
+    import oracle
+    x = W.workload_inputs("prefill")
+    threads = os.cpu_count() or 1
+    arr = {n: x[n].double().numpy() for n in ("q", "k", "v", "g", "beta")}
+    S0 = x["S0"].double().numpy()
+    t0 = time.perf_counter()
+    oracle.recurrence_c(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], S0, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return {"value": 4096 * 16 / dt, "unit": UNIT, "cores": min(threads, 16), "kind": "oracle",
+            "sample": "the whole prefill workload (16 heads x 4096 tokens), FP64 C, one thread per head",
+            "seconds": dt}
+
+
+def rows_n1(K, flush, hbm_peak):
+    """Per-row measurements beyond the headline (rank 0, N=1)."""
+    rows = {}
+    W.set_device("cuda")
+    try:
+        # a1-a4: fused prologue + chunk forward, length sweep at T = 8192
+        T, H, d = 8192, 96, 128
+        x = W.sweep_inputs(T)
+        args = [x[n] for n in ("q_pre", "k_pre", "v_pre", "conv_w", "z", "A", "b_logit")]
+        opts0 = K.make_opts(torch.bfloat16)
+        ws = torch.empty(K.kda_prologue_workspace_bytes(1, T, H, d, d, opts0), dtype=torch.uint8,
+                         device="cuda")
+        out = torch.empty((1, T, H, d), dtype=torch.bfloat16, device="cuda")
+        S_T = torch.empty((1, H, d, d), dtype=torch.float32, device="cuda")
+        opts = K.make_opts(torch.bfloat16, workspace=ws)
+        fn = lambda: K.kda_chunk_fwd_prologue(*args, x["S0"], out, S_T, opts)
+        fn()
+        ms = statistics.median(time_calls(fn, 3, flush))
+        nbytes = T * H * (4 * d * 2 + 4 + d * 2) + H * (2 * d * d * 4 + 3 * d * 4 * 2)
+        rows["sweep_T8192_prologue"] = {
+            "ms": ms, "tokens_per_s": T / (ms * 1e-3), "token_heads_per_s": T * H / (ms * 1e-3),
+            "roofline_bytes": nbytes, "roofline_flops": PREFILL_FLOP_PER_TOKEN_HEAD * T * H,
+            "frac_of_hbm_roofline": (nbytes / (ms * 1e-3) / 1e9) / hbm_peak}
+        del x, args, ws, out, S_T
+        torch.cuda.empty_cache()
+
+        # a5: decode step, N = 256, H = 96, 64 steps with S carried in HBM
+        D = W.DECODE
+        N, H = D["N"], D["H"]
+        S = W.decode_state(N, H, d, d, S_std=D["S_std"])
+        A = W.decode_log_scale(H)
+        toks = [W.decode_step_inputs(N, H, d, d, s, A=A) for s in range(4)]
+        outd = torch.empty((N, H, d), dtype=torch.bfloat16, device="cuda")
+        optd = K.make_opts(torch.bfloat16)
+        it = [0]
+
+        def dstep():
+            t = toks[it[0] % 4]
+            it[0] += 1
+            K.kda_recurrent_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, outd, optd)
+        for _ in range(3):
+            dstep()
+        ms = statistics.median(time_calls(dstep, D["steps"]))
+        nbytes = N * H * (2 * d * d * 4 + token_head_bytes(d))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        rows["decode_step"] = {"ms": ms, "GB_per_s": gbs, "bytes_per_step": nbytes,
+                               "frac_of_hbm": gbs / hbm_peak, "steps": D["steps"],
+                               "note": "state 3.2 GB > L2, no flush needed"}
+        del S, toks, outd
+        torch.cuda.empty_cache()
+
+        # a6: Complex-KDA vs unsigned KDA at B=8, T=8192, H=32
+        cfg = W.WORKLOADS["ckda"]
+        res = {}
+        for cplx in (True, False):
+            x = W.chunk_inputs(cfg["B"], cfg["T"], cfg["H"], d, d, dtype=torch.bfloat16,
+                               S0_std=cfg["S0_std"], seed=0, complex_gate=cplx)
+            o0 = K.make_opts(torch.bfloat16, complex_gate=cplx)
+            wsz = K.kda_chunk_workspace_bytes(cfg["B"], cfg["T"], cfg["H"], d, d, o0)
+            ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device="cuda")
+            o = K.make_opts(torch.bfloat16, complex_gate=cplx, workspace=ws)
+            out = torch.empty_like(x["v"])
+            S_T = torch.empty((cfg["B"], cfg["H"], d, d), dtype=torch.float32, device="cuda")
+            fn = lambda: K.kda_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], out, S_T, o)
+            fn()
+            ms = statistics.median(time_calls(fn, 3))
+            th = cfg["B"] * cfg["T"] * cfg["H"]
+            nbytes = th * token_head_bytes(d) + cfg["B"] * cfg["H"] * 2 * d * d * 4
+            res["ckda" if cplx else "kda"] = {
+                "ms": ms, "tokens_per_s": cfg["B"] * cfg["T"] / (ms * 1e-3),
+                "frac_of_hbm_roofline": (nbytes / (ms * 1e-3) / 1e9) / hbm_peak}
+            del x, ws, out, S_T
+            torch.cuda.empty_cache()
+        res["ckda_over_kda_throughput"] = res["kda"]["ms"] / res["ckda"]["ms"]
+        rows["complex_kda_B8_T8192_H32"] = res
+    finally:
+        W.set_device("cpu")
+    return rows
+
+
+def run_ours(args, ws, rank, local):
+    import gated_delta_rule_73_b200 as K
+    dev = torch.device("cuda", local)
+    hbm_peak, tf_peak, peak_kind = peaks()
+    cfg = W.WORKLOADS["prefill"]
+    B, T, H, dk, dv = cfg["B"], cfg["T"], cfg["H"], cfg["dk"], cfg["dv"]
+    x = W.chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, S0_std=cfg["S0_std"], seed=rank)
+    names = ("q", "k", "v", "g", "beta", "S0")
+    host = {n: x[n].pin_memory() for n in names}
+    d = {n: x[n].to(dev) for n in names}
+    out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    opts0 = K.make_opts(torch.bfloat16)
+    wsz = K.kda_chunk_workspace_bytes(B, T, H, dk, dv, opts0)
+    wsb = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    max_launch = 4
+    # per-step event arrays: events[i] before launch i, events[L] after the last
+    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(max_launch + 1)]
+              for _ in range(args.steps)]
+    for evs in evsets:
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+
+    def call(evs=None):
+        o = K.make_opts(torch.bfloat16, workspace=wsb, events=evs)
+        K.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], out, S_T, o)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize()
+    # launches per call: count events written (those whose timestamps advance)
+    probe = [torch.cuda.Event(enable_timing=True) for _ in range(max_launch + 1)]
+    for e in probe:
+        e.record()
+    torch.cuda.synchronize()
+    t_mark = torch.cuda.Event(enable_timing=True)
+    t_mark.record()
+    call(probe)
+    torch.cuda.synchronize()
+    launches = sum(1 for e in probe[1:] if t_mark.elapsed_time(e) > 0.0)
+
+    sampler = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with sampler:
+        w0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            call(evsets[i])
+        torch.cuda.synchronize()
+        w1 = time.perf_counter()
+    barrier(ws)
+    step_ms = [evs[0].elapsed_time(evs[launches]) for evs in evsets]
+    kern_ms = [[evs[j].elapsed_time(evs[j + 1]) for evs in evsets] for j in range(launches)]
+    total_ms = sum(step_ms)
+    total_ms_max = max_over_ranks(total_ms, ws)
+    ms_per_step = total_ms_max / args.steps
+    tokens_per_step = B * T
+    value = ws * tokens_per_step * args.steps / (total_ms_max * 1e-3)
+
+    # roofline of the step's kernels (the chunk path's algorithmic bytes)
+    alg_bytes = B * T * H * token_head_bytes(dk) + B * H * 2 * dk * dv * 4
+    alg_flops = PREFILL_FLOP_PER_TOKEN_HEAD * B * T * H
+    mean_k = [statistics.mean(km) for km in kern_ms]
+    dom = max(range(launches), key=lambda j: mean_k[j])
+    achieved = alg_bytes / (statistics.mean(step_ms) * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None, "peak_kind": peak_kind,
+                "algorithmic_bytes_per_step": alg_bytes, "algorithmic_flops_per_step": alg_flops,
+                "tensor_frac_of_bf16_peak": alg_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / tf_peak,
+                "kernel_ms": mean_k, "dominant_launch": dom,
+                "note": "achieved = algorithmic bytes of the whole call / its device time"}
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hS = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+
+    def e2e_step():
+        for n in names:
+            d[n].copy_(host[n], non_blocking=True)
+        call()
+        hout.copy_(out, non_blocking=True)
+        hS.copy_(S_T, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = time_calls(e2e_step, args.steps, flush)
+    e2e_max = max_over_ranks(sum(e2e_ms), ws)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = hout.numel() * hout.element_size() + hS.numel() * hS.element_size()
+    e2e = {"value": ws * tokens_per_step * args.steps / (e2e_max * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prefill (chunk_kda fwd) B=1 T=4096 H=16 dk=dv=128 bf16, FP32 state",
+                       "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+                       "l2": "256 MiB buffer written between timed steps",
+                       "parallelism": f"replicas x{ws}: each rank runs its own batch, no collective"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches * args.steps,
+            "clocks": sampler.summary(), "wall_s_timed": w1 - w0}
+    if ws == 1 and rank == 0 and not args.no_rows:
+        line["rows"] = rows_n1(K, flush, hbm_peak)
+    if ws == 1 and rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline_prefill()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    ws, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, ws, rank)
+        return run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,12 @@
+"""B200-native (sm_100a) Kimi Delta Attention hot path.
+
+The product is the C-ABI library ``libkda_b200.so`` (declared in
+``include/kda.h``); this package holds its CUDA sources (``csrc/``), the
+in-tree build (``build.py``) and a thin ctypes binding (``kda.py``).
+"""
+from .kda import (  # noqa: F401
+    KDA_BF16, KDA_F32, KDA_QK_L2NORM, KDA_COMPLEX, KdaError, kda_opts, make_opts,
+    kda_chunk_fwd, kda_recurrent_step, kda_chunk_fwd_prologue, kda_chunk_workspace_bytes,
+    kda_prologue_workspace_bytes, kda_abi_version, status_string, chunk_fwd, recurrent_step,
+    chunk_fwd_prologue, LIB_PATH,
+)

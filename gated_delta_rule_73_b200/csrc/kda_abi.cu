@@ -1,0 +1,245 @@
+// kda_abi.cu -- the C ABI: argument checks, workspace sizing and dispatch.
+//
+// Every check runs on the host before the first CUDA call, so a rejected call
+// touches no device state.  See include/kda.h for the contract.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/kda.h"
+#include "kda_internal.h"
+
+using namespace kda;
+
+namespace {
+
+constexpr size_t kAlignWs = 256;
+constexpr long long kMaxElems = 1LL << 40;   // refuse sizes whose byte offsets could overflow
+
+kda_opts resolve(const kda_opts *o) {
+    kda_opts r;
+    memset(&r, 0, sizeof(r));
+    r.dtype = KDA_BF16;
+    r.flags = KDA_QK_L2NORM;
+    r.scale = 1.0f;
+    if (o) r = *o;
+    return r;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int check_opts(const kda_opts &o) {
+    if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
+    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX)) return KDA_ERR_ARG;
+    if (!isfinite(o.scale)) return KDA_ERR_ARG;
+    if (o.n_events < 0 || (o.n_events > 0 && !o.events)) return KDA_ERR_ARG;
+    return KDA_OK;
+}
+
+int check_dims(long long B, long long T, long long H, int dk, int dv) {
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    const long long d = dk > dv ? dk : dv;
+    if (B > 0 && T > 0 && H > 0) {
+        if (B > kMaxElems / T) return KDA_ERR_SHAPE;
+        const long long bt = B * T;
+        if (bt > kMaxElems / H) return KDA_ERR_SHAPE;
+        if (bt * H > kMaxElems / d) return KDA_ERR_SHAPE;
+    }
+    if (B * H > 65535) return KDA_ERR_UNSUPPORTED;   // grid y of the chunk kernels
+    return KDA_OK;
+}
+
+KernelFlags kflags(const kda_opts &o) {
+    KernelFlags f;
+    f.l2norm = (o.flags & KDA_QK_L2NORM) ? 1 : 0;
+    f.complex_gate = (o.flags & KDA_COMPLEX) ? 1 : 0;
+    f.scale = o.scale;
+    return f;
+}
+
+size_t chunk_ws(int B, int T, int H, int dk, int dv) {
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    return round_up(chunk_ref_workspace_bytes(B, T, H, dk, dv), kAlignWs);
+}
+
+size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, size_t *off) {
+    // off[0..5]: qc, kc, vc, g, beta, chunk workspace
+    const size_t rows = (size_t)B * T * H;
+    size_t o = 0;
+    off[0] = o; o = round_up(o + rows * dk * 4, kAlignWs);
+    off[1] = o; o = round_up(o + rows * dk * 4, kAlignWs);
+    off[2] = o; o = round_up(o + rows * dv * 4, kAlignWs);
+    off[3] = o; o = round_up(o + rows * dk * 4, kAlignWs);
+    off[4] = o; o = round_up(o + rows * 4, kAlignWs);
+    off[5] = o; o += chunk_ws(B, T, H, dk, dv);
+    return o;
+}
+
+int finish_identity(const float *S0, float *S_T, int B, int H, int dk, int dv, cudaStream_t st) {
+    if (!S_T || B == 0 || H == 0) return KDA_OK;
+    const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+    cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, st)
+                       : cudaMemsetAsync(S_T, 0, bytes, st);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int run_chunk(ChunkArgs &a, cudaStream_t st) {
+    int launches = 0;
+    a.launch_idx = &launches;
+    cudaError_t e = launch_chunk_ref(a, st);
+    if (e == cudaSuccess && a.events && launches < a.n_events) cudaEventRecord(a.events[launches], st);
+    if (e == cudaErrorInvalidValue) return KDA_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_abi_version(void) { return 100; }
+
+const char *kda_status_string(int s) {
+    switch (s) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_ARG: return "invalid argument (NULL pointer, negative size or unknown flag)";
+        case KDA_ERR_SHAPE: return "inconsistent or overflowing sizes";
+        case KDA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case KDA_ERR_UNSUPPORTED: return "unsupported configuration (dk/dv must be 64 or 128)";
+        case KDA_ERR_CUDA: return "CUDA launch or copy failed";
+        case KDA_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, const kda_opts *opts) {
+    const kda_opts o = resolve(opts);
+    if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
+    return chunk_ws(B, T, H, dk, dv);
+}
+
+size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, const kda_opts *opts) {
+    const kda_opts o = resolve(opts);
+    if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    size_t off[6];
+    return prologue_ws_parts(B, T, H, dk, dv, off);
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  const float *S0, void *out, float *S_T, int B, int T, int H, int dk, int dv,
+                  const kda_opts *opts, cudaStream_t stream) {
+    const kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if ((s = check_dims(B, T, H, dk, dv)) != KDA_OK) return s;
+    if (B == 0 || H == 0) return KDA_OK;
+    if (T == 0) {
+        if (!aligned16(S0) || !aligned16(S_T)) return KDA_ERR_ALIGN;
+        return finish_identity(S0, S_T, B, H, dk, dv, stream);
+    }
+    if (!q || !k || !v || !g || !beta || !out) return KDA_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, out, S_T, o.workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    const size_t need = chunk_ws(B, T, H, dk, dv);
+    if (need > 0 && (!o.workspace || o.workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+
+    ChunkArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+    const Elt t = o.dtype == KDA_BF16 ? Elt::BF16 : Elt::F32;
+    a.t_qkv = a.t_g = a.t_beta = a.t_out = t;
+    a.S0 = S0; a.out = out; a.S_T = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+    a.fl = kflags(o);
+    a.workspace = o.workspace; a.workspace_bytes = o.workspace_bytes;
+    a.events = o.events; a.n_events = o.n_events;
+    return run_chunk(a, stream);
+}
+
+int kda_recurrent_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                       float *S, void *out, int N, int H, int dk, int dv, const kda_opts *opts,
+                       cudaStream_t stream) {
+    const kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if (N < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    const long long units = (long long)N * H;
+    if (units == 0) return KDA_OK;
+    if (units > 0x7fffffffLL) return KDA_ERR_SHAPE;
+    if (!q || !k || !v || !g || !beta || !S || !out) return KDA_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
+    a.units = units; a.dk = dk; a.dv = dv;
+    a.bf16 = o.dtype == KDA_BF16;
+    a.fl = kflags(o);
+    if (o.events && o.n_events > 0) cudaEventRecord(o.events[0], stream);
+    cudaError_t e = launch_decode(a, stream);
+    if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
+                           const void *conv_w, const void *z, const float *A,
+                           const float *beta_logit, const float *S0, void *out, float *S_T, int B,
+                           int T, int H, int dk, int dv, const kda_opts *opts, cudaStream_t stream) {
+    kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if ((s = check_dims(B, T, H, dk, dv)) != KDA_OK) return s;
+    if (o.flags & KDA_COMPLEX) return KDA_ERR_UNSUPPORTED;
+    if (dk != dv) return KDA_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return KDA_OK;
+    if (T == 0) {
+        if (!aligned16(S0) || !aligned16(S_T)) return KDA_ERR_ALIGN;
+        return finish_identity(S0, S_T, B, H, dk, dv, stream);
+    }
+    if (!q_pre || !k_pre || !v_pre || !conv_w || !z || !A || !beta_logit || !out) return KDA_ERR_ARG;
+    const void *ptrs[] = {q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, out, S_T, o.workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    size_t off[6];
+    const size_t need = prologue_ws_parts(B, T, H, dk, dv, off);
+    if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    char *ws = (char *)o.workspace;
+
+    PrologueArgs p;
+    p.q_pre = q_pre; p.k_pre = k_pre; p.v_pre = v_pre; p.conv_w = conv_w; p.z = z;
+    p.A = A; p.beta_logit = beta_logit;
+    p.bf16 = o.dtype == KDA_BF16;
+    p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
+    p.qc = (float *)(ws + off[0]); p.kc = (float *)(ws + off[1]); p.vc = (float *)(ws + off[2]);
+    p.g = (float *)(ws + off[3]); p.beta = (float *)(ws + off[4]);
+
+    int launches = 0;
+    if (o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
+    ++launches;
+    cudaError_t e = launch_prologue(p, stream);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+
+    ChunkArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = p.qc; a.k = p.kc; a.v = p.vc; a.g = p.g; a.beta = p.beta;
+    a.t_qkv = a.t_g = a.t_beta = Elt::F32;
+    a.t_out = p.bf16 ? Elt::BF16 : Elt::F32;
+    a.S0 = S0; a.out = out; a.S_T = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+    o.flags |= KDA_QK_L2NORM;
+    a.fl = kflags(o);
+    a.workspace = ws + off[5];
+    a.workspace_bytes = need - off[5];
+    a.events = o.events; a.n_events = o.n_events;
+    a.launch_idx = &launches;
+    e = launch_chunk_ref(a, stream);
+    if (e == cudaSuccess && o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

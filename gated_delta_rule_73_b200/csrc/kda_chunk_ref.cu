@@ -1,0 +1,341 @@
+// kda_chunk_ref.cu -- FP32 CUDA-core chunkwise KDA forward (two phases).
+//
+// This is the exact-FP32 path: it serves fp32 inputs (where tensor-core TF32
+// or BF16 operands would not meet a 1e-4 relative bound) and any shape the
+// tensor-core kernel does not take.  It follows the chunkwise form of page
+// "Kimi K3 模型结构（2）：序列维度（下），chunkwise 并行与下界衰减" (Q&A items on
+// the chunkwise algorithm and on the intra-chunk matrix A):
+//
+// Phase 1 (one CTA per chunk and head, all chunks in parallel):
+//   gamma_r = sum_{s<=r} log|alpha_s| per key channel (chunk-local),
+//   sigma_r = prod_{s<=r} sign(alpha_s) (Complex-KDA; folded into q and k),
+//   A_kk[r,i] = beta_r sum_c k_rc k_ic e^{gamma_rc - gamma_ic}   (i < r)
+//   A_qk[r,i] =        sum_c q_rc k_ic e^{gamma_rc - gamma_ic}   (i <= r)
+//   Tm = (I + A_kk)^{-1} by forward substitution (the UT transform)
+//   W = Tm diag(beta) (K e^gamma),  U = Tm diag(beta) V    (WY vectors)
+//   Qg = Q e^gamma,  Kd = sigma_C K e^{gamma_C - gamma},  gC = sigma_C e^{gamma_C}
+// Every exponent above is <= 0, so nothing overflows in FP32.
+//
+// Phase 2 (one CTA per head and slice of value columns, chunks in order):
+//   V~ = U - W S;   O = scale (Qg S + A_qk V~);   S <- diag(gC) S + Kd^T V~
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+namespace {
+constexpr int C = kChunk;
+constexpr int CP = C + 1;
+
+__device__ __forceinline__ float ldx(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ldx(const __nv_bfloat16 *p, size_t i) { return to_f32(p[i]); }
+
+template <int DK, int DV>
+struct RefLayout {
+    static constexpr size_t per_chunk = (size_t)C * DK * 3 + (size_t)C * DV + (size_t)C * C + DK;
+    static constexpr size_t off_W = 0;
+    static constexpr size_t off_U = off_W + (size_t)C * DK;
+    static constexpr size_t off_Qg = off_U + (size_t)C * DV;
+    static constexpr size_t off_Kd = off_Qg + (size_t)C * DK;
+    static constexpr size_t off_A = off_Kd + (size_t)C * DK;
+    static constexpr size_t off_gC = off_A + (size_t)C * C;
+};
+
+template <int DK, int DV>
+constexpr size_t intra_smem_bytes() {
+    return sizeof(float) * ((size_t)C * (DK + 1) * 3 + (size_t)C * (DV + 1) + (size_t)C * CP * 3 +
+                            C + 2 * DK);
+}
+
+template <typename TQ, typename TG, typename TB, int DK, int DV>
+__global__ void __launch_bounds__(256)
+chunk_intra_kernel(const TQ *__restrict__ q, const TQ *__restrict__ k, const TQ *__restrict__ v,
+                   const TG *__restrict__ g, const TB *__restrict__ beta, int T, int H,
+                   int nchunks, KernelFlags fl, float *__restrict__ ws) {
+    constexpr int DKP = DK + 1, DVP = DV + 1;
+    using L = RefLayout<DK, DV>;
+    extern __shared__ float sm[];
+    float *Qs = sm;
+    float *Ks = Qs + C * DKP;
+    float *Gs = Ks + C * DKP;
+    float *Vs = Gs + C * DKP;
+    float *Akk = Vs + C * DVP;
+    float *Aqk = Akk + C * CP;
+    float *Tm = Aqk + C * CP;
+    float *bs = Tm + C * CP;
+    float *sgnC = bs + C;
+    float *gamC = sgnC + DK;
+
+    const int chunk = blockIdx.x, bh = blockIdx.y;
+    const int b = bh / H, h = bh % H;
+    const int t0 = chunk * C;
+    const int n = min(C, T - t0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int idx = tid; idx < C * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        float qv = 0.f, kv = 0.f, gv = fl.complex_gate ? 1.f : 0.f;
+        if (r < n) {
+            const size_t row = ((size_t)b * T + t0 + r) * H + h;
+            qv = ldx(q, row * DK + c);
+            kv = ldx(k, row * DK + c);
+            gv = ldx(g, row * DK + c);
+        }
+        Qs[r * DKP + c] = qv;
+        Ks[r * DKP + c] = kv;
+        Gs[r * DKP + c] = gv;
+    }
+    for (int idx = tid; idx < C * DV; idx += 256) {
+        const int r = idx / DV, c = idx % DV;
+        float vv = 0.f;
+        if (r < n) vv = ldx(v, (((size_t)b * T + t0 + r) * H + h) * DV + c);
+        Vs[r * DVP + c] = vv;
+    }
+    if (tid < C) bs[tid] = tid < n ? ldx(beta, ((size_t)b * T + t0 + tid) * H + h) : 0.f;
+    __syncthreads();
+
+    if (fl.l2norm) {
+        for (int r = warp; r < n; r += 8) {
+            float sq = 0.f, sk = 0.f;
+            for (int c = lane; c < DK; c += 32) {
+                sq += Qs[r * DKP + c] * Qs[r * DKP + c];
+                sk += Ks[r * DKP + c] * Ks[r * DKP + c];
+            }
+            sq = warp_sum(sq);
+            sk = warp_sum(sk);
+            const float fq = rsqrtf(sq + kL2Eps), fk = rsqrtf(sk + kL2Eps);
+            for (int c = lane; c < DK; c += 32) {
+                Qs[r * DKP + c] *= fq;
+                Ks[r * DKP + c] *= fk;
+            }
+        }
+        __syncthreads();
+    }
+
+    // chunk-local cumulative log-decay (and sign parity for Complex-KDA)
+    if (tid < DK) {
+        const int c = tid;
+        float gam = 0.f, sg = 1.f;
+        for (int r = 0; r < n; ++r) {
+            const float a = Gs[r * DKP + c];
+            float lg = a;
+            if (fl.complex_gate) {
+                lg = logf(fabsf(a));
+                if (a < 0.f) sg = -sg;
+                Qs[r * DKP + c] *= sg;
+                Ks[r * DKP + c] *= sg;
+            }
+            gam += lg;
+            Gs[r * DKP + c] = gam;
+        }
+        for (int r = n; r < C; ++r) Gs[r * DKP + c] = gam;
+        sgnC[c] = sg;
+        gamC[c] = gam;
+    }
+    __syncthreads();
+
+    // A_kk (strict lower, with beta_r) and A_qk (lower with diagonal)
+    for (int p = tid; p < C * C; p += 256) {
+        const int r = p / C, i = p % C;
+        float akk = 0.f, aqk = 0.f;
+        if (i <= r && r < n) {
+            for (int c = 0; c < DK; ++c) {
+                const float e = expf(Gs[r * DKP + c] - Gs[i * DKP + c]);
+                const float kk = Ks[i * DKP + c] * e;
+                akk += Ks[r * DKP + c] * kk;
+                aqk += Qs[r * DKP + c] * kk;
+            }
+        }
+        Akk[r * CP + i] = (i < r) ? bs[r] * akk : 0.f;
+        Aqk[r * CP + i] = aqk;
+    }
+    __syncthreads();
+
+    // Tm = (I + A_kk)^{-1}: column j solves (I + A_kk) x = e_j
+    if (tid < C) {
+        const int j = tid;
+        for (int r = 0; r < C; ++r) {
+            float acc = (r == j) ? 1.f : 0.f;
+            for (int i = j; i < r; ++i) acc -= Akk[r * CP + i] * Tm[i * CP + j];
+            Tm[r * CP + j] = (r < j) ? 0.f : acc;
+        }
+    }
+
+    float *wsb = ws + ((size_t)bh * nchunks + chunk) * L::per_chunk;
+    for (int idx = tid; idx < C * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        const float gr = Gs[r * DKP + c];
+        wsb[L::off_Qg + idx] = Qs[r * DKP + c] * expf(gr);
+        wsb[L::off_Kd + idx] = sgnC[c] * Ks[r * DKP + c] * expf(gamC[c] - gr);
+    }
+    for (int idx = tid; idx < C * C; idx += 256) wsb[L::off_A + idx] = Aqk[(idx / C) * CP + idx % C];
+    if (tid < DK) wsb[L::off_gC + tid] = sgnC[tid] * expf(gamC[tid]);
+    __syncthreads();
+    // EK = diag(beta) K e^gamma into the Q buffer; V <- diag(beta) V
+    for (int idx = tid; idx < C * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        Qs[r * DKP + c] = bs[r] * Ks[r * DKP + c] * expf(Gs[r * DKP + c]);
+    }
+    for (int idx = tid; idx < C * DV; idx += 256) {
+        const int r = idx / DV, c = idx % DV;
+        Vs[r * DVP + c] *= bs[r];
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * DK; idx += 256) {
+        const int r = idx / DK, c = idx % DK;
+        float acc = 0.f;
+        for (int i = 0; i <= r; ++i) acc += Tm[r * CP + i] * Qs[i * DKP + c];
+        wsb[L::off_W + idx] = acc;
+    }
+    for (int idx = tid; idx < C * DV; idx += 256) {
+        const int r = idx / DV, c = idx % DV;
+        float acc = 0.f;
+        for (int i = 0; i <= r; ++i) acc += Tm[r * CP + i] * Vs[i * DVP + c];
+        wsb[L::off_U + idx] = acc;
+    }
+}
+
+template <int DK, int DVS>
+constexpr size_t scan_smem_bytes() {
+    return sizeof(float) * ((size_t)C * (DK + 1) * 3 + (size_t)DK * (DVS + 1) +
+                            (size_t)C * (DVS + 1) * 3 + (size_t)C * CP + DK);
+}
+
+template <typename TO, int DK, int DV, int DVS>
+__global__ void __launch_bounds__(256)
+chunk_scan_kernel(const float *__restrict__ ws, const float *__restrict__ S0, TO *__restrict__ out,
+                  float *__restrict__ S_T, int T, int H, int nchunks, float scale) {
+    constexpr int DKP = DK + 1, SP = DVS + 1;
+    using L = RefLayout<DK, DV>;
+    extern __shared__ float sm[];
+    float *Ws = sm;
+    float *Qgs = Ws + C * DKP;
+    float *Kds = Qgs + C * DKP;
+    float *Ss = Kds + C * DKP;      // DK x SP
+    float *Vt = Ss + DK * SP;       // C x SP
+    float *Os = Vt + C * SP;
+    float *Us = Os + C * SP;
+    float *Aq = Us + C * SP;        // C x CP
+    float *gCs = Aq + C * CP;       // DK
+
+    const int bh = blockIdx.x, j0 = blockIdx.y * DVS;
+    const int b = bh / H, h = bh % H;
+    const int tid = threadIdx.x;
+
+    for (int idx = tid; idx < DK * DVS; idx += 256) {
+        const int c = idx / DVS, j = idx % DVS;
+        Ss[c * SP + j] = S0 ? S0[((size_t)bh * DK + c) * DV + j0 + j] : 0.f;
+    }
+    for (int ch = 0; ch < nchunks; ++ch) {
+        const int t0 = ch * C;
+        const int n = min(C, T - t0);
+        const float *wsb = ws + ((size_t)bh * nchunks + ch) * L::per_chunk;
+        for (int idx = tid; idx < C * DK; idx += 256) {
+            const int r = idx / DK, c = idx % DK;
+            Ws[r * DKP + c] = wsb[L::off_W + idx];
+            Qgs[r * DKP + c] = wsb[L::off_Qg + idx];
+            Kds[r * DKP + c] = wsb[L::off_Kd + idx];
+        }
+        for (int idx = tid; idx < C * DVS; idx += 256) {
+            const int r = idx / DVS, j = idx % DVS;
+            Us[r * SP + j] = wsb[L::off_U + (size_t)r * DV + j0 + j];
+        }
+        for (int idx = tid; idx < C * C; idx += 256) Aq[(idx / C) * CP + idx % C] = wsb[L::off_A + idx];
+        if (tid < DK) gCs[tid] = wsb[L::off_gC + tid];
+        __syncthreads();
+        for (int idx = tid; idx < C * DVS; idx += 256) {
+            const int r = idx / DVS, j = idx % DVS;
+            float w = 0.f, o = 0.f;
+            for (int c = 0; c < DK; ++c) {
+                const float s = Ss[c * SP + j];
+                w += Ws[r * DKP + c] * s;
+                o += Qgs[r * DKP + c] * s;
+            }
+            Vt[r * SP + j] = Us[r * SP + j] - w;
+            Os[r * SP + j] = o;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * DVS; idx += 256) {
+            const int r = idx / DVS, j = idx % DVS;
+            if (r < n) {
+                float acc = Os[r * SP + j];
+                for (int i = 0; i <= r; ++i) acc += Aq[r * CP + i] * Vt[i * SP + j];
+                out[(((size_t)b * T + t0 + r) * H + h) * DV + j0 + j] = from_f32<TO>(scale * acc);
+            }
+        }
+        for (int idx = tid; idx < DK * DVS; idx += 256) {
+            const int c = idx / DVS, j = idx % DVS;
+            float acc = gCs[c] * Ss[c * SP + j];
+            for (int r = 0; r < n; ++r) acc += Kds[r * DKP + c] * Vt[r * SP + j];
+            Ss[c * SP + j] = acc;
+        }
+        __syncthreads();
+    }
+    if (S_T) {
+        for (int idx = tid; idx < DK * DVS; idx += 256) {
+            const int c = idx / DVS, j = idx % DVS;
+            S_T[((size_t)bh * DK + c) * DV + j0 + j] = Ss[c * SP + j];
+        }
+    }
+}
+
+template <typename TQ, typename TG, typename TB, int DK, int DV>
+cudaError_t launch_intra(const ChunkArgs &a, int nchunks, float *ws, cudaStream_t st) {
+    auto kern = chunk_intra_kernel<TQ, TG, TB, DK, DV>;
+    const size_t smem = intra_smem_bytes<DK, DV>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mark_launch(a, st);
+    dim3 grid(nchunks, a.B * a.H);
+    kern<<<grid, 256, smem, st>>>((const TQ *)a.q, (const TQ *)a.k, (const TQ *)a.v, (const TG *)a.g,
+                                  (const TB *)a.beta, a.T, a.H, nchunks, a.fl, ws);
+    return cudaGetLastError();
+}
+
+template <typename TO, int DK, int DV>
+cudaError_t launch_scan(const ChunkArgs &a, int nchunks, const float *ws, cudaStream_t st) {
+    constexpr int DVS = 32;
+    auto kern = chunk_scan_kernel<TO, DK, DV, DVS>;
+    const size_t smem = scan_smem_bytes<DK, DVS>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mark_launch(a, st);
+    dim3 grid(a.B * a.H, DV / DVS);
+    kern<<<grid, 256, smem, st>>>(ws, a.S0, (TO *)a.out, a.S_T, a.T, a.H, nchunks, a.fl.scale);
+    return cudaGetLastError();
+}
+
+template <int DK, int DV>
+cudaError_t launch_ref_dims(const ChunkArgs &a, cudaStream_t st) {
+    const int nchunks = (a.T + C - 1) / C;
+    float *ws = (float *)a.workspace;
+    cudaError_t e;
+    // phase 1: input element types
+    if (a.t_qkv == Elt::BF16 && a.t_g == Elt::BF16 && a.t_beta == Elt::BF16)
+        e = launch_intra<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16, DK, DV>(a, nchunks, ws, st);
+    else if (a.t_qkv == Elt::F32 && a.t_g == Elt::F32 && a.t_beta == Elt::F32)
+        e = launch_intra<float, float, float, DK, DV>(a, nchunks, ws, st);
+    else
+        return cudaErrorInvalidValue;
+    if (e != cudaSuccess) return e;
+    // phase 2: output element type
+    if (a.t_out == Elt::BF16) e = launch_scan<__nv_bfloat16, DK, DV>(a, nchunks, ws, st);
+    else e = launch_scan<float, DK, DV>(a, nchunks, ws, st);
+    return e;
+}
+}  // namespace
+
+size_t chunk_ref_workspace_bytes(int B, int T, int H, int dk, int dv) {
+    const size_t nchunks = ((size_t)T + C - 1) / C;
+    const size_t per = (size_t)C * dk * 3 + (size_t)C * dv + (size_t)C * C + dk;
+    return sizeof(float) * per * nchunks * (size_t)B * (size_t)H;
+}
+
+cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st) {
+    if (a.dk == 128 && a.dv == 128) return launch_ref_dims<128, 128>(a, st);
+    if (a.dk == 128 && a.dv == 64) return launch_ref_dims<128, 64>(a, st);
+    if (a.dk == 64 && a.dv == 128) return launch_ref_dims<64, 128>(a, st);
+    return launch_ref_dims<64, 64>(a, st);
+}
+
+}  // namespace kda

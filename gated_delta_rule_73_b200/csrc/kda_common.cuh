@@ -1,0 +1,34 @@
+// kda_common.cuh -- small device helpers shared by the KDA kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kda {
+
+constexpr float kL2Eps = 1e-6f;   // epsilon inside the square root of the L2 norm
+constexpr int kChunk = 64;        // chunk length C
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Options the kernels see (a device-side copy of the host flags).
+struct KernelFlags {
+    int l2norm;
+    int complex_gate;
+    float scale;
+};
+
+}  // namespace kda

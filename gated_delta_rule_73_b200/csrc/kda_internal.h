@@ -1,0 +1,59 @@
+// kda_internal.h -- launch descriptors passed from the C ABI layer to kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include "kda_common.cuh"
+
+namespace kda {
+
+struct DecodeArgs {
+    const void *q, *k, *v, *g, *beta;
+    float *S;
+    void *out;
+    long long units;   // N * H
+    int dk, dv;
+    bool bf16;
+    KernelFlags fl;
+};
+
+// Element types of the chunk path's inputs.
+enum class Elt : int { BF16 = 0, F32 = 1 };
+
+struct ChunkArgs {
+    const void *q, *k, *v, *g, *beta;   // inputs ([B,T,H,*])
+    Elt t_qkv, t_g, t_beta, t_out;
+    const float *S0;                     // nullable
+    void *out;
+    float *S_T;                          // nullable
+    int B, T, H, dk, dv;
+    KernelFlags fl;
+    void *workspace;
+    size_t workspace_bytes;
+    cudaEvent_t *events;
+    int n_events;
+    int *launch_idx;                     // running launch counter for events
+};
+
+struct PrologueArgs {
+    const void *q_pre, *k_pre, *v_pre, *conv_w, *z;
+    const float *A, *beta_logit;
+    bool bf16;
+    int B, T, H, dk, dv;
+    float *qc, *kc, *vc, *g, *beta;      // FP32 outputs in the workspace
+};
+
+// Workspace of the FP32 two-phase chunk path.
+size_t chunk_ref_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st);
+cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st);
+
+// Record a.events[*a.launch_idx] (if requested) and advance the counter.
+inline void mark_launch(const ChunkArgs &a, cudaStream_t st) {
+    if (a.events && a.launch_idx && *a.launch_idx < a.n_events)
+        cudaEventRecord(a.events[*a.launch_idx], st);
+    if (a.launch_idx) ++*a.launch_idx;
+}
+
+}  // namespace kda

@@ -1,0 +1,216 @@
+"""Thin ctypes binding of ``libkda_b200.so`` (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it checks tensor dtypes/devices/contiguity, reads the
+sizes off the shapes, passes raw device pointers and the current CUDA stream,
+and turns a negative status into ``KdaError``.  PyTorch only provides device
+memory, streams and events.  If the shared library is missing the import
+fails loudly -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
+
+KDA_BF16, KDA_F32 = 0, 1
+KDA_QK_L2NORM, KDA_COMPLEX = 1, 2
+STATUS = {0: "KDA_OK", -1: "KDA_ERR_ARG", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_ALIGN",
+          -4: "KDA_ERR_UNSUPPORTED", -5: "KDA_ERR_CUDA", -6: "KDA_ERR_TIMEOUT",
+          -7: "KDA_ERR_WORKSPACE"}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({status_string(status)})")
+
+
+class kda_opts(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("flags", ctypes.c_uint), ("scale", ctypes.c_float),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("events", ctypes.POINTER(ctypes.c_void_p)), ("n_events", ctypes.c_int)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m gated_delta_rule_73_b200.build` (no CPU fallback exists)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, ip, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    op = ctypes.POINTER(kda_opts)
+    lib.kda_chunk_fwd.argtypes = [vp] * 8 + [ip] * 5 + [op, vp]
+    lib.kda_chunk_fwd.restype = ip
+    lib.kda_recurrent_step.argtypes = [vp] * 7 + [ip] * 4 + [op, vp]
+    lib.kda_recurrent_step.restype = ip
+    lib.kda_chunk_fwd_prologue.argtypes = [vp] * 10 + [ip] * 5 + [op, vp]
+    lib.kda_chunk_fwd_prologue.restype = ip
+    lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
+    lib.kda_chunk_workspace_bytes.restype = sz
+    lib.kda_prologue_workspace_bytes.argtypes = [ip] * 5 + [op]
+    lib.kda_prologue_workspace_bytes.restype = sz
+    lib.kda_status_string.argtypes = [ip]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_abi_version.argtypes = []
+    lib.kda_abi_version.restype = ip
+    return lib
+
+
+_lib = _load()
+
+
+def status_string(status: int) -> str:
+    return _lib.kda_status_string(int(status)).decode()
+
+
+def kda_abi_version() -> int:
+    return _lib.kda_abi_version()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return KDA_BF16
+    if t == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported activation dtype {t}; use bfloat16 or float32")
+
+
+def make_opts(dtype: torch.dtype = torch.bfloat16, *, l2norm: bool = True, complex_gate: bool = False,
+              scale: float = 1.0, workspace: torch.Tensor | None = None, events=None) -> kda_opts:
+    o = kda_opts()
+    o.dtype = _dtype_code(dtype)
+    o.flags = (KDA_QK_L2NORM if l2norm else 0) | (KDA_COMPLEX if complex_gate else 0)
+    o.scale = float(scale)
+    if workspace is not None:
+        o.workspace = workspace.data_ptr()
+        o.workspace_bytes = workspace.numel() * workspace.element_size()
+    if events:
+        arr = (ctypes.c_void_p * len(events))()
+        for i, ev in enumerate(events):
+            if not ev.cuda_event:
+                ev.record()          # torch creates the CUDA event lazily
+            arr[i] = ev.cuda_event
+        o.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+        o.n_events = len(events)
+        o._keep = arr                # keep the array alive with the struct
+    return o
+
+
+def _ptr(t, name, dtype=None, device_required=True):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if device_required and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def kda_chunk_workspace_bytes(B, T, H, dk, dv, opts: kda_opts | None = None) -> int:
+    return int(_lib.kda_chunk_workspace_bytes(B, T, H, dk, dv, ctypes.byref(opts) if opts else None))
+
+
+def kda_prologue_workspace_bytes(B, T, H, dk, dv, opts: kda_opts | None = None) -> int:
+    return int(_lib.kda_prologue_workspace_bytes(B, T, H, dk, dv, ctypes.byref(opts) if opts else None))
+
+
+def kda_chunk_fwd(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_chunk_fwd``; q,k,g [B,T,H,dk], v,out [B,T,H,dv], beta [B,T,H]."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
+            _ptr(S_T, "S_T", torch.float32)]
+    st = _lib.kda_chunk_fwd(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_chunk_fwd", st)
+
+
+def kda_recurrent_step(q, k, v, g, beta, S, out, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_recurrent_step``; q,k,g [N,H,dk], v,out [N,H,dv], beta [N,H], S [N,H,dk,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(S, "S", torch.float32), _ptr(out, "out", dt)]
+    st = _lib.kda_recurrent_step(*args, N, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_recurrent_step", st)
+
+
+def kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, out, S_T,
+                           opts: kda_opts, stream=None) -> None:
+    """Call ``kda_chunk_fwd_prologue`` (raw branch inputs; see include/kda.h)."""
+    B, T, H, dk = q_pre.shape
+    dv = v_pre.shape[-1]
+    dt = q_pre.dtype
+    args = [_ptr(q_pre, "q_pre", dt), _ptr(k_pre, "k_pre", dt), _ptr(v_pre, "v_pre", dt),
+            _ptr(conv_w, "conv_w", dt), _ptr(z, "z", dt), _ptr(A, "A", torch.float32),
+            _ptr(beta_logit, "beta_logit", torch.float32), _ptr(S0, "S0", torch.float32),
+            _ptr(out, "out", dt), _ptr(S_T, "S_T", torch.float32)]
+    st = _lib.kda_chunk_fwd_prologue(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_chunk_fwd_prologue", st)
+
+
+# ------------------------------------------------------------------ conveniences
+def chunk_fwd(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False, scale=1.0,
+              workspace=None, out=None, S_T=None, stream=None):
+    """Allocate out / S_T / workspace with torch and run ``kda_chunk_fwd``."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale)
+    if workspace is None:
+        nbytes = kda_chunk_workspace_bytes(B, T, H, dk, dv, opts)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale,
+                     workspace=workspace)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    kda_chunk_fwd(q, k, v, g, beta, S0, out, S_T, opts, stream)
+    return out, S_T
+
+
+def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scale=1.0,
+                   out=None, stream=None):
+    """Run ``kda_recurrent_step`` (S updated in place); returns out."""
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale)
+    kda_recurrent_step(q, k, v, g, beta, S, out, opts, stream)
+    return out
+
+
+def chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0=None, *, scale=1.0,
+                       workspace=None, out=None, S_T=None, stream=None):
+    """Allocate and run ``kda_chunk_fwd_prologue``."""
+    B, T, H, dk = q_pre.shape
+    dv = v_pre.shape[-1]
+    opts = make_opts(q_pre.dtype, scale=scale)
+    if workspace is None:
+        nbytes = kda_prologue_workspace_bytes(B, T, H, dk, dv, opts)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q_pre.device)
+    opts = make_opts(q_pre.dtype, scale=scale, workspace=workspace)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q_pre.dtype, device=q_pre.device)
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q_pre.device)
+    kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, out, S_T, opts, stream)
+    return out, S_T

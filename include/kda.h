@@ -1,0 +1,173 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) library.
+ *
+ * The library computes the forward hot path of KDA for one GPU:
+ *
+ *   decay   St  = Diag(alpha_t) S_{t-1}               alpha_t per key channel
+ *   erase + write  S_t = St + beta_t k_t (v_t - St^T k_t)^T
+ *   read    o_t = scale * S_t^T q_t                   (post-write state)
+ *
+ * Page "Kimi K3 の KDA(1): KDA が Gated MLA と AttnRes とどのように連携するか",
+ * section 1.2.1 (decay -> erase -> write; the read sees S_t; q and k are L2
+ * normalised per head inside the kernel); page "GDN, KDA の整理", section
+ * "Kimi Delta Attention" (S_t in R^{dk x dv}, o_t = S_t^T q_t, per-channel
+ * decay D_t = Diag(alpha_t)).  Complex-KDA (signed gate in [-1, 1], beta in
+ * [0, 2]): page "Complex KDA: 理解并增强 Kimi Delta Attention 的表达能力".
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - Memory: every tensor pointer is DEVICE memory owned by the caller.  The
+ *    library never allocates or frees memory and keeps no state between calls.
+ *  - Asynchrony: work is enqueued on `stream`; the return value reports
+ *    argument and launch errors only.  Kernel faults surface at the caller's
+ *    next synchronisation.
+ *  - Errors: a negative status (see kda_status); no exception and no device
+ *    trap ever crosses the ABI.  Arguments are checked on the host before any
+ *    CUDA call is made.
+ *  - Alignment: every pointer must be 16-byte aligned (KDA_ERR_ALIGN).
+ *  - Layouts (contiguous, row-major, "BTHD"):
+ *        q, k, g      [B, T, H, dk]
+ *        v, out       [B, T, H, dv]
+ *        beta         [B, T, H]
+ *        S0, S_T, S   [B, H, dk, dv]  FP32, rows = key channels
+ *  - Element types: opts->dtype selects the type of q, k, v, g, beta and out
+ *    (bf16 or fp32).  The recurrent state is always FP32 and all arithmetic
+ *    is FP32 (or BF16 tensor-core operands with FP32 accumulation).
+ *  - Shapes: dk and dv must each be 64 or 128 (KDA_ERR_UNSUPPORTED otherwise).
+ *    T need not be a multiple of the 64-token chunk.  T == 0 is the identity:
+ *    S_T = S0 (zero when S0 is NULL).  B == 0 or H == 0 is a no-op.
+ */
+#ifndef KDA_B200_KDA_H
+#define KDA_B200_KDA_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of the activation tensors. */
+typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_ARG = -1,          /* NULL pointer, negative size, unknown flag bit */
+    KDA_ERR_SHAPE = -2,        /* inconsistent sizes, size overflow            */
+    KDA_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned             */
+    KDA_ERR_UNSUPPORTED = -4,  /* valid but not implemented (dk/dv, flags)     */
+    KDA_ERR_CUDA = -5,         /* a CUDA launch or copy reported an error      */
+    KDA_ERR_TIMEOUT = -6,      /* reserved: a bounded device wait gave up      */
+    KDA_ERR_WORKSPACE = -7     /* workspace missing or smaller than required   */
+} kda_status;
+
+/* Flag bits of kda_opts.flags. */
+enum {
+    KDA_QK_L2NORM = 1u,  /* q, k <- x / sqrt(sum x^2 + 1e-6) per head, in-kernel
+                            (use_qk_l2norm_in_kernel, "Kimi K3 の KDA(1)" 1.2.1) */
+    KDA_COMPLEX = 2u     /* Complex-KDA: `g` holds the signed gate alpha itself,
+                            |alpha| in [e^-5, 1], alpha != 0; beta in [0, 2]   */
+};
+
+/* Options.  Passing NULL means {KDA_BF16, KDA_QK_L2NORM, 1.0f, NULL, 0, NULL, 0}. */
+typedef struct {
+    kda_dtype dtype;        /* type of q, k, v, g, beta, out                  */
+    unsigned flags;         /* KDA_QK_L2NORM | KDA_COMPLEX                     */
+    float scale;            /* read-out scale; the pages use 1                 */
+    void *workspace;        /* device scratch, >= kda_*_workspace_bytes()     */
+    size_t workspace_bytes;
+    /* Optional instrumentation: when non-NULL, events[i] is recorded on
+       `stream` just before the i-th kernel launch of the call and
+       events[launches] right after the last one, for i < n_events. */
+    cudaEvent_t *events;
+    int n_events;
+} kda_opts;
+
+/*
+ * kda_chunk_fwd -- chunkwise-parallel forward (chunk_kda; training/prefill).
+ *
+ * Page "Kimi K3 模型结构（2）：序列维度（下），chunkwise 并行与下界衰减",
+ * Q&A items: the sequence is cut into chunks of C = 64 tokens, one state
+ * update per chunk, matmuls inside a chunk through the WY representation and
+ * one C x C triangular (UT) inverse; A = Tril[(Q*Gamma)(K/Gamma)^T] with its
+ * diagonal and O = (Gamma*Q) S + A V~.  The result equals the token
+ * recurrence above up to rounding.
+ *
+ *   q, k     [B,T,H,dk]  queries/keys (normalised in-kernel if KDA_QK_L2NORM)
+ *   v        [B,T,H,dv]  values
+ *   g        [B,T,H,dk]  log-decay g = log(alpha), expected in (-5, 0] for
+ *                        unsigned KDA (bounded decay); with KDA_COMPLEX, the
+ *                        signed gate alpha itself
+ *   beta     [B,T,H]     write strength (already through the sigmoid)
+ *   S0       [B,H,dk,dv] FP32 initial state, NULL means zero
+ *   out      [B,T,H,dv]  outputs o_t
+ *   S_T      [B,H,dk,dv] FP32 final state, NULL to skip
+ *   opts->workspace must hold kda_chunk_workspace_bytes(...) bytes (may be
+ *   NULL when that is 0).
+ */
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
+                  const void *beta, const float *S0, void *out, float *S_T,
+                  int B, int T, int H, int dk, int dv, const kda_opts *opts,
+                  cudaStream_t stream);
+
+/* Workspace bytes kda_chunk_fwd needs for these sizes and options. */
+size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv,
+                                 const kda_opts *opts);
+
+/*
+ * kda_recurrent_step -- one-token recurrent step (fused_recurrent_kda; decode).
+ *
+ * Page "Kimi K3 模型结构（2）", Q&A item on train/prefill vs decode: decode
+ * generates one token at a time with the recurrent form.  One call advances
+ * N independent sequences by one token, updating S in place.
+ *
+ *   q, k, g  [N,H,dk]   v, out [N,H,dv]   beta [N,H]
+ *   S        [N,H,dk,dv] FP32, read and overwritten with S_t
+ * Needs no workspace.
+ */
+int kda_recurrent_step(const void *q, const void *k, const void *v, const void *g,
+                       const void *beta, float *S, void *out, int N, int H, int dk,
+                       int dv, const kda_opts *opts, cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_prologue -- the branch prologue fused ahead of kda_chunk_fwd.
+ *
+ * Page "Kimi K3 の KDA(1)", section 1.2.1: q, k and v each pass a causal
+ * depthwise ShortConvolution (kernel 4, SiLU): every channel independent,
+ * the current token and the three before it (zero history before t = 0, no
+ * bias); the tap order is that of a causal Conv1d weight [channels, 4], tap 3
+ * multiplying the current token.  The decay is the bounded map
+ * g = -5 * sigmoid(exp(A_h) * z) (page "Kimi K3 模型结构（2）", Q&A on the
+ * decay function) and beta = sigmoid(beta_logit) in FP32 (section 1.2.1,
+ * `.float()` of b_proj).  q and k are then L2 normalised in the chunk kernel
+ * (KDA_QK_L2NORM is implied).
+ *
+ *   q_pre, k_pre [B,T,H,dk], v_pre [B,T,H,dv]   pre-conv activations (dtype)
+ *   conv_w       [3, H*dk, 4]  taps for q, k, v (dtype); needs dk == dv
+ *   z            [B,T,H,dk]   decay logits (dtype)
+ *   A            [H]          per-head log-scale A_h (FP32)
+ *   beta_logit   [B,T,H]      FP32
+ *   S0, out, S_T as in kda_chunk_fwd.
+ * KDA_COMPLEX is not supported here (the pages define no signed-gate map).
+ */
+int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
+                           const void *conv_w, const void *z, const float *A,
+                           const float *beta_logit, const float *S0, void *out,
+                           float *S_T, int B, int T, int H, int dk, int dv,
+                           const kda_opts *opts, cudaStream_t stream);
+
+/* Workspace bytes kda_chunk_fwd_prologue needs. */
+size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv,
+                                    const kda_opts *opts);
+
+/* Static description of a status code (never NULL). */
+const char *kda_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+int kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_B200_KDA_H */

@@ -49,18 +49,28 @@ SWEEP = dict(B=1, H=96, dk=128, dv=128, dtype=torch.bfloat16, S0_std=0.01)
 LOG_DECAY_FLOOR = -5.0
 
 
+_DEVICE = "cpu"
+
+
+def set_device(device: str) -> None:
+    """Draw on another device (the benchmark draws its timing-only inputs on
+    the GPU to save host time; every parity test draws on the CPU)."""
+    global _DEVICE
+    _DEVICE = device
+
+
 def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+    g = torch.Generator(device=_DEVICE)
     g.manual_seed(int(seed))
     return g
 
 
 def _randn(shape, gen):
-    return torch.randn(shape, generator=gen, dtype=torch.float32)
+    return torch.randn(shape, generator=gen, dtype=torch.float32, device=gen.device)
 
 
 def _uniform(shape, lo, hi, gen):
-    return torch.rand(shape, generator=gen, dtype=torch.float32) * (hi - lo) + lo
+    return torch.rand(shape, generator=gen, dtype=torch.float32, device=gen.device) * (hi - lo) + lo
 
 
 def _sampled_log_decay(z, A):
@@ -96,7 +106,7 @@ def chunk_inputs(B, T, H, dk, dv, *, dtype=torch.bfloat16, S0_std=0.01, seed=0,
     if complex_gate:
         g = cast(g)
         # keep |alpha| >= exp(-5) after rounding to the run dtype
-        floor = torch.tensor(math.exp(LOG_DECAY_FLOOR), dtype=dtype)
+        floor = torch.tensor(math.exp(LOG_DECAY_FLOOR), dtype=dtype, device=g.device)
         g = torch.where(g.abs() < floor, torch.where(g < 0, -floor, floor), g).contiguous()
     else:
         g = cast(g)

@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute call made).
+
+The library must load, export every function ``include/kda.h`` declares, and
+reject bad arguments on the host before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kda():
+    from gated_delta_rule_73_b200 import build as B
+    B.build()
+    import gated_delta_rule_73_b200.kda as K
+    return K
+
+
+def _declared_functions():
+    names = []
+    for hdr in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not hdr.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", hdr)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[a-z_]+\s*\*?\s*(kda_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_prologue",
+              "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_status_string",
+              "kda_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(kda):
+    lib = ctypes.CDLL(kda.LIB_PATH)
+    for n in _declared_functions():
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings_and_version(kda):
+    assert kda.kda_abi_version() == 100
+    for s in (0, -1, -2, -3, -4, -5, -6, -7):
+        assert kda.status_string(s) and kda.status_string(s) != "unknown status"
+    assert kda.status_string(-99) == "unknown status"
+
+
+def _call_chunk(kda, ptr=0x1000, **kw):
+    d = dict(B=1, T=64, H=2, dk=128, dv=128)
+    d.update(kw.pop("dims", {}))
+    opts = kw.pop("opts", kda.make_opts())
+    p = [ctypes.c_void_p(ptr)] * 8
+    for i, name in enumerate(("q", "k", "v", "g", "beta", "S0", "out", "S_T")):
+        if name in kw:
+            p[i] = ctypes.c_void_p(kw[name])
+    return kda._lib.kda_chunk_fwd(*p, d["B"], d["T"], d["H"], d["dk"], d["dv"],
+                                  ctypes.byref(opts), None)
+
+
+def test_chunk_fwd_rejects_bad_arguments_on_host(kda):
+    # NULL required pointers
+    assert _call_chunk(kda, q=0) == -1
+    assert _call_chunk(kda, out=0) == -1
+    # negative sizes
+    assert _call_chunk(kda, dims=dict(T=-1)) == -1
+    assert _call_chunk(kda, dims=dict(B=-2)) == -1
+    # unsupported head dims
+    assert _call_chunk(kda, dims=dict(dk=96)) == -4
+    assert _call_chunk(kda, dims=dict(dv=256)) == -4
+    # misaligned pointer (never dereferenced)
+    assert _call_chunk(kda, k=0x1004) == -3
+    # unknown flag bit / bad dtype / non-finite scale
+    o = kda.make_opts(); o.flags = 8
+    assert _call_chunk(kda, opts=o) == -1
+    o = kda.make_opts(); o.dtype = 7
+    assert _call_chunk(kda, opts=o) == -1
+    o = kda.make_opts(); o.scale = float("nan")
+    assert _call_chunk(kda, opts=o) == -1
+    # workspace missing for a shape that needs one
+    assert _call_chunk(kda) == -7
+    # overflowing sizes
+    assert _call_chunk(kda, dims=dict(B=1, T=2**30, H=2**10)) == -2
+
+
+def test_empty_calls_are_noops(kda):
+    # B == 0 or H == 0: nothing to do; T == 0 with S_T == NULL: nothing to write
+    assert _call_chunk(kda, dims=dict(B=0)) == 0
+    assert _call_chunk(kda, dims=dict(H=0)) == 0
+    assert _call_chunk(kda, dims=dict(T=0), S_T=0) == 0
+
+
+def test_workspace_sizes(kda):
+    o = kda.make_opts()
+    a = kda.kda_chunk_workspace_bytes(1, 64, 1, 128, 128, o)
+    b = kda.kda_chunk_workspace_bytes(1, 128, 1, 128, 128, o)
+    c = kda.kda_chunk_workspace_bytes(2, 65, 3, 128, 128, o)
+    assert a >= 0 and b >= a and c >= b
+    assert kda.kda_chunk_workspace_bytes(1, 0, 1, 128, 128, o) == 0
+    assert kda.kda_chunk_workspace_bytes(1, 64, 1, 96, 128, o) == 0      # unsupported -> 0
+    p = kda.kda_prologue_workspace_bytes(1, 64, 2, 128, 128, o)
+    assert p > 3 * 64 * 2 * 128 * 4
+
+
+def test_recurrent_step_rejects_bad_arguments_on_host(kda):
+    vp = ctypes.c_void_p
+    o = kda.make_opts()
+    call = lambda ptrs, N=4, H=2, dk=128, dv=128: kda._lib.kda_recurrent_step(
+        *[vp(p) for p in ptrs], N, H, dk, dv, ctypes.byref(o), None)
+    good = [0x1000] * 7
+    assert call([0] + good[1:]) == -1
+    assert call(good[:5] + [0] + good[6:]) == -1          # S is required
+    assert call(good[:2] + [0x1008] + good[3:]) == -3
+    assert call(good, dk=32) == -4
+    assert call(good, N=-1) == -1
+    assert call(good, N=0) == 0
+
+
+def test_prologue_rejects_complex_and_unequal_dims(kda):
+    vp = ctypes.c_void_p
+    call = lambda opts, dk=128, dv=128: kda._lib.kda_chunk_fwd_prologue(
+        *[vp(0x1000)] * 10, 1, 64, 2, dk, dv, ctypes.byref(opts), None)
+    assert call(kda.make_opts(complex_gate=True)) == -4
+    assert call(kda.make_opts(), dk=64, dv=128) == -4
+    assert call(kda.make_opts()) == -7                     # needs a workspace

@@ -1,0 +1,121 @@
+"""GPU parity of ``kda_chunk_fwd`` against the FP64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import kda_workloads as W
+import oracle
+from tests._util import cuda, f64, rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def K():
+    from gated_delta_rule_73_b200 import build
+    build.build()
+    import gated_delta_rule_73_b200 as K
+    return K
+
+
+def _run(K, x, **kw):
+    q, k, v, g, beta = (cuda(x[n]) for n in ("q", "k", "v", "g", "beta"))
+    S0 = cuda(x["S0"])
+    B, T, H, dk = x["q"].shape
+    dv = x["v"].shape[-1]
+    out = torch.full((B, T, H, dv), float("nan"), dtype=q.dtype, device="cuda")
+    S_T = torch.full((B, H, dk, dv), float("nan"), dtype=torch.float32, device="cuda")
+    K.chunk_fwd(q, k, v, g, beta, S0, out=out, S_T=S_T, **kw)
+    torch.cuda.synchronize()
+    return out, S_T
+
+
+def _oracle(x, heads=None, **kw):
+    """Oracle on all heads, or on the listed (b, h) pairs only (stacked as B=1, H=len)."""
+    arr = {n: f64(x[n]) for n in ("q", "k", "v", "g", "beta")}
+    S0 = f64(x["S0"])
+    if heads is None:
+        return oracle.recurrence_c(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], S0, **kw)
+    sel = lambda a: np.stack([a[b, :, h] for b, h in heads], axis=1)[None]
+    S0s = None if S0 is None else np.stack([S0[b, h] for b, h in heads])[None]
+    return oracle.recurrence_c(*(sel(arr[n]) for n in ("q", "k", "v", "g")),
+                               np.stack([arr["beta"][b, :, h] for b, h in heads], axis=1)[None],
+                               S0s, **kw)
+
+
+def _check(out, S_T, ref, dtype, heads=None):
+    o, s = f64(out), f64(S_T)
+    if heads is not None:
+        o = np.stack([o[b, :, h] for b, h in heads], axis=1)[None]
+        s = np.stack([s[b, h] for b, h in heads])[None]
+    tol = tol_for(dtype)
+    eo, es = rel_err(o, ref[0]), rel_err(s, ref[1])
+    assert eo <= tol and es <= tol, (eo, es, tol)
+    return eo, es
+
+
+def test_tiny_fp32_workload(K):
+    """tiny workload: B=1, T=256, H=2, d=64, fp32, S0 = 0; bound 1e-4."""
+    x = W.workload_inputs("tiny")
+    out, S_T = _run(K, x)
+    _check(out, S_T, _oracle(x), torch.float32)
+
+
+def test_prefill_workload_full(K):
+    """prefill workload at full size: B=1, T=4096, H=16, d=128, bf16; every output."""
+    x = W.workload_inputs("prefill")
+    out, S_T = _run(K, x)
+    _check(out, S_T, _oracle(x), torch.bfloat16)
+
+
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 63, 64, 65, 130, 200])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_ragged_lengths(K, T, dtype):
+    x = W.chunk_inputs(2, T, 3, 128, 128, dtype=dtype, seed=T)
+    out, S_T = _run(K, x)
+    _check(out, S_T, _oracle(x), dtype)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_head_dims(K, dk, dv, dtype):
+    x = W.chunk_inputs(1, 150, 2, dk, dv, dtype=dtype, seed=dk + dv)
+    out, S_T = _run(K, x)
+    _check(out, S_T, _oracle(x), dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_complex_kda_small(K, dtype):
+    x = W.chunk_inputs(2, 190, 2, 128, 128, dtype=dtype, seed=5, complex_gate=True)
+    out, S_T = _run(K, x, complex_gate=True)
+    _check(out, S_T, _oracle(x, complex_gate=True), dtype)
+
+
+def test_complex_kda_workload_sampled(K):
+    """Complex-KDA workload at full size (B=8, T=8192, H=32, d=128), sampled heads."""
+    x = W.workload_inputs("ckda")
+    out, S_T = _run(K, x, complex_gate=True)
+    heads = [(0, 0), (3, 17), (7, 31)]
+    _check(out, S_T, _oracle(x, heads, complex_gate=True), torch.bfloat16, heads)
+
+
+def test_options_no_l2norm_scale_and_no_S0(K):
+    x = W.chunk_inputs(1, 100, 2, 128, 128, dtype=torch.float32, seed=9, S0_std=0.0)
+    # without the in-kernel norm the inputs must be normalised by the caller
+    for n in ("q", "k"):
+        x[n] = (x[n] / x[n].norm(dim=-1, keepdim=True)).contiguous()
+    out, S_T = _run(K, x, l2norm=False, scale=0.5)
+    _check(out, S_T, _oracle(x, l2norm=False, scale=0.5), torch.float32)
+
+
+def test_empty_sequence_is_identity(K):
+    """T = 0: S_T = S0 (the empty chunk is the identity of the monoid)."""
+    x = W.chunk_inputs(2, 0, 3, 128, 128, seed=1)
+    S0 = cuda(x["S0"])
+    S_T = torch.full_like(S0, float("nan"))
+    opts = K.make_opts(torch.bfloat16)
+    e = lambda *s: torch.empty(*s, dtype=torch.bfloat16, device="cuda")
+    K.kda_chunk_fwd(e(2, 0, 3, 128), e(2, 0, 3, 128), e(2, 0, 3, 128), e(2, 0, 3, 128),
+                    e(2, 0, 3), S0, e(2, 0, 3, 128), S_T, opts)
+    torch.cuda.synchronize()
+    assert torch.equal(S_T, S0)
