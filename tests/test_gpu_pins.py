@@ -64,6 +64,7 @@ def test_decay_only_on_gpu(K):
     """beta = 0: S_T = Diag(exp(sum g)) S0 and o_t = S0^T (exp(cumsum g)_t * q_t)."""
     x = W.chunk_inputs(1, 130, 2, 128, 128, dtype=torch.float32, seed=22)
     x["beta"][:] = 0.0
+    x["g"] = (x["g"] * 0.02).contiguous()   # keep exp(sum g) inside the FP32 range
     out, ST = _chunk(K, x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"])
     g = f64(x["g"])
     S0 = f64(x["S0"])
