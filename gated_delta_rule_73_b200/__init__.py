@@ -2,11 +2,24 @@
 
 The product is the C-ABI library ``libkda_b200.so`` (declared in
 ``include/kda.h``); this package holds its CUDA sources (``csrc/``), the
-in-tree build (``build.py``) and a thin ctypes binding (``kda.py``).
+in-tree build (``build.py``) and a thin ctypes binding (``kda.py``).  The
+binding is loaded on first attribute access, so ``build`` can run before the
+library exists.
 """
-from .kda import (  # noqa: F401
-    KDA_BF16, KDA_F32, KDA_QK_L2NORM, KDA_COMPLEX, KdaError, kda_opts, make_opts,
-    kda_chunk_fwd, kda_recurrent_step, kda_chunk_fwd_prologue, kda_chunk_workspace_bytes,
-    kda_prologue_workspace_bytes, kda_abi_version, status_string, chunk_fwd, recurrent_step,
-    chunk_fwd_prologue, LIB_PATH,
+_EXPORTS = (
+    "KDA_BF16", "KDA_F32", "KDA_QK_L2NORM", "KDA_COMPLEX", "KdaError", "kda_opts", "make_opts",
+    "kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_prologue",
+    "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_abi_version",
+    "status_string", "chunk_fwd", "recurrent_step", "chunk_fwd_prologue", "LIB_PATH",
 )
+
+
+def __getattr__(name):
+    if name in _EXPORTS or name == "kda":
+        import importlib
+        mod = importlib.import_module(".kda", __name__)
+        return mod if name == "kda" else getattr(mod, name)
+    raise AttributeError(name)
+
+
+__all__ = list(_EXPORTS)
