@@ -49,6 +49,8 @@ def _load():
     lib.kda_recurrent_step.restype = ip
     lib.kda_chunk_fwd_prologue.argtypes = [vp] * 10 + [ip] * 5 + [op, vp]
     lib.kda_chunk_fwd_prologue.restype = ip
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 8 + [ip] * 5 + [op, vp]
+    lib.kda_chunk_fwd_noalloc.restype = ip
     lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_chunk_workspace_bytes.restype = sz
     lib.kda_prologue_workspace_bytes.argtypes = [ip] * 5 + [op]
@@ -139,6 +141,20 @@ def kda_chunk_fwd(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -
     st = _lib.kda_chunk_fwd(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
     if st != 0:
         raise KdaError("kda_chunk_fwd", st)
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_chunk_fwd_noalloc``: kda_chunk_fwd with the library's fixed
+    device scratch instead of a workspace, for callers that cannot allocate."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
+            _ptr(S_T, "S_T", torch.float32)]
+    st = _lib.kda_chunk_fwd_noalloc(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_chunk_fwd_noalloc", st)
 
 
 def kda_recurrent_step(q, k, v, g, beta, S, out, opts: kda_opts, stream=None) -> None:

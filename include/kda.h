@@ -161,6 +161,34 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
 size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv,
                                     const kda_opts *opts);
 
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
+ *
+ * The pages have no counterpart: this is a deployment variant, not part of
+ * the method.  Some callers cannot call cudaMalloc -- code that must not
+ * synchronise the device, loops that forbid allocation once running, host
+ * applications that own the device pool and give a component no allocator.
+ * This entry point takes the same arguments as kda_chunk_fwd (opts->workspace
+ * is ignored) and runs the FP32 two-phase chunk path with its scratch in a
+ * fixed device array of KDA_NOALLOC_SCRATCH_BYTES, which every GPU that loads
+ * the library holds until the process exits.  It calls no allocator.
+ *
+ *  - Sizes whose scratch (kda_chunk_workspace_bytes of the FP32 path: about
+ *    148 KB per 64-token chunk and head at dk = dv = 128) exceeds the array
+ *    are rejected with KDA_ERR_WORKSPACE before any CUDA call.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address once; make that first call before any stream
+ *    capture.
+ *  - All calls share the array.  Calls whose work overlaps on the GPU race;
+ *    serialise them (one stream per device).  No scratch content carries over:
+ *    each call writes every element it reads.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const void *g,
+                          const void *beta, const float *S0, void *out, float *S_T,
+                          int B, int T, int H, int dk, int dv, const kda_opts *opts,
+                          cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
