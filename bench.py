@@ -400,8 +400,49 @@ def run_ours(args, ws, rank, local):
     return 0
 
 
+CASES = ("prefill", "decode", "sweep", "ckda")
+
+
+def run_case(args):
+    """Run one workload's call a few times and exit (a small case for ncu captures):
+    prefill = B=1 T=4096 H=16; decode = N=64 H=96 (800 MB of state);
+    sweep = prologue path at T=2048 H=96; ckda = B=2 T=8192 H=32 signed gate."""
+    import gated_delta_rule_73_b200 as K
+    torch.cuda.set_device(0)
+    W.set_device("cuda")
+    d = 128
+    if args.case == "decode":
+        N, H = 64, 96
+        S = W.decode_state(N, H, d, d)
+        t = W.decode_step_inputs(N, H, d, d, 0)
+        out = torch.empty((N, H, d), dtype=torch.bfloat16, device="cuda")
+        o = K.make_opts(torch.bfloat16)
+        fn = lambda: K.kda_recurrent_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, out, o)
+    elif args.case == "sweep":
+        T, H = 2048, 96
+        x = W.sweep_inputs(T)
+        a = [x[n] for n in ("q_pre", "k_pre", "v_pre", "conv_w", "z", "A", "b_logit")]
+        fn = lambda: K.chunk_fwd_prologue(*a, x["S0"])
+    else:
+        if args.case == "prefill":
+            x = W.workload_inputs("prefill")
+            cplx = False
+        else:
+            x = W.chunk_inputs(2, 8192, 32, d, d, dtype=torch.bfloat16, seed=0, complex_gate=True)
+            cplx = True
+        fn = lambda: K.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], complex_gate=cplx)
+    for _ in range(args.case_reps):
+        fn()
+    torch.cuda.synchronize()
+    W.set_device("cpu")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run one small workload a few times (for profiler captures) and exit")
+    ap.add_argument("--case-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
@@ -409,6 +450,8 @@ def main():
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
+    if args.case:
+        return run_case(args)
     ws, rank, local = dist_setup()
     try:
         if args.impl == "reference":
