@@ -59,6 +59,9 @@ KernelFlags kflags(const kda_opts &o) {
     return f;
 }
 
+// the bf16 dk = dv = 128 chunk forward runs the fused tensor-core kernel (no workspace)
+bool use_tc(const kda_opts &o, int dk, int dv) { return o.dtype == KDA_BF16 && dk == 128 && dv == 128; }
+
 size_t chunk_ws(int B, int T, int H, int dk, int dv) {
     if (B <= 0 || T <= 0 || H <= 0) return 0;
     return round_up(chunk_ref_workspace_bytes(B, T, H, dk, dv), kAlignWs);
@@ -88,7 +91,7 @@ int finish_identity(const float *S0, float *S_T, int B, int H, int dk, int dv, c
 int run_chunk(ChunkArgs &a, cudaStream_t st) {
     int launches = 0;
     a.launch_idx = &launches;
-    cudaError_t e = launch_chunk_ref(a, st);
+    cudaError_t e = chunk_tc_supported(a) ? launch_chunk_tc(a, st) : launch_chunk_ref(a, st);
     if (e == cudaSuccess && a.events && launches < a.n_events) cudaEventRecord(a.events[launches], st);
     if (e == cudaErrorInvalidValue) return KDA_ERR_UNSUPPORTED;
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -117,6 +120,7 @@ const char *kda_status_string(int s) {
 size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, const kda_opts *opts) {
     const kda_opts o = resolve(opts);
     if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
+    if (use_tc(o, dk, dv)) return 0;
     return chunk_ws(B, T, H, dk, dv);
 }
 
@@ -144,7 +148,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     const void *ptrs[] = {q, k, v, g, beta, S0, out, S_T, o.workspace};
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_ALIGN;
-    const size_t need = chunk_ws(B, T, H, dk, dv);
+    const size_t need = use_tc(o, dk, dv) ? 0 : chunk_ws(B, T, H, dk, dv);
     if (need > 0 && (!o.workspace || o.workspace_bytes < need)) return KDA_ERR_WORKSPACE;
 
     ChunkArgs a;

@@ -46,6 +46,10 @@ struct PrologueArgs {
 size_t chunk_ref_workspace_bytes(int B, int T, int H, int dk, int dv);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+// Fused tensor-core chunk path (bf16, dk = dv = 128); needs no workspace.
+bool chunk_tc_supported(const ChunkArgs &a);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t st);
+int chunk_tc_read_error();
 cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st);
 
