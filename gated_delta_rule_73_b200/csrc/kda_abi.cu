@@ -67,16 +67,19 @@ size_t chunk_ws(int B, int T, int H, int dk, int dv) {
     return round_up(chunk_ref_workspace_bytes(B, T, H, dk, dv), kAlignWs);
 }
 
-size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, size_t *off) {
+// The prologue's outputs are bf16 when the tensor-core chunk kernel follows
+// (bf16 activations, dk = dv = 128; it needs no further workspace), FP32 otherwise.
+size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, bool tc, size_t *off) {
     // off[0..5]: qc, kc, vc, g, beta, chunk workspace
     const size_t rows = (size_t)B * T * H;
+    const size_t e = tc ? 2 : 4;
     size_t o = 0;
-    off[0] = o; o = round_up(o + rows * dk * 4, kAlignWs);
-    off[1] = o; o = round_up(o + rows * dk * 4, kAlignWs);
-    off[2] = o; o = round_up(o + rows * dv * 4, kAlignWs);
-    off[3] = o; o = round_up(o + rows * dk * 4, kAlignWs);
-    off[4] = o; o = round_up(o + rows * 4, kAlignWs);
-    off[5] = o; o += chunk_ws(B, T, H, dk, dv);
+    off[0] = o; o = round_up(o + rows * dk * e, kAlignWs);
+    off[1] = o; o = round_up(o + rows * dk * e, kAlignWs);
+    off[2] = o; o = round_up(o + rows * dv * e, kAlignWs);
+    off[3] = o; o = round_up(o + rows * dk * e, kAlignWs);
+    off[4] = o; o = round_up(o + rows * e, kAlignWs);
+    off[5] = o; o += tc ? 0 : chunk_ws(B, T, H, dk, dv);
     return o;
 }
 
@@ -129,7 +132,7 @@ size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, const k
     if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
     if (B <= 0 || T <= 0 || H <= 0) return 0;
     size_t off[6];
-    return prologue_ws_parts(B, T, H, dk, dv, off);
+    return prologue_ws_parts(B, T, H, dk, dv, use_tc(o, dk, dv), off);
 }
 
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -210,7 +213,8 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_ALIGN;
     size_t off[6];
-    const size_t need = prologue_ws_parts(B, T, H, dk, dv, off);
+    const bool tc = use_tc(o, dk, dv);
+    const size_t need = prologue_ws_parts(B, T, H, dk, dv, tc, off);
     if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
     char *ws = (char *)o.workspace;
 
@@ -218,9 +222,10 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     p.q_pre = q_pre; p.k_pre = k_pre; p.v_pre = v_pre; p.conv_w = conv_w; p.z = z;
     p.A = A; p.beta_logit = beta_logit;
     p.bf16 = o.dtype == KDA_BF16;
+    p.out_bf16 = tc;
     p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
-    p.qc = (float *)(ws + off[0]); p.kc = (float *)(ws + off[1]); p.vc = (float *)(ws + off[2]);
-    p.g = (float *)(ws + off[3]); p.beta = (float *)(ws + off[4]);
+    p.qc = ws + off[0]; p.kc = ws + off[1]; p.vc = ws + off[2];
+    p.g = ws + off[3]; p.beta = ws + off[4];
 
     int launches = 0;
     if (o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
@@ -231,7 +236,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     ChunkArgs a;
     memset(&a, 0, sizeof(a));
     a.q = p.qc; a.k = p.kc; a.v = p.vc; a.g = p.g; a.beta = p.beta;
-    a.t_qkv = a.t_g = a.t_beta = Elt::F32;
+    a.t_qkv = a.t_g = a.t_beta = tc ? Elt::BF16 : Elt::F32;
     a.t_out = p.bf16 ? Elt::BF16 : Elt::F32;
     a.S0 = S0; a.out = out; a.S_T = S_T;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
@@ -241,7 +246,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     a.workspace_bytes = need - off[5];
     a.events = o.events; a.n_events = o.n_events;
     a.launch_idx = &launches;
-    e = launch_chunk_ref(a, stream);
+    e = tc ? launch_chunk_tc(a, stream) : launch_chunk_ref(a, stream);
     if (e == cudaSuccess && o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -44,7 +44,7 @@ using namespace sm100;
 
 constexpr int D = 128;          // dk = dv
 constexpr int C = 64;           // chunk
-constexpr int NT = 256;         // threads
+constexpr int NT = 512;         // threads: 16 warps, 4 per TMEM lane quarter
 constexpr uint32_t kTmaBytes = 4u * C * D * 2u;   // q, k, v, g tiles per chunk
 
 // shared memory map (bytes from a 1024-aligned base)
@@ -52,41 +52,53 @@ constexpr uint32_t OFF_STG_Q = 0;
 constexpr uint32_t OFF_STG_K = 16384;
 constexpr uint32_t OFF_STG_V = 32768;
 constexpr uint32_t OFF_STG_G = 49152;
-constexpr uint32_t OFF_GAM = 65536;           // fp32 gamma [64][132]; later AKK/TMF/RS; later VT
-constexpr uint32_t GAM_STRIDE = 132;          // floats per row (conflict-free 16-byte row reads)
-constexpr uint32_t OFF_AKK = OFF_GAM;         // fp32 [64][65]
-constexpr uint32_t OFF_TMF = OFF_GAM + 16640; // fp32 [64][65]
-constexpr uint32_t OFF_RS = OFF_GAM + 33280;  // fp32 [3][16][17]
+constexpr uint32_t OFF_GAM = 65536;           // fp32 E = e^{band-local cumsum} [64][132]; later AKK/TMF; later V~^T
+constexpr uint32_t E_STRIDE = 132;            // floats per row (conflict-free 16-byte row reads)
+constexpr uint32_t AS = 68;                   // row stride (floats) of AKK / TMF
+constexpr uint32_t OFF_AKK = OFF_GAM;         // fp32 [64][68]
+constexpr uint32_t OFF_TMF = OFF_GAM + 17408; // fp32 [64][68]
 constexpr uint32_t OFF_VT = OFF_GAM;          // bf16 V~^T, K-major [128 j][64 r]
-constexpr uint32_t OFF_QG = OFF_GAM + 36864;  // bf16 Q e^gamma, [64 r][128 c]
-constexpr uint32_t OFF_XR = OFF_QG + 16384;   // bf16 K e^{p-gamma} [64][128]; later A_qk + Tm'
+constexpr uint32_t OFF_QG = OFF_GAM + 36864;  // bf16 Q e^gamma [64 r][128 c]; later O staging [64][128]
+constexpr uint32_t OFF_XR = OFF_QG + 16384;   // bf16 K e^{p-gamma} [64][128]; later A_qk + (scratch, Tm')
 constexpr uint32_t OFF_AQK = OFF_XR;          // bf16 [64 r][64 i]
 constexpr uint32_t OFF_TMB = OFF_XR + 8192;   // bf16 [64 r][64 i]
+constexpr uint32_t OFF_RZ = OFF_XR + 8192;    // fp32 inverse scratch: R [2][16][20], Z [32][36]
 constexpr uint32_t OFF_YR = OFF_XR + 16384;   // bf16 K e^gamma [64][128]; later W^T [128][64]
 constexpr uint32_t OFF_KD = OFF_YR + 16384;   // bf16 K e^{gamma_C-gamma} [64][128]
 constexpr uint32_t OFF_SB = OFF_KD + 16384;   // bf16 S [128 c][128 j]
-constexpr uint32_t OFF_TAB = OFF_SB + 32768;  // fp32 tables
-constexpr uint32_t TAB_P = 0;                 // [4][128]
-constexpr uint32_t TAB_F = TAB_P + 2048;      // [4][4][128]
-constexpr uint32_t TAB_G = TAB_F + 8192;      // [4][128]
-constexpr uint32_t TAB_H = TAB_G + 2048;      // [4][128]
-constexpr uint32_t TAB_GC = TAB_H + 2048;     // [128]
-constexpr uint32_t TAB_NRM = TAB_GC + 512;    // [128]
-constexpr uint32_t TAB_BET = TAB_NRM + 512;   // [64]
-constexpr uint32_t TAB_SGN = TAB_BET + 256;   // uint32 [64][4]
-constexpr uint32_t TAB_SGNC = TAB_SGN + 1024; // uint32 [4]
+constexpr uint32_t OFF_TAB = OFF_SB + 32768;  // tables
+constexpr uint32_t TAB_TOT = 0;               // fp32 [4][128] band sums of log-decay
+constexpr uint32_t TAB_F = TAB_TOT + 2048;    // fp32 [4][4][128] e^{p_b - p_j}
+constexpr uint32_t TAB_G = TAB_F + 8192;      // fp32 [4][128] e^{gamma_C - p_b}
+constexpr uint32_t TAB_H = TAB_G + 2048;      // fp32 [4][128] e^{p_b}
+constexpr uint32_t TAB_GC = TAB_H + 2048;     // fp32 [128] sigma_C e^{gamma_C}
+constexpr uint32_t TAB_NRM = TAB_GC + 512;    // fp32 [128] inverse norms (q rows, k rows)
+constexpr uint32_t TAB_BET = TAB_NRM + 512;   // fp32 [64]
+constexpr uint32_t TAB_SGNL = TAB_BET + 256;  // u32 [64][4] band-local sign parity bits
+constexpr uint32_t TAB_BPAR = TAB_SGNL + 1024;// u32 [4][4] parity of each band
+constexpr uint32_t TAB_PP = TAB_BPAR + 256;   // u32 [4][4] parity of the bands before
+constexpr uint32_t TAB_SGNC = TAB_PP + 256;   // u32 [4] parity of the whole chunk
 constexpr uint32_t TAB_BYTES = TAB_SGNC + 256;
 constexpr uint32_t SMEM_USED = OFF_TAB + TAB_BYTES;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for the 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_TMF + 64 * AS * 4 <= OFF_QG, "inverse scratch fits");
 
-// TMEM columns (512 allocated)
-constexpr uint32_t TC_AOP = 0;     // A operands of the A_qk/A_kk products: band j at 64 j
-constexpr uint32_t TC_S = 0;       // dS accumulator (after the band products)
-constexpr uint32_t TC_O = 128;     // O^T
-constexpr uint32_t TC_A = 256;     // A_qk (lanes 0-63) / A_kk (lanes 64-127)
-constexpr uint32_t TC_W = 320;     // W^T
-constexpr uint32_t TC_U = 384;     // U^T, then V~^T
+// TMEM columns (512 allocated).  Every product is split over two accumulators
+// (even / odd K-steps) so that consecutive MMAs never wait on each other; the
+// halves are summed when read back.  Regions are reused once they are dead:
+//   [0,256)   band operands (step 3-4) | W^T_b [0,64), U^T_b [64,128) (7-10),
+//             O^T_a [128,192), O^T_b [192,256) (9-12) | dS_a [0,128) (11-12)
+//   [256,320) A_a (4-5)  | dS_b [256,384) (11-12)
+//   [320,384) W^T_a (7-8)
+//   [384,448) U^T_a, then V~^T_a (7-10)
+//   [448,512) A_b (4-5)
+constexpr uint32_t TC_AOP = 0;
+constexpr uint32_t TC_A_A = 256, TC_A_B = 448;
+constexpr uint32_t TC_W_A = 320, TC_W_B = 0;
+constexpr uint32_t TC_U_A = 384, TC_U_B = 64;
+constexpr uint32_t TC_O_A = 128, TC_O_B = 192;
+constexpr uint32_t TC_S_A = 0, TC_S_B = 256;
 
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -131,6 +143,10 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
     u.w = pack_bf16(x[6], x[7]);
     return u;
 }
+__device__ __forceinline__ void ld8f(const float *p, float (&x)[8]) {
+    *reinterpret_cast<float4 *>(x) = *reinterpret_cast<const float4 *>(p);
+    *reinterpret_cast<float4 *>(x + 4) = *reinterpret_cast<const float4 *>(p + 4);
+}
 
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -143,23 +159,27 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
-    float *GAM = reinterpret_cast<float *>(smem + OFF_GAM);
+    float *EX = reinterpret_cast<float *>(smem + OFF_GAM);
     float *AKK = reinterpret_cast<float *>(smem + OFF_AKK);
     float *TMF = reinterpret_cast<float *>(smem + OFF_TMF);
-    float *RS = reinterpret_cast<float *>(smem + OFF_RS);
-    float *TP = reinterpret_cast<float *>(smem + OFF_TAB + TAB_P);
+    float *RR = reinterpret_cast<float *>(smem + OFF_RZ);          // [2][16][20]
+    float *ZZ = reinterpret_cast<float *>(smem + OFF_RZ + 2560);   // [32][36]
+    float *TOT = reinterpret_cast<float *>(smem + OFF_TAB + TAB_TOT);
     float *TF = reinterpret_cast<float *>(smem + OFF_TAB + TAB_F);
     float *TG = reinterpret_cast<float *>(smem + OFF_TAB + TAB_G);
     float *TH = reinterpret_cast<float *>(smem + OFF_TAB + TAB_H);
     float *TGC = reinterpret_cast<float *>(smem + OFF_TAB + TAB_GC);
     float *NRM = reinterpret_cast<float *>(smem + OFF_TAB + TAB_NRM);
     float *BET = reinterpret_cast<float *>(smem + OFF_TAB + TAB_BET);
-    uint32_t *SGN = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGN);
+    float *BET_S = BET;
+    uint32_t *SGNL = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNL);
+    uint32_t *BPAR = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_BPAR);
+    uint32_t *PP = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_PP);
     uint32_t *SGNC = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNC);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int row = quad * 32 + lane;                 // TMEM lane owned by this thread
+    const int quad = warp & 3, qq = warp >> 2;       // lane quarter; column quarter
+    const int row = quad * 32 + lane;                // TMEM lane owned by this thread
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int nch = (T + C - 1) / C;
@@ -180,17 +200,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sh.tmem_base;
+    // descriptor bases (start address = the smem base); a tile at byte offset `off`
+    // is base + (off >> 4) since every address stays below 256 KB
+    const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);    // K-major [rows][128]
+    const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);   // MN-major [K rows][128]
+    const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);    // K-major [rows][64]
+    const uint64_t dMN32 = sdesc(sbase, 1024, 128, kSwizzleNone);   // MN-major [K rows][64]
+    const uint64_t dV = sdesc(sbase, 8192, 1024, kSwizzle128B);     // MN-major TMA v tile
+    auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
 
-    auto issue_tma = [&](int ch) {
+    // the next chunk's q, k, g tiles are requested as soon as this chunk's operands are
+    // built (they are free then), its v tile once the U product has read it
+    auto issue_tma_qkg = [&](int ch) {
         mbar_arrive_expect_tx(bar_tma, kTmaBytes);
         const int t0 = ch * C;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             tma_load_4d(sbase + OFF_STG_Q + hf * 8192, &tm_q, bar_tma, hf * 64, h, t0, b);
             tma_load_4d(sbase + OFF_STG_K + hf * 8192, &tm_k, bar_tma, hf * 64, h, t0, b);
-            tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_tma, hf * 64, h, t0, b);
             tma_load_4d(sbase + OFF_STG_G + hf * 8192, &tm_g, bar_tma, hf * 64, h, t0, b);
         }
+    };
+    auto issue_tma_v = [&](int ch) {
+        const int t0 = ch * C;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_tma, hf * 64, h, t0, b);
     };
     // every thread waits; a give-up anywhere makes the whole CTA stop together
     auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
@@ -201,24 +236,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncthreads();
         return sh.abort == 0;
     };
-    if (tid == 0 && nch > 0) issue_tma(0);
+    if (tid == 0 && nch > 0) {
+        issue_tma_qkg(0);
+        issue_tma_v(0);
+    }
+    // beta of the first chunk; later chunks' beta is fetched a chunk ahead
+    if (tid < C) BET_S[tid] = tid < T ? __bfloat162float(beta[((size_t)b * T + tid) * H + h]) : 0.f;
 
-    // the FP32 state: thread (row = key channel c, half) owns S[c][64 half .. 64 half + 63]
-    float S[64];
+    // the FP32 state: thread (row = key channel c, qq) owns S[c][32 qq .. 32 qq + 31]
+    float S[32];
     {
         const int c = row;
-        const float *src = S0 ? S0 + ((size_t)bh * D + c) * D + 64 * half : nullptr;
+        const float *src = S0 ? S0 + ((size_t)bh * D + c) * D + 32 * qq : nullptr;
 #pragma unroll
-        for (int j = 0; j < 64; j += 4) {
+        for (int j = 0; j < 32; j += 4) {
             float4 v4 = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
             S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
         }
 #pragma unroll
-        for (int jg = 0; jg < 8; ++jg) {
+        for (int jg = 0; jg < 4; ++jg) {
             float x[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e];
-            *reinterpret_cast<uint4 *>(smem + OFF_SB + off_r128(c, 64 * half + 8 * jg)) = pack8(x);
+            *reinterpret_cast<uint4 *>(smem + OFF_SB + off_r128(c, 32 * qq + 8 * jg)) = pack8(x);
         }
     }
 
@@ -230,73 +270,95 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!(ok = wait_all(bar_tma, ph_tma))) break;
         ph_tma ^= 1;
 
-        // ---- step 1: cumulative log-decay per key channel | row norms and beta
-        if (tid < D) {
-            const int c = tid;
-            float gam = 0.f;
+        // ---- step 1: band-local cumulative log-decay (4 bands x 128 channels) | row norms | beta
+        {
+            const int c = tid & 127, p = tid >> 7;
+            float gv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                gv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                    smem + OFF_STG_G + off_sw128(16 * p + i, c)));
+            float loc = 0.f;
             uint32_t par = 0;
-            for (int r = 0; r < C; ++r) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * p + i;
                 float lg = 0.f;
                 if (r < n) {
-                    const float a = __bfloat162float(
-                        *reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_STG_G + off_sw128(r, c)));
                     if (fl.complex_gate) {
-                        lg = __logf(fabsf(a));
-                        par ^= (a < 0.f) ? 1u : 0u;
+                        lg = __logf(fabsf(gv[i]));
+                        par ^= (gv[i] < 0.f) ? 1u : 0u;
                     } else {
-                        lg = a;
+                        lg = gv[i];
                     }
                 }
-                gam += lg;
-                GAM[r * GAM_STRIDE + c] = gam;
+                loc += lg;
+                EX[r * E_STRIDE + c] = __expf(fmaxf(loc, -85.f));
                 if (fl.complex_gate) {
                     const uint32_t bits = __ballot_sync(0xffffffffu, par != 0);
-                    if (lane == 0) SGN[r * 4 + warp] = bits;
+                    if (lane == 0) SGNL[r * 4 + quad] = bits;
                 }
-                if ((r & 15) == 15 && r < 63) TP[((r + 1) >> 4) * D + c] = gam;
             }
-            TP[c] = 0.f;
-            const uint32_t bits = __ballot_sync(0xffffffffu, par != 0);
-            if (lane == 0) SGNC[warp] = fl.complex_gate ? bits : 0u;
-        } else {
-            const int rr = tid - D;      // 0..63 q rows, 64..127 k rows
+            TOT[p * D + c] = loc;
+            const uint32_t bp = __ballot_sync(0xffffffffu, par != 0);
+            if (lane == 0) BPAR[p * 4 + quad] = bp;
+        }
+        {
+            const int rr = tid >> 2, part = tid & 3;     // 4 lanes per row, 32 channels each
             const int r = rr & 63;
             const uint32_t tile = rr < 64 ? OFF_STG_Q : OFF_STG_K;
             float ss = 0.f;
 #pragma unroll
-            for (int cg = 0; cg < 16; ++cg) {
+            for (int m = 0; m < 4; ++m) {
                 float x[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, cg * 8)), x);
+                unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, 32 * part + 8 * m)), x);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
             }
-            NRM[rr] = fl.l2norm ? rsqrtf(ss + kL2Eps) : 1.f;
-            if (rr < 64)
-                BET[r] = r < n ? __bfloat162float(beta[((size_t)b * T + t0 + r) * H + h]) : 0.f;
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            if (part == 0) NRM[rr] = fl.l2norm ? rsqrtf(ss + kL2Eps) : 1.f;
         }
         __syncthreads();
 
-        // ---- step 2: per-band factor tables
-        for (int idx = tid; idx < 11 * D; idx += NT) {
-            const int e = idx / D, c = idx % D;
-            const float gC = GAM[63 * GAM_STRIDE + c];
-            if (e < 6) {
-                const int bb = e < 1 ? 1 : (e < 3 ? 2 : 3);
-                const int jj = e < 1 ? 0 : (e < 3 ? e - 1 : e - 3);
-                TF[(bb * 4 + jj) * D + c] = __expf(TP[bb * D + c] - TP[jj * D + c]);
-            } else if (e < 10) {
-                const int bb = e - 6;
-                TG[bb * D + c] = __expf(gC - TP[bb * D + c]);
-                TH[bb * D + c] = __expf(TP[bb * D + c]);
-                TF[(bb * 4 + bb) * D + c] = 1.f;
-            } else {
-                const float sg = ((SGNC[c >> 5] >> (c & 31)) & 1u) ? -1.f : 1.f;
-                TGC[c] = sg * __expf(gC);
+        // ---- step 2: per-channel band factors from the four band sums
+        if (tid < D) {
+            const int c = tid;
+            float et[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) et[p] = __expf(TOT[p * D + c]);
+            // H[b] = e^{p_b}, F[b][j] = e^{p_b - p_j}, G[b] = e^{gamma_C - p_b}
+            TH[0 * D + c] = 1.f;
+            TH[1 * D + c] = et[0];
+            TH[2 * D + c] = et[0] * et[1];
+            TH[3 * D + c] = et[0] * et[1] * et[2];
+            const float eC = et[0] * et[1] * et[2] * et[3];
+            TG[0 * D + c] = eC;
+            TG[1 * D + c] = et[1] * et[2] * et[3];
+            TG[2 * D + c] = et[2] * et[3];
+            TG[3 * D + c] = et[3];
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) TF[(bb * 4 + bb) * D + c] = 1.f;
+            TF[(1 * 4 + 0) * D + c] = et[0];
+            TF[(2 * 4 + 1) * D + c] = et[1];
+            TF[(2 * 4 + 0) * D + c] = et[0] * et[1];
+            TF[(3 * 4 + 2) * D + c] = et[2];
+            TF[(3 * 4 + 1) * D + c] = et[1] * et[2];
+            TF[(3 * 4 + 0) * D + c] = et[0] * et[1] * et[2];
+            const int w = c >> 5, bit = c & 31;
+            const uint32_t pc = BPAR[0 * 4 + w] ^ BPAR[1 * 4 + w] ^ BPAR[2 * 4 + w] ^ BPAR[3 * 4 + w];
+            TGC[c] = ((pc >> bit) & 1u) ? -eC : eC;
+            if (c < 4) {
+                PP[0 * 4 + c] = 0u;
+                PP[1 * 4 + c] = BPAR[0 * 4 + c];
+                PP[2 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c];
+                PP[3 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c];
+                SGNC[c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c] ^ BPAR[3 * 4 + c];
             }
         }
         __syncthreads();
 
-        // ---- step 3: band-scaled operands (thread = row, half = 64 channels)
+        // ---- step 3: band-scaled operands (thread = row, 32 channels)
         {
             const bool isq = row < 64;
             const int r = row & 63;
@@ -304,54 +366,48 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const float nrm = NRM[row];
             const float bet = BET[r];
             const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
-#pragma unroll 1
-            for (int cg = 0; cg < 8; ++cg) {
-                const int c0 = 64 * half + 8 * cg;
-                float x[8], gm[8], pb[8];
+            const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
+            const uint32_t swc = SGNC[qq];
+#pragma unroll
+            for (int cg = 0; cg < 4; ++cg) {
+                const int c0 = 32 * qq + 8 * cg;
+                float x[8], E[8], hb[8];
                 unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, c0)), x);
-                *reinterpret_cast<float4 *>(gm) = *reinterpret_cast<const float4 *>(GAM + r * GAM_STRIDE + c0);
-                *reinterpret_cast<float4 *>(gm + 4) = *reinterpret_cast<const float4 *>(GAM + r * GAM_STRIDE + c0 + 4);
-                *reinterpret_cast<float4 *>(pb) = *reinterpret_cast<const float4 *>(TP + band * D + c0);
-                *reinterpret_cast<float4 *>(pb + 4) = *reinterpret_cast<const float4 *>(TP + band * D + c0 + 4);
-                const uint32_t sb = fl.complex_gate ? (SGN[r * 4 + (c0 >> 5)] >> (c0 & 31)) : 0u;
-                const uint32_t sbc = SGNC[c0 >> 5] >> (c0 & 31);
-                float xe[8], inv[8];
+                ld8f(EX + r * E_STRIDE + c0, E);
+                ld8f(TH + band * D + c0, hb);
+                float xe[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float xv = x[e] * nrm * (((sb >> e) & 1u) ? -1.f : 1.f);
-                    const float E = __expf(fmaxf(gm[e] - pb[e], -85.f));
-                    xe[e] = xv * E;
-                    inv[e] = isq ? 0.f : __fdividef(xv, E);
+                    x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
+                    xe[e] = x[e] * E[e];
                 }
-                // A operands of the band products, bands j <= band(r), in TMEM
+                const float rs = isq ? 1.f : bet;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    float y[8];
+                    uint32_t pk[4];
+                    if (j <= band) {
+                        float f[8];
+                        ld8f(TF + (band * 4 + j) * D + c0, f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float f = (j <= band) ? TF[(band * 4 + j) * D + c0 + e] : 0.f;
-                        y[e] = (isq ? xe[e] : bet * xe[e]) * f;
+                        for (int e = 0; e < 4; ++e)
+                            pk[e] = pack_bf16(rs * xe[2 * e] * f[2 * e], rs * xe[2 * e + 1] * f[2 * e + 1]);
+                    } else {
+                        pk[0] = pk[1] = pk[2] = pk[3] = 0u;
                     }
-                    tmem_st4(tbase + lane_off + TC_AOP + 64 * j + 32 * half + 4 * cg,
-                             pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
-                             pack_bf16(y[6], y[7]));
+                    tmem_st4(tbase + lane_off + TC_AOP + 64 * j + 16 * qq + 4 * cg, pk[0], pk[1], pk[2], pk[3]);
                 }
-                float hb[8];
-                *reinterpret_cast<float4 *>(hb) = *reinterpret_cast<const float4 *>(TH + band * D + c0);
-                *reinterpret_cast<float4 *>(hb + 4) = *reinterpret_cast<const float4 *>(TH + band * D + c0 + 4);
-                if (isq) {
-                    float y[8];
+                float y1[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = xe[e] * hb[e];
-                    *reinterpret_cast<uint4 *>(smem + OFF_QG + off_r128(r, c0)) = pack8(y);
+                for (int e = 0; e < 8; ++e) y1[e] = xe[e] * hb[e];
+                if (isq) {
+                    *reinterpret_cast<uint4 *>(smem + OFF_QG + off_r128(r, c0)) = pack8(y1);
                 } else {
-                    float gb[8], y1[8], y2[8];
-                    *reinterpret_cast<float4 *>(gb) = *reinterpret_cast<const float4 *>(TG + band * D + c0);
-                    *reinterpret_cast<float4 *>(gb + 4) = *reinterpret_cast<const float4 *>(TG + band * D + c0 + 4);
+                    float gb[8], inv[8], y2[8];
+                    ld8f(TG + band * D + c0, gb);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        y1[e] = xe[e] * hb[e];
-                        y2[e] = (((sbc >> e) & 1u) ? -1.f : 1.f) * inv[e] * gb[e];
+                        inv[e] = __fdividef(x[e], E[e]);
+                        y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
                     }
                     *reinterpret_cast<uint4 *>(smem + OFF_XR + off_r128(r, c0)) = pack8(inv);
                     *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
@@ -365,16 +421,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncthreads();
 
         // ---- step 4: A_qk / A_kk band products
+        // one thread issues the next chunk's q, k, g loads, another the band MMAs
+        if (tid == 32 && ch + 1 < nch) issue_tma_qkg(ch + 1);
         if (tid == 0) {
             tc_fence_after();
             constexpr uint32_t id = idesc_bf16(128, 16, 0, 0, 0);
-#pragma unroll 1
-            for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_ts(tbase + TC_A + 16 * j, tbase + TC_AOP + 64 * j + 8 * s,
-                           sdesc(sbase + OFF_XR + 4096 * j + 256 * s, 128, 2048, kSwizzleNone), id,
-                           s > 0);
+            for (int s = 0; s < 8; ++s)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_ts(tbase + ((s & 1) ? TC_A_B : TC_A_A) + 16 * j, tbase + TC_AOP + 64 * j + 8 * s,
+                           at(dK64, OFF_XR + 4096 * j + 256 * s), id, s > 1);
             mma_commit(bar_mma);
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
@@ -383,76 +440,142 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ---- step 5: A_qk -> bf16 (lower with diagonal); A_kk -> FP32 (strictly lower)
         {
-            float v[32];
-            tmem_ld32(tbase + lane_off + TC_A + 32 * half, v);
+            float v[16], v2[16];
+            tmem_ld16(tbase + lane_off + TC_A_A + 16 * qq, v);
+            tmem_ld16(tbase + lane_off + TC_A_B + 16 * qq, v2);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += v2[e];
             const int r = row & 63;
             if (row < 64) {
 #pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
+                for (int g8 = 0; g8 < 2; ++g8) {
                     float y[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int i = 32 * half + 8 * g8 + e;
+                        const int i = 16 * qq + 8 * g8 + e;
                         y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
                     }
-                    *reinterpret_cast<uint4 *>(smem + OFF_AQK + off_r64(r, 32 * half + 8 * g8)) = pack8(y);
+                    *reinterpret_cast<uint4 *>(smem + OFF_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = 32 * half + e;
-                    AKK[r * 65 + i] = (i < r) ? v[e] : 0.f;
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    float4 y;
+                    const int i = 16 * qq + 4 * e4;
+                    y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
+                    y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
+                    y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
+                    y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
                 }
             }
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- step 6: Tm = (I + A_kk)^{-1}, 16x16 blocks, FP32; Tm' = Tm diag(beta) -> bf16
+        // ---- step 6: Tm = (I + A_kk)^{-1} in FP32
+        // (a) 16x16 diagonal blocks, one column per thread, right-looking substitution in registers
         if (tid < 64) {
             const int bb = tid >> 4, jj = tid & 15;
-            float x[16];
+            float acc[16], x[16];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                float acc = 0.f;
+            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll
-                for (int i = 0; i < rr; ++i)
-                    if (i >= jj) acc += AKK[(16 * bb + rr) * 65 + 16 * bb + i] * x[i];
-                x[rr] = rr < jj ? 0.f : (rr == jj ? 1.f : -acc);
+            for (int i = 0; i < 16; ++i) {
+                x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
             }
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) TMF[(16 * bb + rr) * 65 + 16 * bb + jj] = x[rr];
+            for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
         }
         __syncthreads();
-#pragma unroll 1
-        for (int bb = 1; bb < 4; ++bb) {
-            for (int o = tid; o < bb * 256; o += NT) {
-                const int j = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-                float acc = 0.f;
-                for (int m = j; m < bb; ++m)
+        // (b) T10 = -D1 (A10 D0), T32 = -D3 (A32 D2); thread = 1 row x 4 columns
+        if (tid < 128) {
+            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
+            float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        acc += AKK[(16 * bb + rr) * 65 + 16 * m + k] * TMF[(16 * m + k) * 65 + 16 * j + cc];
-                RS[(j * 16 + rr) * 17 + cc] = acc;
-            }
-            __syncthreads();
-            for (int o = tid; o < bb * 256; o += NT) {
-                const int j = o >> 8, rr = (o >> 4) & 15, cc = o & 15;
-                float acc = 0.f;
+            for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    if (k <= rr) acc += TMF[(16 * bb + rr) * 65 + 16 * bb + k] * RS[(j * 16 + k) * 17 + cc];
-                TMF[(16 * bb + rr) * 65 + 16 * j + cc] = -acc;
+            for (int k = 0; k < 16; ++k) {
+                const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
+                acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
             }
-            __syncthreads();
+            *reinterpret_cast<float4 *>(RR + (which * 16 + rr) * 20 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         }
-        for (int o = tid; o < 64 * 8; o += NT) {
-            const int r = o >> 3, ig = o & 7;
+        __syncthreads();
+        if (tid < 128) {
+            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
+            float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float ak = k <= rr ? a[k] : 0.f;
+                const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
+                t[0] += ak * z.x; t[1] += ak * z.y; t[2] += ak * z.z; t[3] += ak * z.w;
+            }
+            *reinterpret_cast<float4 *>(TMF + (16 * bi + rr) * AS + 16 * bj + c4) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+        }
+        __syncthreads();
+        // (c) lower-left 32x32: -Y (A_BL X) with X = Tm[0:32,0:32], Y = Tm[32:64,32:64];
+        //     thread = 2 rows x 4 columns of a 32x32 product
+        if (tid < 128) {
+            const int r2 = (tid >> 3) * 2, c4 = (tid & 7) * 4;
+            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int k0 = 0; k0 < 32; k0 += 4) {
+                float a0[4], a1[4];
+                *reinterpret_cast<float4 *>(a0) = *reinterpret_cast<const float4 *>(AKK + (32 + r2) * AS + k0);
+                *reinterpret_cast<float4 *>(a1) = *reinterpret_cast<const float4 *>(AKK + (33 + r2) * AS + k0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int k = k0 + kk;
+                    float4 x = *reinterpret_cast<const float4 *>(TMF + k * AS + c4);
+                    // X is lower triangular: entries above its diagonal are not stored
+                    x.x = k >= c4 + 0 ? x.x : 0.f; x.y = k >= c4 + 1 ? x.y : 0.f;
+                    x.z = k >= c4 + 2 ? x.z : 0.f; x.w = k >= c4 + 3 ? x.w : 0.f;
+                    acc[0][0] += a0[kk] * x.x; acc[0][1] += a0[kk] * x.y; acc[0][2] += a0[kk] * x.z; acc[0][3] += a0[kk] * x.w;
+                    acc[1][0] += a1[kk] * x.x; acc[1][1] += a1[kk] * x.y; acc[1][2] += a1[kk] * x.z; acc[1][3] += a1[kk] * x.w;
+                }
+            }
+            *reinterpret_cast<float4 *>(ZZ + r2 * 36 + c4) = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+            *reinterpret_cast<float4 *>(ZZ + (r2 + 1) * 36 + c4) = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int r2 = (tid >> 3) * 2, c4 = (tid & 7) * 4;
+            float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int k0 = 0; k0 < 32; k0 += 4) {
+                float y0[4], y1[4];
+                *reinterpret_cast<float4 *>(y0) = *reinterpret_cast<const float4 *>(TMF + (32 + r2) * AS + 32 + k0);
+                *reinterpret_cast<float4 *>(y1) = *reinterpret_cast<const float4 *>(TMF + (33 + r2) * AS + 32 + k0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int k = k0 + kk;
+                    const float4 z = *reinterpret_cast<const float4 *>(ZZ + k * 36 + c4);
+                    const float w0 = k <= r2 ? y0[kk] : 0.f, w1 = k <= r2 + 1 ? y1[kk] : 0.f;
+                    t[0][0] += w0 * z.x; t[0][1] += w0 * z.y; t[0][2] += w0 * z.z; t[0][3] += w0 * z.w;
+                    t[1][0] += w1 * z.x; t[1][1] += w1 * z.y; t[1][2] += w1 * z.z; t[1][3] += w1 * z.w;
+                }
+            }
+            *reinterpret_cast<float4 *>(TMF + (32 + r2) * AS + c4) = make_float4(-t[0][0], -t[0][1], -t[0][2], -t[0][3]);
+            *reinterpret_cast<float4 *>(TMF + (33 + r2) * AS + c4) = make_float4(-t[1][0], -t[1][1], -t[1][2], -t[1][3]);
+        }
+        __syncthreads();
+        // (d) Tm' = Tm diag(beta) -> bf16, K-major [r][i]
+        {
+            const int r = tid >> 3, ig = tid & 7;
             float y[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int i = 8 * ig + e;
-                y[e] = (i <= r) ? TMF[r * 65 + i] * BET[i] : 0.f;
+                y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
             }
             *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pack8(y);
         }
@@ -465,9 +588,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t id = idesc_bf16(128, 64, 1, 0, 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
-                const uint64_t bdesc = sdesc(sbase + OFF_TMB + 256 * s, 128, 1024, kSwizzleNone);
-                mma_ss(tbase + TC_W, sdesc(sbase + OFF_YR + 4096 * s, 2048, 128, kSwizzleNone), bdesc, id, s > 0);
-                mma_ss(tbase + TC_U, sdesc(sbase + OFF_STG_V + 2048 * s, 8192, 1024, kSwizzle128B), bdesc, id, s > 0);
+                const uint64_t bdesc = at(dK32, OFF_TMB + 256 * s);
+                mma_ss(tbase + ((s & 1) ? TC_W_B : TC_W_A), at(dMN64, OFF_YR + 4096 * s), bdesc, id, s > 1);
+                mma_ss(tbase + ((s & 1) ? TC_U_B : TC_U_A), at(dV, OFF_STG_V + 2048 * s), bdesc, id, s > 1);
             }
             mma_commit(bar_mma);
         }
@@ -476,17 +599,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
 
         // ---- step 8: prefetch the next chunk; W^T -> bf16 (MN-major [c][r])
-        if (tid == 0 && ch + 1 < nch) issue_tma(ch + 1);
+        if (tid == 32 && ch + 1 < nch) issue_tma_v(ch + 1);
+        float beta_next = 0.f;
+        if (tid < C && ch + 1 < nch && t0 + C + tid < T)
+            beta_next = __bfloat162float(beta[((size_t)b * T + t0 + C + tid) * H + h]);
         {
-            float v[32];
-            tmem_ld32(tbase + lane_off + TC_W + 32 * half, v);
+            float v[16], v2[16];
+            tmem_ld16(tbase + lane_off + TC_W_A + 16 * qq, v);
+            tmem_ld16(tbase + lane_off + TC_W_B + 16 * qq, v2);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += v2[e];
             const int c = row;
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
+            for (int g8 = 0; g8 < 2; ++g8) {
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = v[8 * g8 + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r64(c, 32 * half + 8 * g8)) = pack8(y);
+                *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r64(c, 16 * qq + 8 * g8)) = pack8(y);
             }
         }
         fence_proxy_async();
@@ -500,9 +629,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t id_o = idesc_bf16(128, 64, 1, 0, 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-                const uint64_t adesc = sdesc(sbase + OFF_SB + 4096 * s, 2048, 128, kSwizzleNone);
-                mma_ss(tbase + TC_U, adesc, sdesc(sbase + OFF_YR + 2048 * s, 1024, 128, kSwizzleNone), id_v, 1);
-                mma_ss(tbase + TC_O, adesc, sdesc(sbase + OFF_QG + 256 * s, 128, 2048, kSwizzleNone), id_o, s > 0);
+                const uint64_t adesc = at(dMN64, OFF_SB + 4096 * s);
+                mma_ss(tbase + ((s & 1) ? TC_U_B : TC_U_A), adesc, at(dMN32, OFF_YR + 2048 * s), id_v, 1);
+                mma_ss(tbase + ((s & 1) ? TC_O_B : TC_O_A), adesc, at(dK64, OFF_QG + 256 * s), id_o, s > 1);
             }
             mma_commit(bar_mma);
         }
@@ -512,15 +641,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ---- step 10: V~^T -> bf16 (K-major [j][r])
         {
-            float v[32];
-            tmem_ld32(tbase + lane_off + TC_U + 32 * half, v);
+            float v[16], v2[16];
+            tmem_ld16(tbase + lane_off + TC_U_A + 16 * qq, v);
+            tmem_ld16(tbase + lane_off + TC_U_B + 16 * qq, v2);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += v2[e];
             const int j = row;
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
+            for (int g8 = 0; g8 < 2; ++g8) {
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = v[8 * g8 + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r64(j, 32 * half + 8 * g8)) = pack8(y);
+                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r64(j, 16 * qq + 8 * g8)) = pack8(y);
             }
         }
         fence_proxy_async();
@@ -534,9 +666,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 0, 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
-                const uint64_t vt = sdesc(sbase + OFF_VT + 256 * s, 128, 1024, kSwizzleNone);
-                mma_ss(tbase + TC_O, vt, sdesc(sbase + OFF_AQK + 256 * s, 128, 1024, kSwizzleNone), id_o, 1);
-                mma_ss(tbase + TC_S, sdesc(sbase + OFF_KD + 4096 * s, 2048, 128, kSwizzleNone), vt, id_s, s > 0);
+                const uint64_t vt = at(dK32, OFF_VT + 256 * s);
+                mma_ss(tbase + ((s & 1) ? TC_O_B : TC_O_A), vt, at(dK32, OFF_AQK + 256 * s), id_o, 1);
+                mma_ss(tbase + ((s & 1) ? TC_S_B : TC_S_A), at(dMN64, OFF_KD + 4096 * s), vt, id_s, s > 1);
             }
             mma_commit(bar_mma);
         }
@@ -544,43 +676,55 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---- step 12: outputs; S <- gC * S + dS (FP32) and its bf16 copy
+        // ---- step 12: outputs through a smem staging tile; S <- gC * S + dS (FP32) and its bf16 copy
         {
-            float v[32];
-            tmem_ld32(tbase + lane_off + TC_O + 32 * half, v);
-            const int j = row;
+            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_QG);   // [64 r][128 j]
+            {
+                float o1[16], o2[16];
+                tmem_ld16(tbase + lane_off + TC_O_A + 16 * qq, o1);
+                tmem_ld16(tbase + lane_off + TC_O_B + 16 * qq, o2);
+                const int j = row;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int r = 32 * half + e;
-                if (r < n)
-                    out[(((size_t)b * T + t0 + r) * H + h) * D + j] = __float2bfloat16_rn(fl.scale * v[e]);
+                for (int e = 0; e < 16; ++e)
+                    ost[(16 * qq + e) * D + j] = __float2bfloat16_rn(fl.scale * (o1[e] + o2[e]));
             }
             const int c = row;
             const float gc = TGC[c];
+            float v[32];
+            tmem_ld32(tbase + lane_off + TC_S_A + 32 * qq, v);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                tmem_ld32(tbase + lane_off + TC_S + 64 * half + 32 * part, v);
+            for (int e = 0; e < 32; ++e) S[e] = fmaf(gc, S[e], v[e]);
+            tmem_ld32(tbase + lane_off + TC_S_B + 32 * qq, v);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) S[32 * part + e] = fmaf(gc, S[32 * part + e], v[e]);
-            }
+            for (int e = 0; e < 32; ++e) S[e] += v[e];
 #pragma unroll
-            for (int jg = 0; jg < 8; ++jg) {
+            for (int jg = 0; jg < 4; ++jg) {
                 float x[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_SB + off_r128(c, 64 * half + 8 * jg)) = pack8(x);
+                *reinterpret_cast<uint4 *>(smem + OFF_SB + off_r128(c, 32 * qq + 8 * jg)) = pack8(x);
             }
         }
+        if (tid < C) BET_S[tid] = beta_next;
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+            const int q16 = tid + NT * m, r = q16 >> 4, cj = q16 & 15;
+            if (r < n) {
+                const uint4 val = *reinterpret_cast<const uint4 *>(smem + OFF_QG + r * 256 + cj * 16);
+                *reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 8 * cj) = val;
+            }
+        }
+        __syncthreads();
     }
 
     if (ok && S_T) {
-        float *dst = S_T + ((size_t)bh * D + row) * D + 64 * half;
+        float *dst = S_T + ((size_t)bh * D + row) * D + 32 * qq;
 #pragma unroll
-        for (int j = 0; j < 64; j += 4)
+        for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
     if (!ok) {

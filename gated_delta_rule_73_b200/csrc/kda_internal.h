@@ -37,9 +37,10 @@ struct ChunkArgs {
 struct PrologueArgs {
     const void *q_pre, *k_pre, *v_pre, *conv_w, *z;
     const float *A, *beta_logit;
-    bool bf16;
+    bool bf16;                           // element type of the raw inputs
+    bool out_bf16;                       // outputs in bf16 (tensor-core path) or FP32
     int B, T, H, dk, dv;
-    float *qc, *kc, *vc, *g, *beta;      // FP32 outputs in the workspace
+    void *qc, *kc, *vc, *g, *beta;       // outputs in the workspace
 };
 
 // Workspace of the FP32 two-phase chunk path.

@@ -11,8 +11,9 @@
 // Page "Kimi K3 模型结构（2）", Q&A on the decay function: the bounded log-decay
 // g = -5 * sigmoid(exp(A_h) * z), g in (-5, 0).
 //
-// Outputs are FP32 (so the cumulative decay is not rounded before the chunk
-// kernel takes it); the L2 norm of q and k is applied by the chunk kernel.
+// Outputs are bf16 when the tensor-core chunk kernel follows (its operands are
+// bf16 anyway) and FP32 for the FP32 chunk path; the L2 norm of q and k is
+// applied by the chunk kernel.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -21,14 +22,14 @@ namespace kda {
 namespace {
 __device__ __forceinline__ float sigm(float x) { return 1.f / (1.f + expf(-x)); }
 
-template <typename T>
+template <typename T, typename TO>
 __global__ void __launch_bounds__(256)
 prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
                 const T *__restrict__ v_pre, const T *__restrict__ conv_w,
                 const T *__restrict__ z, const float *__restrict__ A,
                 const float *__restrict__ b_logit, int T_, int H, int D, long long total,
-                float *__restrict__ qc, float *__restrict__ kc, float *__restrict__ vc,
-                float *__restrict__ g, float *__restrict__ beta) {
+                TO *__restrict__ qc, TO *__restrict__ kc, TO *__restrict__ vc,
+                TO *__restrict__ g, TO *__restrict__ beta) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= total) return;
     const int d = (int)(idx % D);
@@ -39,7 +40,7 @@ prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
     const long long nch = HD;                    // channels per branch
     const long long ch = (long long)h * D + d;
     const T *src[3] = {q_pre, k_pre, v_pre};
-    float *dst[3] = {qc, kc, vc};
+    TO *dst[3] = {qc, kc, vc};
 #pragma unroll
     for (int s = 0; s < 3; ++s) {
         const T *w = conv_w + ((long long)s * nch + ch) * 4;
@@ -49,27 +50,28 @@ prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
             const int tt = t - 3 + j;
             if (tt >= 0) acc += to_f32(w[j]) * to_f32(src[s][idx - (long long)(3 - j) * HD]);
         }
-        dst[s][idx] = acc * sigm(acc);
+        dst[s][idx] = from_f32<TO>(acc * sigm(acc));
     }
-    g[idx] = -5.f * sigm(expf(A[h]) * to_f32(z[idx]));
-    if (d == 0) beta[bth] = sigm(b_logit[bth]);
+    g[idx] = from_f32<TO>(-5.f * sigm(expf(A[h]) * to_f32(z[idx])));
+    if (d == 0) beta[bth] = from_f32<TO>(sigm(b_logit[bth]));
 }
 }  // namespace
+
+template <typename T, typename TO>
+static void launch_t(const PrologueArgs &a, long long total, unsigned blocks, cudaStream_t st) {
+    prologue_kernel<T, TO><<<blocks, 256, 0, st>>>(
+        (const T *)a.q_pre, (const T *)a.k_pre, (const T *)a.v_pre, (const T *)a.conv_w,
+        (const T *)a.z, a.A, a.beta_logit, a.T, a.H, a.dk, total, (TO *)a.qc, (TO *)a.kc,
+        (TO *)a.vc, (TO *)a.g, (TO *)a.beta);
+}
 
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st) {
     const long long total = (long long)a.B * a.T * a.H * a.dk;
     const unsigned blocks = (unsigned)((total + 255) / 256);
-    if (a.bf16)
-        prologue_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)a.q_pre, (const __nv_bfloat16 *)a.k_pre,
-            (const __nv_bfloat16 *)a.v_pre, (const __nv_bfloat16 *)a.conv_w,
-            (const __nv_bfloat16 *)a.z, a.A, a.beta_logit, a.T, a.H, a.dk, total, a.qc, a.kc, a.vc,
-            a.g, a.beta);
-    else
-        prologue_kernel<float><<<blocks, 256, 0, st>>>(
-            (const float *)a.q_pre, (const float *)a.k_pre, (const float *)a.v_pre,
-            (const float *)a.conv_w, (const float *)a.z, a.A, a.beta_logit, a.T, a.H, a.dk, total,
-            a.qc, a.kc, a.vc, a.g, a.beta);
+    if (a.bf16 && a.out_bf16) launch_t<__nv_bfloat16, __nv_bfloat16>(a, total, blocks, st);
+    else if (a.bf16) launch_t<__nv_bfloat16, float>(a, total, blocks, st);
+    else if (a.out_bf16) launch_t<float, __nv_bfloat16>(a, total, blocks, st);
+    else launch_t<float, float>(a, total, blocks, st);
     return cudaGetLastError();
 }
 
