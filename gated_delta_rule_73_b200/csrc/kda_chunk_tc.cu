@@ -59,14 +59,13 @@ constexpr uint32_t OFF_AKK = OFF_GAM;         // fp32 [64][68]
 constexpr uint32_t OFF_TMF = OFF_GAM + 17408; // fp32 [64][68]
 constexpr uint32_t OFF_VT = OFF_GAM;          // bf16 V~^T, K-major [128 j][64 r]
 constexpr uint32_t OFF_QG = OFF_GAM + 36864;  // bf16 Q e^gamma [64 r][128 c]; later O staging [64][128]
-constexpr uint32_t OFF_XR = OFF_QG + 16384;   // bf16 K e^{p-gamma} [64][128]; later A_qk + (scratch, Tm')
-constexpr uint32_t OFF_AQK = OFF_XR;          // bf16 [64 r][64 i]
-constexpr uint32_t OFF_TMB = OFF_XR + 8192;   // bf16 [64 r][64 i]
-constexpr uint32_t OFF_RZ = OFF_XR + 8192;    // fp32 inverse scratch: R [2][16][20], Z [32][36]
-constexpr uint32_t OFF_YR = OFF_XR + 16384;   // bf16 K e^gamma [64][128]; later W^T [128][64]
+constexpr uint32_t OFF_BOP = OFF_QG + 16384;  // bf16 band-pair B operand [160][128]; later A_qk, scratch, Tm'
+constexpr uint32_t OFF_AQK = OFF_BOP;         // bf16 [64 r][64 i]
+constexpr uint32_t OFF_TMB = OFF_BOP + 8192;  // bf16 [64 r][64 i]
+constexpr uint32_t OFF_RZ = OFF_BOP + 8192;   // fp32 inverse scratch: R [2][16][20], Z [32][36]
+constexpr uint32_t OFF_YR = OFF_BOP + 40960;  // bf16 K e^gamma [64][128]; later W^T [128][64]
 constexpr uint32_t OFF_KD = OFF_YR + 16384;   // bf16 K e^{gamma_C-gamma} [64][128]
-constexpr uint32_t OFF_SB = OFF_KD + 16384;   // bf16 S [128 c][128 j]
-constexpr uint32_t OFF_TAB = OFF_SB + 32768;  // tables
+constexpr uint32_t OFF_TAB = OFF_KD + 16384;  // tables
 constexpr uint32_t TAB_TOT = 0;               // fp32 [4][128] band sums of log-decay
 constexpr uint32_t TAB_F = TAB_TOT + 2048;    // fp32 [4][4][128] e^{p_b - p_j}
 constexpr uint32_t TAB_G = TAB_F + 8192;      // fp32 [4][128] e^{gamma_C - p_b}
@@ -83,22 +82,19 @@ constexpr uint32_t SMEM_USED = OFF_TAB + TAB_BYTES;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for the 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_TMF + 64 * AS * 4 <= OFF_QG, "inverse scratch fits");
+static_assert(OFF_RZ + 7168 <= OFF_BOP + 16384, "inverse scratch fits");
 
-// TMEM columns (512 allocated).  Every product is split over two accumulators
-// (even / odd K-steps) so that consecutive MMAs never wait on each other; the
-// halves are summed when read back.  Regions are reused once they are dead:
-//   [0,256)   band operands (step 3-4) | W^T_b [0,64), U^T_b [64,128) (7-10),
-//             O^T_a [128,192), O^T_b [192,256) (9-12) | dS_a [0,128) (11-12)
-//   [256,320) A_a (4-5)  | dS_b [256,384) (11-12)
-//   [320,384) W^T_a (7-8)
-//   [384,448) U^T_a, then V~^T_a (7-10)
-//   [448,512) A_b (4-5)
-constexpr uint32_t TC_AOP = 0;
-constexpr uint32_t TC_A_A = 256, TC_A_B = 448;
-constexpr uint32_t TC_W_A = 320, TC_W_B = 0;
-constexpr uint32_t TC_U_A = 384, TC_U_B = 64;
-constexpr uint32_t TC_O_A = 128, TC_O_B = 192;
-constexpr uint32_t TC_S_A = 0, TC_S_B = 256;
+// The ten (row band b, column band j <= b) pairs of the 64 x 64 intra-chunk
+// matrices, as 16-column groups of one N = 160 product: pair(b, j) = P0[j] + b - j.
+__device__ __forceinline__ int pair_of(int b, int j) { return (j == 0 ? 0 : j == 1 ? 4 : j == 2 ? 7 : 9) + b - j; }
+
+// TMEM columns (512 allocated)
+//   [0,64)    X: rows scaled by their own band reference (A of the band product), steps 3-4
+//   [64,224)  D: the ten band-pair products, steps 4-5
+//   [224,288) W^T (7-8)   [288,352) U^T, then V~^T (7-10)
+//   [128,192) O^T (9-12)  [0,128) dS^T (11-12)
+//   [448,512) S^T in bf16: the A operand of the state products (persistent)
+constexpr uint32_t TC_X = 0, TC_D = 64, TC_W = 224, TC_U = 288, TC_O = 128, TC_S = 0, TC_SOP = 448;
 
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -171,7 +167,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *TGC = reinterpret_cast<float *>(smem + OFF_TAB + TAB_GC);
     float *NRM = reinterpret_cast<float *>(smem + OFF_TAB + TAB_NRM);
     float *BET = reinterpret_cast<float *>(smem + OFF_TAB + TAB_BET);
-    float *BET_S = BET;
     uint32_t *SGNL = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNL);
     uint32_t *BPAR = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_BPAR);
     uint32_t *PP = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_PP);
@@ -200,6 +195,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sh.tmem_base;
+    const uint32_t tl = tbase + lane_off;             // this warp's lane quarter
     // descriptor bases (start address = the smem base); a tile at byte offset `off`
     // is base + (off >> 4) since every address stays below 256 KB
     const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);    // K-major [rows][128]
@@ -212,6 +208,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // the next chunk's q, k, g tiles are requested as soon as this chunk's operands are
     // built (they are free then), its v tile once the U product has read it
     auto issue_tma_qkg = [&](int ch) {
+        fence_proxy_async();   // order the threads' earlier reads of the tiles before the overwrite
         mbar_arrive_expect_tx(bar_tma, kTmaBytes);
         const int t0 = ch * C;
 #pragma unroll
@@ -222,44 +219,46 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     };
     auto issue_tma_v = [&](int ch) {
+        fence_proxy_async();
         const int t0 = ch * C;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_tma, hf * 64, h, t0, b);
     };
-    // every thread waits; a give-up anywhere makes the whole CTA stop together
+    // one thread polls the mbarrier (512 pollers would compete with the tensor core for
+    // shared memory); the rest wait at the CTA barrier.  A give-up stops the whole CTA.
     auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
-        if (!mbar_wait_bounded(bar, phase, kWaitLimit)) {
+        if (tid == 0 && !mbar_wait_bounded(bar, phase, kWaitLimit)) {
             sh.abort = 1;
             g_kda_tc_error = 1;
         }
         __syncthreads();
         return sh.abort == 0;
     };
-    if (tid == 0 && nch > 0) {
+    if (tid == 32 && nch > 0) {
         issue_tma_qkg(0);
         issue_tma_v(0);
     }
     // beta of the first chunk; later chunks' beta is fetched a chunk ahead
-    if (tid < C) BET_S[tid] = tid < T ? __bfloat162float(beta[((size_t)b * T + tid) * H + h]) : 0.f;
+    if (tid < C) BET[tid] = tid < T ? __bfloat162float(beta[((size_t)b * T + tid) * H + h]) : 0.f;
 
-    // the FP32 state: thread (row = key channel c, qq) owns S[c][32 qq .. 32 qq + 31]
+    // The FP32 state, transposed: thread (lane j, qq) owns S^T[j][32 qq .. 32 qq + 31],
+    // i.e. S[c][j] for its 32 key channels c; its bf16 copy lives in TMEM.
     float S[32];
+    auto store_state_operand = [&]() {
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4)
+            tmem_st4(tl + TC_SOP + 16 * qq + 4 * e4, pack_bf16(S[8 * e4], S[8 * e4 + 1]),
+                     pack_bf16(S[8 * e4 + 2], S[8 * e4 + 3]), pack_bf16(S[8 * e4 + 4], S[8 * e4 + 5]),
+                     pack_bf16(S[8 * e4 + 6], S[8 * e4 + 7]));
+    };
     {
-        const int c = row;
-        const float *src = S0 ? S0 + ((size_t)bh * D + c) * D + 32 * qq : nullptr;
+        const int j = row;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            float4 v4 = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
-            S[j] = v4.x; S[j + 1] = v4.y; S[j + 2] = v4.z; S[j + 3] = v4.w;
-        }
-#pragma unroll
-        for (int jg = 0; jg < 4; ++jg) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e];
-            *reinterpret_cast<uint4 *>(smem + OFF_SB + off_r128(c, 32 * qq + 8 * jg)) = pack8(x);
-        }
+        for (int e = 0; e < 32; ++e)
+            S[e] = S0 ? S0[((size_t)bh * D + 32 * qq + e) * D + j] : 0.f;
+        store_state_operand();
+        tmem_wait_st();
     }
 
     uint32_t ph_tma = 0, ph_mma = 0;
@@ -270,7 +269,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!(ok = wait_all(bar_tma, ph_tma))) break;
         ph_tma ^= 1;
 
-        // ---- step 1: band-local cumulative log-decay (4 bands x 128 channels) | row norms | beta
+        // ---- step 1: band-local cumulative log-decay (4 bands x 128 channels) | row norms
         {
             const int c = tid & 127, p = tid >> 7;
             float gv[16];
@@ -358,7 +357,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         __syncthreads();
 
-        // ---- step 3: band-scaled operands (thread = row, 32 channels)
+        // ---- step 3: operands (thread = row, 32 channels).  Rows are scaled by their own
+        //      band reference; the band-pair factor e^{p_b - p_j} goes onto the B operand.
         {
             const bool isq = row < 64;
             const int r = row & 63;
@@ -375,30 +375,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, c0)), x);
                 ld8f(EX + r * E_STRIDE + c0, E);
                 ld8f(TH + band * D + c0, hb);
-                float xe[8];
+                float xe[8], y1[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
                     xe[e] = x[e] * E[e];
+                    y1[e] = xe[e] * hb[e];
                 }
                 const float rs = isq ? 1.f : bet;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t pk[4];
-                    if (j <= band) {
-                        float f[8];
-                        ld8f(TF + (band * 4 + j) * D + c0, f);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            pk[e] = pack_bf16(rs * xe[2 * e] * f[2 * e], rs * xe[2 * e + 1] * f[2 * e + 1]);
-                    } else {
-                        pk[0] = pk[1] = pk[2] = pk[3] = 0u;
-                    }
-                    tmem_st4(tbase + lane_off + TC_AOP + 64 * j + 16 * qq + 4 * cg, pk[0], pk[1], pk[2], pk[3]);
-                }
-                float y1[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) y1[e] = xe[e] * hb[e];
+                tmem_st4(tl + TC_X + 16 * qq + 4 * cg, pack_bf16(rs * xe[0], rs * xe[1]),
+                         pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
+                         pack_bf16(rs * xe[6], rs * xe[7]));
                 if (isq) {
                     *reinterpret_cast<uint4 *>(smem + OFF_QG + off_r128(r, c0)) = pack8(y1);
                 } else {
@@ -409,43 +396,57 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         inv[e] = __fdividef(x[e], E[e]);
                         y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
                     }
-                    *reinterpret_cast<uint4 *>(smem + OFF_XR + off_r128(r, c0)) = pack8(inv);
                     *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
                     *reinterpret_cast<uint4 *>(smem + OFF_KD + off_r128(r, c0)) = pack8(y2);
+                    // B rows of the pairs (b, band) for b = band..3
+                    for (int bb = band; bb < 4; ++bb) {
+                        float f[8], y3[8];
+                        ld8f(TF + (bb * 4 + band) * D + c0, f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
+                        const int brow = 16 * pair_of(bb, band) + (r & 15);
+                        *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
+                    }
                 }
             }
         }
         tmem_wait_st();
-        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // ---- step 4: A_qk / A_kk band products
-        // one thread issues the next chunk's q, k, g loads, another the band MMAs
-        if (tid == 32 && ch + 1 < nch) issue_tma_qkg(ch + 1);
+        // ---- step 4: all ten band-pair products in one N = 160 product
+        //      (one thread issues the next chunk's q, k, g loads, another the MMAs)
         if (tid == 0) {
+            fence_proxy_async();   // the threads' smem writes (ordered by the barrier) -> async proxy
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 16, 0, 0, 0);
+            constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_ts(tbase + ((s & 1) ? TC_A_B : TC_A_A) + 16 * j, tbase + TC_AOP + 64 * j + 8 * s,
-                           at(dK64, OFF_XR + 4096 * j + 256 * s), id, s > 1);
+                mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
             mma_commit(bar_mma);
         }
         if (!(ok = wait_all(bar_mma, ph_mma))) break;
         ph_mma ^= 1;
         tc_fence_after();
+        if (tid == 32 && ch + 1 < nch) issue_tma_qkg(ch + 1);
 
-        // ---- step 5: A_qk -> bf16 (lower with diagonal); A_kk -> FP32 (strictly lower)
+        // ---- step 5: A_qk -> bf16 (lower with diagonal); A_kk -> FP32 (strictly lower).
+        //      A warp's 32 rows span two row bands; it reads both bands' columns for
+        //      column band j = qq and each thread keeps its own.
         {
+            const int r = row & 63, band = r >> 4;
+            const int b_lo = (quad & 1) * 2;
             float v[16], v2[16];
-            tmem_ld16(tbase + lane_off + TC_A_A + 16 * qq, v);
-            tmem_ld16(tbase + lane_off + TC_A_B + 16 * qq, v2);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] += v2[e];
-            const int r = row & 63;
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
+            if (qq <= b_lo + 1) {
+                tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, qq), v2);
+                if (band == b_lo + 1) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                }
+            }
             if (row < 64) {
 #pragma unroll
                 for (int g8 = 0; g8 < 2; ++g8) {
@@ -579,18 +580,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pack8(y);
         }
-        fence_proxy_async();
         __syncthreads();
 
         // ---- step 7: W^T = KG^T Tm'^T,  U^T = V^T Tm'^T
         if (tid == 0) {
+            fence_proxy_async();   // the threads' smem writes (ordered by the barrier) -> async proxy
             tc_fence_after();
             constexpr uint32_t id = idesc_bf16(128, 64, 1, 0, 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const uint64_t bdesc = at(dK32, OFF_TMB + 256 * s);
-                mma_ss(tbase + ((s & 1) ? TC_W_B : TC_W_A), at(dMN64, OFF_YR + 4096 * s), bdesc, id, s > 1);
-                mma_ss(tbase + ((s & 1) ? TC_U_B : TC_U_A), at(dV, OFF_STG_V + 2048 * s), bdesc, id, s > 1);
+                mma_ss(tbase + TC_W, at(dMN64, OFF_YR + 4096 * s), bdesc, id, s > 0);
+                mma_ss(tbase + TC_U, at(dV, OFF_STG_V + 2048 * s), bdesc, id, s > 0);
             }
             mma_commit(bar_mma);
         }
@@ -598,17 +599,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---- step 8: prefetch the next chunk; W^T -> bf16 (MN-major [c][r])
+        // ---- step 8: prefetch the next chunk's v and beta; W^T -> bf16 (MN-major [c][r])
         if (tid == 32 && ch + 1 < nch) issue_tma_v(ch + 1);
         float beta_next = 0.f;
         if (tid < C && ch + 1 < nch && t0 + C + tid < T)
             beta_next = __bfloat162float(beta[((size_t)b * T + t0 + C + tid) * H + h]);
         {
-            float v[16], v2[16];
-            tmem_ld16(tbase + lane_off + TC_W_A + 16 * qq, v);
-            tmem_ld16(tbase + lane_off + TC_W_B + 16 * qq, v2);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] += v2[e];
+            float v[16];
+            tmem_ld16(tl + TC_W + 16 * qq, v);
             const int c = row;
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
@@ -618,20 +616,19 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r64(c, 16 * qq + 8 * g8)) = pack8(y);
             }
         }
-        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // ---- step 9: V~^T = U^T - S^T W^T;  O^T = S^T Qg^T
+        // ---- step 9: V~^T = U^T - S^T W^T;  O^T = S^T Qg^T  (S^T from TMEM)
         if (tid == 0) {
+            fence_proxy_async();   // the threads' smem writes (ordered by the barrier) -> async proxy
             tc_fence_after();
-            constexpr uint32_t id_v = idesc_bf16(128, 64, 1, 1, 1);
-            constexpr uint32_t id_o = idesc_bf16(128, 64, 1, 0, 0);
+            constexpr uint32_t id_v = idesc_bf16(128, 64, 0, 1, 1);
+            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-                const uint64_t adesc = at(dMN64, OFF_SB + 4096 * s);
-                mma_ss(tbase + ((s & 1) ? TC_U_B : TC_U_A), adesc, at(dMN32, OFF_YR + 2048 * s), id_v, 1);
-                mma_ss(tbase + ((s & 1) ? TC_O_B : TC_O_A), adesc, at(dK64, OFF_QG + 256 * s), id_o, s > 1);
+                mma_ts(tbase + TC_U, tbase + TC_SOP + 8 * s, at(dMN32, OFF_YR + 2048 * s), id_v, 1);
+                mma_ts(tbase + TC_O, tbase + TC_SOP + 8 * s, at(dK64, OFF_QG + 256 * s), id_o, s > 0);
             }
             mma_commit(bar_mma);
         }
@@ -641,11 +638,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ---- step 10: V~^T -> bf16 (K-major [j][r])
         {
-            float v[16], v2[16];
-            tmem_ld16(tbase + lane_off + TC_U_A + 16 * qq, v);
-            tmem_ld16(tbase + lane_off + TC_U_B + 16 * qq, v2);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] += v2[e];
+            float v[16];
+            tmem_ld16(tl + TC_U + 16 * qq, v);
             const int j = row;
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
@@ -655,20 +649,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r64(j, 16 * qq + 8 * g8)) = pack8(y);
             }
         }
-        fence_proxy_async();
         tc_fence_before();
         __syncthreads();
 
-        // ---- step 11: O^T += V~^T A_qk^T;  dS = Kd^T V~
+        // ---- step 11: O^T += V~^T A_qk^T;  dS^T = V~^T Kd
         if (tid == 0) {
+            fence_proxy_async();   // the threads' smem writes (ordered by the barrier) -> async proxy
             tc_fence_after();
             constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
-            constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 0, 0);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1, 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 const uint64_t vt = at(dK32, OFF_VT + 256 * s);
-                mma_ss(tbase + ((s & 1) ? TC_O_B : TC_O_A), vt, at(dK32, OFF_AQK + 256 * s), id_o, 1);
-                mma_ss(tbase + ((s & 1) ? TC_S_B : TC_S_A), at(dMN64, OFF_KD + 4096 * s), vt, id_s, s > 1);
+                mma_ss(tbase + TC_O, vt, at(dK32, OFF_AQK + 256 * s), id_o, 1);
+                mma_ss(tbase + TC_S, vt, at(dMN64, OFF_KD + 4096 * s), id_s, s > 0);
             }
             mma_commit(bar_mma);
         }
@@ -676,37 +670,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ph_mma ^= 1;
         tc_fence_after();
 
-        // ---- step 12: outputs through a smem staging tile; S <- gC * S + dS (FP32) and its bf16 copy
+        // ---- step 12: outputs through a smem staging tile; S <- diag(gC) S + dS in FP32
+        //      and its bf16 copy back into TMEM
         {
             __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_QG);   // [64 r][128 j]
             {
-                float o1[16], o2[16];
-                tmem_ld16(tbase + lane_off + TC_O_A + 16 * qq, o1);
-                tmem_ld16(tbase + lane_off + TC_O_B + 16 * qq, o2);
+                float o[16];
+                tmem_ld16(tl + TC_O + 16 * qq, o);
                 const int j = row;
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    ost[(16 * qq + e) * D + j] = __float2bfloat16_rn(fl.scale * (o1[e] + o2[e]));
+                for (int e = 0; e < 16; ++e) ost[(16 * qq + e) * D + j] = __float2bfloat16_rn(fl.scale * o[e]);
             }
-            const int c = row;
-            const float gc = TGC[c];
-            float v[32];
-            tmem_ld32(tbase + lane_off + TC_S_A + 32 * qq, v);
+            float v[32], gcv[32];
+            tmem_ld32(tl + TC_S + 32 * qq, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) S[e] = fmaf(gc, S[e], v[e]);
-            tmem_ld32(tbase + lane_off + TC_S_B + 32 * qq, v);
+            for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4 *>(gcv + e) = *reinterpret_cast<const float4 *>(TGC + 32 * qq + e);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) S[e] += v[e];
-#pragma unroll
-            for (int jg = 0; jg < 4; ++jg) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = S[jg * 8 + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_SB + off_r128(c, 32 * qq + 8 * jg)) = pack8(x);
-            }
+            for (int e = 0; e < 32; ++e) S[e] = fmaf(gcv[e], S[e], v[e]);
+            store_state_operand();
+            tmem_wait_st();
         }
-        if (tid < C) BET_S[tid] = beta_next;
-        fence_proxy_async();
+        if (tid < C) BET[tid] = beta_next;
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
@@ -722,10 +707,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 
     if (ok && S_T) {
-        float *dst = S_T + ((size_t)bh * D + row) * D + 32 * qq;
+        const int j = row;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        for (int e = 0; e < 32; ++e) S_T[((size_t)bh * D + 32 * qq + e) * D + j] = S[e];
     }
     if (!ok) {
         // drain what may still be in flight (bounded), then release TMEM
