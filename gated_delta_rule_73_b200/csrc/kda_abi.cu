@@ -31,7 +31,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int check_opts(const kda_opts &o) {
     if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
-    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX)) return KDA_ERR_ARG;
+    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED)) return KDA_ERR_ARG;
     if (!isfinite(o.scale)) return KDA_ERR_ARG;
     if (o.n_events < 0 || (o.n_events > 0 && !o.events)) return KDA_ERR_ARG;
     return KDA_OK;
@@ -59,8 +59,15 @@ KernelFlags kflags(const kda_opts &o) {
     return f;
 }
 
-// the bf16 dk = dv = 128 chunk forward runs the fused tensor-core kernel (no workspace)
+// the bf16 dk = dv = 128 chunk forward runs on tensor cores: by default a parallel
+// per-chunk prep kernel and a per-head scan (workspace: one record per chunk and
+// head); with KDA_FUSED one fused kernel per sequence (no workspace)
 bool use_tc(const kda_opts &o, int dk, int dv) { return o.dtype == KDA_BF16 && dk == 128 && dv == 128; }
+bool use_fused(const kda_opts &o) { return (o.flags & KDA_FUSED) != 0; }
+size_t tc_ws(const kda_opts &o, int B, int T, int H) {
+    if (use_fused(o) || B <= 0 || T <= 0 || H <= 0) return 0;
+    return round_up(chunk_tc2_workspace_bytes(B, T, H), kAlignWs);
+}
 
 size_t chunk_ws(int B, int T, int H, int dk, int dv) {
     if (B <= 0 || T <= 0 || H <= 0) return 0;
@@ -69,7 +76,7 @@ size_t chunk_ws(int B, int T, int H, int dk, int dv) {
 
 // The prologue's outputs are bf16 when the tensor-core chunk kernel follows
 // (bf16 activations, dk = dv = 128; it needs no further workspace), FP32 otherwise.
-size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, bool tc, size_t *off) {
+size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, bool tc, size_t tc_extra, size_t *off) {
     // off[0..5]: qc, kc, vc, g, beta, chunk workspace
     const size_t rows = (size_t)B * T * H;
     const size_t e = tc ? 2 : 4;
@@ -79,7 +86,7 @@ size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, bool tc, size_t *o
     off[2] = o; o = round_up(o + rows * dv * e, kAlignWs);
     off[3] = o; o = round_up(o + rows * dk * e, kAlignWs);
     off[4] = o; o = round_up(o + rows * e, kAlignWs);
-    off[5] = o; o += tc ? 0 : chunk_ws(B, T, H, dk, dv);
+    off[5] = o; o += tc ? tc_extra : chunk_ws(B, T, H, dk, dv);
     return o;
 }
 
@@ -91,10 +98,12 @@ int finish_identity(const float *S0, float *S_T, int B, int H, int dk, int dv, c
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-int run_chunk(ChunkArgs &a, cudaStream_t st) {
+int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
     int launches = 0;
     a.launch_idx = &launches;
-    cudaError_t e = chunk_tc_supported(a) ? launch_chunk_tc(a, st) : launch_chunk_ref(a, st);
+    cudaError_t e = !chunk_tc_supported(a) ? launch_chunk_ref(a, st)
+                    : fused                 ? launch_chunk_tc(a, st)
+                                            : launch_chunk_tc2(a, st);
     if (e == cudaSuccess && a.events && launches < a.n_events) cudaEventRecord(a.events[launches], st);
     if (e == cudaErrorInvalidValue) return KDA_ERR_UNSUPPORTED;
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -123,7 +132,7 @@ const char *kda_status_string(int s) {
 size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, const kda_opts *opts) {
     const kda_opts o = resolve(opts);
     if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
-    if (use_tc(o, dk, dv)) return 0;
+    if (use_tc(o, dk, dv)) return tc_ws(o, B, T, H);
     return chunk_ws(B, T, H, dk, dv);
 }
 
@@ -132,7 +141,7 @@ size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, const k
     if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
     if (B <= 0 || T <= 0 || H <= 0) return 0;
     size_t off[6];
-    return prologue_ws_parts(B, T, H, dk, dv, use_tc(o, dk, dv), off);
+    return prologue_ws_parts(B, T, H, dk, dv, use_tc(o, dk, dv), tc_ws(o, B, T, H), off);
 }
 
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -151,7 +160,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     const void *ptrs[] = {q, k, v, g, beta, S0, out, S_T, o.workspace};
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_ALIGN;
-    const size_t need = use_tc(o, dk, dv) ? 0 : chunk_ws(B, T, H, dk, dv);
+    const size_t need = use_tc(o, dk, dv) ? tc_ws(o, B, T, H) : chunk_ws(B, T, H, dk, dv);
     if (need > 0 && (!o.workspace || o.workspace_bytes < need)) return KDA_ERR_WORKSPACE;
 
     ChunkArgs a;
@@ -164,7 +173,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     a.fl = kflags(o);
     a.workspace = o.workspace; a.workspace_bytes = o.workspace_bytes;
     a.events = o.events; a.n_events = o.n_events;
-    return run_chunk(a, stream);
+    return run_chunk(a, use_fused(o), stream);
 }
 
 int kda_recurrent_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -214,7 +223,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
         if (!aligned16(p)) return KDA_ERR_ALIGN;
     size_t off[6];
     const bool tc = use_tc(o, dk, dv);
-    const size_t need = prologue_ws_parts(B, T, H, dk, dv, tc, off);
+    const size_t need = prologue_ws_parts(B, T, H, dk, dv, tc, tc ? tc_ws(o, B, T, H) : 0, off);
     if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
     char *ws = (char *)o.workspace;
 
@@ -246,7 +255,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     a.workspace_bytes = need - off[5];
     a.events = o.events; a.n_events = o.n_events;
     a.launch_idx = &launches;
-    e = tc ? launch_chunk_tc(a, stream) : launch_chunk_ref(a, stream);
+    e = !tc ? launch_chunk_ref(a, stream) : use_fused(o) ? launch_chunk_tc(a, stream) : launch_chunk_tc2(a, stream);
     if (e == cudaSuccess && o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

@@ -1,0 +1,805 @@
+// kda_chunk_tc2.cu -- two-kernel tensor-core chunkwise KDA forward for sm_100a.
+//
+// The chunkwise form (page "Kimi K3 模型结构（2）：序列维度（下），chunkwise 并行与
+// 下界衰减", Q&A items on the chunkwise algorithm, the -5 decay floor and the
+// intra-chunk matrix A) splits into work that does not depend on the state --
+// everything up to the WY vectors -- and a short state-dependent scan.  The
+// first kernel runs the former for every (chunk, head) in parallel, so it fills
+// the GPU however few heads there are; the second walks each head's chunks in
+// order with nothing but the scan on its critical path.
+//
+// Kernel 1 (one CTA per chunk and head), with the same arithmetic as the fused
+// kernel of kda_chunk_tc.cu:
+//   gamma = band-local cumsum of log|alpha|, E = e^{gamma - p_band}, band factors
+//   A_qk / A_kk: all ten (row band, column band) pairs as one N = 160 tcgen05 product
+//   Tm = (I + A_kk)^{-1} in FP32;  W^T = (K e^gamma)^T Tm'^T,  U^T = V^T Tm'^T
+//   writes, per chunk and head, a 74,240-byte record of bf16 tiles already in the
+//   shared-memory layouts the scan's tensor-core products read:
+//     W^T (MN-major [c][r]), Q e^gamma (K-major [r][c]), K e^{gamma_C-gamma} ([r][c]),
+//     U^T ([j][r] row-major), A_qk (K-major [r][i]) and sigma_C e^{gamma_C} (FP32 [128]).
+// Kernel 2 (one CTA per head): per chunk, one bulk copy of the record (double
+// buffered), then
+//   V~^T = U^T - S^T W^T,  O^T = S^T (Q e^gamma)^T      (S^T in TMEM as bf16)
+//   O^T += V~^T A_qk^T,    dS^T = V~^T Kd
+//   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32 registers;  O -> HBM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+#include "kda_sm100.cuh"
+
+namespace kda {
+
+namespace {
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int C = 64;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// the per-(chunk, head) record written by kernel 1 and read by kernel 2
+constexpr uint32_t IMG_WT = 0;          // bf16 W^T, MN-major [128 c][64 r]
+constexpr uint32_t IMG_QG = 16384;      // bf16 Q e^gamma, K-major [64 r][128 c]
+constexpr uint32_t IMG_KD = 32768;      // bf16 K e^{gamma_C - gamma}, [64 r][128 c]
+constexpr uint32_t IMG_U = 49152;       // bf16 U^T, row-major [128 j][64 r]
+constexpr uint32_t IMG_AQK = 65536;     // bf16 A_qk, K-major [64 r][64 i]
+constexpr uint32_t IMG_GC = 73728;      // fp32 sigma_C e^{gamma_C} [128]
+constexpr uint32_t IMG_BYTES = 74240;
+
+__device__ __forceinline__ uint32_t off_r128(int r, int c) {
+    return (uint32_t)((r & 7) * 16 + (r >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 2);
+}
+__device__ __forceinline__ uint32_t off_r64(int r, int c) {
+    return (uint32_t)((r & 7) * 16 + (r >> 3) * 1024 + (c >> 3) * 128 + (c & 7) * 2);
+}
+__device__ __forceinline__ uint32_t off_sw128(int r, int c) {
+    const int hf = c >> 6, cc = c & 63;
+    return (uint32_t)(hf * 8192 + r * 128 + ((((cc >> 3) ^ (r & 7))) << 4) + (cc & 7) * 2);
+}
+__device__ __forceinline__ int pair_of(int b, int j) { return (j == 0 ? 0 : j == 1 ? 4 : j == 2 ? 7 : 9) + b - j; }
+
+__device__ __forceinline__ void unpack8(uint4 raw, float (&x)[8]) {
+    const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
+    uint4 u;
+    u.x = pack_bf16(x[0], x[1]);
+    u.y = pack_bf16(x[2], x[3]);
+    u.z = pack_bf16(x[4], x[5]);
+    u.w = pack_bf16(x[6], x[7]);
+    return u;
+}
+__device__ __forceinline__ void ld8f(const float *p, float (&x)[8]) {
+    *reinterpret_cast<float4 *>(x) = *reinterpret_cast<const float4 *>(p);
+    *reinterpret_cast<float4 *>(x + 4) = *reinterpret_cast<const float4 *>(p + 4);
+}
+
+__device__ int g_kda_tc2_error;   // set when a bounded wait gives up
+
+struct alignas(8) Bars {
+    uint64_t bar0;
+    uint64_t bar1;
+    uint64_t bar_mma;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// ============================================================== kernel 1: per-chunk prep
+namespace prep {
+constexpr int NT = 512;
+constexpr uint32_t kTmaBytes = 4u * C * D * 2u;
+constexpr uint32_t OFF_STG_Q = 0, OFF_STG_K = 16384, OFF_STG_V = 32768, OFF_STG_G = 49152;
+constexpr uint32_t OFF_GAM = 65536;            // fp32 E [64][132]; later AKK / TMF
+constexpr uint32_t E_STRIDE = 132;
+constexpr uint32_t AS = 68;
+constexpr uint32_t OFF_AKK = OFF_GAM;
+constexpr uint32_t OFF_TMF = OFF_GAM + 17408;
+constexpr uint32_t OFF_BOP = OFF_GAM + 36864;  // bf16 band-pair B operand [160][128]; later Tm' + scratch
+constexpr uint32_t OFF_TMB = OFF_BOP;          // bf16 [64 r][64 i]
+constexpr uint32_t OFF_RZ = OFF_BOP + 8192;    // fp32 inverse scratch
+constexpr uint32_t OFF_YR = OFF_BOP + 40960;   // bf16 K e^gamma [64][128]
+constexpr uint32_t OFF_TAB = OFF_YR + 16384;
+constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_GC = 14336,
+                   TAB_NRM = 14848, TAB_BET = 15360, TAB_SGNL = 15616, TAB_BPAR = 16640,
+                   TAB_PP = 16896, TAB_SGNC = 17152, TAB_BYTES = 17408;
+constexpr uint32_t SMEM_BYTES = OFF_TAB + TAB_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// TMEM: X [0,64), D [64,224), W^T [224,288), U^T [288,352)
+constexpr uint32_t TC_X = 0, TC_D = 64, TC_W = 224, TC_U = 288;
+}  // namespace prep
+
+__global__ void __launch_bounds__(prep::NT, 1)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                  const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
+                  KernelFlags fl) {
+    using namespace prep;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ Bars sh;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    float *EX = reinterpret_cast<float *>(smem + OFF_GAM);
+    float *AKK = reinterpret_cast<float *>(smem + OFF_AKK);
+    float *TMF = reinterpret_cast<float *>(smem + OFF_TMF);
+    float *RR = reinterpret_cast<float *>(smem + OFF_RZ);
+    float *ZZ = reinterpret_cast<float *>(smem + OFF_RZ + 2560);
+    float *TOT = reinterpret_cast<float *>(smem + OFF_TAB + TAB_TOT);
+    float *TF = reinterpret_cast<float *>(smem + OFF_TAB + TAB_F);
+    float *TG = reinterpret_cast<float *>(smem + OFF_TAB + TAB_G);
+    float *TH = reinterpret_cast<float *>(smem + OFF_TAB + TAB_H);
+    float *TGC = reinterpret_cast<float *>(smem + OFF_TAB + TAB_GC);
+    float *NRM = reinterpret_cast<float *>(smem + OFF_TAB + TAB_NRM);
+    float *BET = reinterpret_cast<float *>(smem + OFF_TAB + TAB_BET);
+    uint32_t *SGNL = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNL);
+    uint32_t *BPAR = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_BPAR);
+    uint32_t *PP = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_PP);
+    uint32_t *SGNC = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNC);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, qq = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int ch = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
+    const int nch = gridDim.x;
+    const int t0 = ch * C, n = min(C, T - t0);
+    uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
+    const uint32_t bar_tma = smem_u32(&sh.bar0), bar_mma = smem_u32(&sh.bar_mma);
+
+    if (tid == 0) {
+        mbar_init(bar_tma, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        sh.abort = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sh.tmem_base;
+    const uint32_t tl = tbase + ((uint32_t)(quad * 32) << 16);
+    const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
+    const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
+    const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
+    const uint64_t dV = sdesc(sbase, 8192, 1024, kSwizzle128B);
+    auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
+    auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
+        if (tid == 0 && !mbar_wait_bounded(bar, phase, kWaitLimit)) {
+            sh.abort = 1;
+            g_kda_tc2_error = 1;
+        }
+        __syncthreads();
+        return sh.abort == 0;
+    };
+
+    if (tid == 0) {
+        mbar_arrive_expect_tx(bar_tma, kTmaBytes);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(sbase + OFF_STG_Q + hf * 8192, &tm_q, bar_tma, hf * 64, h, t0, b);
+            tma_load_4d(sbase + OFF_STG_K + hf * 8192, &tm_k, bar_tma, hf * 64, h, t0, b);
+            tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_tma, hf * 64, h, t0, b);
+            tma_load_4d(sbase + OFF_STG_G + hf * 8192, &tm_g, bar_tma, hf * 64, h, t0, b);
+        }
+    }
+    if (tid < C) BET[tid] = tid < n ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
+    bool ok = wait_all(bar_tma, 0);
+
+    if (ok) {
+        // ---- band-local cumulative log-decay | row norms
+        {
+            const int c = tid & 127, p = tid >> 7;
+            float gv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                gv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                    smem + OFF_STG_G + off_sw128(16 * p + i, c)));
+            float loc = 0.f;
+            uint32_t par = 0;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * p + i;
+                float lg = 0.f;
+                if (r < n) {
+                    if (fl.complex_gate) {
+                        lg = __logf(fabsf(gv[i]));
+                        par ^= (gv[i] < 0.f) ? 1u : 0u;
+                    } else {
+                        lg = gv[i];
+                    }
+                }
+                loc += lg;
+                EX[r * E_STRIDE + c] = __expf(fmaxf(loc, -85.f));
+                if (fl.complex_gate) {
+                    const uint32_t bits = __ballot_sync(0xffffffffu, par != 0);
+                    if (lane == 0) SGNL[r * 4 + quad] = bits;
+                }
+            }
+            TOT[p * D + c] = loc;
+            const uint32_t bp = __ballot_sync(0xffffffffu, par != 0);
+            if (lane == 0) BPAR[p * 4 + quad] = bp;
+        }
+        {
+            const int rr = tid >> 2, part = tid & 3;
+            const int r = rr & 63;
+            const uint32_t tile = rr < 64 ? OFF_STG_Q : OFF_STG_K;
+            float ss = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                float x[8];
+                unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, 32 * part + 8 * m)), x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            if (part == 0) NRM[rr] = fl.l2norm ? rsqrtf(ss + kL2Eps) : 1.f;
+        }
+        __syncthreads();
+
+        // ---- per-channel band factors
+        if (tid < D) {
+            const int c = tid;
+            float et[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) et[p] = __expf(TOT[p * D + c]);
+            TH[0 * D + c] = 1.f;
+            TH[1 * D + c] = et[0];
+            TH[2 * D + c] = et[0] * et[1];
+            TH[3 * D + c] = et[0] * et[1] * et[2];
+            const float eC = et[0] * et[1] * et[2] * et[3];
+            TG[0 * D + c] = eC;
+            TG[1 * D + c] = et[1] * et[2] * et[3];
+            TG[2 * D + c] = et[2] * et[3];
+            TG[3 * D + c] = et[3];
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) TF[(bb * 4 + bb) * D + c] = 1.f;
+            TF[(1 * 4 + 0) * D + c] = et[0];
+            TF[(2 * 4 + 1) * D + c] = et[1];
+            TF[(2 * 4 + 0) * D + c] = et[0] * et[1];
+            TF[(3 * 4 + 2) * D + c] = et[2];
+            TF[(3 * 4 + 1) * D + c] = et[1] * et[2];
+            TF[(3 * 4 + 0) * D + c] = et[0] * et[1] * et[2];
+            const int w = c >> 5, bit = c & 31;
+            const uint32_t pc = BPAR[0 * 4 + w] ^ BPAR[1 * 4 + w] ^ BPAR[2 * 4 + w] ^ BPAR[3 * 4 + w];
+            const float gc = ((pc >> bit) & 1u) ? -eC : eC;
+            TGC[c] = gc;
+            reinterpret_cast<float *>(img + IMG_GC)[c] = gc;
+            if (c < 4) {
+                PP[0 * 4 + c] = 0u;
+                PP[1 * 4 + c] = BPAR[0 * 4 + c];
+                PP[2 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c];
+                PP[3 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c];
+                SGNC[c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c] ^ BPAR[3 * 4 + c];
+            }
+        }
+        __syncthreads();
+
+        // ---- operands (thread = row, 32 channels); Q e^gamma and Kd go straight to the record
+        {
+            const bool isq = row < 64;
+            const int r = row & 63;
+            const int band = r >> 4;
+            const float nrm = NRM[row];
+            const float bet = BET[r];
+            const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
+            const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
+            const uint32_t swc = SGNC[qq];
+#pragma unroll
+            for (int cg = 0; cg < 4; ++cg) {
+                const int c0 = 32 * qq + 8 * cg;
+                float x[8], E[8], hb[8];
+                unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, c0)), x);
+                ld8f(EX + r * E_STRIDE + c0, E);
+                ld8f(TH + band * D + c0, hb);
+                float xe[8], y1[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
+                    xe[e] = x[e] * E[e];
+                    y1[e] = xe[e] * hb[e];
+                }
+                const float rs = isq ? 1.f : bet;
+                tmem_st4(tl + TC_X + 16 * qq + 4 * cg, pack_bf16(rs * xe[0], rs * xe[1]),
+                         pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
+                         pack_bf16(rs * xe[6], rs * xe[7]));
+                if (isq) {
+                    *reinterpret_cast<uint4 *>(img + IMG_QG + off_r128(r, c0)) = pack8(y1);
+                } else {
+                    float gb[8], inv[8], y2[8];
+                    ld8f(TG + band * D + c0, gb);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        inv[e] = __fdividef(x[e], E[e]);
+                        y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
+                    }
+                    *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
+                    *reinterpret_cast<uint4 *>(img + IMG_KD + off_r128(r, c0)) = pack8(y2);
+                    for (int bb = band; bb < 4; ++bb) {
+                        float f[8], y3[8];
+                        ld8f(TF + (bb * 4 + band) * D + c0, f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
+                        const int brow = 16 * pair_of(bb, band) + (r & 15);
+                        *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
+                    }
+                }
+            }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- all ten band-pair products as one N = 160 product
+        if (tid == 0) {
+            fence_proxy_async();
+            tc_fence_after();
+            constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
+            mma_commit(bar_mma);
+        }
+        ok = wait_all(bar_mma, 0);
+    }
+    if (ok) {
+        tc_fence_after();
+        // ---- A_qk -> the record (bf16, lower with diagonal); A_kk -> FP32 (strictly lower)
+        {
+            const int r = row & 63, band = r >> 4;
+            const int b_lo = (quad & 1) * 2;
+            float v[16], v2[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
+            if (qq <= b_lo + 1) {
+                tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, qq), v2);
+                if (band == b_lo + 1) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                }
+            }
+            if (row < 64) {
+#pragma unroll
+                for (int g8 = 0; g8 < 2; ++g8) {
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 16 * qq + 8 * g8 + e;
+                        y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(img + IMG_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
+                }
+            } else {
+#pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    float4 y;
+                    const int i = 16 * qq + 4 * e4;
+                    y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
+                    y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
+                    y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
+                    y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- Tm = (I + A_kk)^{-1} in FP32 (16x16 diagonal blocks, then the block products)
+        if (tid < 64) {
+            const int bb = tid >> 4, jj = tid & 15;
+            float acc[16], x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
+            float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
+                acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
+            }
+            *reinterpret_cast<float4 *>(RR + (which * 16 + rr) * 20 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
+            float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float ak = k <= rr ? a[k] : 0.f;
+                const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
+                t[0] += ak * z.x; t[1] += ak * z.y; t[2] += ak * z.z; t[3] += ak * z.w;
+            }
+            *reinterpret_cast<float4 *>(TMF + (16 * bi + rr) * AS + 16 * bj + c4) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+        }
+        __syncthreads();
+        {
+            // Z = A_BL X (32x32), one output pair per thread
+            const int rr = tid >> 4, c2 = (tid & 15) * 2;
+            float a[32];
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (32 + rr) * AS + k);
+            float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float2 x = *reinterpret_cast<const float2 *>(TMF + k * AS + c2);
+                z0 += (k >= c2 ? a[k] : 0.f) * x.x;
+                z1 += (k >= c2 + 1 ? a[k] : 0.f) * x.y;
+            }
+            *reinterpret_cast<float2 *>(ZZ + rr * 36 + c2) = make_float2(z0, z1);
+        }
+        __syncthreads();
+        {
+            // lower-left block = -Y Z
+            const int rr = tid >> 4, c2 = (tid & 15) * 2;
+            float y[32];
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+                *reinterpret_cast<float4 *>(y + k) = *reinterpret_cast<const float4 *>(TMF + (32 + rr) * AS + 32 + k);
+            float t0v = 0.f, t1v = 0.f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                const float2 z = *reinterpret_cast<const float2 *>(ZZ + k * 36 + c2);
+                const float w = k <= rr ? y[k] : 0.f;
+                t0v += w * z.x;
+                t1v += w * z.y;
+            }
+            *reinterpret_cast<float2 *>(TMF + (32 + rr) * AS + c2) = make_float2(-t0v, -t1v);
+        }
+        __syncthreads();
+        {
+            const int r = tid >> 3, ig = tid & 7;
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int i = 8 * ig + e;
+                y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
+            }
+            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pack8(y);
+        }
+        __syncthreads();
+
+        // ---- W^T = KG^T Tm'^T,  U^T = V^T Tm'^T
+        if (tid == 0) {
+            fence_proxy_async();
+            tc_fence_after();
+            constexpr uint32_t id = idesc_bf16(128, 64, 1, 0, 0);
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const uint64_t bdesc = at(dK32, OFF_TMB + 256 * s);
+                mma_ss(tbase + TC_W, at(dMN64, OFF_YR + 4096 * s), bdesc, id, s > 0);
+                mma_ss(tbase + TC_U, at(dV, OFF_STG_V + 2048 * s), bdesc, id, s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ok = wait_all(bar_mma, 1);
+    }
+    if (ok) {
+        tc_fence_after();
+        // ---- W^T (MN-major [c][r]) and U^T ([j][r] row-major) -> the record
+        float w[16], u[16];
+        tmem_ld16(tl + TC_W + 16 * qq, w);
+        tmem_ld16(tl + TC_U + 16 * qq, u);
+#pragma unroll
+        for (int g8 = 0; g8 < 2; ++g8) {
+            float y[8], z[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                y[e] = w[8 * g8 + e];
+                z[e] = u[8 * g8 + e];
+            }
+            *reinterpret_cast<uint4 *>(img + IMG_WT + off_r64(row, 16 * qq + 8 * g8)) = pack8(y);
+            *reinterpret_cast<uint4 *>(img + IMG_U + row * 128 + (16 * qq + 8 * g8) * 2) = pack8(z);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================== kernel 2: the scan
+namespace scan {
+constexpr int NT = 256;                          // 8 warps: lane quarter x column half
+constexpr uint32_t STAGE = 74752;                // record, rounded up to 1 KB
+constexpr uint32_t OFF_ST0 = 0, OFF_ST1 = STAGE;
+constexpr uint32_t OFF_VT = 2 * STAGE;           // bf16 V~^T, K-major [128 j][64 r]
+constexpr uint32_t OFF_OST = OFF_VT + 16384;     // bf16 O staging [64 r][128 j]
+constexpr uint32_t SMEM_BYTES = OFF_OST + 16384 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// TMEM: S^T operand [0,64), U^T / V~^T [64,128), O^T [128,192), dS^T [256,384)
+constexpr uint32_t TC_SOP = 0, TC_U = 64, TC_O = 128, TC_S = 256;
+}  // namespace scan
+
+__global__ void __launch_bounds__(scan::NT, 1)
+chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
+                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
+                     float scale) {
+    using namespace scan;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ Bars sh;
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, hh = warp >> 2;
+    const int row = quad * 32 + lane;
+    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int nch = (T + C - 1) / C;
+    const uint8_t *recs = ws + (size_t)bh * nch * IMG_BYTES;
+    const uint32_t bars[2] = {smem_u32(&sh.bar0), smem_u32(&sh.bar1)};
+    const uint32_t bar_mma = smem_u32(&sh.bar_mma);
+
+    if (tid == 0) {
+        mbar_init(bars[0], 1);
+        mbar_init(bars[1], 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        sh.abort = 0;
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sh.tmem_base;
+    const uint32_t tl = tbase + ((uint32_t)(quad * 32) << 16);
+    const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
+    const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
+    const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
+    const uint64_t dMN32 = sdesc(sbase, 1024, 128, kSwizzleNone);
+    auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
+    auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
+        if (tid == 0 && !mbar_wait_bounded(bar, phase, kWaitLimit)) {
+            sh.abort = 1;
+            g_kda_tc2_error = 1;
+        }
+        __syncthreads();
+        return sh.abort == 0;
+    };
+    auto fetch = [&](int ch) {
+        const int s = ch & 1;
+        mbar_arrive_expect_tx(bars[s], IMG_BYTES);
+        bulk_load(sbase + (s ? OFF_ST1 : OFF_ST0), recs + (size_t)ch * IMG_BYTES, IMG_BYTES, bars[s]);
+    };
+    if (tid == 0) {
+        if (nch > 0) fetch(0);
+        if (nch > 1) fetch(1);
+    }
+
+    // FP32 state, transposed: thread (lane j, hh) owns S^T[j][64 hh .. 64 hh + 63]
+    float S[64];
+    auto store_state_operand = [&]() {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(S[32 * half + 2 * e], S[32 * half + 2 * e + 1]);
+            tmem_st16(tl + TC_SOP + 32 * hh + 16 * half, pk);
+        }
+    };
+    {
+        const int j = row;
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+            S[e] = S0 ? S0[((size_t)bh * D + 64 * hh + e) * D + j] : 0.f;
+        store_state_operand();
+        tmem_wait_st();
+    }
+
+    uint32_t ph[2] = {0u, 0u}, ph_mma = 0;
+    bool ok = true;
+    for (int ch = 0; ch < nch && ok; ++ch) {
+        const int s = ch & 1;
+        const uint32_t st = s ? OFF_ST1 : OFF_ST0;
+        const int t0 = ch * C, n = min(C, T - t0);
+        if (!(ok = wait_all(bars[s], ph[s]))) break;
+        ph[s] ^= 1;
+
+        // U^T -> TMEM (FP32), the accumulator V~^T starts from
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(smem + st + IMG_U + row * 128 + 64 * hh);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                uint32_t pk[16];
+                float x[8];
+                unpack8(src[2 * part], x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[e] = __float_as_uint(x[e]);
+                unpack8(src[2 * part + 1], x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pk[8 + e] = __float_as_uint(x[e]);
+                tmem_st16(tl + TC_U + 32 * hh + 16 * part, pk);
+            }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+
+        // V~^T = U^T - S^T W^T;  O^T = S^T Qg^T
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t id_v = idesc_bf16(128, 64, 0, 1, 1);
+            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                mma_ts(tbase + TC_U, tbase + TC_SOP + 8 * k, at(dMN32, st + IMG_WT + 2048 * k), id_v, 1);
+                mma_ts(tbase + TC_O, tbase + TC_SOP + 8 * k, at(dK64, st + IMG_QG + 256 * k), id_o, k > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // V~^T -> bf16 (K-major [j][r])
+        {
+            float v[32];
+            tmem_ld32(tl + TC_U + 32 * hh, v);
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = v[8 * g8 + e];
+                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r64(row, 32 * hh + 8 * g8)) = pack8(y);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // O^T += V~^T A_qk^T;  dS^T = V~^T Kd
+        if (tid == 0) {
+            fence_proxy_async();
+            tc_fence_after();
+            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1, 0);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t vt = at(dK32, OFF_VT + 256 * k);
+                mma_ss(tbase + TC_O, vt, at(dK32, st + IMG_AQK + 256 * k), id_o, 1);
+                mma_ss(tbase + TC_S, vt, at(dMN64, st + IMG_KD + 4096 * k), id_s, k > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        if (!(ok = wait_all(bar_mma, ph_mma))) break;
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // S <- diag(gC) S + dS (FP32) and its bf16 copy; O^T -> staging tile
+        {
+            const float *gcv = reinterpret_cast<const float *>(smem + st + IMG_GC) + 64 * hh;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float v[32];
+                tmem_ld32(tl + TC_S + 64 * hh + 32 * part, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[32 * part + e] = fmaf(gcv[32 * part + e], S[32 * part + e], v[e]);
+            }
+            store_state_operand();
+            float o[32];
+            tmem_ld32(tl + TC_O + 32 * hh, o);
+            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_OST);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ost[(32 * hh + e) * D + row] = __float2bfloat16_rn(scale * o[e]);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // the stage is free: fetch chunk ch + 2 into it; write the outputs
+        if (tid == 0 && ch + 2 < nch) {
+            fence_proxy_async();
+            fetch(ch + 2);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int q16 = tid + NT * m, r = q16 >> 4, cj = q16 & 15;
+            if (r < n) {
+                const uint4 val = *reinterpret_cast<const uint4 *>(smem + OFF_OST + r * 256 + cj * 16);
+                *reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 8 * cj) = val;
+            }
+        }
+        __syncthreads();
+    }
+
+    if (ok && S_T) {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) S_T[((size_t)bh * D + 64 * hh + e) * D + row] = S[e];
+    }
+    if (!ok) {
+        mbar_wait_bounded(bars[0], ph[0], kWaitLimit);
+        mbar_wait_bounded(bars[1], ph[1], kWaitLimit);
+        mbar_wait_bounded(bar_mma, ph_mma, kWaitLimit);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }
+    return fn;
+}
+
+bool make_map2(CUtensorMap *m, const void *ptr, int B, int T, int H) {
+    auto enc = encode_fn2();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+size_t chunk_tc2_workspace_bytes(int B, int T, int H) {
+    const size_t nch = ((size_t)T + C - 1) / C;
+    return nch * (size_t)B * (size_t)H * IMG_BYTES;
+}
+
+cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mg;
+    if (!make_map2(&mq, a.q, a.B, a.T, a.H) || !make_map2(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map2(&mv, a.v, a.B, a.T, a.H) || !make_map2(&mg, a.g, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)prep::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)scan::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int nch = (a.T + C - 1) / C;
+    uint8_t *ws = (uint8_t *)a.workspace;
+    mark_launch(a, st);
+    chunk_prep_kernel<<<dim3(nch, a.B * a.H), prep::NT, prep::SMEM_BYTES, st>>>(
+        mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.fl);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mark_launch(a, st);
+    chunk_scan_tc_kernel<<<a.B * a.H, scan::NT, scan::SMEM_BYTES, st>>>(
+        ws, a.S0, (__nv_bfloat16 *)a.out, a.S_T, a.T, a.H, a.fl.scale);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

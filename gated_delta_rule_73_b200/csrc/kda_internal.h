@@ -51,6 +51,9 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 bool chunk_tc_supported(const ChunkArgs &a);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t st);
 int chunk_tc_read_error();
+// Two-kernel tensor-core chunk path (parallel prep + per-head scan); needs a workspace.
+size_t chunk_tc2_workspace_bytes(int B, int T, int H);
+cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st);
 

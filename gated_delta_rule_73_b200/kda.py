@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
 
 KDA_BF16, KDA_F32 = 0, 1
-KDA_QK_L2NORM, KDA_COMPLEX = 1, 2
+KDA_QK_L2NORM, KDA_COMPLEX, KDA_FUSED = 1, 2, 4
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_ARG", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_ALIGN",
           -4: "KDA_ERR_UNSUPPORTED", -5: "KDA_ERR_CUDA", -6: "KDA_ERR_TIMEOUT",
           -7: "KDA_ERR_WORKSPACE"}
@@ -82,10 +82,12 @@ def _dtype_code(t: torch.dtype) -> int:
 
 
 def make_opts(dtype: torch.dtype = torch.bfloat16, *, l2norm: bool = True, complex_gate: bool = False,
-              scale: float = 1.0, workspace: torch.Tensor | None = None, events=None) -> kda_opts:
+              scale: float = 1.0, workspace: torch.Tensor | None = None, events=None,
+              fused: bool = False) -> kda_opts:
     o = kda_opts()
     o.dtype = _dtype_code(dtype)
-    o.flags = (KDA_QK_L2NORM if l2norm else 0) | (KDA_COMPLEX if complex_gate else 0)
+    o.flags = ((KDA_QK_L2NORM if l2norm else 0) | (KDA_COMPLEX if complex_gate else 0)
+               | (KDA_FUSED if fused else 0))
     o.scale = float(scale)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -186,16 +188,16 @@ def kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, ou
 
 # ------------------------------------------------------------------ conveniences
 def chunk_fwd(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False, scale=1.0,
-              workspace=None, out=None, S_T=None, stream=None):
+              fused=False, workspace=None, out=None, S_T=None, stream=None):
     """Allocate out / S_T / workspace with torch and run ``kda_chunk_fwd``."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale)
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused)
     if workspace is None:
         nbytes = kda_chunk_workspace_bytes(B, T, H, dk, dv, opts)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale,
-                     workspace=workspace)
+                     workspace=workspace, fused=fused)
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if S_T is None:
@@ -215,15 +217,15 @@ def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scal
 
 
 def chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0=None, *, scale=1.0,
-                       workspace=None, out=None, S_T=None, stream=None):
+                       fused=False, workspace=None, out=None, S_T=None, stream=None):
     """Allocate and run ``kda_chunk_fwd_prologue``."""
     B, T, H, dk = q_pre.shape
     dv = v_pre.shape[-1]
-    opts = make_opts(q_pre.dtype, scale=scale)
+    opts = make_opts(q_pre.dtype, scale=scale, fused=fused)
     if workspace is None:
         nbytes = kda_prologue_workspace_bytes(B, T, H, dk, dv, opts)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q_pre.device)
-    opts = make_opts(q_pre.dtype, scale=scale, workspace=workspace)
+    opts = make_opts(q_pre.dtype, scale=scale, workspace=workspace, fused=fused)
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q_pre.dtype, device=q_pre.device)
     if S_T is None:

@@ -66,8 +66,11 @@ typedef enum {
 enum {
     KDA_QK_L2NORM = 1u,  /* q, k <- x / sqrt(sum x^2 + 1e-6) per head, in-kernel
                             (use_qk_l2norm_in_kernel, "Kimi K3 の KDA(1)" 1.2.1) */
-    KDA_COMPLEX = 2u     /* Complex-KDA: `g` holds the signed gate alpha itself,
+    KDA_COMPLEX = 2u,    /* Complex-KDA: `g` holds the signed gate alpha itself,
                             |alpha| in [e^-5, 1], alpha != 0; beta in [0, 2]   */
+    KDA_FUSED = 4u       /* bf16 dk = dv = 128 only: run the chunk forward as one
+                            fused kernel per sequence (no workspace) instead of
+                            the default parallel-prep + scan pair             */
 };
 
 /* Options.  Passing NULL means {KDA_BF16, KDA_QK_L2NORM, 1.0f, NULL, 0, NULL, 0}. */

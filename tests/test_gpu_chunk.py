@@ -119,3 +119,19 @@ def test_empty_sequence_is_identity(K):
                     e(2, 0, 3), S0, e(2, 0, 3, 128), S_T, opts)
     torch.cuda.synchronize()
     assert torch.equal(S_T, S0)
+
+
+@pytest.mark.parametrize("T", [1, 64, 130, 333])
+@pytest.mark.parametrize("complex_gate", [False, True])
+def test_fused_single_kernel_path(K, T, complex_gate):
+    """KDA_FUSED: the one-kernel-per-sequence tensor-core path (no workspace)."""
+    x = W.chunk_inputs(2, T, 3, 128, 128, dtype=torch.bfloat16, seed=40 + T, complex_gate=complex_gate)
+    out, S_T = _run(K, x, complex_gate=complex_gate, fused=True)
+    _check(out, S_T, _oracle(x, complex_gate=complex_gate), torch.bfloat16)
+
+
+def test_prefill_workload_fused(K):
+    """prefill workload through the fused path, every output."""
+    x = W.workload_inputs("prefill")
+    out, S_T = _run(K, x, fused=True)
+    _check(out, S_T, _oracle(x), torch.bfloat16)
