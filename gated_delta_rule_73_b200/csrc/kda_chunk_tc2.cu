@@ -15,13 +15,15 @@
 //   Tm = (I + A_kk)^{-1} in FP32;  W^T = (K e^gamma)^T Tm'^T,  U^T = V^T Tm'^T
 //   writes, per chunk and head, a 74,240-byte record of bf16 tiles already in the
 //   shared-memory layouts the scan's tensor-core products read:
-//     W^T (MN-major [c][r]), Q e^gamma (K-major [r][c]), K e^{gamma_C-gamma} ([r][c]),
-//     U^T ([j][r] row-major), A_qk (K-major [r][i]) and sigma_C e^{gamma_C} (FP32 [128]).
-// Kernel 2 (one CTA per head): per chunk, one bulk copy of the record (double
-// buffered), then
-//   V~^T = U^T - S^T W^T,  O^T = S^T (Q e^gamma)^T      (S^T in TMEM as bf16)
-//   O^T += V~^T A_qk^T,    dS^T = V~^T Kd
-//   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32 registers;  O -> HBM.
+//     W and Q e^gamma (K-major [r][c], stacked into one [128][128] tile),
+//     K e^{gamma_C-gamma} ([r][c]), U^T (K-major [j][r]), A_qk (K-major [r][i]) and
+//     sigma_C e^{gamma_C} (FP32 [128]).
+// Kernel 2 (one CTA per head): per chunk, one bulk copy of the record (three-stage
+// ring), then
+//   [P | O^T] = S^T [W ; Q e^gamma]^T                    (S^T in TMEM as bf16)
+//   V~^T = U^T - P;  dS^T = V~^T Kd;  O^T += V~^T A_qk^T (V~^T in TMEM as bf16)
+//   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32 registers;  O -> HBM while the
+//   next chunk's first product runs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -39,10 +41,10 @@ constexpr int C = 64;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 // the per-(chunk, head) record written by kernel 1 and read by kernel 2
-constexpr uint32_t IMG_WT = 0;          // bf16 W^T, MN-major [128 c][64 r]
+constexpr uint32_t IMG_W = 0;           // bf16 W, K-major [64 r][128 c] (with Q e^gamma: one [128][128] tile)
 constexpr uint32_t IMG_QG = 16384;      // bf16 Q e^gamma, K-major [64 r][128 c]
 constexpr uint32_t IMG_KD = 32768;      // bf16 K e^{gamma_C - gamma}, [64 r][128 c]
-constexpr uint32_t IMG_U = 49152;       // bf16 U^T, row-major [128 j][64 r]
+constexpr uint32_t IMG_U = 49152;       // bf16 U^T, K-major [128 j][64 r]
 constexpr uint32_t IMG_AQK = 65536;     // bf16 A_qk, K-major [64 r][64 i]
 constexpr uint32_t IMG_GC = 73728;      // fp32 sigma_C e^{gamma_C} [128]
 constexpr uint32_t IMG_BYTES = 74240;
@@ -102,7 +104,7 @@ constexpr uint32_t AS = 68;
 constexpr uint32_t OFF_AKK = OFF_GAM;
 constexpr uint32_t OFF_TMF = OFF_GAM + 17408;
 constexpr uint32_t OFF_BOP = OFF_GAM + 36864;  // bf16 band-pair B operand [160][128]; later Tm' + scratch
-constexpr uint32_t OFF_TMB = OFF_BOP;          // bf16 [64 r][64 i]
+constexpr uint32_t OFF_TMB = OFF_BOP;          // bf16 [128][64 i]: Tm' rows r, then the same rows again
 constexpr uint32_t OFF_RZ = OFF_BOP + 8192;    // fp32 inverse scratch
 constexpr uint32_t OFF_YR = OFF_BOP + 40960;   // bf16 K e^gamma [64][128]
 constexpr uint32_t OFF_TAB = OFF_YR + 16384;
@@ -111,8 +113,8 @@ constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_
                    TAB_PP = 16896, TAB_SGNC = 17152, TAB_BYTES = 17408;
 constexpr uint32_t SMEM_BYTES = OFF_TAB + TAB_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM: X [0,64), D [64,224), W^T [224,288), U^T [288,352)
-constexpr uint32_t TC_X = 0, TC_D = 64, TC_W = 224, TC_U = 288;
+// TMEM: X [0,64), D [64,224), U^T [288,352), W (lanes 0-63; 64-127 repeat them) [352,480)
+constexpr uint32_t TC_X = 0, TC_D = 64, TC_U = 288, TC_W = 352;
 }  // namespace prep
 
 __global__ void __launch_bounds__(prep::NT, 1)
@@ -273,7 +275,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint32_t pc = BPAR[0 * 4 + w] ^ BPAR[1 * 4 + w] ^ BPAR[2 * 4 + w] ^ BPAR[3 * 4 + w];
             const float gc = ((pc >> bit) & 1u) ? -eC : eC;
             TGC[c] = gc;
-            reinterpret_cast<float *>(img + IMG_GC)[c] = gc;
             if (c < 4) {
                 PP[0 * 4 + c] = 0u;
                 PP[1 * 4 + c] = BPAR[0 * 4 + c];
@@ -294,6 +295,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
             const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
             const uint32_t swc = SGNC[qq];
+            uint4 rec[4];   // this row's Q e^gamma or Kd slice of the record, stored after the fence
 #pragma unroll
             for (int cg = 0; cg < 4; ++cg) {
                 const int c0 = 32 * qq + 8 * cg;
@@ -313,7 +315,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                          pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
                          pack_bf16(rs * xe[6], rs * xe[7]));
                 if (isq) {
-                    *reinterpret_cast<uint4 *>(img + IMG_QG + off_r128(r, c0)) = pack8(y1);
+                    rec[cg] = pack8(y1);
                 } else {
                     float gb[8], inv[8], y2[8];
                     ld8f(TG + band * D + c0, gb);
@@ -323,7 +325,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
                     }
                     *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
-                    *reinterpret_cast<uint4 *>(img + IMG_KD + off_r128(r, c0)) = pack8(y2);
+                    rec[cg] = pack8(y2);
                     for (int bb = band; bb < 4; ++bb) {
                         float f[8], y3[8];
                         ld8f(TF + (bb * 4 + band) * D + c0, f);
@@ -334,6 +336,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
             }
+            // Each writer orders its shared-memory operands before the tensor-core reads.  The
+            // fence waits for this thread's outstanding stores, so the record's global stores
+            // come after it.
+            fence_proxy_async();
+#pragma unroll
+            for (int cg = 0; cg < 4; ++cg)
+                *reinterpret_cast<uint4 *>(img + (isq ? IMG_QG : IMG_KD) + off_r128(r, 32 * qq + 8 * cg)) = rec[cg];
+            if (tid < D) reinterpret_cast<float *>(img + IMG_GC)[tid] = TGC[tid];
         }
         tmem_wait_st();
         tc_fence_before();
@@ -341,7 +351,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         // ---- all ten band-pair products as one N = 160 product
         if (tid == 0) {
-            fence_proxy_async();
             tc_fence_after();
             constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
 #pragma unroll
@@ -353,11 +362,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (ok) {
         tc_fence_after();
-        // ---- A_qk -> the record (bf16, lower with diagonal); A_kk -> FP32 (strictly lower)
-        {
+        // ---- A_kk -> FP32 (strictly lower); A_qk goes to the record while W/U are on the tensor cores
+        auto band_rows = [&](float (&v)[16]) {
             const int r = row & 63, band = r >> 4;
             const int b_lo = (quad & 1) * 2;
-            float v[16], v2[16];
+            float v2[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0.f;
             if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
@@ -368,28 +377,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     for (int e = 0; e < 16; ++e) v[e] = v2[e];
                 }
             }
-            if (row < 64) {
+        };
+        if (row >= 64) {
+            const int r = row & 63;
+            float v[16];
+            band_rows(v);
 #pragma unroll
-                for (int g8 = 0; g8 < 2; ++g8) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = 16 * qq + 8 * g8 + e;
-                        y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
-                    }
-                    *reinterpret_cast<uint4 *>(img + IMG_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
-                }
-            } else {
-#pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    float4 y;
-                    const int i = 16 * qq + 4 * e4;
-                    y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
-                    y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
-                    y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
-                    y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
-                }
+            for (int e4 = 0; e4 < 4; ++e4) {
+                float4 y;
+                const int i = 16 * qq + 4 * e4;
+                y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
+                y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
+                y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
+                y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
+                *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
             }
         }
         tc_fence_before();
@@ -485,41 +486,67 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int i = 8 * ig + e;
                 y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
             }
-            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pack8(y);
+            const uint4 pk = pack8(y);
+            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pk;
+            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r + 64, 8 * ig)) = pk;
+            fence_proxy_async();   // Tm' is read by the tensor cores next
         }
         __syncthreads();
 
-        // ---- W^T = KG^T Tm'^T,  U^T = V^T Tm'^T
+        // ---- W = Tm' (K e^gamma) (M = 128: Tm' stacked twice),  U^T = V^T Tm'^T
         if (tid == 0) {
-            fence_proxy_async();
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 64, 1, 0, 0);
+            constexpr uint32_t id_w = idesc_bf16(128, 128, 0, 1, 0);
+            constexpr uint32_t id_u = idesc_bf16(128, 64, 1, 0, 0);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
-                const uint64_t bdesc = at(dK32, OFF_TMB + 256 * s);
-                mma_ss(tbase + TC_W, at(dMN64, OFF_YR + 4096 * s), bdesc, id, s > 0);
-                mma_ss(tbase + TC_U, at(dV, OFF_STG_V + 2048 * s), bdesc, id, s > 0);
+                const uint64_t tdesc = at(dK32, OFF_TMB + 256 * s);
+                mma_ss(tbase + TC_W, tdesc, at(dMN64, OFF_YR + 4096 * s), id_w, s > 0);
+                mma_ss(tbase + TC_U, at(dV, OFF_STG_V + 2048 * s), tdesc, id_u, s > 0);
             }
             mma_commit(bar_mma);
+        }
+        __syncwarp();
+        if (row < 64) {
+            // A_qk (lower with diagonal) -> the record, bf16
+            const int r = row;
+            float v[16];
+            band_rows(v);
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 16 * qq + 8 * g8 + e;
+                    y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
+                }
+                *reinterpret_cast<uint4 *>(img + IMG_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
+            }
         }
         ok = wait_all(bar_mma, 1);
     }
     if (ok) {
         tc_fence_after();
-        // ---- W^T (MN-major [c][r]) and U^T ([j][r] row-major) -> the record
-        float w[16], u[16];
-        tmem_ld16(tl + TC_W + 16 * qq, w);
+        // ---- W (K-major [r][c]) and U^T (K-major [j][r]) -> the record
+        if (row < 64) {
+            float w[32];
+            tmem_ld32(tl + TC_W + 32 * qq, w);
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
+                *reinterpret_cast<uint4 *>(img + IMG_W + off_r128(row, 32 * qq + 8 * g8)) = pack8(y);
+            }
+        }
+        float u[16];
         tmem_ld16(tl + TC_U + 16 * qq, u);
 #pragma unroll
         for (int g8 = 0; g8 < 2; ++g8) {
-            float y[8], z[8];
+            float z[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                y[e] = w[8 * g8 + e];
-                z[e] = u[8 * g8 + e];
-            }
-            *reinterpret_cast<uint4 *>(img + IMG_WT + off_r64(row, 16 * qq + 8 * g8)) = pack8(y);
-            *reinterpret_cast<uint4 *>(img + IMG_U + row * 128 + (16 * qq + 8 * g8) * 2) = pack8(z);
+            for (int e = 0; e < 8; ++e) z[e] = u[8 * g8 + e];
+            *reinterpret_cast<uint4 *>(img + IMG_U + off_r64(row, 16 * qq + 8 * g8)) = pack8(z);
         }
     }
     tc_fence_before();
@@ -528,17 +555,29 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ============================================================== kernel 2: the scan
+// One CTA per (b, h), 256 threads: thread (lane j, half hh) owns the FP32 state column
+// S^T[j][64 hh .. 64 hh + 63].  Per chunk, with the record of chunk ch in stage ch % 3:
+//   [P | O] = S^T [W ; Q e^gamma]^T      one N = 128 product, into D[ch & 1]
+//   (meanwhile: the outputs of chunk ch - 1 leave D[(ch - 1) & 1]; the record of ch + 2 is fetched)
+//   V~^T = U^T - P                       -> TMEM (bf16), the A operand of the next two products
+//   dS^T = V~^T Kd;  O += V~^T A_qk^T
+//   S <- diag(sigma_C e^{gamma_C}) S + dS, and its bf16 copy for the next chunk's product.
 namespace scan {
-constexpr int NT = 256;                          // 8 warps: lane quarter x column half
+constexpr int NT = 256;
+constexpr int NSTAGE = 3;
 constexpr uint32_t STAGE = 74752;                // record, rounded up to 1 KB
-constexpr uint32_t OFF_ST0 = 0, OFF_ST1 = STAGE;
-constexpr uint32_t OFF_VT = 2 * STAGE;           // bf16 V~^T, K-major [128 j][64 r]
-constexpr uint32_t OFF_OST = OFF_VT + 16384;     // bf16 O staging [64 r][128 j]
-constexpr uint32_t SMEM_BYTES = OFF_OST + 16384 + 1024;
+constexpr uint32_t SMEM_BYTES = NSTAGE * STAGE + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM: S^T operand [0,64), U^T / V~^T [64,128), O^T [128,192), dS^T [256,384)
-constexpr uint32_t TC_SOP = 0, TC_U = 64, TC_O = 128, TC_S = 256;
+// TMEM columns: bf16 S^T [0,64), bf16 V~^T [64,96), D0 = [P | O] [128,256), D1 [256,384),
+// dS^T [384,512)
+constexpr uint32_t TC_SOP = 0, TC_VT = 64, TC_D0 = 128, TC_D1 = 256, TC_S = 384;
 }  // namespace scan
+
+struct alignas(8) ScanBars {
+    uint64_t stage[scan::NSTAGE];
+    uint64_t mV, mS, mO;
+    uint32_t tmem_base;
+};
 
 __global__ void __launch_bounds__(scan::NT, 1)
 chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
@@ -546,25 +585,24 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                      float scale) {
     using namespace scan;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ Bars sh;
+    __shared__ ScanBars sh;
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, hh = warp >> 2;
-    const int row = quad * 32 + lane;
+    const int row = quad * 32 + lane;                // TMEM lane = j
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int nch = (T + C - 1) / C;
     const uint8_t *recs = ws + (size_t)bh * nch * IMG_BYTES;
-    const uint32_t bars[2] = {smem_u32(&sh.bar0), smem_u32(&sh.bar1)};
-    const uint32_t bar_mma = smem_u32(&sh.bar_mma);
+    const uint32_t b_mV = smem_u32(&sh.mV), b_mS = smem_u32(&sh.mS), b_mO = smem_u32(&sh.mO);
 
     if (tid == 0) {
-        mbar_init(bars[0], 1);
-        mbar_init(bars[1], 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < NSTAGE; ++i) mbar_init(smem_u32(&sh.stage[i]), 1);
+        mbar_init(b_mV, 1);
+        mbar_init(b_mS, 1);
+        mbar_init(b_mO, 1);
         mbar_fence_init();
-        sh.abort = 0;
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(&sh.tmem_base), 512);
@@ -578,169 +616,143 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
     const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
-    const uint64_t dMN32 = sdesc(sbase, 1024, 128, kSwizzleNone);
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
-    auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
-        if (tid == 0 && !mbar_wait_bounded(bar, phase, kWaitLimit)) {
-            sh.abort = 1;
+    auto stage_off = [](int ch) -> uint32_t { return (uint32_t)(ch % NSTAGE) * STAGE; };
+    auto fetch = [&](int ch) {
+        const uint32_t bar = smem_u32(&sh.stage[ch % NSTAGE]);
+        mbar_arrive_expect_tx(bar, IMG_BYTES);
+        bulk_load(sbase + stage_off(ch), recs + (size_t)ch * IMG_BYTES, IMG_BYTES, bar);
+    };
+    // every thread waits on the barrier itself; a wait that gives up marks this thread, and
+    // the whole CTA leaves the loop at the next block-wide barrier (__syncthreads_or)
+    int failed = 0;
+    auto wait = [&](uint32_t bar, uint32_t phase) {
+        if (!mbar_wait_bounded(bar, phase, kWaitLimit)) {
+            failed = 1;
             g_kda_tc2_error = 1;
         }
-        __syncthreads();
-        return sh.abort == 0;
     };
-    auto fetch = [&](int ch) {
-        const int s = ch & 1;
-        mbar_arrive_expect_tx(bars[s], IMG_BYTES);
-        bulk_load(sbase + (s ? OFF_ST1 : OFF_ST0), recs + (size_t)ch * IMG_BYTES, IMG_BYTES, bars[s]);
+    // outputs of chunk c: O^T[j][r] in D[c & 1] + 64, this thread's 32 tokens r
+    auto emit = [&](int c) {
+        const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 64 + 32 * hh;
+        float o[32];
+        __syncwarp();
+        tmem_ld32(tl + dcol, o);
+        const int t0 = c * C, n = min(C, T - t0);
+        __nv_bfloat16 *dst = out + (((size_t)b * T + t0) * H + h) * D + row;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int r = 32 * hh + e;
+            if (r < n) dst[(size_t)r * H * D] = __float2bfloat16_rn(scale * o[e]);
+        }
     };
-    if (tid == 0) {
-        if (nch > 0) fetch(0);
-        if (nch > 1) fetch(1);
-    }
 
-    // FP32 state, transposed: thread (lane j, hh) owns S^T[j][64 hh .. 64 hh + 63]
-    float S[64];
+    if (tid == 0) {
+        for (int c = 0; c < NSTAGE && c < nch; ++c) fetch(c);
+    }
+    float S[64];   // S^T[j][64 hh + e]
     auto store_state_operand = [&]() {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int q2 = 0; q2 < 2; ++q2) {
             uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(S[32 * half + 2 * e], S[32 * half + 2 * e + 1]);
-            tmem_st16(tl + TC_SOP + 32 * hh + 16 * half, pk);
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(S[32 * q2 + 2 * e], S[32 * q2 + 2 * e + 1]);
+            tmem_st16(tl + TC_SOP + 32 * hh + 16 * q2, pk);
         }
     };
-    {
-        const int j = row;
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-            S[e] = S0 ? S0[((size_t)bh * D + 64 * hh + e) * D + j] : 0.f;
-        store_state_operand();
-        tmem_wait_st();
-    }
+    for (int e = 0; e < 64; ++e) S[e] = S0 ? S0[((size_t)bh * D + 64 * hh + e) * D + row] : 0.f;
+    store_state_operand();
+    tmem_wait_st();
+    tc_fence_before();
+    __syncthreads();
 
-    uint32_t ph[2] = {0u, 0u}, ph_mma = 0;
-    bool ok = true;
-    for (int ch = 0; ch < nch && ok; ++ch) {
-        const int s = ch & 1;
-        const uint32_t st = s ? OFF_ST1 : OFF_ST0;
-        const int t0 = ch * C, n = min(C, T - t0);
-        if (!(ok = wait_all(bars[s], ph[s]))) break;
-        ph[s] ^= 1;
-
-        // U^T -> TMEM (FP32), the accumulator V~^T starts from
-        {
-            const uint4 *src = reinterpret_cast<const uint4 *>(smem + st + IMG_U + row * 128 + 64 * hh);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                uint32_t pk[16];
-                float x[8];
-                unpack8(src[2 * part], x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pk[e] = __float_as_uint(x[e]);
-                unpack8(src[2 * part + 1], x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pk[8 + e] = __float_as_uint(x[e]);
-                tmem_st16(tl + TC_U + 32 * hh + 16 * part, pk);
-            }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
-
-        // V~^T = U^T - S^T W^T;  O^T = S^T Qg^T
+    for (int ch = 0; ch < nch; ++ch) {
+        const uint32_t st = stage_off(ch);
+        const uint32_t sbar = smem_u32(&sh.stage[ch % NSTAGE]);
+        const uint32_t sph = (uint32_t)(ch / NSTAGE) & 1u;
+        const uint32_t dbuf = (ch & 1) ? TC_D1 : TC_D0;
+        const uint32_t par = (uint32_t)ch & 1u;
+        // [P | O] = S^T [W ; Qg]^T: 8 products of N = 128
         if (tid == 0) {
+            wait(sbar, sph);
             tc_fence_after();
-            constexpr uint32_t id_v = idesc_bf16(128, 64, 0, 1, 1);
-            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
+            constexpr uint32_t id_pq = idesc_bf16(128, 128, 0, 0, 0);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                mma_ts(tbase + TC_U, tbase + TC_SOP + 8 * k, at(dMN32, st + IMG_WT + 2048 * k), id_v, 1);
-                mma_ts(tbase + TC_O, tbase + TC_SOP + 8 * k, at(dK64, st + IMG_QG + 256 * k), id_o, k > 0);
-            }
-            mma_commit(bar_mma);
+            for (int k = 0; k < 8; ++k)
+                mma_ts(tbase + dbuf, tbase + TC_SOP + 8 * k, at(dK64, st + IMG_W + 256 * k), id_pq, k > 0);
+            mma_commit(b_mV);
         }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
-        ph_mma ^= 1;
+        // the previous chunk's outputs leave while the product runs; its stage is refilled
+        if (ch > 0) {
+            wait(b_mO, par ^ 1u);
+            tc_fence_after();
+            if (tid == 0 && ch + 2 < nch && ch + 2 >= NSTAGE) fetch(ch + 2);
+            emit(ch - 1);
+        }
+        // V~^T = U^T - P -> bf16 in TMEM (this thread: tokens 32 hh .. 32 hh + 31)
+        wait(sbar, sph);
+        wait(b_mV, par);
         tc_fence_after();
-
-        // V~^T -> bf16 (K-major [j][r])
         {
-            float v[32];
-            tmem_ld32(tl + TC_U + 32 * hh, v);
+            float p[32];
+            __syncwarp();
+            tmem_ld32(tl + dbuf + 32 * hh, p);
+            uint32_t pk[16];
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
-                float y[8];
+                float u[8];
+                unpack8(*reinterpret_cast<const uint4 *>(smem + st + IMG_U + off_r64(row, 32 * hh + 8 * g8)), u);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = v[8 * g8 + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r64(row, 32 * hh + 8 * g8)) = pack8(y);
+                for (int e = 0; e < 4; ++e)
+                    pk[4 * g8 + e] = pack_bf16(u[2 * e] - p[8 * g8 + 2 * e], u[2 * e + 1] - p[8 * g8 + 2 * e + 1]);
             }
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // O^T += V~^T A_qk^T;  dS^T = V~^T Kd
-        if (tid == 0) {
-            fence_proxy_async();
-            tc_fence_after();
-            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
-            constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1, 0);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint64_t vt = at(dK32, OFF_VT + 256 * k);
-                mma_ss(tbase + TC_O, vt, at(dK32, st + IMG_AQK + 256 * k), id_o, 1);
-                mma_ss(tbase + TC_S, vt, at(dMN64, st + IMG_KD + 4096 * k), id_s, k > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!(ok = wait_all(bar_mma, ph_mma))) break;
-        ph_mma ^= 1;
-        tc_fence_after();
-
-        // S <- diag(gC) S + dS (FP32) and its bf16 copy; O^T -> staging tile
-        {
-            const float *gcv = reinterpret_cast<const float *>(smem + st + IMG_GC) + 64 * hh;
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                float v[32];
-                tmem_ld32(tl + TC_S + 64 * hh + 32 * part, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[32 * part + e] = fmaf(gcv[32 * part + e], S[32 * part + e], v[e]);
-            }
-            store_state_operand();
-            float o[32];
-            tmem_ld32(tl + TC_O + 32 * hh, o);
-            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_OST);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ost[(32 * hh + e) * D + row] = __float2bfloat16_rn(scale * o[e]);
+            tmem_st16(tl + TC_VT + 16 * hh, pk);
             tmem_wait_st();
         }
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // the stage is free: fetch chunk ch + 2 into it; write the outputs
-        if (tid == 0 && ch + 2 < nch) {
-            fence_proxy_async();
-            fetch(ch + 2);
-        }
+        if (__syncthreads_or(failed)) { failed = 1; break; }
+        // dS^T = V~^T Kd (the state's path), then O^T += V~^T A_qk^T
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1, 0);
+            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int q16 = tid + NT * m, r = q16 >> 4, cj = q16 & 15;
-            if (r < n) {
-                const uint4 val = *reinterpret_cast<const uint4 *>(smem + OFF_OST + r * 256 + cj * 16);
-                *reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 8 * cj) = val;
-            }
+            for (int k = 0; k < 4; ++k)
+                mma_ts(tbase + TC_S, tbase + TC_VT + 8 * k, at(dMN64, st + IMG_KD + 4096 * k), id_s, k > 0);
+            mma_commit(b_mS);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                mma_ts(tbase + dbuf + 64, tbase + TC_VT + 8 * k, at(dK32, st + IMG_AQK + 256 * k), id_o, 1);
+            mma_commit(b_mO);
         }
-        __syncthreads();
+        // S <- diag(gC) S + dS in FP32, and its bf16 copy
+        wait(b_mS, par);
+        tc_fence_after();
+        {
+            const float *gcv = reinterpret_cast<const float *>(smem + st + IMG_GC) + 64 * hh;
+            __syncwarp();
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                float v[32];
+                tmem_ld32(tl + TC_S + 64 * hh + 32 * q2, v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[32 * q2 + e] = fmaf(gcv[32 * q2 + e], S[32 * q2 + e], v[e]);
+            }
+            store_state_operand();
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        if (__syncthreads_or(failed)) { failed = 1; break; }
     }
-
-    if (ok && S_T) {
+    if (!failed && nch > 0) {
+        wait(b_mO, (uint32_t)(nch - 1) & 1u);
+        tc_fence_after();
+        if (!failed) emit(nch - 1);
+    }
+    if (!failed && S_T) {
 #pragma unroll
         for (int e = 0; e < 64; ++e) S_T[((size_t)bh * D + 64 * hh + e) * D + row] = S[e];
-    }
-    if (!ok) {
-        mbar_wait_bounded(bars[0], ph[0], kWaitLimit);
-        mbar_wait_bounded(bars[1], ph[1], kWaitLimit);
-        mbar_wait_bounded(bar_mma, ph_mma, kWaitLimit);
     }
     tc_fence_before();
     __syncthreads();
