@@ -12,20 +12,22 @@
 // kernel of kda_chunk_tc.cu:
 //   gamma = band-local cumsum of log|alpha|, E = e^{gamma - p_band}, band factors
 //   A_qk / A_kk: all ten (row band, column band) pairs as one N = 160 tcgen05 product
-//   Tm = (I + A_kk)^{-1} in FP32;  W^T = (K e^gamma)^T Tm'^T,  U^T = V^T Tm'^T
+//   Tm = (I + A_kk)^{-1} in FP32;  W = Tm' (K e^gamma),  U = Tm' V
 //   writes, per chunk and head, a 74,240-byte record of bf16 tiles already in the
 //   shared-memory layouts the scan's tensor-core products read:
 //     W and Q e^gamma (K-major [r][c], stacked into one [128][128] tile),
-//     K e^{gamma_C-gamma} ([r][c]), U^T (K-major [j][r]), A_qk (K-major [r][i]) and
+//     K e^{gamma_C-gamma} ([r][c]), U ([r][j]), A_qk (K-major [r][i]) and
 //     sigma_C e^{gamma_C} (FP32 [128]).
-// Kernel 2 (one CTA per head): per chunk, one bulk copy of the record (three-stage
-// ring), then
-//   [P | O^T] = S^T [W ; Q e^gamma]^T                    (S^T in TMEM as bf16)
-//   V~^T = U^T - P;  dS^T = V~^T Kd;  O^T += V~^T A_qk^T (V~^T in TMEM as bf16)
+// Kernel 2 (one CTA per head): per chunk, the record is bulk-copied into one of two
+// stages, then
+//   [P ; O] = [W ; Q e^gamma] S                          (S in shared memory as bf16)
+//   V~ = U - P;  dS = Kd^T V~;  O += A_qk V~             (V~ in shared memory as bf16)
 //   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32 registers;  O -> HBM while the
 //   next chunk's first product runs.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -44,7 +46,7 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr uint32_t IMG_W = 0;           // bf16 W, K-major [64 r][128 c] (with Q e^gamma: one [128][128] tile)
 constexpr uint32_t IMG_QG = 16384;      // bf16 Q e^gamma, K-major [64 r][128 c]
 constexpr uint32_t IMG_KD = 32768;      // bf16 K e^{gamma_C - gamma}, [64 r][128 c]
-constexpr uint32_t IMG_U = 49152;       // bf16 U^T, K-major [128 j][64 r]
+constexpr uint32_t IMG_U = 49152;       // bf16 U, [64 r][128 j] (same core layout as W)
 constexpr uint32_t IMG_AQK = 65536;     // bf16 A_qk, K-major [64 r][64 i]
 constexpr uint32_t IMG_GC = 73728;      // fp32 sigma_C e^{gamma_C} [128]
 constexpr uint32_t IMG_BYTES = 74240;
@@ -96,7 +98,6 @@ struct alignas(8) Bars {
 // ============================================================== kernel 1: per-chunk prep
 namespace prep {
 constexpr int NT = 512;
-constexpr uint32_t kTmaBytes = 4u * C * D * 2u;
 constexpr uint32_t OFF_STG_Q = 0, OFF_STG_K = 16384, OFF_STG_V = 32768, OFF_STG_G = 49152;
 constexpr uint32_t OFF_GAM = 65536;            // fp32 E [64][132]; later AKK / TMF
 constexpr uint32_t E_STRIDE = 132;
@@ -113,15 +114,16 @@ constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_
                    TAB_PP = 16896, TAB_SGNC = 17152, TAB_BYTES = 17408;
 constexpr uint32_t SMEM_BYTES = OFF_TAB + TAB_BYTES + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM: X [0,64), D [64,224), U^T [288,352), W (lanes 0-63; 64-127 repeat them) [352,480)
-constexpr uint32_t TC_X = 0, TC_D = 64, TC_U = 288, TC_W = 352;
+// TMEM: X [0,64), D [64,224), then W and U, each in lanes 0-63 with lanes 64-127 repeating
+// them: U [224,352), W [352,480)
+constexpr uint32_t TC_X = 0, TC_D = 64, TC_U = 224, TC_W = 352;
 }  // namespace prep
 
 __global__ void __launch_bounds__(prep::NT, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                  KernelFlags fl) {
+                  int BH, KernelFlags fl) {
     using namespace prep;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Bars sh;
@@ -148,14 +150,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, qq = warp >> 2;
     const int row = quad * 32 + lane;
-    const int ch = blockIdx.x, bh = blockIdx.y, b = bh / H, h = bh % H;
-    const int nch = gridDim.x;
-    const int t0 = ch * C, n = min(C, T - t0);
-    uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
-    const uint32_t bar_tma = smem_u32(&sh.bar0), bar_mma = smem_u32(&sh.bar_mma);
+    const int nch = (T + C - 1) / C;
+    const int nitems = nch * BH;
+    const uint32_t bar_tma = smem_u32(&sh.bar0), bar_v = smem_u32(&sh.bar1), bar_mma = smem_u32(&sh.bar_mma);
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
+        mbar_init(bar_v, 1);
         mbar_init(bar_mma, 1);
         mbar_fence_init();
         sh.abort = 0;
@@ -183,371 +184,397 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         return sh.abort == 0;
     };
 
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_tma, kTmaBytes);
+    // work item = (chunk, b * H + h), chunk fastest; each CTA walks items with a stride of the
+    // grid and fetches the next item's tiles as soon as their staging buffers are free
+    auto issue_qkg = [&](int item) {
+        const int ich = item % nch, ibh = item / nch;
+        const int ib = ibh / H, ih = ibh % H, it0 = ich * C;
+        mbar_arrive_expect_tx(bar_tma, 3u * C * D * 2u);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(sbase + OFF_STG_Q + hf * 8192, &tm_q, bar_tma, hf * 64, h, t0, b);
-            tma_load_4d(sbase + OFF_STG_K + hf * 8192, &tm_k, bar_tma, hf * 64, h, t0, b);
-            tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_tma, hf * 64, h, t0, b);
-            tma_load_4d(sbase + OFF_STG_G + hf * 8192, &tm_g, bar_tma, hf * 64, h, t0, b);
+            tma_load_4d(sbase + OFF_STG_Q + hf * 8192, &tm_q, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_K + hf * 8192, &tm_k, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_G + hf * 8192, &tm_g, bar_tma, hf * 64, ih, it0, ib);
         }
+    };
+    auto issue_v = [&](int item) {
+        const int ich = item % nch, ibh = item / nch;
+        const int ib = ibh / H, ih = ibh % H, it0 = ich * C;
+        mbar_arrive_expect_tx(bar_v, (uint32_t)C * D * 2u);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_v, hf * 64, ih, it0, ib);
+    };
+    if (tid == 0 && (int)blockIdx.x < nitems) {
+        issue_qkg(blockIdx.x);
+        issue_v(blockIdx.x);
     }
-    if (tid < C) BET[tid] = tid < n ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
-    bool ok = wait_all(bar_tma, 0);
+    bool ok = true;
+    uint32_t li = 0;   // items done by this CTA: parity of the TMA barriers
+    for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+        const int ch = item % nch, bh = item / nch, b = bh / H, h = bh % H;
+        const int t0 = ch * C, n = min(C, T - t0);
+        const int next = item + (int)gridDim.x;
+        uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
+        if (tid < C) BET[tid] = tid < n ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
+        ok = wait_all(bar_tma, li & 1u);
 
-    if (ok) {
-        // ---- band-local cumulative log-decay | row norms
-        {
-            const int c = tid & 127, p = tid >> 7;
-            float gv[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                gv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                    smem + OFF_STG_G + off_sw128(16 * p + i, c)));
-            float loc = 0.f;
-            uint32_t par = 0;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * p + i;
-                float lg = 0.f;
-                if (r < n) {
+        if (ok) {
+            // ---- band-local cumulative log-decay | row norms
+            {
+                const int c = tid & 127, p = tid >> 7;
+                float gv[16];
+    #pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    gv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                        smem + OFF_STG_G + off_sw128(16 * p + i, c)));
+                float loc = 0.f;
+                uint32_t par = 0;
+    #pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 16 * p + i;
+                    float lg = 0.f;
+                    if (r < n) {
+                        if (fl.complex_gate) {
+                            lg = __logf(fabsf(gv[i]));
+                            par ^= (gv[i] < 0.f) ? 1u : 0u;
+                        } else {
+                            lg = gv[i];
+                        }
+                    }
+                    loc += lg;
+                    EX[r * E_STRIDE + c] = __expf(fmaxf(loc, -85.f));
                     if (fl.complex_gate) {
-                        lg = __logf(fabsf(gv[i]));
-                        par ^= (gv[i] < 0.f) ? 1u : 0u;
-                    } else {
-                        lg = gv[i];
+                        const uint32_t bits = __ballot_sync(0xffffffffu, par != 0);
+                        if (lane == 0) SGNL[r * 4 + quad] = bits;
                     }
                 }
-                loc += lg;
-                EX[r * E_STRIDE + c] = __expf(fmaxf(loc, -85.f));
-                if (fl.complex_gate) {
-                    const uint32_t bits = __ballot_sync(0xffffffffu, par != 0);
-                    if (lane == 0) SGNL[r * 4 + quad] = bits;
+                TOT[p * D + c] = loc;
+                const uint32_t bp = __ballot_sync(0xffffffffu, par != 0);
+                if (lane == 0) BPAR[p * 4 + quad] = bp;
+            }
+            {
+                const int rr = tid >> 2, part = tid & 3;
+                const int r = rr & 63;
+                const uint32_t tile = rr < 64 ? OFF_STG_Q : OFF_STG_K;
+                float ss = 0.f;
+    #pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    float x[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, 32 * part + 8 * m)), x);
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+                if (part == 0) NRM[rr] = fl.l2norm ? rsqrtf(ss + kL2Eps) : 1.f;
+            }
+            __syncthreads();
+
+            // ---- per-channel band factors
+            if (tid < D) {
+                const int c = tid;
+                float et[4];
+    #pragma unroll
+                for (int p = 0; p < 4; ++p) et[p] = __expf(TOT[p * D + c]);
+                TH[0 * D + c] = 1.f;
+                TH[1 * D + c] = et[0];
+                TH[2 * D + c] = et[0] * et[1];
+                TH[3 * D + c] = et[0] * et[1] * et[2];
+                const float eC = et[0] * et[1] * et[2] * et[3];
+                TG[0 * D + c] = eC;
+                TG[1 * D + c] = et[1] * et[2] * et[3];
+                TG[2 * D + c] = et[2] * et[3];
+                TG[3 * D + c] = et[3];
+    #pragma unroll
+                for (int bb = 0; bb < 4; ++bb) TF[(bb * 4 + bb) * D + c] = 1.f;
+                TF[(1 * 4 + 0) * D + c] = et[0];
+                TF[(2 * 4 + 1) * D + c] = et[1];
+                TF[(2 * 4 + 0) * D + c] = et[0] * et[1];
+                TF[(3 * 4 + 2) * D + c] = et[2];
+                TF[(3 * 4 + 1) * D + c] = et[1] * et[2];
+                TF[(3 * 4 + 0) * D + c] = et[0] * et[1] * et[2];
+                const int w = c >> 5, bit = c & 31;
+                const uint32_t pc = BPAR[0 * 4 + w] ^ BPAR[1 * 4 + w] ^ BPAR[2 * 4 + w] ^ BPAR[3 * 4 + w];
+                const float gc = ((pc >> bit) & 1u) ? -eC : eC;
+                TGC[c] = gc;
+                if (c < 4) {
+                    PP[0 * 4 + c] = 0u;
+                    PP[1 * 4 + c] = BPAR[0 * 4 + c];
+                    PP[2 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c];
+                    PP[3 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c];
+                    SGNC[c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c] ^ BPAR[3 * 4 + c];
                 }
             }
-            TOT[p * D + c] = loc;
-            const uint32_t bp = __ballot_sync(0xffffffffu, par != 0);
-            if (lane == 0) BPAR[p * 4 + quad] = bp;
-        }
-        {
-            const int rr = tid >> 2, part = tid & 3;
-            const int r = rr & 63;
-            const uint32_t tile = rr < 64 ? OFF_STG_Q : OFF_STG_K;
-            float ss = 0.f;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                float x[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, 32 * part + 8 * m)), x);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
-            }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-            if (part == 0) NRM[rr] = fl.l2norm ? rsqrtf(ss + kL2Eps) : 1.f;
-        }
-        __syncthreads();
+            __syncthreads();
 
-        // ---- per-channel band factors
-        if (tid < D) {
-            const int c = tid;
-            float et[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) et[p] = __expf(TOT[p * D + c]);
-            TH[0 * D + c] = 1.f;
-            TH[1 * D + c] = et[0];
-            TH[2 * D + c] = et[0] * et[1];
-            TH[3 * D + c] = et[0] * et[1] * et[2];
-            const float eC = et[0] * et[1] * et[2] * et[3];
-            TG[0 * D + c] = eC;
-            TG[1 * D + c] = et[1] * et[2] * et[3];
-            TG[2 * D + c] = et[2] * et[3];
-            TG[3 * D + c] = et[3];
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) TF[(bb * 4 + bb) * D + c] = 1.f;
-            TF[(1 * 4 + 0) * D + c] = et[0];
-            TF[(2 * 4 + 1) * D + c] = et[1];
-            TF[(2 * 4 + 0) * D + c] = et[0] * et[1];
-            TF[(3 * 4 + 2) * D + c] = et[2];
-            TF[(3 * 4 + 1) * D + c] = et[1] * et[2];
-            TF[(3 * 4 + 0) * D + c] = et[0] * et[1] * et[2];
-            const int w = c >> 5, bit = c & 31;
-            const uint32_t pc = BPAR[0 * 4 + w] ^ BPAR[1 * 4 + w] ^ BPAR[2 * 4 + w] ^ BPAR[3 * 4 + w];
-            const float gc = ((pc >> bit) & 1u) ? -eC : eC;
-            TGC[c] = gc;
-            if (c < 4) {
-                PP[0 * 4 + c] = 0u;
-                PP[1 * 4 + c] = BPAR[0 * 4 + c];
-                PP[2 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c];
-                PP[3 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c];
-                SGNC[c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c] ^ BPAR[3 * 4 + c];
-            }
-        }
-        __syncthreads();
-
-        // ---- operands (thread = row, 32 channels); Q e^gamma and Kd go straight to the record
-        {
-            const bool isq = row < 64;
-            const int r = row & 63;
-            const int band = r >> 4;
-            const float nrm = NRM[row];
-            const float bet = BET[r];
-            const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
-            const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
-            const uint32_t swc = SGNC[qq];
-            uint4 rec[4];   // this row's Q e^gamma or Kd slice of the record, stored after the fence
-#pragma unroll
-            for (int cg = 0; cg < 4; ++cg) {
-                const int c0 = 32 * qq + 8 * cg;
-                float x[8], E[8], hb[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, c0)), x);
-                ld8f(EX + r * E_STRIDE + c0, E);
-                ld8f(TH + band * D + c0, hb);
-                float xe[8], y1[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
-                    xe[e] = x[e] * E[e];
-                    y1[e] = xe[e] * hb[e];
-                }
-                const float rs = isq ? 1.f : bet;
-                tmem_st4(tl + TC_X + 16 * qq + 4 * cg, pack_bf16(rs * xe[0], rs * xe[1]),
-                         pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
-                         pack_bf16(rs * xe[6], rs * xe[7]));
-                if (isq) {
-                    rec[cg] = pack8(y1);
-                } else {
-                    float gb[8], inv[8], y2[8];
-                    ld8f(TG + band * D + c0, gb);
-#pragma unroll
+            // ---- operands (thread = row, 32 channels); Q e^gamma and Kd go straight to the record
+            {
+                const bool isq = row < 64;
+                const int r = row & 63;
+                const int band = r >> 4;
+                const float nrm = NRM[row];
+                const float bet = BET[r];
+                const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
+                const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
+                const uint32_t swc = SGNC[qq];
+                uint4 rec[4];   // this row's Q e^gamma or Kd slice of the record, stored after the fence
+    #pragma unroll
+                for (int cg = 0; cg < 4; ++cg) {
+                    const int c0 = 32 * qq + 8 * cg;
+                    float x[8], E[8], hb[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, c0)), x);
+                    ld8f(EX + r * E_STRIDE + c0, E);
+                    ld8f(TH + band * D + c0, hb);
+                    float xe[8], y1[8];
+    #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        inv[e] = __fdividef(x[e], E[e]);
-                        y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
+                        x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
+                        xe[e] = x[e] * E[e];
+                        y1[e] = xe[e] * hb[e];
                     }
-                    *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
-                    rec[cg] = pack8(y2);
-                    for (int bb = band; bb < 4; ++bb) {
-                        float f[8], y3[8];
-                        ld8f(TF + (bb * 4 + band) * D + c0, f);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
-                        const int brow = 16 * pair_of(bb, band) + (r & 15);
-                        *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
+                    const float rs = isq ? 1.f : bet;
+                    tmem_st4(tl + TC_X + 16 * qq + 4 * cg, pack_bf16(rs * xe[0], rs * xe[1]),
+                             pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
+                             pack_bf16(rs * xe[6], rs * xe[7]));
+                    if (isq) {
+                        rec[cg] = pack8(y1);
+                    } else {
+                        float gb[8], inv[8], y2[8];
+                        ld8f(TG + band * D + c0, gb);
+    #pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            inv[e] = __fdividef(x[e], E[e]);
+                            y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
+                        }
+                        *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
+                        rec[cg] = pack8(y2);
+                        for (int bb = band; bb < 4; ++bb) {
+                            float f[8], y3[8];
+                            ld8f(TF + (bb * 4 + band) * D + c0, f);
+    #pragma unroll
+                            for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
+                            const int brow = 16 * pair_of(bb, band) + (r & 15);
+                            *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
+                        }
                     }
                 }
+                // Each writer orders its shared-memory operands before the tensor-core reads.  The
+                // fence waits for this thread's outstanding stores, so the record's global stores
+                // come after it.
+                fence_proxy_async();
+    #pragma unroll
+                for (int cg = 0; cg < 4; ++cg)
+                    *reinterpret_cast<uint4 *>(img + (isq ? IMG_QG : IMG_KD) + off_r128(r, 32 * qq + 8 * cg)) = rec[cg];
+                if (tid < D) reinterpret_cast<float *>(img + IMG_GC)[tid] = TGC[tid];
             }
-            // Each writer orders its shared-memory operands before the tensor-core reads.  The
-            // fence waits for this thread's outstanding stores, so the record's global stores
-            // come after it.
-            fence_proxy_async();
-#pragma unroll
-            for (int cg = 0; cg < 4; ++cg)
-                *reinterpret_cast<uint4 *>(img + (isq ? IMG_QG : IMG_KD) + off_r128(r, 32 * qq + 8 * cg)) = rec[cg];
-            if (tid < D) reinterpret_cast<float *>(img + IMG_GC)[tid] = TGC[tid];
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
+            tmem_wait_st();
+            tc_fence_before();
+            __syncthreads();
 
-        // ---- all ten band-pair products as one N = 160 product
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
-            mma_commit(bar_mma);
+            // ---- all ten band-pair products as one N = 160 product
+            if (tid == 0) {
+                if (next < nitems) issue_qkg(next);   // q, k, g staging is free from here on
+                tc_fence_after();
+                constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
+    #pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
+                mma_commit(bar_mma);
+            }
+            ok = wait_all(bar_mma, 0);
         }
-        ok = wait_all(bar_mma, 0);
-    }
-    if (ok) {
-        tc_fence_after();
-        // ---- A_kk -> FP32 (strictly lower); A_qk goes to the record while W/U are on the tensor cores
-        auto band_rows = [&](float (&v)[16]) {
-            const int r = row & 63, band = r >> 4;
-            const int b_lo = (quad & 1) * 2;
-            float v2[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
-            if (qq <= b_lo + 1) {
-                tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, qq), v2);
-                if (band == b_lo + 1) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = v2[e];
+        if (ok) {
+            tc_fence_after();
+            // ---- A_kk -> FP32 (strictly lower); A_qk goes to the record while W/U are on the tensor cores
+            auto band_rows = [&](float (&v)[16]) {
+                const int r = row & 63, band = r >> 4;
+                const int b_lo = (quad & 1) * 2;
+                float v2[16];
+    #pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
+                if (qq <= b_lo + 1) {
+                    tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, qq), v2);
+                    if (band == b_lo + 1) {
+    #pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                    }
+                }
+            };
+            if (row >= 64) {
+                const int r = row & 63;
+                float v[16];
+                band_rows(v);
+    #pragma unroll
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    float4 y;
+                    const int i = 16 * qq + 4 * e4;
+                    y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
+                    y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
+                    y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
+                    y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
                 }
             }
-        };
-        if (row >= 64) {
-            const int r = row & 63;
-            float v[16];
-            band_rows(v);
-#pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) {
-                float4 y;
-                const int i = 16 * qq + 4 * e4;
-                y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
-                y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
-                y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
-                y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
-                *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
+            tc_fence_before();
+            __syncthreads();
 
-        // ---- Tm = (I + A_kk)^{-1} in FP32 (16x16 diagonal blocks, then the block products)
-        if (tid < 64) {
-            const int bb = tid >> 4, jj = tid & 15;
-            float acc[16], x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
-#pragma unroll
-                for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
+            // ---- Tm = (I + A_kk)^{-1} in FP32 (16x16 diagonal blocks, then the block products)
+            if (tid < 64) {
+                const int bb = tid >> 4, jj = tid & 15;
+                float acc[16], x[16];
+    #pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    #pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
+    #pragma unroll
+                    for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
+                }
+    #pragma unroll
+                for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
             }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
-            float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k = 0; k < 16; k += 4)
-                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
-                acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
+            __syncthreads();
+            if (tid < 128) {
+                const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+                const int bi = which ? 3 : 1, bj = which ? 2 : 0;
+                float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                for (int k = 0; k < 16; k += 4)
+                    *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
+    #pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
+                    acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
+                }
+                *reinterpret_cast<float4 *>(RR + (which * 16 + rr) * 20 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
             }
-            *reinterpret_cast<float4 *>(RR + (which * 16 + rr) * 20 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
-            float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k = 0; k < 16; k += 4)
-                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float ak = k <= rr ? a[k] : 0.f;
-                const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
-                t[0] += ak * z.x; t[1] += ak * z.y; t[2] += ak * z.z; t[3] += ak * z.w;
+            __syncthreads();
+            if (tid < 128) {
+                const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
+                const int bi = which ? 3 : 1, bj = which ? 2 : 0;
+                float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                for (int k = 0; k < 16; k += 4)
+                    *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
+    #pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float ak = k <= rr ? a[k] : 0.f;
+                    const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
+                    t[0] += ak * z.x; t[1] += ak * z.y; t[2] += ak * z.z; t[3] += ak * z.w;
+                }
+                *reinterpret_cast<float4 *>(TMF + (16 * bi + rr) * AS + 16 * bj + c4) = make_float4(-t[0], -t[1], -t[2], -t[3]);
             }
-            *reinterpret_cast<float4 *>(TMF + (16 * bi + rr) * AS + 16 * bj + c4) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-        }
-        __syncthreads();
-        {
-            // Z = A_BL X (32x32), one output pair per thread
-            const int rr = tid >> 4, c2 = (tid & 15) * 2;
-            float a[32];
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (32 + rr) * AS + k);
-            float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const float2 x = *reinterpret_cast<const float2 *>(TMF + k * AS + c2);
-                z0 += (k >= c2 ? a[k] : 0.f) * x.x;
-                z1 += (k >= c2 + 1 ? a[k] : 0.f) * x.y;
+            __syncthreads();
+            {
+                // Z = A_BL X (32x32), one output pair per thread
+                const int rr = tid >> 4, c2 = (tid & 15) * 2;
+                float a[32];
+    #pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (32 + rr) * AS + k);
+                float z0 = 0.f, z1 = 0.f;
+    #pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const float2 x = *reinterpret_cast<const float2 *>(TMF + k * AS + c2);
+                    z0 += (k >= c2 ? a[k] : 0.f) * x.x;
+                    z1 += (k >= c2 + 1 ? a[k] : 0.f) * x.y;
+                }
+                *reinterpret_cast<float2 *>(ZZ + rr * 36 + c2) = make_float2(z0, z1);
             }
-            *reinterpret_cast<float2 *>(ZZ + rr * 36 + c2) = make_float2(z0, z1);
-        }
-        __syncthreads();
-        {
-            // lower-left block = -Y Z
-            const int rr = tid >> 4, c2 = (tid & 15) * 2;
-            float y[32];
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<float4 *>(y + k) = *reinterpret_cast<const float4 *>(TMF + (32 + rr) * AS + 32 + k);
-            float t0v = 0.f, t1v = 0.f;
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const float2 z = *reinterpret_cast<const float2 *>(ZZ + k * 36 + c2);
-                const float w = k <= rr ? y[k] : 0.f;
-                t0v += w * z.x;
-                t1v += w * z.y;
+            __syncthreads();
+            {
+                // lower-left block = -Y Z
+                const int rr = tid >> 4, c2 = (tid & 15) * 2;
+                float y[32];
+    #pragma unroll
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<float4 *>(y + k) = *reinterpret_cast<const float4 *>(TMF + (32 + rr) * AS + 32 + k);
+                float t0v = 0.f, t1v = 0.f;
+    #pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const float2 z = *reinterpret_cast<const float2 *>(ZZ + k * 36 + c2);
+                    const float w = k <= rr ? y[k] : 0.f;
+                    t0v += w * z.x;
+                    t1v += w * z.y;
+                }
+                *reinterpret_cast<float2 *>(TMF + (32 + rr) * AS + c2) = make_float2(-t0v, -t1v);
             }
-            *reinterpret_cast<float2 *>(TMF + (32 + rr) * AS + c2) = make_float2(-t0v, -t1v);
-        }
-        __syncthreads();
-        {
-            const int r = tid >> 3, ig = tid & 7;
-            float y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int i = 8 * ig + e;
-                y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
-            }
-            const uint4 pk = pack8(y);
-            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pk;
-            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r + 64, 8 * ig)) = pk;
-            fence_proxy_async();   // Tm' is read by the tensor cores next
-        }
-        __syncthreads();
-
-        // ---- W = Tm' (K e^gamma) (M = 128: Tm' stacked twice),  U^T = V^T Tm'^T
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id_w = idesc_bf16(128, 128, 0, 1, 0);
-            constexpr uint32_t id_u = idesc_bf16(128, 64, 1, 0, 0);
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint64_t tdesc = at(dK32, OFF_TMB + 256 * s);
-                mma_ss(tbase + TC_W, tdesc, at(dMN64, OFF_YR + 4096 * s), id_w, s > 0);
-                mma_ss(tbase + TC_U, at(dV, OFF_STG_V + 2048 * s), tdesc, id_u, s > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        __syncwarp();
-        if (row < 64) {
-            // A_qk (lower with diagonal) -> the record, bf16
-            const int r = row;
-            float v[16];
-            band_rows(v);
-#pragma unroll
-            for (int g8 = 0; g8 < 2; ++g8) {
+            __syncthreads();
+            {
+                const int r = tid >> 3, ig = tid & 7;
                 float y[8];
-#pragma unroll
+    #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int i = 16 * qq + 8 * g8 + e;
-                    y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
+                    const int i = 8 * ig + e;
+                    y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
                 }
-                *reinterpret_cast<uint4 *>(img + IMG_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
+                const uint4 pk = pack8(y);
+                *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pk;
+                *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r + 64, 8 * ig)) = pk;
+                fence_proxy_async();   // Tm' is read by the tensor cores next
+            }
+            __syncthreads();
+
+            // ---- W = Tm' (K e^gamma),  U = Tm' V  (M = 128: Tm' stacked twice)
+            if (tid == 0) {
+                if (!mbar_wait_bounded(bar_v, li & 1u, kWaitLimit)) {
+                    sh.abort = 1;
+                    g_kda_tc2_error = 1;
+                }
+                tc_fence_after();
+                constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
+    #pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint64_t tdesc = at(dK32, OFF_TMB + 256 * s);
+                    mma_ss(tbase + TC_W, tdesc, at(dMN64, OFF_YR + 4096 * s), id, s > 0);
+                    mma_ss(tbase + TC_U, tdesc, at(dV, OFF_STG_V + 2048 * s), id, s > 0);
+                }
+                mma_commit(bar_mma);
+            }
+            __syncwarp();
+            if (row < 64) {
+                // A_qk (lower with diagonal) -> the record, bf16
+                const int r = row;
+                float v[16];
+                band_rows(v);
+    #pragma unroll
+                for (int g8 = 0; g8 < 2; ++g8) {
+                    float y[8];
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int i = 16 * qq + 8 * g8 + e;
+                        y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(img + IMG_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
+                }
+            }
+            ok = wait_all(bar_mma, 1);
+            if (ok && tid == 0 && next < nitems) issue_v(next);   // the v staging is free again
+        }
+        if (ok) {
+            tc_fence_after();
+            // ---- W and U ([r][c] and [r][j], K-major core layout) -> the record; lanes 0-63
+            // write W, lanes 64-127 (the repeated rows) write U
+            {
+                const int r = row & 63;
+                float w[32];
+                tmem_ld32(tl + (row < 64 ? TC_W : TC_U) + 32 * qq, w);
+                uint8_t *dst = img + (row < 64 ? IMG_W : IMG_U);
+    #pragma unroll
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    float y[8];
+    #pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
+                    *reinterpret_cast<uint4 *>(dst + off_r128(r, 32 * qq + 8 * g8)) = pack8(y);
+                }
             }
         }
-        ok = wait_all(bar_mma, 1);
-    }
-    if (ok) {
+        // the next item rewrites TMEM and shared memory: everyone is done with this one
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
-        // ---- W (K-major [r][c]) and U^T (K-major [j][r]) -> the record
-        if (row < 64) {
-            float w[32];
-            tmem_ld32(tl + TC_W + 32 * qq, w);
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                float y[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
-                *reinterpret_cast<uint4 *>(img + IMG_W + off_r128(row, 32 * qq + 8 * g8)) = pack8(y);
-            }
-        }
-        float u[16];
-        tmem_ld16(tl + TC_U + 16 * qq, u);
-#pragma unroll
-        for (int g8 = 0; g8 < 2; ++g8) {
-            float z[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) z[e] = u[8 * g8 + e];
-            *reinterpret_cast<uint4 *>(img + IMG_U + off_r64(row, 16 * qq + 8 * g8)) = pack8(z);
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -555,26 +582,34 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ============================================================== kernel 2: the scan
-// One CTA per (b, h), 256 threads: thread (lane j, half hh) owns the FP32 state column
-// S^T[j][64 hh .. 64 hh + 63].  Per chunk, with the record of chunk ch in stage ch % 3:
-//   [P | O] = S^T [W ; Q e^gamma]^T      one N = 128 product, into D[ch & 1]
-//   (meanwhile: the outputs of chunk ch - 1 leave D[(ch - 1) & 1]; the record of ch + 2 is fetched)
-//   V~^T = U^T - P                       -> TMEM (bf16), the A operand of the next two products
-//   dS^T = V~^T Kd;  O += V~^T A_qk^T
-//   S <- diag(sigma_C e^{gamma_C}) S + dS, and its bf16 copy for the next chunk's product.
+// One CTA per (b, h), 256 threads.  TMEM lane = key channel c for the state and = token
+// row for the chunk products; thread (lane, hh) owns the FP32 state row S[c][64 hh .. 64 hh + 63].
+// Per chunk ch (record in stage ch & 1):
+//   [P ; O] = [W ; Q e^gamma] S          one M = 128, N = 128 product into D[ch & 1]
+//   lanes 0-63:   V~ = U - P -> bf16 shared memory
+//   lanes 64-127: the outputs of chunk ch - 1 leave D[(ch - 1) & 1] (16-byte stores)
+//   dS = Kd^T V~;  O += A_qk V~          (A_qk padded with 64 zero rows to M = 128)
+//   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32, and its bf16 copy for the next product.
 namespace scan {
 constexpr int NT = 256;
-constexpr int NSTAGE = 3;
-constexpr uint32_t STAGE = 74752;                // record, rounded up to 1 KB
-constexpr uint32_t SMEM_BYTES = NSTAGE * STAGE + 1024;
+// stage: the record's first 65,536 bytes, 8 KB of zeros, then A_qk and sigma_C e^{gamma_C}
+constexpr uint32_t ST_HEAD = IMG_AQK;                       // [W;Qg], Kd, U
+constexpr uint32_t ST_ZERO = IMG_AQK;
+constexpr uint32_t ST_AQK = IMG_AQK + 8192;
+constexpr uint32_t ST_GC = ST_AQK + (IMG_GC - IMG_AQK);
+constexpr uint32_t ST_TAIL_BYTES = IMG_BYTES - IMG_AQK;     // A_qk and sigma_C e^{gamma_C}
+constexpr uint32_t STAGE = 82944;                           // 81 KB
+static_assert(ST_GC + 512 <= STAGE, "stage layout");
+constexpr uint32_t OFF_S = 2 * STAGE;                       // bf16 S [128 c][128 j]
+constexpr uint32_t OFF_VT = OFF_S + 32768;                  // bf16 V~ [64 r][128 j]
+constexpr uint32_t SMEM_BYTES = OFF_VT + 16384 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM columns: bf16 S^T [0,64), bf16 V~^T [64,96), D0 = [P | O] [128,256), D1 [256,384),
-// dS^T [384,512)
-constexpr uint32_t TC_SOP = 0, TC_VT = 64, TC_D0 = 128, TC_D1 = 256, TC_S = 384;
+// TMEM columns: D0 = [P ; O] [0,128), D1 [128,256), dS [256,384)
+constexpr uint32_t TC_D0 = 0, TC_D1 = 128, TC_S = 256;
 }  // namespace scan
 
 struct alignas(8) ScanBars {
-    uint64_t stage[scan::NSTAGE];
+    uint64_t stage[2];
     uint64_t mV, mS, mO;
     uint32_t tmem_base;
 };
@@ -591,23 +626,29 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, hh = warp >> 2;
-    const int row = quad * 32 + lane;                // TMEM lane = j
+    const int row = quad * 32 + lane;                // TMEM lane
+    const bool p_lane = row < 64;                    // warp-uniform: rows of P (else of O)
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
     const int nch = (T + C - 1) / C;
     const uint8_t *recs = ws + (size_t)bh * nch * IMG_BYTES;
     const uint32_t b_mV = smem_u32(&sh.mV), b_mS = smem_u32(&sh.mS), b_mO = smem_u32(&sh.mO);
 
     if (tid == 0) {
-        for (int i = 0; i < NSTAGE; ++i) mbar_init(smem_u32(&sh.stage[i]), 1);
+        mbar_init(smem_u32(&sh.stage[0]), 1);
+        mbar_init(smem_u32(&sh.stage[1]), 1);
         mbar_init(b_mV, 1);
         mbar_init(b_mS, 1);
         mbar_init(b_mO, 1);
         mbar_fence_init();
     }
+    // the zero rows under each stage's A_qk
+    for (int i = tid; i < 2 * 512; i += NT)
+        *reinterpret_cast<uint4 *>(smem + (i >> 9) * STAGE + ST_ZERO + (i & 511) * 16) = make_uint4(0, 0, 0, 0);
     if (warp == 0) {
         tmem_alloc(smem_u32(&sh.tmem_base), 512);
         tmem_relinquish();
     }
+    fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -617,11 +658,13 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
-    auto stage_off = [](int ch) -> uint32_t { return (uint32_t)(ch % NSTAGE) * STAGE; };
     auto fetch = [&](int ch) {
-        const uint32_t bar = smem_u32(&sh.stage[ch % NSTAGE]);
+        const int s = ch & 1;
+        const uint32_t bar = smem_u32(&sh.stage[s]);
+        const uint8_t *src = recs + (size_t)ch * IMG_BYTES;
         mbar_arrive_expect_tx(bar, IMG_BYTES);
-        bulk_load(sbase + stage_off(ch), recs + (size_t)ch * IMG_BYTES, IMG_BYTES, bar);
+        bulk_load(sbase + s * STAGE, src, ST_HEAD, bar);
+        bulk_load(sbase + s * STAGE + ST_AQK, src + IMG_AQK, ST_TAIL_BYTES, bar);
     };
     // every thread waits on the barrier itself; a wait that gives up marks this thread, and
     // the whole CTA leaves the loop at the next block-wide barrier (__syncthreads_or)
@@ -632,127 +675,140 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             g_kda_tc2_error = 1;
         }
     };
-    // outputs of chunk c: O^T[j][r] in D[c & 1] + 64, this thread's 32 tokens r
+    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, 64 values
     auto emit = [&](int c) {
-        const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 64 + 32 * hh;
-        float o[32];
+        const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 64 * hh;
+        const int r = row - 64, t0 = c * C;
+        float o[64];
         __syncwarp();
-        tmem_ld32(tl + dcol, o);
-        const int t0 = c * C, n = min(C, T - t0);
-        __nv_bfloat16 *dst = out + (((size_t)b * T + t0) * H + h) * D + row;
+        tmem_ld32(tl + dcol, *reinterpret_cast<float(*)[32]>(o));
+        tmem_ld32(tl + dcol + 32, *reinterpret_cast<float(*)[32]>(o + 32));
+        if (t0 + r < T) {
+            uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 64 * hh);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const int r = 32 * hh + e;
-            if (r < n) dst[(size_t)r * H * D] = __float2bfloat16_rn(scale * o[e]);
+            for (int m = 0; m < 8; ++m) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = scale * o[8 * m + e];
+                dst[m] = pack8(y);
+            }
         }
+    };
+    // FP32 state row S[c = row][64 hh + e] and its bf16 copy (B operand, [c][j] core layout)
+    float S[64];
+    auto store_state_operand = [&]() {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = S[8 * m + e];
+            *reinterpret_cast<uint4 *>(smem + OFF_S + off_r128(row, 64 * hh + 8 * m)) = pack8(y);
+        }
+        fence_proxy_async();
     };
 
     if (tid == 0) {
-        for (int c = 0; c < NSTAGE && c < nch; ++c) fetch(c);
+        if (nch > 0) fetch(0);
+        if (nch > 1) fetch(1);
     }
-    float S[64];   // S^T[j][64 hh + e]
-    auto store_state_operand = [&]() {
+    if (S0) {
+        const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + 64 * hh);
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-            uint32_t pk[16];
+        for (int m = 0; m < 16; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
+    } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(S[32 * q2 + 2 * e], S[32 * q2 + 2 * e + 1]);
-            tmem_st16(tl + TC_SOP + 32 * hh + 16 * q2, pk);
-        }
-    };
-#pragma unroll
-    for (int e = 0; e < 64; ++e) S[e] = S0 ? S0[((size_t)bh * D + 64 * hh + e) * D + row] : 0.f;
+        for (int e = 0; e < 64; ++e) S[e] = 0.f;
+    }
     store_state_operand();
-    tmem_wait_st();
-    tc_fence_before();
     __syncthreads();
 
     for (int ch = 0; ch < nch; ++ch) {
-        const uint32_t st = stage_off(ch);
-        const uint32_t sbar = smem_u32(&sh.stage[ch % NSTAGE]);
-        const uint32_t sph = (uint32_t)(ch / NSTAGE) & 1u;
-        const uint32_t dbuf = (ch & 1) ? TC_D1 : TC_D0;
+        const int s = ch & 1;
+        const uint32_t st = s * STAGE;
+        const uint32_t sbar = smem_u32(&sh.stage[s]);
+        const uint32_t sph = (uint32_t)(ch >> 1) & 1u;
+        const uint32_t dbuf = s ? TC_D1 : TC_D0;
         const uint32_t par = (uint32_t)ch & 1u;
-        // [P | O] = S^T [W ; Qg]^T: 8 products of N = 128
+        // [P ; O] = [W ; Qg] S
         if (tid == 0) {
             wait(sbar, sph);
             tc_fence_after();
-            constexpr uint32_t id_pq = idesc_bf16(128, 128, 0, 0, 0);
+            constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                mma_ts(tbase + dbuf, tbase + TC_SOP + 8 * k, at(dK64, st + IMG_W + 256 * k), id_pq, k > 0);
+                mma_ss(tbase + dbuf, at(dK64, st + 256 * k), at(dMN64, OFF_S + 4096 * k), id, k > 0);
             mma_commit(b_mV);
         }
-        // the previous chunk's outputs leave while the product runs; its stage is refilled
-        if (ch > 0) {
+        if (p_lane) {
+            // the stage of chunk ch - 1 is free once its last products are done: refill it
+            if (tid == 0 && ch >= 1 && ch + 1 < nch) {
+                wait(b_mO, par ^ 1u);
+                fetch(ch + 1);
+            }
+            // V~ = U - P (this thread: token row, columns 64 hh .. 64 hh + 63)
+            wait(sbar, sph);
+            wait(b_mV, par);
+            tc_fence_after();
+            float p[64];
+            __syncwarp();
+            tmem_ld32(tl + dbuf + 64 * hh, *reinterpret_cast<float(*)[32]>(p));
+            tmem_ld32(tl + dbuf + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(p + 32));
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                float u[8], y[8];
+                unpack8(*reinterpret_cast<const uint4 *>(smem + st + IMG_U + off_r128(row, 64 * hh + 8 * m)), u);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = u[e] - p[8 * m + e];
+                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r128(row, 64 * hh + 8 * m)) = pack8(y);
+            }
+            fence_proxy_async();
+        } else if (ch > 0) {
             wait(b_mO, par ^ 1u);
             tc_fence_after();
-            if (tid == 0 && ch + 2 < nch && ch + 2 >= NSTAGE) fetch(ch + 2);
             emit(ch - 1);
-        }
-        // V~^T = U^T - P -> bf16 in TMEM (this thread: tokens 32 hh .. 32 hh + 31)
-        wait(sbar, sph);
-        wait(b_mV, par);
-        tc_fence_after();
-        {
-            float p[32];
-            __syncwarp();
-            tmem_ld32(tl + dbuf + 32 * hh, p);
-            uint32_t pk[16];
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                float u[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + st + IMG_U + off_r64(row, 32 * hh + 8 * g8)), u);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    pk[4 * g8 + e] = pack_bf16(u[2 * e] - p[8 * g8 + 2 * e], u[2 * e + 1] - p[8 * g8 + 2 * e + 1]);
-            }
-            tmem_st16(tl + TC_VT + 16 * hh, pk);
-            tmem_wait_st();
         }
         tc_fence_before();
         if (__syncthreads_or(failed)) { failed = 1; break; }
-        // dS^T = V~^T Kd (the state's path), then O^T += V~^T A_qk^T
+        // dS = Kd^T V~ (the state's path), then O += [0 ; A_qk] V~
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id_s = idesc_bf16(128, 128, 0, 1, 0);
-            constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
+            constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1, 0);
+            constexpr uint32_t id_o = idesc_bf16(128, 128, 0, 1, 0);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                mma_ts(tbase + TC_S, tbase + TC_VT + 8 * k, at(dMN64, st + IMG_KD + 4096 * k), id_s, k > 0);
+                mma_ss(tbase + TC_S, at(dMN64, st + IMG_KD + 4096 * k), at(dMN64, OFF_VT + 4096 * k), id_s, k > 0);
             mma_commit(b_mS);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                mma_ts(tbase + dbuf + 64, tbase + TC_VT + 8 * k, at(dK32, st + IMG_AQK + 256 * k), id_o, 1);
+                mma_ss(tbase + dbuf, at(dK32, st + ST_ZERO + 256 * k), at(dMN64, OFF_VT + 4096 * k), id_o, 1);
             mma_commit(b_mO);
         }
-        // S <- diag(gC) S + dS in FP32, and its bf16 copy
+        // S <- diag(gC) S + dS (FP32) and its bf16 copy
+        wait(sbar, sph);
         wait(b_mS, par);
         tc_fence_after();
         {
-            const float *gcv = reinterpret_cast<const float *>(smem + st + IMG_GC) + 64 * hh;
+            const float gc = reinterpret_cast<const float *>(smem + st + ST_GC)[row];
+            float v[64];
             __syncwarp();
+            tmem_ld32(tl + TC_S + 64 * hh, *reinterpret_cast<float(*)[32]>(v));
+            tmem_ld32(tl + TC_S + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(v + 32));
 #pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float v[32];
-                tmem_ld32(tl + TC_S + 64 * hh + 32 * q2, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[32 * q2 + e] = fmaf(gcv[32 * q2 + e], S[32 * q2 + e], v[e]);
-            }
+            for (int e = 0; e < 64; ++e) S[e] = fmaf(gc, S[e], v[e]);
             store_state_operand();
-            tmem_wait_st();
         }
         tc_fence_before();
         if (__syncthreads_or(failed)) { failed = 1; break; }
     }
-    if (!failed && nch > 0) {
+    if (!failed && nch > 0 && !p_lane) {
         wait(b_mO, (uint32_t)(nch - 1) & 1u);
         tc_fence_after();
         if (!failed) emit(nch - 1);
     }
     if (!failed && S_T) {
+        float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + 64 * hh);
 #pragma unroll
-        for (int e = 0; e < 64; ++e) S_T[((size_t)bh * D + 64 * hh + e) * D + row] = S[e];
+        for (int m = 0; m < 16; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
     }
     tc_fence_before();
     __syncthreads();
@@ -785,6 +841,14 @@ bool make_map2(CUtensorMap *m, const void *ptr, int B, int T, int H) {
 }
 }  // namespace
 
+static int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    return n;
+}
+
 size_t chunk_tc2_workspace_bytes(int B, int T, int H) {
     const size_t nch = ((size_t)T + C - 1) / C;
     return nch * (size_t)B * (size_t)H * IMG_BYTES;
@@ -804,8 +868,9 @@ cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
     const int nch = (a.T + C - 1) / C;
     uint8_t *ws = (uint8_t *)a.workspace;
     mark_launch(a, st);
-    chunk_prep_kernel<<<dim3(nch, a.B * a.H), prep::NT, prep::SMEM_BYTES, st>>>(
-        mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.fl);
+    const int nitems = nch * a.B * a.H;
+    chunk_prep_kernel<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
+        mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark_launch(a, st);

@@ -13,7 +13,8 @@
 //
 // Outputs are bf16 when the tensor-core chunk kernel follows (its operands are
 // bf16 anyway) and FP32 for the FP32 chunk path; the L2 norm of q and k is
-// applied by the chunk kernel.
+// applied by the chunk kernel.  The bf16 -> bf16 case has a vectorised kernel
+// (8 channels x a run of tokens per thread); the others use the one-element kernel.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -55,6 +56,106 @@ prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
     g[idx] = from_f32<TO>(-5.f * sigm(expf(A[h]) * to_f32(z[idx])));
     if (d == 0) beta[bth] = from_f32<TO>(sigm(b_logit[bth]));
 }
+
+// bf16 in, bf16 out (the tensor-core path): thread = 8 consecutive channels of one head
+// over a run of RUN tokens.  The three previous input rows of each branch stay in
+// registers as the window slides, so every input row is read once per run (plus a
+// three-row halo); loads and stores are 16 bytes.
+constexpr int RUN = 16;
+
+__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&x)[8]) {
+    const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h2[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void st8(__nv_bfloat16 *p, const float (&x)[8]) {
+    uint4 raw;
+    __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h2[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = raw;
+}
+
+__global__ void __launch_bounds__(256)
+prologue_bf16_kernel(const __nv_bfloat16 *__restrict__ q_pre, const __nv_bfloat16 *__restrict__ k_pre,
+                     const __nv_bfloat16 *__restrict__ v_pre, const __nv_bfloat16 *__restrict__ conv_w,
+                     const __nv_bfloat16 *__restrict__ z, const float *__restrict__ A,
+                     const float *__restrict__ b_logit, int T_, int H, int D, int nruns,
+                     long long total, __nv_bfloat16 *__restrict__ qc, __nv_bfloat16 *__restrict__ kc,
+                     __nv_bfloat16 *__restrict__ vc, __nv_bfloat16 *__restrict__ g,
+                     __nv_bfloat16 *__restrict__ beta) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const int HD = H * D, ngroups = HD / 8;
+    const int cgrp = (int)(idx % ngroups);
+    const long long rest = idx / ngroups;
+    const int run = (int)(rest % nruns), b = (int)(rest / nruns);
+    const int ch0 = cgrp * 8, h = ch0 / D;
+    const int t0 = run * RUN, t1 = min(T_, t0 + RUN);
+    const long long rowstride = HD;
+    const long long base = ((long long)b * T_) * HD + ch0;
+    // one branch at a time keeps only its taps and window live
+#pragma unroll 1
+    for (int s = 0; s < 3; ++s) {
+        const __nv_bfloat16 *src = s == 0 ? q_pre : s == 1 ? k_pre : v_pre;
+        __nv_bfloat16 *dst = s == 0 ? qc : s == 1 ? kc : vc;
+        float w[4][8];   // [tap][channel]
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float x8[8];   // channels 2m, 2m+1, taps 0-3 each
+            ld8(conv_w + ((long long)s * HD + ch0) * 4 + 8 * m, x8);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                w[j][2 * m] = x8[j];
+                w[j][2 * m + 1] = x8[4 + j];
+            }
+        }
+        float win[3][8];   // x_{t-3}, x_{t-2}, x_{t-1}
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            const int tt = t0 - 3 + j;
+            if (tt >= 0) {
+                ld8(src + base + tt * rowstride, win[j]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) win[j][c] = 0.f;
+            }
+        }
+        for (int t = t0; t < t1; ++t) {
+            const long long off = base + t * rowstride;
+            float x[8], y[8];
+            ld8(src + off, x);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float acc = w[0][c] * win[0][c] + w[1][c] * win[1][c] + w[2][c] * win[2][c] +
+                                  w[3][c] * x[c];
+                y[c] = acc * sigm(acc);
+                win[0][c] = win[1][c];
+                win[1][c] = win[2][c];
+                win[2][c] = x[c];
+            }
+            st8(dst + off, y);
+        }
+    }
+    const float ea = expf(A[h]);
+    for (int t = t0; t < t1; ++t) {
+        const long long off = base + t * rowstride;
+        float zz[8], gg[8];
+        ld8(z + off, zz);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) gg[c] = -5.f * sigm(ea * zz[c]);
+        st8(g + off, gg);
+        if (ch0 % D == 0) {
+            const long long bth = ((long long)b * T_ + t) * H + h;
+            beta[bth] = __float2bfloat16_rn(sigm(b_logit[bth]));
+        }
+    }
+}
 }  // namespace
 
 template <typename T, typename TO>
@@ -66,6 +167,16 @@ static void launch_t(const PrologueArgs &a, long long total, unsigned blocks, cu
 }
 
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st) {
+    if (a.bf16 && a.out_bf16 && a.dk % 8 == 0) {
+        const int nruns = (a.T + RUN - 1) / RUN;
+        const long long total = (long long)a.B * nruns * (a.H * a.dk / 8);
+        prologue_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(
+            (const __nv_bfloat16 *)a.q_pre, (const __nv_bfloat16 *)a.k_pre, (const __nv_bfloat16 *)a.v_pre,
+            (const __nv_bfloat16 *)a.conv_w, (const __nv_bfloat16 *)a.z, a.A, a.beta_logit, a.T, a.H,
+            a.dk, nruns, total, (__nv_bfloat16 *)a.qc, (__nv_bfloat16 *)a.kc, (__nv_bfloat16 *)a.vc,
+            (__nv_bfloat16 *)a.g, (__nv_bfloat16 *)a.beta);
+        return cudaGetLastError();
+    }
     const long long total = (long long)a.B * a.T * a.H * a.dk;
     const unsigned blocks = (unsigned)((total + 255) / 256);
     if (a.bf16 && a.out_bf16) launch_t<__nv_bfloat16, __nv_bfloat16>(a, total, blocks, st);
