@@ -224,13 +224,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             {
                 const int c = tid & 127, p = tid >> 7;
                 float gv[16];
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 16; ++i)
                     gv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
                         smem + OFF_STG_G + off_sw128(16 * p + i, c)));
                 float loc = 0.f;
                 uint32_t par = 0;
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int r = 16 * p + i;
                     float lg = 0.f;
@@ -258,11 +258,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int r = rr & 63;
                 const uint32_t tile = rr < 64 ? OFF_STG_Q : OFF_STG_K;
                 float ss = 0.f;
-    #pragma unroll
+#pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     float x[8];
                     unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, 32 * part + 8 * m)), x);
-    #pragma unroll
+#pragma unroll
                     for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
                 }
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
@@ -275,7 +275,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (tid < D) {
                 const int c = tid;
                 float et[4];
-    #pragma unroll
+#pragma unroll
                 for (int p = 0; p < 4; ++p) et[p] = __expf(TOT[p * D + c]);
                 TH[0 * D + c] = 1.f;
                 TH[1 * D + c] = et[0];
@@ -286,7 +286,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 TG[1 * D + c] = et[1] * et[2] * et[3];
                 TG[2 * D + c] = et[2] * et[3];
                 TG[3 * D + c] = et[3];
-    #pragma unroll
+#pragma unroll
                 for (int bb = 0; bb < 4; ++bb) TF[(bb * 4 + bb) * D + c] = 1.f;
                 TF[(1 * 4 + 0) * D + c] = et[0];
                 TF[(2 * 4 + 1) * D + c] = et[1];
@@ -319,7 +319,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
                 const uint32_t swc = SGNC[qq];
                 uint4 rec[4];   // this row's Q e^gamma or Kd slice of the record, stored after the fence
-    #pragma unroll
+#pragma unroll
                 for (int cg = 0; cg < 4; ++cg) {
                     const int c0 = 32 * qq + 8 * cg;
                     float x[8], E[8], hb[8];
@@ -327,7 +327,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     ld8f(EX + r * E_STRIDE + c0, E);
                     ld8f(TH + band * D + c0, hb);
                     float xe[8], y1[8];
-    #pragma unroll
+#pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
                         xe[e] = x[e] * E[e];
@@ -342,19 +342,38 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     } else {
                         float gb[8], inv[8], y2[8];
                         ld8f(TG + band * D + c0, gb);
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             inv[e] = __fdividef(x[e], E[e]);
                             y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
                         }
                         *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
                         rec[cg] = pack8(y2);
-                        for (int bb = band; bb < 4; ++bb) {
+                    }
+                }
+                // The band-pair B rows k_i e^{p_b - gamma_i} (one copy per row band b >= band(i)),
+                // spread evenly: warp = 8-channel group, lane = key row i in bands 0-1 plus the
+                // mirrored row 63 - i in bands 3-2, five copies per lane.
+                {
+                    const int c0 = 8 * warp;
+                    const int w32 = c0 >> 5, sh8 = c0 & 31;
+#pragma unroll
+                    for (int side = 0; side < 2; ++side) {
+                        const int i = side ? 63 - lane : lane;
+                        const int bi = i >> 4;
+                        const float nk = NRM[64 + i];
+                        const uint32_t swi = fl.complex_gate ? (SGNL[i * 4 + w32] ^ PP[bi * 4 + w32]) >> sh8 : 0u;
+                        float x[8], E[8], inv[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_STG_K + off_sw128(i, c0)), x);
+                        ld8f(EX + i * E_STRIDE + c0, E);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) inv[e] = __fdividef(((swi >> e) & 1u) ? -nk * x[e] : nk * x[e], E[e]);
+                        for (int bb = bi; bb < 4; ++bb) {
                             float f[8], y3[8];
-                            ld8f(TF + (bb * 4 + band) * D + c0, f);
-    #pragma unroll
+                            ld8f(TF + (bb * 4 + bi) * D + c0, f);
+#pragma unroll
                             for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
-                            const int brow = 16 * pair_of(bb, band) + (r & 15);
+                            const int brow = 16 * pair_of(bb, bi) + (i & 15);
                             *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
                         }
                     }
@@ -363,7 +382,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // fence waits for this thread's outstanding stores, so the record's global stores
                 // come after it.
                 fence_proxy_async();
-    #pragma unroll
+#pragma unroll
                 for (int cg = 0; cg < 4; ++cg)
                     *reinterpret_cast<uint4 *>(img + (isq ? IMG_QG : IMG_KD) + off_r128(r, 32 * qq + 8 * cg)) = rec[cg];
                 if (tid < D) reinterpret_cast<float *>(img + IMG_GC)[tid] = TGC[tid];
@@ -377,7 +396,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (next < nitems) issue_qkg(next);   // q, k, g staging is free from here on
                 tc_fence_after();
                 constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
-    #pragma unroll
+#pragma unroll
                 for (int s = 0; s < 8; ++s)
                     mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
                 mma_commit(bar_mma);
@@ -391,13 +410,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int r = row & 63, band = r >> 4;
                 const int b_lo = (quad & 1) * 2;
                 float v2[16];
-    #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 16; ++e) v[e] = 0.f;
                 if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
                 if (qq <= b_lo + 1) {
                     tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, qq), v2);
                     if (band == b_lo + 1) {
-    #pragma unroll
+#pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = v2[e];
                     }
                 }
@@ -406,7 +425,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int r = row & 63;
                 float v[16];
                 band_rows(v);
-    #pragma unroll
+#pragma unroll
                 for (int e4 = 0; e4 < 4; ++e4) {
                     float4 y;
                     const int i = 16 * qq + 4 * e4;
@@ -424,15 +443,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (tid < 64) {
                 const int bb = tid >> 4, jj = tid & 15;
                 float acc[16], x[16];
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
-    #pragma unroll
+#pragma unroll
                     for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
                 }
-    #pragma unroll
+#pragma unroll
                 for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
             }
             __syncthreads();
@@ -440,10 +459,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
                 const int bi = which ? 3 : 1, bj = which ? 2 : 0;
                 float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 16; k += 4)
                     *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
                     acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
@@ -455,10 +474,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
                 const int bi = which ? 3 : 1, bj = which ? 2 : 0;
                 float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 16; k += 4)
                     *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const float ak = k <= rr ? a[k] : 0.f;
                     const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
@@ -471,11 +490,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // Z = A_BL X (32x32), one output pair per thread
                 const int rr = tid >> 4, c2 = (tid & 15) * 2;
                 float a[32];
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 32; k += 4)
                     *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (32 + rr) * AS + k);
                 float z0 = 0.f, z1 = 0.f;
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     const float2 x = *reinterpret_cast<const float2 *>(TMF + k * AS + c2);
                     z0 += (k >= c2 ? a[k] : 0.f) * x.x;
@@ -488,11 +507,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // lower-left block = -Y Z
                 const int rr = tid >> 4, c2 = (tid & 15) * 2;
                 float y[32];
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 32; k += 4)
                     *reinterpret_cast<float4 *>(y + k) = *reinterpret_cast<const float4 *>(TMF + (32 + rr) * AS + 32 + k);
                 float t0v = 0.f, t1v = 0.f;
-    #pragma unroll
+#pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     const float2 z = *reinterpret_cast<const float2 *>(ZZ + k * 36 + c2);
                     const float w = k <= rr ? y[k] : 0.f;
@@ -505,7 +524,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             {
                 const int r = tid >> 3, ig = tid & 7;
                 float y[8];
-    #pragma unroll
+#pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int i = 8 * ig + e;
                     y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
@@ -525,7 +544,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
                 tc_fence_after();
                 constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
-    #pragma unroll
+#pragma unroll
                 for (int s = 0; s < 4; ++s) {
                     const uint64_t tdesc = at(dK32, OFF_TMB + 256 * s);
                     mma_ss(tbase + TC_W, tdesc, at(dMN64, OFF_YR + 4096 * s), id, s > 0);
@@ -539,10 +558,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int r = row;
                 float v[16];
                 band_rows(v);
-    #pragma unroll
+#pragma unroll
                 for (int g8 = 0; g8 < 2; ++g8) {
                     float y[8];
-    #pragma unroll
+#pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int i = 16 * qq + 8 * g8 + e;
                         y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
@@ -562,10 +581,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float w[32];
                 tmem_ld32(tl + (row < 64 ? TC_W : TC_U) + 32 * qq, w);
                 uint8_t *dst = img + (row < 64 ? IMG_W : IMG_U);
-    #pragma unroll
+#pragma unroll
                 for (int g8 = 0; g8 < 4; ++g8) {
                     float y[8];
-    #pragma unroll
+#pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
                     *reinterpret_cast<uint4 *>(dst + off_r128(r, 32 * qq + 8 * g8)) = pack8(y);
                 }
@@ -582,8 +601,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ============================================================== kernel 2: the scan
-// One CTA per (b, h), 256 threads.  TMEM lane = key channel c for the state and = token
-// row for the chunk products; thread (lane, hh) owns the FP32 state row S[c][64 hh .. 64 hh + 63].
+// One CTA per (b, h), 512 threads.  TMEM lane = key channel c for the state and = token
+// row for the chunk products; thread (lane, cq) owns the FP32 state row slice
+// S[c][32 cq .. 32 cq + 31].
 // Per chunk ch (record in stage ch & 1):
 //   [P ; O] = [W ; Q e^gamma] S          one M = 128, N = 128 product into D[ch & 1]
 //   lanes 0-63:   V~ = U - P -> bf16 shared memory
@@ -591,7 +611,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 //   dS = Kd^T V~;  O += A_qk V~          (A_qk padded with 64 zero rows to M = 128)
 //   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32, and its bf16 copy for the next product.
 namespace scan {
-constexpr int NT = 256;
+constexpr int NT = 512;
 // stage: the record's first 65,536 bytes, 8 KB of zeros, then A_qk and sigma_C e^{gamma_C}
 constexpr uint32_t ST_HEAD = IMG_AQK;                       // [W;Qg], Kd, U
 constexpr uint32_t ST_ZERO = IMG_AQK;
@@ -625,7 +645,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, hh = warp >> 2;
+    const int quad = warp & 3, cq = warp >> 2;   // lane quadrant, 32-column quarter
     const int row = quad * 32 + lane;                // TMEM lane
     const bool p_lane = row < 64;                    // warp-uniform: rows of P (else of O)
     const int bh = blockIdx.x, b = bh / H, h = bh % H;
@@ -675,18 +695,17 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             g_kda_tc2_error = 1;
         }
     };
-    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, 64 values
+    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, 32 values
     auto emit = [&](int c) {
-        const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 64 * hh;
+        const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 32 * cq;
         const int r = row - 64, t0 = c * C;
-        float o[64];
+        float o[32];
         __syncwarp();
-        tmem_ld32(tl + dcol, *reinterpret_cast<float(*)[32]>(o));
-        tmem_ld32(tl + dcol + 32, *reinterpret_cast<float(*)[32]>(o + 32));
+        tmem_ld32(tl + dcol, o);
         if (t0 + r < T) {
-            uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 64 * hh);
+            uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 32 * cq);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
+            for (int m = 0; m < 4; ++m) {
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = scale * o[8 * m + e];
@@ -694,15 +713,15 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             }
         }
     };
-    // FP32 state row S[c = row][64 hh + e] and its bf16 copy (B operand, [c][j] core layout)
-    float S[64];
+    // FP32 state row S[c = row][32 cq + e] and its bf16 copy (B operand, [c][j] core layout)
+    float S[32];
     auto store_state_operand = [&]() {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
+        for (int m = 0; m < 4; ++m) {
             float y[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] = S[8 * m + e];
-            *reinterpret_cast<uint4 *>(smem + OFF_S + off_r128(row, 64 * hh + 8 * m)) = pack8(y);
+            *reinterpret_cast<uint4 *>(smem + OFF_S + off_r128(row, 32 * cq + 8 * m)) = pack8(y);
         }
         fence_proxy_async();
     };
@@ -712,12 +731,12 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         if (nch > 1) fetch(1);
     }
     if (S0) {
-        const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + 64 * hh);
+        const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + 32 * cq);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
+        for (int m = 0; m < 8; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
     } else {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) S[e] = 0.f;
+        for (int e = 0; e < 32; ++e) S[e] = 0.f;
     }
     store_state_operand();
     __syncthreads();
@@ -745,21 +764,20 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                 wait(b_mO, par ^ 1u);
                 fetch(ch + 1);
             }
-            // V~ = U - P (this thread: token row, columns 64 hh .. 64 hh + 63)
+            // V~ = U - P (this thread: token row, columns 32 cq .. 32 cq + 31)
             wait(sbar, sph);
             wait(b_mV, par);
             tc_fence_after();
-            float p[64];
+            float p[32];
             __syncwarp();
-            tmem_ld32(tl + dbuf + 64 * hh, *reinterpret_cast<float(*)[32]>(p));
-            tmem_ld32(tl + dbuf + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(p + 32));
+            tmem_ld32(tl + dbuf + 32 * cq, p);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
+            for (int m = 0; m < 4; ++m) {
                 float u[8], y[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + st + IMG_U + off_r128(row, 64 * hh + 8 * m)), u);
+                unpack8(*reinterpret_cast<const uint4 *>(smem + st + IMG_U + off_r128(row, 32 * cq + 8 * m)), u);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = u[e] - p[8 * m + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r128(row, 64 * hh + 8 * m)) = pack8(y);
+                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r128(row, 32 * cq + 8 * m)) = pack8(y);
             }
             fence_proxy_async();
         } else if (ch > 0) {
@@ -789,12 +807,11 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         tc_fence_after();
         {
             const float gc = reinterpret_cast<const float *>(smem + st + ST_GC)[row];
-            float v[64];
+            float v[32];
             __syncwarp();
-            tmem_ld32(tl + TC_S + 64 * hh, *reinterpret_cast<float(*)[32]>(v));
-            tmem_ld32(tl + TC_S + 64 * hh + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tmem_ld32(tl + TC_S + 32 * cq, v);
 #pragma unroll
-            for (int e = 0; e < 64; ++e) S[e] = fmaf(gc, S[e], v[e]);
+            for (int e = 0; e < 32; ++e) S[e] = fmaf(gc, S[e], v[e]);
             store_state_operand();
         }
         tc_fence_before();
@@ -806,9 +823,9 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         if (!failed) emit(nch - 1);
     }
     if (!failed && S_T) {
-        float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + 64 * hh);
+        float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + 32 * cq);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
+        for (int m = 0; m < 8; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
     }
     tc_fence_before();
     __syncthreads();
