@@ -31,7 +31,8 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int check_opts(const kda_opts &o) {
     if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
-    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED)) return KDA_ERR_ARG;
+    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT)) return KDA_ERR_ARG;
+    if ((o.flags & KDA_FUSED) && (o.flags & KDA_SPLIT)) return KDA_ERR_ARG;
     if (!isfinite(o.scale)) return KDA_ERR_ARG;
     if (o.n_events < 0 || (o.n_events > 0 && !o.events)) return KDA_ERR_ARG;
     return KDA_OK;
@@ -59,13 +60,31 @@ KernelFlags kflags(const kda_opts &o) {
     return f;
 }
 
-// the bf16 dk = dv = 128 chunk forward runs on tensor cores: by default a parallel
-// per-chunk prep kernel and a per-head scan (workspace: one record per chunk and
-// head); with KDA_FUSED one fused kernel per sequence (no workspace)
+// The bf16 dk = dv = 128 chunk forward runs on tensor cores, in one of two forms:
+//  * split: a parallel per-chunk prep kernel and a per-sequence scan (workspace: one
+//    record per chunk and head).  Cost ~ B*H*nch*t_prep / SMs + waves * nch * t_scan.
+//  * fused: one kernel per sequence, prep and scan step serially in one CTA (no
+//    workspace).  Cost ~ waves * nch * t_fused, waves = ceil(B*H / SMs).
+// Measured on B200 at d = 128 (per chunk and head): t_fused = 14.0 us, t_prep = 14.8 us,
+// t_scan = 2.8 us; the model uses their ratios.  KDA_FUSED / KDA_SPLIT override it.
 bool use_tc(const kda_opts &o, int dk, int dv) { return o.dtype == KDA_BF16 && dk == 128 && dv == 128; }
-bool use_fused(const kda_opts &o) { return (o.flags & KDA_FUSED) != 0; }
+int device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        return 148;
+    return n;
+}
+bool use_fused(const kda_opts &o, int B, int H) {
+    if (o.flags & KDA_FUSED) return true;
+    if (o.flags & KDA_SPLIT) return false;
+    const double x = (double)B * H / device_sms();
+    const double waves = ceil(x);
+    const double t_fused = 1.0, t_prep = 14.8 / 14.0, t_scan = 2.8 / 14.0;
+    return waves * t_fused < x * t_prep + waves * t_scan;
+}
 size_t tc_ws(const kda_opts &o, int B, int T, int H) {
-    if (use_fused(o) || B <= 0 || T <= 0 || H <= 0) return 0;
+    if (B <= 0 || T <= 0 || H <= 0 || use_fused(o, B, H)) return 0;
     return round_up(chunk_tc2_workspace_bytes(B, T, H), kAlignWs);
 }
 
@@ -113,7 +132,7 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 100; }
+int kda_abi_version(void) { return 101; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -173,7 +192,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, co
     a.fl = kflags(o);
     a.workspace = o.workspace; a.workspace_bytes = o.workspace_bytes;
     a.events = o.events; a.n_events = o.n_events;
-    return run_chunk(a, use_fused(o), stream);
+    return run_chunk(a, use_fused(o, B, H), stream);
 }
 
 int kda_recurrent_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -255,7 +274,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     a.workspace_bytes = need - off[5];
     a.events = o.events; a.n_events = o.n_events;
     a.launch_idx = &launches;
-    e = !tc ? launch_chunk_ref(a, stream) : use_fused(o) ? launch_chunk_tc(a, stream) : launch_chunk_tc2(a, stream);
+    e = !tc ? launch_chunk_ref(a, stream) : use_fused(o, B, H) ? launch_chunk_tc(a, stream) : launch_chunk_tc2(a, stream);
     if (e == cudaSuccess && o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

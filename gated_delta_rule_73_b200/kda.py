@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
 
 KDA_BF16, KDA_F32 = 0, 1
-KDA_QK_L2NORM, KDA_COMPLEX, KDA_FUSED = 1, 2, 4
+KDA_QK_L2NORM, KDA_COMPLEX, KDA_FUSED, KDA_SPLIT = 1, 2, 4, 8
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_ARG", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_ALIGN",
           -4: "KDA_ERR_UNSUPPORTED", -5: "KDA_ERR_CUDA", -6: "KDA_ERR_TIMEOUT",
           -7: "KDA_ERR_WORKSPACE"}
@@ -83,11 +83,11 @@ def _dtype_code(t: torch.dtype) -> int:
 
 def make_opts(dtype: torch.dtype = torch.bfloat16, *, l2norm: bool = True, complex_gate: bool = False,
               scale: float = 1.0, workspace: torch.Tensor | None = None, events=None,
-              fused: bool = False) -> kda_opts:
+              fused: bool | None = None) -> kda_opts:
     o = kda_opts()
     o.dtype = _dtype_code(dtype)
     o.flags = ((KDA_QK_L2NORM if l2norm else 0) | (KDA_COMPLEX if complex_gate else 0)
-               | (KDA_FUSED if fused else 0))
+               | (0 if fused is None else KDA_FUSED if fused else KDA_SPLIT))
     o.scale = float(scale)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -188,7 +188,7 @@ def kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, ou
 
 # ------------------------------------------------------------------ conveniences
 def chunk_fwd(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False, scale=1.0,
-              fused=False, workspace=None, out=None, S_T=None, stream=None):
+              fused=None, workspace=None, out=None, S_T=None, stream=None):
     """Allocate out / S_T / workspace with torch and run ``kda_chunk_fwd``."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -217,7 +217,7 @@ def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scal
 
 
 def chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0=None, *, scale=1.0,
-                       fused=False, workspace=None, out=None, S_T=None, stream=None):
+                       fused=None, workspace=None, out=None, S_T=None, stream=None):
     """Allocate and run ``kda_chunk_fwd_prologue``."""
     B, T, H, dk = q_pre.shape
     dv = v_pre.shape[-1]

@@ -68,15 +68,20 @@ enum {
                             (use_qk_l2norm_in_kernel, "Kimi K3 の KDA(1)" 1.2.1) */
     KDA_COMPLEX = 2u,    /* Complex-KDA: `g` holds the signed gate alpha itself,
                             |alpha| in [e^-5, 1], alpha != 0; beta in [0, 2]   */
-    KDA_FUSED = 4u       /* bf16 dk = dv = 128 only: run the chunk forward as one
-                            fused kernel per sequence (no workspace) instead of
-                            the default parallel-prep + scan pair             */
+    KDA_FUSED = 4u,      /* bf16 dk = dv = 128 only: run the chunk forward as one
+                            fused kernel per sequence (no workspace)          */
+    KDA_SPLIT = 8u       /* bf16 dk = dv = 128 only: run it as the parallel
+                            per-chunk prep kernel + per-sequence scan pair
+                            (workspace: one record per chunk and head).
+                            With neither flag the library picks the one its
+                            cost model, from B*H and the device's SM count,
+                            says is faster; KDA_FUSED | KDA_SPLIT is an error */
 };
 
 /* Options.  Passing NULL means {KDA_BF16, KDA_QK_L2NORM, 1.0f, NULL, 0, NULL, 0}. */
 typedef struct {
     kda_dtype dtype;        /* type of q, k, v, g, beta, out                  */
-    unsigned flags;         /* KDA_QK_L2NORM | KDA_COMPLEX                     */
+    unsigned flags;         /* KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT */
     float scale;            /* read-out scale; the pages use 1                 */
     void *workspace;        /* device scratch, >= kda_*_workspace_bytes()     */
     size_t workspace_bytes;

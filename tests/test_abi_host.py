@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 100
+    assert kda.kda_abi_version() == 101   # 1.1: KDA_SPLIT and the automatic path choice
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
@@ -77,7 +77,9 @@ def test_chunk_fwd_rejects_bad_arguments_on_host(kda):
     # misaligned pointer (never dereferenced)
     assert _call_chunk(kda, k=0x1004) == -3
     # unknown flag bit / bad dtype / non-finite scale
-    o = kda.make_opts(); o.flags = 8
+    o = kda.make_opts(); o.flags = 16
+    assert _call_chunk(kda, opts=o) == -1
+    o = kda.make_opts(); o.flags = kda.KDA_QK_L2NORM | kda.KDA_FUSED | kda.KDA_SPLIT   # both paths forced
     assert _call_chunk(kda, opts=o) == -1
     o = kda.make_opts(); o.dtype = 7
     assert _call_chunk(kda, opts=o) == -1
@@ -106,6 +108,22 @@ def test_workspace_sizes(kda):
     assert kda.kda_chunk_workspace_bytes(1, 64, 1, 96, 128, o) == 0      # unsupported -> 0
     p = kda.kda_prologue_workspace_bytes(1, 64, 2, 128, 128, o)
     assert p > 3 * 64 * 2 * 128 * 4
+
+
+def test_workspace_follows_the_tensor_core_path(kda):
+    """bf16 d=128: the split path needs one 74,240-byte record per chunk and head, the
+    fused path none; without a flag the cost model picks split for few sequences and
+    fused once B*H fills most of a second wave of SMs (148 SMs assumed without a GPU)."""
+    import torch
+    split = kda.make_opts(torch.bfloat16, fused=False)
+    fused = kda.make_opts(torch.bfloat16, fused=True)
+    auto = kda.make_opts(torch.bfloat16)
+    nch = 3   # T = 130
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, split) >= 2 * 3 * nch * 74240
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, fused) == 0
+    assert kda.kda_chunk_workspace_bytes(1, 4096, 16, 128, 128, auto) > 0
+    if not torch.cuda.is_available():
+        assert kda.kda_chunk_workspace_bytes(8, 8192, 32, 128, 128, auto) == 0
 
 
 def test_recurrent_step_rejects_bad_arguments_on_host(kda):

@@ -91,10 +91,12 @@ def test_complex_kda_small(K, dtype):
     _check(out, S_T, _oracle(x, complex_gate=True), dtype)
 
 
-def test_complex_kda_workload_sampled(K):
-    """Complex-KDA workload at full size (B=8, T=8192, H=32, d=128), sampled heads."""
+@pytest.mark.parametrize("fused", [None, False], ids=["auto", "split"])
+def test_complex_kda_workload_sampled(K, fused):
+    """Complex-KDA workload at full size (B=8, T=8192, H=32, d=128), sampled heads, through
+    the path the library picks (fused on a 148-SM B200) and through the split path."""
     x = W.workload_inputs("ckda")
-    out, S_T = _run(K, x, complex_gate=True)
+    out, S_T = _run(K, x, complex_gate=True, fused=fused)
     heads = [(0, 0), (3, 17), (7, 31)]
     _check(out, S_T, _oracle(x, heads, complex_gate=True), torch.bfloat16, heads)
 
