@@ -398,15 +398,33 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
                     *reinterpret_cast<uint4 *>(smem + OFF_KD + off_r128(r, c0)) = pack8(y2);
-                    // B rows of the pairs (b, band) for b = band..3
-                    for (int bb = band; bb < 4; ++bb) {
-                        float f[8], y3[8];
-                        ld8f(TF + (bb * 4 + band) * D + c0, f);
+                }
+            }
+        }
+        // B rows of the pairs (b, band(i)) for b = band(i)..3, spread evenly: warp = 8-channel
+        // group, lane = key row i in bands 0-1 plus the mirrored row 63 - i in bands 3-2
+        // (five copies per lane)
+        {
+            const int c0 = 8 * warp;
+            const int w32 = c0 >> 5, sh8 = c0 & 31;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
-                        const int brow = 16 * pair_of(bb, band) + (r & 15);
-                        *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
-                    }
+            for (int side = 0; side < 2; ++side) {
+                const int i = side ? 63 - lane : lane;
+                const int bi = i >> 4;
+                const float nk = NRM[64 + i];
+                const uint32_t swi = fl.complex_gate ? (SGNL[i * 4 + w32] ^ PP[bi * 4 + w32]) >> sh8 : 0u;
+                float x[8], E[8], inv[8];
+                unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_STG_K + off_sw128(i, c0)), x);
+                ld8f(EX + i * E_STRIDE + c0, E);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) inv[e] = __fdividef(((swi >> e) & 1u) ? -nk * x[e] : nk * x[e], E[e]);
+                for (int bb = bi; bb < 4; ++bb) {
+                    float f[8], y3[8];
+                    ld8f(TF + (bb * 4 + bi) * D + c0, f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
+                    const int brow = 16 * pair_of(bb, bi) + (i & 15);
+                    *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
                 }
             }
         }
