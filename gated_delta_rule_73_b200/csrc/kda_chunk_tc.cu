@@ -11,10 +11,11 @@
 //   CUDA     gamma = chunk-local cumsum of log|alpha| per key channel; band
 //   cores    references p_j = gamma just before 16-token band j; per row the
 //            factor E = e^{gamma_r - p_band(r)} in [e^-80, 1] (bounded decay)
-//   tcgen05  A_qk / A_kk sub-tiles: for column band j, D[:, 16j..] =
-//            [Q e^{gamma - p_j}; beta K e^{gamma - p_j}] (A in TMEM) x
-//            (K e^{p_j - gamma})^T -- every factor stays inside the bf16 range
-//            because a band spans 16 tokens and g > -5 (cumulative >= -80)
+//   tcgen05  A_qk / A_kk: all ten (row band b, column band j <= b) pairs as one
+//            N = 160 product.  A = [Q E; beta K E] (rows scaled by their own band
+//            reference, in TMEM); the B rows of pair (b, j) are k_i e^{p_b - gamma_i}
+//            for the 16 tokens i of band j.  Every factor stays inside the bf16
+//            range because a band spans 16 tokens and g > -5 (cumulative >= -80)
 //   CUDA     Tm = (I + A_kk)^{-1} (UT transform) in FP32, 16x16 blocks
 //   tcgen05  W^T = (K e^gamma)^T Tm'^T,  U^T = V^T Tm'^T   (Tm' = Tm diag(beta))
 //   tcgen05  V~^T = U^T - S^T W^T,  O^T = S^T (Q e^gamma)^T
