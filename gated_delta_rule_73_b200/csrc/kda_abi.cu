@@ -95,8 +95,14 @@ size_t chunk_ws(int B, int T, int H, int dk, int dv) {
 
 // The prologue's outputs are bf16 when the tensor-core chunk kernel follows
 // (bf16 activations, dk = dv = 128; it needs no further workspace), FP32 otherwise.
-size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, bool tc, size_t tc_extra, size_t *off) {
-    // off[0..5]: qc, kc, vc, g, beta, chunk workspace
+size_t prologue_ws_parts(int B, int T, int H, int dk, int dv, bool tc, size_t tc_extra, size_t *off,
+                         bool fused_pro = false) {
+    // off[0..5]: qc, kc, vc, g, beta, chunk workspace.  With the prologue fused into the
+    // split form's prep kernel there are no intermediates: only the chunk workspace.
+    if (fused_pro) {
+        for (int i = 0; i < 6; ++i) off[i] = 0;
+        return tc_extra;
+    }
     const size_t rows = (size_t)B * T * H;
     const size_t e = tc ? 2 : 4;
     size_t o = 0;
@@ -160,7 +166,8 @@ size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, const k
     if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
     if (B <= 0 || T <= 0 || H <= 0) return 0;
     size_t off[6];
-    return prologue_ws_parts(B, T, H, dk, dv, use_tc(o, dk, dv), tc_ws(o, B, T, H), off);
+    const bool tc = use_tc(o, dk, dv);
+    return prologue_ws_parts(B, T, H, dk, dv, tc, tc_ws(o, B, T, H), off, tc && !use_fused(o, B, H));
 }
 
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -242,7 +249,8 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
         if (!aligned16(p)) return KDA_ERR_ALIGN;
     size_t off[6];
     const bool tc = use_tc(o, dk, dv);
-    const size_t need = prologue_ws_parts(B, T, H, dk, dv, tc, tc ? tc_ws(o, B, T, H) : 0, off);
+    const bool fused_pro = tc && !use_fused(o, B, H);   // split form: prologue inside its prep
+    const size_t need = prologue_ws_parts(B, T, H, dk, dv, tc, tc ? tc_ws(o, B, T, H) : 0, off, fused_pro);
     if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
     char *ws = (char *)o.workspace;
 
@@ -256,6 +264,23 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     p.g = ws + off[3]; p.beta = ws + off[4];
 
     int launches = 0;
+    if (fused_pro) {
+        ChunkArgs a;
+        memset(&a, 0, sizeof(a));
+        a.t_qkv = a.t_g = a.t_beta = a.t_out = Elt::BF16;
+        a.S0 = S0; a.out = out; a.S_T = S_T;
+        a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+        o.flags |= KDA_QK_L2NORM;
+        a.fl = kflags(o);
+        a.workspace = ws;
+        a.workspace_bytes = need;
+        a.events = o.events; a.n_events = o.n_events;
+        a.launch_idx = &launches;
+        cudaError_t e = launch_chunk_tc2_prologue(p, a, stream);
+        if (e == cudaSuccess && o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
+        if (e == cudaErrorInvalidValue) return KDA_ERR_UNSUPPORTED;
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
     if (o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
     ++launches;
     cudaError_t e = launch_prologue(p, stream);

@@ -57,9 +57,12 @@ __device__ __forceinline__ uint32_t off_r128(int r, int c) {
 __device__ __forceinline__ uint32_t off_r64(int r, int c) {
     return (uint32_t)((r & 7) * 16 + (r >> 3) * 1024 + (c >> 3) * 128 + (c & 7) * 2);
 }
+// staging tile of 64 (or, with the halo of the fused prologue, 67) token rows x 128 channels
+// as two 64-channel halves of 128-byte-swizzled rows, the halves 9 KB apart
+constexpr uint32_t kHalf = 9216;
 __device__ __forceinline__ uint32_t off_sw128(int r, int c) {
     const int hf = c >> 6, cc = c & 63;
-    return (uint32_t)(hf * 8192 + r * 128 + ((((cc >> 3) ^ (r & 7))) << 4) + (cc & 7) * 2);
+    return (uint32_t)(hf * kHalf + r * 128 + ((((cc >> 3) ^ (r & 7))) << 4) + (cc & 7) * 2);
 }
 __device__ __forceinline__ int pair_of(int b, int j) { return (j == 0 ? 0 : j == 1 ? 4 : j == 2 ? 7 : 9) + b - j; }
 
@@ -98,8 +101,10 @@ struct alignas(8) Bars {
 // ============================================================== kernel 1: per-chunk prep
 namespace prep {
 constexpr int NT = 512;
-constexpr uint32_t OFF_STG_Q = 0, OFF_STG_K = 16384, OFF_STG_V = 32768, OFF_STG_G = 49152;
-constexpr uint32_t OFF_GAM = 65536;            // fp32 E [64][132]; later AKK / TMF
+constexpr uint32_t kTile = 2 * kHalf;         // one staged tensor
+constexpr uint32_t OFF_STG_Q = 0, OFF_STG_K = kTile, OFF_STG_V = 2 * kTile, OFF_STG_G = 3 * kTile;
+constexpr int kHalo = 3;                       // rows before the chunk the short convolution reads
+constexpr uint32_t OFF_GAM = 4 * kTile;        // fp32 E [64][132]; later AKK / TMF
 constexpr uint32_t E_STRIDE = 132;
 constexpr uint32_t AS = 68;
 constexpr uint32_t OFF_AKK = OFF_GAM;
@@ -119,11 +124,19 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 constexpr uint32_t TC_X = 0, TC_D = 64, TC_U = 224, TC_W = 352;
 }  // namespace prep
 
+// Inputs of the prologue fused into the prep kernel (kda_chunk_fwd_prologue on the split
+// form).  conv_w == nullptr: the tiles are q, k, v, g and beta is given.
+struct PrepPrologue {
+    const __nv_bfloat16 *conv_w;   // [3, H * D, 4]: taps of q, k, v
+    const float *A;                // [H] per-head log-scale of the gate
+    const float *b_logit;          // [B, T, H] beta logits (FP32)
+};
+
 __global__ void __launch_bounds__(prep::NT, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                  int BH, KernelFlags fl) {
+                  int BH, KernelFlags fl, PrepPrologue pro) {
     using namespace prep;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Bars sh;
@@ -173,7 +186,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
     const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
-    const uint64_t dV = sdesc(sbase, 8192, 1024, kSwizzle128B);
+    const uint64_t dV = sdesc(sbase, kHalf, 1024, kSwizzle128B);
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
     auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
         if (tid == 0 && !mbar_wait_bounded(bar, phase, kWaitLimit)) {
@@ -186,24 +199,29 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     // work item = (chunk, b * H + h), chunk fastest; each CTA walks items with a stride of the
     // grid and fetches the next item's tiles as soon as their staging buffers are free
+    // with the fused prologue the maps cover the raw inputs and their boxes are 67 rows high,
+    // starting 3 rows before the chunk (rows before t = 0 read as zeros: no history)
+    const bool fused_pro = pro.conv_w != nullptr;
+    const int rows = fused_pro ? C + kHalo : C, row0 = fused_pro ? -kHalo : 0;
+    const uint32_t tile_bytes = (uint32_t)rows * D * 2u;
     auto issue_qkg = [&](int item) {
         const int ich = item % nch, ibh = item / nch;
-        const int ib = ibh / H, ih = ibh % H, it0 = ich * C;
-        mbar_arrive_expect_tx(bar_tma, 3u * C * D * 2u);
+        const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
+        mbar_arrive_expect_tx(bar_tma, 3u * tile_bytes);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(sbase + OFF_STG_Q + hf * 8192, &tm_q, bar_tma, hf * 64, ih, it0, ib);
-            tma_load_4d(sbase + OFF_STG_K + hf * 8192, &tm_k, bar_tma, hf * 64, ih, it0, ib);
-            tma_load_4d(sbase + OFF_STG_G + hf * 8192, &tm_g, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_Q + hf * kHalf, &tm_q, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_K + hf * kHalf, &tm_k, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_G + hf * kHalf, &tm_g, bar_tma, hf * 64, ih, it0, ib);
         }
     };
     auto issue_v = [&](int item) {
         const int ich = item % nch, ibh = item / nch;
-        const int ib = ibh / H, ih = ibh % H, it0 = ich * C;
-        mbar_arrive_expect_tx(bar_v, (uint32_t)C * D * 2u);
+        const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
+        mbar_arrive_expect_tx(bar_v, tile_bytes);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + OFF_STG_V + hf * 8192, &tm_v, bar_v, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_V + hf * kHalf, &tm_v, bar_v, hf * 64, ih, it0, ib);
     };
     if (tid == 0 && (int)blockIdx.x < nitems) {
         issue_qkg(blockIdx.x);
@@ -216,8 +234,77 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int t0 = ch * C, n = min(C, T - t0);
         const int next = item + (int)gridDim.x;
         uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
-        if (tid < C) BET[tid] = tid < n ? __bfloat162float(beta[((size_t)b * T + t0 + tid) * H + h]) : 0.f;
+        if (tid < C) {
+            float bv = 0.f;
+            if (tid < n) {
+                const size_t bth = ((size_t)b * T + t0 + tid) * H + h;
+                // the fused prologue rounds beta to bf16 like the standalone prologue kernel
+                bv = fused_pro ? __bfloat162float(__float2bfloat16_rn(sigmoid_fast(pro.b_logit[bth])))
+                               : __bfloat162float(beta[bth]);
+            }
+            BET[tid] = bv;
+        }
         ok = wait_all(bar_tma, li & 1u);
+        if (ok && fused_pro) ok = wait_all(bar_v, li & 1u);
+        if (ok && fused_pro) {
+            // ---- fused prologue: short convolution k = 4 + SiLU of q, k, v and the bounded
+            // gate, in place on the staged tiles (halo row i = token t0 - 3 + i; output row r
+            // = token t0 + r).  Thread = (branch, 8-channel group, 8-row segment); every input
+            // row it needs is read before the barrier, so in-place writes cannot race.
+            const int br = tid >> 7, cg = tid & 15, seg = (tid >> 4) & 7;
+            const int c0 = 8 * cg, r0 = 8 * seg;
+            const uint32_t tile = br == 0 ? OFF_STG_Q : br == 1 ? OFF_STG_K : br == 2 ? OFF_STG_V : OFF_STG_G;
+            uint4 raw[C / 8 + kHalo];
+#pragma unroll
+            for (int i = 0; i < C / 8 + kHalo; ++i)
+                raw[i] = *reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r0 + i, c0));
+            __syncthreads();
+            float w[4][8];   // [tap][channel]; the gate branch needs none
+            if (br < 3) {
+                const __nv_bfloat16 *wsrc = pro.conv_w + ((size_t)br * H * D + (size_t)h * D + c0) * 4;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    float x8[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(wsrc + 8 * m), x8);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        w[j][2 * m] = x8[j];
+                        w[j][2 * m + 1] = x8[4 + j];
+                    }
+                }
+            }
+            const float ea = br == 3 ? expf(pro.A[h]) : 0.f;
+            if (br < 3) {
+                float x0[8], x1[8], x2[8];   // sliding window: each staged row is unpacked once
+                unpack8(raw[0], x0);
+                unpack8(raw[1], x1);
+                unpack8(raw[2], x2);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float x3[8], y[8];
+                    unpack8(raw[i + kHalo], x3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float acc = w[0][e] * x0[e] + w[1][e] * x1[e] + w[2][e] * x2[e] + w[3][e] * x3[e];
+                        y[e] = silu_fast(acc);
+                        x0[e] = x1[e];
+                        x1[e] = x2[e];
+                        x2[e] = x3[e];
+                    }
+                    *reinterpret_cast<uint4 *>(smem + tile + off_sw128(r0 + i, c0)) = pack8(y);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float x3[8], y[8];
+                    unpack8(raw[i + kHalo], x3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = -5.f * sigmoid_fast(ea * x3[e]);
+                    *reinterpret_cast<uint4 *>(smem + tile + off_sw128(r0 + i, c0)) = pack8(y);
+                }
+            }
+            __syncthreads();
+        }
 
         if (ok) {
             // ---- band-local cumulative log-decay | row norms
@@ -844,12 +931,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
     return fn;
 }
 
-bool make_map2(CUtensorMap *m, const void *ptr, int B, int T, int H) {
+bool make_map2(CUtensorMap *m, const void *ptr, int B, int T, int H, int rows = C) {
     auto enc = encode_fn2();
     if (!enc) return false;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)T * H * D * 2};
-    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box,
                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -871,11 +958,31 @@ size_t chunk_tc2_workspace_bytes(int B, int T, int H) {
     return nch * (size_t)B * (size_t)H * IMG_BYTES;
 }
 
+static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                                const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
+                                cudaStream_t st);
+
 cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mg;
     if (!make_map2(&mq, a.q, a.B, a.T, a.H) || !make_map2(&mk, a.k, a.B, a.T, a.H) ||
         !make_map2(&mv, a.v, a.B, a.T, a.H) || !make_map2(&mg, a.g, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
+    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr}, st);
+}
+
+cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mz;
+    const int rows = C + prep::kHalo;
+    if (!make_map2(&mq, p.q_pre, a.B, a.T, a.H, rows) || !make_map2(&mk, p.k_pre, a.B, a.T, a.H, rows) ||
+        !make_map2(&mv, p.v_pre, a.B, a.T, a.H, rows) || !make_map2(&mz, p.z, a.B, a.T, a.H, rows))
+        return cudaErrorInvalidValue;
+    return launch_split(a, mq, mk, mv, mz,
+                        PrepPrologue{(const __nv_bfloat16 *)p.conv_w, p.A, p.beta_logit}, st);
+}
+
+static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                                const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
+                                cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)prep::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -887,7 +994,7 @@ cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
     mark_launch(a, st);
     const int nitems = nch * a.B * a.H;
     chunk_prep_kernel<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
-        mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl);
+        mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl, pro);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark_launch(a, st);

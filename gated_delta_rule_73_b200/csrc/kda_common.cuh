@@ -24,6 +24,13 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// Activations of the bf16 prologue (standalone and fused into the split form's prep):
+// __expf and a hardware reciprocal (x * rcp(1 + e^-x)).  Both errors are a few ulp, far below
+// the bf16 rounding of the outputs; for x -> -inf the reciprocal of inf is 0, so the limits
+// stay exact (sigmoid -> 0, SiLU -> -0).
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
 // Options the kernels see (a device-side copy of the host flags).
 struct KernelFlags {
     int l2norm;

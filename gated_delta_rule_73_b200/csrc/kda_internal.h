@@ -54,6 +54,10 @@ int chunk_tc_read_error();
 // Two-kernel tensor-core chunk path (parallel prep + per-head scan); needs a workspace.
 size_t chunk_tc2_workspace_bytes(int B, int T, int H);
 cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st);
+// The split form with the prologue fused into its prep kernel: the prep stages the raw
+// q, k, v, z tiles with a 3-row halo and applies the short convolution, SiLU, the gate and
+// beta = sigmoid(logit) on chip.  Uses a.out, a.S0, a.S_T, sizes, flags, workspace, events.
+cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st);
 

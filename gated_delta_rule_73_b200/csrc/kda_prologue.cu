@@ -57,11 +57,6 @@ prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
     if (d == 0) beta[bth] = from_f32<TO>(sigm(b_logit[bth]));
 }
 
-// Sigmoid for the bf16-output kernel: __expf (a few ulp) and a correctly rounded
-// reciprocal; both errors are far below the bf16 rounding of the result, and
-// 1 / (1 + inf) = 0 keeps the large-negative limit exact.
-__device__ __forceinline__ float sigm_fast(float x) { return __frcp_rn(1.f + __expf(-x)); }
-
 // bf16 in, bf16 out (the tensor-core path): thread = 8 consecutive channels of one head
 // over a run of RUN tokens.  The three previous input rows of each branch stay in
 // registers as the window slides, so every input row is read once per run (plus a
@@ -150,7 +145,7 @@ prologue_bf16_kernel(const __nv_bfloat16 *__restrict__ q_pre, const __nv_bfloat1
                 for (int c = 0; c < 8; ++c) {
                     const float acc = w[0][c] * win[0][c] + w[1][c] * win[1][c] + w[2][c] * win[2][c] +
                                       w[3][c] * x[i][c];
-                    y[c] = acc * sigm_fast(acc);
+                    y[c] = silu_fast(acc);
                     win[0][c] = win[1][c];
                     win[1][c] = win[2][c];
                     win[2][c] = x[i][c];
@@ -170,11 +165,11 @@ prologue_bf16_kernel(const __nv_bfloat16 *__restrict__ q_pre, const __nv_bfloat1
             if (tb + i >= t1) break;
             float gg[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) gg[c] = -5.f * sigm_fast(ea * zz[i][c]);
+            for (int c = 0; c < 8; ++c) gg[c] = -5.f * sigmoid_fast(ea * zz[i][c]);
             st8(g + base + (tb + i) * rowstride, gg);
             if (ch0 % D == 0) {
                 const long long bth = ((long long)b * T_ + tb + i) * H + h;
-                beta[bth] = __float2bfloat16_rn(sigm_fast(b_logit[bth]));
+                beta[bth] = __float2bfloat16_rn(sigmoid_fast(b_logit[bth]));
             }
         }
     }

@@ -106,8 +106,18 @@ def test_workspace_sizes(kda):
     assert a >= 0 and b >= a and c >= b
     assert kda.kda_chunk_workspace_bytes(1, 0, 1, 128, 128, o) == 0
     assert kda.kda_chunk_workspace_bytes(1, 64, 1, 96, 128, o) == 0      # unsupported -> 0
-    p = kda.kda_prologue_workspace_bytes(1, 64, 2, 128, 128, o)
+    # FP32 path: the prologue's FP32 intermediates come first
+    import torch
+    f = kda.make_opts(torch.float32)
+    p = kda.kda_prologue_workspace_bytes(1, 64, 2, 128, 128, f)
     assert p > 3 * 64 * 2 * 128 * 4
+    # bf16 d=128, split form: the prologue runs inside the prep kernel, only records are needed
+    split = kda.make_opts(torch.bfloat16, fused=False)
+    assert (kda.kda_prologue_workspace_bytes(1, 64, 2, 128, 128, split)
+            == kda.kda_chunk_workspace_bytes(1, 64, 2, 128, 128, split))
+    # bf16 d=128, fused form: bf16 intermediates of the standalone prologue kernel
+    fused = kda.make_opts(torch.bfloat16, fused=True)
+    assert kda.kda_prologue_workspace_bytes(1, 64, 2, 128, 128, fused) >= 4 * 64 * 2 * 128 * 2
 
 
 def test_workspace_follows_the_tensor_core_path(kda):

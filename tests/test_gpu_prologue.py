@@ -37,9 +37,9 @@ def _oracle_heads(x, heads):
     return np.stack(outs, axis=2), np.stack(states, axis=1)
 
 
-def _run(K, x):
+def _run(K, x, **kw):
     args = [cuda(x[n]) for n in ("q_pre", "k_pre", "v_pre", "conv_w", "z", "A", "b_logit")]
-    out, S_T = K.chunk_fwd_prologue(*args, cuda(x["S0"]))
+    out, S_T = K.chunk_fwd_prologue(*args, cuda(x["S0"]), **kw)
     torch.cuda.synchronize()
     return out, S_T
 
@@ -53,6 +53,19 @@ def test_prologue_small(K, T, dtype):
     tol = tol_for(dtype)
     assert rel_err(f64(out), ref[0]) <= tol
     assert rel_err(f64(S_T), ref[1]) <= tol
+
+
+@pytest.mark.parametrize("T", [1, 3, 5, 64, 67, 130, 200])
+@pytest.mark.parametrize("fused", [None, True], ids=["prologue-in-prep", "fused-kernel"])
+def test_prologue_tensor_core(K, T, fused):
+    """bf16 d=128: the split form applies the convolution to TMA tiles with a 3-row halo
+    inside its prep kernel (rows before t = 0, or of the previous batch, must read as
+    zeros); the fused form runs the standalone prologue kernel first."""
+    x = W.prologue_inputs(2, T, 3, 128, 128, dtype=torch.bfloat16, seed=100 + T)
+    out, S_T = _run(K, x, fused=fused)
+    ref = _oracle_heads(x, range(3))
+    assert rel_err(f64(out), ref[0]) <= 2e-2
+    assert rel_err(f64(S_T), ref[1]) <= 2e-2
 
 
 def test_sweep_T2048_full(K):
