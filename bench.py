@@ -255,7 +255,26 @@ def rows_n1(K, flush, hbm_peak):
         rows["decode_step"] = {"ms": ms, "GB_per_s": gbs, "bytes_per_step": nbytes,
                                "frac_of_hbm": gbs / hbm_peak, "steps": D["steps"],
                                "note": "state 3.2 GB > L2, no flush needed"}
-        del S, toks, outd
+
+        # decode step with the prologue fused in (conv state carried in HBM), same shapes
+        par = W.decode_prologue_params(H, d)
+        ptoks = [W.decode_prologue_step_inputs(N, H, d, s) for s in range(4)]
+        cstate = torch.zeros((N, 3, 3, H * d), dtype=torch.bfloat16, device="cuda")
+
+        def pstep():
+            t = ptoks[it[0] % 4]
+            it[0] += 1
+            K.kda_recurrent_step_prologue(t["q_pre"], t["k_pre"], t["v_pre"], par["conv_w"], cstate,
+                                          t["z"], par["A"], t["b_logit"], S, outd, optd)
+        for _ in range(3):
+            pstep()
+        ms = statistics.median(time_calls(pstep, D["steps"]))
+        # state read + write, raw q, k, v, z in, out, beta logit, conv state read + write
+        nbytes = N * H * (2 * d * d * 4 + 5 * d * 2 + 4 + 2 * 9 * d * 2) + H * 3 * d * 4 * 2
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        rows["decode_step_prologue"] = {"ms": ms, "GB_per_s": gbs, "bytes_per_step": nbytes,
+                                        "frac_of_hbm": gbs / hbm_peak, "steps": D["steps"]}
+        del S, toks, outd, ptoks, cstate, par
         torch.cuda.empty_cache()
 
         # a6: Complex-KDA vs unsigned KDA at B=8, T=8192, H=32

@@ -138,7 +138,7 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 101; }
+int kda_abi_version(void) { return 102; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -218,6 +218,7 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const void *
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_ALIGN;
     DecodeArgs a;
+    memset(&a, 0, sizeof(a));
     a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.out = out;
     a.units = units; a.dk = dk; a.dv = dv;
     a.bf16 = o.dtype == KDA_BF16;
@@ -225,6 +226,57 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const void *
     if (o.events && o.n_events > 0) cudaEventRecord(o.events[0], stream);
     cudaError_t e = launch_decode(a, stream);
     if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_recurrent_step_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
+                                const void *conv_w, void *conv_state, const void *z, const float *A,
+                                const float *beta_logit, float *S, void *out, int N, int H, int dk,
+                                int dv, const kda_opts *opts, cudaStream_t stream) {
+    kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if (N < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    if (dk != dv || (o.flags & KDA_COMPLEX)) return KDA_ERR_UNSUPPORTED;
+    const long long units = (long long)N * H;
+    if (units == 0) return KDA_OK;
+    if (units > 0x7fffffffLL) return KDA_ERR_SHAPE;
+    if (!q_pre || !k_pre || !v_pre || !conv_w || !conv_state || !z || !A || !beta_logit || !S || !out)
+        return KDA_ERR_ARG;
+    const void *ptrs[] = {q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    DecodeArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q_pre; a.k = k_pre; a.v = v_pre; a.g = z; a.S = S; a.out = out;
+    a.units = units; a.dk = dk; a.dv = dv;
+    a.bf16 = o.dtype == KDA_BF16;
+    o.flags |= KDA_QK_L2NORM;
+    a.fl = kflags(o);
+    a.conv_w = conv_w; a.conv_state = conv_state; a.A = A; a.b_logit = beta_logit; a.H = H;
+    if (o.events && o.n_events > 0) cudaEventRecord(o.events[0], stream);
+    cudaError_t e = launch_decode(a, stream);
+    if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_conv_state_from_prefill(const void *q_pre, const void *k_pre, const void *v_pre,
+                                void *conv_state, int B, int T, int H, int d,
+                                const kda_opts *opts, cudaStream_t stream) {
+    const kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if (B < 0 || T < 0 || H < 0) return KDA_ERR_ARG;
+    if (d != 64 && d != 128) return KDA_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return KDA_OK;
+    if ((long long)B * T * H * d > kMaxElems) return KDA_ERR_SHAPE;
+    if (!conv_state || (T > 0 && (!q_pre || !k_pre || !v_pre))) return KDA_ERR_ARG;
+    const void *ptrs[] = {q_pre, k_pre, v_pre, conv_state};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    cudaError_t e = launch_conv_state_from_prefill(q_pre, k_pre, v_pre, conv_state, B, T, H, d,
+                                                   o.dtype == KDA_BF16, stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

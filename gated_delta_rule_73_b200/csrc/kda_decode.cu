@@ -22,11 +22,34 @@
 
 namespace kda {
 
-template <typename T, int DK, int DV>
+// Decode prologue (page "Kimi K3 の KDA(1)" section 1.2.1 for the short convolution, SiLU and
+// beta = sigmoid(b); page "Kimi K3 模型结构（2）", Q&A on the decay function, for the gate):
+// the new token's raw q, k, v go through the causal k = 4 convolution whose three earlier
+// inputs are the conv state, which is then shifted by one token.
+struct DecodePro {
+    const void *conv_w;
+    void *conv_state;
+    const float *A, *b_logit;
+    int H;
+};
+
+// the four taps of one channel (contiguous) as one vector load
+__device__ __forceinline__ void load_taps(const float *p, float (&w)[4]) {
+    const float4 t = *reinterpret_cast<const float4 *>(p);
+    w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+}
+__device__ __forceinline__ void load_taps(const __nv_bfloat16 *p, float (&w)[4]) {
+    const uint2 t = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&t.y));
+    w[0] = a.x; w[1] = a.y; w[2] = b.x; w[3] = b.y;
+}
+
+template <typename T, int DK, int DV, bool PRO>
 __global__ void __launch_bounds__(256)
 decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                    const T *__restrict__ g, const T *__restrict__ beta, float *__restrict__ S,
-                   T *__restrict__ out, KernelFlags fl) {
+                   T *__restrict__ out, KernelFlags fl, DecodePro pro) {
     constexpr int NT = 256;
     constexpr int CG = DV / 4;        // column groups (float4 each)
     constexpr int RG = NT / CG;       // row groups
@@ -46,13 +69,56 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
 #pragma unroll
     for (int r = 0; r < RPT; ++r) s[r] = __ldcs(&Sp[(size_t)(rg * RPT + r) * CG + cg]);
 
-    if (tid < DK) {
-        qs[tid] = to_f32(q[unit * DK + tid]);
-        ks[tid] = to_f32(k[unit * DK + tid]);
-        const float gv = to_f32(g[unit * DK + tid]);
-        as[tid] = fl.complex_gate ? gv : expf(gv);
+    float bt;
+    if constexpr (PRO) {
+        static_assert(DK == DV, "the decode prologue needs dk == dv");
+        const int H = pro.H, h = (int)(unit % H);
+        const size_t n = unit / H, HD = (size_t)H * DK, ch = (size_t)h * DK + tid;
+        const T *w = static_cast<const T *>(pro.conv_w);
+        T *cs = static_cast<T *>(pro.conv_state) + n * 9 * HD;   // [3 branches][3 taps][H * d]
+        if (tid < DK) {
+            // every load first (one round of latency, overlapping the state's), then the math,
+            // then the shifted conv state
+            float taps[3][4], hist[3][3], x[3];
+#pragma unroll
+            for (int br = 0; br < 3; ++br) {
+                load_taps(w + (br * HD + ch) * 4, taps[br]);
+#pragma unroll
+                for (int j = 0; j < 3; ++j) hist[br][j] = to_f32(cs[(br * 3 + j) * HD + ch]);
+            }
+            x[0] = to_f32(q[unit * DK + tid]);
+            x[1] = to_f32(k[unit * DK + tid]);
+            x[2] = to_f32(v[unit * DV + tid]);
+            const float zv = to_f32(g[unit * DK + tid]), a_h = pro.A[h];
+            float y[3];
+#pragma unroll
+            for (int br = 0; br < 3; ++br) {
+                const float acc = taps[br][0] * hist[br][0] + taps[br][1] * hist[br][1] +
+                                  taps[br][2] * hist[br][2] + taps[br][3] * x[br];
+                y[br] = acc / (1.f + expf(-acc));
+            }
+            qs[tid] = y[0];
+            ks[tid] = y[1];
+            vs[tid] = y[2];
+            as[tid] = expf(-5.f / (1.f + expf(-expf(a_h) * zv)));
+#pragma unroll
+            for (int br = 0; br < 3; ++br) {
+                cs[(br * 3 + 0) * HD + ch] = from_f32<T>(hist[br][1]);
+                cs[(br * 3 + 1) * HD + ch] = from_f32<T>(hist[br][2]);
+                cs[(br * 3 + 2) * HD + ch] = from_f32<T>(x[br]);
+            }
+        }
+        bt = 1.f / (1.f + expf(-pro.b_logit[unit]));
+    } else {
+        if (tid < DK) {
+            qs[tid] = to_f32(q[unit * DK + tid]);
+            ks[tid] = to_f32(k[unit * DK + tid]);
+            const float gv = to_f32(g[unit * DK + tid]);
+            as[tid] = fl.complex_gate ? gv : expf(gv);
+        }
+        if (tid < DV) vs[tid] = to_f32(v[unit * DV + tid]);
+        bt = to_f32(beta[unit]);
     }
-    if (tid < DV) vs[tid] = to_f32(v[unit * DV + tid]);
     __syncthreads();
     const int warp = tid >> 5, lane = tid & 31;
     if (warp < 3) {
@@ -92,7 +158,6 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
             sk += rk[e];
             sq += rq[e];
         }
-        const float bt = to_f32(beta[unit]);
         const float u = bt * (vs[j] - fk * sk);
         us[j] = u;
         out[unit * DV + j] = from_f32<T>(fl.scale * (fq * sq + qk * u));
@@ -109,20 +174,24 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
     }
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int DV, bool PRO>
 static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t st) {
-    decode_step_kernel<T, DK, DV><<<(unsigned)a.units, 256, 0, st>>>(
+    decode_step_kernel<T, DK, DV, PRO><<<(unsigned)a.units, 256, 0, st>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.g, (const T *)a.beta, a.S,
-        (T *)a.out, a.fl);
+        (T *)a.out, a.fl, DecodePro{a.conv_w, a.conv_state, a.A, a.b_logit, a.H});
     return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t st) {
-    if (a.dk == 128 && a.dv == 128) return launch_decode_t<T, 128, 128>(a, st);
-    if (a.dk == 128 && a.dv == 64) return launch_decode_t<T, 128, 64>(a, st);
-    if (a.dk == 64 && a.dv == 128) return launch_decode_t<T, 64, 128>(a, st);
-    return launch_decode_t<T, 64, 64>(a, st);
+    if (a.conv_w) {   // the prologue needs dk == dv (checked by the host)
+        if (a.dk == 128) return launch_decode_t<T, 128, 128, true>(a, st);
+        return launch_decode_t<T, 64, 64, true>(a, st);
+    }
+    if (a.dk == 128 && a.dv == 128) return launch_decode_t<T, 128, 128, false>(a, st);
+    if (a.dk == 128 && a.dv == 64) return launch_decode_t<T, 128, 64, false>(a, st);
+    if (a.dk == 64 && a.dv == 128) return launch_decode_t<T, 64, 128, false>(a, st);
+    return launch_decode_t<T, 64, 64, false>(a, st);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {

@@ -14,7 +14,19 @@ struct DecodeArgs {
     int dk, dv;
     bool bf16;
     KernelFlags fl;
+    // decode prologue (conv_w != nullptr): q, k, v are the raw new token, g is the gate
+    // logit z, beta is unused; the short convolution reads and shifts conv_state
+    const void *conv_w;     // [3, H * d, 4]
+    void *conv_state;       // [N, 3 branches, 3 taps (t-3, t-2, t-1), H * d], dtype of q
+    const float *A;         // [H]
+    const float *b_logit;   // [N, H]
+    int H;
 };
+
+// Last three raw rows of each branch of a prefill, as the decode prologue's conv state.
+cudaError_t launch_conv_state_from_prefill(const void *q_pre, const void *k_pre, const void *v_pre,
+                                           void *conv_state, int B, int T, int H, int d, bool bf16,
+                                           cudaStream_t st);
 
 // Element types of the chunk path's inputs.
 enum class Elt : int { BF16 = 0, F32 = 1 };

@@ -176,12 +176,44 @@ prologue_bf16_kernel(const __nv_bfloat16 *__restrict__ q_pre, const __nv_bfloat1
 }
 }  // namespace
 
+// conv_state[b][branch][j][c] = raw input of that branch at token T - 3 + j (zero before t = 0):
+// the three inputs the next token's short convolution reads.
+template <typename T>
+__global__ void __launch_bounds__(256)
+conv_state_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre, const T *__restrict__ v_pre,
+                  T *__restrict__ cs, int T_, long long HD, long long total) {
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total) return;
+    const long long c = idx % HD, r = idx / HD;   // r = (b * 3 + branch) * 3 + j
+    const int j = (int)(r % 3), br = (int)((r / 3) % 3);
+    const long long b = r / 9;
+    const int t = T_ - 3 + j;
+    const T *src = br == 0 ? q_pre : br == 1 ? k_pre : v_pre;
+    cs[idx] = t >= 0 ? src[(b * T_ + t) * HD + c] : from_f32<T>(0.f);
+}
+
 template <typename T, typename TO>
 static void launch_t(const PrologueArgs &a, long long total, unsigned blocks, cudaStream_t st) {
     prologue_kernel<T, TO><<<blocks, 256, 0, st>>>(
         (const T *)a.q_pre, (const T *)a.k_pre, (const T *)a.v_pre, (const T *)a.conv_w,
         (const T *)a.z, a.A, a.beta_logit, a.T, a.H, a.dk, total, (TO *)a.qc, (TO *)a.kc,
         (TO *)a.vc, (TO *)a.g, (TO *)a.beta);
+}
+
+cudaError_t launch_conv_state_from_prefill(const void *q_pre, const void *k_pre, const void *v_pre,
+                                           void *conv_state, int B, int T, int H, int d, bool bf16,
+                                           cudaStream_t st) {
+    const long long HD = (long long)H * d, total = (long long)B * 9 * HD;
+    const unsigned blocks = (unsigned)((total + 255) / 256);
+    if (bf16)
+        conv_state_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+            (const __nv_bfloat16 *)q_pre, (const __nv_bfloat16 *)k_pre, (const __nv_bfloat16 *)v_pre,
+            (__nv_bfloat16 *)conv_state, T, HD, total);
+    else
+        conv_state_kernel<float><<<blocks, 256, 0, st>>>((const float *)q_pre, (const float *)k_pre,
+                                                         (const float *)v_pre, (float *)conv_state, T,
+                                                         HD, total);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st) {

@@ -49,6 +49,10 @@ def _load():
     lib.kda_recurrent_step.restype = ip
     lib.kda_chunk_fwd_prologue.argtypes = [vp] * 10 + [ip] * 5 + [op, vp]
     lib.kda_chunk_fwd_prologue.restype = ip
+    lib.kda_recurrent_step_prologue.argtypes = [vp] * 10 + [ip] * 4 + [op, vp]
+    lib.kda_recurrent_step_prologue.restype = ip
+    lib.kda_conv_state_from_prefill.argtypes = [vp] * 4 + [ip] * 4 + [op, vp]
+    lib.kda_conv_state_from_prefill.restype = ip
     lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 8 + [ip] * 5 + [op, vp]
     lib.kda_chunk_fwd_noalloc.restype = ip
     lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
@@ -186,6 +190,33 @@ def kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, ou
         raise KdaError("kda_chunk_fwd_prologue", st)
 
 
+def kda_recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, out,
+                                opts: kda_opts, stream=None) -> None:
+    """Call ``kda_recurrent_step_prologue``; q_pre,k_pre,z [N,H,dk], v_pre,out [N,H,dv],
+    conv_w [3,H*dk,4], conv_state [N,3,3,H*dk] (updated), A [H], beta_logit [N,H], S updated."""
+    N, H, dk = q_pre.shape
+    dv = v_pre.shape[-1]
+    dt = q_pre.dtype
+    args = [_ptr(q_pre, "q_pre", dt), _ptr(k_pre, "k_pre", dt), _ptr(v_pre, "v_pre", dt),
+            _ptr(conv_w, "conv_w", dt), _ptr(conv_state, "conv_state", dt), _ptr(z, "z", dt),
+            _ptr(A, "A", torch.float32), _ptr(beta_logit, "beta_logit", torch.float32),
+            _ptr(S, "S", torch.float32), _ptr(out, "out", dt)]
+    st = _lib.kda_recurrent_step_prologue(*args, N, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_recurrent_step_prologue", st)
+
+
+def kda_conv_state_from_prefill(q_pre, k_pre, v_pre, conv_state, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_conv_state_from_prefill``: raw inputs [B,T,H,d] -> conv_state [B,3,3,H*d]."""
+    B, T, H, d = q_pre.shape
+    dt = q_pre.dtype
+    args = [_ptr(q_pre, "q_pre", dt), _ptr(k_pre, "k_pre", dt), _ptr(v_pre, "v_pre", dt),
+            _ptr(conv_state, "conv_state", dt)]
+    st = _lib.kda_conv_state_from_prefill(*args, B, T, H, d, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_conv_state_from_prefill", st)
+
+
 # ------------------------------------------------------------------ conveniences
 def chunk_fwd(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False, scale=1.0,
               fused=None, workspace=None, out=None, S_T=None, stream=None):
@@ -213,6 +244,26 @@ def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scal
         out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale)
     kda_recurrent_step(q, k, v, g, beta, S, out, opts, stream)
+    return out
+
+
+def recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, *,
+                            scale=1.0, out=None, stream=None):
+    """Run ``kda_recurrent_step_prologue`` (S and conv_state updated in place); returns out."""
+    if out is None:
+        out = torch.empty(v_pre.shape, dtype=q_pre.dtype, device=q_pre.device)
+    opts = make_opts(q_pre.dtype, scale=scale)
+    kda_recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, out,
+                                opts, stream)
+    return out
+
+
+def conv_state_from_prefill(q_pre, k_pre, v_pre, *, out=None, stream=None):
+    """Return the decode conv state [B,3,3,H*d] continuing a prefill over q_pre, k_pre, v_pre."""
+    B, T, H, d = q_pre.shape
+    if out is None:
+        out = torch.empty((B, 3, 3, H * d), dtype=q_pre.dtype, device=q_pre.device)
+    kda_conv_state_from_prefill(q_pre, k_pre, v_pre, out, make_opts(q_pre.dtype), stream)
     return out
 
 

@@ -170,6 +170,42 @@ size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv,
                                     const kda_opts *opts);
 
 /*
+ * kda_recurrent_step_prologue -- the decode step with its branch prologue fused in.
+ *
+ * Page "Kimi K3 の KDA(1)", section 1.2.1 (short convolution k = 4 + SiLU on q, k,
+ * v; beta = sigmoid(b) in FP32) and page "Kimi K3 模型结构（2）", Q&A on the decay
+ * function (g = -5 * sigmoid(exp(A_h) * z)), applied to one new token per sequence.
+ * The convolution's three earlier inputs per channel come from conv_state, which
+ * is shifted by the new token in place; then q, k are L2 normalised (implied) and
+ * the recurrent step of kda_recurrent_step runs.  All of it in FP32, in one kernel.
+ *
+ *   q_pre, k_pre, v_pre [N,H,d]   the new token's raw branch inputs (dtype)
+ *   conv_w       [3, H*d, 4]      taps of q, k, v, tap 3 on the current token (dtype)
+ *   conv_state   [N, 3, 3, H*d]   per sequence, branch (q, k, v) and tap
+ *                                 (t-3, t-2, t-1): the previous raw inputs (dtype),
+ *                                 read and overwritten.  Zeros = no history.
+ *   z            [N,H,d]          gate logits (dtype);  A [H] FP32;  beta_logit [N,H] FP32
+ *   S, out       as in kda_recurrent_step
+ * Needs dk == dv; KDA_COMPLEX is not supported (no signed-gate map on the pages).
+ */
+int kda_recurrent_step_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
+                                const void *conv_w, void *conv_state, const void *z,
+                                const float *A, const float *beta_logit, float *S, void *out,
+                                int N, int H, int dk, int dv, const kda_opts *opts,
+                                cudaStream_t stream);
+
+/*
+ * kda_conv_state_from_prefill -- the handoff from a prefill to decode: writes the
+ * conv state [B, 3, 3, H*d] that kda_recurrent_step_prologue continues from, i.e.
+ * the raw q, k, v inputs [B,T,H,d] of tokens T-3, T-2, T-1 (zeros where t < 0).
+ * With the final state S_T of kda_chunk_fwd_prologue, decode then continues the
+ * same sequence exactly.  opts->dtype gives the element type; d is 64 or 128.
+ */
+int kda_conv_state_from_prefill(const void *q_pre, const void *k_pre, const void *v_pre,
+                                void *conv_state, int B, int T, int H, int d,
+                                const kda_opts *opts, cudaStream_t stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
  *
  * The pages have no counterpart: this is a deployment variant, not part of
@@ -200,7 +236,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
-/* Library ABI version: 100 * major + minor. */
+/* Library ABI version: 100 * major + minor (1.2: decode prologue and conv-state handoff). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

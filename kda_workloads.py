@@ -151,6 +151,24 @@ def decode_log_scale(H, *, seed=0):
     return _uniform((H,), -1.0, 0.0, _gen(10_000 + seed))
 
 
+def decode_prologue_params(H, d, *, dtype=torch.bfloat16, seed=0):
+    """Per-head parameters of the decode prologue: conv taps [3, H*d, 4] ~ U(-0.5, 0.5)
+    (the sweep recipe) and A [H] ~ U(-1, 0) FP32."""
+    gen = _gen(500 + seed)
+    conv_w = _uniform((3, H * d, 4), -0.5, 0.5, gen).to(dtype).contiguous()
+    A = _uniform((H,), -1.0, 0.0, gen).contiguous()
+    return dict(conv_w=conv_w, A=A)
+
+
+def decode_prologue_step_inputs(N, H, d, step, *, dtype=torch.bfloat16):
+    """One decode token's raw prologue inputs: q_pre, k_pre, v_pre, z [N, H, d] ~ N(0,1) in
+    the run dtype, beta logits [N, H] ~ N(0,1) FP32."""
+    gen = _gen(700 + step)
+    cast = lambda x: x.to(dtype).contiguous()
+    q_pre, k_pre, v_pre, z = (cast(_randn((N, H, d), gen)) for _ in range(4))
+    return dict(q_pre=q_pre, k_pre=k_pre, v_pre=v_pre, z=z, b_logit=_randn((N, H), gen).contiguous())
+
+
 def decode_step_inputs(N, H, dk, dv, step, *, A=None, dtype=torch.bfloat16):
     """One decode step's token: q, k, v [N, H, d], g [N, H, dk], beta [N, H]."""
     if A is None:

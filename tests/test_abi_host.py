@@ -34,6 +34,7 @@ def _declared_functions():
 def test_header_declares_the_entry_points():
     names = _declared_functions()
     for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_prologue",
+              "kda_recurrent_step_prologue", "kda_conv_state_from_prefill",
               "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_status_string",
               "kda_abi_version"):
         assert n in names
@@ -46,7 +47,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 101   # 1.1: KDA_SPLIT and the automatic path choice
+    assert kda.kda_abi_version() == 102   # 1.2: decode prologue and conv-state handoff
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
@@ -157,3 +158,37 @@ def test_prologue_rejects_complex_and_unequal_dims(kda):
     assert call(kda.make_opts(complex_gate=True)) == -4
     assert call(kda.make_opts(), dk=64, dv=128) == -4
     assert call(kda.make_opts()) == -7                     # needs a workspace
+
+
+def test_decode_prologue_rejects_bad_arguments_on_host(kda):
+    """kda_recurrent_step_prologue / kda_conv_state_from_prefill argument checks (no GPU)."""
+    P = 0x1000
+    lib = kda._lib
+    o = kda.make_opts()
+
+    def step(N=2, H=3, dk=128, dv=128, opts=o, **kw):
+        p = [ctypes.c_void_p(P)] * 10
+        for i, name in enumerate(("q", "k", "v", "w", "cs", "z", "A", "b", "S", "out")):
+            if name in kw:
+                p[i] = ctypes.c_void_p(kw[name])
+        return lib.kda_recurrent_step_prologue(*p, N, H, dk, dv, ctypes.byref(opts), None)
+
+    assert step(dk=128, dv=64) == -4                 # needs dk == dv
+    assert step(dk=96, dv=96) == -4
+    c = kda.make_opts(complex_gate=True)
+    assert step(opts=c) == -4                        # no signed-gate map for the prologue
+    assert step(cs=0) == -1                          # conv state is required
+    assert step(cs=0x1008) == -3                     # misaligned
+    assert step(N=0) == 0 and step(H=0) == 0         # nothing to do
+
+    def handoff(B=2, T=5, H=3, d=128, **kw):
+        p = [ctypes.c_void_p(P)] * 4
+        for i, name in enumerate(("q", "k", "v", "cs")):
+            if name in kw:
+                p[i] = ctypes.c_void_p(kw[name])
+        return lib.kda_conv_state_from_prefill(*p, B, T, H, d, ctypes.byref(o), None)
+
+    assert handoff(d=96) == -4
+    assert handoff(T=-1) == -1
+    assert handoff(cs=0) == -1
+    assert handoff(B=0) == 0
