@@ -233,6 +233,30 @@ def rows_n1(K, flush, hbm_peak):
         del x, args, ws, out, S_T
         torch.cuda.empty_cache()
 
+        # a2-a4 + the output epilogue (RMSNorm * sigmoid gate) on the prefill workload
+        x = W.workload_inputs("prefill")
+        Bp, Tp, Hp = x["q"].shape[:3]
+        gen = torch.Generator().manual_seed(11)
+        gate = torch.randn(x["v"].shape, generator=gen).to(torch.bfloat16).cuda()
+        nw = torch.ones(d, dtype=torch.float32, device="cuda")
+        o1 = K.make_opts(torch.bfloat16)
+        wsg = torch.empty(max(K.kda_chunk_workspace_bytes(Bp, Tp, Hp, d, d, o1), 16), dtype=torch.uint8,
+                          device="cuda")
+        og = K.make_opts(torch.bfloat16, workspace=wsg)
+        outg = torch.empty(x["v"].shape, dtype=torch.bfloat16, device="cuda")
+        Sg = torch.empty((Bp, Hp, d, d), dtype=torch.float32, device="cuda")
+        fg = lambda: K.kda_chunk_fwd_gated(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], outg, Sg,
+                                           gate, nw, 1e-5, og)
+        fp = lambda: K.kda_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], outg, Sg, og)
+        fg(); fp()
+        ms_g = statistics.median(time_calls(fg, 10, flush))
+        ms_p = statistics.median(time_calls(fp, 10, flush))
+        rows["prefill_output_epilogue"] = {"ms_gated": ms_g, "ms_plain": ms_p,
+                                           "extra_bytes": Bp * Tp * Hp * d * 2,
+                                           "note": "kda_chunk_fwd_gated vs kda_chunk_fwd, B=1 T=4096 H=16"}
+        del x, gate, nw, wsg, outg, Sg
+        torch.cuda.empty_cache()
+
         # a5: decode step, N = 256, H = 96, 64 steps with S carried in HBM
         D = W.DECODE
         N, H = D["N"], D["H"]

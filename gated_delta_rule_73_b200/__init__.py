@@ -10,10 +10,10 @@ _EXPORTS = (
     "KDA_BF16", "KDA_F32", "KDA_QK_L2NORM", "KDA_COMPLEX", "KDA_FUSED", "KDA_SPLIT", "KdaError",
     "kda_opts", "make_opts",
     "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_recurrent_step", "kda_chunk_fwd_prologue",
-    "kda_recurrent_step_prologue", "kda_conv_state_from_prefill",
+    "kda_recurrent_step_prologue", "kda_conv_state_from_prefill", "kda_chunk_fwd_gated",
     "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_abi_version",
     "status_string", "chunk_fwd", "recurrent_step", "chunk_fwd_prologue",
-    "recurrent_step_prologue", "conv_state_from_prefill", "LIB_PATH",
+    "recurrent_step_prologue", "conv_state_from_prefill", "chunk_fwd_gated", "LIB_PATH",
 )
 
 

@@ -132,6 +132,7 @@ struct PrepPrologue {
     const float *b_logit;          // [B, T, H] beta logits (FP32)
 };
 
+template <bool PRO>
 __global__ void __launch_bounds__(prep::NT, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -201,7 +202,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // grid and fetches the next item's tiles as soon as their staging buffers are free
     // with the fused prologue the maps cover the raw inputs and their boxes are 67 rows high,
     // starting 3 rows before the chunk (rows before t = 0 read as zeros: no history)
-    const bool fused_pro = pro.conv_w != nullptr;
+    constexpr bool fused_pro = PRO;
     const int rows = fused_pro ? C + kHalo : C, row0 = fused_pro ? -kHalo : 0;
     const uint32_t tile_bytes = (uint32_t)rows * D * 2u;
     auto issue_qkg = [&](int item) {
@@ -715,19 +716,36 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 constexpr uint32_t TC_D0 = 0, TC_D1 = 128, TC_S = 256;
 }  // namespace scan
 
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (relative error about 2^-11, below
+// the bf16 rounding of the epilogue's output)
+__device__ __forceinline__ float sigmoid_tanh(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+
+// barrier over `count` threads (a multiple of 32) of the CTA, id != 0 (0 is __syncthreads)
+__device__ __forceinline__ void named_bar(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 struct alignas(8) ScanBars {
     uint64_t stage[2];
     uint64_t mV, mS, mO;
     uint32_t tmem_base;
 };
 
+template <bool GATED>
 __global__ void __launch_bounds__(scan::NT, 1)
 chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
                      __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
-                     float scale) {
+                     float scale, const __nv_bfloat16 *__restrict__ gate,
+                     const float *__restrict__ norm_w, float norm_eps) {
     using namespace scan;
     extern __shared__ uint8_t smem_raw[];
     __shared__ ScanBars sh;
+    __shared__ float rms_part[C * 4];   // output epilogue: per-row partial sums of squares
+    __shared__ float w_s[D];            // output epilogue: the RMSNorm weight (ones if absent)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
@@ -782,20 +800,56 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             g_kda_tc2_error = 1;
         }
     };
-    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, 32 values
+    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, 32 values.
+    // With the output epilogue (FusedRMSNormGated) the row's RMS is summed over the four warps
+    // that hold its quarters (named barrier of the eight output warps), then
+    // out = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate) leaves the chip directly.
+    if (GATED && tid < D) w_s[tid] = norm_w ? norm_w[tid] : 1.f;   // read after the first barrier
+    // gate rows of the chunk the next emit stores, loaded one chunk ahead (registers)
+    uint4 gpre[4];
+    auto prefetch_gate = [&](int c) {
+        const int r = row - 64, t0 = c * C;
+        if (GATED && c < nch && t0 + r < T) {
+            const uint4 *gsrc = reinterpret_cast<const uint4 *>(gate + (((size_t)b * T + t0 + r) * H + h) * D + 32 * cq);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) gpre[m] = gsrc[m];
+        }
+    };
     auto emit = [&](int c) {
         const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 32 * cq;
         const int r = row - 64, t0 = c * C;
         float o[32];
         __syncwarp();
         tmem_ld32(tl + dcol, o);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] *= scale;
+        const size_t orow = (((size_t)b * T + t0 + r) * H + h) * D + 32 * cq;
+        if constexpr (GATED) {
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ss += o[e] * o[e];
+            rms_part[r * 4 + cq] = ss;
+            named_bar(1, 256);
+            const float rr = rsqrtf((rms_part[r * 4] + rms_part[r * 4 + 1] + rms_part[r * 4 + 2] +
+                                     rms_part[r * 4 + 3]) / D + norm_eps);
+            if (t0 + r < T) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    float gv[8];
+                    unpack8(gpre[m], gv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        o[8 * m + e] *= rr * w_s[32 * cq + 8 * m + e] * sigmoid_tanh(gv[e]);
+                }
+            }
+        }
         if (t0 + r < T) {
-            uint4 *dst = reinterpret_cast<uint4 *>(out + (((size_t)b * T + t0 + r) * H + h) * D + 32 * cq);
+            uint4 *dst = reinterpret_cast<uint4 *>(out + orow);
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
                 float y[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = scale * o[8 * m + e];
+                for (int e = 0; e < 8; ++e) y[e] = o[8 * m + e];
                 dst[m] = pack8(y);
             }
         }
@@ -867,10 +921,13 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                 *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r128(row, 32 * cq + 8 * m)) = pack8(y);
             }
             fence_proxy_async();
-        } else if (ch > 0) {
-            wait(b_mO, par ^ 1u);
-            tc_fence_after();
-            emit(ch - 1);
+        } else {
+            if (ch > 0) {
+                wait(b_mO, par ^ 1u);
+                tc_fence_after();
+                emit(ch - 1);
+            }
+            prefetch_gate(ch);   // consumed by the next emit (chunk ch)
         }
         tc_fence_before();
         if (__syncthreads_or(failed)) { failed = 1; break; }
@@ -983,23 +1040,26 @@ cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a,
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    // the plain instantiations carry none of the prologue or epilogue code
+    auto prep_k = pro.conv_w ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+    auto scan_k = a.out_gate ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)prep::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(chunk_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)scan::SMEM_BYTES);
+    e = cudaFuncSetAttribute(scan_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int nch = (a.T + C - 1) / C;
     uint8_t *ws = (uint8_t *)a.workspace;
     mark_launch(a, st);
     const int nitems = nch * a.B * a.H;
-    chunk_prep_kernel<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
+    prep_k<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
         mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl, pro);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark_launch(a, st);
-    chunk_scan_tc_kernel<<<a.B * a.H, scan::NT, scan::SMEM_BYTES, st>>>(
-        ws, a.S0, (__nv_bfloat16 *)a.out, a.S_T, a.T, a.H, a.fl.scale);
+    scan_k<<<a.B * a.H, scan::NT, scan::SMEM_BYTES, st>>>(
+        ws, a.S0, (__nv_bfloat16 *)a.out, a.S_T, a.T, a.H, a.fl.scale,
+        (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
     return cudaGetLastError();
 }
 

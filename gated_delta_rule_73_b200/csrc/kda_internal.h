@@ -44,7 +44,15 @@ struct ChunkArgs {
     cudaEvent_t *events;
     int n_events;
     int *launch_idx;                     // running launch counter for events
+    // output epilogue (FusedRMSNormGated): out = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate)
+    // per (token, head) row of dv values; out_gate == nullptr: no epilogue
+    const void *out_gate;                // [B,T,H,dv], dtype of out
+    const float *norm_w;                 // [dv], nullable = ones
+    float norm_eps;
 };
+
+// The output epilogue as its own pass over out (in place), for the paths that do not fuse it.
+cudaError_t launch_out_epilogue(const ChunkArgs &a, cudaStream_t st);
 
 struct PrologueArgs {
     const void *q_pre, *k_pre, *v_pre, *conv_w, *z;

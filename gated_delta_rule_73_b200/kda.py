@@ -49,6 +49,8 @@ def _load():
     lib.kda_recurrent_step.restype = ip
     lib.kda_chunk_fwd_prologue.argtypes = [vp] * 10 + [ip] * 5 + [op, vp]
     lib.kda_chunk_fwd_prologue.restype = ip
+    lib.kda_chunk_fwd_gated.argtypes = [vp] * 10 + [ctypes.c_float] + [ip] * 5 + [op, vp]
+    lib.kda_chunk_fwd_gated.restype = ip
     lib.kda_recurrent_step_prologue.argtypes = [vp] * 10 + [ip] * 4 + [op, vp]
     lib.kda_recurrent_step_prologue.restype = ip
     lib.kda_conv_state_from_prefill.argtypes = [vp] * 4 + [ip] * 4 + [op, vp]
@@ -190,6 +192,22 @@ def kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, ou
         raise KdaError("kda_chunk_fwd_prologue", st)
 
 
+def kda_chunk_fwd_gated(q, k, v, g, beta, S0, out, S_T, out_gate, norm_weight, norm_eps: float,
+                        opts: kda_opts, stream=None) -> None:
+    """Call ``kda_chunk_fwd_gated``: kda_chunk_fwd + out = RMSNorm(o) * w * sigmoid(out_gate)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
+            _ptr(S_T, "S_T", torch.float32), _ptr(out_gate, "out_gate", dt),
+            _ptr(norm_weight, "norm_weight", torch.float32)]
+    st = _lib.kda_chunk_fwd_gated(*args, float(norm_eps), B, T, H, dk, dv, ctypes.byref(opts),
+                                  _stream(stream))
+    if st != 0:
+        raise KdaError("kda_chunk_fwd_gated", st)
+
+
 def kda_recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, out,
                                 opts: kda_opts, stream=None) -> None:
     """Call ``kda_recurrent_step_prologue``; q_pre,k_pre,z [N,H,dk], v_pre,out [N,H,dv],
@@ -245,6 +263,22 @@ def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scal
     opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale)
     kda_recurrent_step(q, k, v, g, beta, S, out, opts, stream)
     return out
+
+
+def chunk_fwd_gated(q, k, v, g, beta, S0, out_gate, norm_weight=None, *, norm_eps=1e-5,
+                    l2norm=True, complex_gate=False, scale=1.0, fused=None, stream=None):
+    """Allocate and run ``kda_chunk_fwd_gated``; returns (out, S_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused)
+    nbytes = kda_chunk_workspace_bytes(B, T, H, dk, dv, opts)
+    workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale,
+                     workspace=workspace, fused=fused)
+    out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    kda_chunk_fwd_gated(q, k, v, g, beta, S0, out, S_T, out_gate, norm_weight, norm_eps, opts, stream)
+    return out, S_T
 
 
 def recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, *,

@@ -119,6 +119,28 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g,
                   int B, int T, int H, int dk, int dv, const kda_opts *opts,
                   cudaStream_t stream);
 
+/*
+ * kda_chunk_fwd_gated -- kda_chunk_fwd with the branch's output epilogue fused in.
+ *
+ * Page "Kimi K3 の KDA(1)", section 1.2.1, the full-rank output gate:
+ * o = FusedRMSNormGated(o, g_out) = RMSNorm(o) * sigmoid(g_out), the RMS taken per
+ * (token, head) over the dv values, the norm before the gate.  Computed as
+ *     out = o / sqrt(mean(o^2) + norm_eps) * norm_weight * sigmoid(out_gate)
+ * in FP32 (the pages give neither the weight nor eps; norm_weight is one dv-vector
+ * shared by the heads, NULL = ones).  On the split tensor-core form with B*H >= 64 it
+ * is applied inside the scan, before the outputs leave the chip; otherwise as one
+ * bandwidth-bound pass over out (cheaper when few sequences make the scan the chain).
+ *
+ *   out_gate    [B,T,H,dv] gate logits (dtype of out), required
+ *   norm_weight [dv] FP32 or NULL;  norm_eps >= 0 (1e-5 is the usual choice)
+ * Everything else, the workspace included, as kda_chunk_fwd.
+ */
+int kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *g,
+                        const void *beta, const float *S0, void *out, float *S_T,
+                        const void *out_gate, const float *norm_weight, float norm_eps,
+                        int B, int T, int H, int dk, int dv, const kda_opts *opts,
+                        cudaStream_t stream);
+
 /* Workspace bytes kda_chunk_fwd needs for these sizes and options. */
 size_t kda_chunk_workspace_bytes(int B, int T, int H, int dk, int dv,
                                  const kda_opts *opts);
@@ -236,7 +258,7 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
-/* Library ABI version: 100 * major + minor (1.2: decode prologue and conv-state handoff). */
+/* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

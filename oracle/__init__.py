@@ -29,6 +29,7 @@ Functions
 ``bounded_log_decay`` g = -5 * sigmoid(exp(A_h) * z).
 ``sigmoid``           beta = sigmoid(b).
 ``prologue_np``       the three together (raw inputs -> q, k, v, g, beta).
+``rmsnorm_gate_np``   the output epilogue RMSNorm(o) * w * sigmoid(g_out).
 
 Every function is pinned by tests in ``tests/test_oracle_pins.py`` against
 closed forms, special cases, brute force and the worked example printed on the
@@ -291,3 +292,18 @@ def prologue_np(q_pre, k_pre, v_pre, conv_w, z, A, b_logit):
     g = bounded_log_decay(z, A)
     beta = sigmoid(b_logit)
     return outs[0], outs[1], outs[2], g, beta
+
+
+def rmsnorm_gate_np(o, gate, w=None, eps=1e-5):
+    """Output epilogue of a KDA branch (*Kimi K3 KDA(1)* section 1.2.1, the full-rank output
+    gate: ``o = FusedRMSNormGated(o, g) = RMSNorm(o) * sigmoid(g)``, the RMS per (token,
+    head) over the head_dim values, the norm before the gate).  Readings: the RMSNorm weight
+    ``w`` is one head_dim vector shared by the heads (None = ones) and ``eps`` sits inside
+    the square root.  ``o``, ``gate``: [..., d]."""
+    o = _f64(o)
+    gate = _f64(gate)
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    y = o / np.sqrt(ms + eps)
+    if w is not None:
+        y = y * _f64(w)
+    return y * sigmoid(gate)

@@ -34,7 +34,7 @@ def _declared_functions():
 def test_header_declares_the_entry_points():
     names = _declared_functions()
     for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_prologue",
-              "kda_recurrent_step_prologue", "kda_conv_state_from_prefill",
+              "kda_recurrent_step_prologue", "kda_conv_state_from_prefill", "kda_chunk_fwd_gated",
               "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_status_string",
               "kda_abi_version"):
         assert n in names
@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 102   # 1.2: decode prologue and conv-state handoff
+    assert kda.kda_abi_version() == 103   # 1.3: kda_chunk_fwd_gated
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"

@@ -137,3 +137,53 @@ def test_prefill_workload_fused(K):
     x = W.workload_inputs("prefill")
     out, S_T = _run(K, x, fused=True)
     _check(out, S_T, _oracle(x), torch.bfloat16)
+
+
+def _check_epilogue(out, plain, gate, w, eps, ref_o, tol):
+    """RMSNorm rescales every (token, head) row to unit size, so a row whose o is small
+    carries the chunk kernel's error magnified.  Two checks: (1) the epilogue itself, against
+    the oracle epilogue applied to the same call's plain output; (2) end to end against the
+    oracle on rows holding at least a fifth of the largest row norm (a tenth of the rows
+    or more on these inputs)."""
+    got = f64(out)
+    mine = oracle.rmsnorm_gate_np(f64(plain), f64(gate), None if w is None else f64(w), eps=eps)
+    assert rel_err(got, mine) <= tol
+    ref = oracle.rmsnorm_gate_np(ref_o, f64(gate), None if w is None else f64(w), eps=eps)
+    norms = np.sqrt(np.sum(ref_o * ref_o, axis=-1))
+    keep = norms >= 0.2 * norms.max()
+    assert keep.sum() >= 0.1 * keep.size
+    assert rel_err(got[keep], ref[keep]) <= tol
+
+
+@pytest.mark.parametrize("fused,H", [(False, 3), (False, 32), (True, 3)],
+                         ids=["split-pass", "split-in-scan", "fused"])
+@pytest.mark.parametrize("T", [64, 130])
+def test_output_epilogue_bf16(K, fused, H, T):
+    """kda_chunk_fwd_gated: out = RMSNorm(o) * w * sigmoid(g_out).  The split form applies
+    it inside the scan kernel when B*H >= 64 (here 2 x 32) and as a pass otherwise; the
+    fused form always as a pass."""
+    x = W.chunk_inputs(2, T, H, 128, 128, dtype=torch.bfloat16, seed=60 + T)
+    gen = torch.Generator().manual_seed(61 + T)
+    gate = torch.randn((2, T, H, 128), generator=gen).to(torch.bfloat16)
+    w = (1.0 + 0.5 * torch.randn(128, generator=gen)).float()
+    q, k, v, g, beta = (cuda(x[n]) for n in ("q", "k", "v", "g", "beta"))
+    S0 = cuda(x["S0"])
+    out, S_T = K.chunk_fwd_gated(q, k, v, g, beta, S0, cuda(gate), cuda(w), norm_eps=1e-5, fused=fused)
+    plain, _ = K.chunk_fwd(q, k, v, g, beta, S0, fused=fused)
+    torch.cuda.synchronize()
+    o, s = _oracle(x)
+    _check_epilogue(out, plain, gate, w, 1e-5, o, 2e-2)
+    assert rel_err(f64(S_T), s) <= 2e-2
+
+
+def test_output_epilogue_fp32_and_no_weight(K):
+    """The FP32 path applies the epilogue as its own pass; weight NULL means ones."""
+    x = W.chunk_inputs(1, 100, 2, 64, 64, dtype=torch.float32, seed=62)
+    gen = torch.Generator().manual_seed(63)
+    gate = torch.randn((1, 100, 2, 64), generator=gen)
+    q, k, v, g, beta = (cuda(x[n]) for n in ("q", "k", "v", "g", "beta"))
+    out, _ = K.chunk_fwd_gated(q, k, v, g, beta, cuda(x["S0"]), cuda(gate), None, norm_eps=1e-6)
+    plain, _ = K.chunk_fwd(q, k, v, g, beta, cuda(x["S0"]))
+    torch.cuda.synchronize()
+    o, _ = _oracle(x)
+    _check_epilogue(out, plain, gate, None, 1e-6, o, 1e-4)

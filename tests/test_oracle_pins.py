@@ -416,3 +416,35 @@ def test_prologue_composes_the_pieces():
             assert np.allclose(q[0, :, h, c], yq / (1 + np.exp(-yq)), atol=1e-14)
     assert np.all((g < 0) & (g > -5))
     assert np.allclose(beta, 1 / (1 + np.exp(-b)), atol=1e-16)
+
+
+def test_rmsnorm_gate_hand_values():
+    """Output epilogue pinned by hand arithmetic: o = (3, 4) has mean square 12.5, so with
+    eps = 0 the norm gives (3, 4) / sqrt(12.5) = (0.848528..., 1.131370...); a gate of 0
+    halves it; w scales channel-wise; a very negative gate closes it."""
+    o = np.array([[3.0, 4.0]])
+    r = np.sqrt(12.5)
+    got = oracle.rmsnorm_gate_np(o, np.array([[40.0, 40.0]]), eps=0.0)
+    assert np.allclose(got, [[3.0 / r, 4.0 / r]], rtol=1e-12)
+    got = oracle.rmsnorm_gate_np(o, np.zeros((1, 2)), w=np.array([2.0, -1.0]), eps=0.0)
+    assert np.allclose(got, [[0.5 * 2.0 * 3.0 / r, 0.5 * -1.0 * 4.0 / r]], rtol=1e-12)
+    got = oracle.rmsnorm_gate_np(o, np.array([[-60.0, -60.0]]), eps=0.0)
+    assert np.all(np.abs(got) < 1e-25)
+
+
+def test_rmsnorm_gate_invariances():
+    """RMSNorm is scale invariant (eps = 0), gives unit mean square, and the norm is taken
+    per row over the last axis only; eps damps small rows toward 0."""
+    rng = np.random.default_rng(4)
+    o = rng.normal(size=(5, 3, 128))
+    big = 1e9                                    # sigmoid(big) = 1: the gate is open
+    y = oracle.rmsnorm_gate_np(o, np.full_like(o, big), eps=0.0)
+    assert np.allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-12)
+    assert np.allclose(oracle.rmsnorm_gate_np(7.5 * o, np.full_like(o, big), eps=0.0), y, rtol=1e-12)
+    o2 = o.copy()
+    o2[0, 0] *= 100.0                            # another row changing leaves this one alone
+    y2 = oracle.rmsnorm_gate_np(o2, np.full_like(o, big), eps=0.0)
+    assert np.allclose(y2[1:], y[1:], rtol=1e-12) and np.allclose(y2[0, 1:], y[0, 1:], rtol=1e-12)
+    tiny = 1e-6 * o[0, 0]
+    damped = oracle.rmsnorm_gate_np(tiny, np.full_like(tiny, big), eps=1.0)
+    assert np.max(np.abs(damped)) < 1e-5
