@@ -16,8 +16,8 @@
 //   writes, per chunk and head, a 74,240-byte record of bf16 tiles already in the
 //   shared-memory layouts the scan's tensor-core products read:
 //     W and Q e^gamma (K-major [r][c], stacked into one [128][128] tile),
-//     K e^{gamma_C-gamma} ([r][c]), U ([r][j]), A_qk (K-major [r][i]) and
-//     sigma_C e^{gamma_C} (FP32 [128]).
+//     K e^{gamma_C-gamma} ([r][c]), U (16-column slabs of [r][j]), A_qk (K-major [r][i])
+//     and sigma_C e^{gamma_C} (FP32 [128]).
 // Kernel 2 (one CTA per head): per chunk, the record is bulk-copied into one of two
 // stages, then
 //   [P ; O] = [W ; Q e^gamma] S                          (S in shared memory as bf16)
@@ -46,7 +46,7 @@ constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr uint32_t IMG_W = 0;           // bf16 W, K-major [64 r][128 c] (with Q e^gamma: one [128][128] tile)
 constexpr uint32_t IMG_QG = 16384;      // bf16 Q e^gamma, K-major [64 r][128 c]
 constexpr uint32_t IMG_KD = 32768;      // bf16 K e^{gamma_C - gamma}, [64 r][128 c]
-constexpr uint32_t IMG_U = 49152;       // bf16 U, [64 r][128 j] (same core layout as W)
+constexpr uint32_t IMG_U = 49152;       // bf16 U as eight 16-column slabs of [64 r][16 j] (2 KB each)
 constexpr uint32_t IMG_AQK = 65536;     // bf16 A_qk, K-major [64 r][64 i]
 constexpr uint32_t IMG_GC = 73728;      // fp32 sigma_C e^{gamma_C} [128]
 constexpr uint32_t IMG_BYTES = 74240;
@@ -56,6 +56,16 @@ __device__ __forceinline__ uint32_t off_r128(int r, int c) {
 }
 __device__ __forceinline__ uint32_t off_r64(int r, int c) {
     return (uint32_t)((r & 7) * 16 + (r >> 3) * 1024 + (c >> 3) * 128 + (c & 7) * 2);
+}
+// [rows][n] bf16 tile of n columns in the no-swizzle core-matrix layout (8 rows x 16 bytes per
+// core matrix, row groups n * 16 bytes apart)
+__device__ __forceinline__ uint32_t off_rn(int r, int c, int n) {
+    return (uint32_t)((r & 7) * 16 + (r >> 3) * (n * 16) + (c >> 3) * 128 + (c & 7) * 2);
+}
+// U in the record: value column j lives in slab j / 16, a [64 r][16 j] tile of its own, so any
+// run of 16-column slabs (one value-column slice of the scan) is one contiguous copy
+__device__ __forceinline__ uint32_t off_u(int r, int j) {
+    return (uint32_t)((j >> 4) * 2048) + off_rn(r, j & 15, 16);
 }
 // staging tile of 64 (or, with the halo of the fused prologue, 67) token rows x 128 channels
 // as two 64-channel halves of 128-byte-swizzled rows, the halves 9 KB apart
@@ -184,6 +194,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_after();
     const uint32_t tbase = sh.tmem_base;
     const uint32_t tl = tbase + ((uint32_t)(quad * 32) << 16);
+    // the scan kernel, launched with a programmatic dependency on this one, may be scheduled
+    // now: its CTAs take SMs as this grid's CTAs leave and wait in-kernel for its completion
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
     const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
@@ -228,23 +241,31 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         issue_qkg(blockIdx.x);
         issue_v(blockIdx.x);
     }
+    // beta (with the fused prologue: its logit) of token row tid < C of an item, loaded one
+    // item ahead so its global-memory latency overlaps the current item
+    auto load_beta = [&](int it) -> float {
+        if (tid >= C || it >= nitems) return 0.f;
+        const int ich = it % nch, ibh = it / nch;
+        const int t = ich * C + tid;
+        if (t >= T) return 0.f;
+        const size_t bth = ((size_t)(ibh / H) * T + t) * H + ibh % H;
+        return fused_pro ? pro.b_logit[bth] : __bfloat162float(beta[bth]);
+    };
+    float bpre = load_beta(blockIdx.x);
     bool ok = true;
     uint32_t li = 0;   // items done by this CTA: parity of the TMA barriers
     for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
-        const int ch = item % nch, bh = item / nch, b = bh / H, h = bh % H;
+        const int ch = item % nch, bh = item / nch, h = bh % H;
         const int t0 = ch * C, n = min(C, T - t0);
         const int next = item + (int)gridDim.x;
         uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
         if (tid < C) {
-            float bv = 0.f;
-            if (tid < n) {
-                const size_t bth = ((size_t)b * T + t0 + tid) * H + h;
-                // the fused prologue rounds beta to bf16 like the standalone prologue kernel
-                bv = fused_pro ? __bfloat162float(__float2bfloat16_rn(sigmoid_fast(pro.b_logit[bth])))
-                               : __bfloat162float(beta[bth]);
-            }
-            BET[tid] = bv;
+            // the fused prologue rounds beta to bf16 like the standalone prologue kernel
+            BET[tid] = tid >= n ? 0.f
+                       : fused_pro ? __bfloat162float(__float2bfloat16_rn(sigmoid_fast(bpre)))
+                                   : bpre;
         }
+        bpre = load_beta(next);
         ok = wait_all(bar_tma, li & 1u);
         if (ok && fused_pro) ok = wait_all(bar_v, li & 1u);
         if (ok && fused_pro) {
@@ -662,19 +683,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         if (ok) {
             tc_fence_after();
-            // ---- W and U ([r][c] and [r][j], K-major core layout) -> the record; lanes 0-63
-            // write W, lanes 64-127 (the repeated rows) write U
+            // ---- W ([r][c], K-major core layout) and U (16-column slabs) -> the record; lanes
+            // 0-63 write W, lanes 64-127 (the repeated rows) write U
             {
                 const int r = row & 63;
                 float w[32];
                 tmem_ld32(tl + (row < 64 ? TC_W : TC_U) + 32 * qq, w);
-                uint8_t *dst = img + (row < 64 ? IMG_W : IMG_U);
 #pragma unroll
                 for (int g8 = 0; g8 < 4; ++g8) {
                     float y[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
-                    *reinterpret_cast<uint4 *>(dst + off_r128(r, 32 * qq + 8 * g8)) = pack8(y);
+                    const int c0 = 32 * qq + 8 * g8;
+                    *reinterpret_cast<uint4 *>(img + (row < 64 ? IMG_W + off_r128(r, c0) : IMG_U + off_u(r, c0))) =
+                        pack8(y);
                 }
             }
         }
@@ -689,31 +711,41 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ============================================================== kernel 2: the scan
-// One CTA per (b, h), 512 threads.  TMEM lane = key channel c for the state and = token
-// row for the chunk products; thread (lane, cq) owns the FP32 state row slice
-// S[c][32 cq .. 32 cq + 31].
-// Per chunk ch (record in stage ch & 1):
-//   [P ; O] = [W ; Q e^gamma] S          one M = 128, N = 128 product into D[ch & 1]
+// The value columns of the state evolve independently (column j of S sees only v_{t,j}), so
+// the scan splits a head's dv = 128 columns into slices of NS columns, one CTA each: a slice
+// runs the same dependent chain with N = NS products and 1/(128/NS) of the per-thread work,
+// and few heads still fill the SMs.  One CTA per (b, h, slice), 128 * NS / CPT threads.
+// TMEM lane = key channel c for the state and = token row for the chunk products; thread
+// (lane, cq) owns the FP32 state row slice S[c][j0 + CPT cq .. + CPT - 1] (j0 = the slice's
+// first column).  Per chunk ch (record in stage ch & 1):
+//   [P ; O] = [W ; Q e^gamma] S          one M = 128, N = NS product into D[ch & 1]
 //   lanes 0-63:   V~ = U - P -> bf16 shared memory
 //   lanes 64-127: the outputs of chunk ch - 1 leave D[(ch - 1) & 1] (16-byte stores)
 //   dS = Kd^T V~;  O += A_qk V~          (A_qk padded with 64 zero rows to M = 128)
 //   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32, and its bf16 copy for the next product.
 namespace scan {
-constexpr int NT = 512;
-// stage: the record's first 65,536 bytes, 8 KB of zeros, then A_qk and sigma_C e^{gamma_C}
-constexpr uint32_t ST_HEAD = IMG_AQK;                       // [W;Qg], Kd, U
-constexpr uint32_t ST_ZERO = IMG_AQK;
-constexpr uint32_t ST_AQK = IMG_AQK + 8192;
-constexpr uint32_t ST_GC = ST_AQK + (IMG_GC - IMG_AQK);
-constexpr uint32_t ST_TAIL_BYTES = IMG_BYTES - IMG_AQK;     // A_qk and sigma_C e^{gamma_C}
-constexpr uint32_t STAGE = 82944;                           // 81 KB
-static_assert(ST_GC + 512 <= STAGE, "stage layout");
-constexpr uint32_t OFF_S = 2 * STAGE;                       // bf16 S [128 c][128 j]
-constexpr uint32_t OFF_VT = OFF_S + 32768;                  // bf16 V~ [64 r][128 j]
-constexpr uint32_t SMEM_BYTES = OFF_VT + 16384 + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM columns: D0 = [P ; O] [0,128), D1 [128,256), dS [256,384)
-constexpr uint32_t TC_D0 = 0, TC_D1 = 128, TC_S = 256;
+// stage: [W;Qg] and Kd (the record's first 48 KB), the slice's U slabs, 8 KB of zeros, then
+// A_qk and sigma_C e^{gamma_C}
+template <int NS>
+struct Layout {
+    static constexpr int CPT = NS < 32 ? NS : 32;       // state columns per thread
+    static constexpr int NT = 128 * (NS / CPT);
+    static constexpr uint32_t HEAD = IMG_U;             // [W;Qg], Kd
+    static constexpr uint32_t U = IMG_U;
+    static constexpr uint32_t U_BYTES = (uint32_t)NS * 128;
+    static constexpr uint32_t ZERO = U + U_BYTES;
+    static constexpr uint32_t AQK = ZERO + 8192;
+    static constexpr uint32_t GC = AQK + (IMG_GC - IMG_AQK);
+    static constexpr uint32_t TAIL_BYTES = IMG_BYTES - IMG_AQK;   // A_qk and sigma_C e^{gamma_C}
+    static constexpr uint32_t STAGE = (GC + 512 + 1023) / 1024 * 1024;
+    static constexpr uint32_t OFF_S = 2 * STAGE;                    // bf16 S [128 c][NS j]
+    static constexpr uint32_t OFF_VT = OFF_S + 128u * NS * 2;       // bf16 V~ [64 r][NS j]
+    static constexpr uint32_t SMEM_BYTES = OFF_VT + 64u * NS * 2 + 1024;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    // TMEM columns: D0 = [P ; O] [0,NS), D1 [NS,2NS), dS [2NS,3NS)
+    static constexpr uint32_t TC_D0 = 0, TC_D1 = NS, TC_S = 2 * NS;
+    static constexpr uint32_t TMEM_COLS = NS == 16 ? 64 : NS == 32 ? 128 : NS == 64 ? 256 : 512;
+};
 }  // namespace scan
 
 // sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (relative error about 2^-11, below
@@ -729,31 +761,46 @@ __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N]) {
+    if constexpr (N == 32) tmem_ld32(taddr, v);
+    else tmem_ld16(taddr, v);
+}
+
+// wait until the grids this one depends on (the prep kernel) have completed and their
+// memory is visible; a no-op when the launch has no programmatic dependency
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 struct alignas(8) ScanBars {
     uint64_t stage[2];
     uint64_t mV, mS, mO;
     uint32_t tmem_base;
 };
 
-template <bool GATED>
-__global__ void __launch_bounds__(scan::NT, 1)
+template <int NS, bool GATED>
+__global__ void __launch_bounds__(scan::Layout<NS>::NT, 1)
 chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
                      __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
                      float scale, const __nv_bfloat16 *__restrict__ gate,
                      const float *__restrict__ norm_w, float norm_eps) {
-    using namespace scan;
+    using L = scan::Layout<NS>;
+    constexpr int CPT = L::CPT, NT = L::NT, NSL = D / NS;
+    static_assert(!GATED || NS == D, "the output epilogue normalises whole rows: one slice per head");
     extern __shared__ uint8_t smem_raw[];
     __shared__ ScanBars sh;
-    __shared__ float rms_part[C * 4];   // output epilogue: per-row partial sums of squares
-    __shared__ float w_s[D];            // output epilogue: the RMSNorm weight (ones if absent)
+    __shared__ float rms_part[GATED ? C * 4 : 1];   // output epilogue: per-row partial sums of squares
+    __shared__ float w_s[GATED ? D : 1];            // output epilogue: the RMSNorm weight (ones if absent)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, cq = warp >> 2;   // lane quadrant, 32-column quarter
-    const int row = quad * 32 + lane;                // TMEM lane
-    const bool p_lane = row < 64;                    // warp-uniform: rows of P (else of O)
-    const int bh = blockIdx.x, b = bh / H, h = bh % H;
+    const int quad = warp & 3, cq = warp >> 2;   // lane quadrant, column group of the slice
+    const int row = quad * 32 + lane;            // TMEM lane
+    const bool p_lane = row < 64;                // warp-uniform: rows of P (else of O)
+    const int bh = blockIdx.x / NSL, sl = blockIdx.x % NSL, b = bh / H, h = bh % H;
+    const int j0 = sl * NS;                      // first value column of this slice
     const int nch = (T + C - 1) / C;
     const uint8_t *recs = ws + (size_t)bh * nch * IMG_BYTES;
     const uint32_t b_mV = smem_u32(&sh.mV), b_mS = smem_u32(&sh.mS), b_mO = smem_u32(&sh.mO);
@@ -768,9 +815,9 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     }
     // the zero rows under each stage's A_qk
     for (int i = tid; i < 2 * 512; i += NT)
-        *reinterpret_cast<uint4 *>(smem + (i >> 9) * STAGE + ST_ZERO + (i & 511) * 16) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(smem + (i >> 9) * L::STAGE + L::ZERO + (i & 511) * 16) = make_uint4(0, 0, 0, 0);
     if (warp == 0) {
-        tmem_alloc(smem_u32(&sh.tmem_base), 512);
+        tmem_alloc(smem_u32(&sh.tmem_base), L::TMEM_COLS);
         tmem_relinquish();
     }
     fence_proxy_async();
@@ -782,14 +829,16 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
     const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
+    const uint64_t dMNs = sdesc(sbase, NS * 16, 128, kSwizzleNone);   // S copy and V~: [K rows][NS]
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
     auto fetch = [&](int ch) {
         const int s = ch & 1;
         const uint32_t bar = smem_u32(&sh.stage[s]);
         const uint8_t *src = recs + (size_t)ch * IMG_BYTES;
-        mbar_arrive_expect_tx(bar, IMG_BYTES);
-        bulk_load(sbase + s * STAGE, src, ST_HEAD, bar);
-        bulk_load(sbase + s * STAGE + ST_AQK, src + IMG_AQK, ST_TAIL_BYTES, bar);
+        mbar_arrive_expect_tx(bar, L::HEAD + L::U_BYTES + L::TAIL_BYTES);
+        bulk_load(sbase + s * L::STAGE, src, L::HEAD, bar);
+        bulk_load(sbase + s * L::STAGE + L::U, src + IMG_U + (uint32_t)sl * L::U_BYTES, L::U_BYTES, bar);
+        bulk_load(sbase + s * L::STAGE + L::AQK, src + IMG_AQK, L::TAIL_BYTES, bar);
     };
     // every thread waits on the barrier itself; a wait that gives up marks this thread, and
     // the whole CTA leaves the loop at the next block-wide barrier (__syncthreads_or)
@@ -800,41 +849,41 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             g_kda_tc2_error = 1;
         }
     };
-    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, 32 values.
+    // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, CPT values.
     // With the output epilogue (FusedRMSNormGated) the row's RMS is summed over the four warps
     // that hold its quarters (named barrier of the eight output warps), then
     // out = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate) leaves the chip directly.
     if (GATED && tid < D) w_s[tid] = norm_w ? norm_w[tid] : 1.f;   // read after the first barrier
     // gate rows of the chunk the next emit stores, loaded one chunk ahead (registers)
-    uint4 gpre[4];
+    uint4 gpre[CPT / 8];
     auto prefetch_gate = [&](int c) {
         const int r = row - 64, t0 = c * C;
         if (GATED && c < nch && t0 + r < T) {
             const uint4 *gsrc = reinterpret_cast<const uint4 *>(gate + (((size_t)b * T + t0 + r) * H + h) * D + 32 * cq);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) gpre[m] = gsrc[m];
+            for (int m = 0; m < CPT / 8; ++m) gpre[m] = gsrc[m];
         }
     };
     auto emit = [&](int c) {
-        const uint32_t dcol = ((c & 1) ? TC_D1 : TC_D0) + 32 * cq;
+        const uint32_t dcol = ((c & 1) ? L::TC_D1 : L::TC_D0) + CPT * cq;
         const int r = row - 64, t0 = c * C;
-        float o[32];
+        float o[CPT];
         __syncwarp();
-        tmem_ld32(tl + dcol, o);
+        tmem_ldn<CPT>(tl + dcol, o);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] *= scale;
-        const size_t orow = (((size_t)b * T + t0 + r) * H + h) * D + 32 * cq;
+        for (int e = 0; e < CPT; ++e) o[e] *= scale;
+        const size_t orow = (((size_t)b * T + t0 + r) * H + h) * D + j0 + CPT * cq;
         if constexpr (GATED) {
             float ss = 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ss += o[e] * o[e];
+            for (int e = 0; e < CPT; ++e) ss += o[e] * o[e];
             rms_part[r * 4 + cq] = ss;
             named_bar(1, 256);
             const float rr = rsqrtf((rms_part[r * 4] + rms_part[r * 4 + 1] + rms_part[r * 4 + 2] +
                                      rms_part[r * 4 + 3]) / D + norm_eps);
             if (t0 + r < T) {
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
+                for (int m = 0; m < CPT / 8; ++m) {
                     float gv[8];
                     unpack8(gpre[m], gv);
 #pragma unroll
@@ -846,7 +895,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         if (t0 + r < T) {
             uint4 *dst = reinterpret_cast<uint4 *>(out + orow);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
+            for (int m = 0; m < CPT / 8; ++m) {
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = o[8 * m + e];
@@ -854,49 +903,52 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             }
         }
     };
-    // FP32 state row S[c = row][32 cq + e] and its bf16 copy (B operand, [c][j] core layout)
-    float S[32];
+    // FP32 state row slice S[c = row][j0 + CPT cq + e] and its bf16 copy (B operand, [c][j]
+    // core layout of NS columns)
+    float S[CPT];
     auto store_state_operand = [&]() {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < CPT / 8; ++m) {
             float y[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) y[e] = S[8 * m + e];
-            *reinterpret_cast<uint4 *>(smem + OFF_S + off_r128(row, 32 * cq + 8 * m)) = pack8(y);
+            *reinterpret_cast<uint4 *>(smem + L::OFF_S + off_rn(row, CPT * cq + 8 * m, NS)) = pack8(y);
         }
         fence_proxy_async();
     };
 
+    if (S0) {
+        const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + j0 + CPT * cq);
+#pragma unroll
+        for (int m = 0; m < CPT / 4; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
+    } else {
+#pragma unroll
+        for (int e = 0; e < CPT; ++e) S[e] = 0.f;
+    }
+    store_state_operand();
+    // everything above overlaps the end of the prep kernel; the records are read from here on
+    grid_dependency_wait();
     if (tid == 0) {
         if (nch > 0) fetch(0);
         if (nch > 1) fetch(1);
     }
-    if (S0) {
-        const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + 32 * cq);
-#pragma unroll
-        for (int m = 0; m < 8; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
-    } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) S[e] = 0.f;
-    }
-    store_state_operand();
     __syncthreads();
 
     for (int ch = 0; ch < nch; ++ch) {
         const int s = ch & 1;
-        const uint32_t st = s * STAGE;
+        const uint32_t st = s * L::STAGE;
         const uint32_t sbar = smem_u32(&sh.stage[s]);
         const uint32_t sph = (uint32_t)(ch >> 1) & 1u;
-        const uint32_t dbuf = s ? TC_D1 : TC_D0;
+        const uint32_t dbuf = s ? L::TC_D1 : L::TC_D0;
         const uint32_t par = (uint32_t)ch & 1u;
         // [P ; O] = [W ; Qg] S
         if (tid == 0) {
             wait(sbar, sph);
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
+            constexpr uint32_t id = idesc_bf16(128, NS, 0, 1, 0);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                mma_ss(tbase + dbuf, at(dK64, st + 256 * k), at(dMN64, OFF_S + 4096 * k), id, k > 0);
+                mma_ss(tbase + dbuf, at(dK64, st + 256 * k), at(dMNs, L::OFF_S + NS * 32 * k), id, k > 0);
             mma_commit(b_mV);
         }
         if (p_lane) {
@@ -905,20 +957,21 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                 wait(b_mO, par ^ 1u);
                 fetch(ch + 1);
             }
-            // V~ = U - P (this thread: token row, columns 32 cq .. 32 cq + 31)
+            // V~ = U - P (this thread: token row, CPT columns of the slice)
             wait(sbar, sph);
             wait(b_mV, par);
             tc_fence_after();
-            float p[32];
+            float p[CPT];
             __syncwarp();
-            tmem_ld32(tl + dbuf + 32 * cq, p);
+            tmem_ldn<CPT>(tl + dbuf + CPT * cq, p);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
+            for (int m = 0; m < CPT / 8; ++m) {
+                const int jj = CPT * cq + 8 * m;   // column within the slice
                 float u[8], y[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + st + IMG_U + off_r128(row, 32 * cq + 8 * m)), u);
+                unpack8(*reinterpret_cast<const uint4 *>(smem + st + L::U + off_u(row, jj)), u);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) y[e] = u[e] - p[8 * m + e];
-                *reinterpret_cast<uint4 *>(smem + OFF_VT + off_r128(row, 32 * cq + 8 * m)) = pack8(y);
+                *reinterpret_cast<uint4 *>(smem + L::OFF_VT + off_rn(row, jj, NS)) = pack8(y);
             }
             fence_proxy_async();
         } else {
@@ -934,15 +987,15 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         // dS = Kd^T V~ (the state's path), then O += [0 ; A_qk] V~
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id_s = idesc_bf16(128, 128, 1, 1, 0);
-            constexpr uint32_t id_o = idesc_bf16(128, 128, 0, 1, 0);
+            constexpr uint32_t id_s = idesc_bf16(128, NS, 1, 1, 0);
+            constexpr uint32_t id_o = idesc_bf16(128, NS, 0, 1, 0);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                mma_ss(tbase + TC_S, at(dMN64, st + IMG_KD + 4096 * k), at(dMN64, OFF_VT + 4096 * k), id_s, k > 0);
+                mma_ss(tbase + L::TC_S, at(dMN64, st + IMG_KD + 4096 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_s, k > 0);
             mma_commit(b_mS);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                mma_ss(tbase + dbuf, at(dK32, st + ST_ZERO + 256 * k), at(dMN64, OFF_VT + 4096 * k), id_o, 1);
+                mma_ss(tbase + dbuf, at(dK32, st + L::ZERO + 256 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_o, 1);
             mma_commit(b_mO);
         }
         // S <- diag(gC) S + dS (FP32) and its bf16 copy
@@ -950,12 +1003,12 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         wait(b_mS, par);
         tc_fence_after();
         {
-            const float gc = reinterpret_cast<const float *>(smem + st + ST_GC)[row];
-            float v[32];
+            const float gc = reinterpret_cast<const float *>(smem + st + L::GC)[row];
+            float v[CPT];
             __syncwarp();
-            tmem_ld32(tl + TC_S + 32 * cq, v);
+            tmem_ldn<CPT>(tl + L::TC_S + CPT * cq, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) S[e] = fmaf(gc, S[e], v[e]);
+            for (int e = 0; e < CPT; ++e) S[e] = fmaf(gc, S[e], v[e]);
             store_state_operand();
         }
         tc_fence_before();
@@ -967,13 +1020,13 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         if (!failed) emit(nch - 1);
     }
     if (!failed && S_T) {
-        float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + 32 * cq);
+        float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + j0 + CPT * cq);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
+        for (int m = 0; m < CPT / 4; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 512);
+    if (warp == 0) tmem_dealloc(tbase, L::TMEM_COLS);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
@@ -1037,16 +1090,46 @@ cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a,
                         PrepPrologue{(const __nv_bfloat16 *)p.conv_w, p.A, p.beta_logit}, st);
 }
 
+// Value-column slice width of the scan: the widest slice (fewest redundant record reads)
+// whose B*H*(128/NS) CTAs still fit one wave on the SMs; the output epilogue normalises whole
+// rows and keeps one slice per head.
+int scan_slice_width(int BH, bool gated) {
+    if (gated) return D;
+    const int sms = num_sms();
+    int ns = D;
+    while (ns > 16 && (long long)BH * (D / (ns / 2)) <= sms) ns /= 2;
+    return ns;
+}
+
+template <int NS, bool GATED>
+static cudaError_t launch_scan(const ChunkArgs &a, const uint8_t *ws, cudaStream_t st) {
+    using L = scan::Layout<NS>;
+    auto k = chunk_scan_tc_kernel<NS, GATED>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // programmatic dependency on the prep kernel: the scan's CTAs may start (barriers, TMEM,
+    // S0) on SMs the prep has left and wait in the kernel for its records
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.H * (D / NS)));
+    cfg.blockDim = dim3(L::NT);
+    cfg.dynamicSmemBytes = L::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, ws, a.S0, (__nv_bfloat16 *)a.out, a.S_T, a.T, a.H, a.fl.scale,
+                              (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
+}
+
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st) {
     // the plain instantiations carry none of the prologue or epilogue code
     auto prep_k = pro.conv_w ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
-    auto scan_k = a.out_gate ? chunk_scan_tc_kernel<true> : chunk_scan_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)prep::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(scan_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int nch = (a.T + C - 1) / C;
     uint8_t *ws = (uint8_t *)a.workspace;
@@ -1057,10 +1140,13 @@ static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark_launch(a, st);
-    scan_k<<<a.B * a.H, scan::NT, scan::SMEM_BYTES, st>>>(
-        ws, a.S0, (__nv_bfloat16 *)a.out, a.S_T, a.T, a.H, a.fl.scale,
-        (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
-    return cudaGetLastError();
+    if (a.out_gate) return launch_scan<D, true>(a, ws, st);
+    switch (scan_slice_width(a.B * a.H, false)) {
+        case 16: return launch_scan<16, false>(a, ws, st);
+        case 32: return launch_scan<32, false>(a, ws, st);
+        case 64: return launch_scan<64, false>(a, ws, st);
+        default: return launch_scan<D, false>(a, ws, st);
+    }
 }
 
 }  // namespace kda

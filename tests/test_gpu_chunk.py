@@ -76,6 +76,16 @@ def test_ragged_lengths(K, T, dtype):
     _check(out, S_T, _oracle(x), dtype)
 
 
+@pytest.mark.parametrize("H", [8, 12, 24, 40])
+@pytest.mark.parametrize("T", [1, 200])
+def test_split_scan_value_slices(K, H, T):
+    """The split form's scan runs each head as 128/NS value-column slices, NS picked from B*H
+    and the SM count.  On a 148-SM B200, B*H = 16, 24, 48, 80 take NS = 16, 32, 64, 128."""
+    x = W.chunk_inputs(2, T, H, 128, 128, dtype=torch.bfloat16, seed=70 + H + T)
+    out, S_T = _run(K, x, fused=False)
+    _check(out, S_T, _oracle(x), torch.bfloat16)
+
+
 @pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_head_dims(K, dk, dv, dtype):
