@@ -119,9 +119,8 @@ constexpr uint32_t E_STRIDE = 132;
 constexpr uint32_t AS = 68;
 constexpr uint32_t OFF_AKK = OFF_GAM;
 constexpr uint32_t OFF_TMF = OFF_GAM + 17408;
-constexpr uint32_t OFF_BOP = OFF_GAM + 36864;  // bf16 band-pair B operand [160][128]; later Tm' + scratch
+constexpr uint32_t OFF_BOP = OFF_GAM + 36864;  // bf16 band-pair B operand [160][128]; later Tm'
 constexpr uint32_t OFF_TMB = OFF_BOP;          // bf16 [128][64 i]: Tm' rows r, then the same rows again
-constexpr uint32_t OFF_RZ = OFF_BOP + 8192;    // fp32 inverse scratch
 constexpr uint32_t OFF_YR = OFF_BOP + 40960;   // bf16 K e^gamma [64][128]
 constexpr uint32_t OFF_TAB = OFF_YR + 16384;
 constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_GC = 14336,
@@ -157,8 +156,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float *EX = reinterpret_cast<float *>(smem + OFF_GAM);
     float *AKK = reinterpret_cast<float *>(smem + OFF_AKK);
     float *TMF = reinterpret_cast<float *>(smem + OFF_TMF);
-    float *RR = reinterpret_cast<float *>(smem + OFF_RZ);
-    float *ZZ = reinterpret_cast<float *>(smem + OFF_RZ + 2560);
     float *TOT = reinterpret_cast<float *>(smem + OFF_TAB + TAB_TOT);
     float *TF = reinterpret_cast<float *>(smem + OFF_TAB + TAB_F);
     float *TG = reinterpret_cast<float *>(smem + OFF_TAB + TAB_G);
@@ -548,99 +545,87 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_before();
             __syncthreads();
 
-            // ---- Tm = (I + A_kk)^{-1} in FP32 (16x16 diagonal blocks, then the block products)
-            if (tid < 64) {
-                const int bb = tid >> 4, jj = tid & 15;
-                float acc[16], x[16];
+            // ---- Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks, [T1 0; T21 T2]:
+            //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1}: one warp each, lane = column, the rows
+            //   swept in order in registers (x_r = delta_r - sum_{i<r} A[r][i] x_i);
+            //   Y = A21 T1;  T21 = -T2 Y;  then Tm' = Tm diag(beta) in bf16, stacked twice.
+            // TMF holds T1 (rows 0-31, columns 0-31), Y (rows 0-31, columns 32-63) and T2 (rows
+            // 32-63, columns 32-63).  AKK is zero on and above the diagonal.
+            if (warp < 2) {
+                const int base = 32 * warp;
+                float x[32];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                for (int r = 0; r < 32; ++r) x[r] = 0.f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
+                for (int r = 0; r < 32; ++r) {
+                    const float *arow = AKK + (base + r) * AS + base;
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                    for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
+                    for (int i = 0; i < r; i += 4) {   // terms at i >= r are 0 * 0
+                        const float4 av = *reinterpret_cast<const float4 *>(arow + i);
+                        s0 = fmaf(av.x, x[i], s0);
+                        s1 = fmaf(av.y, x[i + 1], s1);
+                        s2 = fmaf(av.z, x[i + 2], s2);
+                        s3 = fmaf(av.w, x[i + 3], s3);
+                    }
+                    x[r] = (r == lane ? 1.f : 0.f) - ((s0 + s1) + (s2 + s3));
                 }
 #pragma unroll
-                for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
-            }
-            __syncthreads();
-            if (tid < 128) {
-                const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-                const int bi = which ? 3 : 1, bj = which ? 2 : 0;
-                float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int k = 0; k < 16; k += 4)
-                    *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
-                    acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
-                }
-                *reinterpret_cast<float4 *>(RR + (which * 16 + rr) * 20 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            }
-            __syncthreads();
-            if (tid < 128) {
-                const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-                const int bi = which ? 3 : 1, bj = which ? 2 : 0;
-                float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int k = 0; k < 16; k += 4)
-                    *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float ak = k <= rr ? a[k] : 0.f;
-                    const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
-                    t[0] += ak * z.x; t[1] += ak * z.y; t[2] += ak * z.z; t[3] += ak * z.w;
-                }
-                *reinterpret_cast<float4 *>(TMF + (16 * bi + rr) * AS + 16 * bj + c4) = make_float4(-t[0], -t[1], -t[2], -t[3]);
+                for (int r = 0; r < 32; ++r) TMF[(base + r) * AS + base + lane] = x[r];
             }
             __syncthreads();
             {
-                // Z = A_BL X (32x32), one output pair per thread
-                const int rr = tid >> 4, c2 = (tid & 15) * 2;
-                float a[32];
+                // Y = A21 T1: warp w -> rows 2w, 2w + 1, lane = column
+                float t1[32];
 #pragma unroll
-                for (int k = 0; k < 32; k += 4)
-                    *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (32 + rr) * AS + k);
-                float z0 = 0.f, z1 = 0.f;
+                for (int i = 0; i < 32; ++i) t1[i] = TMF[i * AS + lane];
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const float2 x = *reinterpret_cast<const float2 *>(TMF + k * AS + c2);
-                    z0 += (k >= c2 ? a[k] : 0.f) * x.x;
-                    z1 += (k >= c2 + 1 ? a[k] : 0.f) * x.y;
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int r = 2 * warp + rr;
+                    const float *arow = AKK + (32 + r) * AS;
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 av = *reinterpret_cast<const float4 *>(arow + i);
+                        s0 = fmaf(av.x, t1[i], s0);
+                        s1 = fmaf(av.y, t1[i + 1], s1);
+                        s2 = fmaf(av.z, t1[i + 2], s2);
+                        s3 = fmaf(av.w, t1[i + 3], s3);
+                    }
+                    TMF[r * AS + 32 + lane] = (s0 + s1) + (s2 + s3);
                 }
-                *reinterpret_cast<float2 *>(ZZ + rr * 36 + c2) = make_float2(z0, z1);
             }
             __syncthreads();
             {
-                // lower-left block = -Y Z
-                const int rr = tid >> 4, c2 = (tid & 15) * 2;
+                // T21 = -T2 Y and the bf16 Tm' rows 2w, 2w + 1 of each half (lane = column j of
+                // each half): [T1 b | 0 ; T21 b | T2 b'], b = beta_j, b' = beta_{32+j}
                 float y[32];
 #pragma unroll
-                for (int k = 0; k < 32; k += 4)
-                    *reinterpret_cast<float4 *>(y + k) = *reinterpret_cast<const float4 *>(TMF + (32 + rr) * AS + 32 + k);
-                float t0v = 0.f, t1v = 0.f;
+                for (int i = 0; i < 32; ++i) y[i] = TMF[i * AS + 32 + lane];
+                const float b0 = BET[lane], b1 = BET[32 + lane];
+                auto put = [&](int r, int c, float v) {
+                    const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TMB + off_r64(r, c)) = hv;
+                    *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TMB + off_r64(r + 64, c)) = hv;
+                };
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const float2 z = *reinterpret_cast<const float2 *>(ZZ + k * 36 + c2);
-                    const float w = k <= rr ? y[k] : 0.f;
-                    t0v += w * z.x;
-                    t1v += w * z.y;
-                }
-                *reinterpret_cast<float2 *>(TMF + (32 + rr) * AS + c2) = make_float2(-t0v, -t1v);
-            }
-            __syncthreads();
-            {
-                const int r = tid >> 3, ig = tid & 7;
-                float y[8];
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int r = 2 * warp + rr;
+                    const float *trow = TMF + (32 + r) * AS + 32;
+                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int i = 8 * ig + e;
-                    y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 tv = *reinterpret_cast<const float4 *>(trow + i);
+                        s0 = fmaf(tv.x, y[i], s0);
+                        s1 = fmaf(tv.y, y[i + 1], s1);
+                        s2 = fmaf(tv.z, y[i + 2], s2);
+                        s3 = fmaf(tv.w, y[i + 3], s3);
+                    }
+                    put(r, lane, TMF[r * AS + lane] * b0);
+                    put(r, 32 + lane, 0.f);
+                    put(32 + r, lane, -((s0 + s1) + (s2 + s3)) * b0);
+                    put(32 + r, 32 + lane, trow[lane] * b1);
                 }
-                const uint4 pk = pack8(y);
-                *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pk;
-                *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r + 64, 8 * ig)) = pk;
                 fence_proxy_async();   // Tm' is read by the tensor cores next
             }
             __syncthreads();
