@@ -699,22 +699,29 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // The value columns of the state evolve independently (column j of S sees only v_{t,j}), so
 // the scan splits a head's dv = 128 columns into slices of NS columns, one CTA each: a slice
 // runs the same dependent chain with N = NS products and 1/(128/NS) of the per-thread work,
-// and few heads still fill the SMs.  One CTA per (b, h, slice), 128 * NS / CPT threads.
-// TMEM lane = key channel c for the state and = token row for the chunk products; thread
-// (lane, cq) owns the FP32 state row slice S[c][j0 + CPT cq .. + CPT - 1] (j0 = the slice's
-// first column).  Per chunk ch (record in stage ch & 1):
-//   [P ; O] = [W ; Q e^gamma] S          one M = 128, N = NS product into D[ch & 1]
-//   lanes 0-63:   V~ = U - P -> bf16 shared memory
-//   lanes 64-127: the outputs of chunk ch - 1 leave D[(ch - 1) & 1] (16-byte stores)
-//   dS = Kd^T V~;  O += A_qk V~          (A_qk padded with 64 zero rows to M = 128)
-//   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32, and its bf16 copy for the next product.
+// and few heads still fill the SMs.  One CTA per (b, h, slice).
+//
+// Warp roles.  4 * NS / CPT state warps: TMEM lane = key channel c for the state and = token
+// row for the chunk products; thread (lane, cq) owns the FP32 state row slice
+// S[c][j0 + CPT cq .. + CPT - 1] (j0 = the slice's first column).  One MMA warp issues every
+// tensor-core product and keeps the record ring full, so no state thread ever waits for an
+// issuing lane and the chain's hand-offs are mbarrier arrivals, not block-wide barriers.
+// Per chunk ch (record in stage ch % NSTG of a ring refilled NSTG - 1 chunks ahead):
+//   MMA warp:      [P ; O] = [W ; Q e^gamma] S         one M = 128, N = NS product into D[ch & 1]
+//   lanes 0-63:    V~ = U - P -> bf16 shared memory, then arrive on "V~ ready"
+//   lanes 64-127:  the outputs of chunk ch - 1 leave D[(ch - 1) & 1] (16-byte stores)
+//   MMA warp:      dS = Kd^T V~;  O += A_qk V~           (A_qk padded with 64 zero rows to M = 128)
+//   state warps:   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32, its bf16 copy, then arrive
+//                  on "S ready", which releases the next chunk's first product.
 namespace scan {
 // stage: [W;Qg] and Kd (the record's first 48 KB), the slice's U slabs, 8 KB of zeros, then
 // A_qk and sigma_C e^{gamma_C}
 template <int NS>
 struct Layout {
     static constexpr int CPT = NS < 32 ? NS : 32;       // state columns per thread
-    static constexpr int NT = 128 * (NS / CPT);
+    static constexpr int NSW = 4 * (NS / CPT);          // state warps
+    static constexpr int NPW = NSW / 2;                 // of which hold rows 0-63 (P, V~)
+    static constexpr int NT = 32 * NSW + 32;            // + the MMA warp
     static constexpr uint32_t HEAD = IMG_U;             // [W;Qg], Kd
     static constexpr uint32_t U = IMG_U;
     static constexpr uint32_t U_BYTES = (uint32_t)NS * 128;
@@ -723,7 +730,8 @@ struct Layout {
     static constexpr uint32_t GC = AQK + (IMG_GC - IMG_AQK);
     static constexpr uint32_t TAIL_BYTES = IMG_BYTES - IMG_AQK;   // A_qk and sigma_C e^{gamma_C}
     static constexpr uint32_t STAGE = (GC + 512 + 1023) / 1024 * 1024;
-    static constexpr uint32_t OFF_S = 2 * STAGE;                    // bf16 S [128 c][NS j]
+    static constexpr int NSTG = NS <= 32 ? 3 : 2;                   // record stages in the ring
+    static constexpr uint32_t OFF_S = NSTG * STAGE;                 // bf16 S [128 c][NS j]
     static constexpr uint32_t OFF_VT = OFF_S + 128u * NS * 2;       // bf16 V~ [64 r][NS j]
     static constexpr uint32_t SMEM_BYTES = OFF_VT + 64u * NS * 2 + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -759,9 +767,11 @@ __device__ __forceinline__ void grid_dependency_wait() {
 }
 
 struct alignas(8) ScanBars {
-    uint64_t stage[2];
-    uint64_t mV, mS, mO;
+    uint64_t stage[3];
+    uint64_t mV, mS, mO[2];    // tensor-core commits: [P;O], dS, O of D[0] / D[1]
+    uint64_t bV, bS;           // thread arrivals: V~ ready (one per P warp), S ready (one per state warp)
     uint32_t tmem_base;
+    int abort;                 // a bounded wait gave up: every other wait returns at once
 };
 
 template <int NS, bool GATED>
@@ -771,7 +781,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                      float scale, const __nv_bfloat16 *__restrict__ gate,
                      const float *__restrict__ norm_w, float norm_eps) {
     using L = scan::Layout<NS>;
-    constexpr int CPT = L::CPT, NT = L::NT, NSL = D / NS;
+    constexpr int CPT = L::CPT, NSL = D / NS;
     static_assert(!GATED || NS == D, "the output epilogue normalises whole rows: one slice per head");
     extern __shared__ uint8_t smem_raw[];
     __shared__ ScanBars sh;
@@ -781,6 +791,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool mma_warp = warp == L::NSW;
     const int quad = warp & 3, cq = warp >> 2;   // lane quadrant, column group of the slice
     const int row = quad * 32 + lane;            // TMEM lane
     const bool p_lane = row < 64;                // warp-uniform: rows of P (else of O)
@@ -788,18 +799,22 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const int j0 = sl * NS;                      // first value column of this slice
     const int nch = (T + C - 1) / C;
     const uint8_t *recs = ws + (size_t)bh * nch * IMG_BYTES;
-    const uint32_t b_mV = smem_u32(&sh.mV), b_mS = smem_u32(&sh.mS), b_mO = smem_u32(&sh.mO);
+    const uint32_t b_mV = smem_u32(&sh.mV), b_mS = smem_u32(&sh.mS);
+    const uint32_t b_bV = smem_u32(&sh.bV), b_bS = smem_u32(&sh.bS);
 
     if (tid == 0) {
-        mbar_init(smem_u32(&sh.stage[0]), 1);
-        mbar_init(smem_u32(&sh.stage[1]), 1);
+        for (int i = 0; i < L::NSTG; ++i) mbar_init(smem_u32(&sh.stage[i]), 1);
         mbar_init(b_mV, 1);
         mbar_init(b_mS, 1);
-        mbar_init(b_mO, 1);
+        mbar_init(smem_u32(&sh.mO[0]), 1);
+        mbar_init(smem_u32(&sh.mO[1]), 1);
+        mbar_init(b_bV, L::NPW);
+        mbar_init(b_bS, L::NSW);
         mbar_fence_init();
+        sh.abort = 0;
     }
     // the zero rows under each stage's A_qk
-    for (int i = tid; i < 2 * 512; i += NT)
+    for (int i = tid; i < L::NSTG * 512; i += L::NT)
         *reinterpret_cast<uint4 *>(smem + (i >> 9) * L::STAGE + L::ZERO + (i & 511) * 16) = make_uint4(0, 0, 0, 0);
     if (warp == 0) {
         tmem_alloc(smem_u32(&sh.tmem_base), L::TMEM_COLS);
@@ -817,7 +832,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint64_t dMNs = sdesc(sbase, NS * 16, 128, kSwizzleNone);   // S copy and V~: [K rows][NS]
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
     auto fetch = [&](int ch) {
-        const int s = ch & 1;
+        const int s = ch % L::NSTG;
         const uint32_t bar = smem_u32(&sh.stage[s]);
         const uint8_t *src = recs + (size_t)ch * IMG_BYTES;
         mbar_arrive_expect_tx(bar, L::HEAD + L::U_BYTES + L::TAIL_BYTES);
@@ -825,22 +840,26 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         bulk_load(sbase + s * L::STAGE + L::U, src + IMG_U + (uint32_t)sl * L::U_BYTES, L::U_BYTES, bar);
         bulk_load(sbase + s * L::STAGE + L::AQK, src + IMG_AQK, L::TAIL_BYTES, bar);
     };
-    // every thread waits on the barrier itself; a wait that gives up marks this thread, and
-    // the whole CTA leaves the loop at the next block-wide barrier (__syncthreads_or)
-    int failed = 0;
-    auto wait = [&](uint32_t bar, uint32_t phase) {
-        if (!mbar_wait_bounded(bar, phase, kWaitLimit)) {
-            failed = 1;
-            g_kda_tc2_error = 1;
+    // Bounded wait by every calling thread.  A wait that gives up raises the CTA's abort flag;
+    // every wait returns false as soon as it sees the flag, so no warp is left waiting on an
+    // arrival that will not come, and all warps leave their loops.
+    auto wait = [&](uint32_t bar, uint32_t phase) -> bool {
+        for (uint32_t i = 0; i < kWaitLimit; ++i) {
+            if (mbar_try_wait(bar, phase)) return true;
+            if (*reinterpret_cast<volatile int *>(&sh.abort)) return false;
+            if (i > 64) __nanosleep(32);
         }
+        *reinterpret_cast<volatile int *>(&sh.abort) = 1;
+        g_kda_tc2_error = 1;
+        return false;
     };
     // outputs of chunk c (O rows are TMEM lanes 64-127): this thread's token r, CPT values.
     // With the output epilogue (FusedRMSNormGated) the row's RMS is summed over the four warps
     // that hold its quarters (named barrier of the eight output warps), then
     // out = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate) leaves the chip directly.
-    if (GATED && tid < D) w_s[tid] = norm_w ? norm_w[tid] : 1.f;   // read after the first barrier
+    if (GATED && tid < D) w_s[tid] = norm_w ? norm_w[tid] : 1.f;   // read after the next barrier
     // gate rows of the chunk the next emit stores, loaded one chunk ahead (registers)
-    uint4 gpre[CPT / 8];
+    uint4 gpre[GATED ? CPT / 8 : 1];
     auto prefetch_gate = [&](int c) {
         const int r = row - 64, t0 = c * C;
         if (GATED && c < nch && t0 + r < T) {
@@ -876,6 +895,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                         o[8 * m + e] *= rr * w_s[32 * cq + 8 * m + e] * sigmoid_tanh(gv[e]);
                 }
             }
+            named_bar(1, 256);   // rms_part is rewritten by the next emit
         }
         if (t0 + r < T) {
             uint4 *dst = reinterpret_cast<uint4 *>(out + orow);
@@ -902,112 +922,129 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         fence_proxy_async();
     };
 
-    if (S0) {
-        const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + j0 + CPT * cq);
+    if (!mma_warp) {
+        if (S0) {
+            const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + j0 + CPT * cq);
 #pragma unroll
-        for (int m = 0; m < CPT / 4; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
-    } else {
+            for (int m = 0; m < CPT / 4; ++m) *reinterpret_cast<float4 *>(S + 4 * m) = src[m];
+        } else {
 #pragma unroll
-        for (int e = 0; e < CPT; ++e) S[e] = 0.f;
+            for (int e = 0; e < CPT; ++e) S[e] = 0.f;
+        }
+        store_state_operand();
     }
-    store_state_operand();
     // everything above overlaps the end of the prep kernel; the records are read from here on
     grid_dependency_wait();
-    if (tid == 0) {
-        if (nch > 0) fetch(0);
-        if (nch > 1) fetch(1);
-    }
+    if (tid == 0)
+        for (int c = 0; c < L::NSTG && c < nch; ++c) fetch(c);
+    tc_fence_before();
     __syncthreads();
 
-    for (int ch = 0; ch < nch; ++ch) {
-        const int s = ch & 1;
-        const uint32_t st = s * L::STAGE;
-        const uint32_t sbar = smem_u32(&sh.stage[s]);
-        const uint32_t sph = (uint32_t)(ch >> 1) & 1u;
-        const uint32_t dbuf = s ? L::TC_D1 : L::TC_D0;
-        const uint32_t par = (uint32_t)ch & 1u;
-        // [P ; O] = [W ; Qg] S
-        if (tid == 0) {
-            wait(sbar, sph);
+    if (mma_warp) {
+        // ---- the MMA warp: every lane waits, lane 0 issues, the warp reconverges
+        for (int ch = 0; ch < nch; ++ch) {
+            const int s = ch & 1, sg = ch % L::NSTG;
+            const uint32_t st = sg * L::STAGE;
+            const uint32_t dbuf = s ? L::TC_D1 : L::TC_D0;
+            if (ch > 0 && !wait(b_bS, (uint32_t)(ch - 1) & 1u)) break;            // S(ch) is in place
+            if (!wait(smem_u32(&sh.stage[sg]), (uint32_t)(ch / L::NSTG) & 1u)) break;
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, NS, 0, 1, 0);
+            if (lane == 0) {
+                constexpr uint32_t id = idesc_bf16(128, NS, 0, 1, 0);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_ss(tbase + dbuf, at(dK64, st + 256 * k), at(dMNs, L::OFF_S + NS * 32 * k), id, k > 0);
-            mma_commit(b_mV);
-        }
-        if (p_lane) {
-            // the stage of chunk ch - 1 is free once its last products are done: refill it
-            if (tid == 0 && ch >= 1 && ch + 1 < nch) {
-                wait(b_mO, par ^ 1u);
-                fetch(ch + 1);
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tbase + dbuf, at(dK64, st + 256 * k), at(dMNs, L::OFF_S + NS * 32 * k), id, k > 0);
+                mma_commit(b_mV);
             }
-            // V~ = U - P (this thread: token row, CPT columns of the slice)
-            wait(sbar, sph);
-            wait(b_mV, par);
-            tc_fence_after();
-            float p[CPT];
             __syncwarp();
-            tmem_ldn<CPT>(tl + dbuf + CPT * cq, p);
-#pragma unroll
-            for (int m = 0; m < CPT / 8; ++m) {
-                const int jj = CPT * cq + 8 * m;   // column within the slice
-                float u[8], y[8];
-                unpack8(*reinterpret_cast<const uint4 *>(smem + st + L::U + off_u(row, jj)), u);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) y[e] = u[e] - p[8 * m + e];
-                *reinterpret_cast<uint4 *>(smem + L::OFF_VT + off_rn(row, jj, NS)) = pack8(y);
+            // the stage of chunk ch - 1 is free once its last products are done and every state
+            // thread has passed its update (S(ch) ready): refill it
+            if (ch >= 1 && ch - 1 + L::NSTG < nch) {
+                if (!wait(smem_u32(&sh.mO[(ch - 1) & 1]), (uint32_t)((ch - 1) >> 1) & 1u)) break;
+                if (lane == 0) fetch(ch - 1 + L::NSTG);
+                __syncwarp();
             }
-            fence_proxy_async();
-        } else {
-            if (ch > 0) {
-                wait(b_mO, par ^ 1u);
+            if (!wait(b_bV, (uint32_t)ch & 1u)) break;                              // V~(ch) is in place
+            tc_fence_after();
+            if (lane == 0) {
+                // dS = Kd^T V~ (the state's path), then O += [0 ; A_qk] V~
+                constexpr uint32_t id_s = idesc_bf16(128, NS, 1, 1, 0);
+                constexpr uint32_t id_o = idesc_bf16(128, NS, 0, 1, 0);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss(tbase + L::TC_S, at(dMN64, st + IMG_KD + 4096 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_s, k > 0);
+                mma_commit(b_mS);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_ss(tbase + dbuf, at(dK32, st + L::ZERO + 256 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_o, 1);
+                mma_commit(smem_u32(&sh.mO[s]));
+            }
+            __syncwarp();
+        }
+    } else {
+        if (!p_lane) prefetch_gate(0);
+        for (int ch = 0; ch < nch; ++ch) {
+            const int s = ch & 1, sg = ch % L::NSTG;
+            const uint32_t st = sg * L::STAGE;
+            const uint32_t sbar = smem_u32(&sh.stage[sg]);
+            const uint32_t sph = (uint32_t)(ch / L::NSTG) & 1u;
+            const uint32_t dbuf = s ? L::TC_D1 : L::TC_D0;
+            if (p_lane) {
+                // V~ = U - P (this thread: token row, CPT columns of the slice)
+                if (!wait(sbar, sph) || !wait(b_mV, (uint32_t)ch & 1u)) break;
                 tc_fence_after();
-                emit(ch - 1);
+                float p[CPT];
+                __syncwarp();
+                tmem_ldn<CPT>(tl + dbuf + CPT * cq, p);
+#pragma unroll
+                for (int m = 0; m < CPT / 8; ++m) {
+                    const int jj = CPT * cq + 8 * m;   // column within the slice
+                    float u[8], y[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(smem + st + L::U + off_u(row, jj)), u);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = u[e] - p[8 * m + e];
+                    *reinterpret_cast<uint4 *>(smem + L::OFF_VT + off_rn(row, jj, NS)) = pack8(y);
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(b_bV);
+            } else if (ch > 0) {
+                // the outputs of chunk ch - 1, while this chunk's first product runs
+                const int c = ch - 1;
+                if (!wait(smem_u32(&sh.mO[c & 1]), (uint32_t)(c >> 1) & 1u)) break;
+                tc_fence_after();
+                emit(c);
+                prefetch_gate(ch);   // consumed by the next emit (chunk ch)
             }
-            prefetch_gate(ch);   // consumed by the next emit (chunk ch)
-        }
-        tc_fence_before();
-        if (__syncthreads_or(failed)) { failed = 1; break; }
-        // dS = Kd^T V~ (the state's path), then O += [0 ; A_qk] V~
-        if (tid == 0) {
+            // S <- diag(gC) S + dS (FP32) and its bf16 copy
+            if (!wait(sbar, sph) || !wait(b_mS, (uint32_t)ch & 1u)) break;
             tc_fence_after();
-            constexpr uint32_t id_s = idesc_bf16(128, NS, 1, 1, 0);
-            constexpr uint32_t id_o = idesc_bf16(128, NS, 0, 1, 0);
+            {
+                const float gc = reinterpret_cast<const float *>(smem + st + L::GC)[row];
+                float v[CPT];
+                __syncwarp();
+                tmem_ldn<CPT>(tl + L::TC_S + CPT * cq, v);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_ss(tbase + L::TC_S, at(dMN64, st + IMG_KD + 4096 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_s, k > 0);
-            mma_commit(b_mS);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_ss(tbase + dbuf, at(dK32, st + L::ZERO + 256 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_o, 1);
-            mma_commit(b_mO);
-        }
-        // S <- diag(gC) S + dS (FP32) and its bf16 copy
-        wait(sbar, sph);
-        wait(b_mS, par);
-        tc_fence_after();
-        {
-            const float gc = reinterpret_cast<const float *>(smem + st + L::GC)[row];
-            float v[CPT];
+                for (int e = 0; e < CPT; ++e) S[e] = fmaf(gc, S[e], v[e]);
+                store_state_operand();
+            }
+            tc_fence_before();
             __syncwarp();
-            tmem_ldn<CPT>(tl + L::TC_S + CPT * cq, v);
-#pragma unroll
-            for (int e = 0; e < CPT; ++e) S[e] = fmaf(gc, S[e], v[e]);
-            store_state_operand();
+            if (lane == 0) mbar_arrive(b_bS);
         }
-        tc_fence_before();
-        if (__syncthreads_or(failed)) { failed = 1; break; }
-    }
-    if (!failed && nch > 0 && !p_lane) {
-        wait(b_mO, (uint32_t)(nch - 1) & 1u);
-        tc_fence_after();
-        if (!failed) emit(nch - 1);
-    }
-    if (!failed && S_T) {
-        float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + j0 + CPT * cq);
+        if (!p_lane && nch > 0 && !*reinterpret_cast<volatile int *>(&sh.abort)) {
+            const int c = nch - 1;
+            if (wait(smem_u32(&sh.mO[c & 1]), (uint32_t)(c >> 1) & 1u)) {
+                tc_fence_after();
+                emit(c);
+            }
+        }
+        if (S_T && !*reinterpret_cast<volatile int *>(&sh.abort)) {
+            float4 *dst = reinterpret_cast<float4 *>(S_T + ((size_t)bh * D + row) * D + j0 + CPT * cq);
 #pragma unroll
-        for (int m = 0; m < CPT / 4; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
+            for (int m = 0; m < CPT / 4; ++m) dst[m] = *reinterpret_cast<const float4 *>(S + 4 * m);
+        }
     }
     tc_fence_before();
     __syncthreads();
