@@ -511,7 +511,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         if (ok) {
             tc_fence_after();
-            // ---- A_kk -> FP32 (strictly lower); A_qk goes to the record while W/U are on the tensor cores
+            // ---- A_kk -> FP32, transposed (AKK[i][r] = A_kk[r][i] for i < r, else 0); A_qk goes to
+            // the record while W/U are on the tensor cores
             auto band_rows = [&](float (&v)[16]) {
                 const int r = row & 63, band = r >> 4;
                 const int b_lo = (quad & 1) * 2;
@@ -532,43 +533,38 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float v[16];
                 band_rows(v);
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    float4 y;
-                    const int i = 16 * qq + 4 * e4;
-                    y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
-                    y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
-                    y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
-                    y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
+                for (int e = 0; e < 16; ++e) {
+                    const int i = 16 * qq + e;
+                    AKK[i * AS + r] = (i < r) ? v[e] : 0.f;   // a warp writes 32 consecutive r
                 }
             }
             tc_fence_before();
             __syncthreads();
 
             // ---- Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks, [T1 0; T21 T2]:
-            //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1}: one warp each, lane = column, the rows
-            //   swept in order in registers (x_r = delta_r - sum_{i<r} A[r][i] x_i);
+            //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1}: one warp each, lane = column; column
+            //   sweep in registers: x_i is final once the rows above it are done, then
+            //   x_r -= A[r][i] x_i for every r > i (independent updates, loads run ahead);
             //   Y = A21 T1;  T21 = -T2 Y;  then Tm' = Tm diag(beta) in bf16, stacked twice.
             // TMF holds T1 (rows 0-31, columns 0-31), Y (rows 0-31, columns 32-63) and T2 (rows
-            // 32-63, columns 32-63).  AKK is zero on and above the diagonal.
+            // 32-63, columns 32-63).  AKK holds A_kk transposed, zero on and above the diagonal.
             if (warp < 2) {
                 const int base = 32 * warp;
                 float x[32];
 #pragma unroll
-                for (int r = 0; r < 32; ++r) x[r] = 0.f;
+                for (int r = 0; r < 32; ++r) x[r] = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    const float *arow = AKK + (base + r) * AS + base;
-                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+                for (int i = 0; i < 31; ++i) {
+                    const float xi = x[i];
+                    const float *col = AKK + (base + i) * AS + base;   // A[base + r][base + i] over r
 #pragma unroll
-                    for (int i = 0; i < r; i += 4) {   // terms at i >= r are 0 * 0
-                        const float4 av = *reinterpret_cast<const float4 *>(arow + i);
-                        s0 = fmaf(av.x, x[i], s0);
-                        s1 = fmaf(av.y, x[i + 1], s1);
-                        s2 = fmaf(av.z, x[i + 2], s2);
-                        s3 = fmaf(av.w, x[i + 3], s3);
+                    for (int r4 = ((i + 1) >> 2) << 2; r4 < 32; r4 += 4) {   // rows r <= i hold 0
+                        const float4 av = *reinterpret_cast<const float4 *>(col + r4);
+                        x[r4] = fmaf(-av.x, xi, x[r4]);
+                        x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
+                        x[r4 + 2] = fmaf(-av.z, xi, x[r4 + 2]);
+                        x[r4 + 3] = fmaf(-av.w, xi, x[r4 + 3]);
                     }
-                    x[r] = (r == lane ? 1.f : 0.f) - ((s0 + s1) + (s2 + s3));
                 }
 #pragma unroll
                 for (int r = 0; r < 32; ++r) TMF[(base + r) * AS + base + lane] = x[r];
@@ -579,21 +575,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float t1[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) t1[i] = TMF[i * AS + lane];
+                const int r = 2 * warp;
+                float ya0 = 0.f, ya1 = 0.f, yb0 = 0.f, yb1 = 0.f;
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int r = 2 * warp + rr;
-                    const float *arow = AKK + (32 + r) * AS;
-                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 av = *reinterpret_cast<const float4 *>(arow + i);
-                        s0 = fmaf(av.x, t1[i], s0);
-                        s1 = fmaf(av.y, t1[i + 1], s1);
-                        s2 = fmaf(av.z, t1[i + 2], s2);
-                        s3 = fmaf(av.w, t1[i + 3], s3);
-                    }
-                    TMF[r * AS + 32 + lane] = (s0 + s1) + (s2 + s3);
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 a0 = *reinterpret_cast<const float2 *>(AKK + i * AS + 32 + r);
+                    const float2 a1 = *reinterpret_cast<const float2 *>(AKK + (i + 1) * AS + 32 + r);
+                    ya0 = fmaf(a0.x, t1[i], ya0);
+                    yb0 = fmaf(a0.y, t1[i], yb0);
+                    ya1 = fmaf(a1.x, t1[i + 1], ya1);
+                    yb1 = fmaf(a1.y, t1[i + 1], yb1);
                 }
+                TMF[r * AS + 32 + lane] = ya0 + ya1;
+                TMF[(r + 1) * AS + 32 + lane] = yb0 + yb1;
             }
             __syncthreads();
             {
