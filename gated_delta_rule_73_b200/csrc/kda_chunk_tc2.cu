@@ -93,6 +93,9 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
     u.w = pack_bf16(x[6], x[7]);
     return u;
 }
+__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
+    return make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+}
 __device__ __forceinline__ void ld8f(const float *p, float (&x)[8]) {
     *reinterpret_cast<float4 *>(x) = *reinterpret_cast<const float4 *>(p);
     *reinterpret_cast<float4 *>(x + 4) = *reinterpret_cast<const float4 *>(p + 4);
@@ -545,7 +548,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1}: one warp each, lane = column; column
             //   sweep in registers: x_i is final once the rows above it are done, then
             //   x_r -= A[r][i] x_i for every r > i (independent updates, loads run ahead);
-            //   Y = A21 T1;  T21 = -T2 Y;  then Tm' = Tm diag(beta) in bf16, stacked twice.
+            //   Y = A21 T1;  T21 = -T2 Y;  Tm' = Tm diag(beta) in bf16, stacked twice.
             // TMF holds T1 (rows 0-31, columns 0-31), Y (rows 0-31, columns 32-63) and T2 (rows
             // 32-63, columns 32-63).  AKK holds A_kk transposed, zero on and above the diagonal.
             if (warp < 2) {
@@ -570,58 +573,86 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int r = 0; r < 32; ++r) TMF[(base + r) * AS + base + lane] = x[r];
             }
             __syncthreads();
+            // Y = A21 T1 and T21 = -T2 Y as 2 x 4 register tiles (threads 0-127: row pair rg,
+            // column group cg), so a warp's loads of a row of one factor and a column group of
+            // the other are one shared-memory wavefront each.  Meanwhile threads 128-511 pack the
+            // finished blocks of Tm' = [T1 b | 0 ; . | T2 b'] (b = beta_j) to bf16, 16 bytes each.
             {
-                // Y = A21 T1: warp w -> rows 2w, 2w + 1, lane = column
-                float t1[32];
+                const int rg = tid >> 3, cg = tid & 7;
+                if (tid < 128) {
+                    float acc[2][4] = {};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) t1[i] = TMF[i * AS + lane];
-                const int r = 2 * warp;
-                float ya0 = 0.f, ya1 = 0.f, yb0 = 0.f, yb1 = 0.f;
+                    for (int i = 0; i < 32; ++i) {
+                        const float2 av = *reinterpret_cast<const float2 *>(AKK + i * AS + 32 + 2 * rg);   // A21[2rg..][i]
+                        const float4 tv = *reinterpret_cast<const float4 *>(TMF + i * AS + 4 * cg);       // T1[i][4cg..]
+                        acc[0][0] = fmaf(av.x, tv.x, acc[0][0]);
+                        acc[0][1] = fmaf(av.x, tv.y, acc[0][1]);
+                        acc[0][2] = fmaf(av.x, tv.z, acc[0][2]);
+                        acc[0][3] = fmaf(av.x, tv.w, acc[0][3]);
+                        acc[1][0] = fmaf(av.y, tv.x, acc[1][0]);
+                        acc[1][1] = fmaf(av.y, tv.y, acc[1][1]);
+                        acc[1][2] = fmaf(av.y, tv.z, acc[1][2]);
+                        acc[1][3] = fmaf(av.y, tv.w, acc[1][3]);
+                    }
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float2 a0 = *reinterpret_cast<const float2 *>(AKK + i * AS + 32 + r);
-                    const float2 a1 = *reinterpret_cast<const float2 *>(AKK + (i + 1) * AS + 32 + r);
-                    ya0 = fmaf(a0.x, t1[i], ya0);
-                    yb0 = fmaf(a0.y, t1[i], yb0);
-                    ya1 = fmaf(a1.x, t1[i + 1], ya1);
-                    yb1 = fmaf(a1.y, t1[i + 1], yb1);
+                    for (int k = 0; k < 2; ++k)
+                        *reinterpret_cast<float4 *>(TMF + (2 * rg + k) * AS + 32 + 4 * cg) =
+                            make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+                } else {
+                    // unit u: rows 0-31 x eight 8-column groups (T1 b, then zeros), then rows
+                    // 32-63 x the four groups of columns 32-63 (T2 b')
+                    const int u = tid - 128;
+                    const int r = u < 256 ? (u >> 3) : 32 + ((u - 256) >> 2);
+                    const int g = u < 256 ? (u & 7) : 4 + ((u - 256) & 3);
+                    float y[8];
+                    if (r < 32 && g >= 4) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = 0.f;
+                    } else {
+                        float t[8], bb[8];
+                        ld8f(TMF + r * AS + 8 * g, t);
+                        ld8f(BET + 8 * g, bb);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = t[e] * bb[e];
+                    }
+                    const uint4 pk = pack8(y);
+                    *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * g)) = pk;
+                    *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r + 64, 8 * g)) = pk;
                 }
-                TMF[r * AS + 32 + lane] = ya0 + ya1;
-                TMF[(r + 1) * AS + 32 + lane] = yb0 + yb1;
             }
             __syncthreads();
-            {
-                // T21 = -T2 Y and the bf16 Tm' rows 2w, 2w + 1 of each half (lane = column j of
-                // each half): [T1 b | 0 ; T21 b | T2 b'], b = beta_j, b' = beta_{32+j}
-                float y[32];
+            if (tid < 128) {
+                const int rg = tid >> 3, cg = tid & 7;
+                float acc[2][4] = {};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) y[i] = TMF[i * AS + 32 + lane];
-                const float b0 = BET[lane], b1 = BET[32 + lane];
-                auto put = [&](int r, int c, float v) {
-                    const __nv_bfloat16 hv = __float2bfloat16_rn(v);
-                    *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TMB + off_r64(r, c)) = hv;
-                    *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_TMB + off_r64(r + 64, c)) = hv;
-                };
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 ta = *reinterpret_cast<const float4 *>(TMF + (32 + 2 * rg) * AS + 32 + i);   // T2[2rg][i..]
+                    const float4 tb = *reinterpret_cast<const float4 *>(TMF + (33 + 2 * rg) * AS + 32 + i);   // T2[2rg+1][i..]
+                    const float a0[4] = {ta.x, ta.y, ta.z, ta.w}, a1[4] = {tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int r = 2 * warp + rr;
-                    const float *trow = TMF + (32 + r) * AS + 32;
-                    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 tv = *reinterpret_cast<const float4 *>(trow + i);
-                        s0 = fmaf(tv.x, y[i], s0);
-                        s1 = fmaf(tv.y, y[i + 1], s1);
-                        s2 = fmaf(tv.z, y[i + 2], s2);
-                        s3 = fmaf(tv.w, y[i + 3], s3);
+                    for (int k = 0; k < 4; ++k) {
+                        const float4 yv = *reinterpret_cast<const float4 *>(TMF + (i + k) * AS + 32 + 4 * cg);   // Y[i+k][4cg..]
+                        acc[0][0] = fmaf(a0[k], yv.x, acc[0][0]);
+                        acc[0][1] = fmaf(a0[k], yv.y, acc[0][1]);
+                        acc[0][2] = fmaf(a0[k], yv.z, acc[0][2]);
+                        acc[0][3] = fmaf(a0[k], yv.w, acc[0][3]);
+                        acc[1][0] = fmaf(a1[k], yv.x, acc[1][0]);
+                        acc[1][1] = fmaf(a1[k], yv.y, acc[1][1]);
+                        acc[1][2] = fmaf(a1[k], yv.z, acc[1][2]);
+                        acc[1][3] = fmaf(a1[k], yv.w, acc[1][3]);
                     }
-                    put(r, lane, TMF[r * AS + lane] * b0);
-                    put(r, 32 + lane, 0.f);
-                    put(32 + r, lane, -((s0 + s1) + (s2 + s3)) * b0);
-                    put(32 + r, 32 + lane, trow[lane] * b1);
                 }
-                fence_proxy_async();   // Tm' is read by the tensor cores next
+                // T21 b -> Tm' rows 32 + 2rg + k, columns 4cg .. 4cg + 3 (8 bytes, both copies)
+                const float4 bv = *reinterpret_cast<const float4 *>(BET + 4 * cg);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const float y4[4] = {-acc[k][0] * bv.x, -acc[k][1] * bv.y, -acc[k][2] * bv.z, -acc[k][3] * bv.w};
+                    const uint2 pk = pack4(y4);
+                    *reinterpret_cast<uint2 *>(smem + OFF_TMB + off_r64(32 + 2 * rg + k, 4 * cg)) = pk;
+                    *reinterpret_cast<uint2 *>(smem + OFF_TMB + off_r64(96 + 2 * rg + k, 4 * cg)) = pk;
+                }
             }
+            fence_proxy_async();   // Tm' is read by the tensor cores next
             __syncthreads();
 
             // ---- W = Tm' (K e^gamma),  U = Tm' V  (M = 128: Tm' stacked twice)
