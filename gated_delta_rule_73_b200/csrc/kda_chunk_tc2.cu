@@ -129,7 +129,13 @@ constexpr uint32_t OFF_TAB = OFF_YR + 16384;
 constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_GC = 14336,
                    TAB_NRM = 14848, TAB_BET = 15360, TAB_SGNL = 15616, TAB_BPAR = 16640,
                    TAB_PP = 16896, TAB_SGNC = 17152, TAB_BYTES = 17408;
-constexpr uint32_t SMEM_BYTES = OFF_TAB + TAB_BYTES + 1024;
+// the record leaves through shared memory by bulk stores: Q e^gamma and Kd here, A_qk in the
+// band-pair operand's region, W and U in E's, sigma_C e^{gamma_C} in the tables
+constexpr uint32_t OFF_RQG = OFF_TAB + TAB_BYTES;    // bf16 Q e^gamma, the record's layout
+constexpr uint32_t OFF_RKD = OFF_RQG + 16384;        // bf16 Kd
+constexpr uint32_t OFF_RAQ = OFF_BOP + 16384;        // bf16 A_qk (after Tm')
+constexpr uint32_t OFF_RWU = OFF_GAM;                // bf16 W, then U (16-column slabs)
+constexpr uint32_t SMEM_BYTES = OFF_RKD + 16384 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // TMEM: X [0,64), D [64,224), then W and U, each in lanes 0-63 with lanes 64-127 repeating
 // them: U [224,352), W [352,480)
@@ -266,6 +272,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                    : bpre;
         }
         bpre = load_beta(next);
+        if (tid == 0) bulk_wait_read_all();   // the previous record's sources may be rewritten
         ok = wait_all(bar_tma, li & 1u);
         if (ok && fused_pro) ok = wait_all(bar_v, li & 1u);
         if (ok && fused_pro) {
@@ -427,7 +434,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
                 const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
                 const uint32_t swc = SGNC[qq];
-                uint4 rec[4];   // this row's Q e^gamma or Kd slice of the record, stored after the fence
 #pragma unroll
                 for (int cg = 0; cg < 4; ++cg) {
                     const int c0 = 32 * qq + 8 * cg;
@@ -447,7 +453,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                              pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
                              pack_bf16(rs * xe[6], rs * xe[7]));
                     if (isq) {
-                        rec[cg] = pack8(y1);
+                        *reinterpret_cast<uint4 *>(smem + OFF_RQG + off_r128(r, c0)) = pack8(y1);
                     } else {
                         float gb[8], inv[8], y2[8];
                         ld8f(TG + band * D + c0, gb);
@@ -457,7 +463,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
                         }
                         *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
-                        rec[cg] = pack8(y2);
+                        *reinterpret_cast<uint4 *>(smem + OFF_RKD + off_r128(r, c0)) = pack8(y2);
                     }
                 }
                 // The band-pair B rows k_i e^{p_b - gamma_i} (one copy per row band b >= band(i)),
@@ -487,14 +493,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         }
                     }
                 }
-                // Each writer orders its shared-memory operands before the tensor-core reads.  The
-                // fence waits for this thread's outstanding stores, so the record's global stores
-                // come after it.
+                // each writer orders its shared-memory operands (and record parts) before the
+                // tensor-core and bulk-copy reads
                 fence_proxy_async();
-#pragma unroll
-                for (int cg = 0; cg < 4; ++cg)
-                    *reinterpret_cast<uint4 *>(img + (isq ? IMG_QG : IMG_KD) + off_r128(r, 32 * qq + 8 * cg)) = rec[cg];
-                if (tid < D) reinterpret_cast<float *>(img + IMG_GC)[tid] = TGC[tid];
             }
             tmem_wait_st();
             tc_fence_before();
@@ -509,6 +510,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int s = 0; s < 8; ++s)
                     mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
                 mma_commit(bar_mma);
+                bulk_store(img + IMG_QG, sbase + OFF_RQG, 16384);
+                bulk_store(img + IMG_KD, sbase + OFF_RKD, 16384);
+                bulk_store(img + IMG_GC, sbase + OFF_TAB + TAB_GC, 512);
+                bulk_commit();
             }
             ok = wait_all(bar_mma, 0);
         }
@@ -673,7 +678,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             __syncwarp();
             if (row < 64) {
-                // A_qk (lower with diagonal) -> the record, bf16
+                // A_qk (lower with diagonal) -> bf16 in shared memory, then the record
                 const int r = row;
                 float v[16];
                 band_rows(v);
@@ -685,11 +690,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         const int i = 16 * qq + 8 * g8 + e;
                         y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
                     }
-                    *reinterpret_cast<uint4 *>(img + IMG_AQK + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
+                    *reinterpret_cast<uint4 *>(smem + OFF_RAQ + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
                 }
+                fence_proxy_async();
             }
             ok = wait_all(bar_mma, 1);
-            if (ok && tid == 0 && next < nitems) issue_v(next);   // the v staging is free again
+            if (ok && tid == 0) {
+                if (next < nitems) issue_v(next);   // the v staging is free again
+                bulk_store(img + IMG_AQK, sbase + OFF_RAQ, 8192);
+                bulk_commit();
+            }
         }
         if (ok) {
             tc_fence_after();
@@ -705,16 +715,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
                     const int c0 = 32 * qq + 8 * g8;
-                    *reinterpret_cast<uint4 *>(img + (row < 64 ? IMG_W + off_r128(r, c0) : IMG_U + off_u(r, c0))) =
+                    *reinterpret_cast<uint4 *>(smem + OFF_RWU + (row < 64 ? off_r128(r, c0) : 16384 + off_u(r, c0))) =
                         pack8(y);
                 }
+                fence_proxy_async();
             }
         }
         // the next item rewrites TMEM and shared memory: everyone is done with this one
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (ok && tid == 0) {
+            bulk_store(img + IMG_W, sbase + OFF_RWU, 16384);
+            bulk_store(img + IMG_U, sbase + OFF_RWU + 16384, 16384);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();   // the records are complete before the scan reads them
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 512);
