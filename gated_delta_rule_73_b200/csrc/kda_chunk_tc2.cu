@@ -135,7 +135,8 @@ constexpr uint32_t OFF_RQG = OFF_TAB + TAB_BYTES;    // bf16 Q e^gamma, the reco
 constexpr uint32_t OFF_RKD = OFF_RQG + 16384;        // bf16 Kd
 constexpr uint32_t OFF_RAQ = OFF_BOP + 16384;        // bf16 A_qk (after Tm')
 constexpr uint32_t OFF_RWU = OFF_GAM;                // bf16 W, then U (16-column slabs)
-constexpr uint32_t SMEM_BYTES = OFF_RKD + 16384 + 1024;
+constexpr uint32_t OFF_CW = OFF_RKD + 16384;        // bf16 conv taps of q, k, v [3][128 c][4] (prologue)
+constexpr uint32_t SMEM_BYTES = OFF_CW + 3072 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // TMEM: X [0,64), D [64,224), then W and U, each in lanes 0-63 with lanes 64-127 repeating
 // them: U [224,352), W [352,480)
@@ -227,7 +228,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto issue_qkg = [&](int item) {
         const int ich = item % nch, ibh = item / nch;
         const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
-        mbar_arrive_expect_tx(bar_tma, 3u * tile_bytes);
+        mbar_arrive_expect_tx(bar_tma, 3u * tile_bytes + (fused_pro ? 3072u : 0u));
+        if (fused_pro) {
+            // the item's conv taps: 1 KB per branch, [c][tap] for the head's 128 channels
+#pragma unroll
+            for (int br = 0; br < 3; ++br)
+                bulk_load(sbase + OFF_CW + 1024 * br, pro.conv_w + ((size_t)br * H * D + (size_t)ih * D) * 4, 1024, bar_tma);
+        }
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             tma_load_4d(sbase + OFF_STG_Q + hf * kHalf, &tm_q, bar_tma, hf * 64, ih, it0, ib);
@@ -290,11 +297,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncthreads();
             float w[4][8];   // [tap][channel]; the gate branch needs none
             if (br < 3) {
-                const __nv_bfloat16 *wsrc = pro.conv_w + ((size_t)br * H * D + (size_t)h * D + c0) * 4;
+                const uint8_t *wsrc = smem + OFF_CW + 1024 * br + c0 * 8;   // staged with the tiles
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     float x8[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(wsrc + 8 * m), x8);
+                    unpack8(*reinterpret_cast<const uint4 *>(wsrc + 16 * m), x8);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         w[j][2 * m] = x8[j];
