@@ -16,7 +16,7 @@
 //            reference, in TMEM); the B rows of pair (b, j) are k_i e^{p_b - gamma_i}
 //            for the 16 tokens i of band j.  Every factor stays inside the bf16
 //            range because a band spans 16 tokens and g > -5 (cumulative >= -80)
-//   CUDA     Tm = (I + A_kk)^{-1} (UT transform) in FP32, 16x16 blocks
+//   CUDA     Tm = (I + A_kk)^{-1} (UT transform) in FP32, 32x32 blocks
 //   tcgen05  W^T = (K e^gamma)^T Tm'^T,  U^T = V^T Tm'^T   (Tm' = Tm diag(beta))
 //   tcgen05  V~^T = U^T - S^T W^T,  O^T = S^T (Q e^gamma)^T
 //   tcgen05  O^T += V~^T A_qk^T,  dS = (K e^{gamma_C - gamma})^T V~
@@ -60,10 +60,9 @@ constexpr uint32_t OFF_AKK = OFF_GAM;         // fp32 [64][68]
 constexpr uint32_t OFF_TMF = OFF_GAM + 17408; // fp32 [64][68]
 constexpr uint32_t OFF_VT = OFF_GAM;          // bf16 V~^T, K-major [128 j][64 r]
 constexpr uint32_t OFF_QG = OFF_GAM + 36864;  // bf16 Q e^gamma [64 r][128 c]; later O staging [64][128]
-constexpr uint32_t OFF_BOP = OFF_QG + 16384;  // bf16 band-pair B operand [160][128]; later A_qk, scratch, Tm'
+constexpr uint32_t OFF_BOP = OFF_QG + 16384;  // bf16 band-pair B operand [160][128]; later A_qk, Tm'
 constexpr uint32_t OFF_AQK = OFF_BOP;         // bf16 [64 r][64 i]
 constexpr uint32_t OFF_TMB = OFF_BOP + 8192;  // bf16 [64 r][64 i]
-constexpr uint32_t OFF_RZ = OFF_BOP + 8192;   // fp32 inverse scratch: R [2][16][20], Z [32][36]
 constexpr uint32_t OFF_YR = OFF_BOP + 40960;  // bf16 K e^gamma [64][128]; later W^T [128][64]
 constexpr uint32_t OFF_KD = OFF_YR + 16384;   // bf16 K e^{gamma_C-gamma} [64][128]
 constexpr uint32_t OFF_TAB = OFF_KD + 16384;  // tables
@@ -83,7 +82,6 @@ constexpr uint32_t SMEM_USED = OFF_TAB + TAB_BYTES;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for the 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_TMF + 64 * AS * 4 <= OFF_QG, "inverse scratch fits");
-static_assert(OFF_RZ + 7168 <= OFF_BOP + 16384, "inverse scratch fits");
 
 // The ten (row band b, column band j <= b) pairs of the 64 x 64 intra-chunk
 // matrices, as 16-column groups of one N = 160 product: pair(b, j) = P0[j] + b - j.
@@ -159,8 +157,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *EX = reinterpret_cast<float *>(smem + OFF_GAM);
     float *AKK = reinterpret_cast<float *>(smem + OFF_AKK);
     float *TMF = reinterpret_cast<float *>(smem + OFF_TMF);
-    float *RR = reinterpret_cast<float *>(smem + OFF_RZ);          // [2][16][20]
-    float *ZZ = reinterpret_cast<float *>(smem + OFF_RZ + 2560);   // [32][36]
     float *TOT = reinterpret_cast<float *>(smem + OFF_TAB + TAB_TOT);
     float *TF = reinterpret_cast<float *>(smem + OFF_TAB + TAB_F);
     float *TG = reinterpret_cast<float *>(smem + OFF_TAB + TAB_G);
@@ -449,7 +445,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         if (tid == 32 && ch + 1 < nch) issue_tma_qkg(ch + 1);
 
-        // ---- step 5: A_qk -> bf16 (lower with diagonal); A_kk -> FP32 (strictly lower).
+        // ---- step 5: A_qk -> bf16 (lower with diagonal); A_kk -> FP32 (strictly lower), transposed
+        //      (AKK[i][r] = A_kk[r][i]).
         //      A warp's 32 rows span two row bands; it reads both bands' columns for
         //      column band j = qq and each thread keeps its own.
         {
@@ -479,125 +476,110 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             } else {
 #pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    float4 y;
-                    const int i = 16 * qq + 4 * e4;
-                    y.x = (i + 0 < r) ? v[4 * e4 + 0] : 0.f;
-                    y.y = (i + 1 < r) ? v[4 * e4 + 1] : 0.f;
-                    y.z = (i + 2 < r) ? v[4 * e4 + 2] : 0.f;
-                    y.w = (i + 3 < r) ? v[4 * e4 + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(AKK + r * AS + i) = y;
+                for (int e = 0; e < 16; ++e) {
+                    const int i = 16 * qq + e;
+                    AKK[i * AS + r] = (i < r) ? v[e] : 0.f;   // a warp writes 32 consecutive r
                 }
             }
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- step 6: Tm = (I + A_kk)^{-1} in FP32
-        // (a) 16x16 diagonal blocks, one column per thread, right-looking substitution in registers
-        if (tid < 64) {
-            const int bb = tid >> 4, jj = tid & 15;
-            float acc[16], x[16];
+        // ---- step 6: Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks, [T1 0; T21 T2]:
+        //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1}: one warp each, lane = column; column sweep in
+        //   registers (x_i is final once the rows above it are done, then x_r -= A[r][i] x_i for
+        //   every r > i); Y = A21 T1;  T21 = -T2 Y;  Tm' = Tm diag(beta) -> bf16, K-major [r][i].
+        // TMF holds T1 (rows 0-31, columns 0-31), Y (rows 0-31, columns 32-63) and T2 (rows
+        // 32-63, columns 32-63).
+        if (warp < 2) {
+            const int base = 32 * warp;
+            float x[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+            for (int r = 0; r < 32; ++r) x[r] = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                x[i] = i < jj ? 0.f : (i == jj ? 1.f : -acc[i]);
+            for (int i = 0; i < 31; ++i) {
+                const float xi = x[i];
+                const float *col = AKK + (base + i) * AS + base;   // A[base + r][base + i] over r
 #pragma unroll
-                for (int r = i + 1; r < 16; ++r) acc[r] += AKK[(16 * bb + r) * AS + 16 * bb + i] * x[i];
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) TMF[(16 * bb + r) * AS + 16 * bb + jj] = x[r];
-        }
-        __syncthreads();
-        // (b) T10 = -D1 (A10 D0), T32 = -D3 (A32 D2); thread = 1 row x 4 columns
-        if (tid < 128) {
-            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
-            float a[16], acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k = 0; k < 16; k += 4)
-                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(AKK + (16 * bi + rr) * AS + 16 * bj + k);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float4 d = *reinterpret_cast<const float4 *>(TMF + (16 * bj + k) * AS + 16 * bj + c4);
-                acc[0] += a[k] * d.x; acc[1] += a[k] * d.y; acc[2] += a[k] * d.z; acc[3] += a[k] * d.w;
-            }
-            *reinterpret_cast<float4 *>(RR + (which * 16 + rr) * 20 + c4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const int which = tid >> 6, rr = (tid >> 2) & 15, c4 = (tid & 3) * 4;
-            const int bi = which ? 3 : 1, bj = which ? 2 : 0;
-            float a[16], t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int k = 0; k < 16; k += 4)
-                *reinterpret_cast<float4 *>(a + k) = *reinterpret_cast<const float4 *>(TMF + (16 * bi + rr) * AS + 16 * bi + k);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float ak = k <= rr ? a[k] : 0.f;
-                const float4 z = *reinterpret_cast<const float4 *>(RR + (which * 16 + k) * 20 + c4);
-                t[0] += ak * z.x; t[1] += ak * z.y; t[2] += ak * z.z; t[3] += ak * z.w;
-            }
-            *reinterpret_cast<float4 *>(TMF + (16 * bi + rr) * AS + 16 * bj + c4) = make_float4(-t[0], -t[1], -t[2], -t[3]);
-        }
-        __syncthreads();
-        // (c) lower-left 32x32: -Y (A_BL X) with X = Tm[0:32,0:32], Y = Tm[32:64,32:64];
-        //     thread = 2 rows x 4 columns of a 32x32 product
-        if (tid < 128) {
-            const int r2 = (tid >> 3) * 2, c4 = (tid & 7) * 4;
-            float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int k0 = 0; k0 < 32; k0 += 4) {
-                float a0[4], a1[4];
-                *reinterpret_cast<float4 *>(a0) = *reinterpret_cast<const float4 *>(AKK + (32 + r2) * AS + k0);
-                *reinterpret_cast<float4 *>(a1) = *reinterpret_cast<const float4 *>(AKK + (33 + r2) * AS + k0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const int k = k0 + kk;
-                    float4 x = *reinterpret_cast<const float4 *>(TMF + k * AS + c4);
-                    // X is lower triangular: entries above its diagonal are not stored
-                    x.x = k >= c4 + 0 ? x.x : 0.f; x.y = k >= c4 + 1 ? x.y : 0.f;
-                    x.z = k >= c4 + 2 ? x.z : 0.f; x.w = k >= c4 + 3 ? x.w : 0.f;
-                    acc[0][0] += a0[kk] * x.x; acc[0][1] += a0[kk] * x.y; acc[0][2] += a0[kk] * x.z; acc[0][3] += a0[kk] * x.w;
-                    acc[1][0] += a1[kk] * x.x; acc[1][1] += a1[kk] * x.y; acc[1][2] += a1[kk] * x.z; acc[1][3] += a1[kk] * x.w;
+                for (int r4 = ((i + 1) >> 2) << 2; r4 < 32; r4 += 4) {   // rows r <= i hold 0
+                    const float4 av = *reinterpret_cast<const float4 *>(col + r4);
+                    x[r4] = fmaf(-av.x, xi, x[r4]);
+                    x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
+                    x[r4 + 2] = fmaf(-av.z, xi, x[r4 + 2]);
+                    x[r4 + 3] = fmaf(-av.w, xi, x[r4 + 3]);
                 }
             }
-            *reinterpret_cast<float4 *>(ZZ + r2 * 36 + c4) = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
-            *reinterpret_cast<float4 *>(ZZ + (r2 + 1) * 36 + c4) = make_float4(acc[1][0], acc[1][1], acc[1][2], acc[1][3]);
+#pragma unroll
+            for (int r = 0; r < 32; ++r) TMF[(base + r) * AS + base + lane] = x[r];
         }
         __syncthreads();
-        if (tid < 128) {
-            const int r2 = (tid >> 3) * 2, c4 = (tid & 7) * 4;
-            float t[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-            for (int k0 = 0; k0 < 32; k0 += 4) {
-                float y0[4], y1[4];
-                *reinterpret_cast<float4 *>(y0) = *reinterpret_cast<const float4 *>(TMF + (32 + r2) * AS + 32 + k0);
-                *reinterpret_cast<float4 *>(y1) = *reinterpret_cast<const float4 *>(TMF + (33 + r2) * AS + 32 + k0);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const int k = k0 + kk;
-                    const float4 z = *reinterpret_cast<const float4 *>(ZZ + k * 36 + c4);
-                    const float w0 = k <= r2 ? y0[kk] : 0.f, w1 = k <= r2 + 1 ? y1[kk] : 0.f;
-                    t[0][0] += w0 * z.x; t[0][1] += w0 * z.y; t[0][2] += w0 * z.z; t[0][3] += w0 * z.w;
-                    t[1][0] += w1 * z.x; t[1][1] += w1 * z.y; t[1][2] += w1 * z.z; t[1][3] += w1 * z.w;
-                }
-            }
-            *reinterpret_cast<float4 *>(TMF + (32 + r2) * AS + c4) = make_float4(-t[0][0], -t[0][1], -t[0][2], -t[0][3]);
-            *reinterpret_cast<float4 *>(TMF + (33 + r2) * AS + c4) = make_float4(-t[1][0], -t[1][1], -t[1][2], -t[1][3]);
-        }
-        __syncthreads();
-        // (d) Tm' = Tm diag(beta) -> bf16, K-major [r][i]
+        // Y = A21 T1 and T21 = -T2 Y as 2 x 4 register tiles (threads 0-127: row pair rg, column
+        // group cg); meanwhile threads 128-511 pack [T1 b | 0 ; . | T2 b'] (b = beta_j) to bf16
         {
-            const int r = tid >> 3, ig = tid & 7;
-            float y[8];
+            const int rg = tid >> 3, cg = tid & 7;
+            if (tid < 128) {
+                float acc[2][4] = {};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int i = 8 * ig + e;
-                y[e] = (i <= r) ? TMF[r * AS + i] * BET[i] : 0.f;
+                for (int i = 0; i < 32; ++i) {
+                    const float2 av = *reinterpret_cast<const float2 *>(AKK + i * AS + 32 + 2 * rg);   // A21[2rg..][i]
+                    const float4 tv = *reinterpret_cast<const float4 *>(TMF + i * AS + 4 * cg);       // T1[i][4cg..]
+                    acc[0][0] = fmaf(av.x, tv.x, acc[0][0]);
+                    acc[0][1] = fmaf(av.x, tv.y, acc[0][1]);
+                    acc[0][2] = fmaf(av.x, tv.z, acc[0][2]);
+                    acc[0][3] = fmaf(av.x, tv.w, acc[0][3]);
+                    acc[1][0] = fmaf(av.y, tv.x, acc[1][0]);
+                    acc[1][1] = fmaf(av.y, tv.y, acc[1][1]);
+                    acc[1][2] = fmaf(av.y, tv.z, acc[1][2]);
+                    acc[1][3] = fmaf(av.y, tv.w, acc[1][3]);
+                }
+#pragma unroll
+                for (int k = 0; k < 2; ++k)
+                    *reinterpret_cast<float4 *>(TMF + (2 * rg + k) * AS + 32 + 4 * cg) =
+                        make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+            } else {
+                const int u = tid - 128;
+                const int r = u < 256 ? (u >> 3) : 32 + ((u - 256) >> 2);
+                const int g = u < 256 ? (u & 7) : 4 + ((u - 256) & 3);
+                float y[8];
+                if (r < 32 && g >= 4) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = 0.f;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = TMF[r * AS + 8 * g + e] * BET[8 * g + e];
+                }
+                *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * g)) = pack8(y);
             }
-            *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * ig)) = pack8(y);
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int rg = tid >> 3, cg = tid & 7;
+            float acc[2][4] = {};
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 ta = *reinterpret_cast<const float4 *>(TMF + (32 + 2 * rg) * AS + 32 + i);   // T2[2rg][i..]
+                const float4 tb = *reinterpret_cast<const float4 *>(TMF + (33 + 2 * rg) * AS + 32 + i);   // T2[2rg+1][i..]
+                const float a0[4] = {ta.x, ta.y, ta.z, ta.w}, a1[4] = {tb.x, tb.y, tb.z, tb.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 yv = *reinterpret_cast<const float4 *>(TMF + (i + k) * AS + 32 + 4 * cg);   // Y[i+k][4cg..]
+                    acc[0][0] = fmaf(a0[k], yv.x, acc[0][0]);
+                    acc[0][1] = fmaf(a0[k], yv.y, acc[0][1]);
+                    acc[0][2] = fmaf(a0[k], yv.z, acc[0][2]);
+                    acc[0][3] = fmaf(a0[k], yv.w, acc[0][3]);
+                    acc[1][0] = fmaf(a1[k], yv.x, acc[1][0]);
+                    acc[1][1] = fmaf(a1[k], yv.y, acc[1][1]);
+                    acc[1][2] = fmaf(a1[k], yv.z, acc[1][2]);
+                    acc[1][3] = fmaf(a1[k], yv.w, acc[1][3]);
+                }
+            }
+            // T21 b -> Tm' rows 32 + 2rg + k, columns 4cg .. 4cg + 3 (8 bytes)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint32_t lo = pack_bf16(-acc[k][0] * BET[4 * cg], -acc[k][1] * BET[4 * cg + 1]);
+                const uint32_t hi = pack_bf16(-acc[k][2] * BET[4 * cg + 2], -acc[k][3] * BET[4 * cg + 3]);
+                *reinterpret_cast<uint2 *>(smem + OFF_TMB + off_r64(32 + 2 * rg + k, 4 * cg)) = make_uint2(lo, hi);
+            }
         }
         __syncthreads();
 
