@@ -557,23 +557,27 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             __syncthreads();
 
             // ---- Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks, [T1 0; T21 T2]:
-            //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1}: one warp each, lane = column; column
-            //   sweep in registers: x_i is final once the rows above it are done, then
-            //   x_r -= A[r][i] x_i for every r > i (independent updates, loads run ahead);
+            //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1} from their 16 x 16 diagonal blocks (column
+            //   sweeps in registers: x_i is final once the rows above it are done, then
+            //   x_r -= A[r][i] x_i for every r > i) and X = -D1 (A10 D0) below them;
             //   Y = A21 T1;  T21 = -T2 Y;  Tm' = Tm diag(beta) in bf16, stacked twice.
             // TMF holds T1 (rows 0-31, columns 0-31), Y (rows 0-31, columns 32-63) and T2 (rows
             // 32-63, columns 32-63).  AKK holds A_kk transposed, zero on and above the diagonal.
+            // T1 and T2 from their 16 x 16 diagonal blocks: D_b = (I + A_bb)^{-1} by a column sweep
+            // (lane = column, two blocks per warp); then, for each 32-block, Z = A10 D0 and
+            // X = -D1 Z (its lower-left quarter), one output per thread, Z in the columns Y takes
+            // later.  The upper-right quarters are zero.
             if (warp < 2) {
-                const int base = 32 * warp;
-                float x[32];
+                const int blk = 2 * warp + (lane >> 4), base = 16 * blk, j = lane & 15;
+                float x[16];
 #pragma unroll
-                for (int r = 0; r < 32; ++r) x[r] = (r == lane) ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int i = 0; i < 31; ++i) {
+                for (int i = 0; i < 15; ++i) {
                     const float xi = x[i];
                     const float *col = AKK + (base + i) * AS + base;   // A[base + r][base + i] over r
 #pragma unroll
-                    for (int r4 = ((i + 1) >> 2) << 2; r4 < 32; r4 += 4) {   // rows r <= i hold 0
+                    for (int r4 = ((i + 1) >> 2) << 2; r4 < 16; r4 += 4) {   // rows r <= i hold 0
                         const float4 av = *reinterpret_cast<const float4 *>(col + r4);
                         x[r4] = fmaf(-av.x, xi, x[r4]);
                         x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
@@ -582,7 +586,36 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
 #pragma unroll
-                for (int r = 0; r < 32; ++r) TMF[(base + r) * AS + base + lane] = x[r];
+                for (int r = 0; r < 16; ++r) TMF[(base + r) * AS + base + j] = x[r];
+                if ((blk & 1) == 0) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) TMF[(base + r) * AS + base + 16 + j] = 0.f;
+                }
+            }
+            __syncthreads();
+            {
+                // Z = A10 D0 (per 32-block h = tid / 256): row r, column j of the 16 x 16 product
+                const int hb = tid >> 8, r = (tid >> 4) & 15, j = tid & 15, base = 32 * hb;
+                float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) {
+                    z0 = fmaf(AKK[(base + k) * AS + base + 16 + r], TMF[(base + k) * AS + base + j], z0);
+                    z1 = fmaf(AKK[(base + k + 1) * AS + base + 16 + r], TMF[(base + k + 1) * AS + base + j], z1);
+                }
+                TMF[r * AS + 32 + 16 * hb + j] = z0 + z1;
+            }
+            __syncthreads();
+            {
+                // X = -D1 Z -> rows 16-31 of the 32-block, columns 0-15
+                const int hb = tid >> 8, r = (tid >> 4) & 15, j = tid & 15, base = 32 * hb;
+                const float *d1 = TMF + (base + 16 + r) * AS + base + 16;
+                float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; k += 2) {
+                    x0 = fmaf(d1[k], TMF[k * AS + 32 + 16 * hb + j], x0);
+                    x1 = fmaf(d1[k + 1], TMF[(k + 1) * AS + 32 + 16 * hb + j], x1);
+                }
+                TMF[(base + 16 + r) * AS + base + j] = -(x0 + x1);
             }
             __syncthreads();
             // Y = A21 T1 and T21 = -T2 Y as 2 x 4 register tiles (threads 0-127: row pair rg,
