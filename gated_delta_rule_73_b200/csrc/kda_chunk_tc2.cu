@@ -151,12 +151,15 @@ struct PrepPrologue {
     const float *b_logit;          // [B, T, H] beta logits (FP32)
 };
 
-template <bool PRO>
-__global__ void __launch_bounds__(prep::NT, 1)
-chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                  const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                  int BH, KernelFlags fl, PrepPrologue pro) {
+// The prep's work, run by CTA `cta` of `ncta` prep CTAs.  MEGA (the fused prep + scan launch of
+// few-head calls): items are taken chunk-major, so every head's early chunks come first, and
+// each finished record is published by a release of flags[item] once its bulk stores are
+// complete.  Otherwise items are taken chunk-fastest and the scan runs as the next kernel.
+template <bool PRO, bool MEGA>
+__device__ __forceinline__ void
+prep_body(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap *ptm_v,
+          const CUtensorMap *ptm_g, const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T,
+          int H, int BH, KernelFlags fl, PrepPrologue pro, int cta, int ncta, int *__restrict__ flags) {
     using namespace prep;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Bars sh;
@@ -225,8 +228,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     constexpr bool fused_pro = PRO;
     const int rows = fused_pro ? C + kHalo : C, row0 = fused_pro ? -kHalo : 0;
     const uint32_t tile_bytes = (uint32_t)rows * D * 2u;
+    // item -> (chunk, b * H + h)
+    auto item_ch = [&](int item) { return MEGA ? item / BH : item % nch; };
+    auto item_bh = [&](int item) { return MEGA ? item % BH : item / nch; };
     auto issue_qkg = [&](int item) {
-        const int ich = item % nch, ibh = item / nch;
+        const int ich = item_ch(item), ibh = item_bh(item);
         const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
         mbar_arrive_expect_tx(bar_tma, 3u * tile_bytes + (fused_pro ? 3072u : 0u));
         if (fused_pro) {
@@ -237,40 +243,49 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(sbase + OFF_STG_Q + hf * kHalf, &tm_q, bar_tma, hf * 64, ih, it0, ib);
-            tma_load_4d(sbase + OFF_STG_K + hf * kHalf, &tm_k, bar_tma, hf * 64, ih, it0, ib);
-            tma_load_4d(sbase + OFF_STG_G + hf * kHalf, &tm_g, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_Q + hf * kHalf, ptm_q, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_K + hf * kHalf, ptm_k, bar_tma, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_G + hf * kHalf, ptm_g, bar_tma, hf * 64, ih, it0, ib);
         }
     };
     auto issue_v = [&](int item) {
-        const int ich = item % nch, ibh = item / nch;
+        const int ich = item_ch(item), ibh = item_bh(item);
         const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
         mbar_arrive_expect_tx(bar_v, tile_bytes);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + OFF_STG_V + hf * kHalf, &tm_v, bar_v, hf * 64, ih, it0, ib);
+            tma_load_4d(sbase + OFF_STG_V + hf * kHalf, ptm_v, bar_v, hf * 64, ih, it0, ib);
     };
-    if (tid == 0 && (int)blockIdx.x < nitems) {
-        issue_qkg(blockIdx.x);
-        issue_v(blockIdx.x);
+    if (tid == 0 && cta < nitems) {
+        issue_qkg(cta);
+        issue_v(cta);
     }
     // beta (with the fused prologue: its logit) of token row tid < C of an item, loaded one
     // item ahead so its global-memory latency overlaps the current item
     auto load_beta = [&](int it) -> float {
         if (tid >= C || it >= nitems) return 0.f;
-        const int ich = it % nch, ibh = it / nch;
+        const int ich = item_ch(it), ibh = item_bh(it);
         const int t = ich * C + tid;
         if (t >= T) return 0.f;
         const size_t bth = ((size_t)(ibh / H) * T + t) * H + ibh % H;
         return fused_pro ? pro.b_logit[bth] : __bfloat162float(beta[bth]);
     };
-    float bpre = load_beta(blockIdx.x);
+    float bpre = load_beta(cta);
     bool ok = true;
     uint32_t li = 0;   // items done by this CTA: parity of the TMA barriers
-    for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
-        const int ch = item % nch, bh = item / nch, h = bh % H;
+    int done = -1;     // the item whose record is published next (MEGA)
+    // MEGA: the previous record's bulk stores are complete; publish it
+    auto publish = [&]() {
+        bulk_wait_all();
+        if (done >= 0) {
+            fence_proxy_async_global();
+            flag_release(flags + done, 1);
+        }
+    };
+    for (int item = cta; item < nitems && ok; item += ncta, ++li) {
+        const int ch = item_ch(item), bh = item_bh(item), h = bh % H;
         const int t0 = ch * C, n = min(C, T - t0);
-        const int next = item + (int)gridDim.x;
+        const int next = item + ncta;
         uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
         if (tid < C) {
             // the fused prologue rounds beta to bf16 like the standalone prologue kernel
@@ -279,7 +294,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                    : bpre;
         }
         bpre = load_beta(next);
-        if (tid == 0) bulk_wait_read_all();   // the previous record's sources may be rewritten
+        if (tid == 0) {
+            if (MEGA) publish();          // (also: its sources may be rewritten)
+            else bulk_wait_read_all();    // the previous record's sources may be rewritten
+        }
         ok = wait_all(bar_tma, li & 1u);
         if (ok && fused_pro) ok = wait_all(bar_v, li & 1u);
         if (ok && fused_pro) {
@@ -769,12 +787,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             bulk_store(img + IMG_W, sbase + OFF_RWU, 16384);
             bulk_store(img + IMG_U, sbase + OFF_RWU + 16384, 16384);
             bulk_commit();
+            done = item;
         }
     }
-    if (tid == 0) bulk_wait_all();   // the records are complete before the scan reads them
+    if (tid == 0) {
+        if (MEGA) publish();
+        else bulk_wait_all();   // the records are complete before the scan reads them
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+template <bool PRO>
+__global__ void __launch_bounds__(prep::NT, 1)
+chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                  const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
+                  int BH, KernelFlags fl, PrepPrologue pro) {
+    prep_body<PRO, false>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x,
+                          (int)gridDim.x, nullptr);
 }
 
 // ============================================================== kernel 2: the scan
@@ -856,12 +888,15 @@ struct alignas(8) ScanBars {
     int abort;                 // a bounded wait gave up: every other wait returns at once
 };
 
-template <int NS, bool GATED>
-__global__ void __launch_bounds__(scan::Layout<NS>::NT, 1)
-chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
-                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
-                     float scale, const __nv_bfloat16 *__restrict__ gate,
-                     const float *__restrict__ norm_w, float norm_eps) {
+// The scan's work for slice CTA `cta`.  MEGA (run beside the prep in one launch): each record is
+// fetched only after the prep has published it (flags, chunk-major), and the CTA may have more
+// threads than the scan's warps: those warps only join the block-wide barriers.
+template <int NS, bool GATED, bool MEGA>
+__device__ __forceinline__ void
+scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
+          float *__restrict__ S_T, int T, int H, float scale, const __nv_bfloat16 *__restrict__ gate,
+          const float *__restrict__ norm_w, float norm_eps, int cta, const int *__restrict__ flags,
+          int nseq) {
     using L = scan::Layout<NS>;
     constexpr int CPT = L::CPT, NSL = D / NS;
     static_assert(!GATED || NS == D, "the output epilogue normalises whole rows: one slice per head");
@@ -874,10 +909,11 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool mma_warp = warp == L::NSW;
+    const bool state_warp = warp < L::NSW;       // (warps past the MMA warp: MEGA only, idle)
     const int quad = warp & 3, cq = warp >> 2;   // lane quadrant, column group of the slice
     const int row = quad * 32 + lane;            // TMEM lane
     const bool p_lane = row < 64;                // warp-uniform: rows of P (else of O)
-    const int bh = blockIdx.x / NSL, sl = blockIdx.x % NSL, b = bh / H, h = bh % H;
+    const int bh = cta / NSL, sl = cta % NSL, b = bh / H, h = bh % H;
     const int j0 = sl * NS;                      // first value column of this slice
     const int nch = (T + C - 1) / C;
     const uint8_t *recs = ws + (size_t)bh * nch * IMG_BYTES;
@@ -896,7 +932,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         sh.abort = 0;
     }
     // the zero rows under each stage's A_qk
-    for (int i = tid; i < L::NSTG * 512; i += L::NT)
+    for (int i = tid; i < L::NSTG * 512; i += (int)blockDim.x)
         *reinterpret_cast<uint4 *>(smem + (i >> 9) * L::STAGE + L::ZERO + (i & 511) * 16) = make_uint4(0, 0, 0, 0);
     if (warp == 0) {
         tmem_alloc(smem_u32(&sh.tmem_base), L::TMEM_COLS);
@@ -913,7 +949,25 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
     const uint64_t dMNs = sdesc(sbase, NS * 16, 128, kSwizzleNone);   // S copy and V~: [K rows][NS]
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
+    // MEGA: the record of chunk ch is read once the prep has published it (bounded wait; a
+    // wait that gives up raises the abort flag and skips the copy)
+    auto published = [&](int ch) -> bool {
+        if (!MEGA) return true;
+        const int *f = flags + (size_t)ch * (size_t)nseq + bh;   // item (chunk, sequence), chunk-major
+        for (uint32_t i = 0; i < kWaitLimit; ++i) {
+            if (flag_acquire(f)) {
+                fence_proxy_async_global();
+                return true;
+            }
+            if (*reinterpret_cast<volatile int *>(&sh.abort)) return false;
+            __nanosleep(64);
+        }
+        *reinterpret_cast<volatile int *>(&sh.abort) = 1;
+        g_kda_tc2_error = 1;
+        return false;
+    };
     auto fetch = [&](int ch) {
+        if (!published(ch)) return;
         const int s = ch % L::NSTG;
         const uint32_t bar = smem_u32(&sh.stage[s]);
         const uint8_t *src = recs + (size_t)ch * IMG_BYTES;
@@ -1004,7 +1058,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         fence_proxy_async();
     };
 
-    if (!mma_warp) {
+    if (state_warp) {
         if (S0) {
             const float4 *src = reinterpret_cast<const float4 *>(S0 + ((size_t)bh * D + row) * D + j0 + CPT * cq);
 #pragma unroll
@@ -1016,7 +1070,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
         store_state_operand();
     }
     // everything above overlaps the end of the prep kernel; the records are read from here on
-    grid_dependency_wait();
+    if (!MEGA) grid_dependency_wait();
     if (tid == 0)
         for (int c = 0; c < L::NSTG && c < nch; ++c) fetch(c);
     tc_fence_before();
@@ -1063,7 +1117,7 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
             }
             __syncwarp();
         }
-    } else {
+    } else if (state_warp) {
         if (!p_lane) prefetch_gate(0);
         for (int ch = 0; ch < nch; ++ch) {
             const int s = ch & 1, sg = ch % L::NSTG;
@@ -1133,6 +1187,42 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
     if (warp == 0) tmem_dealloc(tbase, L::TMEM_COLS);
 }
 
+template <int NS, bool GATED>
+__global__ void __launch_bounds__(scan::Layout<NS>::NT, 1)
+chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
+                     __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int T, int H,
+                     float scale, const __nv_bfloat16 *__restrict__ gate,
+                     const float *__restrict__ norm_w, float norm_eps) {
+    scan_body<NS, GATED, false>(ws, S0, out, S_T, T, H, scale, gate, norm_w, norm_eps, (int)blockIdx.x,
+                                nullptr, 0);
+}
+
+// One launch for few-head calls: CTAs [0, n_scan) run the scan's slice CTAs, the rest the prep,
+// all resident at once (a cooperative launch), the scan reading each record as soon as the
+// prep has published it.  The block has the prep's 512 threads; a scan CTA uses its first
+// 32 * (NSW + 1).
+// dynamic shared memory of the one-launch form: the larger of the two roles' layouts
+template <int NS>
+constexpr uint32_t mega_smem_bytes() {
+    return prep::SMEM_BYTES > scan::Layout<NS>::SMEM_BYTES ? prep::SMEM_BYTES : scan::Layout<NS>::SMEM_BYTES;
+}
+
+template <bool PRO, int NS>
+__global__ void __launch_bounds__(prep::NT, 1)
+chunk_mega_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                  const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
+                  int BH, KernelFlags fl, PrepPrologue pro, const float *__restrict__ S0,
+                  __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int n_scan,
+                  int *__restrict__ flags) {
+    if ((int)blockIdx.x < n_scan)
+        scan_body<NS, false, true>(ws, S0, out, S_T, T, H, fl.scale, nullptr, nullptr, 0.f, (int)blockIdx.x,
+                                   flags, BH);
+    else
+        prep_body<PRO, true>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro,
+                             (int)blockIdx.x - n_scan, (int)gridDim.x - n_scan, flags);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -1168,8 +1258,8 @@ static int num_sms() {
 }
 
 size_t chunk_tc2_workspace_bytes(int B, int T, int H) {
-    const size_t nch = ((size_t)T + C - 1) / C;
-    return nch * (size_t)B * (size_t)H * IMG_BYTES;
+    const size_t nch = ((size_t)T + C - 1) / C, items = nch * (size_t)B * (size_t)H;
+    return items * IMG_BYTES + (items * sizeof(int) + 255) / 256 * 256;   // records, then one flag per record
 }
 
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
@@ -1227,9 +1317,75 @@ static cudaError_t launch_scan(const ChunkArgs &a, const uint8_t *ws, cudaStream
                               (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
 }
 
+// Per-(chunk, head) prep cost and per-chunk scan chain at d = 128 on a B200 SM (cycles, measured).
+constexpr double kPrepItemCycles = 21000.0;
+static double scan_chunk_cycles(int ns) { return ns == 16 ? 2900.0 : ns == 32 ? 3000.0 : ns == 64 ? 3100.0 : 4900.0; }
+
+// Slice width of the one-launch form (prep and scan CTAs side by side), or 0 when the two
+// launches are faster: prep on all SMs, then the scan, against the prep on the SMs the scan's
+// CTAs leave, overlapped with the scan, plus one item of ramp.
+int mega_slice_width(int BH, int nch, int sms) {
+    const double items = (double)BH * nch;
+    const double two = ceil(items / sms) * kPrepItemCycles + nch * scan_chunk_cycles(scan_slice_width(BH, false));
+    int best = 0;
+    double best_t = 0.9 * two;
+    for (int ns : {32, 64}) {
+        const int n_scan = BH * (D / ns);
+        if (n_scan > sms / 2) continue;
+        const double t = fmax(ceil(items / (sms - n_scan)) * kPrepItemCycles, nch * scan_chunk_cycles(ns)) + kPrepItemCycles;
+        if (t < best_t) {
+            best = ns;
+            best_t = t;
+        }
+    }
+    return best;
+}
+
+template <bool PRO, int NS>
+static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                               const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, cudaStream_t st) {
+    auto k = chunk_mega_kernel<PRO, NS>;
+    constexpr uint32_t smem = mega_smem_bytes<NS>();
+    static_assert(smem <= 232448, "shared memory budget");
+    static_assert(scan::Layout<NS>::NT <= prep::NT, "the scan's warps fit the prep's block");
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int nch = (a.T + C - 1) / C, BH = a.B * a.H, n_scan = BH * (D / NS);
+    uint8_t *ws = (uint8_t *)a.workspace;
+    int *flags = reinterpret_cast<int *>(ws + (size_t)nch * BH * IMG_BYTES);
+    e = cudaMemsetAsync(flags, 0, (size_t)nch * BH * sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    // every CTA resident at once (the scan CTAs wait for records the prep CTAs publish)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)num_sms());
+    cfg.blockDim = dim3(prep::NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    mark_launch(a, st);
+    return cudaLaunchKernelEx(&cfg, k, mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, BH, a.fl, pro,
+                              a.S0, (__nv_bfloat16 *)a.out, a.S_T, n_scan, flags);
+}
+
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st) {
+    if (!a.out_gate) {
+        const int ns = mega_slice_width(a.B * a.H, (a.T + C - 1) / C, num_sms());
+        if (ns) {
+            const bool p = pro.conv_w != nullptr;
+            cudaError_t e = ns == 32 ? (p ? launch_mega<true, 32>(a, mq, mk, mv, mg, pro, st)
+                                          : launch_mega<false, 32>(a, mq, mk, mv, mg, pro, st))
+                                     : (p ? launch_mega<true, 64>(a, mq, mk, mv, mg, pro, st)
+                                          : launch_mega<false, 64>(a, mq, mk, mv, mg, pro, st));
+            if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+            (void)cudaGetLastError();   // not enough room to co-schedule: the two launches below
+        }
+    }
     // the plain instantiations carry none of the prologue or epilogue code
     auto prep_k = pro.conv_w ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -86,6 +86,17 @@ def test_split_scan_value_slices(K, H, T):
     _check(out, S_T, _oracle(x), torch.bfloat16)
 
 
+@pytest.mark.parametrize("complex_gate", [False, True])
+@pytest.mark.parametrize("B,T,H", [(1, 2048, 8), (1, 4096, 16)], ids=["ns32", "ns64"])
+def test_one_launch_form(K, B, T, H, complex_gate):
+    """Few long sequences run prep and scan CTAs side by side in one cooperative launch, the
+    scan reading each record once the prep has published it.  On a 148-SM B200 these shapes
+    take slice widths 32 (8 heads) and 64 (16 heads); every output is checked."""
+    x = W.chunk_inputs(B, T, H, 128, 128, dtype=torch.bfloat16, seed=80 + H, complex_gate=complex_gate)
+    out, S_T = _run(K, x, complex_gate=complex_gate, fused=False)
+    _check(out, S_T, _oracle(x, complex_gate=complex_gate), torch.bfloat16)
+
+
 @pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_head_dims(K, dk, dv, dtype):

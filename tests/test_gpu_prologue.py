@@ -68,6 +68,16 @@ def test_prologue_tensor_core(K, T, fused):
     assert rel_err(f64(S_T), ref[1]) <= 2e-2
 
 
+def test_prologue_one_launch_form(K):
+    """Few long sequences (B=1, T=2048, H=8): the prologue inside the prep of the one-launch
+    form, whose prep CTAs take items chunk-major."""
+    x = W.prologue_inputs(1, 2048, 8, 128, 128, dtype=torch.bfloat16, seed=90)
+    out, S_T = _run(K, x, fused=False)
+    ref = _oracle_heads(x, range(8))
+    assert rel_err(f64(out), ref[0]) <= 2e-2
+    assert rel_err(f64(S_T), ref[1]) <= 2e-2
+
+
 def test_sweep_T2048_full(K):
     """length-sweep workload, T = 2048, B=1, H=96, d=128: every head."""
     x = W.sweep_inputs(2048)
