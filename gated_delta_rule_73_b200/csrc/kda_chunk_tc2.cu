@@ -886,11 +886,13 @@ struct alignas(8) ScanBars {
     uint64_t bV, bS;           // thread arrivals: V~ ready (one per P warp), S ready (one per state warp)
     uint32_t tmem_base;
     int abort;                 // a bounded wait gave up: every other wait returns at once
+    int pub;                   // MEGA: records of chunks [0, pub) are published (the loader warp)
 };
 
 // The scan's work for slice CTA `cta`.  MEGA (run beside the prep in one launch): each record is
-// fetched only after the prep has published it (flags, chunk-major), and the CTA may have more
-// threads than the scan's warps: those warps only join the block-wide barriers.
+// fetched only after the prep has published it (flags, chunk-major).  The warp after the MMA
+// warp watches the flags in chunk order and advances a shared counter, so the MMA warp's refills
+// wait on shared memory only; any further warps only join the block-wide barriers.
 template <int NS, bool GATED, bool MEGA>
 __device__ __forceinline__ void
 scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
@@ -909,7 +911,8 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool mma_warp = warp == L::NSW;
-    const bool state_warp = warp < L::NSW;       // (warps past the MMA warp: MEGA only, idle)
+    const bool state_warp = warp < L::NSW;
+    const bool load_warp = MEGA && warp == L::NSW + 1;   // (later warps: MEGA only, idle)
     const int quad = warp & 3, cq = warp >> 2;   // lane quadrant, column group of the slice
     const int row = quad * 32 + lane;            // TMEM lane
     const bool p_lane = row < 64;                // warp-uniform: rows of P (else of O)
@@ -930,6 +933,7 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
         mbar_init(b_bS, L::NSW);
         mbar_fence_init();
         sh.abort = 0;
+        sh.pub = 0;
     }
     // the zero rows under each stage's A_qk
     for (int i = tid; i < L::NSTG * 512; i += (int)blockDim.x)
@@ -949,18 +953,18 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
     const uint64_t dMNs = sdesc(sbase, NS * 16, 128, kSwizzleNone);   // S copy and V~: [K rows][NS]
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
-    // MEGA: the record of chunk ch is read once the prep has published it (bounded wait; a
-    // wait that gives up raises the abort flag and skips the copy)
+    // MEGA: the record of chunk ch is read once the loader warp has seen it published (bounded
+    // wait; a wait that gives up raises the abort flag and skips the copy)
+    const uint32_t a_pub = smem_u32(&sh.pub);
     auto published = [&](int ch) -> bool {
         if (!MEGA) return true;
-        const int *f = flags + (size_t)ch * (size_t)nseq + bh;   // item (chunk, sequence), chunk-major
         for (uint32_t i = 0; i < kWaitLimit; ++i) {
-            if (flag_acquire(f)) {
-                fence_proxy_async_global();
+            if (smem_acquire_load(a_pub) > ch) {
+                fence_proxy_async_global();   // the bulk copies that follow read what the prep wrote
                 return true;
             }
             if (*reinterpret_cast<volatile int *>(&sh.abort)) return false;
-            __nanosleep(64);
+            if (i > 64) __nanosleep(32);
         }
         *reinterpret_cast<volatile int *>(&sh.abort) = 1;
         g_kda_tc2_error = 1;
@@ -1071,12 +1075,40 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     }
     // everything above overlaps the end of the prep kernel; the records are read from here on
     if (!MEGA) grid_dependency_wait();
-    if (tid == 0)
+    if (!MEGA && tid == 0)
         for (int c = 0; c < L::NSTG && c < nch; ++c) fetch(c);
     tc_fence_before();
     __syncthreads();
 
-    if (mma_warp) {
+    if (load_warp) {
+        // MEGA: the flags of this sequence's records, in chunk order (item = chunk * nseq + bh)
+        if (lane == 0) {
+            for (int c = 0; c < nch; ++c) {
+                const int *f = flags + (size_t)c * (size_t)nseq + bh;
+                bool seen = false;
+                for (uint32_t i = 0; i < kWaitLimit; ++i) {
+                    if (flag_acquire(f)) {
+                        seen = true;
+                        break;
+                    }
+                    if (*reinterpret_cast<volatile int *>(&sh.abort)) break;
+                    __nanosleep(64);
+                }
+                if (!seen) {
+                    *reinterpret_cast<volatile int *>(&sh.abort) = 1;
+                    g_kda_tc2_error = 1;
+                    break;
+                }
+                smem_release_store(a_pub, c + 1);
+            }
+        }
+        __syncwarp();
+    } else if (mma_warp) {
+        if (MEGA) {
+            if (lane == 0)
+                for (int c = 0; c < L::NSTG && c < nch; ++c) fetch(c);
+            __syncwarp();
+        }
         // ---- the MMA warp: every lane waits, lane 0 issues, the warp reconverges
         for (int ch = 0; ch < nch; ++ch) {
             const int s = ch & 1, sg = ch % L::NSTG;
@@ -1200,11 +1232,20 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
 // One launch for few-head calls: CTAs [0, n_scan) run the scan's slice CTAs, the rest the prep,
 // all resident at once (a cooperative launch), the scan reading each record as soon as the
 // prep has published it.  The block has the prep's 512 threads; a scan CTA uses its first
-// 32 * (NSW + 1).
+// 32 * (NSW + 2) (state warps, the MMA warp, the loader warp).
 // dynamic shared memory of the one-launch form: the larger of the two roles' layouts
 template <int NS>
 constexpr uint32_t mega_smem_bytes() {
     return prep::SMEM_BYTES > scan::Layout<NS>::SMEM_BYTES ? prep::SMEM_BYTES : scan::Layout<NS>::SMEM_BYTES;
+}
+
+// The scan's role is kept out of line: inlined beside the prep, its code interleaves with the
+// prep's, and the prep's first item, which runs from a cold instruction cache whenever the
+// call's working set has left L2, takes about twice as long.
+template <int NS>
+__device__ __noinline__ void mega_scan(const uint8_t *ws, const float *S0, __nv_bfloat16 *out, float *S_T, int T,
+                                       int H, float scale, int cta, const int *flags, int BH) {
+    scan_body<NS, false, true>(ws, S0, out, S_T, T, H, scale, nullptr, nullptr, 0.f, cta, flags, BH);
 }
 
 template <bool PRO, int NS>
@@ -1216,8 +1257,7 @@ chunk_mega_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int n_scan,
                   int *__restrict__ flags) {
     if ((int)blockIdx.x < n_scan)
-        scan_body<NS, false, true>(ws, S0, out, S_T, T, H, fl.scale, nullptr, nullptr, 0.f, (int)blockIdx.x,
-                                   flags, BH);
+        mega_scan<NS>(ws, S0, out, S_T, T, H, fl.scale, (int)blockIdx.x, flags, BH);
     else
         prep_body<PRO, true>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro,
                              (int)blockIdx.x - n_scan, (int)gridDim.x - n_scan, flags);
@@ -1347,7 +1387,7 @@ static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const 
     auto k = chunk_mega_kernel<PRO, NS>;
     constexpr uint32_t smem = mega_smem_bytes<NS>();
     static_assert(smem <= 232448, "shared memory budget");
-    static_assert(scan::Layout<NS>::NT <= prep::NT, "the scan's warps fit the prep's block");
+    static_assert(scan::Layout<NS>::NT + 32 <= prep::NT, "the scan's warps and the loader warp fit the prep's block");
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int nch = (a.T + C - 1) / C, BH = a.B * a.H, n_scan = BH * (D / NS);
