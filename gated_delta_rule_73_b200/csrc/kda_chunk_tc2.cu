@@ -129,12 +129,13 @@ constexpr uint32_t OFF_TAB = OFF_YR + 16384;
 constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_GC = 14336,
                    TAB_NRM = 14848, TAB_BET = 15360, TAB_SGNL = 15616, TAB_BPAR = 16640,
                    TAB_PP = 16896, TAB_SGNC = 17152, TAB_BYTES = 17408;
-// the record leaves through shared memory by bulk stores: Q e^gamma and Kd here, A_qk in the
-// band-pair operand's region, W and U in E's, sigma_C e^{gamma_C} in the tables
+// the record leaves through shared memory by bulk stores: Q e^gamma and Kd here, then W and U in
+// the same 32 KB at the item's end (first rewritten by the next item's operands), A_qk in the
+// band-pair operand's region, sigma_C e^{gamma_C} in the tables
 constexpr uint32_t OFF_RQG = OFF_TAB + TAB_BYTES;    // bf16 Q e^gamma, the record's layout
 constexpr uint32_t OFF_RKD = OFF_RQG + 16384;        // bf16 Kd
 constexpr uint32_t OFF_RAQ = OFF_BOP + 16384;        // bf16 A_qk (after Tm')
-constexpr uint32_t OFF_RWU = OFF_GAM;                // bf16 W, then U (16-column slabs)
+constexpr uint32_t OFF_RWU = OFF_RQG;                // bf16 W, then U (16-column slabs)
 constexpr uint32_t OFF_CW = OFF_RKD + 16384;        // bf16 conv taps of q, k, v [3][128 c][4] (prologue)
 constexpr uint32_t SMEM_BYTES = OFF_CW + 3072 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -280,6 +281,7 @@ prep_body(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap 
         if (done >= 0) {
             fence_proxy_async_global();
             flag_release(flags + done, 1);
+            done = -1;
         }
     };
     for (int item = cta; item < nitems && ok; item += ncta, ++li) {
@@ -294,10 +296,9 @@ prep_body(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap 
                                    : bpre;
         }
         bpre = load_beta(next);
-        if (tid == 0) {
-            if (MEGA) publish();          // (also: its sources may be rewritten)
-            else bulk_wait_read_all();    // the previous record's sources may be rewritten
-        }
+        // MEGA: the first record of each CTA is published at once (the scan starts on the first
+        // wave); later ones once the next item reaches its operands, by when the stores are done
+        if (MEGA && tid == 0 && li == 1) publish();
         ok = wait_all(bar_tma, li & 1u);
         if (ok && fused_pro) ok = wait_all(bar_v, li & 1u);
         if (ok && fused_pro) {
@@ -446,6 +447,11 @@ prep_body(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap 
                     PP[3 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c];
                     SGNC[c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c] ^ BPAR[3 * 4 + c];
                 }
+            }
+            // the operands overwrite the previous record's sources (W, U, A_qk)
+            if (tid == 0) {
+                if (MEGA) publish();
+                else bulk_wait_read_all();
             }
             __syncthreads();
 
@@ -752,6 +758,7 @@ prep_body(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap 
                 }
                 fence_proxy_async();
             }
+            if (tid == 0) bulk_wait_read_all();   // W and U are staged where Q e^gamma and Kd left from
             ok = wait_all(bar_mma, 1);
             if (ok && tid == 0) {
                 if (next < nitems) issue_v(next);   // the v staging is free again
