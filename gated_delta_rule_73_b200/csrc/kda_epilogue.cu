@@ -7,43 +7,79 @@
 // weight w of head_dim values shared by the heads (NULL = ones) and eps passed by the caller.
 //
 // The split tensor-core form applies the same epilogue inside its scan kernel, before the
-// outputs leave the chip; this pass serves the fused form and the FP32 path.  One warp per
-// (token, head) row, in place on out.
+// outputs leave the chip; this pass serves the other calls.  In place on out, DV / 8 lanes per
+// (token, head) row, 8 values each.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
 namespace kda {
 
 namespace {
+// 8 consecutive values of one row per thread (16-byte bf16 / 32-byte FP32 accesses)
+template <typename T>
+__device__ __forceinline__ void load8(const T *p, float *x) {
+    if constexpr (sizeof(T) == 2) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    } else {
+        const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+}
+template <typename T>
+__device__ __forceinline__ void store8(T *p, const float *x) {
+    if constexpr (sizeof(T) == 2) {
+        uint4 u;
+        __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(p) = u;
+    } else {
+        reinterpret_cast<float4 *>(p)[0] = make_float4(x[0], x[1], x[2], x[3]);
+        reinterpret_cast<float4 *>(p)[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+}
+
+// DV / 8 lanes per (token, head) row; the row's sum of squares is reduced over those lanes
 template <typename T, int DV>
 __global__ void __launch_bounds__(256)
 out_epilogue_kernel(T *__restrict__ out, const T *__restrict__ gate, const float *__restrict__ w,
                     float eps, long long rows) {
-    constexpr int PER = DV / 32;
-    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const int lane = threadIdx.x & 31;
-    T *o = out + row * DV;
-    const T *g = gate + row * DV;
-    float x[PER], ss = 0.f;
+    constexpr int LPR = DV / 8;
+    const long long gt = (long long)blockIdx.x * 256 + threadIdx.x;
+    const long long row = gt / LPR;
+    const int j0 = (int)(gt % LPR) * 8;
+    const bool live = row < rows;   // whole row groups of lanes share this, so the shuffles below are safe
+    float x[8], g[8], ss = 0.f;
+    if (live) {
+        load8(out + row * DV + j0, x);
+        load8(gate + row * DV + j0, g);
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        x[i] = to_f32(o[lane + 32 * i]);
-        ss += x[i] * x[i];
+        for (int i = 0; i < 8; ++i) ss += x[i] * x[i];
     }
-    const float r = rsqrtf(warp_sum(ss) / DV + eps);
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int j = lane + 32 * i;
-        const float wj = w ? w[j] : 1.f;
-        o[j] = from_f32<T>(x[i] * r * wj / (1.f + expf(-to_f32(g[j]))));
+    for (int m = LPR / 2; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+    if (!live) return;
+    const float r = rsqrtf(ss / DV + eps);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float wj = w ? w[j0 + i] : 1.f;
+        x[i] = x[i] * r * wj / (1.f + expf(-g[i]));
     }
+    store8(out + row * DV + j0, x);
 }
 
 template <typename T>
 cudaError_t launch_t(const ChunkArgs &a, cudaStream_t st) {
     const long long rows = (long long)a.B * a.T * a.H;
-    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    const unsigned blocks = (unsigned)((rows * (a.dv / 8) + 255) / 256);
     if (a.dv == 128)
         out_epilogue_kernel<T, 128><<<blocks, 256, 0, st>>>((T *)a.out, (const T *)a.out_gate, a.norm_w,
                                                             a.norm_eps, rows);
