@@ -413,7 +413,7 @@ def run_ours(args, ws, rank, local):
     # kernel's algorithmic bytes per launch are the call's; the whole call is reported beside.
     achieved = alg_bytes / (mean_k[dom] * 1e-3) / 1e9
     call_achieved = alg_bytes / (statistics.mean(step_ms) * 1e-3) / 1e9
-    kernel_names = SPLIT_KERNELS if launches == len(SPLIT_KERNELS) else [None] * launches
+    kernel_names = PREFILL_KERNELS.get(launches, [None] * launches)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak, "traffic": KERNEL_TRAFFIC.get(kernel_names[dom]),
                 "peak_kind": peak_kind, "kernel": kernel_names[dom],
@@ -466,11 +466,12 @@ def run_ours(args, ws, rank, local):
 
 CASES = ("prefill", "decode", "sweep", "ckda")
 
-# Launch order of the split tensor-core form of kda_chunk_fwd on the prefill workload, and the
-# DRAM bytes (read + write) of one launch of each, from one ncu capture
-# (profiles/chunk_tc_split_prefill_T4096_H16.md).  Re-capture when a kernel changes.
-SPLIT_KERNELS = ["chunk_prep_kernel", "chunk_scan_tc_kernel"]
-KERNEL_TRAFFIC = {"chunk_prep_kernel": 95_886_336, "chunk_scan_tc_kernel": 81_324_544}
+# Kernels of kda_chunk_fwd on the prefill workload by launches per call: the one-launch form
+# (prep and scan CTAs side by side) that few-head calls take, or the split form's two kernels;
+# and the DRAM bytes (read + write) of one launch of each from one ncu capture (profiles/),
+# None where no capture of the kernel as it stands exists.  Re-capture when a kernel changes.
+PREFILL_KERNELS = {1: ["chunk_mega_kernel"], 2: ["chunk_prep_kernel", "chunk_scan_tc_kernel"]}
+KERNEL_TRAFFIC = {"chunk_mega_kernel": 112_173_568, "chunk_prep_kernel": None, "chunk_scan_tc_kernel": None}
 
 
 def run_case(args):
