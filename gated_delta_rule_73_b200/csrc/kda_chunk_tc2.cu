@@ -893,13 +893,16 @@ struct alignas(8) ScanBars {
     uint64_t bV, bS;           // thread arrivals: V~ ready (one per P warp), S ready (one per state warp)
     uint32_t tmem_base;
     int abort;                 // a bounded wait gave up: every other wait returns at once
-    int pub;                   // MEGA: records of chunks [0, pub) are published (the loader warp)
+    int s_done;                // MEGA: state-warp updates done (NSW per chunk)
+    int o_done;                // MEGA: O products seen complete by the output warps (NSW / 2 per chunk)
 };
 
 // The scan's work for slice CTA `cta`.  MEGA (run beside the prep in one launch): each record is
-// fetched only after the prep has published it (flags, chunk-major).  The warp after the MMA
-// warp watches the flags in chunk order and advances a shared counter, so the MMA warp's refills
-// wait on shared memory only; any further warps only join the block-wide barriers.
+// fetched only after the prep has published it (flags, chunk-major).  There the warp after the
+// MMA warp issues every stage refill: it watches the flags in chunk order and two shared
+// counters that tell when a stage's last readers are done, which keeps the bulk copies (and
+// the stall of the warp that issues them) off the MMA warp and the chain; any further warps
+// only join the block-wide barriers.
 template <int NS, bool GATED, bool MEGA>
 __device__ __forceinline__ void
 scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
@@ -940,7 +943,8 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
         mbar_init(b_bS, L::NSW);
         mbar_fence_init();
         sh.abort = 0;
-        sh.pub = 0;
+        sh.s_done = 0;
+        sh.o_done = 0;
     }
     // the zero rows under each stage's A_qk
     for (int i = tid; i < L::NSTG * 512; i += (int)blockDim.x)
@@ -960,25 +964,8 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
     const uint64_t dMNs = sdesc(sbase, NS * 16, 128, kSwizzleNone);   // S copy and V~: [K rows][NS]
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
-    // MEGA: the record of chunk ch is read once the loader warp has seen it published (bounded
-    // wait; a wait that gives up raises the abort flag and skips the copy)
-    const uint32_t a_pub = smem_u32(&sh.pub);
-    auto published = [&](int ch) -> bool {
-        if (!MEGA) return true;
-        for (uint32_t i = 0; i < kWaitLimit; ++i) {
-            if (smem_acquire_load(a_pub) > ch) {
-                fence_proxy_async_global();   // the bulk copies that follow read what the prep wrote
-                return true;
-            }
-            if (*reinterpret_cast<volatile int *>(&sh.abort)) return false;
-            if (i > 64) __nanosleep(32);
-        }
-        *reinterpret_cast<volatile int *>(&sh.abort) = 1;
-        g_kda_tc2_error = 1;
-        return false;
-    };
+    const uint32_t a_sdone = smem_u32(&sh.s_done), a_odone = smem_u32(&sh.o_done);
     auto fetch = [&](int ch) {
-        if (!published(ch)) return;
         const int s = ch % L::NSTG;
         const uint32_t bar = smem_u32(&sh.stage[s]);
         const uint8_t *src = recs + (size_t)ch * IMG_BYTES;
@@ -1088,34 +1075,37 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     __syncthreads();
 
     if (load_warp) {
-        // MEGA: the flags of this sequence's records, in chunk order (item = chunk * nseq + bh)
+        // MEGA: chunk c's record goes into stage c % NSTG once the prep has published it (item =
+        // chunk * nseq + sequence) and, from c = NSTG on, once every reader of chunk c - NSTG
+        // is done: the state warps' updates (sigma_C, U) and its O product (A_qk; the output
+        // warps count it when they see it complete).  Counters, not barrier phases: this warp
+        // may fall any number of chunks behind without mistaking a phase.
         if (lane == 0) {
             for (int c = 0; c < nch; ++c) {
                 const int *f = flags + (size_t)c * (size_t)nseq + bh;
-                bool seen = false;
+                const int need = c - L::NSTG + 1;   // chunks whose stage must be free
+                bool go = false;
                 for (uint32_t i = 0; i < kWaitLimit; ++i) {
-                    if (flag_acquire(f)) {
-                        seen = true;
+                    if ((need <= 0 || (smem_acquire_load(a_sdone) >= need * L::NSW &&
+                                       smem_acquire_load(a_odone) >= need * L::NPW)) &&
+                        flag_acquire(f)) {
+                        go = true;
                         break;
                     }
                     if (*reinterpret_cast<volatile int *>(&sh.abort)) break;
-                    __nanosleep(64);
+                    __nanosleep(32);
                 }
-                if (!seen) {
+                if (!go) {
                     *reinterpret_cast<volatile int *>(&sh.abort) = 1;
                     g_kda_tc2_error = 1;
                     break;
                 }
-                smem_release_store(a_pub, c + 1);
+                fence_proxy_async_global();   // the bulk copies read what the prep wrote
+                fetch(c);
             }
         }
         __syncwarp();
     } else if (mma_warp) {
-        if (MEGA) {
-            if (lane == 0)
-                for (int c = 0; c < L::NSTG && c < nch; ++c) fetch(c);
-            __syncwarp();
-        }
         // ---- the MMA warp: every lane waits, lane 0 issues, the warp reconverges
         for (int ch = 0; ch < nch; ++ch) {
             const int s = ch & 1, sg = ch % L::NSTG;
@@ -1133,8 +1123,8 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
             }
             __syncwarp();
             // the stage of chunk ch - 1 is free once its last products are done and every state
-            // thread has passed its update (S(ch) ready): refill it
-            if (ch >= 1 && ch - 1 + L::NSTG < nch) {
+            // thread has passed its update (S(ch) ready): refill it (MEGA: the loader warp does)
+            if (!MEGA && ch >= 1 && ch - 1 + L::NSTG < nch) {
                 if (!wait(smem_u32(&sh.mO[(ch - 1) & 1]), (uint32_t)((ch - 1) >> 1) & 1u)) break;
                 if (lane == 0) fetch(ch - 1 + L::NSTG);
                 __syncwarp();
@@ -1188,6 +1178,7 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
                 // the outputs of chunk ch - 1, while this chunk's first product runs
                 const int c = ch - 1;
                 if (!wait(smem_u32(&sh.mO[c & 1]), (uint32_t)(c >> 1) & 1u)) break;
+                if (MEGA && lane == 0) smem_release_add(a_odone, 1);   // the O product has read A_qk
                 tc_fence_after();
                 emit(c);
                 prefetch_gate(ch);   // consumed by the next emit (chunk ch)
@@ -1206,7 +1197,10 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(b_bS);
+            if (lane == 0) {
+                mbar_arrive(b_bS);
+                if (MEGA) smem_release_add(a_sdone, 1);   // this warp is done with the stage's sigma_C
+            }
         }
         if (!p_lane && nch > 0 && !*reinterpret_cast<volatile int *>(&sh.abort)) {
             const int c = nch - 1;

@@ -170,9 +170,9 @@ __device__ __forceinline__ int flag_acquire(const int *p) {
 __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
-// a counter in shared memory handed between warps of one CTA (release / acquire at CTA scope)
-__device__ __forceinline__ void smem_release_store(uint32_t addr, int v) {
-    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// counters in shared memory handed between warps of one CTA (release / acquire at CTA scope)
+__device__ __forceinline__ void smem_release_add(uint32_t addr, int v) {
+    asm volatile("red.release.cta.shared::cta.add.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ int smem_acquire_load(uint32_t addr) {
     int v;
