@@ -27,12 +27,19 @@ kda_opts resolve(const kda_opts *o) {
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+// g without the -5 floor (Kimi Linear's softplus gate, or the caller says so): the tensor-core
+// forms' band-referenced decay factors could leave the bf16/FP32 range, the FP32 path cannot
+bool unbounded(const kda_opts &o) { return (o.flags & (KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS)) != 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int check_opts(const kda_opts &o) {
     if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
-    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT)) return KDA_ERR_ARG;
+    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT |
+                              KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS))
+        return KDA_ERR_ARG;
     if ((o.flags & KDA_FUSED) && (o.flags & KDA_SPLIT)) return KDA_ERR_ARG;
+    if (unbounded(o) && (o.flags & (KDA_FUSED | KDA_SPLIT))) return KDA_ERR_ARG;
+    if ((o.flags & KDA_GATE_SOFTPLUS) && (o.flags & KDA_COMPLEX)) return KDA_ERR_ARG;
     if (!isfinite(o.scale)) return KDA_ERR_ARG;
     if (o.n_events < 0 || (o.n_events > 0 && !o.events)) return KDA_ERR_ARG;
     return KDA_OK;
@@ -67,7 +74,9 @@ KernelFlags kflags(const kda_opts &o) {
 //    workspace).  Cost ~ waves * nch * t_fused, waves = ceil(B*H / SMs).
 // Measured on B200 at d = 128 (per chunk and head): t_fused = 14.0 us, t_prep = 14.8 us,
 // t_scan = 2.8 us; the model uses their ratios.  KDA_FUSED / KDA_SPLIT override it.
-bool use_tc(const kda_opts &o, int dk, int dv) { return o.dtype == KDA_BF16 && dk == 128 && dv == 128; }
+bool use_tc(const kda_opts &o, int dk, int dv) {
+    return o.dtype == KDA_BF16 && dk == 128 && dv == 128 && !unbounded(o);
+}
 int device_sms() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -130,11 +139,12 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
     // every sequence (about 1 us per chunk); a separate pass costs the bytes of out and the
     // gate instead.  Measured on B200 the chain wins from about 64 sequences on (T=8192:
     // 96 heads 0.14 vs 0.22 ms; T=4096, 16 heads: 0.048 vs 0.020 ms).
-    const bool split = chunk_tc_supported(a) && !fused;
+    const bool tc = chunk_tc_supported(a) && !a.exact_decay;
+    const bool split = tc && !fused;
     const bool fuse_epi = split && a.out_gate && (long long)a.B * a.H >= 64;
     const void *gate = a.out_gate;
     if (split && !fuse_epi) a.out_gate = nullptr;
-    cudaError_t e = !chunk_tc_supported(a) ? launch_chunk_ref(a, st)
+    cudaError_t e = !tc                     ? launch_chunk_ref(a, st)
                     : fused                 ? launch_chunk_tc(a, st)
                                             : launch_chunk_tc2(a, st);
     a.out_gate = gate;
@@ -148,7 +158,7 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 103; }
+int kda_abi_version(void) { return 104; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -211,6 +221,7 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
     a.workspace = o.workspace; a.workspace_bytes = o.workspace_bytes;
     a.events = o.events; a.n_events = o.n_events;
     a.out_gate = out_gate; a.norm_w = norm_w; a.norm_eps = norm_eps;
+    a.exact_decay = unbounded(o);
     return run_chunk(a, use_fused(o, B, H), stream);
 }
 
@@ -284,6 +295,7 @@ int kda_recurrent_step_prologue(const void *q_pre, const void *k_pre, const void
     o.flags |= KDA_QK_L2NORM;
     a.fl = kflags(o);
     a.conv_w = conv_w; a.conv_state = conv_state; a.A = A; a.b_logit = beta_logit; a.H = H;
+    a.gate_softplus = (o.flags & KDA_GATE_SOFTPLUS) ? 1 : 0;
     if (o.events && o.n_events > 0) cudaEventRecord(o.events[0], stream);
     cudaError_t e = launch_decode(a, stream);
     if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
@@ -343,6 +355,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
     p.qc = ws + off[0]; p.kc = ws + off[1]; p.vc = ws + off[2];
     p.g = ws + off[3]; p.beta = ws + off[4];
+    p.gate_softplus = (o.flags & KDA_GATE_SOFTPLUS) ? 1 : 0;
 
     int launches = 0;
     if (fused_pro) {
@@ -378,6 +391,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
     a.fl = kflags(o);
     a.workspace = ws + off[5];
     a.workspace_bytes = need - off[5];
+    a.exact_decay = unbounded(o);
     a.events = o.events; a.n_events = o.n_events;
     a.launch_idx = &launches;
     e = !tc ? launch_chunk_ref(a, stream) : use_fused(o, B, H) ? launch_chunk_tc(a, stream) : launch_chunk_tc2(a, stream);

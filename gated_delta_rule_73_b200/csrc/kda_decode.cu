@@ -31,6 +31,7 @@ struct DecodePro {
     void *conv_state;
     const float *A, *b_logit;
     int H;
+    int gate_softplus;   // g = -exp(A_h) softplus(z) (Kimi Linear) instead of -5 sigmoid(exp(A_h) z)
 };
 
 // the four taps of one channel (contiguous) as one vector load
@@ -100,7 +101,10 @@ decode_step_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
             qs[tid] = y[0];
             ks[tid] = y[1];
             vs[tid] = y[2];
-            as[tid] = expf(-5.f / (1.f + expf(-expf(a_h) * zv)));
+            // alpha = e^g; softplus(z) = max(z, 0) + log1p(e^-|z|)
+            as[tid] = pro.gate_softplus
+                          ? expf(-expf(a_h) * (fmaxf(zv, 0.f) + log1pf(expf(-fabsf(zv)))))
+                          : expf(-5.f / (1.f + expf(-expf(a_h) * zv)));
 #pragma unroll
             for (int br = 0; br < 3; ++br) {
                 cs[(br * 3 + 0) * HD + ch] = from_f32<T>(hist[br][1]);
@@ -178,7 +182,7 @@ template <typename T, int DK, int DV, bool PRO>
 static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t st) {
     decode_step_kernel<T, DK, DV, PRO><<<(unsigned)a.units, 256, 0, st>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.g, (const T *)a.beta, a.S,
-        (T *)a.out, a.fl, DecodePro{a.conv_w, a.conv_state, a.A, a.b_logit, a.H});
+        (T *)a.out, a.fl, DecodePro{a.conv_w, a.conv_state, a.A, a.b_logit, a.H, a.gate_softplus});
     return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@ struct DecodeArgs {
     const float *A;         // [H]
     const float *b_logit;   // [N, H]
     int H;
+    int gate_softplus;      // gate g = -exp(A_h) softplus(z) instead of -5 sigmoid(exp(A_h) z)
 };
 
 // Last three raw rows of each branch of a prefill, as the decode prologue's conv state.
@@ -49,6 +50,8 @@ struct ChunkArgs {
     const void *out_gate;                // [B,T,H,dv], dtype of out
     const float *norm_w;                 // [dv], nullable = ones
     float norm_eps;
+    // g may fall below -5 per token: only the exact-FP32 path takes such inputs
+    bool exact_decay;
 };
 
 // The output epilogue as its own pass over out (in place), for the paths that do not fuse it.
@@ -61,6 +64,7 @@ struct PrologueArgs {
     bool out_bf16;                       // outputs in bf16 (tensor-core path) or FP32
     int B, T, H, dk, dv;
     void *qc, *kc, *vc, *g, *beta;       // outputs in the workspace
+    int gate_softplus;                   // g = -exp(A_h) softplus(z) (unbounded; FP32 outputs)
 };
 
 // Workspace of the FP32 two-phase chunk path.

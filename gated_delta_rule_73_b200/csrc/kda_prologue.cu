@@ -9,7 +9,8 @@
 //     history before t = 0, no bias.
 //   * beta = sigmoid(b) per head, in FP32 (b_proj(...).float()).
 // Page "Kimi K3 模型结构（2）", Q&A on the decay function: the bounded log-decay
-// g = -5 * sigmoid(exp(A_h) * z), g in (-5, 0).
+// g = -5 * sigmoid(exp(A_h) * z), g in (-5, 0); with gate_softplus the Kimi Linear map the
+// same Q&A item contrasts it with, g = -exp(A_h) * softplus(z), g in (-inf, 0).
 //
 // Outputs are bf16 when the tensor-core chunk kernel follows (its operands are
 // bf16 anyway) and FP32 for the FP32 chunk path; the L2 norm of q and k is
@@ -22,6 +23,9 @@ namespace kda {
 
 namespace {
 __device__ __forceinline__ float sigm(float x) { return 1.f / (1.f + expf(-x)); }
+// softplus(x) = log(1 + e^x) = max(x, 0) + log1p(e^-|x|): no overflow for large x, and
+// log1p keeps the tail e^x accurate for very negative x
+__device__ __forceinline__ float softplus(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
 
 template <typename T, typename TO>
 __global__ void __launch_bounds__(256)
@@ -30,7 +34,7 @@ prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
                 const T *__restrict__ z, const float *__restrict__ A,
                 const float *__restrict__ b_logit, int T_, int H, int D, long long total,
                 TO *__restrict__ qc, TO *__restrict__ kc, TO *__restrict__ vc,
-                TO *__restrict__ g, TO *__restrict__ beta) {
+                TO *__restrict__ g, TO *__restrict__ beta, int gate_softplus) {
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= total) return;
     const int d = (int)(idx % D);
@@ -53,7 +57,8 @@ prologue_kernel(const T *__restrict__ q_pre, const T *__restrict__ k_pre,
         }
         dst[s][idx] = from_f32<TO>(acc * sigm(acc));
     }
-    g[idx] = from_f32<TO>(-5.f * sigm(expf(A[h]) * to_f32(z[idx])));
+    const float zv = to_f32(z[idx]);
+    g[idx] = from_f32<TO>(gate_softplus ? -expf(A[h]) * softplus(zv) : -5.f * sigm(expf(A[h]) * zv));
     if (d == 0) beta[bth] = from_f32<TO>(sigm(b_logit[bth]));
 }
 
@@ -197,7 +202,7 @@ static void launch_t(const PrologueArgs &a, long long total, unsigned blocks, cu
     prologue_kernel<T, TO><<<blocks, 256, 0, st>>>(
         (const T *)a.q_pre, (const T *)a.k_pre, (const T *)a.v_pre, (const T *)a.conv_w,
         (const T *)a.z, a.A, a.beta_logit, a.T, a.H, a.dk, total, (TO *)a.qc, (TO *)a.kc,
-        (TO *)a.vc, (TO *)a.g, (TO *)a.beta);
+        (TO *)a.vc, (TO *)a.g, (TO *)a.beta, a.gate_softplus);
 }
 
 cudaError_t launch_conv_state_from_prefill(const void *q_pre, const void *k_pre, const void *v_pre,
@@ -217,7 +222,7 @@ cudaError_t launch_conv_state_from_prefill(const void *q_pre, const void *k_pre,
 }
 
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st) {
-    if (a.bf16 && a.out_bf16 && a.dk % 8 == 0) {
+    if (a.bf16 && a.out_bf16 && a.dk % 8 == 0 && !a.gate_softplus) {
         const int nruns = (a.T + RUN - 1) / RUN;
         const long long total = (long long)a.B * nruns * (a.H * a.dk / 8);
         prologue_bf16_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libkda_b200.so")
 
 KDA_BF16, KDA_F32 = 0, 1
 KDA_QK_L2NORM, KDA_COMPLEX, KDA_FUSED, KDA_SPLIT = 1, 2, 4, 8
+KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS = 16, 32
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_ARG", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_ALIGN",
           -4: "KDA_ERR_UNSUPPORTED", -5: "KDA_ERR_CUDA", -6: "KDA_ERR_TIMEOUT",
           -7: "KDA_ERR_WORKSPACE"}
@@ -89,11 +90,14 @@ def _dtype_code(t: torch.dtype) -> int:
 
 def make_opts(dtype: torch.dtype = torch.bfloat16, *, l2norm: bool = True, complex_gate: bool = False,
               scale: float = 1.0, workspace: torch.Tensor | None = None, events=None,
-              fused: bool | None = None) -> kda_opts:
+              fused: bool | None = None, unbounded: bool = False,
+              gate_softplus: bool = False) -> kda_opts:
     o = kda_opts()
     o.dtype = _dtype_code(dtype)
     o.flags = ((KDA_QK_L2NORM if l2norm else 0) | (KDA_COMPLEX if complex_gate else 0)
-               | (0 if fused is None else KDA_FUSED if fused else KDA_SPLIT))
+               | (0 if fused is None else KDA_FUSED if fused else KDA_SPLIT)
+               | (KDA_UNBOUNDED_DECAY if unbounded else 0)
+               | (KDA_GATE_SOFTPLUS if gate_softplus else 0))
     o.scale = float(scale)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
@@ -237,16 +241,17 @@ def kda_conv_state_from_prefill(q_pre, k_pre, v_pre, conv_state, opts: kda_opts,
 
 # ------------------------------------------------------------------ conveniences
 def chunk_fwd(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False, scale=1.0,
-              fused=None, workspace=None, out=None, S_T=None, stream=None):
+              fused=None, unbounded=False, workspace=None, out=None, S_T=None, stream=None):
     """Allocate out / S_T / workspace with torch and run ``kda_chunk_fwd``."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused)
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused,
+                     unbounded=unbounded)
     if workspace is None:
         nbytes = kda_chunk_workspace_bytes(B, T, H, dk, dv, opts)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale,
-                     workspace=workspace, fused=fused)
+                     workspace=workspace, fused=fused, unbounded=unbounded)
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if S_T is None:
@@ -282,11 +287,11 @@ def chunk_fwd_gated(q, k, v, g, beta, S0, out_gate, norm_weight=None, *, norm_ep
 
 
 def recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, *,
-                            scale=1.0, out=None, stream=None):
+                            scale=1.0, gate_softplus=False, out=None, stream=None):
     """Run ``kda_recurrent_step_prologue`` (S and conv_state updated in place); returns out."""
     if out is None:
         out = torch.empty(v_pre.shape, dtype=q_pre.dtype, device=q_pre.device)
-    opts = make_opts(q_pre.dtype, scale=scale)
+    opts = make_opts(q_pre.dtype, scale=scale, gate_softplus=gate_softplus)
     kda_recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, beta_logit, S, out,
                                 opts, stream)
     return out
@@ -302,15 +307,17 @@ def conv_state_from_prefill(q_pre, k_pre, v_pre, *, out=None, stream=None):
 
 
 def chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0=None, *, scale=1.0,
-                       fused=None, workspace=None, out=None, S_T=None, stream=None):
+                       fused=None, gate_softplus=False, workspace=None, out=None, S_T=None,
+                       stream=None):
     """Allocate and run ``kda_chunk_fwd_prologue``."""
     B, T, H, dk = q_pre.shape
     dv = v_pre.shape[-1]
-    opts = make_opts(q_pre.dtype, scale=scale, fused=fused)
+    opts = make_opts(q_pre.dtype, scale=scale, fused=fused, gate_softplus=gate_softplus)
     if workspace is None:
         nbytes = kda_prologue_workspace_bytes(B, T, H, dk, dv, opts)
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q_pre.device)
-    opts = make_opts(q_pre.dtype, scale=scale, workspace=workspace, fused=fused)
+    opts = make_opts(q_pre.dtype, scale=scale, workspace=workspace, fused=fused,
+                     gate_softplus=gate_softplus)
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q_pre.dtype, device=q_pre.device)
     if S_T is None:

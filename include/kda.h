@@ -70,18 +70,33 @@ enum {
                             |alpha| in [e^-5, 1], alpha != 0; beta in [0, 2]   */
     KDA_FUSED = 4u,      /* bf16 dk = dv = 128 only: run the chunk forward as one
                             fused kernel per sequence (no workspace)          */
-    KDA_SPLIT = 8u       /* bf16 dk = dv = 128 only: run it as the parallel
+    KDA_SPLIT = 8u,      /* bf16 dk = dv = 128 only: run it as the parallel
                             per-chunk prep kernel + per-sequence scan pair
                             (workspace: one record per chunk and head).
                             With neither flag the library picks the one its
                             cost model, from B*H and the device's SM count,
                             says is faster; KDA_FUSED | KDA_SPLIT is an error */
+    KDA_UNBOUNDED_DECAY = 16u, /* g may lie anywhere in (-inf, 0]: no -5 floor.
+                            The bf16 dk = dv = 128 tensor-core forms need the
+                            floor (16 tokens of decay must stay inside e^-80,
+                            page "Kimi K3 模型结构（2）", Q&A on the -5 bound), so
+                            the chunk forward runs on the exact-FP32 chunk path
+                            instead (every decay factor taken pairwise,
+                            exponent <= 0).  Cannot be combined with
+                            KDA_FUSED or KDA_SPLIT (KDA_ERR_ARG).  The decode
+                            step is exact for any g and ignores the flag.   */
+    KDA_GATE_SOFTPLUS = 32u /* prologue entry points: the Kimi Linear gate
+                            g = -exp(A_h) * softplus(z), range (-inf, 0), in
+                            place of the bounded -5 * sigmoid(exp(A_h) z)
+                            (same Q&A item, "与 Kimi Linear 的负 softplus 有何
+                            不同").  Implies KDA_UNBOUNDED_DECAY everywhere. */
 };
 
 /* Options.  Passing NULL means {KDA_BF16, KDA_QK_L2NORM, 1.0f, NULL, 0, NULL, 0}. */
 typedef struct {
     kda_dtype dtype;        /* type of q, k, v, g, beta, out                  */
-    unsigned flags;         /* KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT */
+    unsigned flags;         /* KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT |
+                               KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS */
     float scale;            /* read-out scale; the pages use 1                 */
     void *workspace;        /* device scratch, >= kda_*_workspace_bytes()     */
     size_t workspace_bytes;
@@ -104,8 +119,9 @@ typedef struct {
  *
  *   q, k     [B,T,H,dk]  queries/keys (normalised in-kernel if KDA_QK_L2NORM)
  *   v        [B,T,H,dv]  values
- *   g        [B,T,H,dk]  log-decay g = log(alpha), expected in (-5, 0] for
- *                        unsigned KDA (bounded decay); with KDA_COMPLEX, the
+ *   g        [B,T,H,dk]  log-decay g = log(alpha), expected in [-5, 0] for
+ *                        unsigned KDA (bounded decay) unless
+ *                        KDA_UNBOUNDED_DECAY is set; with KDA_COMPLEX, the
  *                        signed gate alpha itself
  *   beta     [B,T,H]     write strength (already through the sigmoid)
  *   S0       [B,H,dk,dv] FP32 initial state, NULL means zero
@@ -180,6 +196,8 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const void *
  *   beta_logit   [B,T,H]      FP32
  *   S0, out, S_T as in kda_chunk_fwd.
  * KDA_COMPLEX is not supported here (the pages define no signed-gate map).
+ * KDA_GATE_SOFTPLUS selects the Kimi Linear gate g = -exp(A_h) * softplus(z)
+ * (unbounded below) and the exact-FP32 chunk path with it.
  */
 int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
                            const void *conv_w, const void *z, const float *A,
@@ -209,6 +227,7 @@ size_t kda_prologue_workspace_bytes(int B, int T, int H, int dk, int dv,
  *   z            [N,H,d]          gate logits (dtype);  A [H] FP32;  beta_logit [N,H] FP32
  *   S, out       as in kda_recurrent_step
  * Needs dk == dv; KDA_COMPLEX is not supported (no signed-gate map on the pages).
+ * KDA_GATE_SOFTPLUS selects the Kimi Linear gate g = -exp(A_h) * softplus(z).
  */
 int kda_recurrent_step_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
                                 const void *conv_w, void *conv_state, const void *z,
@@ -258,7 +277,8 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
-/* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated). */
+/* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
+   1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -24,6 +24,10 @@ ckda       B=8, T=8192, H=32, d=128, bf16.  alpha = tanh(N(0,1)) with its
            magnitude clamped to >= exp(-5), sign kept; beta = 2*sigmoid(N(0,1));
            q,k,v ~ N(0,1); S0 ~ N(0, 0.01) (not stated by the workload; chosen
            so that the S0 path is exercised).  Seed 0.
+softplus   any of the above with Kimi Linear's gate (``gate="softplus"``):
+           g = -exp(A_h) softplus(z), z ~ N(0,1), A_h = log U(1,16) (the
+           A_log initialisation printed on the Kimi K3 page); g is unbounded
+           below (typically -0.7 x [1, 16], tail far below -5).
 =========  ==================================================================
 
 Tensors are drawn in fp32 on the CPU from one ``torch.Generator`` and then
@@ -78,8 +82,22 @@ def _sampled_log_decay(z, A):
     return LOG_DECAY_FLOOR * torch.sigmoid(torch.exp(A)[:, None] * z)
 
 
+def _sampled_softplus_decay(z, A):
+    # the softplus workloads' sampling recipe for g (pushforward of z and A_h)
+    return -torch.exp(A)[:, None] * torch.nn.functional.softplus(z)
+
+
+def _log_scale(H, gen, gate):
+    # A_h ~ U(-1, 0) for the bounded gate; log U(1, 16) for Kimi Linear's softplus gate
+    if gate == "softplus":
+        return torch.log(_uniform((H,), 1.0, 16.0, gen))
+    if gate != "bounded":
+        raise ValueError(f"unknown gate {gate!r}")
+    return _uniform((H,), -1.0, 0.0, gen)
+
+
 def chunk_inputs(B, T, H, dk, dv, *, dtype=torch.bfloat16, S0_std=0.01, seed=0,
-                 complex_gate=False):
+                 complex_gate=False, gate="bounded"):
     """Inputs of ``kda_chunk_fwd``: q, k, v, g, beta (run dtype), S0 (fp32 or None).
 
     Unsigned KDA: g is the log-decay in (-5, 0).  Complex-KDA: g holds the
@@ -96,8 +114,8 @@ def chunk_inputs(B, T, H, dk, dv, *, dtype=torch.bfloat16, S0_std=0.01, seed=0,
         beta = 2.0 * torch.sigmoid(_randn((B, T, H), gen))
     else:
         z = _randn((B, T, H, dk), gen)
-        A = _uniform((H,), -1.0, 0.0, gen)
-        g = _sampled_log_decay(z, A)
+        A = _log_scale(H, gen, gate)
+        g = _sampled_log_decay(z, A) if gate == "bounded" else _sampled_softplus_decay(z, A)
         beta = torch.sigmoid(_randn((B, T, H), gen))
     S0 = None
     if S0_std > 0:
@@ -121,15 +139,16 @@ def workload_inputs(name, **overrides):
                         complex_gate=(name == "ckda") or overrides.get("complex_gate", False))
 
 
-def prologue_inputs(B, T, H, dk, dv, *, dtype=torch.bfloat16, S0_std=0.01, seed=0):
-    """Raw inputs of ``kda_chunk_fwd_prologue`` (sweep recipe)."""
+def prologue_inputs(B, T, H, dk, dv, *, dtype=torch.bfloat16, S0_std=0.01, seed=0,
+                    gate="bounded"):
+    """Raw inputs of ``kda_chunk_fwd_prologue`` (sweep recipe; ``gate`` picks A_h's law)."""
     gen = _gen(seed)
     q_pre = _randn((B, T, H, dk), gen)
     k_pre = _randn((B, T, H, dk), gen)
     v_pre = _randn((B, T, H, dv), gen)
     conv_w = _uniform((3, H * dk, 4), -0.5, 0.5, gen)
     z = _randn((B, T, H, dk), gen)
-    A = _uniform((H,), -1.0, 0.0, gen)
+    A = _log_scale(H, gen, gate)
     b_logit = _randn((B, T, H), gen)
     S0 = _randn((B, H, dk, dv), gen) * S0_std if S0_std > 0 else None
     cast = lambda x: x.to(dtype).contiguous()

@@ -27,6 +27,7 @@ Functions
                       UT inverse, WY vectors, inter-chunk state update).
 ``conv_silu_np``      causal depthwise short convolution + SiLU.
 ``bounded_log_decay`` g = -5 * sigmoid(exp(A_h) * z).
+``softplus_log_decay`` g = -exp(A_h) * softplus(z) (Kimi Linear's unbounded gate).
 ``sigmoid``           beta = sigmoid(b).
 ``prologue_np``       the three together (raw inputs -> q, k, v, g, beta).
 ``rmsnorm_gate_np``   the output epilogue RMSNorm(o) * w * sigmoid(g_out).
@@ -249,6 +250,19 @@ def bounded_log_decay(z, A):
     return G_MIN * sigmoid(np.exp(A)[:, None] * z)
 
 
+def softplus_log_decay(z, A):
+    """g = -exp(A_h) * softplus(z), softplus(z) = log(1 + e^z); range (-inf, 0).
+
+    Kimi K3 structure (2), Q&A "衰减函数与 Kimi Linear 的负 softplus 有何不同": the
+    gate Kimi Linear uses, with no lower bound, against which the pages set K3's
+    bounded map.  ``log1p(exp(.))`` is evaluated as ``logaddexp(0, z)`` (no overflow).
+    ``z``: [..., H, dk]; ``A``: [H].
+    """
+    z = _f64(z)
+    A = _f64(A)
+    return -np.exp(A)[:, None] * np.logaddexp(0.0, z)
+
+
 def conv_silu_np(x, w):
     """Causal depthwise short convolution (kernel 4, no bias, zero history)
     followed by SiLU.
@@ -273,8 +287,11 @@ def conv_silu_np(x, w):
     return y * sigmoid(y)
 
 
-def prologue_np(q_pre, k_pre, v_pre, conv_w, z, A, b_logit):
+def prologue_np(q_pre, k_pre, v_pre, conv_w, z, A, b_logit, *, gate="bounded"):
     """Raw branch inputs -> (q, k, v, g, beta), FP64.
+
+    ``gate``: ``"bounded"`` (K3: :func:`bounded_log_decay`) or ``"softplus"``
+    (Kimi Linear: :func:`softplus_log_decay`).
 
     ``q_pre, k_pre``: [B, T, H, dk]; ``v_pre``: [B, T, H, dv];
     ``conv_w``: [3, H*dk, 4] (q, k, v taps; requires dk == dv);
@@ -289,7 +306,12 @@ def prologue_np(q_pre, k_pre, v_pre, conv_w, z, A, b_logit):
         d = x.shape[-1]
         y = conv_silu_np(x.reshape(B, T, H * d), cw[i])
         outs.append(y.reshape(B, T, H, d))
-    g = bounded_log_decay(z, A)
+    if gate == "bounded":
+        g = bounded_log_decay(z, A)
+    elif gate == "softplus":
+        g = softplus_log_decay(z, A)
+    else:
+        raise ValueError(f"unknown gate {gate!r}")
     beta = sigmoid(b_logit)
     return outs[0], outs[1], outs[2], g, beta
 

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 103   # 1.3: kda_chunk_fwd_gated
+    assert kda.kda_abi_version() == 104   # 1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
@@ -78,7 +78,7 @@ def test_chunk_fwd_rejects_bad_arguments_on_host(kda):
     # misaligned pointer (never dereferenced)
     assert _call_chunk(kda, k=0x1004) == -3
     # unknown flag bit / bad dtype / non-finite scale
-    o = kda.make_opts(); o.flags = 16
+    o = kda.make_opts(); o.flags = 64
     assert _call_chunk(kda, opts=o) == -1
     o = kda.make_opts(); o.flags = kda.KDA_QK_L2NORM | kda.KDA_FUSED | kda.KDA_SPLIT   # both paths forced
     assert _call_chunk(kda, opts=o) == -1
@@ -192,3 +192,26 @@ def test_decode_prologue_rejects_bad_arguments_on_host(kda):
     assert handoff(T=-1) == -1
     assert handoff(cs=0) == -1
     assert handoff(B=0) == 0
+
+
+def test_unbounded_decay_flags_on_host(kda):
+    """KDA_UNBOUNDED_DECAY / KDA_GATE_SOFTPLUS: the tensor-core forms cannot take a gate
+    without the -5 floor, so forcing one of them is an argument error; the softplus map has
+    no signed form; the workspace becomes the exact-FP32 path's (the same with either flag)."""
+    import torch
+    for fl in (kda.KDA_UNBOUNDED_DECAY, kda.KDA_GATE_SOFTPLUS):
+        for forced in (kda.KDA_FUSED, kda.KDA_SPLIT):
+            o = kda.make_opts(); o.flags = kda.KDA_QK_L2NORM | fl | forced
+            assert _call_chunk(kda, opts=o) == -1
+    o = kda.make_opts(complex_gate=True, gate_softplus=True)
+    assert _call_chunk(kda, opts=o) == -1
+    unb = kda.make_opts(torch.bfloat16, unbounded=True)
+    sp = kda.make_opts(torch.bfloat16, gate_softplus=True)
+    f32 = kda.make_opts(torch.float32)
+    ref = kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, f32)
+    assert ref > 0
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, unb) == ref
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, sp) == ref
+    # the prologue with the softplus gate keeps FP32 intermediates ahead of that workspace
+    assert kda.kda_prologue_workspace_bytes(2, 130, 3, 128, 128, sp) > ref + 4 * 2 * 130 * 3 * 128 * 4
+    assert _call_chunk(kda, opts=unb) == -7                # still needs its workspace

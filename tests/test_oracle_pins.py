@@ -448,3 +448,40 @@ def test_rmsnorm_gate_invariances():
     tiny = 1e-6 * o[0, 0]
     damped = oracle.rmsnorm_gate_np(tiny, np.full_like(tiny, big), eps=1.0)
     assert np.max(np.abs(damped)) < 1e-5
+
+
+def test_softplus_gate_values():
+    """Kimi Linear's gate g = -exp(A_h) softplus(z), pinned by textbook facts: softplus(0) =
+    ln 2 (so g = -exp(A_h) ln 2 at z = 0); softplus(z) - softplus(-z) = z; its slope is the
+    logistic sigmoid (central differences); softplus(z) -> z for large z and -> e^z for very
+    negative z; the map has no lower bound (it passes -5 once exp(A_h) softplus(z) > 5)."""
+    A = np.array([-0.3, 0.0, math.log(16.0)])
+    z0 = np.zeros((1, 1, 3, 2))
+    g0 = oracle.softplus_log_decay(z0, A)
+    assert np.allclose(g0[0, 0, :, 0], -np.exp(A) * math.log(2.0), rtol=1e-15)
+    zs = np.linspace(-6, 6, 25).reshape(1, 25, 1, 1) * np.ones((1, 25, 3, 1))
+    sp = -oracle.softplus_log_decay(zs, A) / np.exp(A)[:, None]
+    spm = -oracle.softplus_log_decay(-zs, A) / np.exp(A)[:, None]
+    assert np.allclose(sp - spm, zs, atol=1e-13)
+    h = 1e-5
+    slope = (oracle.softplus_log_decay(zs + h, A) - oracle.softplus_log_decay(zs - h, A)) / (2 * h)
+    assert np.allclose(slope, -np.exp(A)[:, None] / (1 + np.exp(-zs)), atol=1e-8)
+    big = -oracle.softplus_log_decay(np.full((1, 1, 3, 1), 800.0), A)[0, 0, :, 0]
+    assert np.allclose(big, 800.0 * np.exp(A), rtol=1e-15)      # no overflow in e^z
+    tail = -oracle.softplus_log_decay(np.full((1, 1, 3, 1), -40.0), A)[0, 0, :, 0]
+    assert np.allclose(tail, math.exp(-40.0) * np.exp(A), rtol=1e-12)
+    assert np.all(oracle.softplus_log_decay(zs, A) < 0)
+    assert oracle.softplus_log_decay(np.full((1, 1, 3, 1), 3.0), A)[0, 0, 2, 0] < -5.0
+    # the prologue takes the gate it is asked for and nothing else changes
+    rng = np.random.default_rng(5)
+    B, T, H, d = 1, 5, 3, 2
+    qp, kp, vp, z = (rng.standard_normal((B, T, H, d)) for _ in range(4))
+    cw = rng.uniform(-0.5, 0.5, (3, H * d, 4))
+    b = rng.standard_normal((B, T, H))
+    p1 = oracle.prologue_np(qp, kp, vp, cw, z, A, b)
+    p2 = oracle.prologue_np(qp, kp, vp, cw, z, A, b, gate="softplus")
+    for x1, x2 in zip(p1[:3] + p1[4:], p2[:3] + p2[4:]):
+        assert np.array_equal(x1, x2)
+    assert np.array_equal(p2[3], oracle.softplus_log_decay(z, A))
+    with pytest.raises(ValueError):
+        oracle.prologue_np(qp, kp, vp, cw, z, A, b, gate="relu")
