@@ -254,7 +254,52 @@ def rows_n1(K, flush, hbm_peak):
         rows["prefill_output_epilogue"] = {"ms_gated": ms_g, "ms_plain": ms_p,
                                            "extra_bytes": Bp * Tp * Hp * d * 2,
                                            "note": "kda_chunk_fwd_gated vs kda_chunk_fwd, B=1 T=4096 H=16"}
-        del x, gate, nw, wsg, outg, Sg
+        del gate, nw, wsg, outg, Sg
+        torch.cuda.empty_cache()
+
+        # backward (kda_chunk_bwd) on the prefill workload: FP32 gradients of q, k, v, g, beta, S0
+        gr = W.grad_inputs(Bp, Tp, Hp, d, d, dtype=torch.bfloat16, seed=0)
+        ob = K.make_opts(torch.bfloat16)
+        wsb = torch.empty(K.kda_chunk_bwd_workspace_bytes(Bp, Tp, Hp, d, d, ob), dtype=torch.uint8,
+                          device="cuda")
+        ob = K.make_opts(torch.bfloat16, workspace=wsb)
+        e = lambda *shape: torch.empty(shape, dtype=torch.float32, device="cuda")
+        grads = (e(Bp, Tp, Hp, d), e(Bp, Tp, Hp, d), e(Bp, Tp, Hp, d), e(Bp, Tp, Hp, d),
+                 e(Bp, Tp, Hp), e(Bp, Hp, d, d))
+        fb = lambda: K.kda_chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gr["dout"],
+                                     gr["dS_T"], *grads, ob)
+        fb()
+        ms_b = statistics.median(time_calls(fb, 5, flush))
+        th = Bp * Tp * Hp
+        # in: q, k, v, g, dout (bf16), beta (bf16); out: dq, dk, dv, dg (FP32), dbeta (FP32);
+        # per head S0, dS_T in and dS0 out (FP32)
+        nb = th * (5 * d * 2 + 2 + 4 * d * 4 + 4) + Bp * Hp * 3 * d * d * 4
+        rows["prefill_backward"] = {
+            "ms": ms_b, "tokens_per_s": Bp * Tp / (ms_b * 1e-3), "algorithmic_bytes": nb,
+            "frac_of_hbm_roofline": (nb / (ms_b * 1e-3) / 1e9) / hbm_peak,
+            "workspace_bytes": wsb.numel(),
+            "note": "kda_chunk_bwd, B=1 T=4096 H=16 d=128 bf16 in, FP32 gradients out"}
+        del gr, wsb, grads
+        torch.cuda.empty_cache()
+
+        # unbounded decay (Kimi Linear softplus gate) on the prefill shape: exact-FP32 chunk path
+        xs = W.chunk_inputs(Bp, Tp, Hp, d, d, dtype=torch.bfloat16, seed=0, gate="softplus")
+        ou = K.make_opts(torch.bfloat16, unbounded=True)
+        wsu = torch.empty(K.kda_chunk_workspace_bytes(Bp, Tp, Hp, d, d, ou), dtype=torch.uint8,
+                          device="cuda")
+        ou = K.make_opts(torch.bfloat16, unbounded=True, workspace=wsu)
+        outu = torch.empty(xs["v"].shape, dtype=torch.bfloat16, device="cuda")
+        Su = torch.empty((Bp, Hp, d, d), dtype=torch.float32, device="cuda")
+        fu = lambda: K.kda_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["S0"], outu,
+                                     Su, ou)
+        fu()
+        ms_u = statistics.median(time_calls(fu, 5, flush))
+        nbu = th * token_head_bytes(d) + Bp * Hp * 2 * d * d * 4
+        rows["prefill_softplus_gate"] = {
+            "ms": ms_u, "tokens_per_s": Bp * Tp / (ms_u * 1e-3),
+            "frac_of_hbm_roofline": (nbu / (ms_u * 1e-3) / 1e9) / hbm_peak,
+            "note": "kda_chunk_fwd with KDA_UNBOUNDED_DECAY (exact-FP32 path), softplus-gate inputs"}
+        del x, xs, wsu, outu, Su
         torch.cuda.empty_cache()
 
         # a5: decode step, N = 256, H = 96, 64 steps with S carried in HBM
@@ -464,7 +509,7 @@ def run_ours(args, ws, rank, local):
     return 0
 
 
-CASES = ("prefill", "decode", "sweep", "ckda")
+CASES = ("prefill", "decode", "sweep", "ckda", "bwd")
 
 # Kernels of kda_chunk_fwd on the prefill workload by launches per call: the one-launch form
 # (prep and scan CTAs side by side) that few-head calls take, or the split form's two kernels;
@@ -477,7 +522,8 @@ KERNEL_TRAFFIC = {"chunk_mega_kernel": 112_173_568, "chunk_prep_kernel": None, "
 def run_case(args):
     """Run one workload's call a few times and exit (a small case for ncu captures):
     prefill = B=1 T=4096 H=16; decode = N=64 H=96 (800 MB of state);
-    sweep = prologue path at T=2048 H=96; ckda = B=2 T=8192 H=32 signed gate."""
+    sweep = prologue path at T=2048 H=96; ckda = B=2 T=8192 H=32 signed gate;
+    bwd = kda_chunk_bwd at B=1 T=1024 H=16."""
     import gated_delta_rule_73_b200 as K
     torch.cuda.set_device(0)
     W.set_device("cuda")
@@ -489,6 +535,11 @@ def run_case(args):
         out = torch.empty((N, H, d), dtype=torch.bfloat16, device="cuda")
         o = K.make_opts(torch.bfloat16)
         fn = lambda: K.kda_recurrent_step(t["q"], t["k"], t["v"], t["g"], t["beta"], S, out, o)
+    elif args.case == "bwd":
+        x = W.workload_inputs("prefill", T=1024)
+        gr = W.grad_inputs(1, 1024, 16, d, d, dtype=torch.bfloat16, seed=0)
+        fn = lambda: K.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], gr["dout"],
+                                 gr["dS_T"])
     elif args.case == "sweep":
         T, H = 2048, 96
         x = W.sweep_inputs(T)

@@ -158,7 +158,7 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 104; }
+int kda_abi_version(void) { return 105; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -240,6 +240,52 @@ int kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void 
     if (!out_gate && B > 0 && T > 0 && H > 0) return KDA_ERR_ARG;
     return chunk_fwd_impl(q, k, v, g, beta, S0, out, S_T, out_gate, norm_weight, norm_eps, B, T, H,
                           dk, dv, opts, stream);
+}
+
+size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, const kda_opts *opts) {
+    const kda_opts o = resolve(opts);
+    if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    return round_up(chunk_bwd_workspace_bytes(B, T, H, dk, dv), kAlignWs);
+}
+
+int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  const float *S0, const void *dout, const float *dS_T, float *grad_q,
+                  float *grad_k, float *grad_v, float *grad_g, float *grad_beta, float *grad_S0,
+                  int B, int T, int H, int dk, int dv, const kda_opts *opts, cudaStream_t stream) {
+    const kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if ((s = check_dims(B, T, H, dk, dv)) != KDA_OK) return s;
+    if (B == 0 || H == 0) return KDA_OK;
+    if (T == 0) {   // the identity: dS0 = dS_T, nothing else to write
+        if (!aligned16(dS_T) || !aligned16(grad_S0)) return KDA_ERR_ALIGN;
+        if (!grad_S0) return KDA_OK;
+        const size_t bytes = (size_t)B * H * dk * dv * sizeof(float);
+        cudaError_t e = dS_T ? cudaMemcpyAsync(grad_S0, dS_T, bytes, cudaMemcpyDeviceToDevice, stream)
+                             : cudaMemsetAsync(grad_S0, 0, bytes, stream);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    if (!q || !k || !v || !g || !beta || !dout || !grad_q || !grad_k || !grad_v || !grad_g || !grad_beta)
+        return KDA_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, S0, dout, dS_T, grad_q, grad_k, grad_v, grad_g,
+                          grad_beta, grad_S0, o.workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    const size_t need = round_up(chunk_bwd_workspace_bytes(B, T, H, dk, dv), kAlignWs);
+    if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    BwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.dout = dout; a.dS_T = dS_T;
+    a.dq = grad_q; a.dk = grad_k; a.dv = grad_v; a.dg = grad_g; a.dbeta = grad_beta; a.dS0 = grad_S0;
+    a.workspace = o.workspace;
+    a.B = B; a.T = T; a.H = H; a.dk_ = dk; a.dv_ = dv;
+    a.bf16 = o.dtype == KDA_BF16;
+    a.fl = kflags(o);
+    if (o.events && o.n_events > 0) cudaEventRecord(o.events[0], stream);
+    cudaError_t e = launch_chunk_bwd(a, stream);
+    if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 int kda_recurrent_step(const void *q, const void *k, const void *v, const void *g, const void *beta,

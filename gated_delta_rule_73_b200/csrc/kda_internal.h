@@ -85,6 +85,22 @@ cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a,
 cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st);
 
+// Backward of the chunk forward (kda_chunk_bwd): gradients in FP32.
+struct BwdArgs {
+    const void *q, *k, *v, *g, *beta;    // forward inputs ([B,T,H,*], dtype)
+    const float *S0;                     // nullable
+    const void *dout;                    // [B,T,H,dv], dtype
+    const float *dS_T;                   // nullable
+    float *dq, *dk, *dv, *dg, *dbeta;    // [B,T,H,dk] x3 / [B,T,H,dv] / [B,T,H]
+    float *dS0;                          // nullable
+    void *workspace;                     // chunk_bwd_workspace_bytes
+    int B, T, H, dk_, dv_;
+    bool bf16;
+    KernelFlags fl;
+};
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st);
+
 // Record a.events[*a.launch_idx] (if requested) and advance the counter.
 inline void mark_launch(const ChunkArgs &a, cudaStream_t st) {
     if (a.events && a.launch_idx && *a.launch_idx < a.n_events)

@@ -58,6 +58,10 @@ def _load():
     lib.kda_conv_state_from_prefill.restype = ip
     lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 8 + [ip] * 5 + [op, vp]
     lib.kda_chunk_fwd_noalloc.restype = ip
+    lib.kda_chunk_bwd.argtypes = [vp] * 14 + [ip] * 5 + [op, vp]
+    lib.kda_chunk_bwd.restype = ip
+    lib.kda_chunk_bwd_workspace_bytes.argtypes = [ip] * 5 + [op]
+    lib.kda_chunk_bwd_workspace_bytes.restype = sz
     lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_chunk_workspace_bytes.restype = sz
     lib.kda_prologue_workspace_bytes.argtypes = [ip] * 5 + [op]
@@ -153,6 +157,26 @@ def kda_chunk_fwd(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -
     st = _lib.kda_chunk_fwd(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
     if st != 0:
         raise KdaError("kda_chunk_fwd", st)
+
+
+def kda_chunk_bwd_workspace_bytes(B, T, H, dk, dv, opts: kda_opts | None = None) -> int:
+    return int(_lib.kda_chunk_bwd_workspace_bytes(B, T, H, dk, dv, ctypes.byref(opts) if opts else None))
+
+
+def kda_chunk_bwd(q, k, v, g, beta, S0, dout, dS_T, grad_q, grad_k, grad_v, grad_g, grad_beta,
+                  grad_S0, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_chunk_bwd``: FP32 gradients of <dout, O> + <dS_T, S_T> of kda_chunk_fwd."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    f = torch.float32
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(S0, "S0", f), _ptr(dout, "dout", dt), _ptr(dS_T, "dS_T", f),
+            _ptr(grad_q, "grad_q", f), _ptr(grad_k, "grad_k", f), _ptr(grad_v, "grad_v", f),
+            _ptr(grad_g, "grad_g", f), _ptr(grad_beta, "grad_beta", f), _ptr(grad_S0, "grad_S0", f)]
+    st = _lib.kda_chunk_bwd(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_chunk_bwd", st)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -> None:
@@ -258,6 +282,25 @@ def chunk_fwd(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False, sca
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     kda_chunk_fwd(q, k, v, g, beta, S0, out, S_T, opts, stream)
     return out, S_T
+
+
+def chunk_bwd(q, k, v, g, beta, S0, dout, dS_T=None, *, l2norm=True, complex_gate=False,
+              scale=1.0, workspace=None, want_dS0=True, stream=None):
+    """Allocate the FP32 gradients and the workspace with torch and run ``kda_chunk_bwd``;
+    returns (dq, dk, dv, dg, dbeta, dS0 or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale)
+    if workspace is None:
+        nbytes = kda_chunk_bwd_workspace_bytes(B, T, H, dk, dv, opts)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale,
+                     workspace=workspace)
+    e = lambda *shape: torch.empty(shape, dtype=torch.float32, device=q.device)
+    grads = (e(B, T, H, dk), e(B, T, H, dk), e(B, T, H, dv), e(B, T, H, dk), e(B, T, H),
+             e(B, H, dk, dv) if want_dS0 else None)
+    kda_chunk_bwd(q, k, v, g, beta, S0, dout, dS_T, *grads, opts, stream)
+    return grads
 
 
 def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scale=1.0,

@@ -274,11 +274,44 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
                           int B, int T, int H, int dk, int dv, const kda_opts *opts,
                           cudaStream_t stream);
 
+/*
+ * kda_chunk_bwd -- backward of the chunk forward (chunk_kda training).
+ *
+ * Page "Kimi K3 模型结构（2）", Q&A on the train / prefill / decode forms: training
+ * runs chunk_kda, so it needs the gradient of the forward.  Given the upstream
+ * gradients dout = dL/dO and dS_T = dL/dS_T of a call of kda_chunk_fwd with the
+ * same q, k, v, g, beta, S0 and opts, this writes the gradients of
+ * L = <dout, O> + <dS_T, S_T> with respect to every input:
+ *
+ *   grad_q, grad_k, grad_g [B,T,H,dk] FP32   (q, k before the in-kernel L2 norm
+ *                                             when KDA_QK_L2NORM is set; g as
+ *                                             passed: log-decay, or with
+ *                                             KDA_COMPLEX the signed gate alpha)
+ *   grad_v [B,T,H,dv] FP32,  grad_beta [B,T,H] FP32
+ *   grad_S0 [B,H,dk,dv] FP32, NULL to skip
+ *
+ * dout has the activation dtype (bf16 or fp32) with the layout of out; dS_T is
+ * FP32 [B,H,dk,dv], NULL meaning zero; S0 NULL means zero.  All arithmetic is
+ * FP32 and exact for any g <= 0 (no -5 floor needed).  The gradient outputs
+ * are written, not accumulated.  opts->workspace must hold
+ * kda_chunk_bwd_workspace_bytes(...) bytes: FP32 states every 16 tokens,
+ * B*H*ceil(T/16)*dk*dv*4 bytes.  T == 0 writes grad_S0 = dS_T only.
+ */
+int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
+                  const void *beta, const float *S0, const void *dout,
+                  const float *dS_T, float *grad_q, float *grad_k, float *grad_v,
+                  float *grad_g, float *grad_beta, float *grad_S0, int B, int T,
+                  int H, int dk, int dv, const kda_opts *opts, cudaStream_t stream);
+
+/* Workspace bytes kda_chunk_bwd needs. */
+size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv,
+                                     const kda_opts *opts);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
 /* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
-   1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS). */
+   1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -201,3 +201,12 @@ def decode_step_inputs(N, H, dk, dv, step, *, A=None, dtype=torch.bfloat16):
     beta = torch.sigmoid(_randn((N, H), gen))
     cast = lambda x: x.to(dtype).contiguous()
     return dict(q=cast(q), k=cast(k), v=cast(v), g=cast(g), beta=cast(beta))
+
+
+def grad_inputs(B, T, H, dk, dv, *, dtype=torch.bfloat16, dST_std=0.01, seed=0):
+    """Upstream gradients of the backward workloads: dout ~ N(0,1) [B,T,H,dv] in the run
+    dtype and dS_T ~ N(0, dST_std) [B,H,dk,dv] FP32 (None when dST_std is 0)."""
+    gen = _gen(20_000 + seed)
+    dout = _randn((B, T, H, dv), gen).to(dtype).contiguous()
+    dST = _randn((B, H, dk, dv), gen) * dST_std if dST_std > 0 else None
+    return dict(dout=dout, dS_T=dST)

@@ -23,6 +23,8 @@ Functions
 ``recurrence_np``     numpy FP64 twin of the same recurrence (vectorised over
                       sequences, loop over tokens).
 ``recurrence_loops``  pure-Python loops, for tiny cases only.
+``recurrence_bwd_np`` FP64 reverse-mode gradient of the token recurrence
+                      (dq, dk, dv, dg, dbeta, dS0 from dO and dS_T).
 ``chunkwise_np``      FP64 chunkwise-algebra form (cumulative decay, A_kk,
                       UT inverse, WY vectors, inter-chunk state update).
 ``conv_silu_np``      causal depthwise short convolution + SiLU.
@@ -142,6 +144,75 @@ def recurrence_np(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False,
         S = St + beta[:, t, :, None, None] * k[:, t, :, :, None] * r[:, :, None, :]
         out[:, t] = scale * np.einsum("bhij,bhi->bhj", S, q[:, t])
     return out, S
+
+
+def recurrence_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, l2norm=True,
+                      complex_gate=False, scale=1.0, eps=L2NORM_EPS):
+    """FP64 gradient of ``L = <dO, O> + <dS_T, S_T>`` with respect to every input of the
+    recurrence: returns ``(dq, dk, dv, dg, dbeta, dS0)`` with the shapes of q, k, v, g,
+    beta and S (dS0 is returned even when ``S0`` is None, meaning zero).
+
+    The forward is the recurrence of :func:`recurrence_np` (Kimi K3 KDA(1) section 1.2.1:
+    decay, erase, write, read the post-write state; GDN, KDA notes section "Kimi Delta
+    Attention").  Its reverse pass, token by token from t = T down to 1, with
+    ``St = Diag(alpha_t) S_{t-1}``, ``r = v_t - St^T k_t`` and ``G = dS_t + scale q_t do_t^T``
+    (dS_t: the gradient reaching S_t from later tokens, dS_T at the end):
+
+      dq_t = scale S_t do_t            a = G^T k_t        dbeta_t = a . r
+      dv_t = beta_t a                  dk_t = beta_t G r - St dv_t
+      dSt  = G - k_t dv_t^T            dalpha_t = rowsum(dSt * S_{t-1})
+      dS_{t-1} = Diag(alpha_t) dSt
+
+    then ``dg = alpha * dalpha`` (alpha = e^g) or ``dalpha`` (Complex-KDA, g = alpha), and
+    through the in-kernel L2 norm ``x_hat = x / n``, ``n = sqrt(|x|^2 + eps)``:
+    ``dx = (dx_hat - x_hat (x_hat . dx_hat)) / n``.  Every state S_0..S_T is kept (tiny and
+    moderate sizes only).
+    """
+    q, k, v, g, beta, dO = map(_f64, (q, k, v, g, beta, dO))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if l2norm:
+        nq = np.sqrt(np.sum(q * q, axis=-1, keepdims=True) + eps)
+        nk = np.sqrt(np.sum(k * k, axis=-1, keepdims=True) + eps)
+        qh, kh = q / nq, k / nk
+    else:
+        qh, kh = q, k
+    alpha = g if complex_gate else np.exp(g)
+    S = np.zeros((B, H, dk, dv)) if S0 is None else _f64(S0).copy()
+    states = [S]
+    resid = []
+    for t in range(T):
+        St = alpha[:, t, :, :, None] * S
+        r = v[:, t] - np.einsum("bhij,bhi->bhj", St, kh[:, t])
+        S = St + beta[:, t, :, None, None] * kh[:, t, :, :, None] * r[:, :, None, :]
+        states.append(S)
+        resid.append(r)
+    dS = np.zeros((B, H, dk, dv)) if dS_T is None else _f64(dS_T).copy()
+    dqh, dkh, dalpha = np.zeros_like(q), np.zeros_like(k), np.zeros_like(g)
+    dvv, dbeta = np.zeros_like(v), np.zeros_like(beta)
+    for t in range(T - 1, -1, -1):
+        Sp, St_post, r = states[t], states[t + 1], resid[t]
+        a_t, k_t, q_t, b_t = alpha[:, t], kh[:, t], qh[:, t], beta[:, t]
+        do = scale * dO[:, t]
+        St = a_t[..., None] * Sp
+        G = dS + q_t[..., :, None] * do[..., None, :]
+        dqh[:, t] = np.einsum("bhij,bhj->bhi", St_post, do)
+        a = np.einsum("bhij,bhi->bhj", G, k_t)
+        dbeta[:, t] = np.sum(a * r, axis=-1)
+        dr = b_t[..., None] * a
+        dvv[:, t] = dr
+        dkh[:, t] = (b_t[..., None] * np.einsum("bhij,bhj->bhi", G, r)
+                     - np.einsum("bhij,bhj->bhi", St, dr))
+        dSt = G - k_t[..., :, None] * dr[..., None, :]
+        dalpha[:, t] = np.sum(dSt * Sp, axis=-1)
+        dS = a_t[..., None] * dSt
+    dg = dalpha if complex_gate else alpha * dalpha
+    if l2norm:
+        dq = (dqh - qh * np.sum(qh * dqh, axis=-1, keepdims=True)) / nq
+        dk_ = (dkh - kh * np.sum(kh * dkh, axis=-1, keepdims=True)) / nk
+    else:
+        dq, dk_ = dqh, dkh
+    return dq, dk_, dvv, dg, dbeta, dS
 
 
 def recurrence_loops(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False,

@@ -36,7 +36,7 @@ def test_header_declares_the_entry_points():
     for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_prologue",
               "kda_recurrent_step_prologue", "kda_conv_state_from_prefill", "kda_chunk_fwd_gated",
               "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_status_string",
-              "kda_abi_version"):
+              "kda_abi_version", "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes"):
         assert n in names
 
 
@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 104   # 1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS
+    assert kda.kda_abi_version() == 105   # 1.5: kda_chunk_bwd
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
@@ -215,3 +215,28 @@ def test_unbounded_decay_flags_on_host(kda):
     # the prologue with the softplus gate keeps FP32 intermediates ahead of that workspace
     assert kda.kda_prologue_workspace_bytes(2, 130, 3, 128, 128, sp) > ref + 4 * 2 * 130 * 3 * 128 * 4
     assert _call_chunk(kda, opts=unb) == -7                # still needs its workspace
+
+
+def test_chunk_bwd_host_checks(kda):
+    """kda_chunk_bwd: argument checks before any CUDA call, and its workspace (FP32 states
+    every 16 tokens: B*H*ceil(T/16)*dk*dv*4 bytes, 256-byte rounded)."""
+    vp = ctypes.c_void_p
+    o = kda.make_opts()
+
+    def call(ptrs=None, B=1, T=64, H=2, dk=128, dv=128, opts=o):
+        p = [vp(x) for x in (ptrs or [0x1000] * 14)]
+        return kda._lib.kda_chunk_bwd(*p, B, T, H, dk, dv, ctypes.byref(opts), None)
+
+    good = [0x1000] * 14
+    assert call(good[:6] + [0] + good[7:]) == -1           # dout is required
+    assert call(good[:8] + [0] + good[9:]) == -1           # grad_q is required
+    assert call(good[:10] + [0x1004] + good[11:]) == -3    # misaligned grad_v
+    assert call(dk=96) == -4
+    assert call(T=-1) == -1
+    assert call() == -7                                    # needs its workspace
+    assert call(B=0) == 0
+    assert call(good[:13] + [0], T=0) == 0                 # T = 0 without grad_S0: nothing to do
+    bad = kda.make_opts(); bad.flags = 64
+    assert call(opts=bad) == -1
+    assert kda.kda_chunk_bwd_workspace_bytes(2, 33, 3, 128, 64, o) == 2 * 3 * 3 * 128 * 64 * 4
+    assert kda.kda_chunk_bwd_workspace_bytes(1, 0, 3, 128, 128, o) == 0

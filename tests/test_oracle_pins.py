@@ -485,3 +485,66 @@ def test_softplus_gate_values():
     assert np.array_equal(p2[3], oracle.softplus_log_decay(z, A))
     with pytest.raises(ValueError):
         oracle.prologue_np(qp, kp, vp, cw, z, A, b, gate="relu")
+
+
+# ---------------------------------------------------------------- backward
+def _loss(fwd_inputs, dO, dST, **kw):
+    o, s = oracle.recurrence_np(*fwd_inputs, **kw)
+    return float(np.sum(o * dO) + np.sum(s * dST))
+
+
+@pytest.mark.parametrize("complex_gate,l2norm,scale", [(False, True, 1.0), (False, False, 0.7),
+                                                       (True, True, 1.0), (True, False, 1.3)])
+def test_backward_equals_finite_differences(complex_gate, l2norm, scale):
+    """Every gradient of the oracle's backward agrees with central differences of the
+    forward oracle (an independent route: only the forward definition is used), for
+    every element of q, k, v, g, beta and S0, including a token past a chunk-sized
+    stretch and both gates."""
+    rng = np.random.default_rng(11 + int(complex_gate) + 2 * int(l2norm))
+    q, k, v, g, beta, S0 = _rand_case(rng, B=1, T=6, H=2, dk=4, dv=3, complex_gate=complex_gate)
+    dO = rng.standard_normal((1, 6, 2, 3))
+    dST = rng.standard_normal((1, 2, 4, 3))
+    kw = dict(l2norm=l2norm, complex_gate=complex_gate, scale=scale)
+    grads = oracle.recurrence_bwd_np(q, k, v, g, beta, S0, dO, dST, **kw)
+    inputs = [q, k, v, g, beta, S0]
+    h = 1e-6
+    for idx, (x, gx) in enumerate(zip(inputs, grads)):
+        assert gx.shape == x.shape
+        fd = np.zeros_like(x)
+        for pos in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[pos] += h
+            xm[pos] -= h
+            ip = list(inputs); ip[idx] = xp
+            im = list(inputs); im[idx] = xm
+            fd[pos] = (_loss(ip, dO, dST, **kw) - _loss(im, dO, dST, **kw)) / (2 * h)
+        assert np.max(np.abs(fd - gx)) <= 1e-7 * max(1.0, np.max(np.abs(fd))), idx
+
+
+def test_backward_frozen_state_closed_form():
+    """beta = 0 freezes the write: o_t = scale S0^T (Gamma_t * q_t) with Gamma_t the
+    decay accumulated from the start and S_T = Diag(Gamma_T) S0.  So by hand:
+    dq_t = scale Diag(Gamma_t) S0 do_t, dv = 0, dS0 = sum_t scale Diag(Gamma_t) q_t do_t^T
+    + Diag(Gamma_T) dS_T, and dg_{t,c} = sum_{s >= t} (the terms of o_s and S_T on channel c),
+    i.e. the reverse cumulative sum of Gamma_s,c q_s,c (S0 scale do_s)_c (+ the S_T term)."""
+    rng = np.random.default_rng(3)
+    B, T, H, dk, dv = 1, 5, 1, 4, 3
+    q, k, v, g, beta, S0 = _rand_case(rng, B=B, T=T, H=H, dk=dk, dv=dv)
+    beta = np.zeros_like(beta)
+    dO = rng.standard_normal((B, T, H, dv))
+    dST = rng.standard_normal((B, H, dk, dv))
+    sc = 0.9
+    dq, dk_, dvv, dg, db, dS0 = oracle.recurrence_bwd_np(q, k, v, g, beta, S0, dO, dST,
+                                                         l2norm=False, scale=sc)
+    Gam = np.exp(np.cumsum(g[0, :, 0], axis=0))          # [T, dk], from the start
+    S = S0[0, 0]
+    for t in range(T):
+        assert np.allclose(dq[0, t, 0], sc * Gam[t] * (S @ dO[0, t, 0]), atol=1e-13)
+    assert np.all(dvv == 0) and np.all(dk_ == 0)
+    want_S0 = sum(sc * (Gam[t] * q[0, t, 0])[:, None] * dO[0, t, 0][None, :] for t in range(T))
+    want_S0 = want_S0 + Gam[-1][:, None] * dST[0, 0]
+    assert np.allclose(dS0[0, 0], want_S0, atol=1e-13)
+    per_t = np.array([sc * Gam[t] * q[0, t, 0] * (S @ dO[0, t, 0]) for t in range(T)])
+    per_t[-1] += Gam[-1] * np.sum(S * dST[0, 0], axis=1)
+    want_g = np.cumsum(per_t[::-1], axis=0)[::-1]
+    assert np.allclose(dg[0, :, 0], want_g, atol=1e-13)
