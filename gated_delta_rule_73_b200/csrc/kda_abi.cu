@@ -158,7 +158,7 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 105; }
+int kda_abi_version(void) { return 106; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -225,11 +225,92 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
     return run_chunk(a, use_fused(o, B, H), stream);
 }
 
+// Workspace of kda_segment_pair: a zero v [B,T,H,dk] and an identity S0 [B,H,dk,dk] for the
+// run that yields M, a scratch out [B,T,H,max(dk,dv)] both runs write, and the chunk
+// forward's own workspace (the larger of the two runs').
+static size_t segment_ws_parts(const kda_opts &o, int B, int T, int H, int dk, int dv, size_t *off) {
+    const size_t e = o.dtype == KDA_BF16 ? 2 : 4;
+    const size_t rows = (size_t)B * T * H;
+    const int dmax = dk > dv ? dk : dv;
+    auto cws = [&](int dvv) { return use_tc(o, dk, dvv) ? tc_ws(o, B, T, H) : chunk_ws(B, T, H, dk, dvv); };
+    const size_t c1 = cws(dv), c2 = cws(dk);
+    size_t x = 0;
+    off[0] = x; x = round_up(x + rows * dk * e, kAlignWs);
+    off[1] = x; x = round_up(x + (size_t)B * H * dk * dk * 4, kAlignWs);
+    off[2] = x; x = round_up(x + rows * dmax * e, kAlignWs);
+    off[3] = x; x += c1 > c2 ? c1 : c2;
+    return x;
+}
+
+size_t kda_segment_pair_workspace_bytes(int B, int T, int H, int dk, int dv, const kda_opts *opts) {
+    const kda_opts o = resolve(opts);
+    if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
+    if (B <= 0 || T <= 0 || H <= 0) return 0;
+    size_t off[4];
+    return segment_ws_parts(o, B, T, H, dk, dv, off);
+}
+
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const void *g, const void *beta,
                   const float *S0, void *out, float *S_T, int B, int T, int H, int dk, int dv,
                   const kda_opts *opts, cudaStream_t stream) {
     return chunk_fwd_impl(q, k, v, g, beta, S0, out, S_T, nullptr, nullptr, 0.f, B, T, H, dk, dv,
                           opts, stream);
+}
+
+int kda_segment_pair(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                     float *M_out, float *B_out, int B, int T, int H, int dk, int dv,
+                     const kda_opts *opts, cudaStream_t stream) {
+    const kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if ((s = check_dims(B, T, H, dk, dv)) != KDA_OK) return s;
+    if (B == 0 || H == 0) return KDA_OK;
+    if (!M_out || !B_out) return KDA_ERR_ARG;
+    if (!aligned16(M_out) || !aligned16(B_out)) return KDA_ERR_ALIGN;
+    if (T == 0) {   // the empty segment is the identity pair (I, 0)
+        if (launch_identity(M_out, (long long)B * H, dk, stream) != cudaSuccess) return KDA_ERR_CUDA;
+        return cudaMemsetAsync(B_out, 0, (size_t)B * H * dk * dv * 4, stream) == cudaSuccess ? KDA_OK
+                                                                                         : KDA_ERR_CUDA;
+    }
+    if (!q || !k || !v || !g || !beta) return KDA_ERR_ARG;
+    const void *ptrs[] = {q, k, v, g, beta, o.workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    size_t off[4];
+    const size_t need = segment_ws_parts(o, B, T, H, dk, dv, off);
+    if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    char *ws = (char *)o.workspace;
+    void *zv = ws + off[0];
+    float *eye = (float *)(ws + off[1]);
+    void *scratch_out = ws + off[2];
+    kda_opts oc = o;
+    oc.workspace = ws + off[3];
+    oc.workspace_bytes = need - off[3];
+    oc.events = nullptr;
+    oc.n_events = 0;
+    const size_t e = o.dtype == KDA_BF16 ? 2 : 4;
+    if (cudaMemsetAsync(zv, 0, (size_t)B * T * H * dk * e, stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (launch_identity(eye, (long long)B * H, dk, stream) != cudaSuccess) return KDA_ERR_CUDA;
+    // B: the segment's final state from S0 = 0
+    s = chunk_fwd_impl(q, k, v, g, beta, nullptr, scratch_out, B_out, nullptr, nullptr, 0.f, B, T, H,
+                       dk, dv, &oc, stream);
+    if (s != KDA_OK) return s;
+    // M: from S0 = I with v = 0 (column i of the final state is M e_i)
+    return chunk_fwd_impl(q, k, zv, g, beta, eye, scratch_out, M_out, nullptr, nullptr, 0.f, B, T, H,
+                          dk, dk, &oc, stream);
+}
+
+int kda_affine_combine(const float *M, const float *Bp, int n, const float *S0, float *S_out, int BH,
+                       int dk, int dv, cudaStream_t stream) {
+    if (n < 0 || BH < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    if (BH == 0) return KDA_OK;
+    if (!S_out || (n > 0 && (!M || !Bp))) return KDA_ERR_ARG;
+    const void *ptrs[] = {M, Bp, S0, S_out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    return launch_affine_combine(M, Bp, n, S0, S_out, BH, dk, dv, stream) == cudaSuccess ? KDA_OK
+                                                                                      : KDA_ERR_CUDA;
 }
 
 int kda_chunk_fwd_gated(const void *q, const void *k, const void *v, const void *g, const void *beta,

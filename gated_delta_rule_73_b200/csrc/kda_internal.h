@@ -101,6 +101,12 @@ struct BwdArgs {
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st);
 
+// Affine pairs of segments (context parallelism over T): the identity start state and the
+// ordered fold S <- M_r S + B_r of n pairs ([n, BH, dk, dk] and [n, BH, dk, dv], FP32).
+cudaError_t launch_identity(float *S, long long count, int d, cudaStream_t st);
+cudaError_t launch_affine_combine(const float *M, const float *Bp, int n, const float *S0, float *S_out,
+                                  int BH, int dk, int dv, cudaStream_t st);
+
 // Record a.events[*a.launch_idx] (if requested) and advance the counter.
 inline void mark_launch(const ChunkArgs &a, cudaStream_t st) {
     if (a.events && a.launch_idx && *a.launch_idx < a.n_events)

@@ -62,6 +62,12 @@ def _load():
     lib.kda_chunk_bwd.restype = ip
     lib.kda_chunk_bwd_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_chunk_bwd_workspace_bytes.restype = sz
+    lib.kda_segment_pair.argtypes = [vp] * 7 + [ip] * 5 + [op, vp]
+    lib.kda_segment_pair.restype = ip
+    lib.kda_segment_pair_workspace_bytes.argtypes = [ip] * 5 + [op]
+    lib.kda_segment_pair_workspace_bytes.restype = sz
+    lib.kda_affine_combine.argtypes = [vp, vp, ip, vp, vp, ip, ip, ip, vp]
+    lib.kda_affine_combine.restype = ip
     lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_chunk_workspace_bytes.restype = sz
     lib.kda_prologue_workspace_bytes.argtypes = [ip] * 5 + [op]
@@ -177,6 +183,38 @@ def kda_chunk_bwd(q, k, v, g, beta, S0, dout, dS_T, grad_q, grad_k, grad_v, grad
     st = _lib.kda_chunk_bwd(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
     if st != 0:
         raise KdaError("kda_chunk_bwd", st)
+
+
+def kda_segment_pair_workspace_bytes(B, T, H, dk, dv, opts: kda_opts | None = None) -> int:
+    return int(_lib.kda_segment_pair_workspace_bytes(B, T, H, dk, dv,
+                                                     ctypes.byref(opts) if opts else None))
+
+
+def kda_segment_pair(q, k, v, g, beta, M_out, B_out, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_segment_pair``: the segment's affine pair (M [B,H,dk,dk], B [B,H,dk,dv])."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    f = torch.float32
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(M_out, "M_out", f), _ptr(B_out, "B_out", f)]
+    st = _lib.kda_segment_pair(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_segment_pair", st)
+
+
+def kda_affine_combine(M, Bp, n, S0, S_out, stream=None) -> None:
+    """Call ``kda_affine_combine``: S_out = fold of pairs 0..n-1 of M [R,BH,dk,dk], Bp
+    [R,BH,dk,dv] onto S0 [BH,dk,dv] (None = zero)."""
+    dk, dv = S_out.shape[-2], S_out.shape[-1]
+    BH = S_out.numel() // (dk * dv)
+    f = torch.float32
+    if n > M.shape[0] or n > Bp.shape[0]:
+        raise ValueError("n exceeds the number of pairs")
+    st = _lib.kda_affine_combine(_ptr(M, "M", f), _ptr(Bp, "Bp", f), int(n), _ptr(S0, "S0", f),
+                                 _ptr(S_out, "S_out", f), BH, dk, dv, _stream(stream))
+    if st != 0:
+        raise KdaError("kda_affine_combine", st)
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -> None:
@@ -301,6 +339,28 @@ def chunk_bwd(q, k, v, g, beta, S0, dout, dS_T=None, *, l2norm=True, complex_gat
              e(B, H, dk, dv) if want_dS0 else None)
     kda_chunk_bwd(q, k, v, g, beta, S0, dout, dS_T, *grads, opts, stream)
     return grads
+
+
+def segment_pair(q, k, v, g, beta, *, l2norm=True, complex_gate=False, fused=None,
+                 unbounded=False, stream=None):
+    """Allocate and run ``kda_segment_pair``; returns (M, B)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    kw = dict(l2norm=l2norm, complex_gate=complex_gate, fused=fused, unbounded=unbounded)
+    nbytes = kda_segment_pair_workspace_bytes(B, T, H, dk, dv, make_opts(q.dtype, **kw))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    M = torch.empty((B, H, dk, dk), dtype=torch.float32, device=q.device)
+    Bm = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    kda_segment_pair(q, k, v, g, beta, M, Bm, make_opts(q.dtype, workspace=ws, **kw), stream)
+    return M, Bm
+
+
+def affine_combine(Ms, Bs, n, S0=None, *, out=None, stream=None):
+    """Run ``kda_affine_combine`` over stacked pairs Ms [R,B,H,dk,dk], Bs [R,B,H,dk,dv]."""
+    if out is None:
+        out = torch.empty(Bs.shape[1:], dtype=torch.float32, device=Bs.device)
+    kda_affine_combine(Ms, Bs, n, S0, out, stream)
+    return out
 
 
 def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scale=1.0,

@@ -307,11 +307,51 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
 size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv,
                                      const kda_opts *opts);
 
+/*
+ * kda_segment_pair -- the affine pair of a segment of tokens (for splitting one long
+ * sequence over several GPUs: context parallelism over T).
+ *
+ * Page "Kimi K3 の KDA(1)", section 2.3 (the algebraic view): each token maps the
+ * state by S -> T_t S + beta_t k_t v_t^T, T_t = (I - beta_t k_t k_t^T) Diag(alpha_t),
+ * so a segment maps it by one affine pair S -> M S + B, and pairs compose in order.
+ * For the segment held in q, k, v, g, beta ([B,T,H,*], as kda_chunk_fwd) this writes
+ *
+ *   M_out [B,H,dk,dk] FP32   M = T_T ... T_1   (the final state from S0 = I, v = 0)
+ *   B_out [B,H,dk,dv] FP32   B = the final state from S0 = 0
+ *
+ * by two runs of the chunk forward (same paths, flags and tolerances as
+ * kda_chunk_fwd).  opts->workspace must hold kda_segment_pair_workspace_bytes(...):
+ * a zero v, the identity start state, a scratch output and the chunk workspace.
+ * T == 0 gives the identity pair (I, 0).
+ */
+int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
+                     const void *beta, float *M_out, float *B_out, int B, int T, int H,
+                     int dk, int dv, const kda_opts *opts, cudaStream_t stream);
+
+/* Workspace bytes kda_segment_pair needs. */
+size_t kda_segment_pair_workspace_bytes(int B, int T, int H, int dk, int dv,
+                                        const kda_opts *opts);
+
+/*
+ * kda_affine_combine -- fold the first n segment pairs onto a start state, in order:
+ * S <- M_r S + B_r for r = 0, ..., n-1 (same page and section as kda_segment_pair).
+ * With the pairs of segments 0..r-1 of a sequence this gives the state at the start of
+ * segment r; with all of them, the sequence's final state.
+ *
+ *   M  [n, BH, dk, dk] FP32,  Bp [n, BH, dk, dv] FP32  (BH independent sequences)
+ *   S0 [BH, dk, dv] FP32 start state, NULL means zero;  S_out [BH, dk, dv] FP32
+ *      (may be S0 itself).
+ * n == 0 copies S0 (or zeros) to S_out.  FP32 arithmetic on CUDA cores.
+ */
+int kda_affine_combine(const float *M, const float *Bp, int n, const float *S0,
+                       float *S_out, int BH, int dk, int dv, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
 /* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
-   1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd). */
+   1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd;
+   1.6: kda_segment_pair, kda_affine_combine). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -25,6 +25,8 @@ Functions
 ``recurrence_loops``  pure-Python loops, for tiny cases only.
 ``recurrence_bwd_np`` FP64 reverse-mode gradient of the token recurrence
                       (dq, dk, dv, dg, dbeta, dS0 from dO and dS_T).
+``transition_product_np``  dense product of a segment's per-token transitions.
+``affine_combine_np`` fold of (M, B) segment pairs onto a start state.
 ``chunkwise_np``      FP64 chunkwise-algebra form (cumulative decay, A_kk,
                       UT inverse, WY vectors, inter-chunk state update).
 ``conv_silu_np``      causal depthwise short convolution + SiLU.
@@ -213,6 +215,41 @@ def recurrence_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, l2norm=True,
     else:
         dq, dk_ = dqh, dkh
     return dq, dk_, dvv, dg, dbeta, dS
+
+
+def transition_product_np(k, g, beta, *, l2norm=True, complex_gate=False, eps=L2NORM_EPS):
+    """M = T_T ... T_2 T_1 with T_t = (I - beta_t k_t k_t^T) Diag(alpha_t), [B, H, dk, dk].
+
+    Kimi K3 KDA(1) section 2.3 (the algebraic view): every token acts on the state by the
+    affine map S -> T_t S + beta_t k_t v_t^T, and a segment of tokens composes to one
+    affine map S -> M S + B (the monoid of affine pairs), so a long sequence can be cut
+    into segments whose pairs are combined in order.  M is formed here as the explicit
+    product of dense dk x dk matrices; B is the segment's final state from S = 0.
+    """
+    k, g, beta = map(_f64, (k, g, beta))
+    B, T, H, dk = k.shape
+    if l2norm:
+        k = _normalise(k, eps)
+    alpha = g if complex_gate else np.exp(g)
+    M = np.broadcast_to(np.eye(dk), (B, H, dk, dk)).copy()
+    eye = np.eye(dk)
+    for t in range(T):
+        kt = k[:, t]
+        E = eye - beta[:, t, :, None, None] * kt[..., :, None] * kt[..., None, :]
+        Tt = E * alpha[:, t, :, None, :]            # (I - b k k^T) Diag(alpha): scale columns
+        M = np.einsum("bhij,bhjk->bhik", Tt, M)
+    return M
+
+
+def affine_combine_np(Ms, Bs, S0=None):
+    """Apply the segment pairs in order to a start state: S <- M_r S + B_r for
+    r = 0, 1, ..., returning S (Kimi K3 KDA(1) section 2.3, composition of affine pairs).
+    ``Ms``: [R, B, H, dk, dk]; ``Bs``: [R, B, H, dk, dv]; ``S0``: [B, H, dk, dv] or None."""
+    Ms, Bs = _f64(Ms), _f64(Bs)
+    S = np.zeros(Bs.shape[1:]) if S0 is None else _f64(S0).copy()
+    for M, Bm in zip(Ms, Bs):
+        S = np.einsum("bhij,bhjk->bhik", M, S) + Bm
+    return S
 
 
 def recurrence_loops(q, k, v, g, beta, S0=None, *, l2norm=True, complex_gate=False,

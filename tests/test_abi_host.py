@@ -36,7 +36,8 @@ def test_header_declares_the_entry_points():
     for n in ("kda_chunk_fwd", "kda_recurrent_step", "kda_chunk_fwd_prologue",
               "kda_recurrent_step_prologue", "kda_conv_state_from_prefill", "kda_chunk_fwd_gated",
               "kda_chunk_workspace_bytes", "kda_prologue_workspace_bytes", "kda_status_string",
-              "kda_abi_version", "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes"):
+              "kda_abi_version", "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes",
+              "kda_segment_pair", "kda_segment_pair_workspace_bytes", "kda_affine_combine"):
         assert n in names
 
 
@@ -47,7 +48,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 105   # 1.5: kda_chunk_bwd
+    assert kda.kda_abi_version() == 106   # 1.6: kda_segment_pair, kda_affine_combine
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
@@ -240,3 +241,29 @@ def test_chunk_bwd_host_checks(kda):
     assert call(opts=bad) == -1
     assert kda.kda_chunk_bwd_workspace_bytes(2, 33, 3, 128, 64, o) == 2 * 3 * 3 * 128 * 64 * 4
     assert kda.kda_chunk_bwd_workspace_bytes(1, 0, 3, 128, 128, o) == 0
+
+
+def test_segment_pair_and_combine_host_checks(kda):
+    """kda_segment_pair / kda_affine_combine argument checks before any CUDA call, and the
+    pair's workspace: zero v, identity start, scratch out, then the chunk workspace."""
+    import torch
+    vp = ctypes.c_void_p
+    o = kda.make_opts(torch.float32)
+    pair = lambda ptrs, T=64, dk=128, dv=128, opts=o: kda._lib.kda_segment_pair(
+        *[vp(p) for p in ptrs], 1, T, 2, dk, dv, ctypes.byref(opts), None)
+    good = [0x1000] * 7
+    assert pair(good[:5] + [0] + good[6:]) == -1           # M_out required
+    assert pair(good[:6] + [0x1008]) == -3                 # misaligned B_out
+    assert pair(good, dk=96) == -4
+    assert pair(good) == -7                                # needs a workspace
+    ws = kda.kda_segment_pair_workspace_bytes(1, 64, 2, 128, 128, o)
+    chunk = kda.kda_chunk_workspace_bytes(1, 64, 2, 128, 128, o)
+    assert ws >= 64 * 2 * 128 * 4 + 2 * 128 * 128 * 4 + 64 * 2 * 128 * 4 + chunk
+    comb = lambda M=0x1000, Bp=0x1000, n=2, S0=0x1000, out=0x1000, BH=3, dk=128, dv=128: \
+        kda._lib.kda_affine_combine(vp(M), vp(Bp), n, vp(S0), vp(out), BH, dk, dv, None)
+    assert comb(out=0) == -1
+    assert comb(M=0) == -1
+    assert comb(n=-1) == -1
+    assert comb(dv=32) == -4
+    assert comb(Bp=0x1004) == -3
+    assert comb(BH=0) == 0

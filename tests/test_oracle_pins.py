@@ -548,3 +548,42 @@ def test_backward_frozen_state_closed_form():
     per_t[-1] += Gam[-1] * np.sum(S * dST[0, 0], axis=1)
     want_g = np.cumsum(per_t[::-1], axis=0)[::-1]
     assert np.allclose(dg[0, :, 0], want_g, atol=1e-13)
+
+
+# ---------------------------------------------------------------- segments (affine pairs)
+@pytest.mark.parametrize("complex_gate", [False, True])
+def test_segment_pair_reproduces_the_recurrence(complex_gate):
+    """A segment acts on its start state as S -> M S + B: M from the dense transition
+    product, B = the recurrence's final state from S = 0; M S0 + B must equal the
+    recurrence run from S0, and M must equal the recurrence's final state from S0 = I
+    with v = 0 (each column of the state evolves on its own)."""
+    rng = np.random.default_rng(21 + int(complex_gate))
+    q, k, v, g, beta, S0 = _rand_case(rng, B=2, T=11, H=2, dk=4, dv=3, complex_gate=complex_gate)
+    M = oracle.transition_product_np(k, g, beta, complex_gate=complex_gate)
+    _, Bseg = oracle.recurrence_c(q, k, v, g, beta, None, complex_gate=complex_gate)
+    _, ST = oracle.recurrence_c(q, k, v, g, beta, S0, complex_gate=complex_gate)
+    assert _rel(np.einsum("bhij,bhjk->bhik", M, S0) + Bseg, ST) < RTOL
+    eye = np.broadcast_to(np.eye(4), (2, 2, 4, 4)).copy()
+    _, MI = oracle.recurrence_c(q, k, np.zeros((2, 11, 2, 4)), g, beta, eye,
+                                complex_gate=complex_gate)
+    assert _rel(M, MI) < RTOL
+
+
+def test_affine_combine_is_the_sequential_run():
+    """Cut one sequence into segments of lengths 5, 1, 7 and 3: folding the segments'
+    (M, B) pairs onto S0 gives the state after the whole sequence, every prefix fold gives
+    the state at that segment's start, and an empty fold returns S0."""
+    rng = np.random.default_rng(31)
+    q, k, v, g, beta, S0 = _rand_case(rng, B=1, T=16, H=2, dk=5, dv=3)
+    cuts = [0, 5, 6, 13, 16]
+    Ms, Bs = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        sl = lambda x: x[:, a:b]
+        Ms.append(oracle.transition_product_np(sl(k), sl(g), sl(beta)))
+        Bs.append(oracle.recurrence_c(sl(q), sl(k), sl(v), sl(g), sl(beta), None)[1])
+    for r, c in enumerate(cuts):
+        want = S0 if c == 0 else oracle.recurrence_c(q[:, :c], k[:, :c], v[:, :c], g[:, :c],
+                                                     beta[:, :c], S0)[1]
+        got = oracle.affine_combine_np(np.array(Ms[:r]).reshape(r, 1, 2, 5, 5),
+                                       np.array(Bs[:r]).reshape(r, 1, 2, 5, 3), S0)
+        assert _rel(got, want) < RTOL
