@@ -16,8 +16,9 @@
 //   Qg = Q e^gamma,  Kd = sigma_C K e^{gamma_C - gamma},  gC = sigma_C e^{gamma_C}
 // Every exponent above is <= 0, so nothing overflows in FP32.
 //
-// Phase 2 (one CTA per head and slice of value columns, chunks in order):
+// Phase 2 (one CTA per head and slice of 16 value columns, chunks in order):
 //   V~ = U - W S;   O = scale (Qg S + A_qk V~);   S <- diag(gC) S + Kd^T V~
+// as register-tiled products (2 x 2 and RPT x 2 outputs per thread) over shared memory.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -181,18 +182,39 @@ chunk_intra_kernel(const TQ *__restrict__ q, const TQ *__restrict__ k, const TQ 
         Vs[r * DVP + c] *= bs[r];
     }
     __syncthreads();
-    for (int idx = tid; idx < C * DK; idx += 256) {
-        const int r = idx / DK, c = idx % DK;
-        float acc = 0.f;
-        for (int i = 0; i <= r; ++i) acc += Tm[r * CP + i] * Qs[i * DKP + c];
-        wsb[L::off_W + idx] = acc;
-    }
-    for (int idx = tid; idx < C * DV; idx += 256) {
-        const int r = idx / DV, c = idx % DV;
-        float acc = 0.f;
-        for (int i = 0; i <= r; ++i) acc += Tm[r * CP + i] * Vs[i * DVP + c];
-        wsb[L::off_U + idx] = acc;
-    }
+    // W = Tm EK and U = Tm V as register tiles: thread = 4 rows (4 rg .. 4 rg + 3) x N / 16
+    // columns (cg, cg + 16, ...); Tm is zero above its diagonal, so the sum may run to the
+    // tile's last row.
+    auto tm_product = [&](const float *X, int ldx, int N, size_t off) {
+        const int rg = tid >> 4, cg = tid & 15;
+        const float *t0 = Tm + (4 * rg) * CP;
+        float acc[4][8];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[m][e] = 0.f;
+        const int ne = N / 16;
+        for (int i = 0; i <= 4 * rg + 3; ++i) {
+            const float a0 = t0[i], a1 = t0[CP + i], a2 = t0[2 * CP + i], a3 = t0[3 * CP + i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (e < ne) {
+                    const float x = X[i * ldx + cg + 16 * e];
+                    acc[0][e] = fmaf(a0, x, acc[0][e]);
+                    acc[1][e] = fmaf(a1, x, acc[1][e]);
+                    acc[2][e] = fmaf(a2, x, acc[2][e]);
+                    acc[3][e] = fmaf(a3, x, acc[3][e]);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (e < ne) wsb[off + (size_t)(4 * rg + m) * N + cg + 16 * e] = acc[m][e];
+    };
+    tm_product(Qs, DKP, DK, L::off_W);
+    tm_product(Vs, DVP, DV, L::off_U);
 }
 
 template <int DK, int DVS>
@@ -243,31 +265,80 @@ chunk_scan_kernel(const float *__restrict__ ws, const float *__restrict__ S0, TO
         for (int idx = tid; idx < C * C; idx += 256) Aq[(idx / C) * CP + idx % C] = wsb[L::off_A + idx];
         if (tid < DK) gCs[tid] = wsb[L::off_gC + tid];
         __syncthreads();
-        for (int idx = tid; idx < C * DVS; idx += 256) {
-            const int r = idx / DVS, j = idx % DVS;
-            float w = 0.f, o = 0.f;
+        // Register tiles: thread = (row pair 2rg, 2rg+1; column pair 2jg, 2jg+1) of the
+        // 64 x DVS products, and (RPT key rows, column pair) of the DK x DVS state update.
+        const int rg = tid >> 3, jg = tid & 7, ja = 2 * jg;
+        static_assert(DVS == 16, "the tiles cover 64 x 16 outputs with 256 threads");
+        {
+            // V~ = U - W S,  O = Qg S
+            float w[2][2] = {}, o[2][2] = {};
+            const float *w0 = Ws + (2 * rg) * DKP, *w1 = w0 + DKP;
+            const float *q0 = Qgs + (2 * rg) * DKP, *q1 = q0 + DKP;
+#pragma unroll 4
             for (int c = 0; c < DK; ++c) {
-                const float s = Ss[c * SP + j];
-                w += Ws[r * DKP + c] * s;
-                o += Qgs[r * DKP + c] * s;
+                const float s0 = Ss[c * SP + ja], s1 = Ss[c * SP + ja + 1];
+                const float a0 = w0[c], a1 = w1[c], b0 = q0[c], b1 = q1[c];
+                w[0][0] = fmaf(a0, s0, w[0][0]); w[0][1] = fmaf(a0, s1, w[0][1]);
+                w[1][0] = fmaf(a1, s0, w[1][0]); w[1][1] = fmaf(a1, s1, w[1][1]);
+                o[0][0] = fmaf(b0, s0, o[0][0]); o[0][1] = fmaf(b0, s1, o[0][1]);
+                o[1][0] = fmaf(b1, s0, o[1][0]); o[1][1] = fmaf(b1, s1, o[1][1]);
             }
-            Vt[r * SP + j] = Us[r * SP + j] - w;
-            Os[r * SP + j] = o;
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = 2 * rg + m, j = ja + e;
+                    Vt[r * SP + j] = Us[r * SP + j] - w[m][e];
+                    Os[r * SP + j] = o[m][e];
+                }
         }
         __syncthreads();
-        for (int idx = tid; idx < C * DVS; idx += 256) {
-            const int r = idx / DVS, j = idx % DVS;
-            if (r < n) {
-                float acc = Os[r * SP + j];
-                for (int i = 0; i <= r; ++i) acc += Aq[r * CP + i] * Vt[i * SP + j];
-                out[(((size_t)b * T + t0 + r) * H + h) * DV + j0 + j] = from_f32<TO>(scale * acc);
+        {
+            // out = scale (O + A_qk V~); A_qk is zero above the diagonal
+            float acc[2][2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) acc[m][e] = Os[(2 * rg + m) * SP + ja + e];
+            const float *a0 = Aq + (2 * rg) * CP, *a1 = a0 + CP;
+            for (int i = 0; i <= 2 * rg + 1; ++i) {
+                const float v0 = Vt[i * SP + ja], v1 = Vt[i * SP + ja + 1];
+                const float x0 = a0[i], x1 = a1[i];
+                acc[0][0] = fmaf(x0, v0, acc[0][0]); acc[0][1] = fmaf(x0, v1, acc[0][1]);
+                acc[1][0] = fmaf(x1, v0, acc[1][0]); acc[1][1] = fmaf(x1, v1, acc[1][1]);
+            }
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int r = 2 * rg + m;
+                if (r < n) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        out[(((size_t)b * T + t0 + r) * H + h) * DV + j0 + ja + e] = from_f32<TO>(scale * acc[m][e]);
+                }
             }
         }
-        for (int idx = tid; idx < DK * DVS; idx += 256) {
-            const int c = idx / DVS, j = idx % DVS;
-            float acc = gCs[c] * Ss[c * SP + j];
-            for (int r = 0; r < n; ++r) acc += Kds[r * DKP + c] * Vt[r * SP + j];
-            Ss[c * SP + j] = acc;
+        {
+            // S <- diag(gC) S + Kd^T V~ (each thread reads and writes only its own entries)
+            constexpr int RPT = DK / 32;
+            const int cb = RPT * rg;
+            float acc[RPT][2];
+#pragma unroll
+            for (int m = 0; m < RPT; ++m)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) acc[m][e] = gCs[cb + m] * Ss[(cb + m) * SP + ja + e];
+            for (int r = 0; r < n; ++r) {
+                const float v0 = Vt[r * SP + ja], v1 = Vt[r * SP + ja + 1];
+#pragma unroll
+                for (int m = 0; m < RPT; ++m) {
+                    const float kd = Kds[r * DKP + cb + m];
+                    acc[m][0] = fmaf(kd, v0, acc[m][0]);
+                    acc[m][1] = fmaf(kd, v1, acc[m][1]);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < RPT; ++m)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) Ss[(cb + m) * SP + ja + e] = acc[m][e];
         }
         __syncthreads();
     }
@@ -294,7 +365,7 @@ cudaError_t launch_intra(const ChunkArgs &a, int nchunks, float *ws, cudaStream_
 
 template <typename TO, int DK, int DV>
 cudaError_t launch_scan(const ChunkArgs &a, int nchunks, const float *ws, cudaStream_t st) {
-    constexpr int DVS = 32;
+    constexpr int DVS = 16;
     auto kern = chunk_scan_kernel<TO, DK, DV, DVS>;
     const size_t smem = scan_smem_bytes<DK, DVS>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
