@@ -282,6 +282,47 @@ def rows_n1(K, flush, hbm_peak):
         del gr, wsb, grads
         torch.cuda.empty_cache()
 
+        # context parallelism over T, emulated on one GPU: the prefill sequence cut into 4
+        # segments; each segment's pair (two forward runs), the fold and the forward from the
+        # folded state, timed per piece (on R GPUs the ranks run their pieces side by side)
+        R = 4
+        Ts = Tp // R
+        segs = [{n: x[n][:, r * Ts:(r + 1) * Ts].contiguous() for n in ("q", "k", "v", "g", "beta")}
+                for r in range(R)]
+        op = K.make_opts(torch.bfloat16)
+        wsp = torch.empty(K.kda_segment_pair_workspace_bytes(Bp, Ts, Hp, d, d, op), dtype=torch.uint8,
+                          device="cuda")
+        op = K.make_opts(torch.bfloat16, workspace=wsp)
+        Ms = torch.empty((R, Bp, Hp, d, d), dtype=torch.float32, device="cuda")
+        Bs = torch.empty((R, Bp, Hp, d, d), dtype=torch.float32, device="cuda")
+        fpair = lambda r: K.kda_segment_pair(*(segs[r][n] for n in ("q", "k", "v", "g", "beta")),
+                                             Ms[r], Bs[r], op)
+        for r in range(R):
+            fpair(r)
+        ms_pair = statistics.median(time_calls(lambda: fpair(R - 1), 5, flush))
+        S_start = torch.empty((Bp, Hp, d, d), dtype=torch.float32, device="cuda")
+        fcomb = lambda: K.kda_affine_combine(Ms, Bs, R - 1, x["S0"], S_start)
+        fcomb()
+        ms_comb = statistics.median(time_calls(fcomb, 5, flush))
+        wsf = torch.empty(max(K.kda_chunk_workspace_bytes(Bp, Ts, Hp, d, d, o1), 16), dtype=torch.uint8,
+                          device="cuda")
+        of = K.make_opts(torch.bfloat16, workspace=wsf)
+        outs = torch.empty((Bp, Ts, Hp, d), dtype=torch.bfloat16, device="cuda")
+        Sseg = torch.empty((Bp, Hp, d, d), dtype=torch.float32, device="cuda")
+        fseg = lambda: K.kda_chunk_fwd(*(segs[R - 1][n] for n in ("q", "k", "v", "g", "beta")), S_start,
+                                       outs, Sseg, of)
+        fseg()
+        ms_seg = statistics.median(time_calls(fseg, 5, flush))
+        pair_bytes = R * Bp * Hp * 2 * d * d * 4
+        rows["context_parallel_prefill_4_segments"] = {
+            "segment_T": Ts, "ms_segment_pair": ms_pair, "ms_fold": ms_comb, "ms_segment_forward": ms_seg,
+            "ms_per_rank_compute": ms_pair + ms_comb + ms_seg, "ms_whole_sequence_one_gpu": ms_p,
+            "all_gather_bytes": pair_bytes,
+            "note": "one GPU, pieces timed separately; per rank = pair + fold + forward of its 1024-token "
+                    "segment; the all-gather of the pairs (all_gather_bytes) is not timed here"}
+        del segs, wsp, Ms, Bs, S_start, wsf, outs, Sseg
+        torch.cuda.empty_cache()
+
         # unbounded decay (Kimi Linear softplus gate) on the prefill shape: exact-FP32 chunk path
         xs = W.chunk_inputs(Bp, Tp, Hp, d, d, dtype=torch.bfloat16, seed=0, gate="softplus")
         ou = K.make_opts(torch.bfloat16, unbounded=True)
@@ -294,9 +335,15 @@ def rows_n1(K, flush, hbm_peak):
                                      Su, ou)
         fu()
         ms_u = statistics.median(time_calls(fu, 5, flush))
+        evu = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        flush.zero_()
+        K.kda_chunk_fwd(xs["q"], xs["k"], xs["v"], xs["g"], xs["beta"], xs["S0"], outu, Su,
+                        K.make_opts(torch.bfloat16, unbounded=True, workspace=wsu, events=evu))
+        torch.cuda.synchronize()
         nbu = th * token_head_bytes(d) + Bp * Hp * 2 * d * d * 4
         rows["prefill_softplus_gate"] = {
             "ms": ms_u, "tokens_per_s": Bp * Tp / (ms_u * 1e-3),
+            "ms_intra_kernel": evu[0].elapsed_time(evu[1]), "ms_scan_kernel": evu[1].elapsed_time(evu[2]),
             "frac_of_hbm_roofline": (nbu / (ms_u * 1e-3) / 1e9) / hbm_peak,
             "note": "kda_chunk_fwd with KDA_UNBOUNDED_DECAY (exact-FP32 path), softplus-gate inputs"}
         del x, xs, wsu, outu, Su
@@ -471,24 +518,81 @@ def run_ours(args, ws, rank, local):
                         "whole_call_* = the same bytes / the call's device time; "
                         "traffic = DRAM bytes of that kernel per launch (ncu)"}
 
-    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hS = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region.
+    # Every step copies its inputs host -> device, runs the call and reads out and S_T back.
+    # Pipelined as a serving loop would run it: the copy-in of step i+1, the call of step i and
+    # the copy-out of step i-1 overlap on three streams, with device inputs and outputs
+    # double-buffered.  The serialised form (copy, call, copy on one stream) is kept beside it.
+    cs = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    dbuf = [d, {n: torch.empty_like(d[n]) for n in names}]
+    obuf = [(out, S_T), (torch.empty_like(out), torch.empty_like(S_T))]
+    hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    hS = [torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() for _ in range(2)]
+
+    def call_on(dd, oo):
+        o = K.make_opts(torch.bfloat16, workspace=wsb)
+        K.kda_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], oo[0], oo[1], o)
+
+    def e2e_pipelined(nsteps):
+        ev_in = [torch.cuda.Event() for _ in range(nsteps)]
+        ev_call = [torch.cuda.Event() for _ in range(nsteps)]
+        ev_out = [torch.cuda.Event() for _ in range(nsteps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(cs)
+        s_in.wait_event(t0)
+        s_out.wait_event(t0)
+        for i in range(nsteps):
+            bi = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_call[i - 2])          # the call of step i-2 read dbuf[bi]
+                for n in names:
+                    dbuf[bi][n].copy_(host[n], non_blocking=True)
+                ev_in[i].record(s_in)
+            cs.wait_event(ev_in[i])
+            if i >= 2:
+                cs.wait_event(ev_out[i - 2])                 # obuf[bi] has been read back
+            call_on(dbuf[bi], obuf[bi])
+            ev_call[i].record(cs)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_call[i])
+                hout[bi].copy_(obuf[bi][0], non_blocking=True)
+                hS[bi].copy_(obuf[bi][1], non_blocking=True)
+                ev_out[i].record(s_out)
+        cs.wait_event(ev_in[nsteps - 1])
+        cs.wait_event(ev_out[nsteps - 1])
+        t1.record(cs)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
 
     def e2e_step():
         for n in names:
             d[n].copy_(host[n], non_blocking=True)
         call()
-        hout.copy_(out, non_blocking=True)
-        hS.copy_(S_T, non_blocking=True)
+        hout[0].copy_(out, non_blocking=True)
+        hS[0].copy_(S_T, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize()
-    e2e_ms = time_calls(e2e_step, args.steps, flush)
-    e2e_max = max_over_ranks(sum(e2e_ms), ws)
+    ref_out, ref_S = hout[0].clone(), hS[0].clone()
+    e2e_serial_ms = time_calls(e2e_step, args.steps, flush)
+    e2e_pipelined(3)
+    e2e_ms = e2e_pipelined(args.steps)
+    last = (args.steps - 1) % 2
+    close = lambda a, b: float((a.float() - b.float()).abs().max()) <= 1e-3 * float(b.float().abs().max())
+    e2e_ok = bool(close(hout[last], ref_out) and close(hS[last], ref_S))
+    e2e_max = max_over_ranks(e2e_ms, ws)
+    e2e_serial_max = max_over_ranks(sum(e2e_serial_ms), ws)
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-    d2h = hout.numel() * hout.element_size() + hS.numel() * hS.element_size()
+    d2h = hout[0].numel() * hout[0].element_size() + hS[0].numel() * hS[0].element_size()
     e2e = {"value": ws * tokens_per_step * args.steps / (e2e_max * 1e-3), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_max / args.steps, "outputs_match_serial": e2e_ok,
+           "serial_value": ws * tokens_per_step * args.steps / (e2e_serial_max * 1e-3),
+           "note": "pipelined over three streams (copy-in of step i+1, call i, copy-out of "
+                   "step i-1), every step's copies inside the timed region; serial_value = one "
+                   "stream, L2 flushed between steps"}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

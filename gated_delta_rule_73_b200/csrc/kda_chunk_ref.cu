@@ -252,18 +252,45 @@ chunk_scan_kernel(const float *__restrict__ ws, const float *__restrict__ S0, TO
         const int t0 = ch * C;
         const int n = min(C, T - t0);
         const float *wsb = ws + ((size_t)bh * nchunks + ch) * L::per_chunk;
-        for (int idx = tid; idx < C * DK; idx += 256) {
-            const int r = idx / DK, c = idx % DK;
-            Ws[r * DKP + c] = wsb[L::off_W + idx];
-            Qgs[r * DKP + c] = wsb[L::off_Qg + idx];
-            Kds[r * DKP + c] = wsb[L::off_Kd + idx];
+        {
+            // the chunk's record: every 16-byte load of a matrix is issued before any of its
+            // stores, so each thread keeps NV loads of three matrices in flight (offsets and the
+            // record size are multiples of 4 floats, so every float4 is aligned)
+            constexpr int NV = C * DK / 4 / 256;
+            const float4 *w4 = reinterpret_cast<const float4 *>(wsb + L::off_W);
+            const float4 *q4 = reinterpret_cast<const float4 *>(wsb + L::off_Qg);
+            const float4 *k4 = reinterpret_cast<const float4 *>(wsb + L::off_Kd);
+            float4 a[NV], bq[NV], bk[NV];
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                a[m] = w4[tid + 256 * m];
+                bq[m] = q4[tid + 256 * m];
+                bk[m] = k4[tid + 256 * m];
+            }
+            const int ur = tid >> 2, up = tid & 3;                  // U: 64 rows x 16 columns
+            const float4 u = *reinterpret_cast<const float4 *>(wsb + L::off_U + (size_t)ur * DV + j0 + 4 * up);
+            float4 av[4];
+            const float4 *a4 = reinterpret_cast<const float4 *>(wsb + L::off_A);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) av[m] = a4[tid + 256 * m];
+#pragma unroll
+            for (int m = 0; m < NV; ++m) {
+                const int e0 = 4 * (tid + 256 * m), r = e0 / DK, c = e0 % DK;
+                float *dw = Ws + r * DKP + c, *dq = Qgs + r * DKP + c, *dk = Kds + r * DKP + c;
+                dw[0] = a[m].x; dw[1] = a[m].y; dw[2] = a[m].z; dw[3] = a[m].w;
+                dq[0] = bq[m].x; dq[1] = bq[m].y; dq[2] = bq[m].z; dq[3] = bq[m].w;
+                dk[0] = bk[m].x; dk[1] = bk[m].y; dk[2] = bk[m].z; dk[3] = bk[m].w;
+            }
+            float *du = Us + ur * SP + 4 * up;
+            du[0] = u.x; du[1] = u.y; du[2] = u.z; du[3] = u.w;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int e0 = 4 * (tid + 256 * m), r = e0 / C, c = e0 % C;
+                float *da = Aq + r * CP + c;
+                da[0] = av[m].x; da[1] = av[m].y; da[2] = av[m].z; da[3] = av[m].w;
+            }
+            if (tid < DK) gCs[tid] = wsb[L::off_gC + tid];
         }
-        for (int idx = tid; idx < C * DVS; idx += 256) {
-            const int r = idx / DVS, j = idx % DVS;
-            Us[r * SP + j] = wsb[L::off_U + (size_t)r * DV + j0 + j];
-        }
-        for (int idx = tid; idx < C * C; idx += 256) Aq[(idx / C) * CP + idx % C] = wsb[L::off_A + idx];
-        if (tid < DK) gCs[tid] = wsb[L::off_gC + tid];
         __syncthreads();
         // Register tiles: thread = (row pair 2rg, 2rg+1; column pair 2jg, 2jg+1) of the
         // 64 x DVS products, and (RPT key rows, column pair) of the DK x DVS state update.

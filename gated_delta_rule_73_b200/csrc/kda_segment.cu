@@ -13,9 +13,9 @@
 //    Both runs are the chunk forward itself (kda_abi.cu).
 //  * affine_combine_kernel folds pairs onto a start state: S <- M_r S + B_r, r = 0..n-1.
 //    One CTA per (sequence, 32 value columns): its slice of S stays in shared memory
-//    (double-buffered); thread = (value column, 16 key rows); rows of M_r are read by the
-//    whole warp at once (a broadcast).  n is small (the number of segments), so this is a
-//    few 128^3 products per sequence.
+//    (double-buffered); each M_r is staged transposed in shared memory by coalesced reads;
+//    thread = 4 (or 2) key rows x 4 value columns, two 16-byte shared loads per 16 FMAs.
+//    n is small (the number of segments), so this is a few 128^3 products per sequence.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -33,42 +33,77 @@ identity_kernel(float *__restrict__ S, long long total, int d) {
 
 constexpr int CW = 32;    // value columns per CTA
 
+// Shared memory of one fold CTA: M_r transposed ([c][i], rows padded to keep float4 reads
+// aligned and the transposing writes at most 4-way conflicted) and the state slice, twice.
+template <int DK>
+struct FoldSmem {
+    static constexpr int MP = DK + 4;
+    float mt[DK][MP];
+    float sb[2][DK][CW];
+};
+
 template <int DK>
 __global__ void __launch_bounds__(256)
 affine_combine_kernel(const float *__restrict__ M, const float *__restrict__ Bp, int n,
                       const float *__restrict__ S0, float *__restrict__ S_out, int BH, int dv) {
-    constexpr int RPT = DK / 8;              // key rows per thread (8 warps)
-    __shared__ float sb[2][DK][CW];
+    // thread = 4 x 4 tile: key rows 4 rg .. 4 rg + 3 (RG groups), value columns 4 cg .. 4 cg + 3
+    constexpr int MP = FoldSmem<DK>::MP;
+    constexpr int RPT = DK / 32;             // rows per thread: 4 (DK = 128) or 2 (DK = 64)
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    FoldSmem<DK> &sm = *reinterpret_cast<FoldSmem<DK> *>(smem_raw);
     const int bh = blockIdx.x, j0 = blockIdx.y * CW;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int tid = threadIdx.x, rg = tid >> 3, cg = tid & 7;
+    const int i0 = RPT * rg, c4 = 4 * cg;
     const size_t sbase = (size_t)bh * DK * dv;
-#pragma unroll
-    for (int m = 0; m < RPT; ++m) {
-        const int i = w + 8 * m;
-        sb[0][i][lane] = S0 ? S0[sbase + (size_t)i * dv + j0 + lane] : 0.f;
+    for (int idx = tid; idx < DK * CW; idx += 256) {
+        const int i = idx / CW, j = idx % CW;
+        sm.sb[0][i][j] = S0 ? S0[sbase + (size_t)i * dv + j0 + j] : 0.f;
     }
-    __syncthreads();
     int cur = 0;
     for (int r = 0; r < n; ++r) {
         const float *Mr = M + ((size_t)r * BH + bh) * DK * DK;
         const float *Br = Bp + ((size_t)r * BH + bh) * DK * dv;
-        float acc[RPT];
+        __syncthreads();   // the previous step's reads of mt are done
+        for (int idx = tid; idx < DK * DK; idx += 256) {
+            const int i = idx / DK, c = idx % DK;      // coalesced read of row i
+            sm.mt[c][i] = Mr[idx];
+        }
+        __syncthreads();
+        float acc[RPT][4];
 #pragma unroll
-        for (int m = 0; m < RPT; ++m) acc[m] = Br[(size_t)(w + 8 * m) * dv + j0 + lane];
+        for (int m = 0; m < RPT; ++m) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(&Br[(size_t)(i0 + m) * dv + j0 + c4]);
+            acc[m][0] = b4.x; acc[m][1] = b4.y; acc[m][2] = b4.z; acc[m][3] = b4.w;
+        }
+#pragma unroll 4
         for (int c = 0; c < DK; ++c) {
-            const float s = sb[cur][c][lane];
+            const float4 s4 = *reinterpret_cast<const float4 *>(&sm.sb[cur][c][c4]);
+            float mv[RPT];
+            if constexpr (RPT == 4) {
+                const float4 m4 = *reinterpret_cast<const float4 *>(&sm.mt[c][i0]);
+                mv[0] = m4.x; mv[1] = m4.y; mv[2] = m4.z; mv[3] = m4.w;
+            } else {
+                const float2 m2 = *reinterpret_cast<const float2 *>(&sm.mt[c][i0]);
+                mv[0] = m2.x; mv[1] = m2.y;
+            }
 #pragma unroll
-            for (int m = 0; m < RPT; ++m) acc[m] = fmaf(__ldg(&Mr[(size_t)(w + 8 * m) * DK + c]), s, acc[m]);
+            for (int m = 0; m < RPT; ++m) {
+                acc[m][0] = fmaf(mv[m], s4.x, acc[m][0]);
+                acc[m][1] = fmaf(mv[m], s4.y, acc[m][1]);
+                acc[m][2] = fmaf(mv[m], s4.z, acc[m][2]);
+                acc[m][3] = fmaf(mv[m], s4.w, acc[m][3]);
+            }
         }
 #pragma unroll
-        for (int m = 0; m < RPT; ++m) sb[cur ^ 1][w + 8 * m][lane] = acc[m];
+        for (int m = 0; m < RPT; ++m)
+            *reinterpret_cast<float4 *>(&sm.sb[cur ^ 1][i0 + m][c4]) =
+                make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
         cur ^= 1;
-        __syncthreads();
     }
-#pragma unroll
-    for (int m = 0; m < RPT; ++m) {
-        const int i = w + 8 * m;
-        S_out[sbase + (size_t)i * dv + j0 + lane] = sb[cur][i][lane];
+    __syncthreads();
+    for (int idx = tid; idx < DK * CW; idx += 256) {
+        const int i = idx / CW, j = idx % CW;
+        S_out[sbase + (size_t)i * dv + j0 + j] = sm.sb[cur][i][j];
     }
 }
 
@@ -81,14 +116,22 @@ cudaError_t launch_identity(float *S, long long count, int d, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <int DK>
+static cudaError_t launch_fold(const float *M, const float *Bp, int n, const float *S0, float *S_out,
+                               int BH, int dv, cudaStream_t st) {
+    const size_t smem = sizeof(FoldSmem<DK>);
+    cudaError_t e = cudaFuncSetAttribute(affine_combine_kernel<DK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)BH, (unsigned)(dv / CW));
+    affine_combine_kernel<DK><<<grid, 256, smem, st>>>(M, Bp, n, S0, S_out, BH, dv);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_affine_combine(const float *M, const float *Bp, int n, const float *S0, float *S_out,
                                   int BH, int dk, int dv, cudaStream_t st) {
-    const dim3 grid((unsigned)BH, (unsigned)(dv / CW));
-    if (dk == 128)
-        affine_combine_kernel<128><<<grid, 256, 0, st>>>(M, Bp, n, S0, S_out, BH, dv);
-    else
-        affine_combine_kernel<64><<<grid, 256, 0, st>>>(M, Bp, n, S0, S_out, BH, dv);
-    return cudaGetLastError();
+    return dk == 128 ? launch_fold<128>(M, Bp, n, S0, S_out, BH, dv, st)
+                     : launch_fold<64>(M, Bp, n, S0, S_out, BH, dv, st);
 }
 
 }  // namespace kda
