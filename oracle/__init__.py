@@ -25,6 +25,9 @@ Functions
 ``recurrence_loops``  pure-Python loops, for tiny cases only.
 ``recurrence_bwd_np`` FP64 reverse-mode gradient of the token recurrence
                       (dq, dk, dv, dg, dbeta, dS0 from dO and dS_T).
+``chunkwise_bwd_np``  the same gradient through the chunkwise form: a reverse scan
+                      of dS over chunks, then the WY / UT and decay derivatives
+                      inside each chunk.
 ``transition_product_np``  dense product of a segment's per-token transitions.
 ``affine_combine_np`` fold of (M, B) segment pairs onto a start state.
 ``chunkwise_np``      FP64 chunkwise-algebra form (cumulative decay, A_kk,
@@ -215,6 +218,112 @@ def recurrence_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, l2norm=True,
     else:
         dq, dk_ = dqh, dkh
     return dq, dk_, dvv, dg, dbeta, dS
+
+
+def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
+                     complex_gate=False, scale=1.0, eps=L2NORM_EPS):
+    """FP64 gradient of ``L = <dO, O> + <dS_T, S_T>`` through the chunkwise form of
+    :func:`chunkwise_np`; returns what :func:`recurrence_bwd_np` returns.
+
+    Kimi K3 structure (2), Q&A items on the chunkwise algorithm (training runs this form).
+    Per chunk, with the forward's Gamma, Kg = K*Gamma, Ki = K/Gamma, Qg = Q*Gamma,
+    A_kk, Tm = (I + A_kk)^{-1}, X = diag(beta) Kg, Y = diag(beta) V, W = Tm X, U = Tm Y,
+    V~ = U - W S, A_qk = tril(Qg Ki^T), Kd = K * Gamma_C / Gamma, the adjoint steps are,
+    chunks in reverse (dS' = the gradient at the chunk's end, dO scaled by ``scale``):
+
+      dV~ = A_qk^T dO + Kd dS'
+      dS  = diag(Gamma_C) dS' + Qg^T dO - W^T dV~          (to the previous chunk)
+      dA_qk = tril(dO V~^T),  dW = -dV~ S^T,  dU = dV~,  dKd = V~ dS'^T
+      dX = Tm^T dW,  dY = Tm^T dU,  dA_kk = strict_tril(-Tm^T (dW X^T + dU Y^T) Tm^T)
+
+    then the products back to Q, K, V, beta and Gamma, Gamma_C = Gamma[last], and
+    Gamma = cumprod(alpha) (dg_s = sum_{r >= s} dGamma_r Gamma_r / alpha_s * dalpha_s/dg_s).
+    FP64 holds exp(+-320), so the plain K / Gamma is used, as in the forward.
+    """
+    q, k, v, g, beta, dO = map(_f64, (q, k, v, g, beta, dO))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if l2norm:
+        nq = np.sqrt(np.sum(q * q, axis=-1, keepdims=True) + eps)
+        nk = np.sqrt(np.sum(k * k, axis=-1, keepdims=True) + eps)
+        qh, kh = q / nq, k / nk
+    else:
+        qh, kh = q, k
+    alpha = g if complex_gate else np.exp(g)
+    dqh, dkh, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dalpha, dbeta = np.zeros_like(g), np.zeros_like(beta)
+    dS0 = np.zeros((B, H, dk, dv))
+    starts = list(range(0, T, C))
+    for b in range(B):
+        for h in range(H):
+            # forward, keeping each chunk's start state
+            S = np.zeros((dk, dv)) if S0 is None else _f64(S0)[b, h].copy()
+            states = []
+            for s in starts:
+                e = min(s + C, T)
+                states.append(S)
+                Q, K, V = qh[b, s:e, h], kh[b, s:e, h], v[b, s:e, h]
+                bt = beta[b, s:e, h]
+                Gam = np.cumprod(alpha[b, s:e, h], axis=0)
+                Kg, Ki = K * Gam, K / Gam
+                Akk = np.tril(bt[:, None] * (Kg @ Ki.T), -1)
+                Tm = np.linalg.inv(np.eye(e - s) + Akk)
+                Vt = Tm @ (bt[:, None] * V) - Tm @ (bt[:, None] * Kg) @ S
+                GC = Gam[-1]
+                S = GC[:, None] * S + (K * (GC[None, :] / Gam)).T @ Vt
+            dS = np.zeros((dk, dv)) if dS_T is None else _f64(dS_T)[b, h].copy()
+            for s, S in zip(reversed(starts), reversed(states)):
+                e = min(s + C, T)
+                n = e - s
+                Q, K, V = qh[b, s:e, h], kh[b, s:e, h], v[b, s:e, h]
+                bt = beta[b, s:e, h]
+                al = alpha[b, s:e, h]
+                Gam = np.cumprod(al, axis=0)
+                GC = Gam[-1]
+                Kg, Ki, Qg = K * Gam, K / Gam, Q * Gam
+                KK = Kg @ Ki.T
+                Akk = np.tril(bt[:, None] * KK, -1)
+                Tm = np.linalg.inv(np.eye(n) + Akk)
+                X, Y = bt[:, None] * Kg, bt[:, None] * V
+                W, U = Tm @ X, Tm @ Y
+                Vt = U - W @ S
+                Aqk = np.tril(Qg @ Ki.T)
+                Kd = K * (GC[None, :] / Gam)
+                dOs = scale * dO[b, s:e, h]
+                # adjoint of the chunk
+                dVt = Aqk.T @ dOs + Kd @ dS
+                dS_prev = GC[:, None] * dS + Qg.T @ dOs - W.T @ dVt
+                dAqk = np.tril(dOs @ Vt.T)
+                dQg = dOs @ S.T + dAqk @ Ki
+                dKi = dAqk.T @ Qg
+                dW, dU = -dVt @ S.T, dVt
+                dKd = Vt @ dS.T
+                dGC = np.sum(S * dS, axis=1) + np.sum(K / Gam * dKd, axis=0)
+                dX, dY = Tm.T @ dW, Tm.T @ dU
+                dTm = dW @ X.T + dU @ Y.T
+                dAkk = np.tril(-Tm.T @ dTm @ Tm.T, -1)
+                bA = bt[:, None] * dAkk
+                dKg = bA @ Ki + bt[:, None] * dX
+                dKi = dKi + bA.T @ Kg
+                dbeta[b, s:e, h] = (np.sum(dAkk * KK, axis=1) + np.sum(Kg * dX, axis=1)
+                                    + np.sum(V * dY, axis=1))
+                dvv[b, s:e, h] = bt[:, None] * dY
+                dqh[b, s:e, h] = Gam * dQg
+                dkh[b, s:e, h] = Gam * dKg + dKi / Gam + (GC[None, :] / Gam) * dKd
+                dGam = Q * dQg + K * dKg - Ki * dKi / Gam - Kd * dKd / Gam
+                dGam[-1] += dGC
+                # Gamma_r = prod_{s <= r} alpha_s:  dalpha_s = sum_{r >= s} dGam_r Gamma_r / alpha_s
+                rc = np.cumsum((dGam * Gam)[::-1], axis=0)[::-1]
+                dalpha[b, s:e, h] = rc / al
+                dS = dS_prev
+            dS0[b, h] = dS
+    dg = dalpha if complex_gate else alpha * dalpha
+    if l2norm:
+        dq = (dqh - qh * np.sum(qh * dqh, axis=-1, keepdims=True)) / nq
+        dk_ = (dkh - kh * np.sum(kh * dkh, axis=-1, keepdims=True)) / nk
+    else:
+        dq, dk_ = dqh, dkh
+    return dq, dk_, dvv, dg, dbeta, dS0
 
 
 def transition_product_np(k, g, beta, *, l2norm=True, complex_gate=False, eps=L2NORM_EPS):

@@ -587,3 +587,20 @@ def test_affine_combine_is_the_sequential_run():
         got = oracle.affine_combine_np(np.array(Ms[:r]).reshape(r, 1, 2, 5, 5),
                                        np.array(Bs[:r]).reshape(r, 1, 2, 5, 3), S0)
         assert _rel(got, want) < RTOL
+
+
+@pytest.mark.parametrize("C", [4, 5, 16])
+@pytest.mark.parametrize("complex_gate,l2norm", [(False, True), (False, False), (True, True)])
+def test_chunkwise_backward_equals_recurrence_backward(C, complex_gate, l2norm):
+    """The gradient through the chunkwise form (reverse scan of dS over chunks, WY / UT and
+    decay derivatives inside each chunk) equals the token-level reverse pass (itself pinned
+    by finite differences above), with ragged last chunks and scale != 1."""
+    rng = np.random.default_rng(40 + C + 3 * int(complex_gate) + int(l2norm))
+    q, k, v, g, beta, S0 = _rand_case(rng, B=2, T=13, H=2, dk=5, dv=3, complex_gate=complex_gate)
+    dO = rng.standard_normal((2, 13, 2, 3))
+    dST = rng.standard_normal((2, 2, 5, 3))
+    kw = dict(complex_gate=complex_gate, l2norm=l2norm, scale=0.8)
+    ref = oracle.recurrence_bwd_np(q, k, v, g, beta, S0, dO, dST, **kw)
+    got = oracle.chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dST, C=C, **kw)
+    for a, b in zip(got, ref):
+        assert _rel(a, b) < 1e-12
