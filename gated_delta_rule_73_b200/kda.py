@@ -138,6 +138,17 @@ def _ptr(t, name, dtype=None, device_required=True):
     return t.data_ptr()
 
 
+def _shapes(**named):
+    """Check every tensor against the shape the C call will assume (None = optional, absent).
+    The library receives raw pointers and sizes only, so a mismatch here would otherwise
+    become an out-of-bounds device access."""
+    for name, (t, shape) in named.items():
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -157,6 +168,8 @@ def kda_chunk_fwd(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
+    _shapes(k=(k, q.shape), g=(g, q.shape), v=(v, (B, T, H, dv)), beta=(beta, (B, T, H)),
+            S0=(S0, (B, H, dk, dv)), out=(out, (B, T, H, dv)), S_T=(S_T, (B, H, dk, dv)))
     args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
             _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
             _ptr(S_T, "S_T", torch.float32)]
@@ -176,6 +189,10 @@ def kda_chunk_bwd(q, k, v, g, beta, S0, dout, dS_T, grad_q, grad_k, grad_v, grad
     dv = v.shape[-1]
     dt = q.dtype
     f = torch.float32
+    sq, sv, sS = (B, T, H, dk), (B, T, H, dv), (B, H, dk, dv)
+    _shapes(k=(k, sq), g=(g, sq), v=(v, sv), beta=(beta, (B, T, H)), S0=(S0, sS), dout=(dout, sv),
+            dS_T=(dS_T, sS), grad_q=(grad_q, sq), grad_k=(grad_k, sq), grad_v=(grad_v, sv),
+            grad_g=(grad_g, sq), grad_beta=(grad_beta, (B, T, H)), grad_S0=(grad_S0, sS))
     args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
             _ptr(beta, "beta", dt), _ptr(S0, "S0", f), _ptr(dout, "dout", dt), _ptr(dS_T, "dS_T", f),
             _ptr(grad_q, "grad_q", f), _ptr(grad_k, "grad_k", f), _ptr(grad_v, "grad_v", f),
@@ -196,6 +213,8 @@ def kda_segment_pair(q, k, v, g, beta, M_out, B_out, opts: kda_opts, stream=None
     dv = v.shape[-1]
     dt = q.dtype
     f = torch.float32
+    _shapes(k=(k, q.shape), g=(g, q.shape), v=(v, (B, T, H, dv)), beta=(beta, (B, T, H)),
+            M_out=(M_out, (B, H, dk, dk)), B_out=(B_out, (B, H, dk, dv)))
     args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
             _ptr(beta, "beta", dt), _ptr(M_out, "M_out", f), _ptr(B_out, "B_out", f)]
     st = _lib.kda_segment_pair(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
@@ -209,8 +228,13 @@ def kda_affine_combine(M, Bp, n, S0, S_out, stream=None) -> None:
     dk, dv = S_out.shape[-2], S_out.shape[-1]
     BH = S_out.numel() // (dk * dv)
     f = torch.float32
-    if n > M.shape[0] or n > Bp.shape[0]:
-        raise ValueError("n exceeds the number of pairs")
+    R = M.shape[0]
+    if Bp.shape[0] != R or not 0 <= n <= R:
+        raise ValueError("M and Bp must stack the same number of pairs R, and 0 <= n <= R")
+    if M.numel() != R * BH * dk * dk or Bp.numel() != R * BH * dk * dv:
+        raise ValueError(f"M must hold [R, {BH}, {dk}, {dk}] and Bp [R, {BH}, {dk}, {dv}] values")
+    if S0 is not None and S0.numel() != BH * dk * dv:
+        raise ValueError("S0 must have the shape of S_out")
     st = _lib.kda_affine_combine(_ptr(M, "M", f), _ptr(Bp, "Bp", f), int(n), _ptr(S0, "S0", f),
                                  _ptr(S_out, "S_out", f), BH, dk, dv, _stream(stream))
     if st != 0:
@@ -223,6 +247,8 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
+    _shapes(k=(k, q.shape), g=(g, q.shape), v=(v, (B, T, H, dv)), beta=(beta, (B, T, H)),
+            S0=(S0, (B, H, dk, dv)), out=(out, (B, T, H, dv)), S_T=(S_T, (B, H, dk, dv)))
     args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
             _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
             _ptr(S_T, "S_T", torch.float32)]
@@ -236,6 +262,8 @@ def kda_recurrent_step(q, k, v, g, beta, S, out, opts: kda_opts, stream=None) ->
     N, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
+    _shapes(k=(k, q.shape), g=(g, q.shape), v=(v, (N, H, dv)), beta=(beta, (N, H)),
+            S=(S, (N, H, dk, dv)), out=(out, (N, H, dv)))
     args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
             _ptr(beta, "beta", dt), _ptr(S, "S", torch.float32), _ptr(out, "out", dt)]
     st = _lib.kda_recurrent_step(*args, N, H, dk, dv, ctypes.byref(opts), _stream(stream))
@@ -249,6 +277,9 @@ def kda_chunk_fwd_prologue(q_pre, k_pre, v_pre, conv_w, z, A, beta_logit, S0, ou
     B, T, H, dk = q_pre.shape
     dv = v_pre.shape[-1]
     dt = q_pre.dtype
+    _shapes(k_pre=(k_pre, q_pre.shape), z=(z, q_pre.shape), v_pre=(v_pre, (B, T, H, dv)),
+            conv_w=(conv_w, (3, H * dk, 4)), A=(A, (H,)), beta_logit=(beta_logit, (B, T, H)),
+            S0=(S0, (B, H, dk, dv)), out=(out, (B, T, H, dv)), S_T=(S_T, (B, H, dk, dv)))
     args = [_ptr(q_pre, "q_pre", dt), _ptr(k_pre, "k_pre", dt), _ptr(v_pre, "v_pre", dt),
             _ptr(conv_w, "conv_w", dt), _ptr(z, "z", dt), _ptr(A, "A", torch.float32),
             _ptr(beta_logit, "beta_logit", torch.float32), _ptr(S0, "S0", torch.float32),
@@ -264,6 +295,9 @@ def kda_chunk_fwd_gated(q, k, v, g, beta, S0, out, S_T, out_gate, norm_weight, n
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
+    _shapes(k=(k, q.shape), g=(g, q.shape), v=(v, (B, T, H, dv)), beta=(beta, (B, T, H)),
+            S0=(S0, (B, H, dk, dv)), out=(out, (B, T, H, dv)), S_T=(S_T, (B, H, dk, dv)),
+            out_gate=(out_gate, (B, T, H, dv)), norm_weight=(norm_weight, (dv,)))
     args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
             _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
             _ptr(S_T, "S_T", torch.float32), _ptr(out_gate, "out_gate", dt),
@@ -281,6 +315,10 @@ def kda_recurrent_step_prologue(q_pre, k_pre, v_pre, conv_w, conv_state, z, A, b
     N, H, dk = q_pre.shape
     dv = v_pre.shape[-1]
     dt = q_pre.dtype
+    _shapes(k_pre=(k_pre, q_pre.shape), z=(z, q_pre.shape), v_pre=(v_pre, (N, H, dv)),
+            conv_w=(conv_w, (3, H * dk, 4)), conv_state=(conv_state, (N, 3, 3, H * dk)),
+            A=(A, (H,)), beta_logit=(beta_logit, (N, H)), S=(S, (N, H, dk, dv)),
+            out=(out, (N, H, dv)))
     args = [_ptr(q_pre, "q_pre", dt), _ptr(k_pre, "k_pre", dt), _ptr(v_pre, "v_pre", dt),
             _ptr(conv_w, "conv_w", dt), _ptr(conv_state, "conv_state", dt), _ptr(z, "z", dt),
             _ptr(A, "A", torch.float32), _ptr(beta_logit, "beta_logit", torch.float32),
@@ -294,6 +332,8 @@ def kda_conv_state_from_prefill(q_pre, k_pre, v_pre, conv_state, opts: kda_opts,
     """Call ``kda_conv_state_from_prefill``: raw inputs [B,T,H,d] -> conv_state [B,3,3,H*d]."""
     B, T, H, d = q_pre.shape
     dt = q_pre.dtype
+    _shapes(k_pre=(k_pre, q_pre.shape), v_pre=(v_pre, q_pre.shape),
+            conv_state=(conv_state, (B, 3, 3, H * d)))
     args = [_ptr(q_pre, "q_pre", dt), _ptr(k_pre, "k_pre", dt), _ptr(v_pre, "v_pre", dt),
             _ptr(conv_state, "conv_state", dt)]
     st = _lib.kda_conv_state_from_prefill(*args, B, T, H, d, ctypes.byref(opts), _stream(stream))
