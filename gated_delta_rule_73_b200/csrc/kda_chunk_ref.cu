@@ -45,7 +45,7 @@ struct RefLayout {
 template <int DK, int DV>
 constexpr size_t intra_smem_bytes() {
     return sizeof(float) * ((size_t)C * (DK + 1) * 3 + (size_t)C * (DV + 1) + (size_t)C * CP * 3 +
-                            C + 2 * DK);
+                            C + 2 * DK + (size_t)64 * (DK + 1));
 }
 
 template <typename TQ, typename TG, typename TB, int DK, int DV>
@@ -66,6 +66,8 @@ chunk_intra_kernel(const TQ *__restrict__ q, const TQ *__restrict__ k, const TQ 
     float *bs = Tm + C * CP;
     float *sgnC = bs + C;
     float *gamC = sgnC + DK;
+    float *RF = gamC + DK;           // [16][DKP] row factors e^{gamma_r - P} of one row band
+    float *KI = RF + 16 * DKP;       // [48][DKP] k_i e^{P - gamma_i} for the rows before it
 
     const int chunk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / H, h = bh % H;
@@ -135,30 +137,82 @@ chunk_intra_kernel(const TQ *__restrict__ q, const TQ *__restrict__ k, const TQ 
     }
     __syncthreads();
 
-    // A_kk (strict lower, with beta_r) and A_qk (lower with diagonal)
+    // A_kk (strict lower, with beta_r) and A_qk (lower with diagonal), exact for any
+    // gamma: a pair inside one 16-token band takes e^{gamma_r - gamma_i} directly; a pair with
+    // i in an earlier band takes e^{gamma_r - P} e^{P - gamma_i}, P = gamma of the row just
+    // before r's band.  gamma does not increase, so both factors are <= 1 for any g <= 0, and
+    // one exponential per (row, channel) replaces one per (pair, channel) there.
     for (int p = tid; p < C * C; p += 256) {
-        const int r = p / C, i = p % C;
-        float akk = 0.f, aqk = 0.f;
-        if (i <= r && r < n) {
+        Akk[(p / C) * CP + p % C] = 0.f;
+        Aqk[(p / C) * CP + p % C] = 0.f;
+    }
+    __syncthreads();
+    for (int p = tid; p < 4 * 136; p += 256) {           // the four diagonal bands, i <= r
+        const int band = p / 136, t = p % 136;
+        int rr = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+        while ((rr + 1) * (rr + 2) / 2 <= t) ++rr;
+        while (rr * (rr + 1) / 2 > t) --rr;
+        const int r = 16 * band + rr, i = 16 * band + (t - rr * (rr + 1) / 2);
+        if (r < n) {
+            float akk = 0.f, aqk = 0.f;
             for (int c = 0; c < DK; ++c) {
                 const float e = expf(Gs[r * DKP + c] - Gs[i * DKP + c]);
                 const float kk = Ks[i * DKP + c] * e;
                 akk += Ks[r * DKP + c] * kk;
                 aqk += Qs[r * DKP + c] * kk;
             }
+            if (i < r) Akk[r * CP + i] = bs[r] * akk;
+            Aqk[r * CP + i] = aqk;
         }
-        Akk[r * CP + i] = (i < r) ? bs[r] * akk : 0.f;
-        Aqk[r * CP + i] = aqk;
+    }
+    for (int rb = 1; rb < 4; ++rb) {                        // row band rb x earlier bands
+        const int r0 = 16 * rb;
+        if (r0 >= n) break;
+        __syncthreads();                                    // RF / KI of the last band are read
+        for (int idx = tid; idx < 16 * DK; idx += 256) {
+            const int rr = idx / DK, c = idx % DK;
+            RF[rr * DKP + c] = expf(Gs[(r0 + rr) * DKP + c] - Gs[(r0 - 1) * DKP + c]);
+        }
+        for (int idx = tid; idx < r0 * DK; idx += 256) {
+            const int i = idx / DK, c = idx % DK;
+            KI[i * DKP + c] = Ks[i * DKP + c] * expf(Gs[(r0 - 1) * DKP + c] - Gs[i * DKP + c]);
+        }
+        __syncthreads();
+        const int rr = tid >> 4, ig = tid & 15, r = r0 + rr;   // columns ig, ig + 16, ...
+        float aq[3] = {0.f, 0.f, 0.f}, ak[3] = {0.f, 0.f, 0.f};
+        for (int c = 0; c < DK; ++c) {
+            const float f = RF[rr * DKP + c];
+            const float qf = Qs[r * DKP + c] * f, kf = Ks[r * DKP + c] * f;
+#pragma unroll
+            for (int m = 0; m < 3; ++m) {
+                if (m < rb) {
+                    const float ki = KI[(ig + 16 * m) * DKP + c];
+                    aq[m] = fmaf(qf, ki, aq[m]);
+                    ak[m] = fmaf(kf, ki, ak[m]);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+            if (m < rb) {
+                Aqk[r * CP + ig + 16 * m] = aq[m];
+                Akk[r * CP + ig + 16 * m] = bs[r] * ak[m];
+            }
+        }
     }
     __syncthreads();
 
-    // Tm = (I + A_kk)^{-1}: column j solves (I + A_kk) x = e_j
-    if (tid < C) {
-        const int j = tid;
+    // Tm = (I + A_kk)^{-1}: column j solves (I + A_kk) x = e_j by forward substitution, row by
+    // row; the four lanes of a column split each row's sum (lanes 4j .. 4j + 3 of one warp)
+    {
+        const int j = tid >> 2, part = tid & 3;
         for (int r = 0; r < C; ++r) {
-            float acc = (r == j) ? 1.f : 0.f;
-            for (int i = j; i < r; ++i) acc -= Akk[r * CP + i] * Tm[i * CP + j];
-            Tm[r * CP + j] = (r < j) ? 0.f : acc;
+            float acc = 0.f;
+            for (int i = j + part; i < r; i += 4) acc = fmaf(Akk[r * CP + i], Tm[i * CP + j], acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (part == 0) Tm[r * CP + j] = (r < j) ? 0.f : ((r == j) ? 1.f : 0.f) - acc;
+            __syncwarp();
         }
     }
 
