@@ -11,6 +11,8 @@
 //   sigma_r = prod_{s<=r} sign(alpha_s) (Complex-KDA; folded into q and k),
 //   A_kk[r,i] = beta_r sum_c k_rc k_ic e^{gamma_rc - gamma_ic}   (i < r)
 //   A_qk[r,i] =        sum_c q_rc k_ic e^{gamma_rc - gamma_ic}   (i <= r)
+//     (inside a 16-token band the factor is taken per pair; across bands as
+//      e^{gamma_r - P} e^{P - gamma_i} with P = gamma just before r's band)
 //   Tm = (I + A_kk)^{-1} by forward substitution (the UT transform)
 //   W = Tm diag(beta) (K e^gamma),  U = Tm diag(beta) V    (WY vectors)
 //   Qg = Q e^gamma,  Kd = sigma_C K e^{gamma_C - gamma},  gC = sigma_C e^{gamma_C}

@@ -267,3 +267,31 @@ def test_segment_pair_and_combine_host_checks(kda):
     assert comb(dv=32) == -4
     assert comb(Bp=0x1004) == -3
     assert comb(BH=0) == 0
+
+
+def test_binding_checks_shapes_before_any_call(kda):
+    """The binding passes sizes read off q and v, so every other tensor must have the shape
+    those sizes imply; a mismatch is refused (ValueError) before any pointer is taken."""
+    import torch
+    B, T, H, d = 1, 8, 2, 128
+    q = torch.zeros(B, T, H, d, dtype=torch.bfloat16)
+    good = dict(k=q, v=q, g=q, beta=torch.zeros(B, T, H, dtype=torch.bfloat16),
+                S0=None, out=q, S_T=torch.zeros(B, H, d, d))
+    o = kda.make_opts()
+    for name, bad in (("k", torch.zeros(B, T, H, 64, dtype=torch.bfloat16)),
+                      ("beta", torch.zeros(B, T, dtype=torch.bfloat16)),
+                      ("S_T", torch.zeros(B, H, d, 64)),
+                      ("out", torch.zeros(B, T + 1, H, d, dtype=torch.bfloat16))):
+        args = dict(good, **{name: bad})
+        with pytest.raises(ValueError, match=name):
+            kda.kda_chunk_fwd(q, args["k"], args["v"], args["g"], args["beta"], args["S0"],
+                              args["out"], args["S_T"], o)
+    f = torch.float32
+    grads = [torch.zeros(B, T, H, d), torch.zeros(B, T, H, d), torch.zeros(B, T, H, d),
+             torch.zeros(B, T, H, d), torch.zeros(B, T, H), None]
+    with pytest.raises(ValueError, match="grad_beta"):
+        kda.kda_chunk_bwd(q, q, q, q, good["beta"], None, q, None, *grads[:4],
+                          torch.zeros(B, T, H, 2), None, o)
+    with pytest.raises(ValueError, match="M and Bp|M must"):
+        kda.kda_affine_combine(torch.zeros(3, B * H, d, d), torch.zeros(2, B * H, d, d), 1, None,
+                               torch.zeros(B * H, d, d))
