@@ -158,7 +158,7 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 106; }
+int kda_abi_version(void) { return 107; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -367,6 +367,12 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g, co
     cudaError_t e = launch_chunk_bwd(a, stream);
     if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_selftest_bounded_wait(unsigned limit, cudaStream_t stream) {
+    int status = 0;
+    if (run_bounded_wait_selftest(limit, &status, stream) != cudaSuccess) return KDA_ERR_CUDA;
+    return status == 3 ? KDA_ERR_TIMEOUT : KDA_ERR_CUDA;
 }
 
 int kda_recurrent_step(const void *q, const void *k, const void *v, const void *g, const void *beta,

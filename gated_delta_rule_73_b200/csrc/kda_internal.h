@@ -107,6 +107,10 @@ cudaError_t launch_identity(float *S, long long count, int d, cudaStream_t st);
 cudaError_t launch_affine_combine(const float *M, const float *Bp, int n, const float *S0, float *S_out,
                                   int BH, int dk, int dv, cudaStream_t st);
 
+// Self-test of the bounded waits: one kernel whose mbarrier wait and flag poll both run out
+// (nothing arrives); *status gets bit 0 / bit 1 for each that gave up.  Synchronises `st`.
+cudaError_t run_bounded_wait_selftest(unsigned limit, int *status, cudaStream_t st);
+
 // Record a.events[*a.launch_idx] (if requested) and advance the counter.
 inline void mark_launch(const ChunkArgs &a, cudaStream_t st) {
     if (a.events && a.launch_idx && *a.launch_idx < a.n_events)

@@ -68,6 +68,8 @@ def _load():
     lib.kda_segment_pair_workspace_bytes.restype = sz
     lib.kda_affine_combine.argtypes = [vp, vp, ip, vp, vp, ip, ip, ip, vp]
     lib.kda_affine_combine.restype = ip
+    lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+    lib.kda_selftest_bounded_wait.restype = ip
     lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_chunk_workspace_bytes.restype = sz
     lib.kda_prologue_workspace_bytes.argtypes = [ip] * 5 + [op]
@@ -239,6 +241,11 @@ def kda_affine_combine(M, Bp, n, S0, S_out, stream=None) -> None:
                                  _ptr(S_out, "S_out", f), BH, dk, dv, _stream(stream))
     if st != 0:
         raise KdaError("kda_affine_combine", st)
+
+
+def kda_selftest_bounded_wait(limit: int, stream=None) -> int:
+    """Call ``kda_selftest_bounded_wait``; returns its status (KDA_ERR_TIMEOUT = -6 expected)."""
+    return int(_lib.kda_selftest_bounded_wait(int(limit), _stream(stream)))
 
 
 def kda_chunk_fwd_noalloc(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -> None:

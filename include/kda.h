@@ -58,7 +58,7 @@ typedef enum {
     KDA_ERR_ALIGN = -3,        /* a pointer is not 16-byte aligned             */
     KDA_ERR_UNSUPPORTED = -4,  /* valid but not implemented (dk/dv, flags)     */
     KDA_ERR_CUDA = -5,         /* a CUDA launch or copy reported an error      */
-    KDA_ERR_TIMEOUT = -6,      /* reserved: a bounded device wait gave up      */
+    KDA_ERR_TIMEOUT = -6,      /* a bounded device wait gave up               */
     KDA_ERR_WORKSPACE = -7     /* workspace missing or smaller than required   */
 } kda_status;
 
@@ -346,12 +346,26 @@ size_t kda_segment_pair_workspace_bytes(int B, int T, int H, int dk, int dv,
 int kda_affine_combine(const float *M, const float *Bp, int n, const float *S0,
                        float *S_out, int BH, int dk, int dv, cudaStream_t stream);
 
+/*
+ * kda_selftest_bounded_wait -- exercises the give-up path of the library's bounded waits.
+ *
+ * The pages have no counterpart: this is a check of the library's failure handling.  The
+ * tensor-core kernels wait only in bounded loops (on mbarriers of their own CTA, and on
+ * flags between CTAs of one launch); a wait that runs out sets an error word and the kernel
+ * returns.  This launches one tiny kernel that waits, with at most `limit` polls each, on an
+ * mbarrier no one arrives at and on a flag no one writes, then reads its status back and
+ * synchronises `stream`.  It returns KDA_ERR_TIMEOUT when both waits gave up (the expected
+ * outcome, for any limit, 0 included) and KDA_ERR_CUDA if the launch or the copy failed.
+ * Nothing faults and nothing can hang; the CUDA context stays usable afterwards.
+ */
+int kda_selftest_bounded_wait(unsigned limit, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
 /* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
    1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd;
-   1.6: kda_segment_pair, kda_affine_combine). */
+   1.6: kda_segment_pair, kda_affine_combine; 1.7: kda_selftest_bounded_wait). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

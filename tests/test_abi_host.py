@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 106   # 1.6: kda_segment_pair, kda_affine_combine
+    assert kda.kda_abi_version() == 107   # 1.7: kda_selftest_bounded_wait
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
