@@ -221,7 +221,7 @@ def recurrence_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, l2norm=True,
 
 
 def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
-                     complex_gate=False, scale=1.0, eps=L2NORM_EPS):
+                     complex_gate=False, scale=1.0, eps=L2NORM_EPS, chunk_stages=False):
     """FP64 gradient of ``L = <dO, O> + <dS_T, S_T>`` through the chunkwise form of
     :func:`chunkwise_np`; returns what :func:`recurrence_bwd_np` returns.
 
@@ -239,6 +239,11 @@ def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
     then the products back to Q, K, V, beta and Gamma, Gamma_C = Gamma[last], and
     Gamma = cumprod(alpha) (dg_s = sum_{r >= s} dGamma_r Gamma_r / alpha_s * dalpha_s/dg_s).
     FP64 holds exp(+-320), so the plain K / Gamma is used, as in the forward.
+
+    With ``chunk_stages=True`` it also returns the two sequences a chunked kernel produces
+    between its stages, each [B, H, n_chunks + 1, dk, dv]: the state at the start of every
+    chunk (the last entry is S_T) and dL/dS there (the reverse scan's output; the last
+    entry is dS_T, the first dS0).
     """
     q, k, v, g, beta, dO = map(_f64, (q, k, v, g, beta, dO))
     B, T, H, dk = q.shape
@@ -254,6 +259,8 @@ def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
     dalpha, dbeta = np.zeros_like(g), np.zeros_like(beta)
     dS0 = np.zeros((B, H, dk, dv))
     starts = list(range(0, T, C))
+    st_all = np.zeros((B, H, len(starts) + 1, dk, dv))
+    gr_all = np.zeros((B, H, len(starts) + 1, dk, dv))
     for b in range(B):
         for h in range(H):
             # forward, keeping each chunk's start state
@@ -271,8 +278,11 @@ def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
                 Vt = Tm @ (bt[:, None] * V) - Tm @ (bt[:, None] * Kg) @ S
                 GC = Gam[-1]
                 S = GC[:, None] * S + (K * (GC[None, :] / Gam)).T @ Vt
+            st_all[b, h, :len(states)] = states
+            st_all[b, h, len(states)] = S
             dS = np.zeros((dk, dv)) if dS_T is None else _f64(dS_T)[b, h].copy()
-            for s, S in zip(reversed(starts), reversed(states)):
+            gr_all[b, h, len(starts)] = dS
+            for ci, s, S in zip(reversed(range(len(starts))), reversed(starts), reversed(states)):
                 e = min(s + C, T)
                 n = e - s
                 Q, K, V = qh[b, s:e, h], kh[b, s:e, h], v[b, s:e, h]
@@ -316,6 +326,7 @@ def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
                 rc = np.cumsum((dGam * Gam)[::-1], axis=0)[::-1]
                 dalpha[b, s:e, h] = rc / al
                 dS = dS_prev
+                gr_all[b, h, ci] = dS
             dS0[b, h] = dS
     dg = dalpha if complex_gate else alpha * dalpha
     if l2norm:
@@ -323,6 +334,8 @@ def chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dS_T=None, *, C=64, l2norm=True,
         dk_ = (dkh - kh * np.sum(kh * dkh, axis=-1, keepdims=True)) / nk
     else:
         dq, dk_ = dqh, dkh
+    if chunk_stages:
+        return (dq, dk_, dvv, dg, dbeta, dS0), st_all, gr_all
     return dq, dk_, dvv, dg, dbeta, dS0
 
 

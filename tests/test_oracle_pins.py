@@ -604,3 +604,30 @@ def test_chunkwise_backward_equals_recurrence_backward(C, complex_gate, l2norm):
     got = oracle.chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dST, C=C, **kw)
     for a, b in zip(got, ref):
         assert _rel(a, b) < 1e-12
+
+
+def test_chunkwise_backward_stage_outputs():
+    """The chunked backward's intermediate sequences, pinned without the chunk algebra: the
+    state at chunk start c is the recurrence run over tokens [0, 16c); dL/dS there is the
+    dS0 of the token-level reverse pass over the suffix [16c, T) started from that state
+    (the adjoint of the suffix is the gradient the prefix hands back)."""
+    rng = np.random.default_rng(77)
+    T, C = 37, 16
+    q, k, v, g, beta, S0 = _rand_case(rng, B=1, T=T, H=2, dk=4, dv=3)
+    dO = rng.standard_normal((1, T, 2, 3))
+    dST = rng.standard_normal((1, 2, 4, 3))
+    grads, states, sgrads = oracle.chunkwise_bwd_np(q, k, v, g, beta, S0, dO, dST, C=C,
+                                                    chunk_stages=True)
+    starts = [0, 16, 32, T]
+    assert states.shape == (1, 2, 4, 4, 3) and sgrads.shape == (1, 2, 4, 4, 3)
+    for ci, t in enumerate(starts):
+        want = S0 if t == 0 else oracle.recurrence_c(q[:, :t], k[:, :t], v[:, :t], g[:, :t],
+                                                     beta[:, :t], S0)[1]
+        assert _rel(states[:, :, ci], want) < RTOL
+        if t == T:
+            assert np.array_equal(sgrads[:, :, ci], dST)
+            continue
+        suffix = oracle.recurrence_bwd_np(q[:, t:], k[:, t:], v[:, t:], g[:, t:], beta[:, t:],
+                                          want, dO[:, t:], dST)[5]
+        assert _rel(sgrads[:, :, ci], suffix) < 1e-12
+    assert np.array_equal(sgrads[:, :, 0], grads[5])
