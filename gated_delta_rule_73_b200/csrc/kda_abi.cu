@@ -166,7 +166,7 @@ const char *kda_status_string(int s) {
         case KDA_ERR_ARG: return "invalid argument (NULL pointer, negative size or unknown flag)";
         case KDA_ERR_SHAPE: return "inconsistent or overflowing sizes";
         case KDA_ERR_ALIGN: return "pointer not 16-byte aligned";
-        case KDA_ERR_UNSUPPORTED: return "unsupported configuration (dk/dv must be 64 or 128)";
+        case KDA_ERR_UNSUPPORTED: return "unsupported configuration (dk, dv other than 64 or 128, or an option the entry point does not take)";
         case KDA_ERR_CUDA: return "CUDA launch or copy failed";
         case KDA_ERR_TIMEOUT: return "a bounded device wait gave up";
         case KDA_ERR_WORKSPACE: return "workspace missing or too small";
