@@ -10,10 +10,14 @@ written between timed steps (outside the timed events).  Under torchrun every
 rank runs its own batch (weak scaling, no collective on the data path);
 ``value`` is the tokens of all ranks over the slowest rank's time.
 
-Also measured on rank 0 at N=1 (the ``rows`` object): the fused-prologue
-length sweep at T=8192 (B=1, H=96), the decode step (N=256, H=96) and the
-Complex-KDA workload (B=8, T=8192, H=32) next to unsigned KDA of the same
-shape.  ``cpu_baseline`` times the FP64 oracle on the host cores.
+Also measured on rank 0 at N=1 (the ``rows`` object):
+  * the fused-prologue length sweep at T=8192 (B=1, H=96);
+  * the output epilogue, the backward, the Kimi Linear softplus gate and the split of
+    one sequence into four segments, all on the prefill shape;
+  * the decode step and the decode step with its prologue (N=256, H=96);
+  * the Complex-KDA workload (B=8, T=8192, H=32) next to unsigned KDA of the same shape.
+``e2e`` is the same metric through the C ABI with host buffers, copies timed.
+``cpu_baseline`` times the FP64 oracle on the host cores.
 """
 from __future__ import annotations
 
@@ -81,18 +85,21 @@ class ClockSampler:
         self._stop = threading.Event()
         self._t = None
 
-    def _run(self):
+    def _sample(self):
         N = self.N
+        try:
+            self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+            r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, attr in self.REASONS.items():
+                if r & getattr(N, attr, 0):
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
-                r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, attr in self.REASONS.items():
-                    if r & getattr(N, attr, 0):
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(0.005)
+            self._sample()
+            time.sleep(0.002)
 
     def __enter__(self):
         if self.ok:
@@ -102,6 +109,7 @@ class ClockSampler:
 
     def __exit__(self, *a):
         if self._t:
+            self._sample()          # one more reading at the end of the timed region
             self._stop.set()
             self._t.join()
 
