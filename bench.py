@@ -225,13 +225,13 @@ def cpu_baseline_prefill(min_seconds=10.0, max_runs=40):
             "seconds": dt, "runs": runs}
 
 
-def rows_n1(K, flush, hbm_peak):
-    """Per-row measurements beyond the headline (rank 0, N=1)."""
-    rows = {}
+def sweep_row(K, T, flush, hbm_peak):
+    """a1-a4 on the length-sweep workload (B=1, H=96, d=128, raw inputs through the fused
+    prologue) at one T: the call's time and its fraction of the HBM roofline."""
+    H, d = 96, 128
+    prev = W._DEVICE
     W.set_device("cuda")
     try:
-        # a1-a4: fused prologue + chunk forward, length sweep at T = 8192
-        T, H, d = 8192, 96, 128
         x = W.sweep_inputs(T)
         args = [x[n] for n in ("q_pre", "k_pre", "v_pre", "conv_w", "z", "A", "b_logit")]
         opts0 = K.make_opts(torch.bfloat16)
@@ -244,12 +244,22 @@ def rows_n1(K, flush, hbm_peak):
         fn()
         ms = statistics.median(time_calls(fn, 3, flush))
         nbytes = T * H * (4 * d * 2 + 4 + d * 2) + H * (2 * d * d * 4 + 3 * d * 4 * 2)
-        rows["sweep_T8192_prologue"] = {
-            "ms": ms, "tokens_per_s": T / (ms * 1e-3), "token_heads_per_s": T * H / (ms * 1e-3),
-            "roofline_bytes": nbytes, "roofline_flops": PREFILL_FLOP_PER_TOKEN_HEAD * T * H,
-            "frac_of_hbm_roofline": (nbytes / (ms * 1e-3) / 1e9) / hbm_peak}
-        del x, args, ws, out, S_T
+        return {"ms": ms, "tokens_per_s": T / (ms * 1e-3), "token_heads_per_s": T * H / (ms * 1e-3),
+                "roofline_bytes": nbytes, "roofline_flops": PREFILL_FLOP_PER_TOKEN_HEAD * T * H,
+                "frac_of_hbm_roofline": (nbytes / (ms * 1e-3) / 1e9) / hbm_peak}
+    finally:
+        W.set_device(prev)
         torch.cuda.empty_cache()
+
+
+def rows_n1(K, flush, hbm_peak, rows):
+    """Per-row measurements beyond the headline (rank 0, N=1), filled into `rows` as they
+    finish (a row that fails leaves the earlier ones in place)."""
+    W.set_device("cuda")
+    try:
+        # a1-a4: fused prologue + chunk forward, length sweep at T = 8192
+        rows["sweep_T8192_prologue"] = sweep_row(K, 8192, flush, hbm_peak)
+        d = 128
 
         # a2-a4 + the output epilogue (RMSNorm * sigmoid gate) on the prefill workload
         x = W.workload_inputs("prefill")
@@ -623,7 +633,17 @@ def run_ours(args, ws, rank, local):
             "step_ms_median": statistics.median(step_ms),
             "clocks": sampler.summary(), "wall_s_timed": w1 - w0}
     if ws == 1 and rank == 0 and not args.no_rows:
-        line["rows"] = rows_n1(K, flush, hbm_peak)
+        rows = {}
+        try:
+            rows_n1(K, flush, hbm_peak, rows)
+        except Exception as e:          # a failed row must not cost the headline its line
+            rows["error"] = f"{type(e).__name__}: {e}"
+        for T in W.SWEEP_T[2:]:           # the longer sweep lengths, memory permitting
+            try:
+                rows[f"sweep_T{T}_prologue"] = sweep_row(K, T, flush, hbm_peak)
+            except Exception as e:
+                rows[f"sweep_T{T}_prologue"] = {"error": f"{type(e).__name__}: {e}"}
+        line["rows"] = rows
     if ws == 1 and rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline_prefill()
     if rank == 0:
