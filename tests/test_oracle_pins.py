@@ -631,3 +631,27 @@ def test_chunkwise_backward_stage_outputs():
                                           want, dO[:, t:], dST)[5]
         assert _rel(sgrads[:, :, ci], suffix) < 1e-12
     assert np.array_equal(sgrads[:, :, 0], grads[5])
+
+
+def test_generated_inputs_follow_their_recipes():
+    """The seeded inputs of the newer workloads are what DESIGN's input table says: Kimi
+    Linear's softplus gate has A_h = log U(1, 16) and no floor (a large share of g below -5,
+    all of it below 0); the prologue inputs take the same A_h law; the upstream gradients
+    of the backward have the run dtype (dout) and FP32 (dS_T); one seed, one draw."""
+    x = W.chunk_inputs(1, 512, 4, 32, 16, seed=9, gate="softplus")
+    g = x["g"].double().numpy()
+    assert g.max() < 0.0 and g.min() < -20.0 and (g < -5.0).mean() > 0.2
+    p = W.prologue_inputs(1, 5, 64, 8, 8, seed=2, gate="softplus")
+    A = p["A"].double().numpy()
+    assert A.min() >= 0.0 and A.max() <= math.log(16.0) + 1e-6 and A.std() > 0.3
+    pb = W.prologue_inputs(1, 5, 64, 8, 8, seed=2)
+    assert pb["A"].max() <= 0.0 and pb["A"].min() >= -1.0
+    with pytest.raises(ValueError):
+        W.chunk_inputs(1, 4, 1, 8, 8, gate="relu")
+    gr = W.grad_inputs(2, 7, 3, 16, 8, seed=4)
+    assert gr["dout"].shape == (2, 7, 3, 8) and gr["dout"].dtype.is_floating_point
+    assert str(gr["dout"].dtype) == "torch.bfloat16" and str(gr["dS_T"].dtype) == "torch.float32"
+    assert gr["dS_T"].shape == (2, 3, 16, 8) and 0.005 < float(gr["dS_T"].std()) < 0.02
+    assert W.grad_inputs(1, 3, 1, 8, 8, dST_std=0.0)["dS_T"] is None
+    again = W.grad_inputs(2, 7, 3, 16, 8, seed=4)
+    assert bool((again["dout"] == gr["dout"]).all()) and bool((again["dS_T"] == gr["dS_T"]).all())
