@@ -8,6 +8,7 @@
 
 #include "../../include/kda.h"
 #include "kda_internal.h"
+#include "kda_checks.h"
 
 using namespace kda;
 
@@ -31,33 +32,6 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 // forms' band-referenced decay factors could leave the bf16/FP32 range, the FP32 path cannot
 bool unbounded(const kda_opts &o) { return (o.flags & (KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS)) != 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-int check_opts(const kda_opts &o) {
-    if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
-    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT |
-                              KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS))
-        return KDA_ERR_ARG;
-    if ((o.flags & KDA_FUSED) && (o.flags & KDA_SPLIT)) return KDA_ERR_ARG;
-    if (unbounded(o) && (o.flags & (KDA_FUSED | KDA_SPLIT))) return KDA_ERR_ARG;
-    if ((o.flags & KDA_GATE_SOFTPLUS) && (o.flags & KDA_COMPLEX)) return KDA_ERR_ARG;
-    if (!isfinite(o.scale)) return KDA_ERR_ARG;
-    if (o.n_events < 0 || (o.n_events > 0 && !o.events)) return KDA_ERR_ARG;
-    return KDA_OK;
-}
-
-int check_dims(long long B, long long T, long long H, int dk, int dv) {
-    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
-    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
-    const long long d = dk > dv ? dk : dv;
-    if (B > 0 && T > 0 && H > 0) {
-        if (B > kMaxElems / T) return KDA_ERR_SHAPE;
-        const long long bt = B * T;
-        if (bt > kMaxElems / H) return KDA_ERR_SHAPE;
-        if (bt * H > kMaxElems / d) return KDA_ERR_SHAPE;
-    }
-    if (B * H > 65535) return KDA_ERR_UNSUPPORTED;   // grid y of the chunk kernels
-    return KDA_OK;
-}
 
 KernelFlags kflags(const kda_opts &o) {
     KernelFlags f;
@@ -155,6 +129,36 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
 }
 
 }  // namespace
+
+namespace kda {
+// Shared by every entry point (kda_noalloc.cu included), so the argument rules cannot drift.
+int check_opts(const kda_opts &o) {
+    if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
+    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX | KDA_FUSED | KDA_SPLIT |
+                              KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS))
+        return KDA_ERR_ARG;
+    if ((o.flags & KDA_FUSED) && (o.flags & KDA_SPLIT)) return KDA_ERR_ARG;
+    if (unbounded(o) && (o.flags & (KDA_FUSED | KDA_SPLIT))) return KDA_ERR_ARG;
+    if ((o.flags & KDA_GATE_SOFTPLUS) && (o.flags & KDA_COMPLEX)) return KDA_ERR_ARG;
+    if (!isfinite(o.scale)) return KDA_ERR_ARG;
+    if (o.n_events < 0 || (o.n_events > 0 && !o.events)) return KDA_ERR_ARG;
+    return KDA_OK;
+}
+
+int check_dims(long long B, long long T, long long H, int dk, int dv) {
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
+    const long long d = dk > dv ? dk : dv;
+    if (B > 0 && T > 0 && H > 0) {
+        if (B > kMaxElems / T) return KDA_ERR_SHAPE;
+        const long long bt = B * T;
+        if (bt > kMaxElems / H) return KDA_ERR_SHAPE;
+        if (bt * H > kMaxElems / d) return KDA_ERR_SHAPE;
+    }
+    if (B * H > 65535) return KDA_ERR_UNSUPPORTED;   // grid y of the chunk kernels
+    return KDA_OK;
+}
+}  // namespace kda
 
 extern "C" {
 

@@ -14,12 +14,16 @@
 // stream capture.  Every call shares the array: calls whose work overlaps on
 // the GPU (different streams, or different host threads on one device) race.
 // Each call writes every scratch element it later reads, so nothing needs to
-// start at zero and the previous call's leftovers are never used.
+// start at zero and the previous call's leftovers are never used.  The cached
+// address belongs to the device's primary context: after cudaDeviceReset (or any
+// other teardown of that context) this entry point must not be called again in
+// the same process.
 #include <mutex>
 #include <string.h>
 
 #include "../../include/kda.h"
 #include "kda_internal.h"
+#include "kda_checks.h"
 
 using namespace kda;
 
@@ -56,12 +60,12 @@ extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v
     o.flags = KDA_QK_L2NORM;
     o.scale = 1.0f;
     if (opts) o = *opts;
-    if (o.dtype != KDA_BF16 && o.dtype != KDA_F32) return KDA_ERR_ARG;
-    if (o.flags & ~(unsigned)(KDA_QK_L2NORM | KDA_COMPLEX)) return KDA_ERR_ARG;
-    if (!(o.scale == o.scale) || o.scale > 3.4e38f || o.scale < -3.4e38f) return KDA_ERR_ARG;
-    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_ARG;
-    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_UNSUPPORTED;
-    if ((long long)B * H > 65535) return KDA_ERR_UNSUPPORTED;
+    // the same argument rules as kda_chunk_fwd; the flags that only choose among its paths
+    // (KDA_FUSED, KDA_SPLIT, KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS) are accepted and have no
+    // effect here: this entry point always runs the exact-FP32 path, which takes any g <= 0
+    int st = check_opts(o);
+    if (st != KDA_OK) return st;
+    if ((st = check_dims(B, T, H, dk, dv)) != KDA_OK) return st;
     if (B == 0 || H == 0) return KDA_OK;
     if (T == 0) {
         if (!aligned16(S0) || !aligned16(S_T)) return KDA_ERR_ALIGN;

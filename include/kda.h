@@ -253,17 +253,22 @@ int kda_conv_state_from_prefill(const void *q_pre, const void *k_pre, const void
  * the method.  Some callers cannot call cudaMalloc -- code that must not
  * synchronise the device, loops that forbid allocation once running, host
  * applications that own the device pool and give a component no allocator.
- * This entry point takes the same arguments as kda_chunk_fwd (opts->workspace
- * is ignored) and runs the FP32 two-phase chunk path with its scratch in a
- * fixed device array of KDA_NOALLOC_SCRATCH_BYTES, which every GPU that loads
- * the library holds until the process exits.  It calls no allocator.
+ * This entry point takes the same arguments as kda_chunk_fwd, checked by the
+ * same rules (opts->workspace is ignored), and runs the exact-FP32 two-phase
+ * chunk path with its scratch in a fixed device array of
+ * KDA_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits.  It calls no allocator.  The flags that only pick
+ * one of kda_chunk_fwd's paths (KDA_FUSED, KDA_SPLIT, KDA_UNBOUNDED_DECAY,
+ * KDA_GATE_SOFTPLUS) are accepted and change nothing: the exact-FP32 path
+ * takes any g <= 0.
  *
  *  - Sizes whose scratch (kda_chunk_workspace_bytes of the FP32 path: about
  *    148 KB per 64-token chunk and head at dk = dv = 128) exceeds the array
  *    are rejected with KDA_ERR_WORKSPACE before any CUDA call.
  *  - The first call on a device (with that device current) looks up the
  *    array's device address once; make that first call before any stream
- *    capture.
+ *    capture.  The address belongs to the device's primary context: after
+ *    cudaDeviceReset, do not call this entry point again in that process.
  *  - All calls share the array.  Calls whose work overlaps on the GPU race;
  *    serialise them (one stream per device).  No scratch content carries over:
  *    each call writes every element it reads.
