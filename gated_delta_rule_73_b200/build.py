@@ -47,7 +47,8 @@ LAST_BUILD = {"compiled": None, "objects_compiled": []}
 
 def _digest(files, flags):
     h = hashlib.sha256()
-    h.update(" ".join(flags).encode())
+    # flags with this checkout's absolute paths made relative, so a copy elsewhere matches
+    h.update(" ".join(f.replace(ROOT, "<root>") for f in flags).encode())
     for f in files:
         h.update(os.path.relpath(f, ROOT).encode())
         with open(f, "rb") as fh:

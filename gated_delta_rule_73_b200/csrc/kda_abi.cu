@@ -162,7 +162,7 @@ int check_dims(long long B, long long T, long long H, int dk, int dv) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 107; }
+int kda_abi_version(void) { return 108; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -372,6 +372,15 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g, co
     if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
+
+int kda_device_status(cudaStream_t stream) {
+    int f1 = 0, f2 = 0;
+    if (chunk_tc_take_error(&f1, stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (chunk_tc2_take_error(&f2, stream) != cudaSuccess) return KDA_ERR_CUDA;
+    return (f1 || f2) ? KDA_ERR_TIMEOUT : KDA_OK;
+}
+
+unsigned kda_set_wait_limit(unsigned polls) { return set_wait_limit(polls); }
 
 int kda_selftest_bounded_wait(unsigned limit, cudaStream_t stream) {
     int status = 0;

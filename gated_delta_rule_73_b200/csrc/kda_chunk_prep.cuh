@@ -1,0 +1,774 @@
+// kda_chunk_prep.cuh -- the split form's per-(chunk, head) prep, two items in flight per SM.
+//
+// Included by kda_chunk_tc2.cu after the record layout.  Everything up to the WY vectors
+// depends on one chunk's inputs only (page "Kimi K3 模型结构（2）：序列维度（下），chunkwise 并行与
+// 下界衰减", Q&A items on the chunkwise algorithm, the -5 decay floor and the intra-chunk matrix
+// A), so the work is cut into (chunk, head) items.  A 512-thread CTA holds two independent item
+// groups of 256 threads, each with its own 112 KB of shared memory, 256 TMEM columns, mbarriers
+// and named barrier: while one group waits (a TMA tile, a tensor-core product, a barrier), the
+// other issues.  Per item:
+//
+//   TMA       q, k (interleaved by 64-channel halves so [q; k] is one 128-row K-major operand),
+//             g and v tiles [64 tokens x 128], 128-byte swizzle
+//   tcgen05   band-local cumulative log-decay: gamma~ = L g with L = [L_band; L_band] (ones on
+//             and below the diagonal inside each 16-token band; constant A operand in TMEM);
+//             exact in FP32 (bf16 g times 1, FP32 sums)
+//   CUDA      row norms of q and k, band totals of g (while the cumsum runs); per-channel band
+//             factors e^{p_b}, e^{gamma_C - p_b}, e^{p_b' - p_b} (p_b = gamma before band b)
+//   CUDA      thread = (token row, 32 channels): E = e^{gamma~} in [e^-80, 1] and 1/E, then in
+//             place Q E and beta K E (the band-pair A operand), K e^gamma over g (the W product's
+//             B operand), the band-pair B rows k_i e^{p_b - gamma_i} for b >= band(i), and the
+//             record's Q e^gamma and K e^{gamma_C - gamma} straight to global memory
+//   tcgen05   A_qk / A_kk: the ten (row band, column band) pairs as one N = 160 product
+//   CUDA      A_qk -> record; Tm = (I + A_kk)^{-1} in FP32 (16x16 diagonal blocks, then 32x32)
+//   tcgen05   [W; U] = [Tm' 0; 0 Tm'] [K e^gamma; V]  (Tm' = Tm diag(beta), block-diagonal A
+//             operand in TMEM, one M = 128, K = 128 product)
+//   CUDA      W, U -> record
+//
+// The record (74,240 bytes per chunk and head) has the layout the scan kernel reads.
+#pragma once
+
+namespace prep2 {
+constexpr int NG = 2;                  // item groups per CTA
+constexpr int GT = 256;                // threads per group
+constexpr int NT = NG * GT;
+// shared memory of one group (bytes from its 1024-aligned base)
+constexpr uint32_t OFF_X = 0;          // q, k staging [q h0][k h0][q h1][k h1] (8 KB each)
+constexpr uint32_t OFF_G = 32768;      // g staging [h0][h1]; later K e^gamma
+constexpr uint32_t OFF_V = 49152;      // v staging [h0][h1]
+constexpr uint32_t OFF_KH = 65536;     // band-pair B operand, K-major 128-byte swizzle, 160 rows per
+                                       // 64-channel half; before it: band totals; after it: the
+                                       // UT inverse's A_kk^T and T (FP32)
+constexpr uint32_t KH_HALF = 20480;
+constexpr uint32_t OFF_TOT = OFF_KH;           // FP32 [4 bands][128]
+constexpr uint32_t AS = 68;                    // row stride (floats) of the UT's FP32 tiles
+constexpr uint32_t OFF_AKT = OFF_KH;           // A_kk^T [64 i][68] (A_kk[r][i] at i * AS + r)
+constexpr uint32_t OFF_TMF = OFF_KH + 17408;   // T [64 r][68]
+constexpr uint32_t OFF_TAB = 106496;
+// per-channel band factors, FP32 rows of 128 (p_b = gamma before band b, e_b = e^{band b's total}):
+// e_0..e_3, e^{p_2}, e^{p_3}, e^{gamma_C - p_0..2}, e^{p_2 - p_0}, e^{p_3 - p_1}, e^{p_3 - p_0}, ones
+constexpr int R_ET = 0, R_EP2 = 4, R_EP3 = 5, R_ECP = 6, R_EM20 = 9, R_EM31 = 10, R_EM30 = 11, R_ONE = 12;
+constexpr uint32_t TAB_F = 0;          // 13 rows x 512 B
+constexpr uint32_t TAB_NRMP = 6656;    // FP32 sums of squares [2 halves][128 rows: q, then k]
+constexpr uint32_t TAB_BET = 7680;     // FP32 beta [64]
+constexpr uint32_t TAB_BAR = 7936;     // mbarriers and the abort flag
+constexpr uint32_t GROUP_USED = OFF_TAB + TAB_BAR + 64;
+constexpr uint32_t GROUP_STRIDE = 114688;
+constexpr uint32_t SMEM_BYTES = 1024 + GROUP_STRIDE + GROUP_USED;
+static_assert(GROUP_USED <= GROUP_STRIDE, "group layout");
+static_assert(OFF_TMF + 17408 <= OFF_TAB, "UT tiles inside the band-pair operand's region");
+static_assert(SMEM_BYTES <= 232448 - 256, "shared memory budget");
+// TMEM columns of a group (its 256): D = cumsum / band pairs / [W; U]; the block-diagonal
+// Tm' operand; the constant cumsum operand L
+constexpr uint32_t TC_D = 0, TC_TM = 160, TC_LM = 224;
+
+struct alignas(8) GroupBars {
+    uint64_t qk, g, v, m1, m2, m3;
+    int abort;
+};
+
+// q / k (t = 0 / 1) unit (token row r, 8-channel group cg) in the interleaved staging
+__device__ __forceinline__ uint32_t off_x(int t, int r, int cg) {
+    return (uint32_t)((cg >> 3) * 16384 + t * 8192 + r * 128 + (((cg & 7) ^ (r & 7)) << 4));
+}
+// g / v staging (and K e^gamma over g): one tile of two 8 KB halves
+__device__ __forceinline__ uint32_t off_t(int r, int cg) {
+    return (uint32_t)((cg >> 3) * 8192 + r * 128 + (((cg & 7) ^ (r & 7)) << 4));
+}
+// band-pair B row n (0..159)
+__device__ __forceinline__ uint32_t off_kh(int n, int cg) {
+    return (uint32_t)((cg >> 3) * KH_HALF + n * 128 + (((cg & 7) ^ (n & 7)) << 4));
+}
+// factor rows: e^{p_b}, e^{gamma_C - p_b}, e^{p_b' - p_b} (b' > b)
+__device__ __forceinline__ int row_ep(int b) { return b == 0 ? R_ONE : b == 1 ? R_ET + 0 : b == 2 ? R_EP2 : R_EP3; }
+__device__ __forceinline__ int row_ecp(int b) { return b == 3 ? R_ET + 3 : R_ECP + b; }
+__device__ __forceinline__ int row_em(int bp, int b) {
+    return bp == b + 1 ? R_ET + b : (bp == 2 ? R_EM20 : b == 1 ? R_EM31 : R_EM30);
+}
+}  // namespace prep2
+
+// Wait for phase `ph` of `bar` with the built-in limit, whatever the run's wait limit: used at
+// exit only, so the copies and products a group has in flight land before its TMEM and shared
+// memory are released, even when the run's waits were set to give up early.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t ph) {
+    (void)mbar_wait_bounded(bar, ph, kWaitLimit);
+}
+
+// Group-local barrier (named barrier 1 + group, 256 threads).
+__device__ __forceinline__ void gbar(int gi) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(prep2::GT) : "memory");
+}
+// The same barrier, returning whether any of the group's threads passed p = true: every thread
+// gets the same answer, so a give-up seen by one thread ends the item loop for all of them.
+__device__ __forceinline__ bool gbar_or(int gi, bool p) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.or.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)p), "r"(1 + gi), "r"(prep2::GT)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+        "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+        "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+// bf16 pair -> two floats (the low element first), one integer op each
+__device__ __forceinline__ float2 bf2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t pk2(float2 v) { return pack_bf16(v.x, v.y); }
+// packed FP32 pair arithmetic (one instruction per pair on sm_100)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+// 2^x with the hardware approximation (relative error about 2^-22)
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float tanh_hw(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// SiLU of a pair: x sigmoid(x), sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh
+__device__ __forceinline__ float2 silu2(float2 x) {
+    const float2 h = mul2(x, dup2(0.5f));
+    const float2 t = make_float2(tanh_hw(h.x), tanh_hw(h.y));
+    return mul2(x, fma2(t, dup2(0.5f), dup2(0.5f)));
+}
+__device__ __forceinline__ uint4 ld16(const uint8_t *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ void st16(uint8_t *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(a, b, c, d);
+}
+__device__ __forceinline__ void ld4f2(const float *p, float2 (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = make_float2(a.x, a.y);
+    v[1] = make_float2(a.z, a.w);
+    v[2] = make_float2(b.x, b.y);
+    v[3] = make_float2(b.z, b.w);
+}
+
+// The prep's work for one item group.  vc / nv: this group's index among all groups of the
+// prep CTAs and their number.  MEGA: items are taken chunk-major and each record is published
+// (flags[item], release) once its stores are visible; otherwise items are taken chunk-fastest
+// and the scan is the next kernel.  PRO: the tiles hold the raw branch inputs and z; the short
+// convolution, SiLU, the gate and beta = sigmoid(logit) run on chip first.
+template <bool PRO, bool MEGA>
+__device__ __forceinline__ void
+prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap *ptm_v,
+            const CUtensorMap *ptm_g, const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws,
+            int T, int H, int BH, KernelFlags fl, PrepPrologue pro, int gi, uint8_t *gsm, uint32_t gtm, int vc,
+            int nv, int *__restrict__ flags, uint32_t wait_limit) {
+    using namespace prep2;
+    const uint32_t gs = smem_u32(gsm);
+    float *TOT = reinterpret_cast<float *>(gsm + OFF_TOT);
+    float *FT = reinterpret_cast<float *>(gsm + OFF_TAB + TAB_F);
+    float *NRMP = reinterpret_cast<float *>(gsm + OFF_TAB + TAB_NRMP);
+    float *BET = reinterpret_cast<float *>(gsm + OFF_TAB + TAB_BET);
+    float *AKT = reinterpret_cast<float *>(gsm + OFF_AKT);
+    float *TMF = reinterpret_cast<float *>(gsm + OFF_TMF);
+    GroupBars *gb = reinterpret_cast<GroupBars *>(gsm + OFF_TAB + TAB_BAR);
+    const uint32_t b_qk = smem_u32(&gb->qk), b_g = smem_u32(&gb->g), b_v = smem_u32(&gb->v),
+                   b_m1 = smem_u32(&gb->m1), b_m2 = smem_u32(&gb->m2), b_m3 = smem_u32(&gb->m3);
+    volatile int *abort_f = &gb->abort;
+
+    const int gt = threadIdx.x - gi * GT;       // thread within the group
+    const int gw = gt >> 5, lane = gt & 31;     // warp within the group (TMEM quadrant gw & 3)
+    const int qd = gw & 3;
+    const uint32_t tl = gtm + ((uint32_t)(qd * 32) << 16);   // this warp's TMEM lanes
+    const int nch = (T + C - 1) / C;
+    const int nitems = nch * BH;
+    constexpr uint32_t kTile = 8192;             // one 64-row x 64-channel box
+
+    if (gt == 0) {
+        mbar_init(b_qk, 1);
+        mbar_init(b_g, 1);
+        mbar_init(b_v, 1);
+        mbar_init(b_m1, 1);
+        mbar_init(b_m2, 1);
+        mbar_init(b_m3, 1);
+        mbar_fence_init();
+        *abort_f = 0;
+    }
+    if (gt < 128) FT[R_ONE * 128 + gt] = 1.f;
+    // constant TMEM operands: L = [L_band; L_band] (lane m, row m & 63: ones at s <= row inside
+    // the row's band), and the zero halves of the block-diagonal Tm' operand
+    if (gw < 4) {
+        const int m = qd * 32 + lane, rr = m & 63;
+        uint32_t lv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int s0 = 2 * j, s1 = 2 * j + 1;
+            const uint32_t lo = ((s0 >> 4) == (rr >> 4) && s0 <= rr) ? 0x3F80u : 0u;
+            const uint32_t hi = ((s1 >> 4) == (rr >> 4) && s1 <= rr) ? 0x3F80u : 0u;
+            lv[j] = lo | (hi << 16);
+        }
+        tmem_st32(tl + TC_LM, lv);
+        uint32_t z[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) z[j] = 0u;
+        tmem_st32(tl + TC_TM + (qd < 2 ? 32 : 0), z);
+        tmem_wait_st();
+    }
+    tc_fence_before();
+    gbar(gi);
+    tc_fence_after();
+
+    // MN-major [K rows][N] tiles (g / K e^gamma, v): 64-channel halves 8 KB apart, 8-row groups 1 KB
+    const uint64_t dT = sdesc(gs, 8192, 1024, kSwizzle128B);
+    auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
+    // A bounded wait by every calling thread.  Giving up (or seeing another thread's give-up)
+    // sets this thread's `bad`; the group leaves the item loop together at the next gbar_or.
+    bool bad = false;
+    auto wait = [&](uint32_t bar, uint32_t phase) -> bool {
+        for (uint32_t i = 0; i < wait_limit; ++i) {
+            if (mbar_try_wait(bar, phase)) return true;
+            if (*abort_f) {
+                bad = true;
+                return false;
+            }
+            if (i > 64) __nanosleep(32);
+        }
+        *abort_f = 1;
+        g_kda_tc2_error = 1;
+        bad = true;
+        return false;
+    };
+
+    auto item_ch = [&](int item) { return MEGA ? item / BH : item % nch; };
+    auto item_bh = [&](int item) { return MEGA ? item % BH : item / nch; };
+    // TMA: q and k on one barrier, g and v on one each
+    auto issue_qk = [&](int item) {
+        const int ich = item_ch(item), ibh = item_bh(item), ib = ibh / H, ih = ibh % H, it0 = ich * C;
+        mbar_arrive_expect_tx(b_qk, 4u * kTile);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(gs + OFF_X + hf * 16384, ptm_q, b_qk, hf * 64, ih, it0, ib);
+            tma_load_4d(gs + OFF_X + hf * 16384 + 8192, ptm_k, b_qk, hf * 64, ih, it0, ib);
+        }
+    };
+    auto issue_gv = [&](int item) {
+        const int ich = item_ch(item), ibh = item_bh(item), ib = ibh / H, ih = ibh % H, it0 = ich * C;
+        mbar_arrive_expect_tx(b_g, 2u * kTile);
+        mbar_arrive_expect_tx(b_v, 2u * kTile);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            tma_load_4d(gs + OFF_G + hf * 8192, ptm_g, b_g, hf * 64, ih, it0, ib);
+            tma_load_4d(gs + OFF_V + hf * 8192, ptm_v, b_v, hf * 64, ih, it0, ib);
+        }
+    };
+    // completions issued and consumed per barrier (thread 0 of the group), for the drain:
+    // qk, g, v, m1, m2, m3
+    uint32_t iss[6] = {0, 0, 0, 0, 0, 0}, con[6] = {0, 0, 0, 0, 0, 0};
+    if (gt == 0 && vc < nitems) {
+        issue_qk(vc);
+        issue_gv(vc);
+        iss[0] = iss[1] = iss[2] = 1;
+    }
+    // beta (or its logit) of token row gt < C, one item ahead
+    auto load_beta = [&](int it) -> float {
+        if (gt >= C || it >= nitems) return 0.f;
+        const int ich = item_ch(it), ibh = item_bh(it), t = ich * C + gt;
+        if (t >= T) return 0.f;
+        const size_t bth = ((size_t)(ibh / H) * T + t) * H + ibh % H;
+        return PRO ? pro.b_logit[bth] : __bfloat162float(beta[bth]);
+    };
+    float bpre = load_beta(vc);
+    uint32_t li = 0;
+    for (int item = vc; item < nitems; item += nv, ++li) {
+        const int ch = item_ch(item), bh = item_bh(item), b = bh / H, h = bh % H;
+        const int t0 = ch * C, n = min(C, T - t0);
+        const int next = item + nv;
+        uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
+        if (gt < C)
+            BET[gt] = gt >= n ? 0.f : PRO ? __bfloat162float(__float2bfloat16_rn(sigmoid_fast(bpre))) : bpre;
+        bpre = load_beta(next);
+        const uint32_t ph = li & 1u;
+        // PRO: the global-memory inputs of the convolution (the three rows before the chunk for
+        // the first segment, the head's taps, A_h) are loaded before the tile wait, so their
+        // latency overlaps it
+        const int br = gt >> 6, pcg = ((gt >> 5) & 1) * 8 + (gt & 7), seg = (gt >> 3) & 3;
+        uint4 halo[3];
+        float a_h = 0.f;
+        if constexpr (PRO) {
+            if (br < 3) {
+                const __nv_bfloat16 *rawp = br == 0 ? pro.raw_q : br == 1 ? pro.raw_k : pro.raw_v;
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    const int t = t0 - 3 + j;
+                    halo[j] = (seg == 0 && t >= 0)
+                                  ? *reinterpret_cast<const uint4 *>(rawp + (((size_t)b * T + t) * H + h) * D + 8 * pcg)
+                                  : make_uint4(0, 0, 0, 0);
+                }
+            } else {
+                a_h = pro.A[h];
+            }
+        }
+        if (wait(b_qk, ph) && gt == 0) ++con[0];
+        if constexpr (PRO) {
+            // ---- short convolution k = 4 + SiLU of q, k, v and the bounded gate, in place.
+            // Thread = (branch, 8-channel group, 16-row segment) for q, k, v (192 threads), or
+            // (8-channel group, 16-row segment) for the gate (64 threads).  The three rows before
+            // a segment come from the segment above (read before the barrier, so the in-place
+            // writes cannot race) or, for the first segment, from global memory (zero before t = 0).
+            if (wait(b_g, ph) && gt == 0) ++con[1];
+            if (wait(b_v, ph) && gt == 0) ++con[2];
+            if (gbar_or(gi, bad)) break;
+            // lanes of a quarter-warp take the 8 channel groups of one row: conflict-free
+            const int cg = pcg, r0 = 16 * seg;
+            const uint32_t ubase = br == 0 ? OFF_X : br == 1 ? OFF_X + 8192 : br == 2 ? OFF_V : OFF_G;
+            auto unit = [&](int r) -> uint32_t {
+                return ubase + (br < 2 ? (uint32_t)((cg >> 3) * 16384) : (uint32_t)((cg >> 3) * 8192)) +
+                       (uint32_t)(r * 128 + (((cg & 7) ^ (r & 7)) << 4));
+            };
+            if (br < 3) {
+                float2 xm[3][4];   // rows r0 - 3 .. r0 - 1, channel pairs
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    const uint4 u = seg > 0 ? ld16(gsm + unit(r0 - 3 + j)) : halo[j];
+                    xm[j][0] = bf2(u.x);
+                    xm[j][1] = bf2(u.y);
+                    xm[j][2] = bf2(u.z);
+                    xm[j][3] = bf2(u.w);
+                }
+                float2 w[4][4];   // [tap][channel pair]: the head's taps, [c][tap] in memory
+                const uint4 *wsrc = reinterpret_cast<const uint4 *>(pro.conv_w + ((size_t)br * H * D + (size_t)h * D + 8 * cg) * 4);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {   // channels 2m, 2m + 1
+                    const uint4 u = wsrc[m];
+                    const float2 a = bf2(u.x), bq = bf2(u.y), c2 = bf2(u.z), d2 = bf2(u.w);   // taps (0,1),(2,3) of 2m; of 2m+1
+                    w[0][m] = make_float2(a.x, c2.x);
+                    w[1][m] = make_float2(a.y, c2.y);
+                    w[2][m] = make_float2(bq.x, d2.x);
+                    w[3][m] = make_float2(bq.y, d2.y);
+                }
+                gbar(gi);
+                const bool tail = n < C;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int r = r0 + i;
+                    const uint4 u = ld16(gsm + unit(r));
+                    const float2 x3[4] = {bf2(u.x), bf2(u.y), bf2(u.z), bf2(u.w)};
+                    uint32_t y[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        float2 acc = mul2(w[0][m], xm[0][m]);
+                        acc = fma2(w[1][m], xm[1][m], acc);
+                        acc = fma2(w[2][m], xm[2][m], acc);
+                        acc = fma2(w[3][m], x3[m], acc);
+                        y[m] = pk2(silu2(acc));
+                        xm[0][m] = xm[1][m];
+                        xm[1][m] = xm[2][m];
+                        xm[2][m] = x3[m];
+                    }
+                    if (tail && r >= n) y[0] = y[1] = y[2] = y[3] = 0u;
+                    st16(gsm + unit(r), y[0], y[1], y[2], y[3]);
+                }
+            } else {
+                const float2 ea = dup2(0.5f * expf(a_h));   // sigmoid(a z) = (1 + tanh(a z / 2)) / 2
+                gbar(gi);
+                const bool tail = n < C;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int r = r0 + i;
+                    const uint4 u = ld16(gsm + unit(r));
+                    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t y[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 hz = mul2(bf2(uw[m]), ea);
+                        const float2 t = make_float2(tanh_hw(hz.x), tanh_hw(hz.y));
+                        y[m] = pk2(fma2(t, dup2(-2.5f), dup2(-2.5f)));   // -5 sigmoid
+                    }
+                    if (tail && r >= n) y[0] = y[1] = y[2] = y[3] = 0u;
+                    st16(gsm + unit(r), y[0], y[1], y[2], y[3]);
+                }
+            }
+            fence_proxy_async();   // g and v are read by the tensor cores
+            gbar(gi);
+        }
+        // ---- band-local cumsum on the tensor cores: D[0,128) = [L_band; L_band] g
+        if (gt == 0) {
+            const bool g_ok = PRO || wait(b_g, ph);
+            if (!PRO && g_ok) ++con[1];
+            tc_fence_after();
+            if (g_ok) {
+                constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_ts(gtm + TC_D, gtm + TC_LM + 8 * s, at(dT, OFF_G + 2048 * s), id, s > 0);
+                mma_commit(b_m1);
+                ++iss[3];
+            }
+        }
+        // ---- meanwhile: sums of squares of the rows of [q; k] (thread = row, one 64-channel half)
+        {
+            const int row = gt & 127, hf = gt >> 7;
+            const int t = row >> 6, r = row & 63;
+            float2 ss = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const uint4 u = ld16(gsm + OFF_X + off_x(t, r, 8 * hf + m));
+                float2 x = bf2(u.x);
+                ss = fma2(x, x, ss);
+                x = bf2(u.y);
+                ss = fma2(x, x, ss);
+                x = bf2(u.z);
+                ss = fma2(x, x, ss);
+                x = bf2(u.w);
+                ss = fma2(x, x, ss);
+            }
+            NRMP[hf * 128 + row] = ss.x + ss.y;
+        }
+        if (gbar_or(gi, bad)) break;
+        if (wait(b_m1, ph) && gt == 0) ++con[3];
+        tc_fence_after();
+        // ---- thread = (row r, channels 32 cq .. 32 cq + 31): the band-local cumsum; the last row of
+        // each band holds the band totals
+        const int r = 32 * (gw & 1) + lane, cq = gw >> 1, band = r >> 4;
+        float gam[32];
+        tmem_ld32(tl + TC_D + 32 * cq, gam);
+        if ((r & 15) == 15) {
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                *reinterpret_cast<float4 *>(TOT + band * 128 + 32 * cq + 4 * m) =
+                    make_float4(gam[4 * m], gam[4 * m + 1], gam[4 * m + 2], gam[4 * m + 3]);
+        }
+        gbar(gi);
+        // ---- per-channel band factors (threads 0-127)
+        if (gt < 128) {
+            const int c = gt;
+            float et[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) et[p] = __expf(fmaxf(TOT[p * 128 + c], -85.f));
+            FT[(R_ET + 0) * 128 + c] = et[0];
+            FT[(R_ET + 1) * 128 + c] = et[1];
+            FT[(R_ET + 2) * 128 + c] = et[2];
+            FT[(R_ET + 3) * 128 + c] = et[3];
+            const float e01 = et[0] * et[1], e12 = et[1] * et[2], e23 = et[2] * et[3];
+            FT[R_EP2 * 128 + c] = e01;
+            FT[R_EP3 * 128 + c] = e01 * et[2];
+            const float eC = e01 * e23;
+            FT[(R_ECP + 0) * 128 + c] = eC;
+            FT[(R_ECP + 1) * 128 + c] = et[1] * e23;
+            FT[(R_ECP + 2) * 128 + c] = e23;
+            FT[R_EM20 * 128 + c] = e01;
+            FT[R_EM31 * 128 + c] = e12;
+            FT[R_EM30 * 128 + c] = e01 * et[2];
+            reinterpret_cast<float *>(img + IMG_GC)[c] = eC;
+        }
+        gbar(gi);
+
+        // ---- operands (thread = row r, 32 channels): E = e^{gamma~}, 1/E; Q E and beta K E in
+        // place; K e^gamma over g; the band-pair B rows k e^{p_b - gamma} for b >= band(r); the
+        // record's Q e^gamma and K e^{gamma_C - gamma}
+        {
+            const float nq = fl.l2norm ? rsqrtf(NRMP[r] + NRMP[128 + r] + kL2Eps) : 1.f;
+            const float nk = fl.l2norm ? rsqrtf(NRMP[64 + r] + NRMP[192 + r] + kL2Eps) : 1.f;
+            const float2 nq2 = dup2(nq), nk2 = dup2(nk), bt2 = dup2(BET[r]);
+            const float *ep = FT + row_ep(band) * 128, *ecp = FT + row_ecp(band) * 128;
+            constexpr float kL2E = 1.4426950408889634f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cg = 4 * cq + m, c0 = 8 * cg;
+                const uint4 uq = ld16(gsm + OFF_X + off_x(0, r, cg));
+                const uint4 uk = ld16(gsm + OFF_X + off_x(1, r, cg));
+                const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
+                float2 fp[4], fc[4];
+                ld4f2(ep + c0, fp);
+                ld4f2(ecp + c0, fc);
+                uint32_t o_qe[4], o_qg[4], o_ke[4], o_kg[4], o_kh[4], o_kd[4];
+                float2 kh[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 sg = mul2(make_float2(fmaxf(gam[8 * m + 2 * e], -85.f), fmaxf(gam[8 * m + 2 * e + 1], -85.f)),
+                                           dup2(kL2E));
+                    const float2 E = make_float2(ex2(sg.x), ex2(sg.y));
+                    const float2 iE = make_float2(ex2(-sg.x), ex2(-sg.y));
+                    const float2 qe = mul2(bf2(wq[e]), mul2(E, nq2));
+                    const float2 kv = bf2(wk[e]);
+                    const float2 ke = mul2(kv, mul2(E, nk2));
+                    kh[e] = mul2(kv, mul2(iE, nk2));
+                    o_qe[e] = pk2(qe);
+                    o_qg[e] = pk2(mul2(qe, fp[e]));
+                    o_ke[e] = pk2(mul2(ke, bt2));
+                    o_kg[e] = pk2(mul2(ke, fp[e]));
+                    o_kh[e] = pk2(kh[e]);
+                    o_kd[e] = pk2(mul2(kh[e], fc[e]));
+                }
+                st16(gsm + OFF_X + off_x(0, r, cg), o_qe[0], o_qe[1], o_qe[2], o_qe[3]);
+                st16(gsm + OFF_X + off_x(1, r, cg), o_ke[0], o_ke[1], o_ke[2], o_ke[3]);
+                st16(gsm + OFF_G + off_t(r, cg), o_kg[0], o_kg[1], o_kg[2], o_kg[3]);
+                st16(gsm + OFF_KH + off_kh(16 * pair_of(band, band) + (r & 15), cg), o_kh[0], o_kh[1], o_kh[2], o_kh[3]);
+                st16(img + IMG_QG + off_r128(r, c0), o_qg[0], o_qg[1], o_qg[2], o_qg[3]);
+                st16(img + IMG_KD + off_r128(r, c0), o_kd[0], o_kd[1], o_kd[2], o_kd[3]);
+                for (int bp = band + 1; bp < 4; ++bp) {
+                    float2 f[4];
+                    ld4f2(FT + row_em(bp, band) * 128 + c0, f);
+                    st16(gsm + OFF_KH + off_kh(16 * pair_of(bp, band) + (r & 15), cg), pk2(mul2(kh[0], f[0])),
+                         pk2(mul2(kh[1], f[1])), pk2(mul2(kh[2], f[2])), pk2(mul2(kh[3], f[3])));
+                }
+            }
+            fence_proxy_async();
+        }
+        tc_fence_before();
+        if (gbar_or(gi, bad)) break;
+        // ---- all ten band pairs: D[0,160) = [Q E; beta K E] (B rows)^T
+        if (gt == 0) {
+            tc_fence_after();
+            constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint64_t da = sdesc(gs + OFF_X + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024, kSwizzle128B);
+                const uint64_t db = sdesc(gs + OFF_KH + (s >> 2) * KH_HALF + (s & 3) * 32, 16, 1024, kSwizzle128B);
+                mma_ss(gtm + TC_D, da, db, id, s > 0);
+            }
+            mma_commit(b_m2);
+            ++iss[4];
+        }
+        const bool m2_ok = wait(b_m2, ph);
+        if (gt == 0 && m2_ok) {
+            ++con[4];
+            if (next < nitems) {   // the q / k staging is free: the next item's tiles
+                issue_qk(next);
+                ++iss[0];
+            }
+        }
+        tc_fence_after();
+        // ---- A_qk -> record (lanes 0-63), A_kk -> FP32 transposed (lanes 64-127); warp gw covers
+        // column bands 2h, 2h + 1 of its 32 rows
+        {
+            const int hh = gw >> 2, b_lo = 2 * (qd & 1);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * hh + jj;
+                float v[16], v2[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                if (j <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, j), v);
+                if (j <= b_lo + 1) {
+                    tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, j), v2);
+                    if (band == b_lo + 1) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                    }
+                }
+                if (qd < 2) {
+#pragma unroll
+                    for (int g8 = 0; g8 < 2; ++g8) {
+                        uint32_t y[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i = 16 * j + 8 * g8 + 2 * e;
+                            y[e] = pk2(make_float2(i <= r ? v[8 * g8 + 2 * e] : 0.f, i + 1 <= r ? v[8 * g8 + 2 * e + 1] : 0.f));
+                        }
+                        st16(img + IMG_AQK + off_r64(r, 16 * j + 8 * g8), y[0], y[1], y[2], y[3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int i = 16 * j + e;
+                        AKT[i * AS + r] = (i < r) ? v[e] : 0.f;   // a warp writes 32 consecutive r
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        if (gbar_or(gi, bad)) break;
+
+        // ---- Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks [T1 0; T21 T2]: the 16 x 16 diagonal
+        // blocks D_b by column sweeps (lane = column, two blocks per warp, x_i final once the rows
+        // above are done, then x_r -= A[r][i] x_i for r > i); per 32-block Z = A10 D0, X = -D1 Z;
+        // then Y = A21 T1, T21 = -T2 Y.  TMF holds T (rows 0-31 hold Z, then Y, in columns 32-63).
+        if (gw < 2) {
+            const int blk = 2 * gw + (lane >> 4), base = 16 * blk, j = lane & 15;
+            float x[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < 15; ++i) {
+                const float xi = x[i];
+                const float *col = AKT + (base + i) * AS + base;   // A[base + rr][base + i] over rr
+#pragma unroll
+                for (int r4 = ((i + 1) >> 2) << 2; r4 < 16; r4 += 4) {   // rows rr <= i hold 0
+                    const float4 av = *reinterpret_cast<const float4 *>(col + r4);
+                    x[r4] = fmaf(-av.x, xi, x[r4]);
+                    x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
+                    x[r4 + 2] = fmaf(-av.z, xi, x[r4 + 2]);
+                    x[r4 + 3] = fmaf(-av.w, xi, x[r4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) TMF[(base + rr) * AS + base + j] = x[rr];
+            if ((blk & 1) == 0) {   // the zero upper-right quarter of each 32-block's T
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) TMF[(base + rr) * AS + base + 16 + j] = 0.f;
+            }
+        }
+        gbar(gi);
+        // Z = A10 D0 per 32-block hb (warps 0-3: block hb = gw >> 1, columns 8 (gw & 1) .. + 7;
+        // 2 x 2 tiles: rows 2 rp, 2 rp + 1, columns 2 cp, 2 cp + 1)
+        if (gw < 4) {
+            const int hb = gw >> 1, base = 32 * hb, rp = lane >> 2, c2 = 8 * (gw & 1) + 2 * (lane & 3);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float2 a = *reinterpret_cast<const float2 *>(AKT + (base + k) * AS + base + 16 + 2 * rp);   // A10[2rp..][k]
+                const float2 d = *reinterpret_cast<const float2 *>(TMF + (base + k) * AS + base + c2);            // D0[k][c2..]
+                acc0 = fma2(dup2(a.x), d, acc0);
+                acc1 = fma2(dup2(a.y), d, acc1);
+            }
+            *reinterpret_cast<float2 *>(TMF + (2 * rp) * AS + 32 + 16 * hb + c2) = acc0;
+            *reinterpret_cast<float2 *>(TMF + (2 * rp + 1) * AS + 32 + 16 * hb + c2) = acc1;
+        }
+        gbar(gi);
+        // X = -D1 Z -> rows 16-31 of the 32-block, columns 0-15 (same split)
+        if (gw < 4) {
+            const int hb = gw >> 1, base = 32 * hb, rp = lane >> 2, c2 = 8 * (gw & 1) + 2 * (lane & 3);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int k4 = 0; k4 < 16; k4 += 4) {
+                const float4 d0 = *reinterpret_cast<const float4 *>(TMF + (base + 16 + 2 * rp) * AS + base + 16 + k4);
+                const float4 d1 = *reinterpret_cast<const float4 *>(TMF + (base + 17 + 2 * rp) * AS + base + 16 + k4);
+                const float a0[4] = {d0.x, d0.y, d0.z, d0.w}, a1[4] = {d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float2 z = *reinterpret_cast<const float2 *>(TMF + (k4 + kk) * AS + 32 + 16 * hb + c2);
+                    acc0 = fma2(dup2(a0[kk]), z, acc0);
+                    acc1 = fma2(dup2(a1[kk]), z, acc1);
+                }
+            }
+            *reinterpret_cast<float2 *>(TMF + (base + 16 + 2 * rp) * AS + base + c2) = make_float2(-acc0.x, -acc0.y);
+            *reinterpret_cast<float2 *>(TMF + (base + 17 + 2 * rp) * AS + base + c2) = make_float2(-acc1.x, -acc1.y);
+        }
+        gbar(gi);
+        // Y = A21 T1 (2 x 2 tiles over 256 threads) -> rows 0-31, columns 32-63 (where Z was)
+        {
+            const int rp = gt >> 4, c2 = 2 * (gt & 15);   // rows 2 rp, 2 rp + 1; columns c2, c2 + 1
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#pragma unroll 8
+            for (int k = 0; k < 32; ++k) {
+                const float2 a = *reinterpret_cast<const float2 *>(AKT + k * AS + 32 + 2 * rp);   // A21[2rp..][k]
+                const float2 t = *reinterpret_cast<const float2 *>(TMF + k * AS + c2);            // T1[k][c2..]
+                acc0 = fma2(dup2(a.x), t, acc0);
+                acc1 = fma2(dup2(a.y), t, acc1);
+            }
+            *reinterpret_cast<float2 *>(TMF + (2 * rp) * AS + 32 + c2) = acc0;
+            *reinterpret_cast<float2 *>(TMF + (2 * rp + 1) * AS + 32 + c2) = acc1;
+        }
+        gbar(gi);
+        // T21 = -T2 Y -> rows 32-63, columns 0-31
+        {
+            const int rp = gt >> 4, c2 = 2 * (gt & 15);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#pragma unroll 2
+            for (int k4 = 0; k4 < 32; k4 += 4) {
+                const float4 d0 = *reinterpret_cast<const float4 *>(TMF + (32 + 2 * rp) * AS + 32 + k4);   // T2[2rp][k4..]
+                const float4 d1 = *reinterpret_cast<const float4 *>(TMF + (33 + 2 * rp) * AS + 32 + k4);
+                const float a0[4] = {d0.x, d0.y, d0.z, d0.w}, a1[4] = {d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const float2 y = *reinterpret_cast<const float2 *>(TMF + (k4 + kk) * AS + 32 + c2);   // Y[k][c2..]
+                    acc0 = fma2(dup2(a0[kk]), y, acc0);
+                    acc1 = fma2(dup2(a1[kk]), y, acc1);
+                }
+            }
+            *reinterpret_cast<float2 *>(TMF + (32 + 2 * rp) * AS + c2) = make_float2(-acc0.x, -acc0.y);
+            *reinterpret_cast<float2 *>(TMF + (33 + 2 * rp) * AS + c2) = make_float2(-acc1.x, -acc1.y);
+        }
+        gbar(gi);
+        // ---- Tm' = Tm diag(beta) -> the block-diagonal operand: lanes 0-63 get [Tm' | 0] (warps 0,
+        // 1), lanes 64-127 get [0 | Tm'] (warps 6, 7); the zero halves were written once
+        if (gw < 2 || gw >= 6) {
+            uint32_t tv[32];
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int i0 = 4 * m;
+                const float4 t4 = *reinterpret_cast<const float4 *>(TMF + r * AS + i0);
+                const float4 b4 = *reinterpret_cast<const float4 *>(BET + i0);
+                // T's upper triangle: zero by construction except rows 0-31 x columns 32-63 (Y)
+                const bool z = (r < 32 && i0 >= 32);
+                tv[2 * m] = z ? 0u : pk2(mul2(make_float2(t4.x, t4.y), make_float2(b4.x, b4.y)));
+                tv[2 * m + 1] = z ? 0u : pk2(mul2(make_float2(t4.z, t4.w), make_float2(b4.z, b4.w)));
+            }
+            tmem_st32(tl + TC_TM + (qd < 2 ? 0 : 32), tv);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        if (gbar_or(gi, bad)) break;
+        // ---- [W; U] = [Tm' 0; 0 Tm'] [K e^gamma; V]
+        if (gt == 0) {
+            bool v_ok = true;
+            if constexpr (!PRO) {
+                v_ok = wait(b_v, ph);
+                if (v_ok) ++con[2];
+            }
+            tc_fence_after();
+            if (v_ok) {
+                constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const uint64_t db = s < 4 ? at(dT, OFF_G + 2048 * s) : at(dT, OFF_V + 2048 * (s - 4));
+                    mma_ts(gtm + TC_D, gtm + TC_TM + 8 * s, db, id, s > 0);
+                }
+                mma_commit(b_m3);
+                ++iss[5];
+            }
+        }
+        const bool m3_ok = wait(b_m3, ph);
+        if (gt == 0 && m3_ok) {
+            ++con[5];
+            if (next < nitems) {   // g and v staging are free again
+                issue_gv(next);
+                ++iss[1];
+                ++iss[2];
+            }
+        }
+        tc_fence_after();
+        // ---- W (lanes 0-63) and U (lanes 64-127) -> record, 64 channels per thread
+        {
+            const int hh = gw >> 2;
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+                float w[32];
+                tmem_ld32(tl + TC_D + 64 * hh + 32 * hc, w);
+#pragma unroll
+                for (int g8 = 0; g8 < 4; ++g8) {
+                    const int c0 = 64 * hh + 32 * hc + 8 * g8;
+                    const float *x = w + 8 * g8;
+                    st16(img + (qd < 2 ? IMG_W + off_r128(r, c0) : IMG_U + off_u(r, c0)), pk2(make_float2(x[0], x[1])),
+                         pk2(make_float2(x[2], x[3])), pk2(make_float2(x[4], x[5])), pk2(make_float2(x[6], x[7])));
+                }
+            }
+        }
+        if constexpr (MEGA) __threadfence();   // this thread's record stores, before the flag
+        tc_fence_before();
+        const bool stop = gbar_or(gi, bad);
+        tc_fence_after();
+        if (stop) break;
+        if (MEGA && gt == 0) flag_release(flags + item, 1);
+    }
+    // drain: let every copy and product this group issued land before TMEM and shared memory go
+    // (each barrier has at most one completion outstanding: the one after those consumed)
+    if (gt == 0) {
+        const uint32_t bars[6] = {b_qk, b_g, b_v, b_m1, b_m2, b_m3};
+#pragma unroll
+        for (int i = 0; i < 6; ++i)
+            if (iss[i] > con[i]) drain_wait(bars[i], con[i] & 1u);
+    }
+    tc_fence_before();
+    gbar(gi);
+}

@@ -768,10 +768,12 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-int chunk_tc_read_error() {
-    int v = 0;
-    cudaMemcpyFromSymbol(&v, g_kda_tc_error, sizeof(int));
-    return v;
+cudaError_t chunk_tc_take_error(int *flag, cudaStream_t st) {
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(flag, g_kda_tc_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_kda_tc_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e;
 }
 
 }  // namespace kda

@@ -28,6 +28,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <stdlib.h>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -150,7 +151,11 @@ struct PrepPrologue {
     const __nv_bfloat16 *conv_w;   // [3, H * D, 4]: taps of q, k, v
     const float *A;                // [H] per-head log-scale of the gate
     const float *b_logit;          // [B, T, H] beta logits (FP32)
+    // the raw branch inputs (the rows before a chunk, for its first convolution outputs)
+    const __nv_bfloat16 *raw_q, *raw_k, *raw_v;
 };
+
+#include "kda_chunk_prep.cuh"
 
 // The prep's work, run by CTA `cta` of `ncta` prep CTAs.  MEGA (the fused prep + scan launch of
 // few-head calls): items are taken chunk-major, so every head's early chunks come first, and
@@ -816,6 +821,46 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                           (int)gridDim.x, nullptr);
 }
 
+// The prep with two item groups per CTA (kda_chunk_prep.cuh): one 512-thread CTA per SM, its
+// TMEM split between the groups.  MEGA: CTA `cta` of `ncta` prep CTAs of the one-launch form.
+template <bool PRO, bool MEGA>
+__device__ __forceinline__ void
+prep2_cta(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap *ptm_v, const CUtensorMap *ptm_g,
+          const __nv_bfloat16 *beta, uint8_t *ws, int T, int H, int BH, KernelFlags fl, PrepPrologue pro,
+          int cta, int ncta, int *flags, uint32_t wait_limit) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t prep_tmem_base;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&prep_tmem_base), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = prep_tmem_base;
+    // the scan kernel, launched with a programmatic dependency on this one, may be scheduled now
+    if (!MEGA) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int gi = threadIdx.x / prep2::GT;
+    prep2_group<PRO, MEGA>(ptm_q, ptm_k, ptm_v, ptm_g, beta, ws, T, H, BH, fl, pro, gi,
+                           smem + gi * prep2::GROUP_STRIDE, tbase + 256u * gi, prep2::NG * cta + gi,
+                           prep2::NG * ncta, flags, wait_limit);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+template <bool PRO>
+__global__ void __launch_bounds__(prep2::NT, 1)
+chunk_prep2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                   const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H, int BH,
+                   KernelFlags fl, PrepPrologue pro, uint32_t wait_limit) {
+    prep2_cta<PRO, false>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x,
+                          (int)gridDim.x, nullptr, wait_limit);
+}
+
 // ============================================================== kernel 2: the scan
 // The value columns of the state evolve independently (column j of S sees only v_{t,j}), so
 // the scan splits a head's dv = 128 columns into slices of NS columns, one CTA each: a slice
@@ -895,6 +940,9 @@ struct alignas(8) ScanBars {
     int abort;                 // a bounded wait gave up: every other wait returns at once
     int s_done;                // MEGA: state-warp updates done (NSW per chunk)
     int o_done;                // MEGA: O products seen complete by the output warps (NSW / 2 per chunk)
+    // completions issued to each barrier (stage[0..2], mV, mS, mO[0], mO[1]): each is written by
+    // the one lane that issues to it, and read at exit to drain what is still in flight
+    int issued[7];
 };
 
 // The scan's work for slice CTA `cta`.  MEGA (run beside the prep in one launch): each record is
@@ -908,7 +956,7 @@ __device__ __forceinline__ void
 scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
           float *__restrict__ S_T, int T, int H, float scale, const __nv_bfloat16 *__restrict__ gate,
           const float *__restrict__ norm_w, float norm_eps, int cta, const int *__restrict__ flags,
-          int nseq) {
+          int nseq, uint32_t poll_limit = kWaitLimit) {
     using L = scan::Layout<NS>;
     constexpr int CPT = L::CPT, NSL = D / NS;
     static_assert(!GATED || NS == D, "the output epilogue normalises whole rows: one slice per head");
@@ -945,6 +993,7 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
         sh.abort = 0;
         sh.s_done = 0;
         sh.o_done = 0;
+        for (int i = 0; i < 7; ++i) sh.issued[i] = 0;
     }
     // the zero rows under each stage's A_qk
     for (int i = tid; i < L::NSTG * 512; i += (int)blockDim.x)
@@ -968,6 +1017,7 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     auto fetch = [&](int ch) {
         const int s = ch % L::NSTG;
         const uint32_t bar = smem_u32(&sh.stage[s]);
+        ++sh.issued[s];
         const uint8_t *src = recs + (size_t)ch * IMG_BYTES;
         mbar_arrive_expect_tx(bar, L::HEAD + L::U_BYTES + L::TAIL_BYTES);
         bulk_load(sbase + s * L::STAGE, src, L::HEAD, bar);
@@ -1085,7 +1135,7 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
                 const int *f = flags + (size_t)c * (size_t)nseq + bh;
                 const int need = c - L::NSTG + 1;   // chunks whose stage must be free
                 bool go = false;
-                for (uint32_t i = 0; i < kWaitLimit; ++i) {
+                for (uint32_t i = 0; i < poll_limit; ++i) {
                     if ((need <= 0 || (smem_acquire_load(a_sdone) >= need * L::NSW &&
                                        smem_acquire_load(a_odone) >= need * L::NPW)) &&
                         flag_acquire(f)) {
@@ -1120,6 +1170,7 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
                 for (int k = 0; k < 8; ++k)
                     mma_ss(tbase + dbuf, at(dK64, st + 256 * k), at(dMNs, L::OFF_S + NS * 32 * k), id, k > 0);
                 mma_commit(b_mV);
+                ++sh.issued[3];
             }
             __syncwarp();
             // the stage of chunk ch - 1 is free once its last products are done and every state
@@ -1139,10 +1190,12 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
                 for (int k = 0; k < 4; ++k)
                     mma_ss(tbase + L::TC_S, at(dMN64, st + IMG_KD + 4096 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_s, k > 0);
                 mma_commit(b_mS);
+                ++sh.issued[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_ss(tbase + dbuf, at(dK32, st + L::ZERO + 256 * k), at(dMNs, L::OFF_VT + NS * 32 * k), id_o, 1);
                 mma_commit(smem_u32(&sh.mO[s]));
+                ++sh.issued[5 + s];
             }
             __syncwarp();
         }
@@ -1217,6 +1270,17 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     }
     tc_fence_before();
     __syncthreads();
+    // drain: after a give-up, copies and products may still be in flight; let each barrier
+    // reach its last issued completion (built-in limit) before TMEM and shared memory go
+    if (tid == 0 && *reinterpret_cast<volatile int *>(&sh.abort)) {
+        const uint32_t bars[7] = {smem_u32(&sh.stage[0]), smem_u32(&sh.stage[1]), smem_u32(&sh.stage[2]),
+                                  b_mV, b_mS, smem_u32(&sh.mO[0]), smem_u32(&sh.mO[1])};
+        for (int i = 0; i < 7; ++i) {
+            const int k = *reinterpret_cast<volatile int *>(&sh.issued[i]);
+            if (k > 0) (void)mbar_wait_bounded(bars[i], (uint32_t)(k - 1) & 1u, kWaitLimit);
+        }
+    }
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, L::TMEM_COLS);
 }
 
@@ -1245,8 +1309,9 @@ constexpr uint32_t mega_smem_bytes() {
 // call's working set has left L2, takes about twice as long.
 template <int NS>
 __device__ __noinline__ void mega_scan(const uint8_t *ws, const float *S0, __nv_bfloat16 *out, float *S_T, int T,
-                                       int H, float scale, int cta, const int *flags, int BH) {
-    scan_body<NS, false, true>(ws, S0, out, S_T, T, H, scale, nullptr, nullptr, 0.f, cta, flags, BH);
+                                       int H, float scale, int cta, const int *flags, int BH,
+                                       uint32_t poll_limit = kWaitLimit) {
+    scan_body<NS, false, true>(ws, S0, out, S_T, T, H, scale, nullptr, nullptr, 0.f, cta, flags, BH, poll_limit);
 }
 
 template <bool PRO, int NS>
@@ -1262,6 +1327,27 @@ chunk_mega_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     else
         prep_body<PRO, true>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro,
                              (int)blockIdx.x - n_scan, (int)gridDim.x - n_scan, flags);
+}
+
+// The one-launch form with the two-group prep: prep CTAs are 512 threads of two item groups.
+template <int NS>
+constexpr uint32_t mega2_smem_bytes() {
+    return prep2::SMEM_BYTES > scan::Layout<NS>::SMEM_BYTES ? prep2::SMEM_BYTES : scan::Layout<NS>::SMEM_BYTES;
+}
+
+template <bool PRO, int NS>
+__global__ void __launch_bounds__(prep2::NT, 1)
+chunk_mega2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                   const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
+                   int BH, KernelFlags fl, PrepPrologue pro, const float *__restrict__ S0,
+                   __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int n_scan,
+                   int *__restrict__ flags, uint32_t wait_limit) {
+    if ((int)blockIdx.x < n_scan)
+        mega_scan<NS>(ws, S0, out, S_T, T, H, fl.scale, (int)blockIdx.x, flags, BH, wait_limit);
+    else
+        prep2_cta<PRO, true>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x - n_scan,
+                             (int)gridDim.x - n_scan, flags, wait_limit);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn2() {
@@ -1306,23 +1392,28 @@ size_t chunk_tc2_workspace_bytes(int B, int T, int H) {
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st);
+static bool use_prep2(const ChunkArgs &a);
 
 cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mg;
     if (!make_map2(&mq, a.q, a.B, a.T, a.H) || !make_map2(&mk, a.k, a.B, a.T, a.H) ||
         !make_map2(&mv, a.v, a.B, a.T, a.H) || !make_map2(&mg, a.g, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr}, st);
+    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr}, st);
 }
 
 cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mz;
-    const int rows = C + prep::kHalo;
+    // the one-group prep stages a 3-row halo with each tile; the two-group prep reads those rows
+    // from global memory and stages 64-row tiles
+    const int rows = use_prep2(a) ? C : C + prep::kHalo;
     if (!make_map2(&mq, p.q_pre, a.B, a.T, a.H, rows) || !make_map2(&mk, p.k_pre, a.B, a.T, a.H, rows) ||
         !make_map2(&mv, p.v_pre, a.B, a.T, a.H, rows) || !make_map2(&mz, p.z, a.B, a.T, a.H, rows))
         return cudaErrorInvalidValue;
     return launch_split(a, mq, mk, mv, mz,
-                        PrepPrologue{(const __nv_bfloat16 *)p.conv_w, p.A, p.beta_logit}, st);
+                        PrepPrologue{(const __nv_bfloat16 *)p.conv_w, p.A, p.beta_logit, (const __nv_bfloat16 *)p.q_pre,
+                                     (const __nv_bfloat16 *)p.k_pre, (const __nv_bfloat16 *)p.v_pre},
+                        st);
 }
 
 // Value-column slice width of the scan: the widest slice (fewest redundant record reads)
@@ -1358,22 +1449,27 @@ static cudaError_t launch_scan(const ChunkArgs &a, const uint8_t *ws, cudaStream
                               (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
 }
 
-// Per-(chunk, head) prep cost and per-chunk scan chain at d = 128 on a B200 SM (cycles, measured).
+// Per-(chunk, head) prep cost per SM (cycles; the two-group prep overlaps two items per SM) and
+// per-chunk scan chain at d = 128 on a B200 SM (measured).
 constexpr double kPrepItemCycles = 21000.0;
+constexpr double kPrep2ItemCycles = 7000.0;
 static double scan_chunk_cycles(int ns) { return ns == 16 ? 2900.0 : ns == 32 ? 3000.0 : ns == 64 ? 3100.0 : 4900.0; }
+
+// Polls of a bounded wait before it gives up (kda_set_wait_limit; failure-handling tests only).
+static uint32_t g_wait_limit = kWaitLimit;
 
 // Slice width of the one-launch form (prep and scan CTAs side by side), or 0 when the two
 // launches are faster: prep on all SMs, then the scan, against the prep on the SMs the scan's
 // CTAs leave, overlapped with the scan, plus one item of ramp.
-int mega_slice_width(int BH, int nch, int sms) {
+int mega_slice_width(int BH, int nch, int sms, double t_item) {
     const double items = (double)BH * nch;
-    const double two = ceil(items / sms) * kPrepItemCycles + nch * scan_chunk_cycles(scan_slice_width(BH, false));
+    const double two = ceil(items / sms) * t_item + nch * scan_chunk_cycles(scan_slice_width(BH, false));
     int best = 0;
     double best_t = 0.9 * two;
     for (int ns : {32, 64}) {
         const int n_scan = BH * (D / ns);
         if (n_scan > sms / 2) continue;
-        const double t = fmax(ceil(items / (sms - n_scan)) * kPrepItemCycles, nch * scan_chunk_cycles(ns)) + kPrepItemCycles;
+        const double t = fmax(ceil(items / (sms - n_scan)) * t_item, nch * scan_chunk_cycles(ns)) + t_item;
         if (t < best_t) {
             best = ns;
             best_t = t;
@@ -1382,14 +1478,36 @@ int mega_slice_width(int BH, int nch, int sms) {
     return best;
 }
 
+cudaError_t chunk_tc2_take_error(int *flag, cudaStream_t st) {
+    const int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(flag, g_kda_tc2_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbolAsync(g_kda_tc2_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e;
+}
+
+uint32_t set_wait_limit(uint32_t polls) {
+    const uint32_t prev = g_wait_limit;
+    g_wait_limit = polls;
+    return prev;
+}
+
+// Whether the two-group prep runs (all unsigned-gate calls; Complex-KDA keeps the one-group prep).
+static bool use_prep2(const ChunkArgs &a) { return !a.fl.complex_gate && getenv("KDA_PREP_FORM") == nullptr; }
+
 template <bool PRO, int NS>
 static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, cudaStream_t st) {
+    const bool v2 = use_prep2(a);
     auto k = chunk_mega_kernel<PRO, NS>;
-    constexpr uint32_t smem = mega_smem_bytes<NS>();
-    static_assert(smem <= 232448, "shared memory budget");
+    auto k2 = chunk_mega2_kernel<PRO, NS>;
+    constexpr uint32_t smem1 = mega_smem_bytes<NS>(), smem2 = mega2_smem_bytes<NS>();
+    static_assert(smem1 <= 232448 && smem2 <= 232448, "shared memory budget");
     static_assert(scan::Layout<NS>::NT + 32 <= prep::NT, "the scan's warps and the loader warp fit the prep's block");
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static_assert(prep::NT == prep2::NT, "one block size for both prep forms");
+    const uint32_t smem = v2 ? smem2 : smem1;
+    cudaError_t e = v2 ? cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                       : cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int nch = (a.T + C - 1) / C, BH = a.B * a.H, n_scan = BH * (D / NS);
     uint8_t *ws = (uint8_t *)a.workspace;
@@ -1408,6 +1526,9 @@ static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     mark_launch(a, st);
+    if (v2)
+        return cudaLaunchKernelEx(&cfg, k2, mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, BH, a.fl,
+                                  pro, a.S0, (__nv_bfloat16 *)a.out, a.S_T, n_scan, flags, g_wait_limit);
     return cudaLaunchKernelEx(&cfg, k, mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, BH, a.fl, pro,
                               a.S0, (__nv_bfloat16 *)a.out, a.S_T, n_scan, flags);
 }
@@ -1415,8 +1536,9 @@ static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const 
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st) {
+    const bool v2 = use_prep2(a);
     if (!a.out_gate) {
-        const int ns = mega_slice_width(a.B * a.H, (a.T + C - 1) / C, num_sms());
+        const int ns = mega_slice_width(a.B * a.H, (a.T + C - 1) / C, num_sms(), v2 ? kPrep2ItemCycles : kPrepItemCycles);
         if (ns) {
             const bool p = pro.conv_w != nullptr;
             cudaError_t e = ns == 32 ? (p ? launch_mega<true, 32>(a, mq, mk, mv, mg, pro, st)
@@ -1428,16 +1550,26 @@ static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const
         }
     }
     // the plain instantiations carry none of the prologue or epilogue code
-    auto prep_k = pro.conv_w ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)prep::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
     const int nch = (a.T + C - 1) / C;
     uint8_t *ws = (uint8_t *)a.workspace;
-    mark_launch(a, st);
     const int nitems = nch * a.B * a.H;
-    prep_k<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
-        mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl, pro);
+    cudaError_t e;
+    if (v2) {
+        auto prep_k = pro.conv_w ? chunk_prep2_kernel<true> : chunk_prep2_kernel<false>;
+        e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep2::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        mark_launch(a, st);
+        const int ctas = std::min((nitems + prep2::NG - 1) / prep2::NG, num_sms());
+        prep_k<<<(unsigned)ctas, prep2::NT, prep2::SMEM_BYTES, st>>>(mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws,
+                                                                    a.T, a.H, a.B * a.H, a.fl, pro, g_wait_limit);
+    } else {
+        auto prep_k = pro.conv_w ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+        e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        mark_launch(a, st);
+        prep_k<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
+            mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl, pro);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark_launch(a, st);

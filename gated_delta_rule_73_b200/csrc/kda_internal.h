@@ -74,10 +74,16 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 // Fused tensor-core chunk path (bf16, dk = dv = 128); needs no workspace.
 bool chunk_tc_supported(const ChunkArgs &a);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t st);
-int chunk_tc_read_error();
+// Read and clear the fused form's device error word (1 = a bounded wait gave up); synchronises st.
+cudaError_t chunk_tc_take_error(int *flag, cudaStream_t st);
 // Two-kernel tensor-core chunk path (parallel prep + per-head scan); needs a workspace.
 size_t chunk_tc2_workspace_bytes(int B, int T, int H);
 cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st);
+// Read and clear the split form's device error word; synchronises st.
+cudaError_t chunk_tc2_take_error(int *flag, cudaStream_t st);
+// Polls before a bounded wait of the split form gives up (the prep's waits, the one-launch
+// scan's wait for published records); returns the previous value.
+uint32_t set_wait_limit(uint32_t polls);
 // The split form with the prologue fused into its prep kernel: the prep stages the raw
 // q, k, v, z tiles with a 3-row halo and applies the short convolution, SiLU, the gate and
 // beta = sigmoid(logit) on chip.  Uses a.out, a.S0, a.S_T, sizes, flags, workspace, events.

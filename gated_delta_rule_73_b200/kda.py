@@ -70,6 +70,10 @@ def _load():
     lib.kda_affine_combine.restype = ip
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
     lib.kda_selftest_bounded_wait.restype = ip
+    lib.kda_device_status.argtypes = [vp]
+    lib.kda_device_status.restype = ip
+    lib.kda_set_wait_limit.argtypes = [ctypes.c_uint]
+    lib.kda_set_wait_limit.restype = ctypes.c_uint
     lib.kda_chunk_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_chunk_workspace_bytes.restype = sz
     lib.kda_prologue_workspace_bytes.argtypes = [ip] * 5 + [op]
@@ -241,6 +245,20 @@ def kda_affine_combine(M, Bp, n, S0, S_out, stream=None) -> None:
                                  _ptr(S_out, "S_out", f), BH, dk, dv, _stream(stream))
     if st != 0:
         raise KdaError("kda_affine_combine", st)
+
+
+KDA_WAIT_LIMIT_DEFAULT = 1 << 22
+
+
+def kda_device_status(stream=None) -> int:
+    """Call ``kda_device_status``: synchronise the stream, read and clear the device error
+    words; returns the status (0, or KDA_ERR_TIMEOUT = -6 when a bounded wait gave up)."""
+    return int(_lib.kda_device_status(_stream(stream)))
+
+
+def kda_set_wait_limit(polls: int) -> int:
+    """Call ``kda_set_wait_limit``; returns the previous limit."""
+    return int(_lib.kda_set_wait_limit(int(polls)))
 
 
 def kda_selftest_bounded_wait(limit: int, stream=None) -> int:

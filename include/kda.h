@@ -20,7 +20,11 @@
  *    library never allocates or frees memory and keeps no state between calls.
  *  - Asynchrony: work is enqueued on `stream`; the return value reports
  *    argument and launch errors only.  Kernel faults surface at the caller's
- *    next synchronisation.
+ *    next synchronisation.  The tensor-core chunk kernels wait on each other
+ *    only through bounded loops (mbarriers of their own CTA; in the one-launch
+ *    form, the scan CTAs on flags the prep CTAs publish); a wait that runs out
+ *    sets a device error word and the kernel returns with its outputs
+ *    unwritten.  kda_device_status() reads and clears that word.
  *  - Errors: a negative status (see kda_status); no exception and no device
  *    trap ever crosses the ABI.  Arguments are checked on the host before any
  *    CUDA call is made.
@@ -365,12 +369,38 @@ int kda_affine_combine(const float *M, const float *Bp, int n, const float *S0,
  */
 int kda_selftest_bounded_wait(unsigned limit, cudaStream_t stream);
 
+/*
+ * kda_device_status -- the outcome of the kernels already enqueued on `stream`.
+ *
+ * The pages have no counterpart: this is the library's failure reporting.  Synchronises
+ * `stream`, then reads and clears the device error words the tensor-core chunk kernels set
+ * when one of their bounded waits gives up.  Returns KDA_OK when none did, KDA_ERR_TIMEOUT
+ * when one did since the last call (that call's out and S_T are not valid), KDA_ERR_CUDA if
+ * the synchronisation or the copies failed.  The words are per device and shared by all
+ * streams: call it with no other chunk work in flight on the device.
+ */
+int kda_device_status(cudaStream_t stream);
+
+/*
+ * kda_set_wait_limit -- polls a bounded wait of the split tensor-core form makes before it
+ * gives up (the prep kernel's waits and the one-launch form's wait for published records).
+ *
+ * The pages have no counterpart: this exists so failure handling can be tested on a GPU
+ * without a fault.  0 makes those waits give up at once: the call then ends early with
+ * KDA_ERR_TIMEOUT reported by kda_device_status(), copies and products already in flight
+ * are drained first, and nothing faults.  KDA_WAIT_LIMIT_DEFAULT restores normal operation.
+ * Returns the previous limit.  Host-global; not thread-safe against concurrent calls.
+ */
+#define KDA_WAIT_LIMIT_DEFAULT (1u << 22)
+unsigned kda_set_wait_limit(unsigned polls);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(int status);
 
 /* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
    1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd;
-   1.6: kda_segment_pair, kda_affine_combine; 1.7: kda_selftest_bounded_wait). */
+   1.6: kda_segment_pair, kda_affine_combine; 1.7: kda_selftest_bounded_wait;
+   1.8: kda_device_status, kda_set_wait_limit). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus
