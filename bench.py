@@ -3,21 +3,24 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one ``kda_chunk_fwd`` over the prefill workload (B=1, T=4096, H=16,
-dk=dv=128, bf16 q/k/v/g/beta, FP32 S0 -> out, S_T), inputs resident in HBM.
-The workload's inputs (86 MB) fit in the 126 MB L2, so a 256 MiB buffer is
-written between timed steps (outside the timed events).  Under torchrun every
-rank runs its own batch (weak scaling, no collective on the data path);
-``value`` is the tokens of all ranks over the slowest rank's time.
+A step is one ``kda_chunk_fwd_prologue`` over the largest length-sweep workload
+(B=1, T=65536, H=96, dk=dv=128, bf16 raw q/k/v/z, FP32 beta logits, conv taps and
+S0 -> out, S_T): the fused prologue (short conv k=4 + SiLU, gate, beta), the
+chunk-local cumsum, A_kk / A_qk / UT / WY and the inter-chunk scan, inputs resident
+in HBM.  Its inputs (8 GB) are larger than the 126 MB L2, so no flush is needed
+between steps.  Under torchrun every rank runs its own batch (weak scaling, no
+collective on the data path); ``value`` is the tokens of all ranks over the
+slowest rank's time.
 
 Also measured on rank 0 at N=1 (the ``rows`` object):
-  * the fused-prologue length sweep at T=8192 (B=1, H=96);
+  * the prefill workload (B=1, T=4096, H=16), 20 timed calls with its own clock record;
+  * the sweep at T=8192 and T=32768;
   * the output epilogue, the backward, the Kimi Linear softplus gate and the split of
     one sequence into four segments, all on the prefill shape;
   * the decode step and the decode step with its prologue (N=256, H=96);
   * the Complex-KDA workload (B=8, T=8192, H=32) next to unsigned KDA of the same shape.
 ``e2e`` is the same metric through the C ABI with host buffers, copies timed.
-``cpu_baseline`` times the FP64 oracle on the host cores.
+``cpu_baseline`` times the FP64 oracle on the host cores on a bounded sample.
 """
 from __future__ import annotations
 
@@ -152,36 +155,65 @@ def max_over_ranks(x, ws):
     return float(t.item())
 
 
+# ---------------------------------------------------------------- the headline workload
+HEADLINE_T = W.SWEEP_T[-1]          # T = 65536, the largest length-sweep config
+SWEEP_H, SWEEP_D = W.SWEEP["H"], W.SWEEP["dk"]
+HEADLINE_WORKLOAD = (f"length sweep with the fused prologue, B=1 T={HEADLINE_T} H={SWEEP_H} dk=dv={SWEEP_D}: "
+                     "kda_chunk_fwd_prologue (short conv k=4 + SiLU, bounded gate, beta, chunk_kda fwd)")
+
+
+def sweep_alg_bytes(T, H=SWEEP_H, d=SWEEP_D):
+    """Algorithmic bytes of kda_chunk_fwd_prologue on the sweep workload: per token-head raw
+    q, k, v, z and out in bf16 and the FP32 beta logit; per head S0 and S_T (FP32) and the
+    conv taps of q, k, v (bf16)."""
+    return T * H * (4 * d * 2 + 4 + d * 2) + H * (2 * d * d * 4 + 3 * d * 4 * 2)
+
+
+def oracle_sweep_sample(heads, tokens, seed):
+    """A bounded sample of the sweep workload for the FP64 oracle: `heads` heads x `tokens`
+    tokens drawn with the sweep recipe (same distributions and shapes per head; the oracle's
+    time does not depend on the values)."""
+    import numpy as np
+    x = W.prologue_inputs(1, tokens, heads, SWEEP_D, SWEEP_D, dtype=torch.bfloat16,
+                          S0_std=W.SWEEP["S0_std"], seed=seed)
+    return {n: (None if x[n] is None else x[n].double().numpy()) for n in x}
+
+
+def run_oracle_sample(smp, threads):
+    import oracle
+    q, k, v, g, beta = oracle.prologue_np(smp["q_pre"], smp["k_pre"], smp["v_pre"], smp["conv_w"],
+                                          smp["z"], smp["A"], smp["b_logit"])
+    return oracle.recurrence_c(q, k, v, g, beta, smp["S0"], nthreads=threads)
+
+
 # ---------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args, ws, rank):
     if rank != 0:
         return 0
-    import numpy as np
-    import oracle
-    cfg = W.WORKLOADS["prefill"]
-    x = W.workload_inputs("prefill")
-    heads = 2       # a bounded sample of the workload per step
-    sel = {n: x[n][:, :, :heads].double().numpy() for n in ("q", "k", "v", "g", "beta")}
-    S0 = x["S0"][:, :heads].double().numpy()
-    threads = os.cpu_count() or 1
+    heads, tokens = 16, 4096          # a bounded sample of the workload per step
+    smp = oracle_sweep_sample(heads, tokens, HEADLINE_T)
+    host_cores = os.cpu_count() or 1
+    threads = min(host_cores, heads)  # the oracle threads over sequences (heads)
     times = []
     for i in range(args.warmup + args.steps):
         t0 = time.perf_counter()
-        oracle.recurrence_c(sel["q"], sel["k"], sel["v"], sel["g"], sel["beta"], S0, nthreads=threads)
+        run_oracle_sample(smp, threads)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     # the sample is `heads` of the workload's H heads: that many tokens of the whole workload
-    tok = cfg["B"] * cfg["T"] * heads / cfg["H"]
+    tok = tokens * heads / SWEEP_H
     value = tok / statistics.mean(times)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "prefill B=1 T=4096 H=16 dk=dv=128 (oracle sample: 2 heads)",
-                       "B": 1, "T": 4096, "H": 16, "dk": 128, "dv": 128},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, heads), "kind": "oracle",
-                             "sample": f"{heads} of 16 heads x 4096 tokens of the prefill workload per step "
-                                       "(counted as the 512 tokens of the whole workload they are)"},
+            "config": {"workload": HEADLINE_WORKLOAD + f" (oracle sample: {heads} heads x {tokens} tokens)",
+                       "B": 1, "T": HEADLINE_T, "H": SWEEP_H, "dk": SWEEP_D, "dv": SWEEP_D},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "host_cores": host_cores,
+                             "kind": "oracle",
+                             "sample": f"{heads} of {SWEEP_H} heads x {tokens} tokens of the sweep recipe per "
+                                       f"step, prologue and recurrence in FP64 (counted as the {tok:.0f} tokens "
+                                       "of the whole workload they are)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -203,25 +235,26 @@ def time_calls(fn, reps, flush=None, stream=None):
     return [a.elapsed_time(b) for a, b in out]
 
 
-def cpu_baseline_prefill(min_seconds=10.0, max_runs=40):
-    """The FP64 oracle on the prefill workload, on the host's cores (one thread per head):
-    the whole workload run repeatedly until about `min_seconds` of CPU work (at most
-    `max_runs` runs), rate = tokens of all runs / their time."""
-    import oracle
-    x = W.workload_inputs("prefill")
-    threads = os.cpu_count() or 1
-    arr = {n: x[n].double().numpy() for n in ("q", "k", "v", "g", "beta")}
-    S0 = x["S0"].double().numpy()
-    T = arr["q"].shape[1]
+def cpu_baseline_sweep(min_seconds=10.0, max_runs=40):
+    """The FP64 oracle (prologue in numpy, recurrence in C threaded over heads) on the host's
+    cores, on a bounded sample of the headline workload: 16 heads x 8192 tokens of the sweep
+    recipe, run repeatedly until about `min_seconds` of CPU work (at most `max_runs` runs);
+    rate = the workload tokens the sample stands for / the time."""
+    heads, tokens = 16, 8192
+    smp = oracle_sweep_sample(heads, tokens, HEADLINE_T)
+    host_cores = os.cpu_count() or 1
+    threads = min(host_cores, heads)
     runs, dt = 0, 0.0
     while runs < max_runs and (runs == 0 or dt < min_seconds):
         t0 = time.perf_counter()
-        oracle.recurrence_c(arr["q"], arr["k"], arr["v"], arr["g"], arr["beta"], S0, nthreads=threads)
+        run_oracle_sample(smp, threads)
         dt += time.perf_counter() - t0
         runs += 1
-    return {"value": runs * T / dt, "unit": UNIT, "cores": min(threads, 16), "kind": "oracle",
-            "sample": f"the whole prefill workload (16 heads x 4096 tokens), FP64 C, one thread per "
-                      f"head, run {runs} times",
+    tok = tokens * heads / SWEEP_H
+    return {"value": runs * tok / dt, "unit": UNIT, "cores": threads, "host_cores": host_cores, "kind": "oracle",
+            "sample": f"{heads} of {SWEEP_H} heads x {tokens} tokens of the sweep recipe (prologue + recurrence, "
+                      f"FP64, one thread per head), run {runs} times; counted as the {tok:.0f} tokens of "
+                      "the whole workload each run stands for",
             "seconds": dt, "runs": runs}
 
 
@@ -257,8 +290,6 @@ def rows_n1(K, flush, hbm_peak, rows):
     finish (a row that fails leaves the earlier ones in place)."""
     W.set_device("cuda")
     try:
-        # a1-a4: fused prologue + chunk forward, length sweep at T = 8192
-        rows["sweep_T8192_prologue"] = sweep_row(K, 8192, flush, hbm_peak)
         d = 128
 
         # a2-a4 + the output epilogue (RMSNorm * sigmoid gate) on the prefill workload
@@ -450,117 +481,160 @@ def rows_n1(K, flush, hbm_peak, rows):
     return rows
 
 
-def run_ours(args, ws, rank, local):
-    import gated_delta_rule_73_b200 as K
-    dev = torch.device("cuda", local)
-    hbm_peak, tf_peak, peak_kind = peaks()
-    cfg = W.WORKLOADS["prefill"]
-    B, T, H, dk, dv = cfg["B"], cfg["T"], cfg["H"], cfg["dk"], cfg["dv"]
-    x = W.chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, S0_std=cfg["S0_std"], seed=rank)
-    names = ("q", "k", "v", "g", "beta", "S0")
-    host = {n: x[n].pin_memory() for n in names}
-    d = {n: x[n].to(dev) for n in names}
-    out = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
-    S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
-    opts0 = K.make_opts(torch.bfloat16)
-    wsz = K.kda_chunk_workspace_bytes(B, T, H, dk, dv, opts0)
-    wsb = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    max_launch = 4
-    # per-step event arrays: events[i] before launch i, events[L] after the last
-    evsets = [[torch.cuda.Event(enable_timing=True) for _ in range(max_launch + 1)]
-              for _ in range(args.steps)]
-    for evs in evsets:
-        for e in evs:
-            e.record()
+def time_steps(call, steps, sampler=None):
+    """`steps` calls, one event pair around each on the current stream; returns the per-call
+    device times (ms) and the wall time of the timed region."""
+    t0s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    t1s = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     torch.cuda.synchronize()
-
-    def call(evs=None):
-        o = K.make_opts(torch.bfloat16, workspace=wsb, events=evs)
-        K.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], out, S_T, o)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        call()
-    torch.cuda.synchronize()
-    # launches per call: count events written (those whose timestamps advance)
-    probe = [torch.cuda.Event(enable_timing=True) for _ in range(max_launch + 1)]
-    for e in probe:
-        e.record()
-    torch.cuda.synchronize()
-    t_mark = torch.cuda.Event(enable_timing=True)
-    t_mark.record()
-    call(probe)
-    torch.cuda.synchronize()
-    launches = sum(1 for e in probe[1:] if t_mark.elapsed_time(e) > 0.0)
-
-    # timed steps: one event pair around each call (the call as a user makes it; events between
-    # its launches would hold back the programmatic overlap of the scan with the prep)
-    sampler = ClockSampler(local)
-    t0s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    t1s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(ws)
-    torch.cuda.synchronize()
-    with sampler:
+    ctx = sampler if sampler is not None else _NullCtx()
+    with ctx:
         w0 = time.perf_counter()
-        for i in range(args.steps):
-            flush.zero_()
+        for i in range(steps):
             t0s[i].record()
             call()
             t1s[i].record()
         torch.cuda.synchronize()
         w1 = time.perf_counter()
-    barrier(ws)
-    step_ms = [a.elapsed_time(b) for a, b in zip(t0s, t1s)]
-    # per-kernel durations from a second pass with an event before each launch
-    for i in range(args.steps):
-        flush.zero_()
-        call(evsets[i])
+    return [a.elapsed_time(b) for a, b in zip(t0s, t1s)], w1 - w0
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def kernel_times(call, steps, max_launch=4):
+    """Launches per call and each launch's mean device time (ms), from calls that record an
+    event before every launch (kda_opts.events)."""
+    probe = [torch.cuda.Event(enable_timing=True) for _ in range(max_launch + 1)]
+    for e in probe:
+        e.record()
     torch.cuda.synchronize()
-    kern_ms = [[evs[j].elapsed_time(evs[j + 1]) for evs in evsets] for j in range(launches)]
+    mark = torch.cuda.Event(enable_timing=True)
+    mark.record()
+    call(probe)
+    torch.cuda.synchronize()
+    launches = sum(1 for e in probe[1:] if mark.elapsed_time(e) > 0.0)
+    sets = [[torch.cuda.Event(enable_timing=True) for _ in range(max_launch + 1)] for _ in range(steps)]
+    for evs in sets:
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+    for evs in sets:
+        call(evs)
+    torch.cuda.synchronize()
+    return launches, [statistics.mean(evs[j].elapsed_time(evs[j + 1]) for evs in sets) for j in range(launches)]
+
+
+def prefill_row(K, flush, hbm_peak, steps=20):
+    """The prefill workload (B=1, T=4096, H=16): `steps` timed calls (L2 flushed between them,
+    its inputs fit in L2) with their own clock record and per-launch times."""
+    cfg = W.WORKLOADS["prefill"]
+    B, T, H, d = cfg["B"], cfg["T"], cfg["H"], cfg["dk"]
+    x = W.workload_inputs("prefill")
+    o0 = K.make_opts(torch.bfloat16)
+    wsb = torch.empty(max(K.kda_chunk_workspace_bytes(B, T, H, d, d, o0), 16), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, T, H, d), dtype=torch.bfloat16, device="cuda")
+    S_T = torch.empty((B, H, d, d), dtype=torch.float32, device="cuda")
+
+    def call(evs=None):
+        o = K.make_opts(torch.bfloat16, workspace=wsb, events=evs)
+        K.kda_chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], out, S_T, o)
+    for _ in range(3):
+        call()
+    sampler = ClockSampler(torch.cuda.current_device())
+    ms = []
+    with sampler:
+        for _ in range(steps):
+            ms += time_calls(call, 1, flush)
+    launches, kms = kernel_times(lambda evs: (flush.zero_(), call(evs)), 5)
+    nbytes = B * T * H * token_head_bytes(d) + B * H * 2 * d * d * 4
+    med = statistics.median(ms)
+    return {"ms": med, "ms_mean": statistics.mean(ms), "tokens_per_s": B * T / (med * 1e-3),
+            "frac_of_hbm_roofline": (nbytes / (med * 1e-3) / 1e9) / hbm_peak, "roofline_bytes": nbytes,
+            "launches": launches, "kernel_ms": kms, "clocks": sampler.summary(), "steps": steps,
+            "note": "kda_chunk_fwd B=1 T=4096 H=16 d=128 bf16; 256 MiB written between calls (inputs fit in L2)"}
+
+
+def run_ours(args, ws, rank, local):
+    import gated_delta_rule_73_b200 as K
+    dev = torch.device("cuda", local)
+    hbm_peak, tf_peak, peak_kind = peaks()
+    T, H, d = HEADLINE_T, SWEEP_H, SWEEP_D
+    W.set_device("cuda")
+    x = W.sweep_inputs(T, seed=T + rank)       # each rank its own batch
+    W.set_device("cpu")
+    names = ("q_pre", "k_pre", "v_pre", "conv_w", "z", "A", "b_logit", "S0")
+    opts0 = K.make_opts(torch.bfloat16)
+    wsz = K.kda_prologue_workspace_bytes(1, T, H, d, d, opts0)
+    wsb = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
+    out = torch.empty((1, T, H, d), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((1, H, d, d), dtype=torch.float32, device=dev)
+
+    def call_on(dd, oo, evs=None):
+        o = K.make_opts(torch.bfloat16, workspace=wsb, events=evs)
+        K.kda_chunk_fwd_prologue(*(dd[n] for n in names[:-1]), dd["S0"], oo[0], oo[1], o)
+
+    def call(evs=None):
+        call_on(x, (out, S_T), evs)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    # timed steps: one event pair around each call (the call as a user makes it; the inputs,
+    # 8 GB, are far larger than L2, so nothing is flushed between steps)
+    sampler = ClockSampler(local)
+    barrier(ws)
+    step_ms, wall = time_steps(call, args.steps, sampler)
+    barrier(ws)
+    # per-kernel durations from a second pass with an event before each launch
+    launches, mean_k = kernel_times(call, args.steps)
     total_ms = sum(step_ms)
     total_ms_max = max_over_ranks(total_ms, ws)
     ms_per_step = total_ms_max / args.steps
-    tokens_per_step = B * T
+    tokens_per_step = T
     value = ws * tokens_per_step * args.steps / (total_ms_max * 1e-3)
 
-    # roofline of the step's kernels (the chunk path's algorithmic bytes)
-    alg_bytes = B * T * H * token_head_bytes(dk) + B * H * 2 * dk * dv * 4
-    alg_flops = PREFILL_FLOP_PER_TOKEN_HEAD * B * T * H
-    mean_k = [statistics.mean(km) for km in kern_ms]
+    # roofline of the dominant kernel: the path's algorithmic bytes (every launch of the split
+    # form processes every token-head of the call) over its mean duration
+    alg_bytes = sweep_alg_bytes(T)
+    alg_flops = PREFILL_FLOP_PER_TOKEN_HEAD * T * H
     dom = max(range(launches), key=lambda j: mean_k[j])
-    # Each launch of the split path processes every token-head of the call, so the dominant
-    # kernel's algorithmic bytes per launch are the call's; the whole call is reported beside.
     achieved = alg_bytes / (mean_k[dom] * 1e-3) / 1e9
     call_achieved = alg_bytes / (statistics.mean(step_ms) * 1e-3) / 1e9
-    kernel_names = PREFILL_KERNELS.get(launches, [None] * launches)
+    kernel_names = SWEEP_KERNELS.get(launches, [None] * launches)
+    items = ((T + 63) // 64) * H
+    per_item = KERNEL_TRAFFIC_PER_ITEM.get(kernel_names[dom])
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": KERNEL_TRAFFIC.get(kernel_names[dom]),
+                "frac": achieved / hbm_peak, "traffic": None if per_item is None else per_item * items,
                 "peak_kind": peak_kind, "kernel": kernel_names[dom],
                 "algorithmic_bytes_per_step": alg_bytes, "algorithmic_flops_per_step": alg_flops,
                 "tensor_frac_of_bf16_peak": alg_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / tf_peak,
-                "kernel_ms": mean_k, "dominant_launch": dom,
+                "kernel_ms": mean_k, "kernel_names": kernel_names, "dominant_launch": dom,
                 "whole_call_achieved": call_achieved, "whole_call_frac": call_achieved / hbm_peak,
-                "note": "achieved = algorithmic bytes per launch / the dominant kernel's mean "
-                        "duration (a second pass, an event before each launch); "
-                        "whole_call_* = the same bytes / the call's device time; "
-                        "traffic = DRAM bytes of that kernel per launch (ncu)"}
+                "note": "achieved = algorithmic bytes per launch (the whole call's: each launch covers every "
+                        "token-head) / the dominant kernel's mean duration (a second pass, an event before "
+                        "each launch); whole_call_* = the same bytes / the call's device time; traffic = that "
+                        "kernel's DRAM bytes per (chunk, head) item from an ncu capture at T=2048, times the "
+                        "items of one launch"}
 
     # end to end through the C ABI with host buffers (pinned), copies inside the timed region.
-    # Every step copies its inputs host -> device, runs the call and reads out and S_T back.
+    # Every step copies all its inputs host -> device, runs the call and reads out and S_T back.
     # Pipelined as a serving loop would run it: the copy-in of step i+1, the call of step i and
-    # the copy-out of step i-1 overlap on three streams, with device inputs and outputs
-    # double-buffered.  The serialised form (copy, call, copy on one stream) is kept beside it.
+    # the copy-out of step i-1 overlap on three streams, device buffers double-buffered.  The
+    # serialised form (copy, call, copy on one stream) is kept beside it.
+    host = {n: x[n].cpu().pin_memory() for n in names}
     cs = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    dbuf = [d, {n: torch.empty_like(d[n]) for n in names}]
+    dbuf = [x, {n: torch.empty_like(x[n]) for n in names}]
     obuf = [(out, S_T), (torch.empty_like(out), torch.empty_like(S_T))]
     hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     hS = [torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() for _ in range(2)]
-
-    def call_on(dd, oo):
-        o = K.make_opts(torch.bfloat16, workspace=wsb)
-        K.kda_chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], oo[0], oo[1], o)
+    e2e_steps = min(args.steps, 10)
 
     def e2e_pipelined(nsteps):
         ev_in = [torch.cuda.Event() for _ in range(nsteps)]
@@ -597,75 +671,86 @@ def run_ours(args, ws, rank, local):
 
     def e2e_step():
         for n in names:
-            d[n].copy_(host[n], non_blocking=True)
+            x[n].copy_(host[n], non_blocking=True)
         call()
         hout[0].copy_(out, non_blocking=True)
         hS[0].copy_(S_T, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize()
     ref_out, ref_S = hout[0].clone(), hS[0].clone()
-    e2e_serial_ms = time_calls(e2e_step, args.steps, flush)
+    e2e_serial_ms = time_calls(e2e_step, e2e_steps)
     e2e_pipelined(3)
-    e2e_ms = e2e_pipelined(args.steps)
-    last = (args.steps - 1) % 2
+    e2e_ms = e2e_pipelined(e2e_steps)
+    last = (e2e_steps - 1) % 2
     close = lambda a, b: float((a.float() - b.float()).abs().max()) <= 1e-3 * float(b.float().abs().max())
     e2e_ok = bool(close(hout[last], ref_out) and close(hS[last], ref_S))
     e2e_max = max_over_ranks(e2e_ms, ws)
     e2e_serial_max = max_over_ranks(sum(e2e_serial_ms), ws)
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
     d2h = hout[0].numel() * hout[0].element_size() + hS[0].numel() * hS[0].element_size()
-    e2e = {"value": ws * tokens_per_step * args.steps / (e2e_max * 1e-3), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": e2e_max / args.steps, "outputs_match_serial": e2e_ok,
-           "serial_value": ws * tokens_per_step * args.steps / (e2e_serial_max * 1e-3),
-           "note": "pipelined over three streams (copy-in of step i+1, call i, copy-out of "
-                   "step i-1), every step's copies inside the timed region; serial_value = one "
-                   "stream, L2 flushed between steps"}
+    e2e = {"value": ws * tokens_per_step * e2e_steps / (e2e_max * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "ms_per_step": e2e_max / e2e_steps, "outputs_match_serial": e2e_ok,
+           "serial_value": ws * tokens_per_step * e2e_steps / (e2e_serial_max * 1e-3),
+           "note": "pipelined over three streams (copy-in of step i+1, call i, copy-out of step i-1), every "
+                   "step's copies inside the timed region; serial_value = one stream; PCIe-bound"}
+    del host, dbuf, obuf, hout, hS
+    torch.cuda.empty_cache()
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "prefill (chunk_kda fwd) B=1 T=4096 H=16 dk=dv=128 bf16, FP32 state",
-                       "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
-                       "l2": "256 MiB buffer written between timed steps",
+            "config": {"workload": HEADLINE_WORKLOAD, "B": 1, "T": T, "H": H, "dk": d, "dv": d,
+                       "l2": "inputs (8 GB) larger than the 126 MB L2; nothing flushed between steps",
                        "parallelism": f"replicas x{ws}: each rank runs its own batch, no collective"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches * args.steps,
             "step_ms_median": statistics.median(step_ms),
-            "clocks": sampler.summary(), "wall_s_timed": w1 - w0}
+            "clocks": sampler.summary(), "wall_s_timed": wall}
+    del x, wsb, out, S_T
+    torch.cuda.empty_cache()
     if ws == 1 and rank == 0 and not args.no_rows:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         rows = {}
         try:
-            rows_n1(K, flush, hbm_peak, rows)
+            W.set_device("cuda")
+            rows["prefill_B1_T4096_H16"] = prefill_row(K, flush, hbm_peak)
         except Exception as e:          # a failed row must not cost the headline its line
+            rows["prefill_B1_T4096_H16"] = {"error": f"{type(e).__name__}: {e}"}
+        finally:
+            W.set_device("cpu")
+        try:
+            rows_n1(K, flush, hbm_peak, rows)
+        except Exception as e:
             rows["error"] = f"{type(e).__name__}: {e}"
-        for T in W.SWEEP_T[2:]:           # the longer sweep lengths, memory permitting
+        for Ts in W.SWEEP_T[1:-1]:         # T = 8192, 32768 (65536 is the headline)
             try:
-                rows[f"sweep_T{T}_prologue"] = sweep_row(K, T, flush, hbm_peak)
+                rows[f"sweep_T{Ts}_prologue"] = sweep_row(K, Ts, flush, hbm_peak)
             except Exception as e:
-                rows[f"sweep_T{T}_prologue"] = {"error": f"{type(e).__name__}: {e}"}
+                rows[f"sweep_T{Ts}_prologue"] = {"error": f"{type(e).__name__}: {e}"}
         line["rows"] = rows
+        del flush
     if ws == 1 and rank == 0 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline_prefill()
+        line["cpu_baseline"] = cpu_baseline_sweep()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
 
 
-CASES = ("prefill", "decode", "sweep", "ckda", "bwd")
+CASES = ("prefill", "decode", "sweep", "ckda", "bwd", "sweep_plain")
 
-# Kernels of kda_chunk_fwd on the prefill workload by launches per call: the one-launch form
-# (prep and scan CTAs side by side) that few-head calls take, or the split form's two kernels;
-# and the DRAM bytes (read + write) of one launch of each from one ncu capture (profiles/),
-# None where no capture of the kernel as it stands exists.  Re-capture when a kernel changes.
-PREFILL_KERNELS = {1: ["chunk_mega_kernel"], 2: ["chunk_prep_kernel", "chunk_scan_tc_kernel"]}
-KERNEL_TRAFFIC = {"chunk_mega_kernel": 112_274_176, "chunk_prep_kernel": None, "chunk_scan_tc_kernel": None}
+# Kernels of kda_chunk_fwd_prologue on the sweep workload (B*H = 96 takes the split form: the
+# two-group prep with the fused prologue, then the scan) by launches per call, and the DRAM
+# bytes (read + write) per (chunk, head) item of each from one ncu capture at T = 2048
+# (profiles/), None where no capture of the kernel as it stands exists.
+SWEEP_KERNELS = {2: ["chunk_prep2_kernel", "chunk_scan_tc_kernel"], 1: ["chunk_mega2_kernel"]}
+KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": 122_745, "chunk_scan_tc_kernel": 86_995, "chunk_mega2_kernel": None}
 
 
 def run_case(args):
     """Run one workload's call a few times and exit (a small case for ncu captures):
     prefill = B=1 T=4096 H=16; decode = N=64 H=96 (800 MB of state);
-    sweep = prologue path at T=2048 H=96; ckda = B=2 T=8192 H=32 signed gate;
-    bwd = kda_chunk_bwd at B=1 T=1024 H=16."""
+    sweep = prologue path at T=2048 H=96; sweep_plain = kda_chunk_fwd at B=1 T=2048 H=96;
+    ckda = B=2 T=8192 H=32 signed gate; bwd = kda_chunk_bwd at B=1 T=1024 H=16."""
     import gated_delta_rule_73_b200 as K
     torch.cuda.set_device(0)
     W.set_device("cuda")
@@ -687,6 +772,9 @@ def run_case(args):
         x = W.sweep_inputs(T)
         a = [x[n] for n in ("q_pre", "k_pre", "v_pre", "conv_w", "z", "A", "b_logit")]
         fn = lambda: K.chunk_fwd_prologue(*a, x["S0"])
+    elif args.case == "sweep_plain":
+        x = W.chunk_inputs(1, 2048, 96, d, d, dtype=torch.bfloat16, seed=0)
+        fn = lambda: K.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], fused=False)
     else:
         if args.case == "prefill":
             x = W.workload_inputs("prefill")
@@ -708,7 +796,7 @@ def main():
                     help="run one small workload a few times (for profiler captures) and exit")
     ap.add_argument("--case-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-rows", action="store_true")

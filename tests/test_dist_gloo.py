@@ -66,8 +66,11 @@ def test_reference_arm_under_torchrun_only_rank0_prints():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle"
-    # tokens of the whole workload: a 2-of-16-head sample of 4096 tokens counts as 512 tokens
-    assert abs(d["value"] * d["ms_per_step"] * 1e-3 - 4096 * 2 / 16) < 1e-6 * 512
+    # tokens of the whole workload: a 16-of-96-head sample of 4096 tokens of the sweep counts
+    # as 4096 * 16 / 96 tokens
+    assert abs(d["value"] * d["ms_per_step"] * 1e-3 - 4096 * 16 / 96) < 1e-6 * 4096
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["host_cores"] >= d["cpu_baseline"]["cores"]
+    assert "T=65536" in d["config"]["workload"]
 
 
 def _cp_worker(rank, world, port, q, cuts):
