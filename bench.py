@@ -739,11 +739,11 @@ def run_ours(args, ws, rank, local):
 CASES = ("prefill", "decode", "sweep", "ckda", "bwd", "sweep_plain")
 
 # Kernels of kda_chunk_fwd_prologue on the sweep workload (B*H = 96 takes the split form: the
-# two-group prep with the fused prologue, then the scan) by launches per call, and the DRAM
+# two-group prep with the fused prologue, then the TMEM scan) by launches per call, and the DRAM
 # bytes (read + write) per (chunk, head) item of each from one ncu capture at T = 2048
 # (profiles/), None where no capture of the kernel as it stands exists.
-SWEEP_KERNELS = {2: ["chunk_prep2_kernel", "chunk_scan_tc_kernel"], 1: ["chunk_mega2_kernel"]}
-KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": 122_745, "chunk_scan_tc_kernel": 86_995, "chunk_mega2_kernel": None}
+SWEEP_KERNELS = {2: ["chunk_prep2_kernel", "chunk_scan3_kernel"], 1: ["chunk_mega2_kernel"]}
+KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": 122_882, "chunk_scan3_kernel": 87_121, "chunk_mega2_kernel": None}
 
 
 def run_case(args):

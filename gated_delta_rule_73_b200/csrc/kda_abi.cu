@@ -46,8 +46,10 @@ KernelFlags kflags(const kda_opts &o) {
 //    record per chunk and head).  Cost ~ B*H*nch*t_prep / SMs + waves * nch * t_scan.
 //  * fused: one kernel per sequence, prep and scan step serially in one CTA (no
 //    workspace).  Cost ~ waves * nch * t_fused, waves = ceil(B*H / SMs).
-// Measured on B200 at d = 128 (per chunk and head): t_fused = 14.0 us, t_prep = 14.8 us,
-// t_scan = 2.8 us; the model uses their ratios.  KDA_FUSED / KDA_SPLIT override it.
+// Measured on B200 at d = 128: t_fused = 14.0 us per chunk of a wave of sequences, t_prep =
+// 6.8 us of one SM per (chunk, head) item (the two-group prep), t_scan = 2.4 us per chunk (one
+// CTA per head); the model uses their ratios.  With the two-group prep the split form wins at
+// every B*H; the fused form stays available through KDA_FUSED.  KDA_SPLIT forces the split.
 bool use_tc(const kda_opts &o, int dk, int dv) {
     return o.dtype == KDA_BF16 && dk == 128 && dv == 128 && !unbounded(o);
 }
@@ -63,7 +65,7 @@ bool use_fused(const kda_opts &o, int B, int H) {
     if (o.flags & KDA_SPLIT) return false;
     const double x = (double)B * H / device_sms();
     const double waves = ceil(x);
-    const double t_fused = 1.0, t_prep = 14.8 / 14.0, t_scan = 2.8 / 14.0;
+    const double t_fused = 1.0, t_prep = 6.8 / 14.0, t_scan = 2.4 / 14.0;
     return waves * t_fused < x * t_prep + waves * t_scan;
 }
 size_t tc_ws(const kda_opts &o, int B, int T, int H) {

@@ -52,7 +52,9 @@ constexpr uint32_t TAB_F = 0;          // 13 rows x 512 B
 constexpr uint32_t TAB_NRMP = 6656;    // FP32 sums of squares [2 halves][128 rows: q, then k]
 constexpr uint32_t TAB_BET = 7680;     // FP32 beta [64]
 constexpr uint32_t TAB_BAR = 7936;     // mbarriers and the abort flag
-constexpr uint32_t GROUP_USED = OFF_TAB + TAB_BAR + 64;
+constexpr uint32_t TAB_PX = TAB_BAR + 64;   // Complex-KDA: sign parity of each warp's 32 rows [8]
+constexpr uint32_t GROUP_USED = OFF_TAB + TAB_PX + 32;
+constexpr uint32_t OFF_LO = OFF_KH;    // Complex-KDA: the low bf16 part of log|alpha| (g's layout)
 constexpr uint32_t GROUP_STRIDE = 114688;
 constexpr uint32_t SMEM_BYTES = 1024 + GROUP_STRIDE + GROUP_USED;
 static_assert(GROUP_USED <= GROUP_STRIDE, "group layout");
@@ -178,6 +180,7 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
     float *FT = reinterpret_cast<float *>(gsm + OFF_TAB + TAB_F);
     float *NRMP = reinterpret_cast<float *>(gsm + OFF_TAB + TAB_NRMP);
     float *BET = reinterpret_cast<float *>(gsm + OFF_TAB + TAB_BET);
+    uint32_t *PX = reinterpret_cast<uint32_t *>(gsm + OFF_TAB + TAB_PX);
     float *AKT = reinterpret_cast<float *>(gsm + OFF_AKT);
     float *TMF = reinterpret_cast<float *>(gsm + OFF_TMF);
     GroupBars *gb = reinterpret_cast<GroupBars *>(gsm + OFF_TAB + TAB_BAR);
@@ -324,9 +327,15 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
             // (8-channel group, 16-row segment) for the gate (64 threads).  The three rows before
             // a segment come from the segment above (read before the barrier, so the in-place
             // writes cannot race) or, for the first segment, from global memory (zero before t = 0).
-            if (wait(b_g, ph) && gt == 0) ++con[1];
-            if (wait(b_v, ph) && gt == 0) ++con[2];
+            // q and k (threads 0-127) start as soon as their tiles are in; v and the gate (threads
+            // 128-255) wait for theirs, which were issued last.  Each half has its own barrier
+            // for the in-place hazard (named barriers 3 + 2 gi and 4 + 2 gi, 128 threads).
             if (gbar_or(gi, bad)) break;
+            if (br >= 2) {
+                wait(b_g, ph);
+                wait(b_v, ph);
+            }
+            const int sub_bar = 3 + 2 * gi + (br >= 2 ? 1 : 0);
             // lanes of a quarter-warp take the 8 channel groups of one row: conflict-free
             const int cg = pcg, r0 = 16 * seg;
             const uint32_t ubase = br == 0 ? OFF_X : br == 1 ? OFF_X + 8192 : br == 2 ? OFF_V : OFF_G;
@@ -355,7 +364,7 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                     w[2][m] = make_float2(bq.x, d2.x);
                     w[3][m] = make_float2(bq.y, d2.y);
                 }
-                gbar(gi);
+                asm volatile("bar.sync %0, %1;" ::"r"(sub_bar), "r"(128) : "memory");
                 const bool tail = n < C;
 #pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
@@ -379,7 +388,7 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 }
             } else {
                 const float2 ea = dup2(0.5f * expf(a_h));   // sigmoid(a z) = (1 + tanh(a z / 2)) / 2
-                gbar(gi);
+                asm volatile("bar.sync %0, %1;" ::"r"(sub_bar), "r"(128) : "memory");
                 const bool tail = n < C;
 #pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
@@ -398,18 +407,70 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 }
             }
             fence_proxy_async();   // g and v are read by the tensor cores
-            gbar(gi);
+            if (gt == 0) {   // by now both have landed: count them for the drain
+                if (wait(b_g, ph)) ++con[1];
+                if (wait(b_v, ph)) ++con[2];
+            }
+            if (gbar_or(gi, bad)) break;   // the gate's g is in place before the cumsum reads it
         }
-        // ---- band-local cumsum on the tensor cores: D[0,128) = [L_band; L_band] g
+        // ---- Complex-KDA: g holds the signed gate alpha.  Thread = (row r, channels 32 cq ..):
+        // log|alpha| split into a bf16 high part (in place) and low part (OFF_LO), so the cumsum
+        // below is exact to ~2^-17; the sign bits become this thread's prefix parity word
+        // sigma_r (bit j: channel 32 cq + j) by an XOR scan over the warp's 32 rows, the carry
+        // of rows 0-31 coming through PX after the barrier.  Rows past T count as alpha = 1.
+        uint32_t sig = 0;
+        if (fl.complex_gate) {
+            if (wait(b_g, ph) && gt == 0) ++con[1];
+            const int r = gt & 63, cq = gt >> 6;
+            uint32_t neg = 0;
+            constexpr float kLn2 = 0.6931471805599453f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cg = 4 * cq + m;
+                const uint4 u = ld16(gsm + OFF_G + off_t(r, cg));
+                const uint32_t wa[4] = {u.x, u.y, u.z, u.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 a = bf2(wa[e]);
+                    neg |= (a.x < 0.f ? 1u : 0u) << (8 * m + 2 * e);
+                    neg |= (a.y < 0.f ? 1u : 0u) << (8 * m + 2 * e + 1);
+                    float l0, l1;
+                    asm("lg2.approx.f32 %0, %1;" : "=f"(l0) : "f"(fabsf(a.x)));
+                    asm("lg2.approx.f32 %0, %1;" : "=f"(l1) : "f"(fabsf(a.y)));
+                    const float2 lg = r < n ? mul2(make_float2(l0, l1), dup2(kLn2)) : make_float2(0.f, 0.f);
+                    hi[e] = pk2(lg);
+                    const float2 h2 = bf2(hi[e]);
+                    lo[e] = pk2(make_float2(lg.x - h2.x, lg.y - h2.y));
+                }
+                st16(gsm + OFF_G + off_t(r, cg), hi[0], hi[1], hi[2], hi[3]);
+                st16(gsm + OFF_LO + off_t(r, cg), lo[0], lo[1], lo[2], lo[3]);
+            }
+            if (r >= n) neg = 0u;
+            uint32_t pfx = neg;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, pfx, o);
+                if (lane >= o) pfx ^= y;
+            }
+            if (lane == 31) PX[gw] = pfx;
+            sig = pfx;
+            fence_proxy_async();   // both parts are read by the tensor cores
+            if (gbar_or(gi, bad)) break;
+            if (gw & 1) sig ^= PX[gw - 1];
+        }
+        // ---- band-local cumsum on the tensor cores: D[0,128) = [L_band; L_band] g (Complex-KDA:
+        // the two parts of log|alpha|, K = 128)
         if (gt == 0) {
-            const bool g_ok = PRO || wait(b_g, ph);
-            if (!PRO && g_ok) ++con[1];
+            const bool g_ok = PRO || fl.complex_gate || wait(b_g, ph);
+            if (!PRO && !fl.complex_gate && g_ok) ++con[1];
             tc_fence_after();
             if (g_ok) {
                 constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_ts(gtm + TC_D, gtm + TC_LM + 8 * s, at(dT, OFF_G + 2048 * s), id, s > 0);
+                const int nk = fl.complex_gate ? 8 : 4;
+                for (int s = 0; s < nk; ++s)
+                    mma_ts(gtm + TC_D, gtm + TC_LM + 8 * (s & 3),
+                           at(dT, (s < 4 ? OFF_G : OFF_LO) + 2048 * (s & 3)), id, s > 0);
                 mma_commit(b_m1);
                 ++iss[3];
             }
@@ -457,18 +518,21 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
             FT[(R_ET + 0) * 128 + c] = et[0];
             FT[(R_ET + 1) * 128 + c] = et[1];
             FT[(R_ET + 2) * 128 + c] = et[2];
-            FT[(R_ET + 3) * 128 + c] = et[3];
+            // Complex-KDA: K e^{gamma_C - gamma} carries sigma_C sigma_r (Gamma_C / Gamma_r), and the
+            // state update sigma_C e^{gamma_C}: fold sigma_C into the e^{gamma_C - p_b} rows
+            const float sc = (fl.complex_gate && (((PX[2 * (c >> 5)] ^ PX[2 * (c >> 5) + 1]) >> (c & 31)) & 1u)) ? -1.f : 1.f;
+            FT[(R_ET + 3) * 128 + c] = sc * et[3];   // e_3 is used only as e^{gamma_C - p_3}
             const float e01 = et[0] * et[1], e12 = et[1] * et[2], e23 = et[2] * et[3];
             FT[R_EP2 * 128 + c] = e01;
             FT[R_EP3 * 128 + c] = e01 * et[2];
             const float eC = e01 * e23;
-            FT[(R_ECP + 0) * 128 + c] = eC;
-            FT[(R_ECP + 1) * 128 + c] = et[1] * e23;
-            FT[(R_ECP + 2) * 128 + c] = e23;
+            FT[(R_ECP + 0) * 128 + c] = sc * eC;
+            FT[(R_ECP + 1) * 128 + c] = sc * et[1] * e23;
+            FT[(R_ECP + 2) * 128 + c] = sc * e23;
             FT[R_EM20 * 128 + c] = e01;
             FT[R_EM31 * 128 + c] = e12;
             FT[R_EM30 * 128 + c] = e01 * et[2];
-            reinterpret_cast<float *>(img + IMG_GC)[c] = eC;
+            reinterpret_cast<float *>(img + IMG_GC)[c] = sc * eC;
         }
         gbar(gi);
 
@@ -486,7 +550,16 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 const int cg = 4 * cq + m, c0 = 8 * cg;
                 const uint4 uq = ld16(gsm + OFF_X + off_x(0, r, cg));
                 const uint4 uk = ld16(gsm + OFF_X + off_x(1, r, cg));
-                const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
+                uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
+                if (fl.complex_gate) {   // sigma_r: flip the signs of q and k channel by channel
+                    const uint32_t sb = sig >> (8 * m);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t mk = (((sb >> (2 * e)) & 1u) << 15) | (((sb >> (2 * e + 1)) & 1u) << 31);
+                        wq[e] ^= mk;
+                        wk[e] ^= mk;
+                    }
+                }
                 float2 fp[4], fc[4];
                 ld4f2(ep + c0, fp);
                 ld4f2(ecp + c0, fc);
@@ -749,7 +822,8 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 for (int g8 = 0; g8 < 4; ++g8) {
                     const int c0 = 64 * hh + 32 * hc + 8 * g8;
                     const float *x = w + 8 * g8;
-                    st16(img + (qd < 2 ? IMG_W + off_r128(r, c0) : IMG_U + off_u(r, c0)), pk2(make_float2(x[0], x[1])),
+                    const uint32_t uoff = pro.u_slabs ? off_u(r, c0) : off_r128(r, c0);
+                    st16(img + (qd < 2 ? IMG_W + off_r128(r, c0) : IMG_U + uoff), pk2(make_float2(x[0], x[1])),
                          pk2(make_float2(x[2], x[3])), pk2(make_float2(x[4], x[5])), pk2(make_float2(x[6], x[7])));
                 }
             }

@@ -1,34 +1,25 @@
-// kda_chunk_tc2.cu -- two-kernel tensor-core chunkwise KDA forward for sm_100a.
+// kda_chunk_tc2.cu -- the split tensor-core chunkwise KDA forward for sm_100a.
 //
 // The chunkwise form (page "Kimi K3 模型结构（2）：序列维度（下），chunkwise 并行与
 // 下界衰减", Q&A items on the chunkwise algorithm, the -5 decay floor and the
 // intra-chunk matrix A) splits into work that does not depend on the state --
-// everything up to the WY vectors -- and a short state-dependent scan.  The
-// first kernel runs the former for every (chunk, head) in parallel, so it fills
-// the GPU however few heads there are; the second walks each head's chunks in
-// order with nothing but the scan on its critical path.
+// everything up to the WY vectors -- and a short state-dependent scan.
 //
-// Kernel 1 (one CTA per chunk and head), with the same arithmetic as the fused
-// kernel of kda_chunk_tc.cu:
-//   gamma = band-local cumsum of log|alpha|, E = e^{gamma - p_band}, band factors
-//   A_qk / A_kk: all ten (row band, column band) pairs as one N = 160 tcgen05 product
-//   Tm = (I + A_kk)^{-1} in FP32;  W = Tm' (K e^gamma),  U = Tm' V
-//   writes, per chunk and head, a 74,240-byte record of bf16 tiles already in the
-//   shared-memory layouts the scan's tensor-core products read:
-//     W and Q e^gamma (K-major [r][c], stacked into one [128][128] tile),
-//     K e^{gamma_C-gamma} ([r][c]), U (16-column slabs of [r][j]), A_qk (K-major [r][i])
-//     and sigma_C e^{gamma_C} (FP32 [128]).
-// Kernel 2 (one CTA per head): per chunk, the record is bulk-copied into one of two
-// stages, then
-//   [P ; O] = [W ; Q e^gamma] S                          (S in shared memory as bf16)
-//   V~ = U - P;  dS = Kd^T V~;  O += A_qk V~             (V~ in shared memory as bf16)
-//   S <- diag(sigma_C e^{gamma_C}) S + dS in FP32 registers;  O -> HBM while the
-//   next chunk's first product runs.
+//   prep (kda_chunk_prep.cuh): every (chunk, head) item in parallel, two items in flight per SM;
+//        writes one 74,240-byte record per item: W and Q e^gamma (one [128][128] K-major tile),
+//        K e^{gamma_C - gamma}, U, A_qk (K-major [r][i]) and sigma_C e^{gamma_C} (FP32 [128]),
+//        bf16 tiles already in the layouts the scan's tensor-core products read
+//   scan, TMEM form (kda_chunk_scan.cuh): one CTA per sequence, the state and the chunk's
+//        products in TMEM; the second launch when the sequences fill the SMs
+//   scan, sliced form (below): one CTA per (sequence, value-column slice), the state in
+//        registers and shared memory; beside the prep in one cooperative launch when the
+//        sequences are few, and with whole-row slices when the output epilogue is fused:
+//          [P ; O] = [W ; Q e^gamma] S;  V~ = U - P;  dS = Kd^T V~;  O += A_qk V~
+//          S <- diag(sigma_C e^{gamma_C}) S + dS in FP32 registers
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <stdlib.h>
 
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -68,13 +59,6 @@ __device__ __forceinline__ uint32_t off_rn(int r, int c, int n) {
 __device__ __forceinline__ uint32_t off_u(int r, int j) {
     return (uint32_t)((j >> 4) * 2048) + off_rn(r, j & 15, 16);
 }
-// staging tile of 64 (or, with the halo of the fused prologue, 67) token rows x 128 channels
-// as two 64-channel halves of 128-byte-swizzled rows, the halves 9 KB apart
-constexpr uint32_t kHalf = 9216;
-__device__ __forceinline__ uint32_t off_sw128(int r, int c) {
-    const int hf = c >> 6, cc = c & 63;
-    return (uint32_t)(hf * kHalf + r * 128 + ((((cc >> 3) ^ (r & 7))) << 4) + (cc & 7) * 2);
-}
 __device__ __forceinline__ int pair_of(int b, int j) { return (j == 0 ? 0 : j == 1 ? 4 : j == 2 ? 7 : 9) + b - j; }
 
 __device__ __forceinline__ void unpack8(uint4 raw, float (&x)[8]) {
@@ -94,56 +78,9 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
     u.w = pack_bf16(x[6], x[7]);
     return u;
 }
-__device__ __forceinline__ uint2 pack4(const float (&x)[4]) {
-    return make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
-}
-__device__ __forceinline__ void ld8f(const float *p, float (&x)[8]) {
-    *reinterpret_cast<float4 *>(x) = *reinterpret_cast<const float4 *>(p);
-    *reinterpret_cast<float4 *>(x + 4) = *reinterpret_cast<const float4 *>(p + 4);
-}
 
 __device__ int g_kda_tc2_error;   // set when a bounded wait gives up
 
-struct alignas(8) Bars {
-    uint64_t bar0;
-    uint64_t bar1;
-    uint64_t bar_mma;
-    uint32_t tmem_base;
-    int abort;
-};
-
-// ============================================================== kernel 1: per-chunk prep
-namespace prep {
-constexpr int NT = 512;
-constexpr uint32_t kTile = 2 * kHalf;         // one staged tensor
-constexpr uint32_t OFF_STG_Q = 0, OFF_STG_K = kTile, OFF_STG_V = 2 * kTile, OFF_STG_G = 3 * kTile;
-constexpr int kHalo = 3;                       // rows before the chunk the short convolution reads
-constexpr uint32_t OFF_GAM = 4 * kTile;        // fp32 E [64][132]; later AKK / TMF
-constexpr uint32_t E_STRIDE = 132;
-constexpr uint32_t AS = 68;
-constexpr uint32_t OFF_AKK = OFF_GAM;
-constexpr uint32_t OFF_TMF = OFF_GAM + 17408;
-constexpr uint32_t OFF_BOP = OFF_GAM + 36864;  // bf16 band-pair B operand [160][128]; later Tm'
-constexpr uint32_t OFF_TMB = OFF_BOP;          // bf16 [128][64 i]: Tm' rows r, then the same rows again
-constexpr uint32_t OFF_YR = OFF_BOP + 40960;   // bf16 K e^gamma [64][128]
-constexpr uint32_t OFF_TAB = OFF_YR + 16384;
-constexpr uint32_t TAB_TOT = 0, TAB_F = 2048, TAB_G = 10240, TAB_H = 12288, TAB_GC = 14336,
-                   TAB_NRM = 14848, TAB_BET = 15360, TAB_SGNL = 15616, TAB_BPAR = 16640,
-                   TAB_PP = 16896, TAB_SGNC = 17152, TAB_BYTES = 17408;
-// the record leaves through shared memory by bulk stores: Q e^gamma and Kd here, then W and U in
-// the same 32 KB at the item's end (first rewritten by the next item's operands), A_qk in the
-// band-pair operand's region, sigma_C e^{gamma_C} in the tables
-constexpr uint32_t OFF_RQG = OFF_TAB + TAB_BYTES;    // bf16 Q e^gamma, the record's layout
-constexpr uint32_t OFF_RKD = OFF_RQG + 16384;        // bf16 Kd
-constexpr uint32_t OFF_RAQ = OFF_BOP + 16384;        // bf16 A_qk (after Tm')
-constexpr uint32_t OFF_RWU = OFF_RQG;                // bf16 W, then U (16-column slabs)
-constexpr uint32_t OFF_CW = OFF_RKD + 16384;        // bf16 conv taps of q, k, v [3][128 c][4] (prologue)
-constexpr uint32_t SMEM_BYTES = OFF_CW + 3072 + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-// TMEM: X [0,64), D [64,224), then W and U, each in lanes 0-63 with lanes 64-127 repeating
-// them: U [224,352), W [352,480)
-constexpr uint32_t TC_X = 0, TC_D = 64, TC_U = 224, TC_W = 352;
-}  // namespace prep
 
 // Inputs of the prologue fused into the prep kernel (kda_chunk_fwd_prologue on the split
 // form).  conv_w == nullptr: the tiles are q, k, v, g and beta is given.
@@ -153,673 +90,11 @@ struct PrepPrologue {
     const float *b_logit;          // [B, T, H] beta logits (FP32)
     // the raw branch inputs (the rows before a chunk, for its first convolution outputs)
     const __nv_bfloat16 *raw_q, *raw_k, *raw_v;
+    // U in the record as 16-column slabs (the sliced scan) rather than rows like W (the TMEM scan)
+    int u_slabs;
 };
 
 #include "kda_chunk_prep.cuh"
-
-// The prep's work, run by CTA `cta` of `ncta` prep CTAs.  MEGA (the fused prep + scan launch of
-// few-head calls): items are taken chunk-major, so every head's early chunks come first, and
-// each finished record is published by a release of flags[item] once its bulk stores are
-// complete.  Otherwise items are taken chunk-fastest and the scan runs as the next kernel.
-template <bool PRO, bool MEGA>
-__device__ __forceinline__ void
-prep_body(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap *ptm_v,
-          const CUtensorMap *ptm_g, const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T,
-          int H, int BH, KernelFlags fl, PrepPrologue pro, int cta, int ncta, int *__restrict__ flags) {
-    using namespace prep;
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ Bars sh;
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const uint32_t sbase = smem_u32(smem);
-    float *EX = reinterpret_cast<float *>(smem + OFF_GAM);
-    float *AKK = reinterpret_cast<float *>(smem + OFF_AKK);
-    float *TMF = reinterpret_cast<float *>(smem + OFF_TMF);
-    float *TOT = reinterpret_cast<float *>(smem + OFF_TAB + TAB_TOT);
-    float *TF = reinterpret_cast<float *>(smem + OFF_TAB + TAB_F);
-    float *TG = reinterpret_cast<float *>(smem + OFF_TAB + TAB_G);
-    float *TH = reinterpret_cast<float *>(smem + OFF_TAB + TAB_H);
-    float *TGC = reinterpret_cast<float *>(smem + OFF_TAB + TAB_GC);
-    float *NRM = reinterpret_cast<float *>(smem + OFF_TAB + TAB_NRM);
-    float *BET = reinterpret_cast<float *>(smem + OFF_TAB + TAB_BET);
-    uint32_t *SGNL = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNL);
-    uint32_t *BPAR = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_BPAR);
-    uint32_t *PP = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_PP);
-    uint32_t *SGNC = reinterpret_cast<uint32_t *>(smem + OFF_TAB + TAB_SGNC);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, qq = warp >> 2;
-    const int row = quad * 32 + lane;
-    const int nch = (T + C - 1) / C;
-    const int nitems = nch * BH;
-    const uint32_t bar_tma = smem_u32(&sh.bar0), bar_v = smem_u32(&sh.bar1), bar_mma = smem_u32(&sh.bar_mma);
-
-    if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_mma, 1);
-        mbar_fence_init();
-        sh.abort = 0;
-    }
-    if (warp == 0) {
-        tmem_alloc(smem_u32(&sh.tmem_base), 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tbase = sh.tmem_base;
-    const uint32_t tl = tbase + ((uint32_t)(quad * 32) << 16);
-    // the scan kernel, launched with a programmatic dependency on this one, may be scheduled
-    // now: its CTAs take SMs as this grid's CTAs leave and wait in-kernel for its completion
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const uint64_t dK64 = sdesc(sbase, 128, 2048, kSwizzleNone);
-    const uint64_t dMN64 = sdesc(sbase, 2048, 128, kSwizzleNone);
-    const uint64_t dK32 = sdesc(sbase, 128, 1024, kSwizzleNone);
-    const uint64_t dV = sdesc(sbase, kHalf, 1024, kSwizzle128B);
-    auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
-    auto wait_all = [&](uint32_t bar, uint32_t phase) -> bool {
-        if (tid == 0 && !mbar_wait_bounded(bar, phase, kWaitLimit)) {
-            sh.abort = 1;
-            g_kda_tc2_error = 1;
-        }
-        __syncthreads();
-        return sh.abort == 0;
-    };
-
-    // work item = (chunk, b * H + h), chunk fastest; each CTA walks items with a stride of the
-    // grid and fetches the next item's tiles as soon as their staging buffers are free
-    // with the fused prologue the maps cover the raw inputs and their boxes are 67 rows high,
-    // starting 3 rows before the chunk (rows before t = 0 read as zeros: no history)
-    constexpr bool fused_pro = PRO;
-    const int rows = fused_pro ? C + kHalo : C, row0 = fused_pro ? -kHalo : 0;
-    const uint32_t tile_bytes = (uint32_t)rows * D * 2u;
-    // item -> (chunk, b * H + h)
-    auto item_ch = [&](int item) { return MEGA ? item / BH : item % nch; };
-    auto item_bh = [&](int item) { return MEGA ? item % BH : item / nch; };
-    auto issue_qkg = [&](int item) {
-        const int ich = item_ch(item), ibh = item_bh(item);
-        const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
-        mbar_arrive_expect_tx(bar_tma, 3u * tile_bytes + (fused_pro ? 3072u : 0u));
-        if (fused_pro) {
-            // the item's conv taps: 1 KB per branch, [c][tap] for the head's 128 channels
-#pragma unroll
-            for (int br = 0; br < 3; ++br)
-                bulk_load(sbase + OFF_CW + 1024 * br, pro.conv_w + ((size_t)br * H * D + (size_t)ih * D) * 4, 1024, bar_tma);
-        }
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(sbase + OFF_STG_Q + hf * kHalf, ptm_q, bar_tma, hf * 64, ih, it0, ib);
-            tma_load_4d(sbase + OFF_STG_K + hf * kHalf, ptm_k, bar_tma, hf * 64, ih, it0, ib);
-            tma_load_4d(sbase + OFF_STG_G + hf * kHalf, ptm_g, bar_tma, hf * 64, ih, it0, ib);
-        }
-    };
-    auto issue_v = [&](int item) {
-        const int ich = item_ch(item), ibh = item_bh(item);
-        const int ib = ibh / H, ih = ibh % H, it0 = ich * C + row0;
-        mbar_arrive_expect_tx(bar_v, tile_bytes);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + OFF_STG_V + hf * kHalf, ptm_v, bar_v, hf * 64, ih, it0, ib);
-    };
-    if (tid == 0 && cta < nitems) {
-        issue_qkg(cta);
-        issue_v(cta);
-    }
-    // beta (with the fused prologue: its logit) of token row tid < C of an item, loaded one
-    // item ahead so its global-memory latency overlaps the current item
-    auto load_beta = [&](int it) -> float {
-        if (tid >= C || it >= nitems) return 0.f;
-        const int ich = item_ch(it), ibh = item_bh(it);
-        const int t = ich * C + tid;
-        if (t >= T) return 0.f;
-        const size_t bth = ((size_t)(ibh / H) * T + t) * H + ibh % H;
-        return fused_pro ? pro.b_logit[bth] : __bfloat162float(beta[bth]);
-    };
-    float bpre = load_beta(cta);
-    bool ok = true;
-    uint32_t li = 0;   // items done by this CTA: parity of the TMA barriers
-    int done = -1;     // the item whose record is published next (MEGA)
-    // MEGA: the previous record's bulk stores are complete; publish it
-    auto publish = [&]() {
-        bulk_wait_all();
-        if (done >= 0) {
-            fence_proxy_async_global();
-            flag_release(flags + done, 1);
-            done = -1;
-        }
-    };
-    for (int item = cta; item < nitems && ok; item += ncta, ++li) {
-        const int ch = item_ch(item), bh = item_bh(item), h = bh % H;
-        const int t0 = ch * C, n = min(C, T - t0);
-        const int next = item + ncta;
-        uint8_t *img = ws + ((size_t)bh * nch + ch) * IMG_BYTES;
-        if (tid < C) {
-            // the fused prologue rounds beta to bf16 like the standalone prologue kernel
-            BET[tid] = tid >= n ? 0.f
-                       : fused_pro ? __bfloat162float(__float2bfloat16_rn(sigmoid_fast(bpre)))
-                                   : bpre;
-        }
-        bpre = load_beta(next);
-        // MEGA: the first record of each CTA is published at once (the scan starts on the first
-        // wave); later ones once the next item reaches its operands, by when the stores are done
-        if (MEGA && tid == 0 && li == 1) publish();
-        ok = wait_all(bar_tma, li & 1u);
-        if (ok && fused_pro) ok = wait_all(bar_v, li & 1u);
-        if (ok && fused_pro) {
-            // ---- fused prologue: short convolution k = 4 + SiLU of q, k, v and the bounded
-            // gate, in place on the staged tiles (halo row i = token t0 - 3 + i; output row r
-            // = token t0 + r).  Thread = (branch, 8-channel group, 8-row segment); every input
-            // row it needs is read before the barrier, so in-place writes cannot race.
-            const int br = tid >> 7, cg = tid & 15, seg = (tid >> 4) & 7;
-            const int c0 = 8 * cg, r0 = 8 * seg;
-            const uint32_t tile = br == 0 ? OFF_STG_Q : br == 1 ? OFF_STG_K : br == 2 ? OFF_STG_V : OFF_STG_G;
-            uint4 raw[C / 8 + kHalo];
-#pragma unroll
-            for (int i = 0; i < C / 8 + kHalo; ++i)
-                raw[i] = *reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r0 + i, c0));
-            __syncthreads();
-            float w[4][8];   // [tap][channel]; the gate branch needs none
-            if (br < 3) {
-                const uint8_t *wsrc = smem + OFF_CW + 1024 * br + c0 * 8;   // staged with the tiles
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    float x8[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(wsrc + 16 * m), x8);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        w[j][2 * m] = x8[j];
-                        w[j][2 * m + 1] = x8[4 + j];
-                    }
-                }
-            }
-            const float ea = br == 3 ? expf(pro.A[h]) : 0.f;
-            if (br < 3) {
-                float x0[8], x1[8], x2[8];   // sliding window: each staged row is unpacked once
-                unpack8(raw[0], x0);
-                unpack8(raw[1], x1);
-                unpack8(raw[2], x2);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float x3[8], y[8];
-                    unpack8(raw[i + kHalo], x3);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float acc = w[0][e] * x0[e] + w[1][e] * x1[e] + w[2][e] * x2[e] + w[3][e] * x3[e];
-                        y[e] = silu_fast(acc);
-                        x0[e] = x1[e];
-                        x1[e] = x2[e];
-                        x2[e] = x3[e];
-                    }
-                    *reinterpret_cast<uint4 *>(smem + tile + off_sw128(r0 + i, c0)) = pack8(y);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    float x3[8], y[8];
-                    unpack8(raw[i + kHalo], x3);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = -5.f * sigmoid_fast(ea * x3[e]);
-                    *reinterpret_cast<uint4 *>(smem + tile + off_sw128(r0 + i, c0)) = pack8(y);
-                }
-            }
-            __syncthreads();
-        }
-
-        if (ok) {
-            // ---- band-local cumulative log-decay | row norms
-            {
-                const int c = tid & 127, p = tid >> 7;
-                float gv[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    gv[i] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                        smem + OFF_STG_G + off_sw128(16 * p + i, c)));
-                float loc = 0.f;
-                uint32_t par = 0;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int r = 16 * p + i;
-                    float lg = 0.f;
-                    if (r < n) {
-                        if (fl.complex_gate) {
-                            lg = __logf(fabsf(gv[i]));
-                            par ^= (gv[i] < 0.f) ? 1u : 0u;
-                        } else {
-                            lg = gv[i];
-                        }
-                    }
-                    loc += lg;
-                    EX[r * E_STRIDE + c] = __expf(fmaxf(loc, -85.f));
-                    if (fl.complex_gate) {
-                        const uint32_t bits = __ballot_sync(0xffffffffu, par != 0);
-                        if (lane == 0) SGNL[r * 4 + quad] = bits;
-                    }
-                }
-                TOT[p * D + c] = loc;
-                const uint32_t bp = __ballot_sync(0xffffffffu, par != 0);
-                if (lane == 0) BPAR[p * 4 + quad] = bp;
-            }
-            {
-                const int rr = tid >> 2, part = tid & 3;
-                const int r = rr & 63;
-                const uint32_t tile = rr < 64 ? OFF_STG_Q : OFF_STG_K;
-                float ss = 0.f;
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    float x[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, 32 * part + 8 * m)), x);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
-                }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-                if (part == 0) NRM[rr] = fl.l2norm ? rsqrtf(ss + kL2Eps) : 1.f;
-            }
-            __syncthreads();
-
-            // ---- per-channel band factors
-            if (tid < D) {
-                const int c = tid;
-                float et[4];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) et[p] = __expf(TOT[p * D + c]);
-                TH[0 * D + c] = 1.f;
-                TH[1 * D + c] = et[0];
-                TH[2 * D + c] = et[0] * et[1];
-                TH[3 * D + c] = et[0] * et[1] * et[2];
-                const float eC = et[0] * et[1] * et[2] * et[3];
-                TG[0 * D + c] = eC;
-                TG[1 * D + c] = et[1] * et[2] * et[3];
-                TG[2 * D + c] = et[2] * et[3];
-                TG[3 * D + c] = et[3];
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb) TF[(bb * 4 + bb) * D + c] = 1.f;
-                TF[(1 * 4 + 0) * D + c] = et[0];
-                TF[(2 * 4 + 1) * D + c] = et[1];
-                TF[(2 * 4 + 0) * D + c] = et[0] * et[1];
-                TF[(3 * 4 + 2) * D + c] = et[2];
-                TF[(3 * 4 + 1) * D + c] = et[1] * et[2];
-                TF[(3 * 4 + 0) * D + c] = et[0] * et[1] * et[2];
-                const int w = c >> 5, bit = c & 31;
-                const uint32_t pc = BPAR[0 * 4 + w] ^ BPAR[1 * 4 + w] ^ BPAR[2 * 4 + w] ^ BPAR[3 * 4 + w];
-                const float gc = ((pc >> bit) & 1u) ? -eC : eC;
-                TGC[c] = gc;
-                if (c < 4) {
-                    PP[0 * 4 + c] = 0u;
-                    PP[1 * 4 + c] = BPAR[0 * 4 + c];
-                    PP[2 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c];
-                    PP[3 * 4 + c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c];
-                    SGNC[c] = BPAR[0 * 4 + c] ^ BPAR[1 * 4 + c] ^ BPAR[2 * 4 + c] ^ BPAR[3 * 4 + c];
-                }
-            }
-            // the operands overwrite the previous record's sources (W, U, A_qk)
-            if (tid == 0) {
-                if (MEGA) publish();
-                else bulk_wait_read_all();
-            }
-            __syncthreads();
-
-            // ---- operands (thread = row, 32 channels); Q e^gamma and Kd go straight to the record
-            {
-                const bool isq = row < 64;
-                const int r = row & 63;
-                const int band = r >> 4;
-                const float nrm = NRM[row];
-                const float bet = BET[r];
-                const uint32_t tile = isq ? OFF_STG_Q : OFF_STG_K;
-                const uint32_t sw = fl.complex_gate ? (SGNL[r * 4 + qq] ^ PP[band * 4 + qq]) : 0u;
-                const uint32_t swc = SGNC[qq];
-#pragma unroll
-                for (int cg = 0; cg < 4; ++cg) {
-                    const int c0 = 32 * qq + 8 * cg;
-                    float x[8], E[8], hb[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(smem + tile + off_sw128(r, c0)), x);
-                    ld8f(EX + r * E_STRIDE + c0, E);
-                    ld8f(TH + band * D + c0, hb);
-                    float xe[8], y1[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        x[e] *= ((sw >> (8 * cg + e)) & 1u) ? -nrm : nrm;
-                        xe[e] = x[e] * E[e];
-                        y1[e] = xe[e] * hb[e];
-                    }
-                    const float rs = isq ? 1.f : bet;
-                    tmem_st4(tl + TC_X + 16 * qq + 4 * cg, pack_bf16(rs * xe[0], rs * xe[1]),
-                             pack_bf16(rs * xe[2], rs * xe[3]), pack_bf16(rs * xe[4], rs * xe[5]),
-                             pack_bf16(rs * xe[6], rs * xe[7]));
-                    if (isq) {
-                        *reinterpret_cast<uint4 *>(smem + OFF_RQG + off_r128(r, c0)) = pack8(y1);
-                    } else {
-                        float gb[8], inv[8], y2[8];
-                        ld8f(TG + band * D + c0, gb);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            inv[e] = __fdividef(x[e], E[e]);
-                            y2[e] = (((swc >> (8 * cg + e)) & 1u) ? -inv[e] : inv[e]) * gb[e];
-                        }
-                        *reinterpret_cast<uint4 *>(smem + OFF_YR + off_r128(r, c0)) = pack8(y1);
-                        *reinterpret_cast<uint4 *>(smem + OFF_RKD + off_r128(r, c0)) = pack8(y2);
-                    }
-                }
-                // The band-pair B rows k_i e^{p_b - gamma_i} (one copy per row band b >= band(i)),
-                // spread evenly: warp = 8-channel group, lane = key row i in bands 0-1 plus the
-                // mirrored row 63 - i in bands 3-2, five copies per lane.
-                {
-                    const int c0 = 8 * warp;
-                    const int w32 = c0 >> 5, sh8 = c0 & 31;
-#pragma unroll
-                    for (int side = 0; side < 2; ++side) {
-                        const int i = side ? 63 - lane : lane;
-                        const int bi = i >> 4;
-                        const float nk = NRM[64 + i];
-                        const uint32_t swi = fl.complex_gate ? (SGNL[i * 4 + w32] ^ PP[bi * 4 + w32]) >> sh8 : 0u;
-                        float x[8], E[8], inv[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_STG_K + off_sw128(i, c0)), x);
-                        ld8f(EX + i * E_STRIDE + c0, E);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) inv[e] = __fdividef(((swi >> e) & 1u) ? -nk * x[e] : nk * x[e], E[e]);
-                        for (int bb = bi; bb < 4; ++bb) {
-                            float f[8], y3[8];
-                            ld8f(TF + (bb * 4 + bi) * D + c0, f);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) y3[e] = inv[e] * f[e];
-                            const int brow = 16 * pair_of(bb, bi) + (i & 15);
-                            *reinterpret_cast<uint4 *>(smem + OFF_BOP + off_r128(brow, c0)) = pack8(y3);
-                        }
-                    }
-                }
-                // each writer orders its shared-memory operands (and record parts) before the
-                // tensor-core and bulk-copy reads
-                fence_proxy_async();
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncthreads();
-
-            // ---- all ten band-pair products as one N = 160 product
-            if (tid == 0) {
-                if (next < nitems) issue_qkg(next);   // q, k, g staging is free from here on
-                tc_fence_after();
-                constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_ts(tbase + TC_D, tbase + TC_X + 8 * s, at(dK64, OFF_BOP + 256 * s), id, s > 0);
-                mma_commit(bar_mma);
-                bulk_store(img + IMG_QG, sbase + OFF_RQG, 16384);
-                bulk_store(img + IMG_KD, sbase + OFF_RKD, 16384);
-                bulk_store(img + IMG_GC, sbase + OFF_TAB + TAB_GC, 512);
-                bulk_commit();
-            }
-            ok = wait_all(bar_mma, 0);
-        }
-        if (ok) {
-            tc_fence_after();
-            // ---- A_kk -> FP32, transposed (AKK[i][r] = A_kk[r][i] for i < r, else 0); A_qk goes to
-            // the record while W/U are on the tensor cores
-            auto band_rows = [&](float (&v)[16]) {
-                const int r = row & 63, band = r >> 4;
-                const int b_lo = (quad & 1) * 2;
-                float v2[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = 0.f;
-                if (qq <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, qq), v);
-                if (qq <= b_lo + 1) {
-                    tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, qq), v2);
-                    if (band == b_lo + 1) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = v2[e];
-                    }
-                }
-            };
-            if (row >= 64) {
-                const int r = row & 63;
-                float v[16];
-                band_rows(v);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int i = 16 * qq + e;
-                    AKK[i * AS + r] = (i < r) ? v[e] : 0.f;   // a warp writes 32 consecutive r
-                }
-            }
-            tc_fence_before();
-            __syncthreads();
-
-            // ---- Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks, [T1 0; T21 T2]:
-            //   T1 = (I + A11)^{-1}, T2 = (I + A22)^{-1} from their 16 x 16 diagonal blocks (column
-            //   sweeps in registers: x_i is final once the rows above it are done, then
-            //   x_r -= A[r][i] x_i for every r > i) and X = -D1 (A10 D0) below them;
-            //   Y = A21 T1;  T21 = -T2 Y;  Tm' = Tm diag(beta) in bf16, stacked twice.
-            // TMF holds T1 (rows 0-31, columns 0-31), Y (rows 0-31, columns 32-63) and T2 (rows
-            // 32-63, columns 32-63).  AKK holds A_kk transposed, zero on and above the diagonal.
-            // T1 and T2 from their 16 x 16 diagonal blocks: D_b = (I + A_bb)^{-1} by a column sweep
-            // (lane = column, two blocks per warp); then, for each 32-block, Z = A10 D0 and
-            // X = -D1 Z (its lower-left quarter), one output per thread, Z in the columns Y takes
-            // later.  The upper-right quarters are zero.
-            if (warp < 2) {
-                const int blk = 2 * warp + (lane >> 4), base = 16 * blk, j = lane & 15;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-                for (int i = 0; i < 15; ++i) {
-                    const float xi = x[i];
-                    const float *col = AKK + (base + i) * AS + base;   // A[base + r][base + i] over r
-#pragma unroll
-                    for (int r4 = ((i + 1) >> 2) << 2; r4 < 16; r4 += 4) {   // rows r <= i hold 0
-                        const float4 av = *reinterpret_cast<const float4 *>(col + r4);
-                        x[r4] = fmaf(-av.x, xi, x[r4]);
-                        x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
-                        x[r4 + 2] = fmaf(-av.z, xi, x[r4 + 2]);
-                        x[r4 + 3] = fmaf(-av.w, xi, x[r4 + 3]);
-                    }
-                }
-#pragma unroll
-                for (int r = 0; r < 16; ++r) TMF[(base + r) * AS + base + j] = x[r];
-                if ((blk & 1) == 0) {
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) TMF[(base + r) * AS + base + 16 + j] = 0.f;
-                }
-            }
-            __syncthreads();
-            {
-                // Z = A10 D0 (per 32-block h = tid / 256): row r, column j of the 16 x 16 product
-                const int hb = tid >> 8, r = (tid >> 4) & 15, j = tid & 15, base = 32 * hb;
-                float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-                for (int k = 0; k < 16; k += 2) {
-                    z0 = fmaf(AKK[(base + k) * AS + base + 16 + r], TMF[(base + k) * AS + base + j], z0);
-                    z1 = fmaf(AKK[(base + k + 1) * AS + base + 16 + r], TMF[(base + k + 1) * AS + base + j], z1);
-                }
-                TMF[r * AS + 32 + 16 * hb + j] = z0 + z1;
-            }
-            __syncthreads();
-            {
-                // X = -D1 Z -> rows 16-31 of the 32-block, columns 0-15
-                const int hb = tid >> 8, r = (tid >> 4) & 15, j = tid & 15, base = 32 * hb;
-                const float *d1 = TMF + (base + 16 + r) * AS + base + 16;
-                float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-                for (int k = 0; k < 16; k += 2) {
-                    x0 = fmaf(d1[k], TMF[k * AS + 32 + 16 * hb + j], x0);
-                    x1 = fmaf(d1[k + 1], TMF[(k + 1) * AS + 32 + 16 * hb + j], x1);
-                }
-                TMF[(base + 16 + r) * AS + base + j] = -(x0 + x1);
-            }
-            __syncthreads();
-            // Y = A21 T1 and T21 = -T2 Y as 2 x 4 register tiles (threads 0-127: row pair rg,
-            // column group cg), so a warp's loads of a row of one factor and a column group of
-            // the other are one shared-memory wavefront each.  Meanwhile threads 128-511 pack the
-            // finished blocks of Tm' = [T1 b | 0 ; . | T2 b'] (b = beta_j) to bf16, 16 bytes each.
-            {
-                const int rg = tid >> 3, cg = tid & 7;
-                if (tid < 128) {
-                    float acc[2][4] = {};
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float2 av = *reinterpret_cast<const float2 *>(AKK + i * AS + 32 + 2 * rg);   // A21[2rg..][i]
-                        const float4 tv = *reinterpret_cast<const float4 *>(TMF + i * AS + 4 * cg);       // T1[i][4cg..]
-                        acc[0][0] = fmaf(av.x, tv.x, acc[0][0]);
-                        acc[0][1] = fmaf(av.x, tv.y, acc[0][1]);
-                        acc[0][2] = fmaf(av.x, tv.z, acc[0][2]);
-                        acc[0][3] = fmaf(av.x, tv.w, acc[0][3]);
-                        acc[1][0] = fmaf(av.y, tv.x, acc[1][0]);
-                        acc[1][1] = fmaf(av.y, tv.y, acc[1][1]);
-                        acc[1][2] = fmaf(av.y, tv.z, acc[1][2]);
-                        acc[1][3] = fmaf(av.y, tv.w, acc[1][3]);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 2; ++k)
-                        *reinterpret_cast<float4 *>(TMF + (2 * rg + k) * AS + 32 + 4 * cg) =
-                            make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
-                } else {
-                    // unit u: rows 0-31 x eight 8-column groups (T1 b, then zeros), then rows
-                    // 32-63 x the four groups of columns 32-63 (T2 b')
-                    const int u = tid - 128;
-                    const int r = u < 256 ? (u >> 3) : 32 + ((u - 256) >> 2);
-                    const int g = u < 256 ? (u & 7) : 4 + ((u - 256) & 3);
-                    float y[8];
-                    if (r < 32 && g >= 4) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = 0.f;
-                    } else {
-                        float t[8], bb[8];
-                        ld8f(TMF + r * AS + 8 * g, t);
-                        ld8f(BET + 8 * g, bb);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = t[e] * bb[e];
-                    }
-                    const uint4 pk = pack8(y);
-                    *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r, 8 * g)) = pk;
-                    *reinterpret_cast<uint4 *>(smem + OFF_TMB + off_r64(r + 64, 8 * g)) = pk;
-                }
-            }
-            __syncthreads();
-            if (tid < 128) {
-                const int rg = tid >> 3, cg = tid & 7;
-                float acc[2][4] = {};
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const float4 ta = *reinterpret_cast<const float4 *>(TMF + (32 + 2 * rg) * AS + 32 + i);   // T2[2rg][i..]
-                    const float4 tb = *reinterpret_cast<const float4 *>(TMF + (33 + 2 * rg) * AS + 32 + i);   // T2[2rg+1][i..]
-                    const float a0[4] = {ta.x, ta.y, ta.z, ta.w}, a1[4] = {tb.x, tb.y, tb.z, tb.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float4 yv = *reinterpret_cast<const float4 *>(TMF + (i + k) * AS + 32 + 4 * cg);   // Y[i+k][4cg..]
-                        acc[0][0] = fmaf(a0[k], yv.x, acc[0][0]);
-                        acc[0][1] = fmaf(a0[k], yv.y, acc[0][1]);
-                        acc[0][2] = fmaf(a0[k], yv.z, acc[0][2]);
-                        acc[0][3] = fmaf(a0[k], yv.w, acc[0][3]);
-                        acc[1][0] = fmaf(a1[k], yv.x, acc[1][0]);
-                        acc[1][1] = fmaf(a1[k], yv.y, acc[1][1]);
-                        acc[1][2] = fmaf(a1[k], yv.z, acc[1][2]);
-                        acc[1][3] = fmaf(a1[k], yv.w, acc[1][3]);
-                    }
-                }
-                // T21 b -> Tm' rows 32 + 2rg + k, columns 4cg .. 4cg + 3 (8 bytes, both copies)
-                const float4 bv = *reinterpret_cast<const float4 *>(BET + 4 * cg);
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const float y4[4] = {-acc[k][0] * bv.x, -acc[k][1] * bv.y, -acc[k][2] * bv.z, -acc[k][3] * bv.w};
-                    const uint2 pk = pack4(y4);
-                    *reinterpret_cast<uint2 *>(smem + OFF_TMB + off_r64(32 + 2 * rg + k, 4 * cg)) = pk;
-                    *reinterpret_cast<uint2 *>(smem + OFF_TMB + off_r64(96 + 2 * rg + k, 4 * cg)) = pk;
-                }
-            }
-            fence_proxy_async();   // Tm' is read by the tensor cores next
-            __syncthreads();
-
-            // ---- W = Tm' (K e^gamma),  U = Tm' V  (M = 128: Tm' stacked twice)
-            if (tid == 0) {
-                if (!mbar_wait_bounded(bar_v, li & 1u, kWaitLimit)) {
-                    sh.abort = 1;
-                    g_kda_tc2_error = 1;
-                }
-                tc_fence_after();
-                constexpr uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const uint64_t tdesc = at(dK32, OFF_TMB + 256 * s);
-                    mma_ss(tbase + TC_W, tdesc, at(dMN64, OFF_YR + 4096 * s), id, s > 0);
-                    mma_ss(tbase + TC_U, tdesc, at(dV, OFF_STG_V + 2048 * s), id, s > 0);
-                }
-                mma_commit(bar_mma);
-            }
-            __syncwarp();
-            if (row < 64) {
-                // A_qk (lower with diagonal) -> bf16 in shared memory, then the record
-                const int r = row;
-                float v[16];
-                band_rows(v);
-#pragma unroll
-                for (int g8 = 0; g8 < 2; ++g8) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int i = 16 * qq + 8 * g8 + e;
-                        y[e] = (i <= r) ? v[8 * g8 + e] : 0.f;
-                    }
-                    *reinterpret_cast<uint4 *>(smem + OFF_RAQ + off_r64(r, 16 * qq + 8 * g8)) = pack8(y);
-                }
-                fence_proxy_async();
-            }
-            if (tid == 0) bulk_wait_read_all();   // W and U are staged where Q e^gamma and Kd left from
-            ok = wait_all(bar_mma, 1);
-            if (ok && tid == 0) {
-                if (next < nitems) issue_v(next);   // the v staging is free again
-                bulk_store(img + IMG_AQK, sbase + OFF_RAQ, 8192);
-                bulk_commit();
-            }
-        }
-        if (ok) {
-            tc_fence_after();
-            // ---- W ([r][c], K-major core layout) and U (16-column slabs) -> the record; lanes
-            // 0-63 write W, lanes 64-127 (the repeated rows) write U
-            {
-                const int r = row & 63;
-                float w[32];
-                tmem_ld32(tl + (row < 64 ? TC_W : TC_U) + 32 * qq, w);
-#pragma unroll
-                for (int g8 = 0; g8 < 4; ++g8) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = w[8 * g8 + e];
-                    const int c0 = 32 * qq + 8 * g8;
-                    *reinterpret_cast<uint4 *>(smem + OFF_RWU + (row < 64 ? off_r128(r, c0) : 16384 + off_u(r, c0))) =
-                        pack8(y);
-                }
-                fence_proxy_async();
-            }
-        }
-        // the next item rewrites TMEM and shared memory: everyone is done with this one
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (ok && tid == 0) {
-            bulk_store(img + IMG_W, sbase + OFF_RWU, 16384);
-            bulk_store(img + IMG_U, sbase + OFF_RWU + 16384, 16384);
-            bulk_commit();
-            done = item;
-        }
-    }
-    if (tid == 0) {
-        if (MEGA) publish();
-        else bulk_wait_all();   // the records are complete before the scan reads them
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 512);
-}
-
-template <bool PRO>
-__global__ void __launch_bounds__(prep::NT, 1)
-chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                  const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                  int BH, KernelFlags fl, PrepPrologue pro) {
-    prep_body<PRO, false>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x,
-                          (int)gridDim.x, nullptr);
-}
 
 // The prep with two item groups per CTA (kda_chunk_prep.cuh): one 512-thread CTA per SM, its
 // TMEM split between the groups.  MEGA: CTA `cta` of `ncta` prep CTAs of the one-launch form.
@@ -1284,6 +559,14 @@ scan_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfl
     if (warp == 0) tmem_dealloc(tbase, L::TMEM_COLS);
 }
 
+#include "kda_chunk_scan.cuh"
+
+__global__ void __launch_bounds__(scan3::NT, 1)
+chunk_scan3_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
+                   float *__restrict__ S_T, int T, int H, float scale) {
+    scan3_body<false>(ws, S0, out, S_T, T, H, scale, (int)blockIdx.x, nullptr, 0, kWaitLimit);
+}
+
 template <int NS, bool GATED>
 __global__ void __launch_bounds__(scan::Layout<NS>::NT, 1)
 chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
@@ -1294,16 +577,6 @@ chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S
                                 nullptr, 0);
 }
 
-// One launch for few-head calls: CTAs [0, n_scan) run the scan's slice CTAs, the rest the prep,
-// all resident at once (a cooperative launch), the scan reading each record as soon as the
-// prep has published it.  The block has the prep's 512 threads; a scan CTA uses its first
-// 32 * (NSW + 2) (state warps, the MMA warp, the loader warp).
-// dynamic shared memory of the one-launch form: the larger of the two roles' layouts
-template <int NS>
-constexpr uint32_t mega_smem_bytes() {
-    return prep::SMEM_BYTES > scan::Layout<NS>::SMEM_BYTES ? prep::SMEM_BYTES : scan::Layout<NS>::SMEM_BYTES;
-}
-
 // The scan's role is kept out of line: inlined beside the prep, its code interleaves with the
 // prep's, and the prep's first item, which runs from a cold instruction cache whenever the
 // call's working set has left L2, takes about twice as long.
@@ -1312,21 +585,6 @@ __device__ __noinline__ void mega_scan(const uint8_t *ws, const float *S0, __nv_
                                        int H, float scale, int cta, const int *flags, int BH,
                                        uint32_t poll_limit = kWaitLimit) {
     scan_body<NS, false, true>(ws, S0, out, S_T, T, H, scale, nullptr, nullptr, 0.f, cta, flags, BH, poll_limit);
-}
-
-template <bool PRO, int NS>
-__global__ void __launch_bounds__(prep::NT, 1)
-chunk_mega_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                  const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                  int BH, KernelFlags fl, PrepPrologue pro, const float *__restrict__ S0,
-                  __nv_bfloat16 *__restrict__ out, float *__restrict__ S_T, int n_scan,
-                  int *__restrict__ flags) {
-    if ((int)blockIdx.x < n_scan)
-        mega_scan<NS>(ws, S0, out, S_T, T, H, fl.scale, (int)blockIdx.x, flags, BH);
-    else
-        prep_body<PRO, true>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro,
-                             (int)blockIdx.x - n_scan, (int)gridDim.x - n_scan, flags);
 }
 
 // The one-launch form with the two-group prep: prep CTAs are 512 threads of two item groups.
@@ -1392,27 +650,25 @@ size_t chunk_tc2_workspace_bytes(int B, int T, int H) {
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st);
-static bool use_prep2(const ChunkArgs &a);
 
 cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mg;
     if (!make_map2(&mq, a.q, a.B, a.T, a.H) || !make_map2(&mk, a.k, a.B, a.T, a.H) ||
         !make_map2(&mv, a.v, a.B, a.T, a.H) || !make_map2(&mg, a.g, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr}, st);
+    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0}, st);
 }
 
 cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mz;
-    // the one-group prep stages a 3-row halo with each tile; the two-group prep reads those rows
-    // from global memory and stages 64-row tiles
-    const int rows = use_prep2(a) ? C : C + prep::kHalo;
+    // 64-row tiles: the prep reads the three rows before a chunk from global memory
+    const int rows = C;
     if (!make_map2(&mq, p.q_pre, a.B, a.T, a.H, rows) || !make_map2(&mk, p.k_pre, a.B, a.T, a.H, rows) ||
         !make_map2(&mv, p.v_pre, a.B, a.T, a.H, rows) || !make_map2(&mz, p.z, a.B, a.T, a.H, rows))
         return cudaErrorInvalidValue;
     return launch_split(a, mq, mk, mv, mz,
                         PrepPrologue{(const __nv_bfloat16 *)p.conv_w, p.A, p.beta_logit, (const __nv_bfloat16 *)p.q_pre,
-                                     (const __nv_bfloat16 *)p.k_pre, (const __nv_bfloat16 *)p.v_pre},
+                                     (const __nv_bfloat16 *)p.k_pre, (const __nv_bfloat16 *)p.v_pre, 0},
                         st);
 }
 
@@ -1449,27 +705,28 @@ static cudaError_t launch_scan(const ChunkArgs &a, const uint8_t *ws, cudaStream
                               (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
 }
 
-// Per-(chunk, head) prep cost per SM (cycles; the two-group prep overlaps two items per SM) and
-// per-chunk scan chain at d = 128 on a B200 SM (measured).
-constexpr double kPrepItemCycles = 21000.0;
-constexpr double kPrep2ItemCycles = 7000.0;
+// Per-(chunk, head) prep cost of one SM (cycles; two items in flight per SM) and the per-chunk
+// chain of the sliced scan at d = 128 on a B200 SM (measured).
+constexpr double kPrepItemCycles = 13300.0;
 static double scan_chunk_cycles(int ns) { return ns == 16 ? 2900.0 : ns == 32 ? 3000.0 : ns == 64 ? 3100.0 : 4900.0; }
 
 // Polls of a bounded wait before it gives up (kda_set_wait_limit; failure-handling tests only).
 static uint32_t g_wait_limit = kWaitLimit;
 
-// Slice width of the one-launch form (prep and scan CTAs side by side), or 0 when the two
-// launches are faster: prep on all SMs, then the scan, against the prep on the SMs the scan's
-// CTAs leave, overlapped with the scan, plus one item of ramp.
-int mega_slice_width(int BH, int nch, int sms, double t_item) {
+// Slice width of the one-launch form (prep and sliced-scan CTAs side by side), or 0 when the two
+// launches are faster: prep on all SMs, then the TMEM scan, against the prep on the SMs the scan's
+// CTAs leave, overlapped with the sliced scan, plus one item of ramp.
+constexpr double kScan3ChunkCycles = 4100.0;   // the TMEM scan's chain, one CTA per sequence
+int mega_slice_width(int BH, int nch, int sms) {
     const double items = (double)BH * nch;
-    const double two = ceil(items / sms) * t_item + nch * scan_chunk_cycles(scan_slice_width(BH, false));
+    const double waves = ceil((double)BH / sms);
+    const double two = ceil(items / sms) * kPrepItemCycles + waves * nch * kScan3ChunkCycles;
     int best = 0;
     double best_t = 0.9 * two;
     for (int ns : {32, 64}) {
         const int n_scan = BH * (D / ns);
         if (n_scan > sms / 2) continue;
-        const double t = fmax(ceil(items / (sms - n_scan)) * t_item, nch * scan_chunk_cycles(ns)) + t_item;
+        const double t = fmax(ceil(items / (sms - n_scan)) * kPrepItemCycles, nch * scan_chunk_cycles(ns)) + kPrepItemCycles;
         if (t < best_t) {
             best = ns;
             best_t = t;
@@ -1492,32 +749,26 @@ uint32_t set_wait_limit(uint32_t polls) {
     return prev;
 }
 
-// Whether the two-group prep runs (all unsigned-gate calls; Complex-KDA keeps the one-group prep).
-static bool use_prep2(const ChunkArgs &a) { return !a.fl.complex_gate && getenv("KDA_PREP_FORM") == nullptr; }
-
+// The one-launch form: CTAs [0, n_scan) are sliced-scan CTAs, the rest prep CTAs of two item
+// groups, all resident at once (a cooperative launch; the scan CTAs wait for the records the
+// prep CTAs publish).
 template <bool PRO, int NS>
 static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, cudaStream_t st) {
-    const bool v2 = use_prep2(a);
-    auto k = chunk_mega_kernel<PRO, NS>;
-    auto k2 = chunk_mega2_kernel<PRO, NS>;
-    constexpr uint32_t smem1 = mega_smem_bytes<NS>(), smem2 = mega2_smem_bytes<NS>();
-    static_assert(smem1 <= 232448 && smem2 <= 232448, "shared memory budget");
-    static_assert(scan::Layout<NS>::NT + 32 <= prep::NT, "the scan's warps and the loader warp fit the prep's block");
-    static_assert(prep::NT == prep2::NT, "one block size for both prep forms");
-    const uint32_t smem = v2 ? smem2 : smem1;
-    cudaError_t e = v2 ? cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                       : cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto k = chunk_mega2_kernel<PRO, NS>;
+    constexpr uint32_t smem = mega2_smem_bytes<NS>();
+    static_assert(smem <= 232448, "shared memory budget");
+    static_assert(scan::Layout<NS>::NT + 32 <= prep2::NT, "the scan's warps and the loader warp fit the prep's block");
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int nch = (a.T + C - 1) / C, BH = a.B * a.H, n_scan = BH * (D / NS);
     uint8_t *ws = (uint8_t *)a.workspace;
     int *flags = reinterpret_cast<int *>(ws + (size_t)nch * BH * IMG_BYTES);
     e = cudaMemsetAsync(flags, 0, (size_t)nch * BH * sizeof(int), st);
     if (e != cudaSuccess) return e;
-    // every CTA resident at once (the scan CTAs wait for records the prep CTAs publish)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)num_sms());
-    cfg.blockDim = dim3(prep::NT);
+    cfg.blockDim = dim3(prep2::NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -1526,21 +777,42 @@ static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     mark_launch(a, st);
-    if (v2)
-        return cudaLaunchKernelEx(&cfg, k2, mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, BH, a.fl,
-                                  pro, a.S0, (__nv_bfloat16 *)a.out, a.S_T, n_scan, flags, g_wait_limit);
     return cudaLaunchKernelEx(&cfg, k, mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, BH, a.fl, pro,
-                              a.S0, (__nv_bfloat16 *)a.out, a.S_T, n_scan, flags);
+                              a.S0, (__nv_bfloat16 *)a.out, a.S_T, n_scan, flags, g_wait_limit);
 }
 
+static cudaError_t launch_scan3(const ChunkArgs &a, const uint8_t *ws, cudaStream_t st) {
+    auto k = chunk_scan3_kernel;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan3::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // programmatic dependency on the prep kernel: the scan's CTAs may start (barriers, TMEM,
+    // S0) on SMs the prep has left and wait in the kernel for its records
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.B * a.H));
+    cfg.blockDim = dim3(scan3::NT);
+    cfg.dynamicSmemBytes = scan3::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, ws, a.S0, (__nv_bfloat16 *)a.out, a.S_T, a.T, a.H, a.fl.scale);
+}
+
+// The split form: few sequences take the one-launch form with value-column slices (its chain is
+// the shorter one there); otherwise the prep kernel, then the TMEM scan (one CTA per sequence),
+// or with the output epilogue the sliced scan with whole-row slices (it normalises rows in its
+// registers).  U's layout in the record follows the scan that reads it.
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st) {
-    const bool v2 = use_prep2(a);
+    const bool p = pro.conv_w != nullptr;
+    const int nch = (a.T + C - 1) / C;
     if (!a.out_gate) {
-        const int ns = mega_slice_width(a.B * a.H, (a.T + C - 1) / C, num_sms(), v2 ? kPrep2ItemCycles : kPrepItemCycles);
+        const int ns = mega_slice_width(a.B * a.H, nch, num_sms());
         if (ns) {
-            const bool p = pro.conv_w != nullptr;
+            pro.u_slabs = 1;
             cudaError_t e = ns == 32 ? (p ? launch_mega<true, 32>(a, mq, mk, mv, mg, pro, st)
                                           : launch_mega<false, 32>(a, mq, mk, mv, mg, pro, st))
                                      : (p ? launch_mega<true, 64>(a, mq, mk, mv, mg, pro, st)
@@ -1549,37 +821,21 @@ static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const
             (void)cudaGetLastError();   // not enough room to co-schedule: the two launches below
         }
     }
-    // the plain instantiations carry none of the prologue or epilogue code
-    const int nch = (a.T + C - 1) / C;
+    pro.u_slabs = a.out_gate ? 1 : 0;
     uint8_t *ws = (uint8_t *)a.workspace;
     const int nitems = nch * a.B * a.H;
-    cudaError_t e;
-    if (v2) {
-        auto prep_k = pro.conv_w ? chunk_prep2_kernel<true> : chunk_prep2_kernel<false>;
-        e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep2::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        mark_launch(a, st);
-        const int ctas = std::min((nitems + prep2::NG - 1) / prep2::NG, num_sms());
-        prep_k<<<(unsigned)ctas, prep2::NT, prep2::SMEM_BYTES, st>>>(mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws,
-                                                                    a.T, a.H, a.B * a.H, a.fl, pro, g_wait_limit);
-    } else {
-        auto prep_k = pro.conv_w ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
-        e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep::SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        mark_launch(a, st);
-        prep_k<<<(unsigned)std::min(nitems, num_sms()), prep::NT, prep::SMEM_BYTES, st>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws, a.T, a.H, a.B * a.H, a.fl, pro);
-    }
+    auto prep_k = p ? chunk_prep2_kernel<true> : chunk_prep2_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep2::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    mark_launch(a, st);
+    const int ctas = std::min((nitems + prep2::NG - 1) / prep2::NG, num_sms());
+    prep_k<<<(unsigned)ctas, prep2::NT, prep2::SMEM_BYTES, st>>>(mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws,
+                                                                a.T, a.H, a.B * a.H, a.fl, pro, g_wait_limit);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     mark_launch(a, st);
     if (a.out_gate) return launch_scan<D, true>(a, ws, st);
-    switch (scan_slice_width(a.B * a.H, false)) {
-        case 16: return launch_scan<16, false>(a, ws, st);
-        case 32: return launch_scan<32, false>(a, ws, st);
-        case 64: return launch_scan<64, false>(a, ws, st);
-        default: return launch_scan<D, false>(a, ws, st);
-    }
+    return launch_scan3(a, ws, st);
 }
 
 }  // namespace kda

@@ -87,9 +87,10 @@ def test_sweep_T2048_full(K):
     assert rel_err(f64(S_T), ref[1]) <= 2e-2
 
 
-@pytest.mark.parametrize("T", [8192, 65536])
+@pytest.mark.parametrize("T", [8192, 32768, 65536])
 def test_sweep_long_sampled(K, T):
-    """length-sweep workload at T = 8192 and 65536, sampled heads."""
+    """length-sweep workload at T = 8192, 32768 and 65536 (every length the benchmark times
+    beyond the fully checked T = 2048), sampled heads."""
     x = W.sweep_inputs(T)
     out, S_T = _run(K, x)
     heads = [0, 47, 95]
