@@ -28,8 +28,9 @@ kda_opts resolve(const kda_opts *o) {
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
-// g without the -5 floor (Kimi Linear's softplus gate, or the caller says so): the tensor-core
-// forms' band-referenced decay factors could leave the bf16/FP32 range, the FP32 path cannot
+// g without the -5 floor (Kimi Linear's softplus gate, or the caller says so): the split
+// tensor-core form takes it with FP32 diagonal blocks (its fused form and its signed-gate steps
+// rely on the floor); with Complex-KDA it runs on the FP32 path
 bool unbounded(const kda_opts &o) { return (o.flags & (KDA_UNBOUNDED_DECAY | KDA_GATE_SOFTPLUS)) != 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -50,8 +51,9 @@ KernelFlags kflags(const kda_opts &o) {
 // 6.8 us of one SM per (chunk, head) item (the two-group prep), t_scan = 2.4 us per chunk (one
 // CTA per head); the model uses their ratios.  With the two-group prep the split form wins at
 // every B*H; the fused form stays available through KDA_FUSED.  KDA_SPLIT forces the split.
+// An unbounded gate always takes the split form.
 bool use_tc(const kda_opts &o, int dk, int dv) {
-    return o.dtype == KDA_BF16 && dk == 128 && dv == 128 && !unbounded(o);
+    return o.dtype == KDA_BF16 && dk == 128 && dv == 128 && !(unbounded(o) && (o.flags & KDA_COMPLEX));
 }
 int device_sms() {
     int dev = 0, n = 0;
@@ -61,6 +63,7 @@ int device_sms() {
     return n;
 }
 bool use_fused(const kda_opts &o, int B, int H) {
+    if (unbounded(o)) return false;
     if (o.flags & KDA_FUSED) return true;
     if (o.flags & KDA_SPLIT) return false;
     const double x = (double)B * H / device_sms();
@@ -115,7 +118,8 @@ int run_chunk(ChunkArgs &a, bool fused, cudaStream_t st) {
     // every sequence (about 1 us per chunk); a separate pass costs the bytes of out and the
     // gate instead.  Measured on B200 the chain wins from about 64 sequences on (T=8192:
     // 96 heads 0.14 vs 0.22 ms; T=4096, 16 heads: 0.048 vs 0.020 ms).
-    const bool tc = chunk_tc_supported(a) && !a.exact_decay;
+    const bool tc = chunk_tc_supported(a) && !(a.exact_decay && a.fl.complex_gate);
+    if (a.exact_decay) fused = false;
     const bool split = tc && !fused;
     const bool fuse_epi = split && a.out_gate && (long long)a.B * a.H >= 64;
     const void *gate = a.out_gate;
@@ -516,6 +520,7 @@ int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_p
         a.fl = kflags(o);
         a.workspace = ws;
         a.workspace_bytes = need;
+        a.exact_decay = unbounded(o);
         a.events = o.events; a.n_events = o.n_events;
         a.launch_idx = &launches;
         cudaError_t e = launch_chunk_tc2_prologue(p, a, stream);

@@ -26,6 +26,13 @@
 //   CUDA      W, U -> record
 //
 // The record (74,240 bytes per chunk and head) has the layout the scan kernel reads.
+//
+// UNB (a gate without the -5 floor: Kimi Linear's softplus map, same page, Q&A on how the decay
+// map differs from Kimi Linear's): the band-referenced factors of the band's own keys,
+// e^{p_b - gamma_i}, have no bound.  Only the six off-diagonal band pairs stay on the tensor
+// cores (N = 96), with every factor formed as one exponential of a non-positive difference;
+// the four diagonal 16 x 16 blocks are FP32 position pairs, sum_c q_rc k_ic prod_{i<s<=r} alpha_sc,
+// with the products of alpha = e^g taken row by row (no factor above 1, underflow harmless).
 #pragma once
 
 namespace prep2 {
@@ -56,10 +63,23 @@ constexpr uint32_t TAB_PX = TAB_BAR + 64;   // Complex-KDA: sign parity of each 
 constexpr uint32_t GROUP_USED = OFF_TAB + TAB_PX + 32;
 constexpr uint32_t OFF_LO = OFF_KH;    // Complex-KDA: the low bf16 part of log|alpha| (g's layout)
 constexpr uint32_t GROUP_STRIDE = 114688;
+// UNB: alpha = e^g (FP32 [64 r][128 c]) after the band totals while the diagonal blocks are
+// formed; the blocks wait in the region's last 6 KB for the readout (the six off-diagonal pairs'
+// B rows are rows 0-95 of each half)
+constexpr uint32_t OFF_ALPHA = OFF_KH + 2048;
+constexpr uint32_t OFF_DQ = OFF_KH + 34816;    // A_qk's diagonal blocks, bf16 [4 bands][16 r][16 i]
+constexpr uint32_t OFF_DK = OFF_KH + 36864;    // A_kk's diagonal blocks, FP32 [4 bands][16 r][16 i]
+constexpr int NPAIR_U = 96;
+// UNB band factors, FP32 rows of 128 (T_b = band b's total, p_b = T_0 + .. + T_{b-1},
+// gamma_C = p_4): as logarithms T_0..T_3, T_0+T_1, T_1+T_2, T_0+T_1+T_2, gamma_C - p_0..2; then
+// e^{p_1}, e^{p_2}, e^{p_3} (each <= 1)
+constexpr int R_LT = 0, R_L01 = 4, R_L12 = 5, R_L012 = 6, R_LC = 7, R_EXP = 10;
 constexpr uint32_t SMEM_BYTES = 1024 + GROUP_STRIDE + GROUP_USED;
 static_assert(GROUP_USED <= GROUP_STRIDE, "group layout");
 static_assert(OFF_TMF + 17408 <= OFF_TAB, "UT tiles inside the band-pair operand's region");
 static_assert(SMEM_BYTES <= 232448 - 256, "shared memory budget");
+static_assert(OFF_ALPHA + 32768 <= OFF_DQ && OFF_DK + 4096 <= OFF_TAB, "UNB staging inside the band-pair region");
+static_assert(OFF_KH + KH_HALF + NPAIR_U * 128 <= OFF_DQ, "UNB B rows clear of the diagonal blocks");
 // TMEM columns of a group (its 256): D = cumsum / band pairs / [W; U]; the block-diagonal
 // Tm' operand; the constant cumsum operand L
 constexpr uint32_t TC_D = 0, TC_TM = 160, TC_LM = 224;
@@ -87,6 +107,13 @@ __device__ __forceinline__ int row_ecp(int b) { return b == 3 ? R_ET + 3 : R_ECP
 __device__ __forceinline__ int row_em(int bp, int b) {
     return bp == b + 1 ? R_ET + b : (bp == 2 ? R_EM20 : b == 1 ? R_EM31 : R_EM30);
 }
+// UNB log rows: gamma_C - p_b, p_b' - p_b (b' > b)
+__device__ __forceinline__ int lrow_c(int b) { return b == 3 ? R_LT + 3 : R_LC + b; }
+__device__ __forceinline__ int lrow_m(int bp, int b) {
+    return bp == b + 1 ? R_LT + b : (bp == 2 ? R_L01 : b == 1 ? R_L12 : R_L012);
+}
+// UNB: TMEM column block (16 columns) of the off-diagonal band pair (row band b, key band j < b)
+__device__ __forceinline__ int pair_u(int b, int j) { return (j == 0 ? 0 : j == 1 ? 3 : 5) + b - j - 1; }
 }  // namespace prep2
 
 // Wait for phase `ph` of `bar` with the built-in limit, whatever the run's wait limit: used at
@@ -167,8 +194,9 @@ __device__ __forceinline__ void ld4f2(const float *p, float2 (&v)[4]) {
 // prep CTAs and their number.  MEGA: items are taken chunk-major and each record is published
 // (flags[item], release) once its stores are visible; otherwise items are taken chunk-fastest
 // and the scan is the next kernel.  PRO: the tiles hold the raw branch inputs and z; the short
-// convolution, SiLU, the gate and beta = sigmoid(logit) run on chip first.
-template <bool PRO, bool MEGA>
+// convolution, SiLU, the gate and beta = sigmoid(logit) run on chip first.  UNB: g has no
+// lower bound (see the top of this file).
+template <bool PRO, bool MEGA, bool UNB>
 __device__ __forceinline__ void
 prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap *ptm_v,
             const CUtensorMap *ptm_g, const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws,
@@ -206,7 +234,7 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
         mbar_fence_init();
         *abort_f = 0;
     }
-    if (gt < 128) FT[R_ONE * 128 + gt] = 1.f;
+    if (!UNB && gt < 128) FT[R_ONE * 128 + gt] = 1.f;
     // constant TMEM operands: L = [L_band; L_band] (lane m, row m & 63: ones at s <= row inside
     // the row's band), and the zero halves of the block-diagonal Tm' operand
     if (gw < 4) {
@@ -386,6 +414,30 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                     if (tail && r >= n) y[0] = y[1] = y[2] = y[3] = 0u;
                     st16(gsm + unit(r), y[0], y[1], y[2], y[3]);
                 }
+            } else if (pro.softplus) {
+                // Kimi Linear's map g = -e^A softplus(z), softplus(z) = max(z, 0) + ln(1 + e^-|z|)
+                const float ea = expf(a_h);
+                constexpr float kL2E = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+                asm volatile("bar.sync %0, %1;" ::"r"(sub_bar), "r"(128) : "memory");
+                const bool tail = n < C;
+#pragma unroll 2
+                for (int i = 0; i < 16; ++i) {
+                    const int r = r0 + i;
+                    const uint4 u = ld16(gsm + unit(r));
+                    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t y[4];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float2 z = bf2(uw[m]);
+                        float l0, l1;
+                        asm("lg2.approx.f32 %0, %1;" : "=f"(l0) : "f"(1.f + ex2(-fabsf(z.x) * kL2E)));
+                        asm("lg2.approx.f32 %0, %1;" : "=f"(l1) : "f"(1.f + ex2(-fabsf(z.y) * kL2E)));
+                        const float2 sp = make_float2(fmaxf(z.x, 0.f) + kLn2 * l0, fmaxf(z.y, 0.f) + kLn2 * l1);
+                        y[m] = pk2(mul2(sp, dup2(-ea)));
+                    }
+                    if (tail && r >= n) y[0] = y[1] = y[2] = y[3] = 0u;
+                    st16(gsm + unit(r), y[0], y[1], y[2], y[3]);
+                }
             } else {
                 const float2 ea = dup2(0.5f * expf(a_h));   // sigmoid(a z) = (1 + tanh(a z / 2)) / 2
                 asm volatile("bar.sync %0, %1;" ::"r"(sub_bar), "r"(128) : "memory");
@@ -509,8 +561,51 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                     make_float4(gam[4 * m], gam[4 * m + 1], gam[4 * m + 2], gam[4 * m + 3]);
         }
         gbar(gi);
-        // ---- per-channel band factors (threads 0-127)
-        if (gt < 128) {
+        // ---- per-channel band factors (threads 0-127); UNB: as logarithms, while threads 128-255
+        // form alpha = e^g for the diagonal blocks
+        if (UNB) {
+            constexpr float kL2E = 1.4426950408889634f;
+            if (gt < 128) {
+                const int c = gt;
+                const float t0 = TOT[c], t1 = TOT[128 + c], t2 = TOT[256 + c], t3 = TOT[384 + c];
+                FT[(R_LT + 0) * 128 + c] = t0;
+                FT[(R_LT + 1) * 128 + c] = t1;
+                FT[(R_LT + 2) * 128 + c] = t2;
+                FT[(R_LT + 3) * 128 + c] = t3;
+                const float p2 = t0 + t1, p3 = p2 + t2;
+                FT[R_L01 * 128 + c] = p2;
+                FT[R_L12 * 128 + c] = t1 + t2;
+                FT[R_L012 * 128 + c] = p3;
+                const float c2 = t2 + t3, c1 = t1 + c2, c0 = t0 + c1;
+                FT[(R_LC + 0) * 128 + c] = c0;
+                FT[(R_LC + 1) * 128 + c] = c1;
+                FT[(R_LC + 2) * 128 + c] = c2;
+                FT[(R_EXP + 0) * 128 + c] = ex2(t0 * kL2E);
+                FT[(R_EXP + 1) * 128 + c] = ex2(p2 * kL2E);
+                FT[(R_EXP + 2) * 128 + c] = ex2(p3 * kL2E);
+                reinterpret_cast<float *>(img + IMG_GC)[c] = ex2(c0 * kL2E);
+            }
+            // alpha = e^g, thread = (8-channel group, rows gt / 16 + 16 m): a warp writes two
+            // whole rows per store
+            if (!PRO) (void)wait(b_g, ph);   // the g tile (already complete: a formality per thread)
+            const int cg = gt & 15;
+            float *AL = reinterpret_cast<float *>(gsm + OFF_ALPHA);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int rr = (gt >> 4) + 16 * m;
+                const uint4 gu = ld16(gsm + OFF_G + off_t(rr, cg));
+                const uint32_t gw4[4] = {gu.x, gu.y, gu.z, gu.w};
+                float a[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 g2 = bf2(gw4[e]);
+                    a[2 * e] = ex2(g2.x * kL2E);
+                    a[2 * e + 1] = ex2(g2.y * kL2E);
+                }
+                *reinterpret_cast<float4 *>(AL + rr * 128 + 8 * cg) = make_float4(a[0], a[1], a[2], a[3]);
+                *reinterpret_cast<float4 *>(AL + rr * 128 + 8 * cg + 4) = make_float4(a[4], a[5], a[6], a[7]);
+            }
+        } else if (gt < 128) {
             const int c = gt;
             float et[4];
 #pragma unroll
@@ -535,11 +630,175 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
             reinterpret_cast<float *>(img + IMG_GC)[c] = sc * eC;
         }
         gbar(gi);
+        if constexpr (UNB) {
+            // ---- the diagonal 16 x 16 blocks as FP32 position pairs.  Thread = (band, row pair
+            // x / 15 - x, 8-channel group e); a warp takes row pairs x = 2 xh' + (lane >> 4) of
+            // one band with xh' = xh, then of another band with xh' = 3 - xh, so every warp walks
+            // 26 key rows.  Walking the key row i down from the row, f = prod_{i<s<=r} alpha_s
+            // grows by one factor per step; sum_c q_rc k_ic f_c (and the same with k_r) for two
+            // steps at a time is reduced over the 16 channel groups of a half-warp by a
+            // transposing butterfly (eight values, eight shuffles).  Keys past the row (i > r) are
+            // masked at the readout.
+            const int xh = gw & 3, tb = gw >> 2, xl = lane >> 4, e = lane & 15;
+            const float *AL = reinterpret_cast<const float *>(gsm + OFF_ALPHA);
+            __nv_bfloat16 *DQ = reinterpret_cast<__nv_bfloat16 *>(gsm + OFF_DQ);
+            float *DK = reinterpret_cast<float *>(gsm + OFF_DK);
+            const bool b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1, b1 = (lane >> 1) & 1;
+            auto norm_qk = [&](int row) -> float2 {
+                return fl.l2norm ? make_float2(rsqrtf(NRMP[row] + NRMP[128 + row] + kL2Eps),
+                                               rsqrtf(NRMP[64 + row] + NRMP[192 + row] + kL2Eps))
+                                 : make_float2(1.f, 1.f);
+            };
+#pragma unroll 1
+            for (int task = 0; task < 2; ++task) {
+                const int xt = task == 0 ? xh : 3 - xh;
+                const int ra = 2 * xt + xl, rb = 15 - ra, ilmax = 15 - 2 * xt;   // ilmax odd
+                const int bnd = tb + 2 * task, bs = 16 * bnd;
+                const float2 na = norm_qk(bs + ra), nb = norm_qk(bs + rb);
+                float2 qa[4], ka[4], qb[4], kb[4], fa[4], fb[4], ap[4];
+                {
+                    const uint4 u0 = ld16(gsm + OFF_X + off_x(0, bs + ra, e));
+                    const uint4 u1 = ld16(gsm + OFF_X + off_x(1, bs + ra, e));
+                    const uint4 u2 = ld16(gsm + OFF_X + off_x(0, bs + rb, e));
+                    const uint4 u3 = ld16(gsm + OFF_X + off_x(1, bs + rb, e));
+                    const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w}, w1[4] = {u1.x, u1.y, u1.z, u1.w};
+                    const uint32_t w2[4] = {u2.x, u2.y, u2.z, u2.w}, w3[4] = {u3.x, u3.y, u3.z, u3.w};
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        qa[m] = mul2(bf2(w0[m]), dup2(na.x));
+                        ka[m] = mul2(bf2(w1[m]), dup2(na.y));
+                        qb[m] = mul2(bf2(w2[m]), dup2(nb.x));
+                        kb[m] = mul2(bf2(w3[m]), dup2(nb.y));
+                        fa[m] = fb[m] = ap[m] = make_float2(1.f, 1.f);
+                    }
+                }
+                // one key step: the q and k sums of rows a and b with key row i (0 where i > row)
+                auto step = [&](int il, float (&v)[4]) {
+                    const uint4 ku = ld16(gsm + OFF_X + off_x(1, bs + il, e));
+                    const uint32_t wk[4] = {ku.x, ku.y, ku.z, ku.w};
+                    float2 av[4];
+                    ld4f2(AL + (bs + il) * 128 + 8 * e, av);
+                    v[0] = v[1] = v[2] = v[3] = 0.f;
+                    if (il <= rb) {
+                        float2 aq = make_float2(0.f, 0.f), ak = aq;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            if (il < rb) fb[m] = mul2(fb[m], ap[m]);
+                            const float2 t = mul2(bf2(wk[m]), fb[m]);
+                            aq = fma2(qb[m], t, aq);
+                            ak = fma2(kb[m], t, ak);
+                        }
+                        v[0] = aq.x + aq.y;
+                        v[1] = ak.x + ak.y;
+                    }
+                    if (il <= ra) {
+                        float2 aq = make_float2(0.f, 0.f), ak = aq;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) {
+                            if (il < ra) fa[m] = mul2(fa[m], ap[m]);
+                            const float2 t = mul2(bf2(wk[m]), fa[m]);
+                            aq = fma2(qa[m], t, aq);
+                            ak = fma2(ka[m], t, ak);
+                        }
+                        v[2] = aq.x + aq.y;
+                        v[3] = ak.x + ak.y;
+                    }
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) ap[m] = av[m];
+                };
+#pragma unroll 1
+                for (int il = ilmax; il > 0; il -= 2) {
+                    float v0[4], v1[4];   // steps il and il - 1: (q, k) sums of row b, then row a
+                    step(il, v0);
+                    step(il - 1, v1);
+                    // value index 4 b3 + 2 b2 + b1: step (b3), row a / b (b2), k / q (b1)
+                    float w4[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float keep = b3 ? v1[j] : v0[j], send = b3 ? v0[j] : v1[j];
+                        w4[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+                    }
+                    float w2[2];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float keep = b2 ? w4[2 + j] : w4[j], send = b2 ? w4[j] : w4[2 + j];
+                        w2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                    }
+                    float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2);
+                    w1 += __shfl_xor_sync(0xffffffffu, w1, 1);
+                    const int i = il - (b3 ? 1 : 0), rr = b2 ? ra : rb;
+                    if ((lane & 1) == 0 && i <= rr) {
+                        const float nki = fl.l2norm ? rsqrtf(NRMP[64 + bs + i] + NRMP[192 + bs + i] + kL2Eps) : 1.f;
+                        const int o = (bnd * 16 + rr) * 16 + i;
+                        if (b1) DK[o] = w1 * nki * BET[bs + rr];
+                        else DQ[o] = __float2bfloat16_rn(w1 * nki);
+                    }
+                }
+            }
+            gbar(gi);
+            tmem_ld32(tl + TC_D + 32 * cq, gam);   // gamma~ again (not kept live across the pairs)
+        }
 
         // ---- operands (thread = row r, 32 channels): E = e^{gamma~}, 1/E; Q E and beta K E in
         // place; K e^gamma over g; the band-pair B rows k e^{p_b - gamma} for b >= band(r); the
-        // record's Q e^gamma and K e^{gamma_C - gamma}
-        {
+        // record's Q e^gamma and K e^{gamma_C - gamma}.  UNB: every factor is one exponential of a
+        // non-positive exponent, or a product of such: E, e^gamma = E e^{p_b}, e^{gamma_C - gamma},
+        // and for the later bands' B rows e^{p_b' - gamma}; the own band's B rows are not formed.
+        if constexpr (UNB) {
+            const float nq = fl.l2norm ? rsqrtf(NRMP[r] + NRMP[128 + r] + kL2Eps) : 1.f;
+            const float nk = fl.l2norm ? rsqrtf(NRMP[64 + r] + NRMP[192 + r] + kL2Eps) : 1.f;
+            const float2 nq2 = dup2(nq), nk2 = dup2(nk), bt2 = dup2(BET[r]);
+            const float *ep = FT + (R_EXP + band - 1) * 128, *lc = FT + lrow_c(band) * 128;
+            constexpr float kL2E = 1.4426950408889634f;
+            auto ex2p = [&](float2 x) { return make_float2(ex2(x.x * kL2E), ex2(x.y * kL2E)); };
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cg = 4 * cq + m, c0 = 8 * cg;
+                const uint4 uq = ld16(gsm + OFF_X + off_x(0, r, cg));
+                const uint4 uk = ld16(gsm + OFF_X + off_x(1, r, cg));
+                const uint32_t wq[4] = {uq.x, uq.y, uq.z, uq.w}, wk[4] = {uk.x, uk.y, uk.z, uk.w};
+                float2 fp[4], fc[4];
+                if (band > 0) {
+                    ld4f2(ep + c0, fp);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) fp[e] = make_float2(1.f, 1.f);
+                }
+                ld4f2(lc + c0, fc);
+                uint32_t o_qe[4], o_qg[4], o_ke[4], o_kg[4], o_kd[4];
+                float2 kn[4], g2v[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 g2 = make_float2(gam[8 * m + 2 * e], gam[8 * m + 2 * e + 1]);
+                    g2v[e] = g2;
+                    const float2 E = ex2p(g2);
+                    const float2 G = mul2(E, fp[e]);   // e^{gamma}: both factors <= 1
+                    const float2 Kf = ex2p(make_float2(fc[e].x - g2.x, fc[e].y - g2.y));
+                    const float2 qn = mul2(bf2(wq[e]), nq2);
+                    kn[e] = mul2(bf2(wk[e]), nk2);
+                    o_qe[e] = pk2(mul2(qn, E));
+                    o_qg[e] = pk2(mul2(qn, G));
+                    o_ke[e] = pk2(mul2(mul2(kn[e], E), bt2));
+                    o_kg[e] = pk2(mul2(kn[e], G));
+                    o_kd[e] = pk2(mul2(kn[e], Kf));
+                }
+                st16(gsm + OFF_X + off_x(0, r, cg), o_qe[0], o_qe[1], o_qe[2], o_qe[3]);
+                st16(gsm + OFF_X + off_x(1, r, cg), o_ke[0], o_ke[1], o_ke[2], o_ke[3]);
+                st16(gsm + OFF_G + off_t(r, cg), o_kg[0], o_kg[1], o_kg[2], o_kg[3]);
+                st16(img + IMG_QG + off_r128(r, c0), o_qg[0], o_qg[1], o_qg[2], o_qg[3]);
+                st16(img + IMG_KD + off_r128(r, c0), o_kd[0], o_kd[1], o_kd[2], o_kd[3]);
+                for (int bp = band + 1; bp < 4; ++bp) {
+                    float2 fm[4];
+                    ld4f2(FT + lrow_m(bp, band) * 128 + c0, fm);
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        o[e] = pk2(mul2(kn[e], ex2p(make_float2(fm[e].x - g2v[e].x, fm[e].y - g2v[e].y))));
+                    st16(gsm + OFF_KH + off_kh(16 * pair_u(bp, band) + (r & 15), cg), o[0], o[1], o[2], o[3]);
+                }
+            }
+            fence_proxy_async();
+        } else {
             const float nq = fl.l2norm ? rsqrtf(NRMP[r] + NRMP[128 + r] + kL2Eps) : 1.f;
             const float nk = fl.l2norm ? rsqrtf(NRMP[64 + r] + NRMP[192 + r] + kL2Eps) : 1.f;
             const float2 nq2 = dup2(nq), nk2 = dup2(nk), bt2 = dup2(BET[r]);
@@ -599,10 +858,11 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
         }
         tc_fence_before();
         if (gbar_or(gi, bad)) break;
-        // ---- all ten band pairs: D[0,160) = [Q E; beta K E] (B rows)^T
+        // ---- all ten band pairs: D[0,160) = [Q E; beta K E] (B rows)^T (UNB: the six off-diagonal
+        // pairs, D[0,96))
         if (gt == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_bf16(128, 160, 0, 0, 0);
+            constexpr uint32_t id = idesc_bf16(128, UNB ? NPAIR_U : 160, 0, 0, 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
                 const uint64_t da = sdesc(gs + OFF_X + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024, kSwizzle128B);
@@ -631,12 +891,48 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 float v[16], v2[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) v[e] = 0.f;
-                if (j <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, j), v);
-                if (j <= b_lo + 1) {
-                    tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, j), v2);
-                    if (band == b_lo + 1) {
+                if constexpr (UNB) {
+                    // key bands before the row's band from the product, the own band's block
+                    // from the FP32 pairs
+                    if (j < b_lo) tmem_ld16(tl + TC_D + 16 * pair_u(b_lo, j), v);
+                    if (j < b_lo + 1) {
+                        tmem_ld16(tl + TC_D + 16 * pair_u(b_lo + 1, j), v2);
+                        if (band == b_lo + 1) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                            for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                        }
+                    }
+                    if (j == band) {
+                        const int o = (band * 16 + (r & 15)) * 16;
+                        if (qd < 2) {
+                            const uint4 d0 = ld16(gsm + OFF_DQ + 2 * o), d1 = ld16(gsm + OFF_DQ + 2 * o + 16);
+                            const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float2 f = bf2(dw[e]);
+                                v[2 * e] = f.x;
+                                v[2 * e + 1] = f.y;
+                            }
+                        } else {
+                            const float *dk = reinterpret_cast<const float *>(gsm + OFF_DK) + o;
+#pragma unroll
+                            for (int e4 = 0; e4 < 4; ++e4) {
+                                const float4 f = *reinterpret_cast<const float4 *>(dk + 4 * e4);
+                                v[4 * e4] = f.x;
+                                v[4 * e4 + 1] = f.y;
+                                v[4 * e4 + 2] = f.z;
+                                v[4 * e4 + 3] = f.w;
+                            }
+                        }
+                    }
+                } else {
+                    if (j <= b_lo) tmem_ld16(tl + TC_D + 16 * pair_of(b_lo, j), v);
+                    if (j <= b_lo + 1) {
+                        tmem_ld16(tl + TC_D + 16 * pair_of(b_lo + 1, j), v2);
+                        if (band == b_lo + 1) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) v[e] = v2[e];
+                        }
                     }
                 }
                 if (qd < 2) {

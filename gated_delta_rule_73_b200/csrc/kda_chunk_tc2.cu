@@ -92,13 +92,16 @@ struct PrepPrologue {
     const __nv_bfloat16 *raw_q, *raw_k, *raw_v;
     // U in the record as 16-column slabs (the sliced scan) rather than rows like W (the TMEM scan)
     int u_slabs;
+    // the gate map: Kimi Linear's g = -e^A softplus(z) instead of -5 sigmoid(e^A z)
+    int softplus;
 };
 
 #include "kda_chunk_prep.cuh"
 
 // The prep with two item groups per CTA (kda_chunk_prep.cuh): one 512-thread CTA per SM, its
 // TMEM split between the groups.  MEGA: CTA `cta` of `ncta` prep CTAs of the one-launch form.
-template <bool PRO, bool MEGA>
+// UNB: g without the -5 floor.
+template <bool PRO, bool MEGA, bool UNB>
 __device__ __forceinline__ void
 prep2_cta(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap *ptm_v, const CUtensorMap *ptm_g,
           const __nv_bfloat16 *beta, uint8_t *ws, int T, int H, int BH, KernelFlags fl, PrepPrologue pro,
@@ -118,7 +121,7 @@ prep2_cta(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap 
     // the scan kernel, launched with a programmatic dependency on this one, may be scheduled now
     if (!MEGA) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int gi = threadIdx.x / prep2::GT;
-    prep2_group<PRO, MEGA>(ptm_q, ptm_k, ptm_v, ptm_g, beta, ws, T, H, BH, fl, pro, gi,
+    prep2_group<PRO, MEGA, UNB>(ptm_q, ptm_k, ptm_v, ptm_g, beta, ws, T, H, BH, fl, pro, gi,
                            smem + gi * prep2::GROUP_STRIDE, tbase + 256u * gi, prep2::NG * cta + gi,
                            prep2::NG * ncta, flags, wait_limit);
     tc_fence_before();
@@ -126,13 +129,13 @@ prep2_cta(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMap 
     if (warp == 0) tmem_dealloc(tbase, 512);
 }
 
-template <bool PRO>
+template <bool PRO, bool UNB>
 __global__ void __launch_bounds__(prep2::NT, 1)
 chunk_prep2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                    const __nv_bfloat16 *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H, int BH,
                    KernelFlags fl, PrepPrologue pro, uint32_t wait_limit) {
-    prep2_cta<PRO, false>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x,
+    prep2_cta<PRO, false, UNB>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x,
                           (int)gridDim.x, nullptr, wait_limit);
 }
 
@@ -593,7 +596,7 @@ constexpr uint32_t mega2_smem_bytes() {
     return prep2::SMEM_BYTES > scan::Layout<NS>::SMEM_BYTES ? prep2::SMEM_BYTES : scan::Layout<NS>::SMEM_BYTES;
 }
 
-template <bool PRO, int NS>
+template <bool PRO, int NS, bool UNB>
 __global__ void __launch_bounds__(prep2::NT, 1)
 chunk_mega2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -604,7 +607,7 @@ chunk_mega2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if ((int)blockIdx.x < n_scan)
         mega_scan<NS>(ws, S0, out, S_T, T, H, fl.scale, (int)blockIdx.x, flags, BH, wait_limit);
     else
-        prep2_cta<PRO, true>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x - n_scan,
+        prep2_cta<PRO, true, UNB>(&tm_q, &tm_k, &tm_v, &tm_g, beta, ws, T, H, BH, fl, pro, (int)blockIdx.x - n_scan,
                              (int)gridDim.x - n_scan, flags, wait_limit);
 }
 
@@ -656,7 +659,7 @@ cudaError_t launch_chunk_tc2(const ChunkArgs &a, cudaStream_t st) {
     if (!make_map2(&mq, a.q, a.B, a.T, a.H) || !make_map2(&mk, a.k, a.B, a.T, a.H) ||
         !make_map2(&mv, a.v, a.B, a.T, a.H) || !make_map2(&mg, a.g, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0}, st);
+    return launch_split(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0}, st);
 }
 
 cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a, cudaStream_t st) {
@@ -668,7 +671,7 @@ cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a,
         return cudaErrorInvalidValue;
     return launch_split(a, mq, mk, mv, mz,
                         PrepPrologue{(const __nv_bfloat16 *)p.conv_w, p.A, p.beta_logit, (const __nv_bfloat16 *)p.q_pre,
-                                     (const __nv_bfloat16 *)p.k_pre, (const __nv_bfloat16 *)p.v_pre, 0},
+                                     (const __nv_bfloat16 *)p.k_pre, (const __nv_bfloat16 *)p.v_pre, 0, p.gate_softplus},
                         st);
 }
 
@@ -705,9 +708,10 @@ static cudaError_t launch_scan(const ChunkArgs &a, const uint8_t *ws, cudaStream
                               (const __nv_bfloat16 *)a.out_gate, a.norm_w, a.norm_eps);
 }
 
-// Per-(chunk, head) prep cost of one SM (cycles; two items in flight per SM) and the per-chunk
-// chain of the sliced scan at d = 128 on a B200 SM (measured).
-constexpr double kPrepItemCycles = 13300.0;
+// Per-(chunk, head) prep cost of one SM (cycles; two items in flight per SM; with the FP32
+// diagonal blocks of an unbounded gate) and the per-chunk chain of the sliced scan at d = 128 on
+// a B200 SM (measured).
+constexpr double kPrepItemCycles = 13300.0, kPrepItemCyclesUnb = 24800.0;
 static double scan_chunk_cycles(int ns) { return ns == 16 ? 2900.0 : ns == 32 ? 3000.0 : ns == 64 ? 3100.0 : 4900.0; }
 
 // Polls of a bounded wait before it gives up (kda_set_wait_limit; failure-handling tests only).
@@ -717,16 +721,17 @@ static uint32_t g_wait_limit = kWaitLimit;
 // launches are faster: prep on all SMs, then the TMEM scan, against the prep on the SMs the scan's
 // CTAs leave, overlapped with the sliced scan, plus one item of ramp.
 constexpr double kScan3ChunkCycles = 4100.0;   // the TMEM scan's chain, one CTA per sequence
-int mega_slice_width(int BH, int nch, int sms) {
+int mega_slice_width(int BH, int nch, int sms, bool unb) {
+    const double t_item = unb ? kPrepItemCyclesUnb : kPrepItemCycles;
     const double items = (double)BH * nch;
     const double waves = ceil((double)BH / sms);
-    const double two = ceil(items / sms) * kPrepItemCycles + waves * nch * kScan3ChunkCycles;
+    const double two = ceil(items / sms) * t_item + waves * nch * kScan3ChunkCycles;
     int best = 0;
     double best_t = 0.9 * two;
     for (int ns : {32, 64}) {
         const int n_scan = BH * (D / ns);
         if (n_scan > sms / 2) continue;
-        const double t = fmax(ceil(items / (sms - n_scan)) * kPrepItemCycles, nch * scan_chunk_cycles(ns)) + kPrepItemCycles;
+        const double t = fmax(ceil(items / (sms - n_scan)) * t_item, nch * scan_chunk_cycles(ns)) + t_item;
         if (t < best_t) {
             best = ns;
             best_t = t;
@@ -752,10 +757,10 @@ uint32_t set_wait_limit(uint32_t polls) {
 // The one-launch form: CTAs [0, n_scan) are sliced-scan CTAs, the rest prep CTAs of two item
 // groups, all resident at once (a cooperative launch; the scan CTAs wait for the records the
 // prep CTAs publish).
-template <bool PRO, int NS>
+template <bool PRO, int NS, bool UNB>
 static cudaError_t launch_mega(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, cudaStream_t st) {
-    auto k = chunk_mega2_kernel<PRO, NS>;
+    auto k = chunk_mega2_kernel<PRO, NS, UNB>;
     constexpr uint32_t smem = mega2_smem_bytes<NS>();
     static_assert(smem <= 232448, "shared memory budget");
     static_assert(scan::Layout<NS>::NT + 32 <= prep2::NT, "the scan's warps and the loader warp fit the prep's block");
@@ -803,20 +808,30 @@ static cudaError_t launch_scan3(const ChunkArgs &a, const uint8_t *ws, cudaStrea
 // The split form: few sequences take the one-launch form with value-column slices (its chain is
 // the shorter one there); otherwise the prep kernel, then the TMEM scan (one CTA per sequence),
 // or with the output epilogue the sliced scan with whole-row slices (it normalises rows in its
-// registers).  U's layout in the record follows the scan that reads it.
+// registers).  U's layout in the record follows the scan that reads it.  An unbounded gate
+// (a.exact_decay) takes the prep with FP32 diagonal blocks; the scans are the same.
+template <bool UNB>
+static cudaError_t launch_mega_any(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                                   const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, int ns,
+                                   cudaStream_t st) {
+    const bool p = pro.conv_w != nullptr;
+    return ns == 32 ? (p ? launch_mega<true, 32, UNB>(a, mq, mk, mv, mg, pro, st)
+                         : launch_mega<false, 32, UNB>(a, mq, mk, mv, mg, pro, st))
+                    : (p ? launch_mega<true, 64, UNB>(a, mq, mk, mv, mg, pro, st)
+                         : launch_mega<false, 64, UNB>(a, mq, mk, mv, mg, pro, st));
+}
+
 static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                 const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro,
                                 cudaStream_t st) {
-    const bool p = pro.conv_w != nullptr;
+    const bool p = pro.conv_w != nullptr, unb = a.exact_decay;
     const int nch = (a.T + C - 1) / C;
     if (!a.out_gate) {
-        const int ns = mega_slice_width(a.B * a.H, nch, num_sms());
+        const int ns = mega_slice_width(a.B * a.H, nch, num_sms(), unb);
         if (ns) {
             pro.u_slabs = 1;
-            cudaError_t e = ns == 32 ? (p ? launch_mega<true, 32>(a, mq, mk, mv, mg, pro, st)
-                                          : launch_mega<false, 32>(a, mq, mk, mv, mg, pro, st))
-                                     : (p ? launch_mega<true, 64>(a, mq, mk, mv, mg, pro, st)
-                                          : launch_mega<false, 64>(a, mq, mk, mv, mg, pro, st));
+            cudaError_t e = unb ? launch_mega_any<true>(a, mq, mk, mv, mg, pro, ns, st)
+                                : launch_mega_any<false>(a, mq, mk, mv, mg, pro, ns, st);
             if (e != cudaErrorCooperativeLaunchTooLarge) return e;
             (void)cudaGetLastError();   // not enough room to co-schedule: the two launches below
         }
@@ -824,7 +839,8 @@ static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const
     pro.u_slabs = a.out_gate ? 1 : 0;
     uint8_t *ws = (uint8_t *)a.workspace;
     const int nitems = nch * a.B * a.H;
-    auto prep_k = p ? chunk_prep2_kernel<true> : chunk_prep2_kernel<false>;
+    auto prep_k = p ? (unb ? chunk_prep2_kernel<true, true> : chunk_prep2_kernel<true, false>)
+                    : (unb ? chunk_prep2_kernel<false, true> : chunk_prep2_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep2::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     mark_launch(a, st);

@@ -439,15 +439,16 @@ def recurrent_step(q, k, v, g, beta, S, *, l2norm=True, complex_gate=False, scal
 
 
 def chunk_fwd_gated(q, k, v, g, beta, S0, out_gate, norm_weight=None, *, norm_eps=1e-5,
-                    l2norm=True, complex_gate=False, scale=1.0, fused=None, stream=None):
+                    l2norm=True, complex_gate=False, scale=1.0, fused=None, unbounded=False,
+                    stream=None):
     """Allocate and run ``kda_chunk_fwd_gated``; returns (out, S_T)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused)
+    kw = dict(l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused, unbounded=unbounded)
+    opts = make_opts(q.dtype, **kw)
     nbytes = kda_chunk_workspace_bytes(B, T, H, dk, dv, opts)
     workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
-    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale,
-                     workspace=workspace, fused=fused)
+    opts = make_opts(q.dtype, workspace=workspace, **kw)
     out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     kda_chunk_fwd_gated(q, k, v, g, beta, S0, out, S_T, out_gate, norm_weight, norm_eps, opts, stream)

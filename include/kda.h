@@ -81,12 +81,16 @@ enum {
                             cost model, from B*H and the device's SM count,
                             says is faster; KDA_FUSED | KDA_SPLIT is an error */
     KDA_UNBOUNDED_DECAY = 16u, /* g may lie anywhere in (-inf, 0]: no -5 floor.
-                            The bf16 dk = dv = 128 tensor-core forms need the
-                            floor (16 tokens of decay must stay inside e^-80,
-                            page "Kimi K3 模型结构（2）", Q&A on the -5 bound), so
-                            the chunk forward runs on the exact-FP32 chunk path
-                            instead (every decay factor taken pairwise,
-                            exponent <= 0).  Cannot be combined with
+                            The bounded tensor-core forms reference decay
+                            factors to 16-token band starts, which needs the
+                            floor (page "Kimi K3 模型结构（2）", Q&A on the -5
+                            bound).  With this flag the bf16 dk = dv = 128
+                            chunk forward takes the split form with the
+                            off-diagonal band pairs on the tensor cores (every
+                            factor one exponential of an exponent <= 0) and the
+                            diagonal 16 x 16 blocks as FP32 position pairs;
+                            with KDA_COMPLEX, fp32 data or d = 64 it takes the
+                            exact-FP32 chunk path.  Cannot be combined with
                             KDA_FUSED or KDA_SPLIT (KDA_ERR_ARG).  The decode
                             step is exact for any g and ignores the flag.   */
     KDA_GATE_SOFTPLUS = 32u /* prologue entry points: the Kimi Linear gate
@@ -201,7 +205,9 @@ int kda_recurrent_step(const void *q, const void *k, const void *v, const void *
  *   S0, out, S_T as in kda_chunk_fwd.
  * KDA_COMPLEX is not supported here (the pages define no signed-gate map).
  * KDA_GATE_SOFTPLUS selects the Kimi Linear gate g = -exp(A_h) * softplus(z)
- * (unbounded below) and the exact-FP32 chunk path with it.
+ * (unbounded below) and the unbounded chunk forward with it (KDA_UNBOUNDED_DECAY):
+ * for bf16 d = 128 the gate is computed inside the split form's prep, otherwise
+ * by the FP32 prologue ahead of the exact-FP32 chunk path.
  */
 int kda_chunk_fwd_prologue(const void *q_pre, const void *k_pre, const void *v_pre,
                            const void *conv_w, const void *z, const float *A,

@@ -209,9 +209,10 @@ def test_decode_prologue_rejects_bad_arguments_on_host(kda):
 
 @host_only
 def test_unbounded_decay_flags_on_host(kda):
-    """KDA_UNBOUNDED_DECAY / KDA_GATE_SOFTPLUS: the tensor-core forms cannot take a gate
-    without the -5 floor, so forcing one of them is an argument error; the softplus map has
-    no signed form; the workspace becomes the exact-FP32 path's (the same with either flag)."""
+    """KDA_UNBOUNDED_DECAY / KDA_GATE_SOFTPLUS: only the split tensor-core form takes a gate
+    without the -5 floor, so forcing a form is an argument error; the softplus map has no signed
+    form.  bf16 d = 128 keeps the split form's workspace (its prep forms the diagonal blocks in
+    FP32); with Complex-KDA, or fp32, the gate runs on the exact-FP32 path and its workspace."""
     import torch
     for fl in (kda.KDA_UNBOUNDED_DECAY, kda.KDA_GATE_SOFTPLUS):
         for forced in (kda.KDA_FUSED, kda.KDA_SPLIT):
@@ -221,13 +222,18 @@ def test_unbounded_decay_flags_on_host(kda):
     assert _call_chunk(kda, opts=o) == -1
     unb = kda.make_opts(torch.bfloat16, unbounded=True)
     sp = kda.make_opts(torch.bfloat16, gate_softplus=True)
+    bounded = kda.make_opts(torch.bfloat16)
+    unb_c = kda.make_opts(torch.bfloat16, unbounded=True, complex_gate=True)
     f32 = kda.make_opts(torch.float32)
+    split = kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, kda.make_opts(torch.bfloat16, fused=False))
     ref = kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, f32)
-    assert ref > 0
-    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, unb) == ref
-    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, sp) == ref
-    # the prologue with the softplus gate keeps FP32 intermediates ahead of that workspace
-    assert kda.kda_prologue_workspace_bytes(2, 130, 3, 128, 128, sp) > ref + 4 * 2 * 130 * 3 * 128 * 4
+    assert split > 0 and ref > 0 and split != ref
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, unb) == split
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, sp) == split
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, bounded) == split
+    assert kda.kda_chunk_workspace_bytes(2, 130, 3, 128, 128, unb_c) == ref
+    # the prologue with the softplus gate is fused into the split form's prep: no intermediates
+    assert kda.kda_prologue_workspace_bytes(2, 130, 3, 128, 128, sp) == split
     assert _call_chunk(kda, opts=unb) == -7                # still needs its workspace
 
 
