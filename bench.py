@@ -341,9 +341,36 @@ def rows_n1(K, flush, hbm_peak, rows):
         del gr, wsb, grads
         torch.cuda.empty_cache()
 
+        # Complex-KDA against KDA, forward + backward, at the shape of the CKDA review's Figure 5
+        # (BF16, 16 heads, dk = dv = 128, 32k tokens per step): context for the pages' 96-97 %
+        fb_ms = {}
+        for cplx in (False, True):
+            xc = W.chunk_inputs(1, 32768, 16, d, d, dtype=torch.bfloat16, seed=5, complex_gate=cplx)
+            gc = W.grad_inputs(1, 32768, 16, d, d, dtype=torch.bfloat16, seed=6)
+            ob = K.make_opts(torch.bfloat16, complex_gate=cplx)
+            wsc = torch.empty(K.kda_chunk_bwd_workspace_bytes(1, 32768, 16, d, d, ob), dtype=torch.uint8,
+                              device="cuda")
+            ff = lambda: K.chunk_fwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], xc["S0"],
+                                     complex_gate=cplx)
+            fbw = lambda: K.chunk_bwd(xc["q"], xc["k"], xc["v"], xc["g"], xc["beta"], xc["S0"], gc["dout"],
+                                      gc["dS_T"], complex_gate=cplx, workspace=wsc)
+            ff(); fbw()
+            torch.cuda.synchronize()
+            t_f = statistics.median(time_calls(ff, 3, flush))
+            t_b = statistics.median(time_calls(fbw, 3, flush))
+            fb_ms["ckda" if cplx else "kda"] = {"fwd_ms": t_f, "bwd_ms": t_b, "fwd_bwd_ms": t_f + t_b}
+            del xc, gc, wsc
+            torch.cuda.empty_cache()
+        fb_ms["ckda_over_kda_throughput_fwd_bwd"] = fb_ms["kda"]["fwd_bwd_ms"] / fb_ms["ckda"]["fwd_bwd_ms"]
+        fb_ms["ckda_over_kda_throughput_fwd"] = fb_ms["kda"]["fwd_ms"] / fb_ms["ckda"]["fwd_ms"]
+        fb_ms["note"] = ("B=1 T=32768 H=16 dk=dv=128 bf16, kda_chunk_fwd + kda_chunk_bwd (FP32 recurrent "
+                         "backward sweep); the pages report 96-97 % on H100 (context only)")
+        rows["complex_kda_fwd_bwd_T32768_H16"] = fb_ms
+
         # context parallelism over T, emulated on one GPU: the prefill sequence cut into 4
-        # segments; each segment's pair (two forward runs), the fold and the forward from the
-        # folded state, timed per piece (on R GPUs the ranks run their pieces side by side)
+        # segments; each segment's pair (one prep pass, two scans over its records), the fold and
+        # the segment's forward from the folded state (a scan over the same records), timed per
+        # piece (on R GPUs the ranks run their pieces side by side)
         R = 4
         Ts = Tp // R
         segs = [{n: x[n][:, r * Ts:(r + 1) * Ts].contiguous() for n in ("q", "k", "v", "g", "beta")}
@@ -363,13 +390,11 @@ def rows_n1(K, flush, hbm_peak, rows):
         fcomb = lambda: K.kda_affine_combine(Ms, Bs, R - 1, x["S0"], S_start)
         fcomb()
         ms_comb = statistics.median(time_calls(fcomb, 5, flush))
-        wsf = torch.empty(max(K.kda_chunk_workspace_bytes(Bp, Ts, Hp, d, d, o1), 16), dtype=torch.uint8,
-                          device="cuda")
-        of = K.make_opts(torch.bfloat16, workspace=wsf)
         outs = torch.empty((Bp, Ts, Hp, d), dtype=torch.bfloat16, device="cuda")
         Sseg = torch.empty((Bp, Hp, d, d), dtype=torch.float32, device="cuda")
-        fseg = lambda: K.kda_chunk_fwd(*(segs[R - 1][n] for n in ("q", "k", "v", "g", "beta")), S_start,
-                                       outs, Sseg, of)
+        # wsp holds the last segment's records (its pair was the last call on it)
+        fseg = lambda: K.kda_segment_forward(*(segs[R - 1][n] for n in ("q", "k", "v", "g", "beta")),
+                                             S_start, outs, Sseg, op)
         fseg()
         ms_seg = statistics.median(time_calls(fseg, 5, flush))
         pair_bytes = R * Bp * Hp * 2 * d * d * 4
@@ -377,9 +402,10 @@ def rows_n1(K, flush, hbm_peak, rows):
             "segment_T": Ts, "ms_segment_pair": ms_pair, "ms_fold": ms_comb, "ms_segment_forward": ms_seg,
             "ms_per_rank_compute": ms_pair + ms_comb + ms_seg, "ms_whole_sequence_one_gpu": ms_p,
             "all_gather_bytes": pair_bytes,
-            "note": "one GPU, pieces timed separately; per rank = pair + fold + forward of its 1024-token "
-                    "segment; the all-gather of the pairs (all_gather_bytes) is not timed here"}
-        del segs, wsp, Ms, Bs, S_start, wsf, outs, Sseg
+            "note": "one GPU, pieces timed separately; per rank = pair + fold of 3 pairs + the segment's "
+                    "forward over its 1024 tokens; the all-gather of the pairs (all_gather_bytes) is not "
+                    "timed here"}
+        del segs, wsp, Ms, Bs, S_start, outs, Sseg
         torch.cuda.empty_cache()
 
         # unbounded decay (Kimi Linear softplus gate) on the prefill shape: the split tensor-core

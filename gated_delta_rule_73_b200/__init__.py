@@ -15,6 +15,7 @@ _EXPORTS = (
     "kda_chunk_bwd", "kda_chunk_bwd_workspace_bytes", "chunk_bwd", "KDA_UNBOUNDED_DECAY",
     "KDA_GATE_SOFTPLUS", "kda_segment_pair", "kda_segment_pair_workspace_bytes",
     "kda_affine_combine", "segment_pair", "affine_combine", "kda_selftest_bounded_wait",
+    "kda_segment_forward", "segment_forward",
     "kda_device_status", "kda_set_wait_limit", "KDA_WAIT_LIMIT_DEFAULT",
     "status_string", "chunk_fwd", "recurrent_step", "chunk_fwd_prologue",
     "recurrent_step_prologue", "conv_state_from_prefill", "chunk_fwd_gated", "LIB_PATH",

@@ -5,10 +5,12 @@ tokens acts on the state as one affine pair S -> M S + B, and pairs compose in o
 rank r only needs the pairs of segments 0..r-1 to know the state its own segment starts
 from.  Per call, every rank
 
-  1. computes its segment's pair (M_r, B_r) with ``kda_segment_pair``   (two chunk passes),
+  1. computes its segment's pair (M_r, B_r) with ``kda_segment_pair``   (one prep pass, two
+     scans over its records),
   2. all-gathers the pairs of all ranks                                  (the one exchange),
   3. folds pairs 0..r-1 onto the sequence's start state S0 with ``kda_affine_combine``,
-  4. runs ``kda_chunk_fwd`` over its segment from that state, and
+  4. runs ``kda_segment_forward`` over its segment from that state       (a third scan over
+     the same records), and
   5. folds all pairs onto S0 for the final state of the whole sequence.
 
 Only step 2 crosses ranks (2 x 64 KiB per head and rank at d = 128, FP32).  The arithmetic
@@ -23,14 +25,25 @@ import torch.distributed as dist
 
 
 class LibraryOps:
-    """The three library calls the context-parallel forward is built from."""
+    """The library calls the context-parallel forward is built from.  The segment's workspace
+    (its chunk records) is kept from ``segment_pair`` for ``segment_forward``."""
 
     def __init__(self, **flags):
         self.flags = flags
+        self.workspace = None
 
     def segment_pair(self, q, k, v, g, beta):
         from . import kda
-        return kda.segment_pair(q, k, v, g, beta, **self.flags)
+        B, T, H, dk = q.shape
+        opts = kda.make_opts(q.dtype, **{n: f for n, f in self.flags.items() if n != "scale"})
+        nbytes = kda.kda_segment_pair_workspace_bytes(B, T, H, dk, v.shape[-1], opts)
+        self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+        return kda.segment_pair(q, k, v, g, beta, workspace=self.workspace,
+                                **{n: f for n, f in self.flags.items() if n != "scale"})
+
+    def segment_forward(self, q, k, v, g, beta, S0):
+        from . import kda
+        return kda.segment_forward(q, k, v, g, beta, S0, self.workspace, **self.flags)
 
     def affine_combine(self, Ms, Bs, n, S0):
         from . import kda
@@ -65,6 +78,6 @@ def chunk_fwd_context_parallel(q, k, v, g, beta, S0=None, *, group=None, ops=Non
     Ms = _all_gather(M, group)                       # [R, B, H, dk, dk]
     Bs = _all_gather(Bm, group)                      # [R, B, H, dk, dv]
     S_start = ops.affine_combine(Ms, Bs, rank, S0)
-    out, _ = ops.chunk_fwd(q, k, v, g, beta, S_start)
+    out, _ = ops.segment_forward(q, k, v, g, beta, S_start)
     S_T = ops.affine_combine(Ms, Bs, world, S0)
     return out, S_T, S_start

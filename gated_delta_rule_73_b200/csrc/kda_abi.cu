@@ -168,7 +168,7 @@ int check_dims(long long B, long long T, long long H, int dk, int dv) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 108; }
+int kda_abi_version(void) { return 109; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -238,6 +238,13 @@ static int chunk_fwd_impl(const void *q, const void *k, const void *v, const voi
 // Workspace of kda_segment_pair: a zero v [B,T,H,dk] and an identity S0 [B,H,dk,dk] for the
 // run that yields M, a scratch out [B,T,H,max(dk,dv)] both runs write, and the chunk
 // forward's own workspace (the larger of the two runs').
+// Split tensor-core form (bf16, d = 128): the chunk records (kept for kda_segment_forward),
+// then the identity start state of the M scan.
+static size_t segment_ws_tc(int B, int T, int H, int dk, size_t *eye_off) {
+    *eye_off = round_up(chunk_tc2_workspace_bytes(B, T, H), kAlignWs);
+    return *eye_off + (size_t)B * H * dk * dk * 4;
+}
+
 static size_t segment_ws_parts(const kda_opts &o, int B, int T, int H, int dk, int dv, size_t *off) {
     const size_t e = o.dtype == KDA_BF16 ? 2 : 4;
     const size_t rows = (size_t)B * T * H;
@@ -257,6 +264,7 @@ size_t kda_segment_pair_workspace_bytes(int B, int T, int H, int dk, int dv, con
     if (check_opts(o) != KDA_OK || check_dims(B, T, H, dk, dv) != KDA_OK) return 0;
     if (B <= 0 || T <= 0 || H <= 0) return 0;
     size_t off[4];
+    if (use_tc(o, dk, dv)) return segment_ws_tc(B, T, H, dk, off);
     return segment_ws_parts(o, B, T, H, dk, dv, off);
 }
 
@@ -287,6 +295,27 @@ int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_ALIGN;
     size_t off[4];
+    if (use_tc(o, dk, dv)) {
+        // one prep pass (its records stay in the workspace for kda_segment_forward), then the
+        // scans from S0 = 0 (B) and from S0 = I with U taken as zero (M) side by side
+        const size_t need = segment_ws_tc(B, T, H, dk, off);
+        if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
+        float *eye = (float *)((char *)o.workspace + off[0]);
+        if (launch_identity(eye, (long long)B * H, dk, stream) != cudaSuccess) return KDA_ERR_CUDA;
+        ChunkArgs a;
+        memset(&a, 0, sizeof(a));
+        a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+        a.t_qkv = a.t_g = a.t_beta = a.t_out = Elt::BF16;
+        a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+        a.fl = kflags(o);
+        a.workspace = o.workspace; a.workspace_bytes = need;
+        a.exact_decay = unbounded(o);
+        int launches = 0;
+        a.launch_idx = &launches;
+        cudaError_t e = launch_segment_pair_tc2(a, eye, M_out, B_out, stream);
+        if (e == cudaErrorInvalidValue) return KDA_ERR_UNSUPPORTED;
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
     const size_t need = segment_ws_parts(o, B, T, H, dk, dv, off);
     if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
     char *ws = (char *)o.workspace;
@@ -308,6 +337,44 @@ int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
     // M: from S0 = I with v = 0 (column i of the final state is M e_i)
     return chunk_fwd_impl(q, k, zv, g, beta, eye, scratch_out, M_out, nullptr, nullptr, 0.f, B, T, H,
                           dk, dk, &oc, stream);
+}
+
+int kda_segment_forward(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                        const float *S0, void *out, float *S_T, int B, int T, int H, int dk, int dv,
+                        const kda_opts *opts, cudaStream_t stream) {
+    const kda_opts o = resolve(opts);
+    int s = check_opts(o);
+    if (s != KDA_OK) return s;
+    if ((s = check_dims(B, T, H, dk, dv)) != KDA_OK) return s;
+    if (!use_tc(o, dk, dv))   // no records on this path: the whole chunk forward
+        return chunk_fwd_impl(q, k, v, g, beta, S0, out, S_T, nullptr, nullptr, 0.f, B, T, H, dk, dv, opts,
+                              stream);
+    if (B == 0 || H == 0) return KDA_OK;
+    if (T == 0) {
+        if (!aligned16(S0) || !aligned16(S_T)) return KDA_ERR_ALIGN;
+        return finish_identity(S0, S_T, B, H, dk, dv, stream);
+    }
+    if (!out) return KDA_ERR_ARG;
+    const void *ptrs[] = {S0, out, S_T, o.workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_ALIGN;
+    size_t eye_off;
+    const size_t need = segment_ws_tc(B, T, H, dk, &eye_off);
+    if (!o.workspace || o.workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    ChunkArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+    a.t_qkv = a.t_g = a.t_beta = a.t_out = Elt::BF16;
+    a.S0 = S0; a.out = out; a.S_T = S_T;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+    a.fl = kflags(o);
+    a.workspace = o.workspace; a.workspace_bytes = need;
+    a.events = o.events; a.n_events = o.n_events;
+    int launches = 0;
+    a.launch_idx = &launches;
+    cudaError_t e = launch_segment_scan_tc2(a, stream);
+    if (e == cudaSuccess && o.events && launches < o.n_events) cudaEventRecord(o.events[launches], stream);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 int kda_affine_combine(const float *M, const float *Bp, int n, const float *S0, float *S_out, int BH,

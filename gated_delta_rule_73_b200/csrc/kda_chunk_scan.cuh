@@ -46,11 +46,13 @@ struct alignas(8) Scan3Bars {
     int issued[scan3::NSTG + 5];   // completions issued per barrier (drain on give-up)
 };
 
+// zero_u: the chunks' U taken as zero (the segment map's linear part: S -> M S from S0 = I);
+// out == nullptr: no outputs (their products are skipped), only the final state.
 template <bool MEGA>
 __device__ __forceinline__ void
 scan3_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bfloat16 *__restrict__ out,
            float *__restrict__ S_T, int T, int H, float scale, int cta, const int *__restrict__ flags, int nseq,
-           uint32_t poll_limit) {
+           uint32_t poll_limit, bool zero_u = false) {
     using namespace scan3;
     extern __shared__ uint8_t smem_raw[];
     __shared__ Scan3Bars sh;
@@ -194,7 +196,7 @@ scan3_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bf
             if (!wait(bar_mO(buf), (uint32_t)(ch >> 1) & 1u)) break;
             __syncwarp();
             tc_fence_after();
-            {
+            if (out) {
                 float o[32];
                 tmem_ld32(tl + tdp + 64 + 32 * hh, o);
                 __nv_bfloat16 *dst = out + (((size_t)b * T + t0 + 32 * hh) * H + h) * D + j;
@@ -231,7 +233,7 @@ scan3_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bf
             if (!wait(bar_st(sg), (uint32_t)(ch / NSTG) & 1u)) break;          // the record is in
             if (ch >= 2 && !wait(bar_bE(buf), (uint32_t)((ch - 2) >> 1) & 1u)) break;   // buffer emitted
             tc_fence_after();
-            if (lane == 0) {
+            if (lane == 0 && !zero_u) {
                 // U^T into the V~^T half: four M = 128, N = 16, K = 16 identity products
                 constexpr uint32_t id_u = idesc_bf16(128, 16, 1, 0, 0);
 #pragma unroll
@@ -241,16 +243,19 @@ scan3_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bf
             if (!wait(b_bS, (uint32_t)ch & 1u)) break;                          // S(ch) is in place
             tc_fence_after();
             if (lane == 0) {
-                // V~^T = U^T - S^T W^T (negated A), then O^T = S^T (Q Gamma)^T
+                // V~^T = U^T - S^T W^T (negated A; zero_u: -S^T W^T), then O^T = S^T (Q Gamma)^T
                 constexpr uint32_t id_p = idesc_bf16(128, 64, 0, 0, 1);
                 constexpr uint32_t id_o = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mma_ts(tdp, tbase + TS_B + 8 * k, at(dK, st + IMG_W + 256 * k), id_p, 1);
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tdp, tbase + TS_B + 8 * k, at(dK, st + IMG_W + 256 * k), id_p, !zero_u || k > 0);
                 mma_commit(bar_mP(buf));
                 ++sh.issued[NSTG + buf];
+                if (out) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ts(tdp + 64, tbase + TS_B + 8 * k, at(dK, st + IMG_QG + 256 * k), id_o, k > 0);
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(tdp + 64, tbase + TS_B + 8 * k, at(dK, st + IMG_QG + 256 * k), id_o, k > 0);
+                }
             }
             __syncwarp();
             // the stage of chunk ch - 1 is free once its O products are done and its sigma_C has
@@ -270,8 +275,11 @@ scan3_body(const uint8_t *__restrict__ ws, const float *__restrict__ S0, __nv_bf
                 for (int k = 0; k < 4; ++k) mma_ts(tbase + TS_S, tbase + TS_V + 8 * k, at(dMN, st + IMG_KD + 4096 * k), id_s, k > 0);
                 mma_commit(b_mS);
                 ++sh.issued[NSTG + 2];
+                if (out) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) mma_ts(tdp + 64, tbase + TS_V + 8 * k, at(dK64, st + IMG_AQK + 256 * k), id_q, 1);
+                    for (int k = 0; k < 4; ++k)
+                        mma_ts(tdp + 64, tbase + TS_V + 8 * k, at(dK64, st + IMG_AQK + 256 * k), id_q, 1);
+                }
                 mma_commit(bar_mO(buf));
                 ++sh.issued[NSTG + 3 + buf];
             }

@@ -570,6 +570,19 @@ chunk_scan3_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
     scan3_body<false>(ws, S0, out, S_T, T, H, scale, (int)blockIdx.x, nullptr, 0, kWaitLimit);
 }
 
+// The affine pair of a segment from its records (kda_segment_pair): CTAs [0, BH) run the scan
+// from S0 = 0 (the final state is B), CTAs [BH, 2 BH) from S0 = I with U taken as zero (the
+// final state is M); no outputs.
+__global__ void __launch_bounds__(scan3::NT, 1)
+chunk_scan3_pair_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ eye, float *__restrict__ B_out,
+                        float *__restrict__ M_out, int T, int H, int BH) {
+    const int cta = (int)blockIdx.x, bh = cta % BH;
+    if (cta < BH)
+        scan3_body<false>(ws, nullptr, nullptr, B_out, T, H, 1.f, bh, nullptr, 0, kWaitLimit, false);
+    else
+        scan3_body<false>(ws, eye, nullptr, M_out, T, H, 1.f, bh, nullptr, 0, kWaitLimit, true);
+}
+
 template <int NS, bool GATED>
 __global__ void __launch_bounds__(scan::Layout<NS>::NT, 1)
 chunk_scan_tc_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ S0,
@@ -810,6 +823,24 @@ static cudaError_t launch_scan3(const ChunkArgs &a, const uint8_t *ws, cudaStrea
 // or with the output epilogue the sliced scan with whole-row slices (it normalises rows in its
 // registers).  U's layout in the record follows the scan that reads it.  An unbounded gate
 // (a.exact_decay) takes the prep with FP32 diagonal blocks; the scans are the same.
+// The prep kernel over every (chunk, head) item: records into a.workspace (U as rows unless
+// pro.u_slabs), unbounded prep when a.exact_decay.
+static cudaError_t launch_prep2(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                                const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, cudaStream_t st) {
+    const bool p = pro.conv_w != nullptr, unb = a.exact_decay;
+    const int nitems = ((a.T + C - 1) / C) * a.B * a.H;
+    auto prep_k = p ? (unb ? chunk_prep2_kernel<true, true> : chunk_prep2_kernel<true, false>)
+                    : (unb ? chunk_prep2_kernel<false, true> : chunk_prep2_kernel<false, false>);
+    cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep2::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    mark_launch(a, st);
+    const int ctas = std::min((nitems + prep2::NG - 1) / prep2::NG, num_sms());
+    prep_k<<<(unsigned)ctas, prep2::NT, prep2::SMEM_BYTES, st>>>(mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta,
+                                                                (uint8_t *)a.workspace, a.T, a.H, a.B * a.H, a.fl,
+                                                                pro, g_wait_limit);
+    return cudaGetLastError();
+}
+
 template <bool UNB>
 static cudaError_t launch_mega_any(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                                    const CUtensorMap &mv, const CUtensorMap &mg, PrepPrologue pro, int ns,
@@ -837,21 +868,47 @@ static cudaError_t launch_split(const ChunkArgs &a, const CUtensorMap &mq, const
         }
     }
     pro.u_slabs = a.out_gate ? 1 : 0;
+    cudaError_t e = launch_prep2(a, mq, mk, mv, mg, pro, st);
+    if (e != cudaSuccess) return e;
+    mark_launch(a, st);
     uint8_t *ws = (uint8_t *)a.workspace;
-    const int nitems = nch * a.B * a.H;
-    auto prep_k = p ? (unb ? chunk_prep2_kernel<true, true> : chunk_prep2_kernel<true, false>)
-                    : (unb ? chunk_prep2_kernel<false, true> : chunk_prep2_kernel<false, false>);
-    cudaError_t e = cudaFuncSetAttribute(prep_k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep2::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    mark_launch(a, st);
-    const int ctas = std::min((nitems + prep2::NG - 1) / prep2::NG, num_sms());
-    prep_k<<<(unsigned)ctas, prep2::NT, prep2::SMEM_BYTES, st>>>(mq, mk, mv, mg, (const __nv_bfloat16 *)a.beta, ws,
-                                                                a.T, a.H, a.B * a.H, a.fl, pro, g_wait_limit);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    mark_launch(a, st);
     if (a.out_gate) return launch_scan<D, true>(a, ws, st);
     return launch_scan3(a, ws, st);
+}
+
+// kda_segment_pair on the split form: the segment's records, then its two scans (B from S0 = 0,
+// M from S0 = I with U taken as zero) side by side in one launch.  The records stay in the
+// workspace for kda_segment_forward.
+cudaError_t launch_segment_pair_tc2(const ChunkArgs &a, const float *eye, float *M_out, float *B_out,
+                                    cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mg;
+    if (!make_map2(&mq, a.q, a.B, a.T, a.H) || !make_map2(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map2(&mv, a.v, a.B, a.T, a.H) || !make_map2(&mg, a.g, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = launch_prep2(a, mq, mk, mv, mg, PrepPrologue{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0}, st);
+    if (e != cudaSuccess) return e;
+    auto k = chunk_scan3_pair_kernel;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan3::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * a.B * a.H));
+    cfg.blockDim = dim3(scan3::NT);
+    cfg.dynamicSmemBytes = scan3::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    mark_launch(a, st);
+    return cudaLaunchKernelEx(&cfg, k, (const uint8_t *)a.workspace, eye, B_out, M_out, a.T, a.H, a.B * a.H);
+}
+
+// kda_segment_forward on the split form: the scan alone, from S0 over the records
+// kda_segment_pair left in the workspace.
+cudaError_t launch_segment_scan_tc2(const ChunkArgs &a, cudaStream_t st) {
+    mark_launch(a, st);
+    return launch_scan3(a, (const uint8_t *)a.workspace, st);
 }
 
 }  // namespace kda

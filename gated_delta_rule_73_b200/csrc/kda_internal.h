@@ -88,6 +88,13 @@ uint32_t set_wait_limit(uint32_t polls);
 // q, k, v, z tiles with a 3-row halo and applies the short convolution, SiLU, the gate and
 // beta = sigmoid(logit) on chip.  Uses a.out, a.S0, a.S_T, sizes, flags, workspace, events.
 cudaError_t launch_chunk_tc2_prologue(const PrologueArgs &p, const ChunkArgs &a, cudaStream_t st);
+// The segment pair on the split form (kda_segment_pair): prep records into a.workspace, then the
+// scans from S0 = 0 (B_out) and from S0 = eye with U taken as zero (M_out) in one launch.
+cudaError_t launch_segment_pair_tc2(const ChunkArgs &a, const float *eye, float *M_out, float *B_out,
+                                    cudaStream_t st);
+// The scan alone from a.S0 over the records a preceding launch_segment_pair_tc2 left in
+// a.workspace (kda_segment_forward).
+cudaError_t launch_segment_scan_tc2(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_chunk_ref(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t st);
 

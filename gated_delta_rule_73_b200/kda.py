@@ -66,6 +66,8 @@ def _load():
     lib.kda_segment_pair.restype = ip
     lib.kda_segment_pair_workspace_bytes.argtypes = [ip] * 5 + [op]
     lib.kda_segment_pair_workspace_bytes.restype = sz
+    lib.kda_segment_forward.argtypes = [vp] * 8 + [ip] * 5 + [op, vp]
+    lib.kda_segment_forward.restype = ip
     lib.kda_affine_combine.argtypes = [vp, vp, ip, vp, vp, ip, ip, ip, vp]
     lib.kda_affine_combine.restype = ip
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
@@ -226,6 +228,22 @@ def kda_segment_pair(q, k, v, g, beta, M_out, B_out, opts: kda_opts, stream=None
     st = _lib.kda_segment_pair(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
     if st != 0:
         raise KdaError("kda_segment_pair", st)
+
+
+def kda_segment_forward(q, k, v, g, beta, S0, out, S_T, opts: kda_opts, stream=None) -> None:
+    """Call ``kda_segment_forward``: the segment's forward from S0 over the records a preceding
+    ``kda_segment_pair`` left in ``opts.workspace`` (same inputs and workspace)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _shapes(k=(k, q.shape), g=(g, q.shape), v=(v, (B, T, H, dv)), beta=(beta, (B, T, H)),
+            S0=(S0, (B, H, dk, dv)), out=(out, (B, T, H, dv)), S_T=(S_T, (B, H, dk, dv)))
+    args = [_ptr(q, "q", dt), _ptr(k, "k", dt), _ptr(v, "v", dt), _ptr(g, "g", dt),
+            _ptr(beta, "beta", dt), _ptr(S0, "S0", torch.float32), _ptr(out, "out", dt),
+            _ptr(S_T, "S_T", torch.float32)]
+    st = _lib.kda_segment_forward(*args, B, T, H, dk, dv, ctypes.byref(opts), _stream(stream))
+    if st != 0:
+        raise KdaError("kda_segment_forward", st)
 
 
 def kda_affine_combine(M, Bp, n, S0, S_out, stream=None) -> None:
@@ -407,17 +425,36 @@ def chunk_bwd(q, k, v, g, beta, S0, dout, dS_T=None, *, l2norm=True, complex_gat
 
 
 def segment_pair(q, k, v, g, beta, *, l2norm=True, complex_gate=False, fused=None,
-                 unbounded=False, stream=None):
-    """Allocate and run ``kda_segment_pair``; returns (M, B)."""
+                 unbounded=False, workspace=None, stream=None):
+    """Run ``kda_segment_pair`` (workspace allocated unless given; pass the same one to
+    ``segment_forward`` afterwards); returns (M, B)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     kw = dict(l2norm=l2norm, complex_gate=complex_gate, fused=fused, unbounded=unbounded)
-    nbytes = kda_segment_pair_workspace_bytes(B, T, H, dk, dv, make_opts(q.dtype, **kw))
-    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    ws = workspace
+    if ws is None:
+        nbytes = kda_segment_pair_workspace_bytes(B, T, H, dk, dv, make_opts(q.dtype, **kw))
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     M = torch.empty((B, H, dk, dk), dtype=torch.float32, device=q.device)
     Bm = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     kda_segment_pair(q, k, v, g, beta, M, Bm, make_opts(q.dtype, workspace=ws, **kw), stream)
     return M, Bm
+
+
+def segment_forward(q, k, v, g, beta, S0, workspace, *, l2norm=True, complex_gate=False, scale=1.0,
+                    fused=None, unbounded=False, out=None, S_T=None, stream=None):
+    """Run ``kda_segment_forward`` with the workspace a ``segment_pair`` call on the same inputs
+    filled; returns (out, S_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    opts = make_opts(q.dtype, l2norm=l2norm, complex_gate=complex_gate, scale=scale, fused=fused,
+                     unbounded=unbounded, workspace=workspace)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    kda_segment_forward(q, k, v, g, beta, S0, out, S_T, opts, stream)
+    return out, S_T
 
 
 def affine_combine(Ms, Bs, n, S0=None, *, out=None, stream=None):

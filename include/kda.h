@@ -334,18 +334,36 @@ size_t kda_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv,
  *   M_out [B,H,dk,dk] FP32   M = T_T ... T_1   (the final state from S0 = I, v = 0)
  *   B_out [B,H,dk,dv] FP32   B = the final state from S0 = 0
  *
- * by two runs of the chunk forward (same paths, flags and tolerances as
- * kda_chunk_fwd).  opts->workspace must hold kda_segment_pair_workspace_bytes(...):
- * a zero v, the identity start state, a scratch output and the chunk workspace.
- * T == 0 gives the identity pair (I, 0).
+ * For bf16 dk = dv = 128 (the split tensor-core form, any gate it takes) one prep pass
+ * writes the segment's chunk records into opts->workspace and two scans over them run
+ * side by side: B from S0 = 0, M from S0 = I with the chunks' U taken as zero (the state's
+ * columns evolve independently, so column i is M e_i).  The records stay in the workspace
+ * for kda_segment_forward.  Otherwise (fp32, d = 64, Complex-KDA with an unbounded gate)
+ * it runs the chunk forward twice, the second time from S0 = I with v = 0.  Same flags
+ * and tolerances as kda_chunk_fwd.  opts->workspace must hold
+ * kda_segment_pair_workspace_bytes(...).  T == 0 gives the identity pair (I, 0).
  */
 int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
                      const void *beta, float *M_out, float *B_out, int B, int T, int H,
                      int dk, int dv, const kda_opts *opts, cudaStream_t stream);
 
-/* Workspace bytes kda_segment_pair needs. */
+/* Workspace bytes kda_segment_pair (and kda_segment_forward after it) needs. */
 size_t kda_segment_pair_workspace_bytes(int B, int T, int H, int dk, int dv,
                                         const kda_opts *opts);
+
+/*
+ * kda_segment_forward -- the segment's chunk forward from a start state S0 (the fold of the
+ * earlier segments' pairs, kda_affine_combine), after kda_segment_pair on the SAME inputs with
+ * the SAME opts (flags and workspace, untouched in between).  Same page and section.
+ *
+ * Arguments as kda_chunk_fwd.  On the split tensor-core form (bf16, dk = dv = 128) only the
+ * scan runs, over the records kda_segment_pair left in opts->workspace (the inputs are not
+ * read); otherwise this is kda_chunk_fwd (opts->workspace large enough for it: a
+ * kda_segment_pair workspace is).  The result equals kda_chunk_fwd from S0 up to rounding.
+ */
+int kda_segment_forward(const void *q, const void *k, const void *v, const void *g,
+                        const void *beta, const float *S0, void *out, float *S_T, int B, int T,
+                        int H, int dk, int dv, const kda_opts *opts, cudaStream_t stream);
 
 /*
  * kda_affine_combine -- fold the first n segment pairs onto a start state, in order:
@@ -406,7 +424,7 @@ const char *kda_status_string(int status);
 /* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
    1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd;
    1.6: kda_segment_pair, kda_affine_combine; 1.7: kda_selftest_bounded_wait;
-   1.8: kda_device_status, kda_set_wait_limit). */
+   1.8: kda_device_status, kda_set_wait_limit; 1.9: kda_segment_forward). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 108   # 1.8: kda_device_status, kda_set_wait_limit
+    assert kda.kda_abi_version() == 109   # 1.9: kda_segment_forward
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"

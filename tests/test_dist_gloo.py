@@ -97,7 +97,7 @@ def _cp_worker(rank, world, port, q, cuts):
             s0 = None if S0 is None else S0.double().numpy()
             return torch.from_numpy(oracle.affine_combine_np(Ms[:n].numpy(), Bs[:n].numpy(), s0))
 
-        def chunk_fwd(self, q, k, v, g, beta, S0):
+        def segment_forward(self, q, k, v, g, beta, S0):
             a = [x.double().numpy() for x in (q, k, v, g, beta)]
             o, s = oracle.recurrence_c(*a, S0.numpy())
             return torch.from_numpy(o), torch.from_numpy(s)

@@ -52,6 +52,36 @@ def test_segment_pair(K, T, d, dtype):
     assert rel_err(f64(Ms), ref_M) <= tol_for(dtype)
 
 
+def _seg_workspace(K, q, **flags):
+    B, T, H, d = q.shape
+    n = K.kda_segment_pair_workspace_bytes(B, T, H, d, d, K.make_opts(q.dtype, **flags))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+
+
+@pytest.mark.parametrize("kind", ["bf16", "complex", "unbounded", "fp32-d64"])
+def test_segment_forward_from_records(K, kind):
+    """kda_segment_forward after kda_segment_pair on the same inputs and workspace: the scan
+    alone over the pair's records (bf16 d=128, Complex-KDA, the unbounded gate) or the whole
+    chunk forward (fp32 d=64), from a given start state; equal to the oracle from that state,
+    and the pair itself still right (M S0 + B = the final state)."""
+    d, dtype = (64, torch.float32) if kind == "fp32-d64" else (128, torch.bfloat16)
+    flags = dict(complex_gate=kind == "complex", unbounded=kind == "unbounded")
+    x = W.chunk_inputs(2, 200, 3, d, d, dtype=dtype, seed=820, complex_gate=flags["complex_gate"],
+                       gate="softplus" if flags["unbounded"] else "bounded")
+    c = {n: (None if x[n] is None else cuda(x[n])) for n in x}
+    ws = _seg_workspace(K, c["q"], **flags)
+    args = [c[n] for n in ("q", "k", "v", "g", "beta")]
+    M, Bm = K.segment_pair(*args, workspace=ws, **flags)
+    out, S_T = K.segment_forward(*args, c["S0"], ws, **flags)
+    torch.cuda.synchronize()
+    a = [f64(x[n]) for n in ("q", "k", "v", "g", "beta")]
+    ref_o, ref_s = oracle.recurrence_c(*a, f64(x["S0"]), complex_gate=flags["complex_gate"])
+    tol = tol_for(dtype)
+    assert rel_err(f64(out), ref_o) <= tol and rel_err(f64(S_T), ref_s) <= tol
+    got_ST = np.einsum("bhij,bhjk->bhik", f64(M), f64(x["S0"])) + f64(Bm)
+    assert rel_err(got_ST, ref_s) <= tol
+
+
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 128), (128, 64)])
 def test_affine_combine(K, dk, dv):
     gen = torch.Generator().manual_seed(dk + dv)
@@ -81,13 +111,15 @@ def test_split_sequence_emulated(K, cuts):
     c = {n: cuda(x[n]) for n in x}
     segs = [(a, b) for a, b in zip(cuts[:-1], cuts[1:])]
     sl = lambda n, a, b: c[n][:, a:b].contiguous()
-    pairs = [K.segment_pair(*(sl(n, a, b) for n in ("q", "k", "v", "g", "beta"))) for a, b in segs]
+    wss = [_seg_workspace(K, sl("q", a, b)) for a, b in segs]
+    pairs = [K.segment_pair(*(sl(n, a, b) for n in ("q", "k", "v", "g", "beta")), workspace=ws)
+             for (a, b), ws in zip(segs, wss)]
     Ms = torch.stack([p[0] for p in pairs])
     Bs = torch.stack([p[1] for p in pairs])
     outs = []
     for r, (a, b) in enumerate(segs):
         S_start = K.affine_combine(Ms, Bs, r, c["S0"])
-        o, _ = K.chunk_fwd(*(sl(n, a, b) for n in ("q", "k", "v", "g", "beta")), S_start)
+        o, _ = K.segment_forward(*(sl(n, a, b) for n in ("q", "k", "v", "g", "beta")), S_start, wss[r])
         outs.append(o)
     S_T = K.affine_combine(Ms, Bs, len(segs), c["S0"])
     torch.cuda.synchronize()
