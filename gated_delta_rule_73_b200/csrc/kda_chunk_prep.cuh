@@ -954,40 +954,39 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                     }
                 }
             }
+            if (gw == 2 || gw == 7) {
+                __syncwarp();   // this warp's own A_kk^T rows
+                const int blk = (gw == 2 ? 0 : 2) + (lane >> 4), base = 16 * blk, j = lane & 15;
+                float x[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int i = 0; i < 15; ++i) {
+                    const float xi = x[i];
+                    const float *col = AKT + (base + i) * AS + base;   // A[base + rr][base + i] over rr
+#pragma unroll
+                    for (int r4 = ((i + 1) >> 2) << 2; r4 < 16; r4 += 4) {   // rows rr <= i hold 0
+                        const float4 av = *reinterpret_cast<const float4 *>(col + r4);
+                        x[r4] = fmaf(-av.x, xi, x[r4]);
+                        x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
+                        x[r4 + 2] = fmaf(-av.z, xi, x[r4 + 2]);
+                        x[r4 + 3] = fmaf(-av.w, xi, x[r4 + 3]);
+                    }
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) TMF[(base + rr) * AS + base + j] = x[rr];
+                if ((blk & 1) == 0) {   // the zero upper-right quarter of each 32-block's T
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) TMF[(base + rr) * AS + base + 16 + j] = 0.f;
+                }
+            }
         }
         tc_fence_before();
         if (gbar_or(gi, bad)) break;
 
         // ---- Tm = (I + A_kk)^{-1} in FP32 by 32 x 32 blocks [T1 0; T21 T2]: the 16 x 16 diagonal
-        // blocks D_b by column sweeps (lane = column, two blocks per warp, x_i final once the rows
-        // above are done, then x_r -= A[r][i] x_i for r > i); per 32-block Z = A10 D0, X = -D1 Z;
+        // blocks D_b were swept at the end of the readout; per 32-block Z = A10 D0, X = -D1 Z;
         // then Y = A21 T1, T21 = -T2 Y.  TMF holds T (rows 0-31 hold Z, then Y, in columns 32-63).
-        if (gw < 2) {
-            const int blk = 2 * gw + (lane >> 4), base = 16 * blk, j = lane & 15;
-            float x[16];
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int i = 0; i < 15; ++i) {
-                const float xi = x[i];
-                const float *col = AKT + (base + i) * AS + base;   // A[base + rr][base + i] over rr
-#pragma unroll
-                for (int r4 = ((i + 1) >> 2) << 2; r4 < 16; r4 += 4) {   // rows rr <= i hold 0
-                    const float4 av = *reinterpret_cast<const float4 *>(col + r4);
-                    x[r4] = fmaf(-av.x, xi, x[r4]);
-                    x[r4 + 1] = fmaf(-av.y, xi, x[r4 + 1]);
-                    x[r4 + 2] = fmaf(-av.z, xi, x[r4 + 2]);
-                    x[r4 + 3] = fmaf(-av.w, xi, x[r4 + 3]);
-                }
-            }
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) TMF[(base + rr) * AS + base + j] = x[rr];
-            if ((blk & 1) == 0) {   // the zero upper-right quarter of each 32-block's T
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) TMF[(base + rr) * AS + base + 16 + j] = 0.f;
-            }
-        }
-        gbar(gi);
         // Z = A10 D0 per 32-block hb (warps 0-3: block hb = gw >> 1, columns 8 (gw & 1) .. + 7;
         // 2 x 2 tiles: rows 2 rp, 2 rp + 1, columns 2 cp, 2 cp + 1)
         if (gw < 4) {
