@@ -761,7 +761,7 @@ def run_ours(args, ws, rank, local):
     return 0
 
 
-CASES = ("prefill", "decode", "sweep", "ckda", "bwd", "sweep_plain")
+CASES = ("prefill", "decode", "sweep", "ckda", "bwd", "sweep_plain", "softplus")
 
 # Kernels of kda_chunk_fwd_prologue on the sweep workload (B*H = 96 takes the split form: the
 # two-group prep with the fused prologue, then the TMEM scan) by launches per call, and the DRAM
@@ -775,6 +775,7 @@ def run_case(args):
     """Run one workload's call a few times and exit (a small case for ncu captures):
     prefill = B=1 T=4096 H=16; decode = N=64 H=96 (800 MB of state);
     sweep = prologue path at T=2048 H=96; sweep_plain = kda_chunk_fwd at B=1 T=2048 H=96;
+    softplus = kda_chunk_fwd with the unbounded (softplus) gate at B=1 T=2048 H=96;
     ckda = B=2 T=8192 H=32 signed gate; bwd = kda_chunk_bwd at B=1 T=1024 H=16."""
     import gated_delta_rule_73_b200 as K
     torch.cuda.set_device(0)
@@ -800,6 +801,9 @@ def run_case(args):
     elif args.case == "sweep_plain":
         x = W.chunk_inputs(1, 2048, 96, d, d, dtype=torch.bfloat16, seed=0)
         fn = lambda: K.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], fused=False)
+    elif args.case == "softplus":
+        x = W.chunk_inputs(1, 2048, 96, d, d, dtype=torch.bfloat16, seed=0, gate="softplus")
+        fn = lambda: K.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["S0"], unbounded=True)
     else:
         if args.case == "prefill":
             x = W.workload_inputs("prefill")

@@ -290,6 +290,32 @@ def test_segment_pair_and_combine_host_checks(kda):
     assert comb(BH=0) == 0
 
 
+@host_only
+def test_segment_forward_host_checks(kda):
+    """kda_segment_forward: argument checks before any CUDA call.  On the split tensor-core
+    form (bf16, d = 128) it needs the segment pair's workspace (the records and the identity
+    start state) and out; the other configurations are kda_chunk_fwd and check as it does."""
+    import torch
+    vp = ctypes.c_void_p
+    ob = kda.make_opts(torch.bfloat16)
+    fwd = lambda ptrs, T=64, dk=128, dv=128, opts=ob: kda._lib.kda_segment_forward(
+        *[vp(p) for p in ptrs], 1, T, 2, dk, dv, ctypes.byref(opts), None)
+    good = [0x1000] * 8
+    assert fwd(good[:6] + [0] + good[7:]) == -1            # out required
+    assert fwd(good[:7] + [0x1008]) == -3                  # misaligned S_T
+    assert fwd(good) == -7                                 # needs the pair's workspace
+    pair_ws = kda.kda_segment_pair_workspace_bytes(1, 64, 2, 128, 128, ob)
+    assert pair_ws > kda.kda_chunk_workspace_bytes(1, 64, 2, 128, 128, ob)   # records + identity
+    small = kda.make_opts(torch.bfloat16)
+    small.workspace, small.workspace_bytes = 0x10000, pair_ws - 16
+    assert fwd(good, opts=small) == -7
+    assert kda.kda_abi_version() >= 109
+    # fp32: the whole chunk forward, with its own checks
+    of = kda.make_opts(torch.float32)
+    assert fwd(good, opts=of) == -7
+    assert fwd(good, dk=96, opts=of) == -4
+
+
 def test_binding_checks_shapes_before_any_call(kda):
     """The binding passes sizes read off q and v, so every other tensor must have the shape
     those sizes imply; a mismatch is refused (ValueError) before any pointer is taken."""
