@@ -768,7 +768,7 @@ CASES = ("prefill", "decode", "sweep", "ckda", "bwd", "sweep_plain", "softplus")
 # bytes (read + write) per (chunk, head) item of each from one ncu capture at T = 2048
 # (profiles/), None where no capture of the kernel as it stands exists.
 SWEEP_KERNELS = {2: ["chunk_prep2_kernel", "chunk_scan3_kernel"], 1: ["chunk_mega2_kernel"]}
-KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": 122_725, "chunk_scan3_kernel": 86_777, "chunk_mega2_kernel": None}
+KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": 122_751, "chunk_scan3_kernel": 86_792, "chunk_mega2_kernel": None}
 
 
 def run_case(args):

