@@ -168,7 +168,7 @@ int check_dims(long long B, long long T, long long H, int dk, int dv) {
 
 extern "C" {
 
-int kda_abi_version(void) { return 109; }
+int kda_abi_version(void) { return 110; }
 
 const char *kda_status_string(int s) {
     switch (s) {
@@ -440,9 +440,9 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g, co
     a.B = B; a.T = T; a.H = H; a.dk_ = dk; a.dv_ = dv;
     a.bf16 = o.dtype == KDA_BF16;
     a.fl = kflags(o);
-    if (o.events && o.n_events > 0) cudaEventRecord(o.events[0], stream);
-    cudaError_t e = launch_chunk_bwd(a, stream);
-    if (e == cudaSuccess && o.events && o.n_events > 1) cudaEventRecord(o.events[1], stream);
+    a.events = o.events; a.n_events = o.n_events;
+    cudaError_t e = launch_chunk_bwd(a, stream);   // two launches: the sweeps, the blocks
+    if (e == cudaSuccess && o.events && o.n_events > 2) cudaEventRecord(o.events[2], stream);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

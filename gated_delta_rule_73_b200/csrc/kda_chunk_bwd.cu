@@ -14,17 +14,20 @@
 // backward dx = (dx_hat - x_hat (x_hat . dx_hat)) / n.
 //
 // Layout of the work.  The value columns of S evolve independently (column j sees only
-// v_{t,j}), so a CTA owns NS = 16 columns of one (b, h): 8 warps, two columns per warp (two
-// independent reduction chains per warp), each lane 4 (or 2) key rows of both in registers.
-// The DV / NS CTAs of a sequence form one thread-block cluster.
+// v_{t,j}), and so do the columns of dS; a CTA owns NS = 16 columns of one (b, h): 8 warps, two
+// columns per warp (two independent reduction chains per warp), each lane 4 (or 2) key rows of
+// both in registers.
 //
-// States are needed in reverse order.  Phase 1 runs the recurrence forward and writes the
-// state at the start of every 16-token block to the workspace (FP32, column-major).  Phase 2
-// walks the blocks backward, each as two 8-token windows, upper window first:
+// The reverse recursion dS_{t-1} = Diag(alpha_t)(G - beta_t k_t (k_t . G)), G = dS_t + q_t do_t^T,
+// needs no state.  So two sequential sweeps over the tokens, one launch side by side, give every
+// 16-token block both of its boundary values: the forward sweep writes S at every block start,
+// the reverse sweep dS at every block end (and dS0).  Then every block's local work is
+// independent, and a second launch runs all blocks of all heads at once: one thread-block
+// cluster of DV / NS CTAs per (block, b, h), the block as two 8-token windows, upper window
+// first:
 //   1. recompute the window's pre-token states S_{t-1} into shared memory, with r_t;
-//   2. reverse pass over the window, the only sequential part: G = dS + q do,
-//      a = k . G (a warp reduction), dv = beta a, dS <- alpha (G - k dv).  It needs no
-//      state, only r_t; it records dv_t and a_t r_t per column;
+//   2. reverse pass over the window from its end's dS: G = dS + q do, a = k . G (a warp
+//      reduction), dv = beta a, dS <- alpha (G - k dv); it records dv_t and a_t r_t per column;
 //   3. post-pass: every (token, key row) sum over the CTA's columns -- dq (S_t do), dk
 //      (beta G r - St dv), dalpha (dSt * S_{t-1}) -- re-running the elementwise dS recursion
 //      from the window's end with the recorded dv (no reduction on it), thread = (key row,
@@ -49,170 +52,309 @@ constexpr int NW = 8;           // warps per CTA, two columns each
 constexpr int NT = NW * 32;     // threads per CTA
 static_assert(WL == NW, "staging gives one warp per token row of a window");
 
+// The inputs of one window of tokens, staged in shared memory.
+template <int DK>
+struct WinIn {
+    float qs[WL][DK], ks[WL][DK], as[WL][DK];   // normalised q, k and alpha
+    float vs[WL][NS], dos[WL][NS];              // v and scale * dO of this CTA's columns
+    float bs[WL], nq[WL], nk[WL];               // beta and the reciprocal norms of q and k
+};
+
 template <int DK>
 struct BwdSmem {
     static constexpr int JQ = NT / DK;           // column groups of the post-pass
+    WinIn<DK> in;
     float win[WL][NS][DK];      // S_{t-1} of each token of the window, per column
     float part[3][JQ][WL][DK];  // post-pass sums (dq, dk, dalpha) per column group
-    float qs[WL][DK], ks[WL][DK], as[WL][DK];    // normalised q, k and alpha of the window
     float dsb[NS][DK];          // dS at the window's end (the post-pass restarts from it)
     float rr[WL][NS], drr[WL][NS], ab[WL][NS];   // r, dv and a*r per token and column
-    float vs[WL][NS], dos[WL][NS];               // v and scale * dO of this CTA's columns
-    float bs[WL], nq[WL], nk[WL];
 };
 
 __device__ __forceinline__ float ldf(const float *p, size_t i) { return p[i]; }
 __device__ __forceinline__ float ldf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
 
-template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(NT, 2)
-chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                 const T *__restrict__ g, const T *__restrict__ beta, const float *__restrict__ S0,
-                 const T *__restrict__ dout, const float *__restrict__ dST,
-                 float *__restrict__ dq, float *__restrict__ dkk, float *__restrict__ dvv,
-                 float *__restrict__ dg, float *__restrict__ dbeta, float *__restrict__ dS0,
-                 float *__restrict__ ckpt, int T_, int H, int nblk, KernelFlags fl) {
-    constexpr int RPL = DK / 32;            // key rows per lane
-    constexpr int CS = DV / NS;             // CTAs per sequence (cluster size)
-    constexpr int JQ = BwdSmem<DK>::JQ;     // post-pass column groups
-    constexpr int CPJ = NS / JQ;            // columns per post-pass thread
-    constexpr int TPC = (WL + CS - 1) / CS; // token rows each CTA finishes per window
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    BwdSmem<DK> &sm = *reinterpret_cast<BwdSmem<DK> *>(smem_raw);
-    cg::cluster_group cluster = cg::this_cluster();
+// A window's inputs as one warp's token row holds them between its global loads and its
+// shared-memory writes (so the loads of the next window can be in flight during this one).
+template <int DK>
+struct RowIn {
+    float q[DK / 32], k[DK / 32], g[DK / 32];
+    float v, dout, beta;
+};
 
-    const int rank = (int)cluster.block_rank();
-    const int bh = blockIdx.x / CS;
+// Load token row ta + (warp index) of the sequence whose token t sits at row row0 + t * H, if
+// it is one of the m rows of the window; the CTA's value columns are [col0, col0 + NS).
+template <typename T, int DK, int DV>
+__device__ __forceinline__ void load_row(RowIn<DK> &r, const T *q, const T *k, const T *v, const T *g,
+                                         const T *beta, const T *dout, size_t row0, int H, int ta,
+                                         int m, int col0) {
+    const int tt = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (tt >= m) return;
+    const size_t row = row0 + (size_t)(ta + tt) * H;
+#pragma unroll
+    for (int i = 0; i < DK / 32; ++i) {
+        const int c = lane + 32 * i;
+        r.q[i] = ldf(q, row * DK + c);
+        r.k[i] = ldf(k, row * DK + c);
+        r.g[i] = ldf(g, row * DK + c);
+    }
+    if (lane < NS) {
+        r.v = ldf(v, row * DV + col0 + lane);
+        r.dout = ldf(dout, row * DV + col0 + lane);
+    }
+    if (lane == 0) r.beta = ldf(beta, row);
+}
+
+// Normalise q and k, form alpha and write the row to the window in shared memory.
+template <int DK>
+__device__ __forceinline__ void commit_row(WinIn<DK> &in, const RowIn<DK> &r, int m,
+                                           const KernelFlags &fl) {
+    constexpr int RPL = DK / 32;
+    const int tt = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (tt >= m) return;
+    float sq = 0.f, sk = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        sq += r.q[i] * r.q[i];
+        sk += r.k[i] * r.k[i];
+        in.as[tt][lane + 32 * i] = fl.complex_gate ? r.g[i] : expf(r.g[i]);
+    }
+    float fq = 1.f, fk = 1.f;
+    if (fl.l2norm) {
+        fq = rsqrtf(warp_sum(sq) + kL2Eps);
+        fk = rsqrtf(warp_sum(sk) + kL2Eps);
+    }
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        in.qs[tt][lane + 32 * i] = r.q[i] * fq;
+        in.ks[tt][lane + 32 * i] = r.k[i] * fk;
+    }
+    if (lane < NS) {
+        in.vs[tt][lane] = r.v;
+        in.dos[tt][lane] = fl.scale * r.dout;
+    }
+    if (lane == 0) {
+        in.bs[tt] = r.beta;
+        in.nq[tt] = fq;
+        in.nk[tt] = fk;
+    }
+}
+
+// Stage tokens [ta, ta + m): one warp per token row.
+template <typename T, int DK, int DV>
+__device__ __forceinline__ void stage_window(WinIn<DK> &in, const T *q, const T *k, const T *v,
+                                             const T *g, const T *beta, const T *dout, size_t row0,
+                                             int H, int ta, int m, int col0, const KernelFlags &fl) {
+    RowIn<DK> r;
+    load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, ta, m, col0);
+    commit_row<DK>(in, r, m, fl);
+}
+
+// One forward step of the warp's two columns lc0, lc0 + 1 (lane holds rows lane + 32 i):
+// S <- alpha S, r = v - S^T k, S += beta k r^T.  With win / rr, S_{t-1} and r are recorded.
+template <int DK>
+__device__ __forceinline__ void fwd_step(const WinIn<DK> &in, int tt, int lc0, int lane,
+                                         float (&s)[2][DK / 32], float (*win)[NS][DK],
+                                         float (*rr)[NS]) {
+    constexpr int RPL = DK / 32;
+    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        const int c = lane + 32 * i;
+        if (win) {
+            win[tt][lc0][c] = s[0][i];
+            win[tt][lc0 + 1][c] = s[1][i];
+        }
+        const float a = in.as[tt][c], kc = in.ks[tt][c];
+        s[0][i] *= a;
+        s[1][i] *= a;
+        d0 = fmaf(kc, s[0][i], d0);
+        d1 = fmaf(kc, s[1][i], d1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+        d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+    }
+    const float r0 = in.vs[tt][lc0] - d0, r1 = in.vs[tt][lc0 + 1] - d1;
+    if (rr && lane == 0) {
+        rr[tt][lc0] = r0;
+        rr[tt][lc0 + 1] = r1;
+    }
+    const float bt = in.bs[tt];
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        const float kc = in.ks[tt][lane + 32 * i];
+        s[0][i] = fmaf(kc, bt * r0, s[0][i]);
+        s[1][i] = fmaf(kc, bt * r1, s[1][i]);
+    }
+}
+
+// One reverse step of the warp's two columns: G = dS + q do, d = k . G, dv = beta d,
+// dS <- alpha (G - k dv).  Returns d and dv of both columns.
+template <int DK>
+__device__ __forceinline__ void rev_step(const WinIn<DK> &in, int tt, int lc0, int lane,
+                                         float (&dS)[2][DK / 32], float (&d)[2], float (&dr)[2]) {
+    constexpr int RPL = DK / 32;
+    const float do0 = in.dos[tt][lc0], do1 = in.dos[tt][lc0 + 1], bt = in.bs[tt];
+    float G0[RPL], G1[RPL], d0 = 0.f, d1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        const int c = lane + 32 * i;
+        const float qc = in.qs[tt][c], kc = in.ks[tt][c];
+        G0[i] = fmaf(qc, do0, dS[0][i]);
+        G1[i] = fmaf(qc, do1, dS[1][i]);
+        d0 = fmaf(kc, G0[i], d0);
+        d1 = fmaf(kc, G1[i], d1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        d0 += __shfl_xor_sync(0xffffffffu, d0, o);
+        d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+    }
+    const float dr0 = bt * d0, dr1 = bt * d1;
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        const int c = lane + 32 * i;
+        const float a = in.as[tt][c], kc = in.ks[tt][c];
+        dS[0][i] = a * fmaf(-kc, dr0, G0[i]);
+        dS[1][i] = a * fmaf(-kc, dr1, G1[i]);
+    }
+    d[0] = d0; d[1] = d1;
+    dr[0] = dr0; dr[1] = dr1;
+}
+
+// Checkpoint of block blk of sequence-head bh, value column j: DK FP32 values (column-major).
+__device__ __forceinline__ size_t ck_off(int bh, int nblk, int blk, int j, int DK, int DV) {
+    return (((size_t)bh * nblk + blk) * DV + j) * DK;
+}
+
+// Launch 1: the two sequential sweeps.  CTAs [0, n) run the forward recurrence and write S at
+// every block start to ckpt; CTAs [n, 2n) run the reverse recursion from dS_T and write dS at
+// every block end to dckpt, then dS0.  n = B * H * (DV / NS).
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(NT, 4)
+chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                       const T *__restrict__ g, const T *__restrict__ beta,
+                       const float *__restrict__ S0, const T *__restrict__ dout,
+                       const float *__restrict__ dST, float *__restrict__ dS0,
+                       float *__restrict__ ckpt, float *__restrict__ dckpt, int T_, int H, int nblk,
+                       KernelFlags fl) {
+    constexpr int RPL = DK / 32;
+    constexpr int CS = DV / NS;
+    __shared__ __align__(16) WinIn<DK> in;
+    const int n = (int)gridDim.x / 2;
+    const bool reverse = (int)blockIdx.x >= n;
+    const int cta = (int)blockIdx.x - (reverse ? n : 0);
+    const int bh = cta / CS, rank = cta % CS;
     const int b = bh / H, h = bh % H;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int lc0 = 2 * w;                  // this warp's local columns lc0, lc0 + 1
-    const int j0 = rank * NS + lc0;         // and global columns j0, j0 + 1
-
-    auto row_of = [&](int t) { return ((size_t)b * T_ + t) * H + h; };
-
-    // One warp per token row: normalised q, k (and 1/n), alpha, beta, this CTA's v and dO.
-    auto stage = [&](int ta, int m) {
-        const int tt = w;
-        if (tt < m) {
-            const size_t row = row_of(ta + tt);
-            float qv[RPL], kv[RPL], sq = 0.f, sk = 0.f;
-#pragma unroll
-            for (int i = 0; i < RPL; ++i) {
-                const int c = lane + 32 * i;
-                qv[i] = ldf(q, row * DK + c);
-                kv[i] = ldf(k, row * DK + c);
-                sq += qv[i] * qv[i];
-                sk += kv[i] * kv[i];
-                const float gv = ldf(g, row * DK + c);
-                sm.as[tt][c] = fl.complex_gate ? gv : expf(gv);
-            }
-            float fq = 1.f, fk = 1.f;
-            if (fl.l2norm) {
-                fq = rsqrtf(warp_sum(sq) + kL2Eps);
-                fk = rsqrtf(warp_sum(sk) + kL2Eps);
-            }
-#pragma unroll
-            for (int i = 0; i < RPL; ++i) {
-                sm.qs[tt][lane + 32 * i] = qv[i] * fq;
-                sm.ks[tt][lane + 32 * i] = kv[i] * fk;
-            }
-            if (lane < NS) {
-                sm.vs[tt][lane] = ldf(v, row * DV + rank * NS + lane);
-                sm.dos[tt][lane] = fl.scale * ldf(dout, row * DV + rank * NS + lane);
-            }
-            if (lane == 0) {
-                sm.bs[tt] = ldf(beta, row);
-                sm.nq[tt] = fq;
-                sm.nk[tt] = fk;
-            }
-        }
-    };
-
-    // one forward step of both columns; with WIN, S_{t-1} goes to the window and r to rr
-    auto fwd_step = [&](int tt, float (&s)[2][RPL], bool store) {
-        float d0 = 0.f, d1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            const int c = lane + 32 * i;
-            if (store) {
-                sm.win[tt][lc0][c] = s[0][i];
-                sm.win[tt][lc0 + 1][c] = s[1][i];
-            }
-            const float a = sm.as[tt][c], kc = sm.ks[tt][c];
-            s[0][i] *= a;
-            s[1][i] *= a;
-            d0 = fmaf(kc, s[0][i], d0);
-            d1 = fmaf(kc, s[1][i], d1);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            d0 += __shfl_xor_sync(0xffffffffu, d0, o);
-            d1 += __shfl_xor_sync(0xffffffffu, d1, o);
-        }
-        const float r0 = sm.vs[tt][lc0] - d0, r1 = sm.vs[tt][lc0 + 1] - d1;
-        if (store && lane == 0) {
-            sm.rr[tt][lc0] = r0;
-            sm.rr[tt][lc0 + 1] = r1;
-        }
-        const float bt = sm.bs[tt];
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            const float kc = sm.ks[tt][lane + 32 * i];
-            s[0][i] = fmaf(kc, bt * r0, s[0][i]);
-            s[1][i] = fmaf(kc, bt * r1, s[1][i]);
-        }
-    };
-
+    const int lc0 = 2 * w, j0 = rank * NS + lc0;
+    const size_t row0 = (size_t)b * T_ * H + h;
     const size_t sbase = (size_t)bh * DK * DV;
-    auto load_ckpt = [&](int blk, float (&s)[2][RPL]) {
-        const float *ck = ckpt + (((size_t)bh * nblk + blk) * DV + j0) * DK;
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            s[0][i] = ck[lane + 32 * i];
-            s[1][i] = ck[DK + lane + 32 * i];
-        }
-    };
 
     float s[2][RPL];
+    const float *init = reverse ? dST : S0;
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
-        s[0][i] = S0 ? S0[rowc] : 0.f;
-        s[1][i] = S0 ? S0[rowc + 1] : 0.f;
+        s[0][i] = init ? init[rowc] : 0.f;
+        s[1][i] = init ? init[rowc + 1] : 0.f;
     }
-
-    // ---- phase 1: forward, checkpoint at every block start
-    for (int blk = 0; blk < nblk; ++blk) {
-        float *ck = ckpt + (((size_t)bh * nblk + blk) * DV + j0) * DK;
+    auto put = [&](float *base, int blk) {
+        float *ck = base + ck_off(bh, nblk, blk, j0, DK, DV);
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
             ck[lane + 32 * i] = s[0][i];
             ck[DK + lane + 32 * i] = s[1][i];
         }
-        if (blk == nblk - 1) break;
-        for (int half = 0; half < 2; ++half) {
-            const int ta = blk * BL + half * WL, m = min(WL, T_ - ta);
-            __syncthreads();
-            stage(ta, m);
-            __syncthreads();
-            for (int tt = 0; tt < m; ++tt) fwd_step(tt, s, false);
-        }
-    }
+    };
 
-    // ---- phase 2: blocks in reverse, each as its upper then its lower window
-    float dS[2][RPL];
+    // Window wi covers tokens [wi WL, min(wi WL + WL, T)).  Each pass stages window wi from
+    // registers loaded during the previous window's steps, then loads the next window's rows.
+    RowIn<DK> r;
+    if (!reverse) {
+        const int nw = 2 * (nblk - 1);          // the last block's state is its start's
+        if (nw > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, 0, WL, rank * NS);
+        for (int wi = 0; wi < nw; ++wi) {
+            if ((wi & 1) == 0) put(ckpt, wi >> 1);
+            __syncthreads();
+            commit_row<DK>(in, r, WL, fl);
+            if (wi + 1 < nw)
+                load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi + 1) * WL, WL, rank * NS);
+            __syncthreads();
+            for (int tt = 0; tt < WL; ++tt) fwd_step<DK>(in, tt, lc0, lane, s, nullptr, nullptr);
+        }
+        put(ckpt, nblk - 1);
+        return;
+    }
+    const int nw = (T_ + WL - 1) / WL;
+    load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (nw - 1) * WL, T_ - (nw - 1) * WL, rank * NS);
+    for (int wi = nw - 1; wi >= 0; --wi) {
+        if ((wi & 1) || wi == nw - 1) {         // the last window of block wi / 2: dS at its end
+            put(dckpt, wi >> 1);
+            if (wi <= 1 && !dS0) return;
+        }
+        const int ta = wi * WL, m = min(WL, T_ - ta);
+        __syncthreads();
+        commit_row<DK>(in, r, m, fl);
+        if (wi > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi - 1) * WL, WL, rank * NS);
+        __syncthreads();
+        float d[2], dr[2];
+        for (int tt = m - 1; tt >= 0; --tt) rev_step<DK>(in, tt, lc0, lane, s, d, dr);
+    }
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
-        dS[0][i] = dST ? dST[rowc] : 0.f;
-        dS[1][i] = dST ? dST[rowc + 1] : 0.f;
+        *reinterpret_cast<float2 *>(&dS0[rowc]) = make_float2(s[0][i], s[1][i]);
     }
+}
+
+// Launch 2: one cluster of DV / NS CTAs per (block, b, h); cluster ci is block ci / (B H) of
+// sequence-head ci % (B H).
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(NT, 2)
+chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                       const T *__restrict__ g, const T *__restrict__ beta, const T *__restrict__ dout,
+                       float *__restrict__ dq, float *__restrict__ dkk, float *__restrict__ dvv,
+                       float *__restrict__ dg, float *__restrict__ dbeta,
+                       const float *__restrict__ ckpt, const float *__restrict__ dckpt, int T_, int H,
+                       int BH, int nblk, KernelFlags fl) {
+    constexpr int RPL = DK / 32;            // key rows per lane
+    constexpr int CS = DV / NS;             // CTAs per cluster
+    constexpr int JQ = BwdSmem<DK>::JQ;     // post-pass column groups
+    constexpr int CPJ = NS / JQ;            // columns per post-pass thread
+    constexpr int TPC = (WL + CS - 1) / CS; // token rows each CTA finishes per window
+    static_assert(CPJ % 4 == 0, "the post-pass reads r, dv and dO four columns at a time");
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    BwdSmem<DK> &sm = *reinterpret_cast<BwdSmem<DK> *>(smem_raw);
+    cg::cluster_group cluster = cg::this_cluster();
+
+    const int rank = (int)cluster.block_rank();
+    const int ci = (int)blockIdx.x / CS;
+    const int bh = ci % BH, blk = ci / BH;
+    const int b = bh / H, h = bh % H;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int lc0 = 2 * w;                  // this warp's local columns lc0, lc0 + 1
+    const int j0 = rank * NS + lc0;         // and global columns j0, j0 + 1
+    const size_t row0 = (size_t)b * T_ * H + h;
+    auto row_of = [&](int t) { return row0 + (size_t)t * H; };
+
+    auto load = [&](const float *base, float (&x)[2][RPL]) {
+        const float *ck = base + ck_off(bh, nblk, blk, j0, DK, DV);
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            x[0][i] = ck[lane + 32 * i];
+            x[1][i] = ck[DK + lane + 32 * i];
+        }
+    };
+    float dS[2][RPL];
+    load(dckpt, dS);
 
     auto window = [&](int ta, int m, float (&st)[2][RPL]) {
         __syncthreads();
-        stage(ta, m);
+        stage_window<T, DK, DV>(sm.in, q, k, v, g, beta, dout, row0, H, ta, m, rank * NS, fl);
         __syncthreads();
-        for (int tt = 0; tt < m; ++tt) fwd_step(tt, st, true);
+        for (int tt = 0; tt < m; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, sm.win, sm.rr);
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
             sm.dsb[lc0][lane + 32 * i] = dS[0][i];
@@ -221,36 +363,14 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         __syncwarp();
         // 2. reverse pass (sequential in t)
         for (int tt = m - 1; tt >= 0; --tt) {
-            const float do0 = sm.dos[tt][lc0], do1 = sm.dos[tt][lc0 + 1], bt = sm.bs[tt];
-            float G0[RPL], G1[RPL], d0 = 0.f, d1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < RPL; ++i) {
-                const int c = lane + 32 * i;
-                const float qc = sm.qs[tt][c], kc = sm.ks[tt][c];
-                G0[i] = fmaf(qc, do0, dS[0][i]);
-                G1[i] = fmaf(qc, do1, dS[1][i]);
-                d0 = fmaf(kc, G0[i], d0);
-                d1 = fmaf(kc, G1[i], d1);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                d0 += __shfl_xor_sync(0xffffffffu, d0, o);
-                d1 += __shfl_xor_sync(0xffffffffu, d1, o);
-            }
-            const float dr0 = bt * d0, dr1 = bt * d1;
+            float d[2], dr[2];
+            rev_step<DK>(sm.in, tt, lc0, lane, dS, d, dr);
             if (lane == 0) {
-                sm.drr[tt][lc0] = dr0;
-                sm.drr[tt][lc0 + 1] = dr1;
-                sm.ab[tt][lc0] = d0 * sm.rr[tt][lc0];
-                sm.ab[tt][lc0 + 1] = d1 * sm.rr[tt][lc0 + 1];
-                *reinterpret_cast<float2 *>(&dvv[row_of(ta + tt) * DV + j0]) = make_float2(dr0, dr1);
-            }
-#pragma unroll
-            for (int i = 0; i < RPL; ++i) {
-                const int c = lane + 32 * i;
-                const float a = sm.as[tt][c], kc = sm.ks[tt][c];
-                dS[0][i] = a * fmaf(-kc, dr0, G0[i]);
-                dS[1][i] = a * fmaf(-kc, dr1, G1[i]);
+                sm.drr[tt][lc0] = dr[0];
+                sm.drr[tt][lc0 + 1] = dr[1];
+                sm.ab[tt][lc0] = d[0] * sm.rr[tt][lc0];
+                sm.ab[tt][lc0 + 1] = d[1] * sm.rr[tt][lc0 + 1];
+                *reinterpret_cast<float2 *>(&dvv[row_of(ta + tt) * DV + j0]) = make_float2(dr[0], dr[1]);
             }
         }
         __syncthreads();
@@ -261,19 +381,26 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
 #pragma unroll
             for (int jj = 0; jj < CPJ; ++jj) dl[jj] = sm.dsb[jq * CPJ + jj][c];
             for (int tt = m - 1; tt >= 0; --tt) {
-                const float a = sm.as[tt][c], kc = sm.ks[tt][c], qc = sm.qs[tt][c], bt = sm.bs[tt];
+                const float a = sm.in.as[tt][c], kc = sm.in.ks[tt][c], qc = sm.in.qs[tt][c];
+                const float bt = sm.in.bs[tt];
+                float r[CPJ], dr[CPJ], dov[CPJ];
+#pragma unroll
+                for (int j4 = 0; j4 < CPJ; j4 += 4) {
+                    const int jl = jq * CPJ + j4;
+                    *reinterpret_cast<float4 *>(&r[j4]) = *reinterpret_cast<const float4 *>(&sm.rr[tt][jl]);
+                    *reinterpret_cast<float4 *>(&dr[j4]) = *reinterpret_cast<const float4 *>(&sm.drr[tt][jl]);
+                    *reinterpret_cast<float4 *>(&dov[j4]) = *reinterpret_cast<const float4 *>(&sm.in.dos[tt][jl]);
+                }
                 float sq = 0.f, sk = 0.f, sa = 0.f;
 #pragma unroll
                 for (int jj = 0; jj < CPJ; ++jj) {
-                    const int jl = jq * CPJ + jj;
-                    const float sp = sm.win[tt][jl][c];
+                    const float sp = sm.win[tt][jq * CPJ + jj][c];
                     const float St = a * sp;
-                    const float r = sm.rr[tt][jl], dr = sm.drr[tt][jl], dov = sm.dos[tt][jl];
-                    const float post = fmaf(bt * kc, r, St);
-                    const float G = fmaf(qc, dov, dl[jj]);
-                    sq = fmaf(post, dov, sq);
-                    sk += bt * G * r - St * dr;
-                    const float dSt = fmaf(-kc, dr, G);
+                    const float post = fmaf(bt * kc, r[jj], St);
+                    const float G = fmaf(qc, dov[jj], dl[jj]);
+                    sq = fmaf(post, dov[jj], sq);
+                    sk += bt * G * r[jj] - St * dr[jj];
+                    const float dSt = fmaf(-kc, dr[jj], G);
                     sa = fmaf(dSt, sp, sa);
                     dl[jj] = a * dSt;
                 }
@@ -313,11 +440,11 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
 #pragma unroll
                 for (int i = 0; i < RPL; ++i) {
                     const int c = lane + 32 * i;
-                    dg[row * DK + c] = fl.complex_gate ? val[i] : sm.as[tt][c] * val[i];
+                    dg[row * DK + c] = fl.complex_gate ? val[i] : sm.in.as[tt][c] * val[i];
                 }
             } else {
-                const float *xh = qty == 0 ? &sm.qs[tt][0] : &sm.ks[tt][0];
-                const float inv = qty == 0 ? sm.nq[tt] : sm.nk[tt];
+                const float *xh = qty == 0 ? &sm.in.qs[tt][0] : &sm.in.ks[tt][0];
+                const float inv = qty == 0 ? sm.in.nq[tt] : sm.in.nk[tt];
                 float proj = 0.f;
                 if (fl.l2norm) {
                     float d = 0.f;
@@ -336,39 +463,39 @@ chunk_bwd_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         cluster.sync();
     };
 
-    for (int blk = nblk - 1; blk >= 0; --blk) {
-        const int t0 = blk * BL, n = min(BL, T_ - t0);
-        float st[2][RPL];
-        load_ckpt(blk, st);
-        if (n > WL) {
-            __syncthreads();
-            stage(t0, WL);
-            __syncthreads();
-            for (int tt = 0; tt < WL; ++tt) fwd_step(tt, st, false);
-            window(t0 + WL, n - WL, st);
-            load_ckpt(blk, st);
-        }
-        window(t0, min(n, WL), st);
+    const int t0 = blk * BL, n = min(BL, T_ - t0);
+    float st[2][RPL];
+    load(ckpt, st);
+    if (n > WL) {
+        __syncthreads();
+        stage_window<T, DK, DV>(sm.in, q, k, v, g, beta, dout, row0, H, t0, WL, rank * NS, fl);
+        __syncthreads();
+        for (int tt = 0; tt < WL; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, nullptr, nullptr);
+        window(t0 + WL, n - WL, st);
+        load(ckpt, st);
     }
-    if (dS0) {
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
-            *reinterpret_cast<float2 *>(&dS0[rowc]) = make_float2(dS[0][i], dS[1][i]);
-        }
-    }
+    window(t0, min(n, WL), st);
 }
 
 template <typename T, int DK, int DV>
 cudaError_t launch_t(const BwdArgs &a, cudaStream_t st) {
     constexpr int CS = DV / NS;
-    const size_t smem = sizeof(BwdSmem<DK>);
-    auto kern = chunk_bwd_kernel<T, DK, DV>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int nblk = (a.T + BL - 1) / BL, BH = a.B * a.H;
+    float *ckpt = (float *)a.workspace;
+    float *dckpt = ckpt + (size_t)BH * nblk * DK * DV;
+    if (a.events && a.n_events > 0) cudaEventRecord(a.events[0], st);
+    chunk_bwd_sweep_kernel<T, DK, DV><<<2 * CS * BH, NT, 0, st>>>(
+        (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.g, (const T *)a.beta, a.S0,
+        (const T *)a.dout, a.dS_T, a.dS0, ckpt, dckpt, a.T, a.H, nblk, a.fl);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int nblk = (a.T + BL - 1) / BL;
+
+    const size_t smem = sizeof(BwdSmem<DK>);
+    auto kern = chunk_bwd_block_kernel<T, DK, DV>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(CS * a.B * a.H));
+    cfg.gridDim = dim3((unsigned)((size_t)CS * BH * nblk));
     cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -379,10 +506,11 @@ cudaError_t launch_t(const BwdArgs &a, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (a.events && a.n_events > 1) cudaEventRecord(a.events[1], st);
     return cudaLaunchKernelEx(&cfg, kern, (const T *)a.q, (const T *)a.k, (const T *)a.v,
-                              (const T *)a.g, (const T *)a.beta, a.S0, (const T *)a.dout, a.dS_T,
-                              a.dq, a.dk, a.dv, a.dg, a.dbeta, a.dS0, (float *)a.workspace, a.T,
-                              a.H, nblk, a.fl);
+                              (const T *)a.g, (const T *)a.beta, (const T *)a.dout, a.dq, a.dk, a.dv,
+                              a.dg, a.dbeta, (const float *)ckpt, (const float *)dckpt, a.T, a.H, BH,
+                              nblk, a.fl);
 }
 
 template <typename T>
@@ -394,9 +522,10 @@ cudaError_t launch_d(const BwdArgs &a, cudaStream_t st) {
 }
 }  // namespace
 
+// S at every block start and dS at every block end, FP32.
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
     const size_t nblk = ((size_t)T + BL - 1) / BL;
-    return (size_t)B * H * nblk * dk * dv * sizeof(float);
+    return 2 * (size_t)B * H * nblk * dk * dv * sizeof(float);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st) {

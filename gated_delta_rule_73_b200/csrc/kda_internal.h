@@ -110,6 +110,8 @@ struct BwdArgs {
     int B, T, H, dk_, dv_;
     bool bf16;
     KernelFlags fl;
+    cudaEvent_t *events;                 // kda_opts.events: one before each launch, one after
+    int n_events;
 };
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st);

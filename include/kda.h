@@ -309,8 +309,9 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
  * FP32 [B,H,dk,dv], NULL meaning zero; S0 NULL means zero.  All arithmetic is
  * FP32 and exact for any g <= 0 (no -5 floor needed).  The gradient outputs
  * are written, not accumulated.  opts->workspace must hold
- * kda_chunk_bwd_workspace_bytes(...) bytes: FP32 states every 16 tokens,
- * B*H*ceil(T/16)*dk*dv*4 bytes.  T == 0 writes grad_S0 = dS_T only.
+ * kda_chunk_bwd_workspace_bytes(...) bytes: the FP32 state at every 16-token
+ * block start and its gradient at every block end, 2*B*H*ceil(T/16)*dk*dv*4
+ * bytes.  T == 0 writes grad_S0 = dS_T only.
  */
 int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,
                   const void *beta, const float *S0, const void *dout,
@@ -424,7 +425,8 @@ const char *kda_status_string(int status);
 /* Library ABI version: 100 * major + minor (1.3: kda_chunk_fwd_gated;
    1.4: KDA_UNBOUNDED_DECAY, KDA_GATE_SOFTPLUS; 1.5: kda_chunk_bwd;
    1.6: kda_segment_pair, kda_affine_combine; 1.7: kda_selftest_bounded_wait;
-   1.8: kda_device_status, kda_set_wait_limit; 1.9: kda_segment_forward). */
+   1.8: kda_device_status, kda_set_wait_limit; 1.9: kda_segment_forward;
+   1.10: the kda_chunk_bwd workspace holds the state gradients too). */
 int kda_abi_version(void);
 
 #ifdef __cplusplus

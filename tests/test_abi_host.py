@@ -55,7 +55,7 @@ def test_library_exports_every_declared_symbol(kda):
 
 
 def test_status_strings_and_version(kda):
-    assert kda.kda_abi_version() == 109   # 1.9: kda_segment_forward
+    assert kda.kda_abi_version() == 110   # 1.10: the backward's workspace holds dS too
     for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert kda.status_string(s) and kda.status_string(s) != "unknown status"
     assert kda.status_string(-99) == "unknown status"
@@ -240,7 +240,7 @@ def test_unbounded_decay_flags_on_host(kda):
 @host_only
 def test_chunk_bwd_host_checks(kda):
     """kda_chunk_bwd: argument checks before any CUDA call, and its workspace (FP32 states
-    every 16 tokens: B*H*ceil(T/16)*dk*dv*4 bytes, 256-byte rounded)."""
+    and state gradients every 16 tokens: 2*B*H*ceil(T/16)*dk*dv*4 bytes, 256-byte rounded)."""
     vp = ctypes.c_void_p
     o = kda.make_opts()
 
@@ -259,7 +259,7 @@ def test_chunk_bwd_host_checks(kda):
     assert call(good[:13] + [0], T=0) == 0                 # T = 0 without grad_S0: nothing to do
     bad = kda.make_opts(); bad.flags = 64
     assert call(opts=bad) == -1
-    assert kda.kda_chunk_bwd_workspace_bytes(2, 33, 3, 128, 64, o) == 2 * 3 * 3 * 128 * 64 * 4
+    assert kda.kda_chunk_bwd_workspace_bytes(2, 33, 3, 128, 64, o) == 2 * 2 * 3 * 3 * 128 * 64 * 4
     assert kda.kda_chunk_bwd_workspace_bytes(1, 0, 3, 128, 128, o) == 0
 
 
@@ -309,7 +309,7 @@ def test_segment_forward_host_checks(kda):
     small = kda.make_opts(torch.bfloat16)
     small.workspace, small.workspace_bytes = 0x10000, pair_ws - 16
     assert fwd(good, opts=small) == -7
-    assert kda.kda_abi_version() >= 109
+    assert kda.kda_abi_version() >= 110
     # fp32: the whole chunk forward, with its own checks
     of = kda.make_opts(torch.float32)
     assert fwd(good, opts=of) == -7
