@@ -45,8 +45,7 @@ namespace cg = cooperative_groups;
 namespace kda {
 
 namespace {
-constexpr int BL = 16;          // tokens per checkpoint block
-constexpr int WL = 8;           // tokens per window (half a block)
+constexpr int WL = 8;           // tokens per window (one checkpoint each)
 constexpr int NS = 16;          // value columns per CTA
 constexpr int NW = 8;           // warps per CTA, two columns each
 constexpr int NT = NW * 32;     // threads per CTA
@@ -149,95 +148,86 @@ __device__ __forceinline__ void stage_window(WinIn<DK> &in, const T *q, const T 
     commit_row<DK>(in, r, m, fl);
 }
 
-// One forward step of the warp's two columns lc0, lc0 + 1 (lane holds rows lane + 32 i):
-// S <- alpha S, r = v - S^T k, S += beta k r^T.  With win / rr, S_{t-1} and r are recorded.
+__device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
+
+// One forward step of the warp's two columns lc0, lc0 + 1 (s[i] holds row lane + 32 i of both,
+// as one packed pair): S <- alpha S, r = v - S^T k, S += beta k r^T.  With win / rr, S_{t-1}
+// and r are recorded.
 template <int DK>
 __device__ __forceinline__ void fwd_step(const WinIn<DK> &in, int tt, int lc0, int lane,
-                                         float (&s)[2][DK / 32], float (*win)[NS][DK],
+                                         float2 (&s)[DK / 32], float (*win)[NS][DK],
                                          float (*rr)[NS]) {
     constexpr int RPL = DK / 32;
-    float d0 = 0.f, d1 = 0.f;
+    float2 d = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const int c = lane + 32 * i;
         if (win) {
-            win[tt][lc0][c] = s[0][i];
-            win[tt][lc0 + 1][c] = s[1][i];
+            win[tt][lc0][c] = s[i].x;
+            win[tt][lc0 + 1][c] = s[i].y;
         }
-        const float a = in.as[tt][c], kc = in.ks[tt][c];
-        s[0][i] *= a;
-        s[1][i] *= a;
-        d0 = fmaf(kc, s[0][i], d0);
-        d1 = fmaf(kc, s[1][i], d1);
+        s[i] = __fmul2_rn(s[i], f2(in.as[tt][c]));
+        d = __ffma2_rn(f2(in.ks[tt][c]), s[i], d);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        d0 += __shfl_xor_sync(0xffffffffu, d0, o);
-        d1 += __shfl_xor_sync(0xffffffffu, d1, o);
-    }
-    const float r0 = in.vs[tt][lc0] - d0, r1 = in.vs[tt][lc0 + 1] - d1;
+    for (int o = 16; o > 0; o >>= 1)
+        d = __fadd2_rn(d, make_float2(__shfl_xor_sync(0xffffffffu, d.x, o),
+                                      __shfl_xor_sync(0xffffffffu, d.y, o)));
+    const float r0 = in.vs[tt][lc0] - d.x, r1 = in.vs[tt][lc0 + 1] - d.y;
     if (rr && lane == 0) {
         rr[tt][lc0] = r0;
         rr[tt][lc0 + 1] = r1;
     }
     const float bt = in.bs[tt];
+    const float2 br = make_float2(bt * r0, bt * r1);
 #pragma unroll
-    for (int i = 0; i < RPL; ++i) {
-        const float kc = in.ks[tt][lane + 32 * i];
-        s[0][i] = fmaf(kc, bt * r0, s[0][i]);
-        s[1][i] = fmaf(kc, bt * r1, s[1][i]);
-    }
+    for (int i = 0; i < RPL; ++i) s[i] = __ffma2_rn(f2(in.ks[tt][lane + 32 * i]), br, s[i]);
 }
 
 // One reverse step of the warp's two columns: G = dS + q do, d = k . G, dv = beta d,
 // dS <- alpha (G - k dv).  Returns d and dv of both columns.
 template <int DK>
 __device__ __forceinline__ void rev_step(const WinIn<DK> &in, int tt, int lc0, int lane,
-                                         float (&dS)[2][DK / 32], float (&d)[2], float (&dr)[2]) {
+                                         float2 (&dS)[DK / 32], float2 &d, float2 &dr) {
     constexpr int RPL = DK / 32;
-    const float do0 = in.dos[tt][lc0], do1 = in.dos[tt][lc0 + 1], bt = in.bs[tt];
-    float G0[RPL], G1[RPL], d0 = 0.f, d1 = 0.f;
+    const float2 dov = make_float2(in.dos[tt][lc0], in.dos[tt][lc0 + 1]);
+    const float bt = in.bs[tt];
+    float2 G[RPL];
+    d = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const int c = lane + 32 * i;
-        const float qc = in.qs[tt][c], kc = in.ks[tt][c];
-        G0[i] = fmaf(qc, do0, dS[0][i]);
-        G1[i] = fmaf(qc, do1, dS[1][i]);
-        d0 = fmaf(kc, G0[i], d0);
-        d1 = fmaf(kc, G1[i], d1);
+        G[i] = __ffma2_rn(f2(in.qs[tt][c]), dov, dS[i]);
+        d = __ffma2_rn(f2(in.ks[tt][c]), G[i], d);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        d0 += __shfl_xor_sync(0xffffffffu, d0, o);
-        d1 += __shfl_xor_sync(0xffffffffu, d1, o);
-    }
-    const float dr0 = bt * d0, dr1 = bt * d1;
+    for (int o = 16; o > 0; o >>= 1)
+        d = __fadd2_rn(d, make_float2(__shfl_xor_sync(0xffffffffu, d.x, o),
+                                      __shfl_xor_sync(0xffffffffu, d.y, o)));
+    dr = __fmul2_rn(f2(bt), d);
+    const float2 ndr = make_float2(-dr.x, -dr.y);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const int c = lane + 32 * i;
-        const float a = in.as[tt][c], kc = in.ks[tt][c];
-        dS[0][i] = a * fmaf(-kc, dr0, G0[i]);
-        dS[1][i] = a * fmaf(-kc, dr1, G1[i]);
+        dS[i] = __fmul2_rn(f2(in.as[tt][c]), __ffma2_rn(f2(in.ks[tt][c]), ndr, G[i]));
     }
-    d[0] = d0; d[1] = d1;
-    dr[0] = dr0; dr[1] = dr1;
 }
 
-// Checkpoint of block blk of sequence-head bh, value column j: DK FP32 values (column-major).
-__device__ __forceinline__ size_t ck_off(int bh, int nblk, int blk, int j, int DK, int DV) {
-    return (((size_t)bh * nblk + blk) * DV + j) * DK;
+// Checkpoint of window wi of sequence-head bh, value column j: DK FP32 values (column-major).
+__device__ __forceinline__ size_t ck_off(int bh, int nwin, int wi, int j, int DK, int DV) {
+    return (((size_t)bh * nwin + wi) * DV + j) * DK;
 }
 
 // Launch 1: the two sequential sweeps.  CTAs [0, n) run the forward recurrence and write S at
-// every block start to ckpt; CTAs [n, 2n) run the reverse recursion from dS_T and write dS at
-// every block end to dckpt, then dS0.  n = B * H * (DV / NS).
+// every window start to ckpt; CTAs [n, 2n) run the reverse recursion from dS_T and write dS at
+// every window end to dckpt, then dS0.  n = B * H * (DV / NS).
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(NT, 4)
 chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                        const T *__restrict__ g, const T *__restrict__ beta,
                        const float *__restrict__ S0, const T *__restrict__ dout,
                        const float *__restrict__ dST, float *__restrict__ dS0,
-                       float *__restrict__ ckpt, float *__restrict__ dckpt, int T_, int H, int nblk,
+                       float *__restrict__ ckpt, float *__restrict__ dckpt, int T_, int H, int nwin,
                        KernelFlags fl) {
     constexpr int RPL = DK / 32;
     constexpr int CS = DV / NS;
@@ -252,20 +242,19 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     const size_t row0 = (size_t)b * T_ * H + h;
     const size_t sbase = (size_t)bh * DK * DV;
 
-    float s[2][RPL];
+    float2 s[RPL];
     const float *init = reverse ? dST : S0;
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
-        s[0][i] = init ? init[rowc] : 0.f;
-        s[1][i] = init ? init[rowc + 1] : 0.f;
+        s[i] = init ? make_float2(init[rowc], init[rowc + 1]) : make_float2(0.f, 0.f);
     }
-    auto put = [&](float *base, int blk) {
-        float *ck = base + ck_off(bh, nblk, blk, j0, DK, DV);
+    auto put = [&](float *base, int wi) {
+        float *ck = base + ck_off(bh, nwin, wi, j0, DK, DV);
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
-            ck[lane + 32 * i] = s[0][i];
-            ck[DK + lane + 32 * i] = s[1][i];
+            ck[lane + 32 * i] = s[i].x;
+            ck[DK + lane + 32 * i] = s[i].y;
         }
     };
 
@@ -273,10 +262,10 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     // registers loaded during the previous window's steps, then loads the next window's rows.
     RowIn<DK> r;
     if (!reverse) {
-        const int nw = 2 * (nblk - 1);          // the last block's state is its start's
+        const int nw = nwin - 1;                // the last window's state is its start's
         if (nw > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, 0, WL, rank * NS);
         for (int wi = 0; wi < nw; ++wi) {
-            if ((wi & 1) == 0) put(ckpt, wi >> 1);
+            put(ckpt, wi);
             __syncthreads();
             commit_row<DK>(in, r, WL, fl);
             if (wi + 1 < nw)
@@ -284,32 +273,30 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             __syncthreads();
             for (int tt = 0; tt < WL; ++tt) fwd_step<DK>(in, tt, lc0, lane, s, nullptr, nullptr);
         }
-        put(ckpt, nblk - 1);
+        put(ckpt, nwin - 1);
         return;
     }
-    const int nw = (T_ + WL - 1) / WL;
-    load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (nw - 1) * WL, T_ - (nw - 1) * WL, rank * NS);
-    for (int wi = nw - 1; wi >= 0; --wi) {
-        if ((wi & 1) || wi == nw - 1) {         // the last window of block wi / 2: dS at its end
-            put(dckpt, wi >> 1);
-            if (wi <= 1 && !dS0) return;
-        }
+    load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (nwin - 1) * WL, T_ - (nwin - 1) * WL,
+                        rank * NS);
+    for (int wi = nwin - 1; wi >= 0; --wi) {
+        put(dckpt, wi);
+        if (wi == 0 && !dS0) return;
         const int ta = wi * WL, m = min(WL, T_ - ta);
         __syncthreads();
         commit_row<DK>(in, r, m, fl);
         if (wi > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi - 1) * WL, WL, rank * NS);
         __syncthreads();
-        float d[2], dr[2];
+        float2 d, dr;
         for (int tt = m - 1; tt >= 0; --tt) rev_step<DK>(in, tt, lc0, lane, s, d, dr);
     }
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
         const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
-        *reinterpret_cast<float2 *>(&dS0[rowc]) = make_float2(s[0][i], s[1][i]);
+        *reinterpret_cast<float2 *>(&dS0[rowc]) = s[i];
     }
 }
 
-// Launch 2: one cluster of DV / NS CTAs per (block, b, h); cluster ci is block ci / (B H) of
+// Launch 2: one cluster of DV / NS CTAs per (window, b, h); cluster ci is window ci / (B H) of
 // sequence-head ci % (B H).
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(NT, 2)
@@ -318,7 +305,7 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                        float *__restrict__ dq, float *__restrict__ dkk, float *__restrict__ dvv,
                        float *__restrict__ dg, float *__restrict__ dbeta,
                        const float *__restrict__ ckpt, const float *__restrict__ dckpt, int T_, int H,
-                       int BH, int nblk, KernelFlags fl) {
+                       int BH, int nwin, KernelFlags fl) {
     constexpr int RPL = DK / 32;            // key rows per lane
     constexpr int CS = DV / NS;             // CTAs per cluster
     constexpr int JQ = BwdSmem<DK>::JQ;     // post-pass column groups
@@ -331,7 +318,7 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
 
     const int rank = (int)cluster.block_rank();
     const int ci = (int)blockIdx.x / CS;
-    const int bh = ci % BH, blk = ci / BH;
+    const int bh = ci % BH, wi = ci / BH;
     const int b = bh / H, h = bh % H;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int lc0 = 2 * w;                  // this warp's local columns lc0, lc0 + 1
@@ -339,74 +326,76 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     const size_t row0 = (size_t)b * T_ * H + h;
     auto row_of = [&](int t) { return row0 + (size_t)t * H; };
 
-    auto load = [&](const float *base, float (&x)[2][RPL]) {
-        const float *ck = base + ck_off(bh, nblk, blk, j0, DK, DV);
+    auto load = [&](const float *base, float2 (&x)[RPL]) {
+        const float *ck = base + ck_off(bh, nwin, wi, j0, DK, DV);
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            x[0][i] = ck[lane + 32 * i];
-            x[1][i] = ck[DK + lane + 32 * i];
-        }
+        for (int i = 0; i < RPL; ++i) x[i] = make_float2(ck[lane + 32 * i], ck[DK + lane + 32 * i]);
     };
-    float dS[2][RPL];
+    float2 dS[RPL];
     load(dckpt, dS);
 
-    auto window = [&](int ta, int m, float (&st)[2][RPL]) {
+    auto window = [&](int ta, int m, float2 (&st)[RPL]) {
         __syncthreads();
         stage_window<T, DK, DV>(sm.in, q, k, v, g, beta, dout, row0, H, ta, m, rank * NS, fl);
         __syncthreads();
         for (int tt = 0; tt < m; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, sm.win, sm.rr);
 #pragma unroll
         for (int i = 0; i < RPL; ++i) {
-            sm.dsb[lc0][lane + 32 * i] = dS[0][i];
-            sm.dsb[lc0 + 1][lane + 32 * i] = dS[1][i];
+            sm.dsb[lc0][lane + 32 * i] = dS[i].x;
+            sm.dsb[lc0 + 1][lane + 32 * i] = dS[i].y;
         }
         __syncwarp();
         // 2. reverse pass (sequential in t)
         for (int tt = m - 1; tt >= 0; --tt) {
-            float d[2], dr[2];
+            float2 d, dr;
             rev_step<DK>(sm.in, tt, lc0, lane, dS, d, dr);
             if (lane == 0) {
-                sm.drr[tt][lc0] = dr[0];
-                sm.drr[tt][lc0 + 1] = dr[1];
-                sm.ab[tt][lc0] = d[0] * sm.rr[tt][lc0];
-                sm.ab[tt][lc0 + 1] = d[1] * sm.rr[tt][lc0 + 1];
-                *reinterpret_cast<float2 *>(&dvv[row_of(ta + tt) * DV + j0]) = make_float2(dr[0], dr[1]);
+                sm.drr[tt][lc0] = dr.x;
+                sm.drr[tt][lc0 + 1] = dr.y;
+                sm.ab[tt][lc0] = d.x * sm.rr[tt][lc0];
+                sm.ab[tt][lc0 + 1] = d.y * sm.rr[tt][lc0 + 1];
+                *reinterpret_cast<float2 *>(&dvv[row_of(ta + tt) * DV + j0]) = dr;
             }
         }
         __syncthreads();
-        // 3. post-pass: thread = (key row c, column group jq)
+        // 3. post-pass: thread = (key row c, column group jq), the columns in packed pairs
         {
+            constexpr int CP = CPJ / 2;
             const int c = threadIdx.x % DK, jq = threadIdx.x / DK;
-            float dl[CPJ];
+            float2 dl[CP];
 #pragma unroll
-            for (int jj = 0; jj < CPJ; ++jj) dl[jj] = sm.dsb[jq * CPJ + jj][c];
+            for (int p = 0; p < CP; ++p)
+                dl[p] = make_float2(sm.dsb[jq * CPJ + 2 * p][c], sm.dsb[jq * CPJ + 2 * p + 1][c]);
             for (int tt = m - 1; tt >= 0; --tt) {
                 const float a = sm.in.as[tt][c], kc = sm.in.ks[tt][c], qc = sm.in.qs[tt][c];
                 const float bt = sm.in.bs[tt];
-                float r[CPJ], dr[CPJ], dov[CPJ];
+                float2 r[CP], dr[CP], dov[CP];
 #pragma unroll
-                for (int j4 = 0; j4 < CPJ; j4 += 4) {
-                    const int jl = jq * CPJ + j4;
+                for (int j4 = 0; j4 < CP; j4 += 2) {
+                    const int jl = jq * CPJ + 2 * j4;
                     *reinterpret_cast<float4 *>(&r[j4]) = *reinterpret_cast<const float4 *>(&sm.rr[tt][jl]);
                     *reinterpret_cast<float4 *>(&dr[j4]) = *reinterpret_cast<const float4 *>(&sm.drr[tt][jl]);
                     *reinterpret_cast<float4 *>(&dov[j4]) = *reinterpret_cast<const float4 *>(&sm.in.dos[tt][jl]);
                 }
-                float sq = 0.f, sk = 0.f, sa = 0.f;
+                const float2 a2 = f2(a), btk = f2(bt * kc), q2 = f2(qc), b2 = f2(bt), nk = f2(-kc);
+                float2 sq = make_float2(0.f, 0.f), sk = sq, sa = sq;
 #pragma unroll
-                for (int jj = 0; jj < CPJ; ++jj) {
-                    const float sp = sm.win[tt][jq * CPJ + jj][c];
-                    const float St = a * sp;
-                    const float post = fmaf(bt * kc, r[jj], St);
-                    const float G = fmaf(qc, dov[jj], dl[jj]);
-                    sq = fmaf(post, dov[jj], sq);
-                    sk += bt * G * r[jj] - St * dr[jj];
-                    const float dSt = fmaf(-kc, dr[jj], G);
-                    sa = fmaf(dSt, sp, sa);
-                    dl[jj] = a * dSt;
+                for (int p = 0; p < CP; ++p) {
+                    const int jl = jq * CPJ + 2 * p;
+                    const float2 sp = make_float2(sm.win[tt][jl][c], sm.win[tt][jl + 1][c]);
+                    const float2 St = __fmul2_rn(a2, sp);
+                    const float2 post = __ffma2_rn(btk, r[p], St);
+                    const float2 G = __ffma2_rn(q2, dov[p], dl[p]);
+                    sq = __ffma2_rn(post, dov[p], sq);
+                    sk = __ffma2_rn(__fmul2_rn(b2, G), r[p], sk);
+                    sk = __ffma2_rn(make_float2(-St.x, -St.y), dr[p], sk);
+                    const float2 dSt = __ffma2_rn(nk, dr[p], G);
+                    sa = __ffma2_rn(dSt, sp, sa);
+                    dl[p] = __fmul2_rn(a2, dSt);
                 }
-                sm.part[0][jq][tt][c] = sq;
-                sm.part[1][jq][tt][c] = sk;
-                sm.part[2][jq][tt][c] = sa;
+                sm.part[0][jq][tt][c] = sq.x + sq.y;
+                sm.part[1][jq][tt][c] = sk.x + sk.y;
+                sm.part[2][jq][tt][c] = sa.x + sa.y;
             }
         }
         __syncthreads();
@@ -463,30 +452,21 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         cluster.sync();
     };
 
-    const int t0 = blk * BL, n = min(BL, T_ - t0);
-    float st[2][RPL];
+    float2 st[RPL];
     load(ckpt, st);
-    if (n > WL) {
-        __syncthreads();
-        stage_window<T, DK, DV>(sm.in, q, k, v, g, beta, dout, row0, H, t0, WL, rank * NS, fl);
-        __syncthreads();
-        for (int tt = 0; tt < WL; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, nullptr, nullptr);
-        window(t0 + WL, n - WL, st);
-        load(ckpt, st);
-    }
-    window(t0, min(n, WL), st);
+    window(wi * WL, min(WL, T_ - wi * WL), st);
 }
 
 template <typename T, int DK, int DV>
 cudaError_t launch_t(const BwdArgs &a, cudaStream_t st) {
     constexpr int CS = DV / NS;
-    const int nblk = (a.T + BL - 1) / BL, BH = a.B * a.H;
+    const int nwin = (a.T + WL - 1) / WL, BH = a.B * a.H;
     float *ckpt = (float *)a.workspace;
-    float *dckpt = ckpt + (size_t)BH * nblk * DK * DV;
+    float *dckpt = ckpt + (size_t)BH * nwin * DK * DV;
     if (a.events && a.n_events > 0) cudaEventRecord(a.events[0], st);
     chunk_bwd_sweep_kernel<T, DK, DV><<<2 * CS * BH, NT, 0, st>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, (const T *)a.g, (const T *)a.beta, a.S0,
-        (const T *)a.dout, a.dS_T, a.dS0, ckpt, dckpt, a.T, a.H, nblk, a.fl);
+        (const T *)a.dout, a.dS_T, a.dS0, ckpt, dckpt, a.T, a.H, nwin, a.fl);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -495,7 +475,7 @@ cudaError_t launch_t(const BwdArgs &a, cudaStream_t st) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((size_t)CS * BH * nblk));
+    cfg.gridDim = dim3((unsigned)((size_t)CS * BH * nwin));
     cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -510,7 +490,7 @@ cudaError_t launch_t(const BwdArgs &a, cudaStream_t st) {
     return cudaLaunchKernelEx(&cfg, kern, (const T *)a.q, (const T *)a.k, (const T *)a.v,
                               (const T *)a.g, (const T *)a.beta, (const T *)a.dout, a.dq, a.dk, a.dv,
                               a.dg, a.dbeta, (const float *)ckpt, (const float *)dckpt, a.T, a.H, BH,
-                              nblk, a.fl);
+                              nwin, a.fl);
 }
 
 template <typename T>
@@ -522,10 +502,10 @@ cudaError_t launch_d(const BwdArgs &a, cudaStream_t st) {
 }
 }  // namespace
 
-// S at every block start and dS at every block end, FP32.
+// S at every window start and dS at every window end, FP32.
 size_t chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
-    const size_t nblk = ((size_t)T + BL - 1) / BL;
-    return 2 * (size_t)B * H * nblk * dk * dv * sizeof(float);
+    const size_t nwin = ((size_t)T + WL - 1) / WL;
+    return 2 * (size_t)B * H * nwin * dk * dv * sizeof(float);
 }
 
 cudaError_t launch_chunk_bwd(const BwdArgs &a, cudaStream_t st) {

@@ -309,8 +309,8 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const voi
  * FP32 [B,H,dk,dv], NULL meaning zero; S0 NULL means zero.  All arithmetic is
  * FP32 and exact for any g <= 0 (no -5 floor needed).  The gradient outputs
  * are written, not accumulated.  opts->workspace must hold
- * kda_chunk_bwd_workspace_bytes(...) bytes: the FP32 state at every 16-token
- * block start and its gradient at every block end, 2*B*H*ceil(T/16)*dk*dv*4
+ * kda_chunk_bwd_workspace_bytes(...) bytes: the FP32 state at every 8-token
+ * window start and its gradient at every window end, 2*B*H*ceil(T/8)*dk*dv*4
  * bytes.  T == 0 writes grad_S0 = dS_T only.
  */
 int kda_chunk_bwd(const void *q, const void *k, const void *v, const void *g,

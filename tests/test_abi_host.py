@@ -240,7 +240,7 @@ def test_unbounded_decay_flags_on_host(kda):
 @host_only
 def test_chunk_bwd_host_checks(kda):
     """kda_chunk_bwd: argument checks before any CUDA call, and its workspace (FP32 states
-    and state gradients every 16 tokens: 2*B*H*ceil(T/16)*dk*dv*4 bytes, 256-byte rounded)."""
+    and state gradients every 8 tokens: 2*B*H*ceil(T/8)*dk*dv*4 bytes, 256-byte rounded)."""
     vp = ctypes.c_void_p
     o = kda.make_opts()
 
@@ -259,7 +259,7 @@ def test_chunk_bwd_host_checks(kda):
     assert call(good[:13] + [0], T=0) == 0                 # T = 0 without grad_S0: nothing to do
     bad = kda.make_opts(); bad.flags = 64
     assert call(opts=bad) == -1
-    assert kda.kda_chunk_bwd_workspace_bytes(2, 33, 3, 128, 64, o) == 2 * 2 * 3 * 3 * 128 * 64 * 4
+    assert kda.kda_chunk_bwd_workspace_bytes(2, 33, 3, 128, 64, o) == 2 * 2 * 3 * 5 * 128 * 64 * 4
     assert kda.kda_chunk_bwd_workspace_bytes(1, 0, 3, 128, 128, o) == 0
 
 
