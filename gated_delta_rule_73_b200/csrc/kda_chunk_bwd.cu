@@ -69,53 +69,99 @@ struct BwdSmem {
     float rr[WL][NS], drr[WL][NS], ab[WL][NS];   // r, dv and a*r per token and column
 };
 
-__device__ __forceinline__ float ldf(const float *p, size_t i) { return p[i]; }
-__device__ __forceinline__ float ldf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
+
+// RPL consecutive FP32 values (RPL = 4 or 2) of 16- or 8-byte aligned memory, and the store.
+template <int RPL>
+__device__ __forceinline__ void ld_rows(const float *p, float (&x)[RPL]) {
+    if constexpr (RPL == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    } else {
+        const float2 t = *reinterpret_cast<const float2 *>(p);
+        x[0] = t.x; x[1] = t.y;
+    }
+}
+template <int RPL>
+__device__ __forceinline__ void st_rows(float *p, const float (&x)[RPL]) {
+    if constexpr (RPL == 4) *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    else *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+}
+
+// RPL consecutive input values as one vector load, kept packed until they are used.
+template <typename T, int RPL> struct RowVec;
+template <> struct RowVec<__nv_bfloat16, 4> {
+    uint2 u;
+    __device__ void unpack(float (&x)[4]) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+    }
+};
+template <> struct RowVec<__nv_bfloat16, 2> {
+    uint32_t u;
+    __device__ void unpack(float (&x)[2]) const {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u));
+        x[0] = a.x; x[1] = a.y;
+    }
+};
+template <> struct RowVec<float, 4> {
+    float4 u;
+    __device__ void unpack(float (&x)[4]) const { x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; }
+};
+template <> struct RowVec<float, 2> {
+    float2 u;
+    __device__ void unpack(float (&x)[2]) const { x[0] = u.x; x[1] = u.y; }
+};
+template <typename T, int RPL>
+__device__ __forceinline__ void ldg_rows(RowVec<T, RPL> &r, const T *p) {
+    r.u = *reinterpret_cast<const decltype(r.u) *>(p);
+}
 
 // A window's inputs as one warp's token row holds them between its global loads and its
 // shared-memory writes (so the loads of the next window can be in flight during this one).
-template <int DK>
+// Lane l holds channels RPL l .. RPL l + RPL - 1.
+template <typename T, int DK>
 struct RowIn {
-    float q[DK / 32], k[DK / 32], g[DK / 32];
-    float v, dout, beta;
+    RowVec<T, DK / 32> q, k, g;
+    T v, dout, beta;
 };
 
 // Load token row ta + (warp index) of the sequence whose token t sits at row row0 + t * H, if
 // it is one of the m rows of the window; the CTA's value columns are [col0, col0 + NS).
 template <typename T, int DK, int DV>
-__device__ __forceinline__ void load_row(RowIn<DK> &r, const T *q, const T *k, const T *v, const T *g,
+__device__ __forceinline__ void load_row(RowIn<T, DK> &r, const T *q, const T *k, const T *v, const T *g,
                                          const T *beta, const T *dout, size_t row0, int H, int ta,
                                          int m, int col0) {
+    constexpr int RPL = DK / 32;
     const int tt = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (tt >= m) return;
     const size_t row = row0 + (size_t)(ta + tt) * H;
-#pragma unroll
-    for (int i = 0; i < DK / 32; ++i) {
-        const int c = lane + 32 * i;
-        r.q[i] = ldf(q, row * DK + c);
-        r.k[i] = ldf(k, row * DK + c);
-        r.g[i] = ldf(g, row * DK + c);
-    }
+    ldg_rows<T, RPL>(r.q, q + row * DK + RPL * lane);
+    ldg_rows<T, RPL>(r.k, k + row * DK + RPL * lane);
+    ldg_rows<T, RPL>(r.g, g + row * DK + RPL * lane);
     if (lane < NS) {
-        r.v = ldf(v, row * DV + col0 + lane);
-        r.dout = ldf(dout, row * DV + col0 + lane);
+        r.v = v[row * DV + col0 + lane];
+        r.dout = dout[row * DV + col0 + lane];
     }
-    if (lane == 0) r.beta = ldf(beta, row);
+    if (lane == 0) r.beta = beta[row];
 }
 
 // Normalise q and k, form alpha and write the row to the window in shared memory.
-template <int DK>
-__device__ __forceinline__ void commit_row(WinIn<DK> &in, const RowIn<DK> &r, int m,
+template <typename T, int DK>
+__device__ __forceinline__ void commit_row(WinIn<DK> &in, const RowIn<T, DK> &r, int m,
                                            const KernelFlags &fl) {
     constexpr int RPL = DK / 32;
     const int tt = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (tt >= m) return;
-    float sq = 0.f, sk = 0.f;
+    float qv[RPL], kv[RPL], gv[RPL], sq = 0.f, sk = 0.f;
+    r.q.unpack(qv);
+    r.k.unpack(kv);
+    r.g.unpack(gv);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        sq += r.q[i] * r.q[i];
-        sk += r.k[i] * r.k[i];
-        in.as[tt][lane + 32 * i] = fl.complex_gate ? r.g[i] : expf(r.g[i]);
+        sq += qv[i] * qv[i];
+        sk += kv[i] * kv[i];
+        gv[i] = fl.complex_gate ? gv[i] : expf(gv[i]);
     }
     float fq = 1.f, fk = 1.f;
     if (fl.l2norm) {
@@ -124,15 +170,18 @@ __device__ __forceinline__ void commit_row(WinIn<DK> &in, const RowIn<DK> &r, in
     }
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        in.qs[tt][lane + 32 * i] = r.q[i] * fq;
-        in.ks[tt][lane + 32 * i] = r.k[i] * fk;
+        qv[i] *= fq;
+        kv[i] *= fk;
     }
+    st_rows<RPL>(&in.as[tt][RPL * lane], gv);
+    st_rows<RPL>(&in.qs[tt][RPL * lane], qv);
+    st_rows<RPL>(&in.ks[tt][RPL * lane], kv);
     if (lane < NS) {
-        in.vs[tt][lane] = r.v;
-        in.dos[tt][lane] = fl.scale * r.dout;
+        in.vs[tt][lane] = to_f32(r.v);
+        in.dos[tt][lane] = fl.scale * to_f32(r.dout);
     }
     if (lane == 0) {
-        in.bs[tt] = r.beta;
+        in.bs[tt] = to_f32(r.beta);
         in.nq[tt] = fq;
         in.nk[tt] = fk;
     }
@@ -143,31 +192,40 @@ template <typename T, int DK, int DV>
 __device__ __forceinline__ void stage_window(WinIn<DK> &in, const T *q, const T *k, const T *v,
                                              const T *g, const T *beta, const T *dout, size_t row0,
                                              int H, int ta, int m, int col0, const KernelFlags &fl) {
-    RowIn<DK> r;
+    RowIn<T, DK> r;
     load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, ta, m, col0);
-    commit_row<DK>(in, r, m, fl);
+    commit_row<T, DK>(in, r, m, fl);
 }
 
 __device__ __forceinline__ float2 f2(float x) { return make_float2(x, x); }
 
-// One forward step of the warp's two columns lc0, lc0 + 1 (s[i] holds row lane + 32 i of both,
-// as one packed pair): S <- alpha S, r = v - S^T k, S += beta k r^T.  With win / rr, S_{t-1}
-// and r are recorded.
+// One forward step of the warp's two columns lc0, lc0 + 1 (s[i] holds row RPL lane + i of
+// both, as one packed pair): S <- alpha S, r = v - S^T k, S += beta k r^T.  With win / rr,
+// S_{t-1} and r are recorded.
 template <int DK>
 __device__ __forceinline__ void fwd_step(const WinIn<DK> &in, int tt, int lc0, int lane,
                                          float2 (&s)[DK / 32], float (*win)[NS][DK],
                                          float (*rr)[NS]) {
     constexpr int RPL = DK / 32;
+    const int c0 = RPL * lane;
+    if (win) {
+        float x0[RPL], x1[RPL];
+#pragma unroll
+        for (int i = 0; i < RPL; ++i) {
+            x0[i] = s[i].x;
+            x1[i] = s[i].y;
+        }
+        st_rows<RPL>(&win[tt][lc0][c0], x0);
+        st_rows<RPL>(&win[tt][lc0 + 1][c0], x1);
+    }
+    float a[RPL], kk[RPL];
+    ld_rows<RPL>(&in.as[tt][c0], a);
+    ld_rows<RPL>(&in.ks[tt][c0], kk);
     float2 d = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        const int c = lane + 32 * i;
-        if (win) {
-            win[tt][lc0][c] = s[i].x;
-            win[tt][lc0 + 1][c] = s[i].y;
-        }
-        s[i] = __fmul2_rn(s[i], f2(in.as[tt][c]));
-        d = __ffma2_rn(f2(in.ks[tt][c]), s[i], d);
+        s[i] = __fmul2_rn(s[i], f2(a[i]));
+        d = __ffma2_rn(f2(kk[i]), s[i], d);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -181,7 +239,7 @@ __device__ __forceinline__ void fwd_step(const WinIn<DK> &in, int tt, int lc0, i
     const float bt = in.bs[tt];
     const float2 br = make_float2(bt * r0, bt * r1);
 #pragma unroll
-    for (int i = 0; i < RPL; ++i) s[i] = __ffma2_rn(f2(in.ks[tt][lane + 32 * i]), br, s[i]);
+    for (int i = 0; i < RPL; ++i) s[i] = __ffma2_rn(f2(kk[i]), br, s[i]);
 }
 
 // One reverse step of the warp's two columns: G = dS + q do, d = k . G, dv = beta d,
@@ -190,15 +248,19 @@ template <int DK>
 __device__ __forceinline__ void rev_step(const WinIn<DK> &in, int tt, int lc0, int lane,
                                          float2 (&dS)[DK / 32], float2 &d, float2 &dr) {
     constexpr int RPL = DK / 32;
+    const int c0 = RPL * lane;
     const float2 dov = make_float2(in.dos[tt][lc0], in.dos[tt][lc0 + 1]);
     const float bt = in.bs[tt];
+    float qq[RPL], kk[RPL], a[RPL];
+    ld_rows<RPL>(&in.qs[tt][c0], qq);
+    ld_rows<RPL>(&in.ks[tt][c0], kk);
+    ld_rows<RPL>(&in.as[tt][c0], a);
     float2 G[RPL];
     d = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        const int c = lane + 32 * i;
-        G[i] = __ffma2_rn(f2(in.qs[tt][c]), dov, dS[i]);
-        d = __ffma2_rn(f2(in.ks[tt][c]), G[i], d);
+        G[i] = __ffma2_rn(f2(qq[i]), dov, dS[i]);
+        d = __ffma2_rn(f2(kk[i]), G[i], d);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -207,10 +269,28 @@ __device__ __forceinline__ void rev_step(const WinIn<DK> &in, int tt, int lc0, i
     dr = __fmul2_rn(f2(bt), d);
     const float2 ndr = make_float2(-dr.x, -dr.y);
 #pragma unroll
+    for (int i = 0; i < RPL; ++i) dS[i] = __fmul2_rn(f2(a[i]), __ffma2_rn(f2(kk[i]), ndr, G[i]));
+}
+
+// A lane's RPL rows of the warp's two columns from / to a column-major checkpoint.
+template <int RPL>
+__device__ __forceinline__ void ck_load(const float *ck, int DK, int lane, float2 (&x)[RPL]) {
+    float a[RPL], b[RPL];
+    ld_rows<RPL>(ck + RPL * lane, a);
+    ld_rows<RPL>(ck + DK + RPL * lane, b);
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) x[i] = make_float2(a[i], b[i]);
+}
+template <int RPL>
+__device__ __forceinline__ void ck_store(float *ck, int DK, int lane, const float2 (&x)[RPL]) {
+    float a[RPL], b[RPL];
+#pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        const int c = lane + 32 * i;
-        dS[i] = __fmul2_rn(f2(in.as[tt][c]), __ffma2_rn(f2(in.ks[tt][c]), ndr, G[i]));
+        a[i] = x[i].x;
+        b[i] = x[i].y;
     }
+    st_rows<RPL>(ck + RPL * lane, a);
+    st_rows<RPL>(ck + DK + RPL * lane, b);
 }
 
 // Checkpoint of window wi of sequence-head bh, value column j: DK FP32 values (column-major).
@@ -246,28 +326,21 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     const float *init = reverse ? dST : S0;
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
-        s[i] = init ? make_float2(init[rowc], init[rowc + 1]) : make_float2(0.f, 0.f);
+        const size_t rowc = sbase + (size_t)(RPL * lane + i) * DV + j0;
+        s[i] = init ? *reinterpret_cast<const float2 *>(&init[rowc]) : make_float2(0.f, 0.f);
     }
-    auto put = [&](float *base, int wi) {
-        float *ck = base + ck_off(bh, nwin, wi, j0, DK, DV);
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            ck[lane + 32 * i] = s[i].x;
-            ck[DK + lane + 32 * i] = s[i].y;
-        }
-    };
+    auto put = [&](float *base, int wi) { ck_store<RPL>(base + ck_off(bh, nwin, wi, j0, DK, DV), DK, lane, s); };
 
     // Window wi covers tokens [wi WL, min(wi WL + WL, T)).  Each pass stages window wi from
     // registers loaded during the previous window's steps, then loads the next window's rows.
-    RowIn<DK> r;
+    RowIn<T, DK> r;
     if (!reverse) {
         const int nw = nwin - 1;                // the last window's state is its start's
         if (nw > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, 0, WL, rank * NS);
         for (int wi = 0; wi < nw; ++wi) {
             put(ckpt, wi);
             __syncthreads();
-            commit_row<DK>(in, r, WL, fl);
+            commit_row<T, DK>(in, r, WL, fl);
             if (wi + 1 < nw)
                 load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi + 1) * WL, WL, rank * NS);
             __syncthreads();
@@ -283,7 +356,7 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         if (wi == 0 && !dS0) return;
         const int ta = wi * WL, m = min(WL, T_ - ta);
         __syncthreads();
-        commit_row<DK>(in, r, m, fl);
+        commit_row<T, DK>(in, r, m, fl);
         if (wi > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi - 1) * WL, WL, rank * NS);
         __syncthreads();
         float2 d, dr;
@@ -291,7 +364,7 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     }
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        const size_t rowc = sbase + (size_t)(lane + 32 * i) * DV + j0;
+        const size_t rowc = sbase + (size_t)(RPL * lane + i) * DV + j0;
         *reinterpret_cast<float2 *>(&dS0[rowc]) = s[i];
     }
 }
@@ -327,9 +400,7 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
     auto row_of = [&](int t) { return row0 + (size_t)t * H; };
 
     auto load = [&](const float *base, float2 (&x)[RPL]) {
-        const float *ck = base + ck_off(bh, nwin, wi, j0, DK, DV);
-#pragma unroll
-        for (int i = 0; i < RPL; ++i) x[i] = make_float2(ck[lane + 32 * i], ck[DK + lane + 32 * i]);
+        ck_load<RPL>(base + ck_off(bh, nwin, wi, j0, DK, DV), DK, lane, x);
     };
     float2 dS[RPL];
     load(dckpt, dS);
@@ -339,10 +410,15 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         stage_window<T, DK, DV>(sm.in, q, k, v, g, beta, dout, row0, H, ta, m, rank * NS, fl);
         __syncthreads();
         for (int tt = 0; tt < m; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, sm.win, sm.rr);
+        {
+            float x0[RPL], x1[RPL];
 #pragma unroll
-        for (int i = 0; i < RPL; ++i) {
-            sm.dsb[lc0][lane + 32 * i] = dS[i].x;
-            sm.dsb[lc0 + 1][lane + 32 * i] = dS[i].y;
+            for (int i = 0; i < RPL; ++i) {
+                x0[i] = dS[i].x;
+                x1[i] = dS[i].y;
+            }
+            st_rows<RPL>(&sm.dsb[lc0][RPL * lane], x0);
+            st_rows<RPL>(&sm.dsb[lc0 + 1][RPL * lane], x1);
         }
         __syncwarp();
         // 2. reverse pass (sequential in t)
