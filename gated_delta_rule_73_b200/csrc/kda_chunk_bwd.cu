@@ -344,6 +344,7 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
             if (wi + 1 < nw)
                 load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi + 1) * WL, WL, rank * NS);
             __syncthreads();
+#pragma unroll
             for (int tt = 0; tt < WL; ++tt) fwd_step<DK>(in, tt, lc0, lane, s, nullptr, nullptr);
         }
         put(ckpt, nwin - 1);
@@ -360,7 +361,12 @@ chunk_bwd_sweep_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         if (wi > 0) load_row<T, DK, DV>(r, q, k, v, g, beta, dout, row0, H, (wi - 1) * WL, WL, rank * NS);
         __syncthreads();
         float2 d, dr;
-        for (int tt = m - 1; tt >= 0; --tt) rev_step<DK>(in, tt, lc0, lane, s, d, dr);
+        if (m == WL) {
+#pragma unroll
+            for (int tt = WL - 1; tt >= 0; --tt) rev_step<DK>(in, tt, lc0, lane, s, d, dr);
+        } else {
+            for (int tt = m - 1; tt >= 0; --tt) rev_step<DK>(in, tt, lc0, lane, s, d, dr);
+        }
     }
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
@@ -409,7 +415,12 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         __syncthreads();
         stage_window<T, DK, DV>(sm.in, q, k, v, g, beta, dout, row0, H, ta, m, rank * NS, fl);
         __syncthreads();
-        for (int tt = 0; tt < m; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, sm.win, sm.rr);
+        if (m == WL) {      // a full window: token loops unrolled
+#pragma unroll
+            for (int tt = 0; tt < WL; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, sm.win, sm.rr);
+        } else {
+            for (int tt = 0; tt < m; ++tt) fwd_step<DK>(sm.in, tt, lc0, lane, st, sm.win, sm.rr);
+        }
         {
             float x0[RPL], x1[RPL];
 #pragma unroll
@@ -422,7 +433,7 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
         }
         __syncwarp();
         // 2. reverse pass (sequential in t)
-        for (int tt = m - 1; tt >= 0; --tt) {
+        auto rev = [&](int tt) {
             float2 d, dr;
             rev_step<DK>(sm.in, tt, lc0, lane, dS, d, dr);
             if (lane == 0) {
@@ -432,6 +443,12 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 sm.ab[tt][lc0 + 1] = d.y * sm.rr[tt][lc0 + 1];
                 *reinterpret_cast<float2 *>(&dvv[row_of(ta + tt) * DV + j0]) = dr;
             }
+        };
+        if (m == WL) {
+#pragma unroll
+            for (int tt = WL - 1; tt >= 0; --tt) rev(tt);
+        } else {
+            for (int tt = m - 1; tt >= 0; --tt) rev(tt);
         }
         __syncthreads();
         // 3. post-pass: thread = (key row c, column group jq), the columns in packed pairs
@@ -442,7 +459,7 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
 #pragma unroll
             for (int p = 0; p < CP; ++p)
                 dl[p] = make_float2(sm.dsb[jq * CPJ + 2 * p][c], sm.dsb[jq * CPJ + 2 * p + 1][c]);
-            for (int tt = m - 1; tt >= 0; --tt) {
+            auto post = [&](int tt) {
                 const float a = sm.in.as[tt][c], kc = sm.in.ks[tt][c], qc = sm.in.qs[tt][c];
                 const float bt = sm.in.bs[tt];
                 float2 r[CP], dr[CP], dov[CP];
@@ -472,6 +489,12 @@ chunk_bwd_block_kernel(const T *__restrict__ q, const T *__restrict__ k, const T
                 sm.part[0][jq][tt][c] = sq.x + sq.y;
                 sm.part[1][jq][tt][c] = sk.x + sk.y;
                 sm.part[2][jq][tt][c] = sa.x + sa.y;
+            };
+            if (m == WL) {
+#pragma unroll
+                for (int tt = WL - 1; tt >= 0; --tt) post(tt);
+            } else {
+                for (int tt = m - 1; tt >= 0; --tt) post(tt);
             }
         }
         __syncthreads();
