@@ -363,8 +363,9 @@ def rows_n1(K, flush, hbm_peak, rows):
             torch.cuda.empty_cache()
         fb_ms["ckda_over_kda_throughput_fwd_bwd"] = fb_ms["kda"]["fwd_bwd_ms"] / fb_ms["ckda"]["fwd_bwd_ms"]
         fb_ms["ckda_over_kda_throughput_fwd"] = fb_ms["kda"]["fwd_ms"] / fb_ms["ckda"]["fwd_ms"]
-        fb_ms["note"] = ("B=1 T=32768 H=16 dk=dv=128 bf16, kda_chunk_fwd + kda_chunk_bwd (FP32 recurrent "
-                         "backward sweep); the pages report 96-97 % on H100 (context only)")
+        fb_ms["note"] = ("B=1 T=32768 H=16 dk=dv=128 bf16, kda_chunk_fwd + kda_chunk_bwd (FP32: sweeps for "
+                         "the 8-token boundary values, then all windows in parallel); the pages report "
+                         "96-97 % on H100 (context only)")
         rows["complex_kda_fwd_bwd_T32768_H16"] = fb_ms
 
         # context parallelism over T, emulated on one GPU: the prefill sequence cut into 4
