@@ -20,11 +20,10 @@
 //
 // The reverse recursion dS_{t-1} = Diag(alpha_t)(G - beta_t k_t (k_t . G)), G = dS_t + q_t do_t^T,
 // needs no state.  So two sequential sweeps over the tokens, one launch side by side, give every
-// 16-token block both of its boundary values: the forward sweep writes S at every block start,
-// the reverse sweep dS at every block end (and dS0).  Then every block's local work is
-// independent, and a second launch runs all blocks of all heads at once: one thread-block
-// cluster of DV / NS CTAs per (block, b, h), the block as two 8-token windows, upper window
-// first:
+// 8-token window both of its boundary values: the forward sweep writes S at every window
+// start, the reverse sweep dS at every window end (and dS0).  Then every window's local work
+// is independent, and a second launch runs all windows of all heads at once, one thread-block
+// cluster of DV / NS CTAs per (window, b, h):
 //   1. recompute the window's pre-token states S_{t-1} into shared memory, with r_t;
 //   2. reverse pass over the window from its end's dS: G = dS + q do, a = k . G (a warp
 //      reduction), dv = beta a, dS <- alpha (G - k dv); it records dv_t and a_t r_t per column;
