@@ -848,12 +848,21 @@ prep2_group(const CUtensorMap *ptm_q, const CUtensorMap *ptm_k, const CUtensorMa
                 st16(gsm + OFF_KH + off_kh(16 * pair_of(band, band) + (r & 15), cg), o_kh[0], o_kh[1], o_kh[2], o_kh[3]);
                 st16(img + IMG_QG + off_r128(r, c0), o_qg[0], o_qg[1], o_qg[2], o_qg[3]);
                 st16(img + IMG_KD + off_r128(r, c0), o_kd[0], o_kd[1], o_kd[2], o_kd[3]);
-                for (int bp = band + 1; bp < 4; ++bp) {
-                    float2 f[4];
-                    ld4f2(FT + row_em(bp, band) * 128 + c0, f);
-                    st16(gsm + OFF_KH + off_kh(16 * pair_of(bp, band) + (r & 15), cg), pk2(mul2(kh[0], f[0])),
-                         pk2(mul2(kh[1], f[1])), pk2(mul2(kh[2], f[2])), pk2(mul2(kh[3], f[3])));
-                }
+            }
+            // the later bands' B rows k_i e^{p_b' - gamma_i} = (band b's own row) e^{p_b' - p_b},
+            // b' > b: 6 band pairs x 16 rows x 16 channel groups, 6 per thread (a row's owner
+            // alone would leave the warps of bands 2-3 idle while those of bands 0-1 form three)
+            gbar(gi);
+#pragma unroll
+            for (int k = 0; k < 6; ++k) {
+                const int it = gt + GT * k, cg = it & 15, pr = it >> 8, ri = (it >> 4) & 15;
+                const int b = pr < 3 ? 0 : pr < 5 ? 1 : 2;
+                const int bp = pr < 3 ? pr + 1 : pr < 5 ? pr - 1 : 3;   // (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+                const uint4 u = ld16(gsm + OFF_KH + off_kh(16 * pair_of(b, b) + ri, cg));
+                float2 f[4];
+                ld4f2(FT + row_em(bp, b) * 128 + 8 * cg, f);
+                st16(gsm + OFF_KH + off_kh(16 * pair_of(bp, b) + ri, cg), pk2(mul2(bf2(u.x), f[0])),
+                     pk2(mul2(bf2(u.y), f[1])), pk2(mul2(bf2(u.z), f[2])), pk2(mul2(bf2(u.w), f[3])));
             }
             fence_proxy_async();
         }
