@@ -769,7 +769,9 @@ CASES = ("prefill", "decode", "sweep", "ckda", "bwd", "sweep_plain", "softplus")
 # bytes (read + write) per (chunk, head) item of each from one ncu capture at T = 2048
 # (profiles/), None where no capture of the kernel as it stands exists.
 SWEEP_KERNELS = {2: ["chunk_prep2_kernel", "chunk_scan3_kernel"], 1: ["chunk_mega2_kernel"]}
-KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": 122_751, "chunk_scan3_kernel": 86_792, "chunk_mega2_kernel": None}
+# (the prep's figure was taken before its later-band B rows were spread over the item group: a
+# change inside the kernel, so no figure is reported for it until it is captured again)
+KERNEL_TRAFFIC_PER_ITEM = {"chunk_prep2_kernel": None, "chunk_scan3_kernel": 86_792, "chunk_mega2_kernel": None}
 
 
 def run_case(args):
